@@ -1,0 +1,395 @@
+"""Benchmark of the AnchorKV codec on B200.
+
+One step = the whole hot path over one synthetic cache: compress every layer
+(observation score, anchors, assignment, coefficients, utilities, top-R
+residual selection, 2-bit codec) and then one decode-attention step over every
+compressed layer at batch 1.  The default workload is the Llama-3.1-8B-shaped
+cache (32 layers, 8 KV / 32 query heads, D = 128, N = 32768 tokens, bf16,
+theta = 0.05).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl anchorkv|reference]
+Under torchrun (N > 1) every rank compresses its own independent cache (weak
+scaling, no collective on the data path); the timed region is bracketed by a
+barrier and device synchronisation and its duration is the max over ranks.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "compress Mtok/s per layer-head; compressed decode attn µs/step and HBM GB/s"
+UNIT = "Mtok/s per layer-head"
+WORKLOAD = "llama8b-n32k-bf16"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sust=d.get("bf16_tflops_sustained"),
+                    sm_max_mhz=d.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, sm_max_mhz=1965.0, source="fallback")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.dev)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows]
+        mx = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
+        loaded = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- algorithmic units per stage
+
+def stage_units(spec, theta, L):
+    """Per-launch algorithmic bytes / flops of each stage (see the design notes).
+    Returns {stage: (kind, amount per launch)}; kind 'bytes' or 'flops'."""
+    H, N, D, G, W = spec.n_kv_heads, spec.n_tokens, spec.head_dim, spec.n_q_heads // spec.n_kv_heads, spec.window
+    e = 2 if spec.dtype == "bf16" else 4
+    k = L["n_anchors"]
+    GW = G * W
+    kv = 2 * H * N * D * e
+    return {
+        "obs_pass1": ("flops", 2 * 2 * H * GW * N * D),            # Q K^T and P V
+        "token_stats": ("flops", 2 * 2 * H * GW * N * D),          # Q K^T and V ybar^T
+        "assign": ("flops", 2 * 2 * H * N * k * D),                 # X A^T, both sides
+        "project": ("bytes", kv + 4 * 2 * H * N * 3),               # K, V + records + utilities
+        "quantize": ("bytes", L["n_residuals"] * (2 * D * e + 34)),
+        "decode_split": ("bytes", L["total_bytes"]),
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="anchorkv", choices=["anchorkv", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        return run_reference(args)
+    return run_gpu(args, world, rank, local)
+
+
+# ---------------------------------------------------------------- oracle (CPU) arm
+
+def _oracle_sample(spec, theta, n_heads):
+    """Compress one layer of the workload (the first n_heads KV heads with
+    their query heads) with the CPU oracle; returns (seconds, layer-head tokens)."""
+    from kv_cache_compression_anchorkv_b200.synthetic import CacheSpec, make_layer
+    from oracle import anchorkv_oracle as O
+    sub = CacheSpec(1, n_heads, n_heads * (spec.n_q_heads // spec.n_kv_heads), spec.n_tokens, spec.head_dim,
+                    spec.window, spec.n_dirs, spec.dtype, spec.seed)
+    K, V, Q = make_layer(sub, 0)
+    K, V, Q = (x.double().numpy() for x in (K, V, Q))
+    p = O.Params(n_tokens=spec.n_tokens, n_kv_heads=n_heads, n_q_heads=sub.n_q_heads, theta=theta,
+                 dtype=spec.dtype)
+    t0 = time.perf_counter()
+    O.compress_layer(K, V, Q, p)
+    dt = time.perf_counter() - t0
+    return dt, spec.n_tokens * n_heads
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(spec, theta, n_heads=2):
+    dt, toks = _oracle_sample(spec, theta, n_heads)
+    return {"value": toks / dt / 1e6, "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "sample": f"one layer, {n_heads} of {spec.n_kv_heads} KV heads (N={spec.n_tokens}), fp64 numpy, "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args):
+    from kv_cache_compression_anchorkv_b200.synthetic import WORKLOADS
+    wl = WORKLOADS[WORKLOAD]
+    spec, theta = wl["spec"], wl["theta"]
+    for _ in range(max(0, min(args.warmup, 1))):
+        _oracle_sample(spec, theta, 1)
+    times, toks = [], 0
+    for _ in range(args.steps):
+        dt, toks = _oracle_sample(spec, theta, 1)
+        times.append(dt)
+    total = sum(times)
+    value = toks * args.steps / total / 1e6
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD, "sample": "one layer, 1 KV head (4 query heads) per step",
+                       "n_tokens": spec.n_tokens, "theta": theta},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": _threads(), "kind": "oracle",
+                             "sample": "one layer, 1 of 8 KV heads per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_gpu(args, world, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    from kv_cache_compression_anchorkv_b200 import api
+    from kv_cache_compression_anchorkv_b200.synthetic import WORKLOADS, make_decode_queries, make_layer
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    wl = WORKLOADS[WORKLOAD]
+    spec, theta = wl["spec"], wl["theta"]
+    spec = type(spec)(**{**spec.__dict__, "seed": spec.seed + rank})     # an independent cache per rank
+    Lr, H, N = spec.n_layers, spec.n_kv_heads, spec.n_tokens
+
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu_base = cpu_baseline(spec, theta)
+
+    # inputs resident in HBM: every layer's K, V, Q_obs (4.3 GB at the 8B shape)
+    Ks, Vs, Qs, qd = [], [], [], []
+    for l in range(Lr):
+        K, V, Q = make_layer(spec, l, device=dev)
+        Ks.append(K); Vs.append(V); Qs.append(Q)
+        qd.append(make_decode_queries(spec, l, step=0, batch=1, device=dev))
+    params = [api.AnchorKVParams(n_tokens=N, n_kv_heads=H, n_q_heads=spec.n_q_heads, theta=theta,
+                                 window=spec.window, dtype=spec.dtype, seed=spec.seed, layer=l) for l in range(Lr)]
+    L = api.anchorkv_bytes(params[0])
+    outs = [torch.empty(L["total_bytes"], dtype=torch.uint8, device=dev) for _ in range(Lr)]
+    ws = torch.empty(api.compress_workspace(params[0])["total_bytes"], dtype=torch.uint8, device=dev)
+    dws = torch.empty(api.decode_workspace_bytes(params[0], 1), dtype=torch.uint8, device=dev)
+    dout = [torch.empty(1, spec.n_q_heads, spec.head_dim, dtype=torch.float32, device=dev) for _ in range(Lr)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for l in range(Lr):
+            api.compress(params[l], Ks[l], Vs[l], Qs[l], out=outs[l], workspace=ws)
+        for l in range(Lr):
+            api.decode_attn(params[l], outs[l], qd[l], out=dout[l], workspace=dws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    status = api.read_status(ws)
+    barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    n0 = api.launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    barrier()
+    launches = api.launch_count() - n0
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+
+    # decode alone and compress alone (same stream, CUDA events) for the metric's parts
+    ev2, ev3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    ev2.record(stream)
+    for _ in range(args.steps):
+        for l in range(Lr):
+            api.decode_attn(params[l], outs[l], qd[l], out=dout[l], workspace=dws)
+    ev3.record(stream)
+    barrier()
+    dec_us = 1e3 * ev2.elapsed_time(ev3) / args.steps
+
+    # per-stage event timing over the same steps, for the roofline of the dominant kernel
+    api.stage_timing(True)
+    barrier()
+    for _ in range(args.steps):
+        step()
+    barrier()
+    stages = api.stage_times()
+    api.stage_timing(False)
+
+    peaks = _peaks()
+    units = stage_units(spec, theta, L)
+    dom = max((s for s in stages if s in units and stages[s][1]), key=lambda s: stages[s][0])
+    kind, amount = units[dom]
+    per_launch_s = stages[dom][0] / stages[dom][1] / 1e3
+    if kind == "flops":
+        achieved = amount / per_launch_s / 1e12
+        if dom == "assign" and os.environ.get("ANCHORKV_TC", "1") != "0" and _tc_assign():
+            roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16"], "unit": "TFLOP/s"}
+        else:
+            alu_peak = 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+            roof = {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s"}
+    else:
+        achieved = amount / per_launch_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = dom
+    roof["peak_source"] = peaks["source"]
+
+    dec_bytes = Lr * L["total_bytes"]
+    tokens_step = N * Lr * H * world
+    value = tokens_step / (ms_step / 1e3) / 1e6
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, spec, theta, params, dev, stream, barrier, world)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": spec.dtype, "data": "synthetic",
+            "config": {"workload": WORKLOAD, "layers": Lr, "kv_heads": H, "q_heads": spec.n_q_heads,
+                       "head_dim": spec.head_dim, "n_tokens": N, "window": spec.window, "theta": theta,
+                       "decode_batch": 1, "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (%.1f GB of K/V per step)" % (Lr * 2 * H * N * 128 * 2 / 1e9)},
+            "decode_us_per_step": dec_us,
+            "decode_hbm_gbs": dec_bytes / (dec_us / 1e6) / 1e9,
+            "compressed_bytes_per_layer": L["total_bytes"],
+            "uncompressed_bytes_per_layer": L["uncompressed_bytes"],
+            "compression_ratio": L["uncompressed_bytes"] / L["total_bytes"],
+            "roofline": roof,
+            "stage_ms_per_step": {s: v[0] / args.steps for s, v in stages.items() if v[1]},
+            "gpu_launches": launches,
+            "clocks": clk,
+            "device_status": status[0],
+            "e2e": e2e,
+        }
+        if cpu_base is not None:
+            line["cpu_baseline"] = cpu_base
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def _tc_assign() -> bool:
+    """True when the library's assignment stage runs on the tensor cores."""
+    return False
+
+
+def run_e2e(args, spec, theta, params, dev, stream, barrier, world):
+    """Same step through the public API with host buffers: per layer, pinned
+    K, V, Q_obs are copied in, compressed and the layout copied back; then the
+    decode step copies each layer's query in and its output back."""
+    import torch
+
+    from kv_cache_compression_anchorkv_b200 import api
+    from kv_cache_compression_anchorkv_b200.synthetic import make_decode_queries, make_layer
+    Lr = spec.n_layers
+    # host copies of the layers (pinned); the step moves all of them
+    host = []
+    for l in range(Lr):
+        K, V, Q = make_layer(spec, l, device=dev)
+        host.append(tuple(x.cpu().pin_memory() for x in (K, V, Q)))
+    qh = [make_decode_queries(spec, l, 0, 1, device=dev).cpu().pin_memory() for l in range(Lr)]
+    comp = api.HostCompressor(api.AnchorKVParams(**{**params[0].__dict__}), device=dev)
+    outs_h = [torch.empty_like(comp.host_out).pin_memory() for _ in range(Lr)]
+    qdev = torch.empty(1, spec.n_q_heads, spec.head_dim, dtype=params[0].torch_dtype, device=dev)
+    odev = torch.empty(1, spec.n_q_heads, spec.head_dim, dtype=torch.float32, device=dev)
+    oh = torch.empty(Lr, 1, spec.n_q_heads, spec.head_dim, dtype=torch.float32).pin_memory()
+    layouts = [torch.empty_like(comp.out) for _ in range(Lr)]
+    dws = torch.empty(api.decode_workspace_bytes(params[0], 1), dtype=torch.uint8, device=dev)
+
+    def step():
+        for l in range(Lr):
+            comp(*host[l], layer=l)
+            layouts[l].copy_(comp.out)
+            outs_h[l].copy_(comp.host_out, non_blocking=True)
+        for l in range(Lr):
+            qdev.copy_(qh[l], non_blocking=True)
+            api.decode_attn(params[l], layouts[l], qdev, out=odev, workspace=dws)
+            oh[l].copy_(odev, non_blocking=True)
+
+    steps = max(1, min(args.steps, 3))
+    step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    barrier()
+    ms = e0.elapsed_time(e1) / steps
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = sum(x.numel() * x.element_size() for t3 in host for x in t3) + sum(q.numel() * q.element_size() for q in qh)
+    d2h = sum(o.numel() for o in outs_h) + oh.numel() * 4
+    tokens = spec.n_tokens * Lr * spec.n_kv_heads * world
+    return {"value": tokens / (ms / 1e3) / 1e6, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": ms, "steps": steps}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,203 @@
+"""Thin PyTorch binding of the AnchorKV C ABI.
+
+PyTorch supplies device memory and the current CUDA stream; every step of the
+codec runs in libanchorkv.so.  Functions mirror the C entry points:
+``anchorkv_bytes``, ``compress`` (anchorkv_compress), ``decode_attn``
+(anchorkv_decode_attn), ``reconstruct`` (anchorkv_reconstruct).
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import capi
+
+_DT = {"fp32": capi.FP32, "bf16": capi.BF16}
+_TORCH_DT = {"fp32": torch.float32, "bf16": torch.bfloat16}
+
+
+@dataclass
+class AnchorKVParams:
+    """One layer's codec parameters (defaults: the pages' hyper-parameters)."""
+    n_tokens: int
+    n_kv_heads: int = 8
+    n_q_heads: int = 32
+    theta: float = 0.05
+    head_dim: int = 128
+    window: int = 32
+    dtype: str = "bf16"
+    seed: int = 0
+    layer: int = 0
+    anchor_div: int = 128
+    rho_num: int = 7
+    rho_den: int = 10
+    pool_kernel: int = 7
+
+    def c(self) -> capi.Params:
+        return capi.Params(self.n_tokens, self.head_dim, self.n_kv_heads, self.n_q_heads, self.window,
+                           _DT[self.dtype], float(self.theta), self.seed, self.layer, self.anchor_div,
+                           self.rho_num, self.rho_den, self.pool_kernel, 0)
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return _TORCH_DT[self.dtype]
+
+
+def anchorkv_bytes(p: AnchorKVParams) -> dict:
+    L = capi.Layout()
+    capi.check("anchorkv_bytes", capi.lib().anchorkv_bytes(ctypes.byref(p.c()), ctypes.byref(L)))
+    return {name: getattr(L, name) for name, _ in capi.Layout._fields_}
+
+
+def compress_workspace(p: AnchorKVParams) -> dict:
+    v = capi.WorkspaceView()
+    capi.check("anchorkv_compress_workspace",
+               capi.lib().anchorkv_compress_workspace(ctypes.byref(p.c()), ctypes.byref(v)))
+    return {name: getattr(v, name) for name, _ in capi.WorkspaceView._fields_}
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
+
+
+def _check_tensor(name, t, shape, dtype):
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
+def compress(p: AnchorKVParams, K: torch.Tensor, V: torch.Tensor, Q_obs: torch.Tensor,
+             out: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+    """Compress one layer.  K, V: [H, N, D]; Q_obs: [H_q, W, D] (CUDA, p.dtype).
+    Returns (compressed uint8 tensor of layout.total_bytes, workspace)."""
+    H, N, D, W = p.n_kv_heads, p.n_tokens, p.head_dim, p.window
+    _check_tensor("K", K, (H, N, D), p.torch_dtype)
+    _check_tensor("V", V, (H, N, D), p.torch_dtype)
+    _check_tensor("Q_obs", Q_obs, (p.n_q_heads, W, D), p.torch_dtype)
+    L = anchorkv_bytes(p)
+    ws = compress_workspace(p)
+    if out is None:
+        out = torch.empty(L["total_bytes"], dtype=torch.uint8, device=K.device)
+    if workspace is None:
+        workspace = torch.empty(ws["total_bytes"], dtype=torch.uint8, device=K.device)
+    st = capi.lib().anchorkv_compress(ctypes.byref(p.c()), _ptr(K), _ptr(V), _ptr(Q_obs), _ptr(out),
+                                      out.numel(), _ptr(workspace), workspace.numel(), _stream(K.device))
+    capi.check("anchorkv_compress", st)
+    return out, workspace
+
+
+def decode_workspace_bytes(p: AnchorKVParams, batch: int) -> int:
+    n = ctypes.c_size_t()
+    capi.check("anchorkv_decode_workspace_bytes",
+               capi.lib().anchorkv_decode_workspace_bytes(ctypes.byref(p.c()), batch, ctypes.byref(n)))
+    return n.value
+
+
+def decode_attn(p: AnchorKVParams, compressed: torch.Tensor, q: torch.Tensor,
+                K_tail: torch.Tensor | None = None, V_tail: torch.Tensor | None = None, tail_len: int = 0,
+                out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Decode attention.  compressed: uint8 [batch, stride] (one layout per
+    row) or [total_bytes]; q: [batch, H_q, D]; tails [batch, H, T_cap, D].
+    Returns fp32 [batch, H_q, D]."""
+    if compressed.dim() == 1:
+        compressed = compressed[None]
+    batch, stride = compressed.shape
+    _check_tensor("q", q, (batch, p.n_q_heads, p.head_dim), p.torch_dtype)
+    cap = 0
+    if K_tail is not None:
+        cap = K_tail.shape[2]
+        _check_tensor("K_tail", K_tail, (batch, p.n_kv_heads, cap, p.head_dim), p.torch_dtype)
+        _check_tensor("V_tail", V_tail, (batch, p.n_kv_heads, cap, p.head_dim), p.torch_dtype)
+    if out is None:
+        out = torch.empty(batch, p.n_q_heads, p.head_dim, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(decode_workspace_bytes(p, batch), dtype=torch.uint8, device=q.device)
+    st = capi.lib().anchorkv_decode_attn(ctypes.byref(p.c()), _ptr(compressed), stride, batch, _ptr(q),
+                                         _ptr(K_tail), _ptr(V_tail), tail_len, cap, _ptr(out), _ptr(workspace),
+                                         workspace.numel(), _stream(q.device))
+    capi.check("anchorkv_decode_attn", st)
+    return out
+
+
+def reconstruct(p: AnchorKVParams, compressed: torch.Tensor):
+    """Dense fp32 K^, V^ [H, N, D] of one compressed layer (inspection hook)."""
+    H, N, D = p.n_kv_heads, p.n_tokens, p.head_dim
+    Kh = torch.empty(H, N, D, dtype=torch.float32, device=compressed.device)
+    Vh = torch.empty_like(Kh)
+    st = capi.lib().anchorkv_reconstruct(ctypes.byref(p.c()), _ptr(compressed), _ptr(Kh), _ptr(Vh),
+                                         _stream(compressed.device))
+    capi.check("anchorkv_reconstruct", st)
+    return Kh, Vh
+
+
+def read_status(workspace: torch.Tensor) -> list[int]:
+    """Device status word and counters of a compress workspace (synchronises
+    the current stream).  Raises if a device-side check failed."""
+    buf = (ctypes.c_int32 * 16)()
+    st = capi.lib().anchorkv_read_device_status(_ptr(workspace), buf, _stream(workspace.device))
+    vals = list(buf)
+    capi.check("anchorkv_read_device_status", st)
+    return vals
+
+
+def codebook() -> tuple[float, float, float, float]:
+    out = (ctypes.c_double * 4)()
+    capi.check("anchorkv_codebook", capi.lib().anchorkv_codebook(out))
+    return tuple(out)
+
+
+class HostCompressor:
+    """End-to-end compress from host (pinned) buffers: per call, the layer's
+    K, V, Q_obs are copied to preallocated device buffers, compressed, and the
+    compressed bytes copied back into a pinned host buffer, all on the current
+    stream.  Allocation happens once, in the constructor."""
+
+    def __init__(self, p: AnchorKVParams, device="cuda"):
+        self.p = p
+        H, N, D = p.n_kv_heads, p.n_tokens, p.head_dim
+        self.K = torch.empty(H, N, D, dtype=p.torch_dtype, device=device)
+        self.V = torch.empty_like(self.K)
+        self.Q = torch.empty(p.n_q_heads, p.window, D, dtype=p.torch_dtype, device=device)
+        L = anchorkv_bytes(p)
+        self.out = torch.empty(L["total_bytes"], dtype=torch.uint8, device=device)
+        self.ws = torch.empty(compress_workspace(p)["total_bytes"], dtype=torch.uint8, device=device)
+        self.host_out = torch.empty(L["total_bytes"], dtype=torch.uint8, pin_memory=True)
+
+    def __call__(self, K_host, V_host, Q_host, layer: int | None = None):
+        if layer is not None:
+            self.p.layer = layer
+        self.K.copy_(K_host, non_blocking=True)
+        self.V.copy_(V_host, non_blocking=True)
+        self.Q.copy_(Q_host, non_blocking=True)
+        compress(self.p, self.K, self.V, self.Q, out=self.out, workspace=self.ws)
+        self.host_out.copy_(self.out, non_blocking=True)
+        return self.host_out
+
+
+N_STAGES = 12
+
+
+def stage_timing(enable: bool) -> None:
+    """Turn the library's per-stage CUDA-event timing on (clearing it) or off."""
+    capi.check("anchorkv_stage_timing", capi.lib().anchorkv_stage_timing(1 if enable else 0))
+
+
+def stage_times() -> dict:
+    """{stage name: (total ms, timed calls)} since the last stage_timing(True)."""
+    ms = (ctypes.c_double * N_STAGES)()
+    calls = (ctypes.c_int64 * N_STAGES)()
+    capi.check("anchorkv_stage_times", capi.lib().anchorkv_stage_times(ms, calls, N_STAGES))
+    return {capi.lib().anchorkv_stage_name(i).decode(): (ms[i], calls[i]) for i in range(N_STAGES)}
+
+
+def launch_count() -> int:
+    n = ctypes.c_int64()
+    capi.check("anchorkv_launch_count", capi.lib().anchorkv_launch_count(ctypes.byref(n)))
+    return n.value

@@ -1,0 +1,465 @@
+// Coefficient/residual/utility, per-layer top-R residual selection, the
+// residual codec and the dense reconstruction hook.
+//
+// Sources ("AnchorKV: Anchor-Residual KV Cache Compression", pith.science
+// review; "AnchorKV-adapted", VeloxQuant-MLX docs):
+//  * gamma_i = <x_i, x_a>/||x_a||^2, x^_i = gamma_i x_a + r~_i
+//    (review, "What carries the argument"); gamma is stored in 2 bytes
+//    (review, "Assumptions & free parameters", codec parameters).
+//  * utilities: first-order softmax expansion under the incoherence model
+//    (review, "Circularity Check"; "Assumptions": Eq. 5, Eq. 6, Eq. 16).
+//    Reading: u^V_t = ||r^V_t||^2 sum_r alpha_rt^2,
+//             u^K_t = ||r^K_t||^2 / D^2 sum_r alpha_rt^2 ||q_r||^2 ||V_t - ybar_r||^2.
+//  * the byte budget buys the R best token-sides of the layer, pooled over
+//    heads and sides (VeloxQuant "Evidence": the budget pools across heads;
+//    review: 17.3% of token-sides get residuals).  Ties -> lower flat index
+//    (side, head, position).
+//  * residuals: randomized Hadamard rotation, one fp16 scale ||r||/sqrt(D),
+//    2-bit Lloyd-Max codes for a unit Gaussian (review, Referee "Summary";
+//    "Assumptions": rotated coordinates ~ N(0, ||r||^2/D)).
+// gamma~, ||r||^2, the scale and the code decisions are taken in fp64 from
+// exact inputs (a bf16/fp32 product is exact in fp64), so each integer the
+// codec stores is decided in the precision of a float64 restatement.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace akv {
+namespace {
+
+// ---------------------------------------------------------------- project
+
+template <typename T>
+__global__ void project_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ anc_k,
+                               const T* __restrict__ anc_v, const double* __restrict__ anc_n2,
+                               const int* __restrict__ slot_of, const float* __restrict__ a2s,
+                               const float* __restrict__ kus, uint32_t* __restrict__ tok,
+                               float* __restrict__ util, int N, int H, int k) {
+  const int lane = threadIdx.x & 31;
+  const int64_t total = 2LL * H * N;
+  for (int64_t f = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); f < total;
+       f += (int64_t)gridDim.x * (blockDim.x >> 5)) {
+    const int side = (int)(f / ((int64_t)H * N));
+    const int h = (int)((f / N) % H);
+    const int t = (int)(f % N);
+    const uint32_t slot = tok[f] & 0xFFFFu;
+    const T* x = (side ? V : K) + ((int64_t)h * N + t) * kD;
+    const T* a = (side ? anc_v : anc_k) + ((int64_t)h * k + slot) * kD;
+    float xf[4], af[4];
+    load4<T>(x + lane * 4, xf);
+    load4<T>(a + lane * 4, af);
+    const bool is_anchor = slot_of[(int64_t)h * N + t] >= 0;
+    double dot = 0.0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dot = fma((double)xf[e], (double)af[e], dot);
+    dot = warp_sum_d(dot);
+    const double n2 = anc_n2[((int64_t)side * H + h) * k + slot];
+    double gamma = (n2 > 0.0) ? dot / n2 : 0.0;
+    if (is_anchor) gamma = 1.0;
+    const uint16_t gb = half_bits_rn(gamma);
+    const double g = (double)half_bits_to_f(gb);
+    double r2 = 0.0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const double r = (double)xf[e] - g * (double)af[e];
+      r2 = fma(r, r, r2);
+    }
+    r2 = warp_sum_d(r2);
+    if (lane == 0) {
+      tok[f] = slot | ((uint32_t)gb << 16);
+      float u;
+      if (is_anchor) {
+        u = -1.0f;
+      } else if (side) {
+        u = (float)(r2 * (double)a2s[(int64_t)h * N + t]);
+      } else {
+        u = (float)(r2 / (double)(kD * kD) * (double)kus[(int64_t)h * N + t]);
+      }
+      util[f] = u;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- top-R select
+// Radix select over the utility bits (eligible utilities are >= 0, so their
+// IEEE bit patterns order like the values).  state[0] = threshold prefix,
+// state[1] = how many keys equal to the final threshold are still to take.
+
+__global__ void rs_hist_kernel(const float* __restrict__ util, int64_t n, const uint32_t* __restrict__ state,
+                               int shift, unsigned int* __restrict__ hist) {
+  __shared__ unsigned int sh[256];
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) sh[i] = 0;
+  __syncthreads();
+  const uint32_t prefix = state[0];
+  const uint32_t mask = (shift == 24) ? 0u : (0xFFFFFFFFu << (shift + 8));
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const float u = util[i];
+    if (!(u >= 0.f)) continue;
+    const uint32_t key = __float_as_uint(u);
+    if ((key & mask) == (prefix & mask)) atomicAdd(&sh[(key >> shift) & 255u], 1u);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 256; i += blockDim.x)
+    if (sh[i]) atomicAdd(&hist[i], sh[i]);
+}
+
+__global__ void rs_pick_kernel(unsigned int* __restrict__ hist, uint32_t* __restrict__ state, int shift) {
+  if (threadIdx.x == 0) {
+    const int need = (int)state[1];
+    int cum = 0, digit = 0;
+    for (int d = 255; d >= 0; --d) {
+      if (cum + (int)hist[d] >= need) { digit = d; break; }
+      cum += (int)hist[d];
+    }
+    state[0] |= (uint32_t)digit << shift;
+    state[1] = (uint32_t)(need - cum);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+}
+
+__global__ void rs_init_kernel(uint32_t* __restrict__ state, unsigned int* __restrict__ hist, int R, int take_all) {
+  if (threadIdx.x == 0) {
+    state[0] = 0;
+    state[1] = take_all ? 0x7fffffffu : (uint32_t)R;
+  }
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+}
+
+// One warp per 128-token tile of one (side, head): counts above/at threshold.
+__global__ void sel_tiles_kernel(const float* __restrict__ util, const uint32_t* __restrict__ state, int N,
+                                 int n_tiles, int n_sh, int* __restrict__ tile_gt, int* __restrict__ tile_eq) {
+  const int lane = threadIdx.x & 31;
+  const int tile = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (tile >= n_sh * n_tiles) return;
+  const int sh = tile / n_tiles, j = tile % n_tiles;
+  const uint32_t T = state[0];
+  int gt = 0, eq = 0;
+  for (int w = 0; w < 4; ++w) {
+    const int t = j * kTile + w * 32 + lane;
+    bool g = false, e = false;
+    if (t < N) {
+      const float u = util[(int64_t)sh * N + t];
+      if (u >= 0.f) {
+        const uint32_t key = __float_as_uint(u);
+        g = key > T;
+        e = key == T;
+      }
+    }
+    gt += __popc(__ballot_sync(0xffffffffu, g));
+    eq += __popc(__ballot_sync(0xffffffffu, e));
+  }
+  if (lane == 0) { tile_gt[tile] = gt; tile_eq[tile] = eq; }
+}
+
+// Single-block exclusive scan of n ints; out has n + 1 entries (out[n] = total).
+// With prefix_layout != 0 the result is written as [n_sh][n_tiles + 1] where
+// entry (sh, n_tiles) is the start of the next (side, head).
+__global__ void scan_kernel(const int* __restrict__ in, int n, int* __restrict__ out, int n_tiles,
+                            int prefix_layout) {
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int base = 0; base <= n; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    const int v = (i < n) ? in[i] : 0;
+    int x = v;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = (lane < nw) ? warp_tot[lane] : 0;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      if (lane < nw) warp_tot[lane] = w;
+    }
+    __syncthreads();
+    const int excl = carry + (warp ? warp_tot[warp - 1] : 0) + x - v;
+    if (i <= n) {
+      if (!prefix_layout) {
+        out[i] = excl;
+      } else {
+        const int sh = i / n_tiles, j = i % n_tiles;
+        if (i < n) out[sh * (n_tiles + 1) + j] = excl;
+        if (j == 0 && sh > 0) out[(sh - 1) * (n_tiles + 1) + n_tiles] = excl;
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) carry += warp_tot[nw - 1];
+    __syncthreads();
+  }
+}
+
+__global__ void sel_bitmap_kernel(const float* __restrict__ util, const uint32_t* __restrict__ state, int N,
+                                  int n_tiles, int n_sh, const int* __restrict__ tie_before,
+                                  uint32_t* __restrict__ bitmap, int* __restrict__ tile_cnt,
+                                  int* __restrict__ counters) {
+  const int lane = threadIdx.x & 31;
+  const int tile = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (tile >= n_sh * n_tiles) return;
+  const int sh = tile / n_tiles, j = tile % n_tiles;
+  const uint32_t T = state[0];
+  const int need = (int)state[1];
+  int rank = tie_before[tile];
+  int cnt = 0, ties = 0;
+  for (int w = 0; w < 4; ++w) {
+    const int t = j * kTile + w * 32 + lane;
+    bool g = false, e = false;
+    if (t < N) {
+      const float u = util[(int64_t)sh * N + t];
+      if (u >= 0.f) {
+        const uint32_t key = __float_as_uint(u);
+        g = key > T;
+        e = key == T;
+      }
+    }
+    const uint32_t eqb = __ballot_sync(0xffffffffu, e);
+    const int my_rank = rank + __popc(eqb & ((1u << lane) - 1u));
+    const bool s = g || (e && my_rank < need);
+    const uint32_t sb = __ballot_sync(0xffffffffu, s);
+    if (lane == 0) bitmap[(int64_t)tile * 4 + w] = sb;
+    rank += __popc(eqb);
+    ties += __popc(eqb);
+    cnt += __popc(sb);
+  }
+  if (lane == 0) {
+    tile_cnt[tile] = cnt;
+    if (ties && need != 0x7fffffff) atomicAdd(&counters[kSelectTies], ties);
+  }
+}
+
+// ---------------------------------------------------------------- quantize
+
+struct CodecConst {
+  double tau, l1, l2;
+  uint32_t sign_bits[4];
+};
+
+__device__ __forceinline__ double sign_of(const CodecConst& cc, int j) {
+  return ((cc.sign_bits[j >> 5] >> (j & 31)) & 1u) ? -1.0 : 1.0;
+}
+
+// One warp per (tile, 32-token word); residual records in flat order.
+template <typename T>
+__global__ void quantize_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ anc_k,
+                                const T* __restrict__ anc_v, const uint32_t* __restrict__ tok,
+                                const uint32_t* __restrict__ bitmap, const int* __restrict__ tile_prefix,
+                                uint8_t* __restrict__ codes, uint16_t* __restrict__ sigma, int N, int H, int k,
+                                int n_tiles, int64_t R, int* __restrict__ counters, CodecConst cc) {
+  const int lane = threadIdx.x & 31;
+  const int n_words = 2 * H * n_tiles * 4;
+  const int wid = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (wid >= n_words) return;
+  const int tile = wid >> 2, w = wid & 3;
+  const int sh = tile / n_tiles, j = tile % n_tiles;
+  const int side = sh / H, h = sh % H;
+  const uint32_t* bw = bitmap + (int64_t)tile * 4;
+  int rec = tile_prefix[sh * (n_tiles + 1) + j];
+  for (int q = 0; q < w; ++q) rec += __popc(bw[q]);
+  uint32_t bits = bw[w];
+  const double inv_sqrt_d = 1.0 / sqrt((double)kD);
+  double sgn[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) sgn[e] = sign_of(cc, lane * 4 + e);
+  while (bits) {
+    const int b = __ffs(bits) - 1;
+    bits &= bits - 1;
+    const int t = j * kTile + w * 32 + b;
+    if (rec >= R || t >= N) {                 // inconsistent selection: never write out of bounds
+      if (lane == 0) latch_error(counters, kDevErrBounds);
+      break;
+    }
+    const uint32_t rec_tok = tok[((int64_t)side * H + h) * N + t];
+    const uint32_t slot = rec_tok & 0xFFFFu;
+    const double g = (double)half_bits_to_f(rec_tok >> 16);
+    float xf[4], af[4];
+    load4<T>((side ? V : K) + ((int64_t)h * N + t) * kD + lane * 4, xf);
+    load4<T>((side ? anc_v : anc_k) + ((int64_t)h * k + slot) * kD + lane * 4, af);
+    double y[4];
+    double r2 = 0.0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const double r = (double)xf[e] - g * (double)af[e];
+      r2 = fma(r, r, r2);
+      y[e] = r * sgn[e];
+    }
+    r2 = warp_sum_d(r2);
+    fwht128<double>(y);
+    const uint16_t sb = half_bits_rn(sqrt(r2 / (double)kD));
+    const double th = cc.tau * (double)half_bits_to_f(sb);
+    uint32_t byte = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const double v = y[e] * inv_sqrt_d;
+      const uint32_t c = (v >= th) ? 3u : (v >= 0.0) ? 2u : (v >= -th) ? 1u : 0u;
+      byte |= c << (2 * e);
+    }
+    codes[(int64_t)rec * kCodeBytes + lane] = (uint8_t)byte;
+    if (lane == 0) sigma[rec] = sb;
+    ++rec;
+  }
+}
+
+// ---------------------------------------------------------------- reconstruct
+
+template <typename T>
+__global__ void reconstruct_kernel(const uint8_t* __restrict__ comp, anchorkv_layout L, int N, int H, int k,
+                                   CodecConst cc, float* __restrict__ Kh, float* __restrict__ Vh) {
+  const int lane = threadIdx.x & 31;
+  const int64_t total = 2LL * H * N;
+  const int n_tiles = L.n_tiles;
+  const uint32_t* tok = reinterpret_cast<const uint32_t*>(comp + L.off_tok);
+  const uint32_t* bitmap = reinterpret_cast<const uint32_t*>(comp + L.off_bitmap);
+  const int* prefix = reinterpret_cast<const int*>(comp + L.off_tile_prefix);
+  const uint8_t* codes = comp + L.off_res_codes;
+  const uint16_t* sigma = reinterpret_cast<const uint16_t*>(comp + L.off_res_sigma);
+  const float lev[4] = {(float)-cc.l2, (float)-cc.l1, (float)cc.l1, (float)cc.l2};
+  for (int64_t f = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); f < total;
+       f += (int64_t)gridDim.x * (blockDim.x >> 5)) {
+    const int sh = (int)(f / N), t = (int)(f % N);
+    const int side = sh / H, h = sh % H;
+    const uint32_t rt = tok[f];
+    const T* a = reinterpret_cast<const T*>(comp + (side ? L.off_anchors_v : L.off_anchors_k)) +
+                 ((int64_t)h * k + (rt & 0xFFFFu)) * kD;
+    float af[4];
+    load4<T>(a + lane * 4, af);
+    const float g = half_bits_to_f(rt >> 16);
+    float o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] = g * af[e];
+    const int j = t / kTile, w = (t % kTile) / 32, b = t % 32;
+    const uint32_t* bw = bitmap + ((int64_t)sh * n_tiles + j) * 4;
+    if ((bw[w] >> b) & 1u) {
+      int rec = prefix[sh * (n_tiles + 1) + j];
+      for (int q = 0; q < w; ++q) rec += __popc(bw[q]);
+      rec += __popc(bw[w] & ((1u << b) - 1u));
+      if (rec >= L.n_residuals) continue;     // corrupt layout: leave the anchor part only
+      const float sg = half_bits_to_f(sigma[rec]);
+      const uint32_t byte = codes[(int64_t)rec * kCodeBytes + lane];
+      float z[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) z[e] = lev[(byte >> (2 * e)) & 3u] * sg;
+      fwht128<float>(z);
+      const float isd = rsqrtf((float)kD);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float s = ((cc.sign_bits[(lane * 4 + e) >> 5] >> ((lane * 4 + e) & 31)) & 1u) ? -1.f : 1.f;
+        o[e] += s * z[e] * isd;
+      }
+    }
+    float* dst = (side ? Vh : Kh) + ((int64_t)h * N + t) * kD + lane * 4;
+    *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+CodecConst make_cc(const Plan& pl) {
+  CodecConst cc;
+  cc.tau = pl.tau; cc.l1 = pl.l1; cc.l2 = pl.l2;
+  for (int i = 0; i < 4; ++i) cc.sign_bits[i] = pl.sign_bits[i];
+  return cc;
+}
+
+}  // namespace
+
+cudaError_t launch_project(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s) {
+  const int blocks = 148 * 8;
+  auto* n2 = reinterpret_cast<const double*>(ws + pl.o_anc_n2);
+  auto* slot_of = reinterpret_cast<const int*>(ws + pl.o_slot_of);
+  auto* a2 = reinterpret_cast<const float*>(ws + pl.o_a2);
+  auto* ku = reinterpret_cast<const float*>(ws + pl.o_ku);
+  auto* tok = reinterpret_cast<uint32_t*>(out + pl.L.off_tok);
+  auto* util = reinterpret_cast<float*>(ws + pl.o_util);
+  if (pl.p.dtype == ANCHORKV_BF16) {
+    project_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+        (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
+        reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_k),
+        reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_v), n2, slot_of, a2, ku, tok, util,
+        pl.N, pl.H, pl.k);
+  } else {
+    project_kernel<float><<<blocks, 256, 0, s>>>(
+        (const float*)K, (const float*)V, reinterpret_cast<const float*>(out + pl.L.off_anchors_k),
+        reinterpret_cast<const float*>(out + pl.L.off_anchors_v), n2, slot_of, a2, ku, tok, util,
+        pl.N, pl.H, pl.k);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const Plan& pl, char* out, char* ws, cudaStream_t s) {
+  const int n_sh = 2 * pl.H, n_t = pl.n_tiles, n_tiles_all = n_sh * n_t;
+  auto* util = reinterpret_cast<const float*>(ws + pl.o_util);
+  auto* state = reinterpret_cast<uint32_t*>(ws + pl.o_sel_state);
+  auto* hist = reinterpret_cast<unsigned int*>(ws + pl.o_hist);
+  auto* gt = reinterpret_cast<int*>(ws + pl.o_tile_gt);
+  auto* eq = reinterpret_cast<int*>(ws + pl.o_tile_eq);
+  auto* tb = reinterpret_cast<int*>(ws + pl.o_tie_before);
+  auto* tc = reinterpret_cast<int*>(ws + pl.o_tile_cnt);
+  auto* cnt = reinterpret_cast<int*>(ws + pl.o_counters);
+  auto* bitmap = reinterpret_cast<uint32_t*>(out + pl.L.off_bitmap);
+  auto* prefix = reinterpret_cast<int*>(out + pl.L.off_tile_prefix);
+  if (pl.R == 0) {
+    cudaMemsetAsync(bitmap, 0, (size_t)n_tiles_all * 16, s);
+    cudaMemsetAsync(prefix, 0, (size_t)n_sh * (n_t + 1) * 4, s);
+    return cudaGetLastError();
+  }
+  const bool take_all = pl.R == pl.cap;
+  rs_init_kernel<<<1, 256, 0, s>>>(state, hist, (int)pl.R, take_all ? 1 : 0);
+  if (!take_all) {
+    const int64_t n = 2LL * pl.H * pl.N;
+    const int blocks = (int)std::min<int64_t>(148 * 4, (n + 255) / 256);
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      rs_hist_kernel<<<blocks, 256, 0, s>>>(util, n, state, shift, hist);
+      rs_pick_kernel<<<1, 256, 0, s>>>(hist, state, shift);
+    }
+  }
+  const int wb = (n_tiles_all + 7) / 8;
+  sel_tiles_kernel<<<wb, 256, 0, s>>>(util, state, pl.N, n_t, n_sh, gt, eq);
+  scan_kernel<<<1, 1024, 0, s>>>(eq, n_tiles_all, tb, n_t, 0);
+  sel_bitmap_kernel<<<wb, 256, 0, s>>>(util, state, pl.N, n_t, n_sh, tb, bitmap, tc, cnt);
+  scan_kernel<<<1, 1024, 0, s>>>(tc, n_tiles_all, prefix, n_t, 1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s) {
+  if (pl.R == 0) return cudaSuccess;
+  const int n_words = 2 * pl.H * pl.n_tiles * 4;
+  const int blocks = (n_words + 7) / 8;
+  auto* tok = reinterpret_cast<const uint32_t*>(out + pl.L.off_tok);
+  auto* bitmap = reinterpret_cast<const uint32_t*>(out + pl.L.off_bitmap);
+  auto* prefix = reinterpret_cast<const int*>(out + pl.L.off_tile_prefix);
+  auto* codes = reinterpret_cast<uint8_t*>(out + pl.L.off_res_codes);
+  auto* sigma = reinterpret_cast<uint16_t*>(out + pl.L.off_res_sigma);
+  const CodecConst cc = make_cc(pl);
+  if (pl.p.dtype == ANCHORKV_BF16) {
+    quantize_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+        (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
+        reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_k),
+        reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_v), tok, bitmap, prefix, codes, sigma,
+        pl.N, pl.H, pl.k, pl.n_tiles, pl.R, reinterpret_cast<int*>(ws + pl.o_counters), cc);
+  } else {
+    quantize_kernel<float><<<blocks, 256, 0, s>>>(
+        (const float*)K, (const float*)V, reinterpret_cast<const float*>(out + pl.L.off_anchors_k),
+        reinterpret_cast<const float*>(out + pl.L.off_anchors_v), tok, bitmap, prefix, codes, sigma,
+        pl.N, pl.H, pl.k, pl.n_tiles, pl.R, reinterpret_cast<int*>(ws + pl.o_counters), cc);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reconstruct(const Plan& pl, const char* comp, float* Kh, float* Vh, cudaStream_t s) {
+  const CodecConst cc = make_cc(pl);
+  const int blocks = 148 * 8;
+  if (pl.p.dtype == ANCHORKV_BF16)
+    reconstruct_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>((const uint8_t*)comp, pl.L, pl.N, pl.H, pl.k, cc, Kh, Vh);
+  else
+    reconstruct_kernel<float><<<blocks, 256, 0, s>>>((const uint8_t*)comp, pl.L, pl.N, pl.H, pl.k, cc, Kh, Vh);
+  return cudaGetLastError();
+}
+
+}  // namespace akv

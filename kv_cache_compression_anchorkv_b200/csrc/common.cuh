@@ -1,0 +1,103 @@
+// Device helpers shared by the AnchorKV kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/anchorkv.h"
+
+namespace akv {
+
+constexpr int kD = 128;          // head_dim supported by every kernel
+constexpr int kTile = 128;       // token tile of the residual bitmap / prefix table
+constexpr int kCodeBytes = kD / 4;
+
+// Counter slots in the compress workspace (int32 [16] at offset 0).
+enum Counter {
+  kStatus = 0,        // non-zero: a device-side check failed (code below)
+  kRefineRows = 1,    // nearest-anchor rows re-decided in fp64
+  kSelectTies = 2,    // token-sides whose utility equals the selection threshold
+  kRefineOverflow = 3,
+  kUniformRetries = 4,
+  kCounterCount = 16
+};
+enum DeviceError { kDevErrNone = 0, kDevErrUniform = 1, kDevErrRefine = 2, kDevErrBounds = 3 };
+
+__device__ __forceinline__ void latch_error(int* counters, int code) {
+  atomicCAS(&counters[kStatus], 0, code);
+}
+
+// SplitMix64 output for state x (Steele, Lea & Flood, OOPSLA 2014).
+__host__ __device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+__device__ __forceinline__ uint64_t anchor_key(uint64_t seed, int layer, int head, int t) {
+  return splitmix64(seed ^ ((uint64_t)layer << 48) ^ ((uint64_t)head << 32) ^ (uint64_t)(uint32_t)t);
+}
+
+template <typename T> __device__ __forceinline__ float to_f(T v);
+template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Four consecutive elements starting at p (16-byte aligned for float, 8 for bf16).
+template <typename T> __device__ __forceinline__ void load4(const T* p, float (&o)[4]);
+template <> __device__ __forceinline__ void load4<float>(const float* p, float (&o)[4]) {
+  float4 v = *reinterpret_cast<const float4*>(p);
+  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+}
+template <> __device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, float (&o)[4]) {
+  uint2 v = *reinterpret_cast<const uint2*>(p);
+  o[0] = __uint_as_float(v.x << 16); o[1] = __uint_as_float(v.x & 0xFFFF0000u);
+  o[2] = __uint_as_float(v.y << 16); o[3] = __uint_as_float(v.y & 0xFFFF0000u);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// fp16 (IEEE half) round-to-nearest-even of a double, saturating at +-65504.
+__device__ __forceinline__ uint16_t half_bits_rn(double v) {
+  v = fmin(fmax(v, -65504.0), 65504.0);
+  return __half_as_ushort(__double2half(v));
+}
+__device__ __forceinline__ float half_bits_to_f(uint32_t bits16) {
+  return __half2float(__ushort_as_half((unsigned short)bits16));
+}
+
+// In-warp orthonormal Walsh-Hadamard transform of a 128-vector held as
+// 4 consecutive coordinates per lane (lane l owns 4l..4l+3), natural order.
+template <typename F>
+__device__ __forceinline__ void fwht128(F (&v)[4]) {
+  F a0 = v[0] + v[1], a1 = v[0] - v[1], a2 = v[2] + v[3], a3 = v[2] - v[3];
+  v[0] = a0 + a2; v[2] = a0 - a2; v[1] = a1 + a3; v[3] = a1 - a3;
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = lane & m;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      F other = __shfl_xor_sync(0xffffffffu, v[i], m);
+      v[i] = upper ? (other - v[i]) : (v[i] + other);
+    }
+  }
+}
+
+}  // namespace akv

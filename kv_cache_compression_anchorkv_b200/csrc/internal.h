@@ -1,0 +1,62 @@
+// Host-side plan shared by the C-ABI entry points and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/anchorkv.h"
+
+namespace akv {
+
+// Stages bracketed by the optional event timing (profile.cu).
+enum Stage {
+  kStObsPass1 = 0, kStObsCombine, kStTokenStats, kStAnchorSelect, kStAssign, kStRefine, kStProject,
+  kStSelect, kStQuantize, kStDecodePrep, kStDecodeSplit, kStDecodeCombine, kStageCount
+};
+void stage_begin(int stage, cudaStream_t s);
+void stage_end(int stage, cudaStream_t s, int kernels);
+
+// Everything one compress call needs to know, derived from the parameters.
+struct Plan {
+  anchorkv_params p;
+  anchorkv_layout L;
+  int N, D, H, Hq, G, W, GW, k, n_s, n_u, n_tiles, elem;
+  int64_t R, cap;
+  bool all_anchors;
+  // pass-1 token chunks
+  int chunk1, n_chunk1;
+  // workspace offsets (bytes from the workspace base)
+  int64_t ws_total;
+  int64_t o_counters, o_row_m, o_row_z, o_ybar, o_part_m, o_part_l, o_part_y;
+  int64_t o_score, o_a2, o_ku, o_pooled, o_slot_of, o_anc_n2, o_anc_inv;
+  int64_t o_util, o_refine, o_sel_state, o_hist, o_tile_gt, o_tile_eq, o_tie_before, o_tile_cnt;
+  // codebook and Hadamard signs (bit j set: s_j = -1)
+  double tau, l1, l2;
+  uint32_t sign_bits[4];
+};
+
+int make_plan(const anchorkv_params* p, Plan* out);
+void codebook(double* tau, double* l1, double* l2, double* mse);
+
+struct DecodePlan {
+  int batch, n_split, split_tokens;
+  int64_t ws_total, o_P, o_qrot, o_part_m, o_part_l, o_part_w, o_part_z;
+};
+int make_decode_plan(const Plan& pl, int batch, DecodePlan* out);
+
+// Kernel launchers (one per hot-path step), all asynchronous on `s`.
+cudaError_t launch_obs_pass1(const Plan& pl, const void* K, const void* V, const void* Q, char* ws, cudaStream_t s);
+cudaError_t launch_obs_combine(const Plan& pl, char* ws, cudaStream_t s);
+cudaError_t launch_token_stats(const Plan& pl, const void* K, const void* V, const void* Q, char* ws, cudaStream_t s);
+cudaError_t launch_anchor_select(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s);
+cudaError_t launch_assign_simt(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s);
+cudaError_t launch_refine(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s);
+cudaError_t launch_project(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s);
+cudaError_t launch_select(const Plan& pl, char* out, char* ws, cudaStream_t s);
+cudaError_t launch_quantize(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s);
+cudaError_t launch_decode(const Plan& pl, const DecodePlan& dp, const char* comp, int64_t stride,
+                          const void* q, const void* Kt, const void* Vt, int tail_len, int tail_cap,
+                          float* out, char* ws, cudaStream_t s);
+cudaError_t launch_reconstruct(const Plan& pl, const char* comp, float* Kh, float* Vh, cudaStream_t s);
+
+}  // namespace akv

@@ -285,7 +285,7 @@ def pool_scores(score: np.ndarray, kappa: int) -> np.ndarray:
 # a2: anchor selection
 # --------------------------------------------------------------------------
 
-def select_anchors(pooled: np.ndarray, p: Params, head: int) -> np.ndarray:
+def select_anchors(pooled: np.ndarray, p: Params, head: int, scored: np.ndarray | None = None) -> np.ndarray:
     """Anchor positions of one KV head, ascending (slot s <-> position).
 
     [PITH] free parameters: the final W positions are always anchors; a
@@ -295,6 +295,8 @@ def select_anchors(pooled: np.ndarray, p: Params, head: int) -> np.ndarray:
     (ties -> lower position), n_u = m - n_s drawn without replacement from the
     remaining non-window positions as the n_u smallest counter-based hash keys
     (ties -> lower position).  If N - W <= m every position is an anchor.
+    ``scored`` may carry the scored positions to use instead of recomputing
+    them (tests use it to check the uniform sample on its own).
     """
     N, W = p.n_tokens, p.window
     L = layout(p)
@@ -302,8 +304,10 @@ def select_anchors(pooled: np.ndarray, p: Params, head: int) -> np.ndarray:
         return np.arange(N, dtype=np.int64)
     n_s, n_u = L["n_s"], L["n_u"]
     t = np.arange(N - W)
-    order = np.lexsort((t, -pooled))            # primary: pooled desc; then t asc
-    scored = order[:n_s]
+    if scored is None:
+        order = np.lexsort((t, -pooled))        # primary: pooled desc; then t asc
+        scored = order[:n_s]
+    scored = np.asarray(scored, dtype=np.int64)
     taken = np.zeros(N - W, dtype=bool)
     taken[scored] = True
     rest = t[~taken]

@@ -1,0 +1,205 @@
+"""Stage-by-stage parity of the CUDA path against the oracle.
+
+Every discrete decision (anchor set, nearest-anchor slot, fp16 coefficient,
+residual selection, 2-bit code, fp16 scale, record order) is compared exactly.
+A mismatch is accepted only as a near-tie: the oracle's own fp64 margin at that
+decision lies inside the kernel's error bound for the quantity that decides it.
+Near-ties are counted and returned; each later stage is checked with the GPU's
+earlier decisions fed to the oracle, so one near-tie does not cascade.
+
+Error bounds (relative):
+  pooled score, utility  EPS_SCORE = 2^-14: both come from an fp32 softmax
+      (fp32 dot products of D = 128 exact products, expf, fp32 sums over the
+      observation rows); the measured relative error is reported and is about
+      1e-6, so 2^-14 leaves a wide margin while staying far below the spacing
+      of distinct values;
+  cosine, coefficient, scale, code  EPS_FP64 = 1e-12: these decisions are taken
+      in fp64 from exact products on the GPU, so only fp64 rounding-order noise
+      can separate them from the oracle.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from kv_cache_compression_anchorkv_b200 import api
+from oracle import anchorkv_oracle as O
+
+EPS_SCORE = 2.0 ** -14
+EPS_FP64 = 1e-12
+
+
+def oracle_params(p: api.AnchorKVParams) -> O.Params:
+    return O.Params(n_tokens=p.n_tokens, n_kv_heads=p.n_kv_heads, n_q_heads=p.n_q_heads, theta=p.theta,
+                    head_dim=p.head_dim, window=p.window, dtype=p.dtype, seed=p.seed, layer=p.layer,
+                    anchor_div=p.anchor_div, rho_num=p.rho_num, rho_den=p.rho_den, pool_kernel=p.pool_kernel)
+
+
+def gpu_compress(p: api.AnchorKVParams, K: torch.Tensor, V: torch.Tensor, Q: torch.Tensor):
+    """Run the CUDA compress on (device copies of) K, V, Q; return host arrays."""
+    Kd, Vd, Qd = (x.cuda() if x.device.type != "cuda" else x for x in (K, V, Q))
+    out, ws = api.compress(p, Kd, Vd, Qd)
+    counters = api.read_status(ws)
+    view = api.compress_workspace(p)
+    wsh = ws.cpu().numpy()
+    H, N, W = p.n_kv_heads, p.n_tokens, p.window
+    pooled = wsh[view["off_pooled"]:view["off_pooled"] + 4 * H * N].view(np.float32).reshape(H, N)[:, :N - W]
+    util = wsh[view["off_utility"]:view["off_utility"] + 8 * H * N].view(np.float32).reshape(2, H, N)
+    return out.cpu().numpy(), pooled.astype(np.float64), util.astype(np.float64), counters
+
+
+def _top_by(values: np.ndarray, n: int) -> np.ndarray:
+    """Indices of the n largest values, ties to the lower index."""
+    idx = np.arange(values.shape[0])
+    return idx[np.lexsort((idx, -values))[:n]]
+
+
+def check_compress(p: api.AnchorKVParams, K: np.ndarray, V: np.ndarray, Q: np.ndarray, gpu_bytes: np.ndarray,
+                   gpu_pooled: np.ndarray, gpu_util: np.ndarray, full_chain: bool = True) -> dict:
+    """Assert parity; K, V, Q are float64 copies of the stored values."""
+    po = oracle_params(p)
+    L = O.layout(po)
+    H, N, D, W, G = p.n_kv_heads, p.n_tokens, p.head_dim, p.window, po.group
+    k = L["k"]
+    rep = dict(near_tie_scored=0, near_tie_slot=0, near_tie_gamma=0, near_tie_select=0, near_tie_code=0,
+               exact_ties_slot=0, max_rel_pooled=0.0, max_rel_util=0.0)
+    assert gpu_bytes.shape[0] == L["total"]
+    g = O.unpack_layout(gpu_bytes, po)
+    eligible = np.ones((2, H, N), bool)
+    att = []
+    for h in range(H):
+        Qh = Q[h * G:(h + 1) * G].reshape(G * W, D)
+        a = O.obs_attention(Qh, K[h], V[h], W)
+        att.append((Qh, a))
+        pooled = O.pool_scores(O.token_scores(a["alpha"], N, W), po.pool_kernel)
+        ap_g = g["anchor_pos"][h]
+        eligible[:, h, ap_g] = False
+        if L["k"] == N:
+            assert np.array_equal(ap_g, np.arange(N))
+            continue
+        scale = pooled.max()
+        rep["max_rel_pooled"] = max(rep["max_rel_pooled"], float(np.abs(gpu_pooled[h] - pooled).max() / scale))
+        assert np.abs(gpu_pooled[h] - pooled).max() <= EPS_SCORE * scale, "pooled scores"
+        # the GPU's scored set is the top n_s of its own pooled values
+        s_g = _top_by(gpu_pooled[h], L["n_s"])
+        s_o = _top_by(pooled, L["n_s"])
+        assert set(s_g.tolist()) <= set(ap_g.tolist()), "scored positions missing from the anchor set"
+        diff = set(s_g.tolist()) ^ set(s_o.tolist())
+        if diff:
+            boundary = np.sort(pooled)[::-1][L["n_s"] - 1]
+            for t in diff:
+                assert abs(pooled[t] - boundary) <= EPS_SCORE * scale, f"scored anchor {t} is not a near-tie"
+            rep["near_tie_scored"] += len(diff) // 2 + len(diff) % 2
+        # uniform sample and window, given the GPU's scored set: exact
+        want = O.select_anchors(pooled, po, h, scored=s_g)
+        assert np.array_equal(ap_g, want), "uniform sample / window / slot order"
+    # anchor rows are the input rows, bit for bit
+    for h in range(H):
+        assert np.array_equal(g["anchors_K"][h], K[h][g["anchor_pos"][h]])
+        assert np.array_equal(g["anchors_V"][h], V[h][g["anchor_pos"][h]])
+    # nearest-anchor slot and coefficient, per side
+    r2 = np.zeros((2, H, N))
+    r_all = np.zeros((2, H, N, D))
+    for h in range(H):
+        ap = g["anchor_pos"][h]
+        for side, X in enumerate((K[h], V[h])):
+            idx_o, dots, cos = O.assign(X, ap)
+            idx_g = g["idx"][side, h]
+            bad = np.nonzero(idx_o != idx_g)[0]
+            xn = np.linalg.norm(X, axis=1)
+            for t in bad:
+                margin = cos[t, idx_o[t]] - cos[t, idx_g[t]]
+                assert margin <= EPS_FP64 * max(xn[t], 1e-300), f"slot of token {t} side {side} head {h}"
+            rep["near_tie_slot"] += len(bad)
+            top2 = np.sort(cos, axis=1)[:, -2:] if k > 1 else None
+            if top2 is not None:
+                non_anchor = np.ones(N, bool)
+                non_anchor[ap] = False
+                rep["exact_ties_slot"] += int(((top2[:, 1] == top2[:, 0]) & non_anchor).sum())
+            gamma, g16_o, r, rr2 = O.project(X, ap, idx_g)
+            g16_g = g["g16"][side, h]
+            badg = np.nonzero(g16_o.view(np.uint16) != g16_g.view(np.uint16))[0]
+            for t in badg:
+                mid = 0.5 * (float(g16_o[t]) + float(g16_g[t]))
+                assert abs(gamma[t] - mid) <= EPS_FP64 * max(abs(gamma[t]), 1e-300), f"gamma of token {t}"
+            rep["near_tie_gamma"] += len(badg)
+            # downstream uses the GPU's stored coefficient
+            xa = X[ap][idx_g]
+            r = X - g16_g.astype(np.float64)[:, None] * xa
+            r[ap] = 0.0
+            r_all[side, h] = r
+            r2[side, h] = (r * r).sum(axis=1)
+    # utilities (oracle formula on the GPU's decisions)
+    u_o = np.zeros((2, H, N))
+    for h in range(H):
+        Qh, a = att[h]
+        uK, uV = O.utilities(a["alpha"], a["ybar"], Qh, V[h], r2[0, h], r2[1, h], g["anchor_pos"][h])
+        u_o[0, h], u_o[1, h] = uK, uV
+    assert np.all(gpu_util[~eligible] == -1.0)
+    el = eligible
+    if el.any():
+        scale_u = u_o[el].max()
+        err = np.abs(gpu_util[el] - u_o[el])
+        rep["max_rel_util"] = float((err / np.maximum(u_o[el], 1e-30 * scale_u)).max())
+        assert np.all(err <= EPS_SCORE * u_o[el] + 1e-30 * scale_u), "utilities"
+    # selection: the GPU picks the top R of its own utilities (exact) ...
+    R = L["R"]
+    flat_gu = np.where(el, gpu_util, -np.inf).reshape(-1)
+    assert g["sel"].sum() == R
+    sel_g = g["sel"].reshape(-1)
+    if R:
+        assert np.array_equal(np.sort(_top_by(flat_gu, R)), np.nonzero(sel_g)[0]), "top-R of GPU utilities"
+    # ... and agrees with the oracle's top R up to near-ties at the boundary
+    sel_o = O.select_residuals(u_o, el, R).reshape(-1)
+    diff = np.nonzero(sel_o != sel_g)[0]
+    if len(diff):
+        fu = u_o.reshape(-1)
+        boundary = np.sort(fu[el.reshape(-1)])[::-1][R - 1]
+        for f in diff:
+            assert abs(fu[f] - boundary) <= EPS_SCORE * boundary, f"selection of token-side {f}"
+        rep["near_tie_select"] += len(diff) // 2 + len(diff) % 2
+    # tile prefix table from the GPU's selection (exact)
+    n_t = L["n_tiles"]
+    per = np.zeros((2, H, n_t * O.TILE), bool)
+    per[:, :, :N] = g["sel"]
+    counts = per.reshape(2 * H, n_t, O.TILE).sum(axis=2).reshape(-1)
+    starts = np.concatenate([[0], np.cumsum(counts)])
+    want_prefix = np.zeros((2 * H, n_t + 1), np.int64)
+    for sh in range(2 * H):
+        want_prefix[sh] = starts[sh * n_t: sh * n_t + n_t + 1]
+    assert np.array_equal(g["tile_prefix"].reshape(2 * H, n_t + 1), want_prefix)
+    # residual codes and scales for the GPU-selected rows, in record order
+    if R:
+        rows = r_all[g["sel"]]
+        sig_o, codes_o, y = O.quantize_residuals(rows, p.seed)
+        assert np.array_equal(sig_o.view(np.uint16), g["sigma16"].view(np.uint16)), "residual scales"
+        badc = np.argwhere(codes_o != g["codes"])
+        tau = O.lloyd_max_gaussian_4()[0]
+        for i, j in badc:
+            s16 = float(sig_o[i])
+            m = min(abs(y[i, j] - tau * s16), abs(y[i, j]), abs(y[i, j] + tau * s16))
+            assert m <= EPS_FP64 * max(np.linalg.norm(rows[i]), 1e-300), f"code {i},{j}"
+        rep["near_tie_code"] += len(badc)
+    near = sum(v for k_, v in rep.items() if k_.startswith("near_tie"))
+    rep["near_ties"] = near
+    if full_chain and near == 0:
+        ref = O.compress_layer(K, V, Q, po)
+        assert np.array_equal(ref["bytes"], gpu_bytes), "independent oracle chain differs"
+        rep["bytes_identical"] = True
+    return rep
+
+
+def check_decode(p: api.AnchorKVParams, layouts: list, q: np.ndarray, Kt, Vt, tail_len: int,
+                 out: np.ndarray, tol: float) -> float:
+    """Decode attention of every sequence vs the oracle on the GPU's layout."""
+    po = oracle_params(p)
+    worst = 0.0
+    for b, buf in enumerate(layouts):
+        parts = O.unpack_layout(buf, po)
+        Kh, Vh = O.reconstruct(parts, po)
+        kt = Kt[b][:, :tail_len] if tail_len else None
+        vt = Vt[b][:, :tail_len] if tail_len else None
+        o = O.decode_attention(q[b], Kh, Vh, kt, vt)
+        worst = max(worst, float(np.abs(o - out[b]).max()))
+    assert worst <= tol, f"decode max-abs error {worst} > {tol}"
+    return worst

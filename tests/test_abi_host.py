@@ -1,0 +1,92 @@
+"""The C-ABI library loads, exports what include/anchorkv.h declares, and its
+host-side (pure) functions agree with the oracle.  No GPU needed."""
+import ctypes
+import math
+
+import pytest
+
+from kv_cache_compression_anchorkv_b200 import api, capi
+from oracle import anchorkv_oracle as O
+
+
+def test_library_exports_every_declared_symbol():
+    L = capi.lib()
+    names = capi.header_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(capi._SIGS), "binding and header disagree"
+
+
+def test_struct_sizes_match_header_layout():
+    assert ctypes.sizeof(capi.Params) == 4 * 6 + 8 + 8 + 4 * 6
+    assert ctypes.sizeof(capi.Layout) == 8 * 7 + 4 * 4 + 8 * 8
+
+
+CASES = [
+    (1024, 1, 4, 0.1, "fp32"), (32768, 8, 32, 0.05, "bf16"), (131072, 8, 64, 0.05, "bf16"),
+    (32768, 8, 32, 0.1, "bf16"), (8192, 8, 32, 0.2, "bf16"), (3000, 2, 8, 0.1, "bf16"),
+    (33, 1, 2, 0.5, "bf16"), (256, 1, 4, 0.05, "bf16"), (777, 2, 4, 1.0, "fp32"), (5000, 3, 6, 0.07, "bf16"),
+]
+
+
+@pytest.mark.parametrize("N,H,Hq,theta,dtype", CASES)
+def test_byte_accounting_matches_oracle(N, H, Hq, theta, dtype):
+    p = api.AnchorKVParams(n_tokens=N, n_kv_heads=H, n_q_heads=Hq, theta=theta, dtype=dtype)
+    got = api.anchorkv_bytes(p)
+    want = O.layout(O.Params(n_tokens=N, n_kv_heads=H, n_q_heads=Hq, theta=theta, dtype=dtype))
+    assert got["total_bytes"] == want["total"]
+    assert got["base_bytes"] == want["base"]
+    assert got["budget_bytes"] == want["B"]
+    assert got["n_residuals"] == want["R"]
+    assert got["residual_cap"] == want["cap"]
+    assert got["n_anchors"] == want["k"]
+    assert got["n_scored"] == want["n_s"] and got["n_uniform"] == want["n_u"]
+    for name, off in want["off"].items():
+        assert got["off_" + name.lower()] == off, name
+
+
+@pytest.mark.parametrize("field,value", [
+    ("head_dim", 64), ("n_kv_heads", 0), ("n_q_heads", 12), ("window", 0), ("n_tokens", 32),
+    ("theta", 0.0), ("theta", float("nan")), ("theta", -1.0), ("pool_kernel", 6), ("rho_num", 11),
+    ("layer", -1), ("anchor_div", 0)])
+def test_invalid_params_rejected(field, value):
+    p = api.AnchorKVParams(n_tokens=1024, n_kv_heads=8, n_q_heads=32)
+    setattr(p, field, value)
+    with pytest.raises(capi.AnchorKVError) as e:
+        api.anchorkv_bytes(p)
+    assert e.value.status in (capi.EINVAL, capi.EUNSUPPORTED)
+
+
+def test_null_arguments_are_errors_not_crashes():
+    L = capi.lib()
+    assert L.anchorkv_bytes(None, None) == capi.EINVAL
+    p = api.AnchorKVParams(n_tokens=1024).c()
+    assert L.anchorkv_compress(ctypes.byref(p), None, None, None, None, 0, None, 0, None) == capi.EINVAL
+    n = ctypes.c_size_t()
+    assert L.anchorkv_decode_workspace_bytes(ctypes.byref(p), -1, ctypes.byref(n)) == capi.EINVAL
+    assert L.anchorkv_read_device_status(None, None, None) == capi.EINVAL
+    assert L.anchorkv_strerror(capi.ENOSPC) == b"buffer too small"
+
+
+def test_small_output_buffer_is_enospc():
+    L = capi.lib()
+    p = api.AnchorKVParams(n_tokens=1024).c()
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: size check fails first
+    st = L.anchorkv_compress(ctypes.byref(p), fake, fake, fake, fake, 16, fake, 16, None)
+    assert st == capi.ENOSPC
+
+
+def test_library_codebook_matches_oracle():
+    tau, l1, l2, mse = api.codebook()
+    o = O.lloyd_max_gaussian_4()
+    for a, b in zip((tau, l1, l2, mse), o):
+        assert abs(a - b) < 1e-13
+
+
+def test_workspace_view():
+    p = api.AnchorKVParams(n_tokens=32768)
+    v = api.compress_workspace(p)
+    assert v["total_bytes"] > v["off_utility"] + 4 * 2 * 8 * 32768
+    assert v["off_counters"] % 256 == 0 and v["off_pooled"] % 256 == 0
+    assert api.decode_workspace_bytes(p, 16) > api.decode_workspace_bytes(p, 1) > 0

@@ -1,0 +1,153 @@
+"""CUDA path vs the oracle, through the C ABI, on seeded synthetic caches."""
+import numpy as np
+import pytest
+import torch
+
+from kv_cache_compression_anchorkv_b200 import api, capi
+from kv_cache_compression_anchorkv_b200.synthetic import (CacheSpec, make_decode_queries, make_layer,
+                                                           make_tail)
+from oracle import anchorkv_oracle as O
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+DECODE_TOL = {"bf16": 2e-3, "fp32": 1e-5}
+
+
+def _params(spec: CacheSpec, theta, layer=0):
+    return api.AnchorKVParams(n_tokens=spec.n_tokens, n_kv_heads=spec.n_kv_heads, n_q_heads=spec.n_q_heads,
+                              theta=theta, window=spec.window, dtype=spec.dtype, seed=spec.seed, layer=layer)
+
+
+def _f64(x):
+    return x.detach().cpu().double().numpy()
+
+
+CASES = {
+    # name: (spec, theta)
+    "tiny-fp32-n1024": (CacheSpec(1, 1, 4, 1024, dtype="fp32", n_dirs=32, seed=0), 0.1),
+    "bf16-ragged-n3000": (CacheSpec(1, 2, 8, 3000, n_dirs=64, seed=1), 0.1),
+    "bf16-gqa8-n2500": (CacheSpec(1, 2, 16, 2500, n_dirs=64, seed=2), 0.15),
+    "bf16-every-residual": (CacheSpec(1, 1, 4, 1100, n_dirs=16, seed=3), 1.0),
+    "bf16-no-residual": (CacheSpec(1, 2, 4, 1000, n_dirs=16, seed=4), 0.01),
+    "fp32-all-anchors": (CacheSpec(1, 2, 4, 33, dtype="fp32", n_dirs=8, seed=5), 0.5),
+    "fp32-window8-n700": (CacheSpec(1, 3, 3, 700, window=8, dtype="fp32", n_dirs=8, seed=6), 0.3),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_compress_parity(name):
+    spec, theta = CASES[name]
+    K, V, Q = make_layer(spec, 0)
+    p = _params(spec, theta, layer=3)
+    gb, gpool, gutil, counters = parity.gpu_compress(p, K, V, Q)
+    assert counters[0] == 0
+    rep = parity.check_compress(p, _f64(K), _f64(V), _f64(Q), gb, gpool, gutil)
+    print(name, rep, "refined rows:", counters[1])
+
+
+def test_compress_exact_ties():
+    """Duplicate rows and zero rows make exact ties: lowest slot / lowest index."""
+    spec = CacheSpec(1, 1, 4, 600, n_dirs=8, seed=7)
+    K, V, Q = make_layer(spec, 0)
+    K[0, 100:140] = K[0, 10]          # many keys identical to one another
+    V[0, 200:260] = V[0, 20]
+    K[0, 300:310] = 0.0               # zero keys: every cosine 0 -> slot 0, gamma 0
+    V[0, 400:405] = 0.0
+    p = _params(spec, 0.3)
+    gb, gpool, gutil, counters = parity.gpu_compress(p, K, V, Q)
+    rep = parity.check_compress(p, _f64(K), _f64(V), _f64(Q), gb, gpool, gutil)
+    g = O.unpack_layout(gb, parity.oracle_params(p))
+    assert np.all(g["idx"][0, 0, 300:310] == 0) or 300 in g["anchor_pos"][0]
+    print(rep)
+
+
+def test_compress_deterministic():
+    spec, theta = CASES["bf16-ragged-n3000"]
+    K, V, Q = (x.cuda() for x in make_layer(spec, 0))
+    p = _params(spec, theta)
+    a, _ = api.compress(p, K, V, Q)
+    b, _ = api.compress(p, K, V, Q)
+    assert torch.equal(a, b)
+
+
+def test_reconstruct_matches_oracle():
+    spec, theta = CASES["bf16-ragged-n3000"]
+    K, V, Q = make_layer(spec, 0)
+    p = _params(spec, theta)
+    out, _ = api.compress(p, K.cuda(), V.cuda(), Q.cuda())
+    Kh, Vh = api.reconstruct(p, out)
+    parts = O.unpack_layout(out.cpu().numpy(), parity.oracle_params(p))
+    Ko, Vo = O.reconstruct(parts, parity.oracle_params(p))
+    assert np.abs(Kh.cpu().double().numpy() - Ko).max() < 1e-5 * max(1.0, np.abs(Ko).max())
+    assert np.abs(Vh.cpu().double().numpy() - Vo).max() < 1e-5 * max(1.0, np.abs(Vo).max())
+    # anchors reconstruct bit for bit
+    ap = parts["anchor_pos"]
+    for h in range(p.n_kv_heads):
+        assert torch.equal(Kh[h][ap[h]].cpu(), K[h][ap[h]].float())
+
+
+@pytest.mark.parametrize("name,batch,tail", [("tiny-fp32-n1024", 1, 0), ("tiny-fp32-n1024", 2, 5),
+                                             ("bf16-ragged-n3000", 3, 17), ("bf16-gqa8-n2500", 2, 0),
+                                             ("bf16-every-residual", 1, 3), ("bf16-no-residual", 2, 1),
+                                             ("fp32-all-anchors", 1, 2)])
+def test_decode_parity(name, batch, tail):
+    spec, theta = CASES[name]
+    p = _params(spec, theta)
+    L = api.anchorkv_bytes(p)
+    stride = (L["total_bytes"] + 255) // 256 * 256
+    comp = torch.zeros(batch, stride, dtype=torch.uint8, device="cuda")
+    layouts = []
+    for b in range(batch):
+        sb = CacheSpec(**{**spec.__dict__, "seed": spec.seed + 100 * b})
+        K, V, Q = make_layer(sb, 0)
+        out, _ = api.compress(p, K.cuda(), V.cuda(), Q.cuda())
+        comp[b, :L["total_bytes"]] = out
+        layouts.append(out.cpu().numpy())
+    q = make_decode_queries(spec, 0, step=0, batch=batch)
+    cap = max(tail, 1) + 3
+    Kt, Vt = make_tail(spec, 0, cap, batch=batch)
+    o = api.decode_attn(p, comp, q.cuda(), Kt.cuda(), Vt.cuda(), tail_len=tail)
+    err = parity.check_decode(p, layouts, _f64(q), _f64(Kt), _f64(Vt), tail, o.cpu().double().numpy(),
+                              DECODE_TOL[spec.dtype])
+    print(name, batch, tail, "max abs err", err)
+
+
+def test_error_paths_on_device():
+    spec, theta = CASES["bf16-ragged-n3000"]
+    K, V, Q = (x.cuda() for x in make_layer(spec, 0))
+    p = _params(spec, theta)
+    L = api.anchorkv_bytes(p)
+    small = torch.empty(L["total_bytes"] - 1, dtype=torch.uint8, device="cuda")
+    with pytest.raises(capi.AnchorKVError) as e:
+        api.compress(p, K, V, Q, out=small)
+    assert e.value.status == capi.ENOSPC
+    buf = torch.empty(K.numel() * 2 + 64, dtype=torch.uint8, device="cuda")
+    lib = capi.lib()
+    ws = torch.empty(api.compress_workspace(p)["total_bytes"], dtype=torch.uint8, device="cuda")
+    out = torch.empty(L["total_bytes"], dtype=torch.uint8, device="cuda")
+    import ctypes
+    st = lib.anchorkv_compress(ctypes.byref(p.c()), ctypes.c_void_p(buf.data_ptr() + 2), ctypes.c_void_p(V.data_ptr()),
+                               ctypes.c_void_p(Q.data_ptr()), ctypes.c_void_p(out.data_ptr()), out.numel(),
+                               ctypes.c_void_p(ws.data_ptr()), ws.numel(), None)
+    assert st == capi.EINVAL
+    assert api.decode_attn(p, torch.zeros(0, 16, dtype=torch.uint8, device="cuda"),
+                           torch.zeros(0, p.n_q_heads, 128, dtype=torch.bfloat16, device="cuda")).shape[0] == 0
+
+
+@pytest.mark.slow
+def test_full_size_layer_llama8b_shape():
+    """One layer of the 8B-shaped cache (8 KV / 32 Q heads, N = 32768, bf16,
+    theta = 0.05), generated on the device as the benchmark does, checked
+    against the oracle in full (every head, both sides), plus a batch-1 decode."""
+    spec = CacheSpec(32, 8, 32, 32768, n_dirs=128, seed=0)
+    layer = 5
+    K, V, Q = make_layer(spec, layer, device="cuda")
+    p = _params(spec, 0.05, layer=layer)
+    gb, gpool, gutil, counters = parity.gpu_compress(p, K, V, Q)
+    rep = parity.check_compress(p, _f64(K), _f64(V), _f64(Q), gb, gpool, gutil, full_chain=False)
+    print("full-size layer", rep, "refined rows:", counters[1])
+    q = make_decode_queries(spec, layer, step=0, batch=1, device="cuda")
+    comp = torch.from_numpy(gb).cuda()
+    o = api.decode_attn(p, comp, q)
+    parity.check_decode(p, [gb], _f64(q), None, None, 0, o.cpu().double().numpy(), DECODE_TOL["bf16"])
