@@ -108,6 +108,7 @@ def main():
     ap.add_argument("--impl", default="anchorkv", choices=["anchorkv", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layers", type=int, default=0, help="compress only the first L layers (profiling runs)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -198,6 +199,8 @@ def run_gpu(args, world, rank, local):
     wl = WORKLOADS[WORKLOAD]
     spec, theta = wl["spec"], wl["theta"]
     spec = type(spec)(**{**spec.__dict__, "seed": spec.seed + rank})     # an independent cache per rank
+    if args.layers:
+        spec = type(spec)(**{**spec.__dict__, "n_layers": min(args.layers, spec.n_layers)})
     Lr, H, N = spec.n_layers, spec.n_kv_heads, spec.n_tokens
 
     cpu_base = None

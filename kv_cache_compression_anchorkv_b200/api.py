@@ -181,7 +181,7 @@ class HostCompressor:
         return self.host_out
 
 
-N_STAGES = 12
+N_STAGES = 14
 
 
 def stage_timing(enable: bool) -> None:

@@ -78,8 +78,9 @@ anchor_select_kernel(const float* __restrict__ score, float* __restrict__ pooled
                      int n_s, int n_u, int k, int all_anchors, unsigned long long seed, int layer,
                      const T* __restrict__ K, const T* __restrict__ V, T* __restrict__ anc_k,
                      T* __restrict__ anc_v, int* __restrict__ anchor_pos, int* __restrict__ slot_of,
-                     double* __restrict__ anc_n2, float* __restrict__ anc_inv, int* __restrict__ counters,
-                     int H, PadList pads) {
+                     double* __restrict__ anc_n2, double* __restrict__ anc_sqrt, float* __restrict__ anc_inv,
+                     int* __restrict__ counters,
+                     int H, int kp16, int obs_rb, PadList pads) {
   __shared__ SelSmem sm;
   const int h = blockIdx.x;
   const int tid = threadIdx.x;
@@ -89,18 +90,22 @@ anchor_select_kernel(const float* __restrict__ score, float* __restrict__ pooled
     if (b < pads.len[i]) pads.base[pads.off[i] + b] = 0;
   }
   const int NW = N - W;
-  const float* sc = score + (int64_t)h * N;
   float* pl = pooled + (int64_t)h * N;
   int* flag = slot_of + (int64_t)h * N;       // flags first, slots after compaction
 
-  // 1. pooling (zero padding outside [0, N-W), divide by kappa)
+  // 1. pooling (zero padding outside [0, N-W), divide by kappa); the score of
+  //    a position is the sum of its observation-row-block partials, in order
   const int half = kappa / 2;
   for (int t = tid; t < N; t += kThreads) {
     if (t < NW) {
       float acc = 0.f;
       for (int d = -half; d <= half; ++d) {
         const int u = t + d;
-        if (u >= 0 && u < NW) acc += sc[u];
+        if (u >= 0 && u < NW) {
+          float s = score[(int64_t)h * N + u];
+          for (int rb = 1; rb < obs_rb; ++rb) s += score[((int64_t)rb * H + h) * N + u];
+          acc += s;
+        }
       }
       pl[t] = acc / (float)kappa;
     }
@@ -253,9 +258,15 @@ anchor_select_kernel(const float* __restrict__ score, float* __restrict__ pooled
       if (lane == 0) {
         const int64_t ai = ((int64_t)side * H + h) * k + s;
         anc_n2[ai] = n2;
-        anc_inv[ai] = (n2 > 0.0) ? (float)(1.0 / sqrt(n2)) : 0.f;
+        anc_sqrt[ai] = sqrt(n2);
+        anc_inv[((int64_t)side * H + h) * kp16 + s] = (n2 > 0.0) ? (float)(1.0 / sqrt(n2)) : 0.f;
       }
     }
+  }
+  // 1/||a|| rows are padded to a multiple of 16 slots with zeros
+  for (int i = tid; i < 2 * (kp16 - k); i += kThreads) {
+    const int side = i / (kp16 - k), s = k + i % (kp16 - k);
+    anc_inv[((int64_t)side * H + h) * kp16 + s] = 0.f;
   }
 }
 
@@ -268,6 +279,7 @@ cudaError_t launch_anchor_select(const Plan& pl, const void* K, const void* V, c
   auto* slot_of = reinterpret_cast<int*>(ws + pl.o_slot_of);
   auto* n2 = reinterpret_cast<double*>(ws + pl.o_anc_n2);
   auto* inv = reinterpret_cast<float*>(ws + pl.o_anc_inv);
+  auto* sq = reinterpret_cast<double*>(ws + pl.o_anc_sqrt);
   auto* cnt = reinterpret_cast<int*>(ws + pl.o_counters);
   // section ends and the next 16-byte boundary
   const int64_t H = pl.H, N = pl.N, k = pl.k, D = kD;
@@ -286,13 +298,13 @@ cudaError_t launch_anchor_select(const Plan& pl, const void* K, const void* V, c
         score, pooled, pl.N, pl.W, pl.p.pool_kernel, pl.n_s, pl.n_u, pl.k, pl.all_anchors ? 1 : 0,
         pl.p.seed, pl.p.layer, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
         reinterpret_cast<__nv_bfloat16*>(out + pl.L.off_anchors_k),
-        reinterpret_cast<__nv_bfloat16*>(out + pl.L.off_anchors_v), apos, slot_of, n2, inv, cnt, pl.H, pads);
+        reinterpret_cast<__nv_bfloat16*>(out + pl.L.off_anchors_v), apos, slot_of, n2, sq, inv, cnt, pl.H, pl.kp16, pl.obs_rb, pads);
   } else {
     anchor_select_kernel<float><<<pl.H, kThreads, 0, s>>>(
         score, pooled, pl.N, pl.W, pl.p.pool_kernel, pl.n_s, pl.n_u, pl.k, pl.all_anchors ? 1 : 0,
         pl.p.seed, pl.p.layer, (const float*)K, (const float*)V,
         reinterpret_cast<float*>(out + pl.L.off_anchors_k), reinterpret_cast<float*>(out + pl.L.off_anchors_v),
-        apos, slot_of, n2, inv, cnt, pl.H, pads);
+        apos, slot_of, n2, sq, inv, cnt, pl.H, pl.kp16, pl.obs_rb, pads);
   }
   return cudaGetLastError();
 }

@@ -1,6 +1,7 @@
 // C-ABI entry points: parameter checks, the byte accounting, workspace plans
 // and the launch sequence of one compress / decode call.
 #include <math.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -112,6 +113,7 @@ int make_plan(const anchorkv_params* p, Plan* pl) {
   st = fill_layout(p, &pl->L, &n_s, &n_u, &all);
   if (st) return st;
   if (n_u > 2048) return ANCHORKV_EUNSUPPORTED;          // uniform-sample candidate buffer
+  if (pl->L.n_anchors > 2048) return ANCHORKV_EUNSUPPORTED;   // fp64 re-decision score buffer
   pl->N = p->n_tokens; pl->D = p->head_dim; pl->H = p->n_kv_heads; pl->Hq = p->n_q_heads;
   pl->G = pl->Hq / pl->H; pl->W = p->window; pl->GW = pl->G * pl->W;
   pl->k = pl->L.n_anchors; pl->n_s = n_s; pl->n_u = n_u; pl->n_tiles = pl->L.n_tiles;
@@ -120,24 +122,47 @@ int make_plan(const anchorkv_params* p, Plan* pl) {
   pl->all_anchors = all;
   pl->chunk1 = 1024;
   pl->n_chunk1 = (pl->N + pl->chunk1 - 1) / pl->chunk1;
+  // tensor-core observation passes: 128-row blocks, token range split so
+  // that the (head, row block, split) items fill the SMs about once
+  pl->tc_rb = (pl->GW + 127) / 128;
+  {
+    const int units = pl->H * pl->tc_rb, row_tiles = (pl->N + 127) / 128;
+    const int want = std::max(1, (148 + units - 1) / units);
+    pl->tc_tps = std::max(1, (row_tiles + want - 1) / want);
+    pl->tc_split = (row_tiles + pl->tc_tps - 1) / pl->tc_tps;
+  }
+  pl->obs_rb = 1;
   const int64_t H = pl->H, N = pl->N, GW = pl->GW, k = pl->k, D = kD;
   const int64_t n_sh_t = 2 * H * pl->n_tiles;
+  const int64_t U = H * pl->tc_rb, nrb = pl->tc_rb;
   int64_t off = 0;
   auto take = [&](int64_t bytes) { int64_t o = off; off += (bytes + 255) / 256 * 256; return o; };
-  pl->o_counters = take(4 * kCounterCount);
+  pl->o_counters = take(4 * (kCounterCount + 2 * H));
   pl->o_row_m = take(4 * H * GW);
   pl->o_row_z = take(4 * H * GW);
   pl->o_ybar = take(4 * H * GW * D);
   pl->o_part_m = take(4 * H * pl->n_chunk1 * GW);
   pl->o_part_l = take(4 * H * pl->n_chunk1 * GW);
   pl->o_part_y = take(4 * H * pl->n_chunk1 * GW * D);
-  pl->o_score = take(4 * H * N);
-  pl->o_a2 = take(4 * H * N);
-  pl->o_ku = take(4 * H * N);
+  pl->o_tc_pm2 = take(4 * U * pl->tc_split * 128);
+  pl->o_tc_pl = take(4 * U * pl->tc_split * 128);
+  pl->o_tc_rm2 = take(4 * U * 128);
+  pl->o_tc_riz = take(4 * U * 128);
+  pl->o_tc_rq2 = take(4 * U * 128);
+  pl->o_tc_ry2 = take(4 * U * 128);
+  pl->o_tc_py = take(4 * U * pl->tc_split * 128 * 128);
+  pl->o_tc_yh = take(2 * U * 128 * 128);
+  pl->o_tc_yl = take(2 * U * 128 * 128);
+  pl->o_score = take(4 * nrb * H * N);
+  pl->o_a2 = take(4 * nrb * H * N);
+  pl->o_ku = take(4 * nrb * H * N);
   pl->o_pooled = take(4 * H * N);
   pl->o_slot_of = take(4 * H * N);
   pl->o_anc_n2 = take(8 * 2 * H * k);
-  pl->o_anc_inv = take(4 * 2 * H * k);
+  pl->kp16 = (pl->k + 15) / 16 * 16;
+  pl->o_anc_inv = take(4 * 2 * H * pl->kp16);
+  pl->o_anc_sqrt = take(8 * 2 * H * k);
+  pl->o_xnorm = take(4 * 2 * H * N);
   pl->o_util = take(4 * 2 * H * N);
   pl->o_refine = take(4 * 2 * H * N);
   pl->o_sel_state = take(64);
@@ -155,6 +180,23 @@ int make_plan(const anchorkv_params* p, Plan* pl) {
     if (z & 1ull) pl->sign_bits[j >> 5] |= 1u << (j & 31);
   }
   return ANCHORKV_OK;
+}
+
+// The tensor-core assignment runs for bf16 caches whose anchors fit in
+// shared memory; ANCHORKV_SIMT_ASSIGN=1 forces the SIMT path (tests use it to
+// compare the two).
+static bool use_tc_assign(const Plan& pl) {
+  const char* e = getenv("ANCHORKV_SIMT_ASSIGN");
+  if (e && e[0] == '1') return false;
+  return assign_tc_supported(pl);
+}
+
+// The tensor-core observation passes run for bf16 caches;
+// ANCHORKV_SIMT_OBS=1 forces the SIMT passes.
+static bool use_tc_obs(const Plan& pl) {
+  const char* e = getenv("ANCHORKV_SIMT_OBS");
+  if (e && e[0] == '1') return false;
+  return obs_tc_supported(pl);
 }
 
 static int check_device() {
@@ -230,14 +272,24 @@ int anchorkv_compress(const anchorkv_params* p, const void* K, const void* V, co
   cudaStream_t s = (cudaStream_t)stream;
   char* o = (char*)out;
   char* w = (char*)ws;
-  AKV_LAUNCH(cudaMemsetAsync(w + pl.o_counters, 0, 4 * kCounterCount, s));
+  AKV_LAUNCH(cudaMemsetAsync(w + pl.o_counters, 0, 4 * (kCounterCount + 2 * (size_t)pl.H), s));
 #define AKV_STAGE(st, nk, expr) \
   do { stage_begin(st, s); AKV_LAUNCH(expr); stage_end(st, s, nk); } while (0)
-  AKV_STAGE(kStObsPass1, 1, launch_obs_pass1(pl, K, V, Q_obs, w, s));
-  AKV_STAGE(kStObsCombine, 1, launch_obs_combine(pl, w, s));
-  AKV_STAGE(kStTokenStats, 1, launch_token_stats(pl, K, V, Q_obs, w, s));
+  if (use_tc_obs(pl)) {
+    pl.obs_rb = pl.tc_rb;
+    AKV_LAUNCH(launch_obs_tc(pl, K, V, Q_obs, w, s));
+  } else {
+    pl.obs_rb = 1;
+    AKV_STAGE(kStObsPass1, 1, launch_obs_pass1(pl, K, V, Q_obs, w, s));
+    AKV_STAGE(kStObsCombine, 1, launch_obs_combine(pl, w, s));
+    AKV_STAGE(kStTokenStats, 1, launch_token_stats(pl, K, V, Q_obs, w, s));
+  }
   AKV_STAGE(kStAnchorSelect, 1, launch_anchor_select(pl, K, V, o, w, s));
-  AKV_STAGE(kStAssign, 1, launch_assign_simt(pl, K, V, o, w, s));
+  if (use_tc_assign(pl)) {
+    AKV_STAGE(kStAssign, 1, launch_assign_tc(pl, K, V, o, w, s));
+  } else {
+    AKV_STAGE(kStAssign, 1, launch_assign_simt(pl, K, V, o, w, s));
+  }
   AKV_STAGE(kStRefine, 1, launch_refine(pl, K, V, o, w, s));
   AKV_STAGE(kStProject, 1, launch_project(pl, K, V, o, w, s));
   const int sel_kernels = pl.R == 0 ? 0 : (pl.R == pl.cap ? 5 : 13);

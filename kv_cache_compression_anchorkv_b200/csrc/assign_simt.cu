@@ -14,6 +14,8 @@
 // Rows closer than that are listed and re-decided by refine_kernel from exact
 // fp64 dots (bf16 and fp32 products are exact in fp64), which takes the
 // decision in the same precision as a float64 restatement of the rule.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -32,38 +34,19 @@ struct AsgSmem {
   float xn[kTM];
 };
 
-struct Best {
-  float b1, b2;
-  int i1;
-};
-
-__device__ __forceinline__ void best_push(Best& b, float v, int i) {
-  // slots arrive in ascending order within a thread: strict > keeps the lowest
-  if (v > b.b1) { b.b2 = b.b1; b.b1 = v; b.i1 = i; }
-  else if (v > b.b2) { b.b2 = v; }
-}
-
-__device__ __forceinline__ Best best_merge(const Best& a, const Best& b) {
-  const bool a_wins = (a.b1 > b.b1) || (a.b1 == b.b1 && a.i1 < b.i1);
-  Best w = a_wins ? a : b;
-  const Best& l = a_wins ? b : a;
-  w.b2 = fmaxf(w.b2, l.b1);
-  return w;
-}
-
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 assign_simt_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ anc_k,
                    const T* __restrict__ anc_v, const float* __restrict__ anc_inv,
                    const int* __restrict__ slot_of, uint32_t* __restrict__ tok, int* __restrict__ refine,
-                   int* __restrict__ counters, int N, int H, int k) {
+                   int* __restrict__ counters, int N, int H, int k, int kp16) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   AsgSmem& sm = *reinterpret_cast<AsgSmem*>(smem_raw);
   const int t0 = blockIdx.x * kTM, h = blockIdx.y, side = blockIdx.z;
   const int nv = min(kTM, N - t0);
   const T* X = (side ? V : K) + (int64_t)h * N * kD;
   const T* A = (side ? anc_v : anc_k) + (int64_t)h * k * kD;
-  const float* inv = anc_inv + ((int64_t)side * H + h) * k;
+  const float* inv = anc_inv + ((int64_t)side * H + h) * kp16;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
 
   for (int i = tid; i < kTM * (kD / 4); i += kThreads) {
@@ -78,8 +61,8 @@ assign_simt_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __
     for (int d = 0; d < kD; ++d) s = fmaf(sm.xs[d][tid], sm.xs[d][tid], s);
     sm.xn[tid] = sqrtf(s);
   }
-  Best best[4];
-  for (int i = 0; i < 4; ++i) best[i] = Best{-INFINITY, -INFINITY, 0x7fffffff};
+  Top3 best[4];
+  for (int i = 0; i < 4; ++i) best[i] = top3_init();
 
   for (int a0 = 0; a0 < k; a0 += kTN) {
     const int na = min(kTN, k - a0);
@@ -111,20 +94,22 @@ assign_simt_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __
       if (a >= na) continue;
       const float iv = sm.inv[a];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) best_push(best[i], acc[i][j] * iv, a0 + a);
+      for (int i = 0; i < 4; ++i) push(best[i], acc[i][j] * iv, a0 + a);
     }
   }
   // merge across the 16 threads (tx) that share the same 4 tokens
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    Best b = best[i];
+    Top3 b = best[i];
 #pragma unroll
     for (int o = 8; o; o >>= 1) {
-      Best other;
+      Top3 other;
       other.b1 = __shfl_xor_sync(0xffffffffu, b.b1, o);
       other.b2 = __shfl_xor_sync(0xffffffffu, b.b2, o);
+      other.b3 = __shfl_xor_sync(0xffffffffu, b.b3, o);
       other.i1 = __shfl_xor_sync(0xffffffffu, b.i1, o);
-      b = best_merge(b, other);
+      other.i2 = __shfl_xor_sync(0xffffffffu, b.i2, o);
+      b = merge(b, other);
     }
     best[i] = b;
   }
@@ -140,48 +125,121 @@ assign_simt_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __
         slot = (uint32_t)own;
       } else {
         slot = (uint32_t)best[i].i1;
-        if (!(best[i].b1 - best[i].b2 > kRefineRel * sm.xn[r])) {
-          const int at = atomicAdd(&counters[kRefineRows], 1);
-          refine[at] = (side * H + h) * N + t;
-        }
+        if (!(best[i].b1 - best[i].b2 > kRefineRel * sm.xn[r])) list_for_refine(refine, counters, side * H + h, N, t);
       }
       tok[((int64_t)side * H + h) * N + t] = slot;
     }
   }
 }
 
-// One warp per listed row: exact fp64 dots against every anchor.
+// Re-decision of the listed rows of one (side, head) per blockIdx.y.
+// The block stages the head's anchors in shared memory transposed as
+// (d, d+1) pairs per slot, so that lanes scoring consecutive slots read
+// consecutive words.  Each warp takes one row: fp32 scores of every slot
+// (sequential FMA over D = 128 exact products: error <= 2^-17 ||x|| after
+// scaling), candidates within 2^-14 ||x|| of the best fp32 score, and the
+// exact fp64 score dot / sqrt(||a||^2) of each candidate (correctly rounded
+// sqrt and division) decides; ties go to the lowest slot.
+constexpr int kRefineWarps = 8;
+constexpr int kRefineMaxK = 2048;
+template <typename T> struct RefineCfg;
+template <> struct RefineCfg<__nv_bfloat16> { using P = __nv_bfloat162; static constexpr int kChunk = 448; };
+template <> struct RefineCfg<float> { using P = float2; static constexpr int kChunk = 192; };
+
+__device__ __forceinline__ float2 pair_f(__nv_bfloat162 p) { return __bfloat1622float2(p); }
+__device__ __forceinline__ float2 pair_f(float2 p) { return p; }
+
 template <typename T>
-__global__ void refine_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ anc_k,
-                              const T* __restrict__ anc_v, const double* __restrict__ anc_n2,
-                              const int* __restrict__ refine, const int* __restrict__ counters,
-                              uint32_t* __restrict__ tok, int N, int H, int k) {
-  const int lane = threadIdx.x & 31;
-  const int n_list = counters[kRefineRows];
-  for (int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); i < n_list;
-       i += gridDim.x * (blockDim.x >> 5)) {
-    const int f = refine[i];
-    const int side = f / (H * N), h = (f / N) % H, t = f % N;
+__global__ void __launch_bounds__(kRefineWarps * 32)
+refine_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ anc_k,
+              const T* __restrict__ anc_v, const float* __restrict__ anc_inv, const double* __restrict__ anc_sqrt,
+              const int* __restrict__ refine, const int* __restrict__ counters, uint32_t* __restrict__ tok, int N,
+              int H, int k, int kp16) {
+  using P = typename RefineCfg<T>::P;
+  constexpr int CH = RefineCfg<T>::kChunk;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  P* aT = reinterpret_cast<P*>(smem_raw);                              // [64][CH]
+  float* xs = reinterpret_cast<float*>(aT + 64 * CH);                  // [8][128]
+  float* sc = xs + kRefineWarps * kD;                                  // [8][kRefineMaxK]
+  const int u = blockIdx.y, side = u / H, h = u % H;
+  const int n = counters[kRefineListBase + u];
+  if ((int)blockIdx.x * kRefineWarps >= n) return;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const T* A = (side ? anc_v : anc_k) + (int64_t)h * k * kD;
+  const float* inv = anc_inv + (int64_t)u * kp16;
+  const double* sq = anc_sqrt + (int64_t)u * k;
+  float* xw = xs + w * kD;
+  float* sw = sc + w * kRefineMaxK;
+  auto stage = [&](int c0, int cn) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < cn * 64; i += blockDim.x) {
+      const int j = i / 64, dp = i % 64;
+      const T* src = A + (int64_t)(c0 + j) * kD + 2 * dp;
+      aT[dp * CH + j] = *reinterpret_cast<const P*>(src);
+    }
+    __syncthreads();
+  };
+  const bool one_chunk = k <= CH;
+  if (one_chunk) stage(0, k);
+  for (int base = blockIdx.x * kRefineWarps; base < n; base += gridDim.x * kRefineWarps) {
+    const int i = base + w;
+    const bool live = i < n;
+    const int t = live ? refine[(int64_t)u * N + i] : 0;
     const T* x = (side ? V : K) + ((int64_t)h * N + t) * kD;
-    const T* A = (side ? anc_v : anc_k) + (int64_t)h * k * kD;
-    const double* n2 = anc_n2 + ((int64_t)side * H + h) * k;
     float xf[4];
     load4<T>(x + lane * 4, xf);
-    double best = -INFINITY;
-    int bi = 0;
-    for (int s = 0; s < k; ++s) {
-      float af[4];
-      load4<T>(A + (int64_t)s * kD + lane * 4, af);
-      double d = 0.0;
+    __syncwarp();
 #pragma unroll
-      for (int e = 0; e < 4; ++e) d = fma((double)xf[e], (double)af[e], d);
-      d = warp_sum_d(d);
-      const double nn = n2[s];
-      const double c = (nn > 0.0) ? d / sqrt(nn) : 0.0;
-      if (c > best) { best = c; bi = s; }
+    for (int e = 0; e < 4; ++e) xw[lane * 4 + e] = xf[e];
+    const float xn = sqrtf(warp_sum(xf[0] * xf[0] + xf[1] * xf[1] + xf[2] * xf[2] + xf[3] * xf[3]));
+    __syncwarp();
+    float best = -INFINITY;
+    for (int c0 = 0; c0 < k; c0 += CH) {
+      const int cn = min(CH, k - c0);
+      if (!one_chunk) stage(c0, cn);
+      for (int j = lane; j < cn; j += 32) {
+        float acc = 0.f;
+#pragma unroll 8
+        for (int dp = 0; dp < 64; ++dp) {
+          const float2 av = pair_f(aT[dp * CH + j]);
+          acc = fmaf(xw[2 * dp], av.x, acc);
+          acc = fmaf(xw[2 * dp + 1], av.y, acc);
+        }
+        const float s = acc * inv[c0 + j];
+        sw[c0 + j] = s;
+        best = fmaxf(best, s);
+      }
     }
-    if (lane == 0) tok[f] = (uint32_t)bi;
+    best = warp_max(best);
+    __syncwarp();
+    const float thr = best - xn * (1.0f / 16384.0f);
+    double cbest = -INFINITY;
+    int cbi = 0x7fffffff;
+    for (int j0 = 0; j0 < k; j0 += 32) {
+      const int j = j0 + lane;
+      uint32_t cand = __ballot_sync(0xffffffffu, j < k && sw[j] >= thr);
+      while (cand) {
+        const int s = j0 + __ffs(cand) - 1;
+        cand &= cand - 1;
+        float af[4];
+        load4<T>(A + (int64_t)s * kD + lane * 4, af);
+        double d = 0.0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) d = fma((double)xf[e], (double)af[e], d);
+        d = warp_sum_d(d);
+        const double nn = sq[s];
+        const double cs = (nn > 0.0) ? d / nn : 0.0;
+        if (cs > cbest) { cbest = cs; cbi = s; }
+      }
+    }
+    if (live && lane == 0 && cbi < k) tok[(int64_t)u * N + t] = (uint32_t)cbi;
   }
+}
+
+template <typename T>
+constexpr int refine_smem() {
+  return 64 * RefineCfg<T>::kChunk * (int)sizeof(typename RefineCfg<T>::P) + kRefineWarps * kD * 4 +
+         kRefineWarps * kRefineMaxK * 4;
 }
 
 }  // namespace
@@ -200,32 +258,40 @@ cudaError_t launch_assign_simt(const Plan& pl, const void* K, const void* V, cha
     kfn<<<grid, kThreads, smem, s>>>((const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
                                      reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_k),
                                      reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_v),
-                                     inv, slot_of, tok, ref, cnt, pl.N, pl.H, pl.k);
+                                     inv, slot_of, tok, ref, cnt, pl.N, pl.H, pl.k, pl.kp16);
   } else {
     auto kfn = assign_simt_kernel<float>;
     cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     kfn<<<grid, kThreads, smem, s>>>((const float*)K, (const float*)V,
                                      reinterpret_cast<const float*>(out + pl.L.off_anchors_k),
                                      reinterpret_cast<const float*>(out + pl.L.off_anchors_v),
-                                     inv, slot_of, tok, ref, cnt, pl.N, pl.H, pl.k);
+                                     inv, slot_of, tok, ref, cnt, pl.N, pl.H, pl.k, pl.kp16);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_refine(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s) {
-  auto* n2 = reinterpret_cast<const double*>(ws + pl.o_anc_n2);
+  auto* sq = reinterpret_cast<const double*>(ws + pl.o_anc_sqrt);
+  auto* inv = reinterpret_cast<const float*>(ws + pl.o_anc_inv);
   auto* ref = reinterpret_cast<const int*>(ws + pl.o_refine);
   auto* cnt = reinterpret_cast<const int*>(ws + pl.o_counters);
   auto* tok = reinterpret_cast<uint32_t*>(out + pl.L.off_tok);
+  // a few CTAs per (side, head) list; the lists are short (about 1% of rows)
+  const dim3 grid(std::max(1, 2 * 148 / (2 * pl.H)), 2 * pl.H);
   if (pl.p.dtype == ANCHORKV_BF16) {
-    refine_kernel<__nv_bfloat16><<<2 * 148, 256, 0, s>>>(
-        (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
-        reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_k),
-        reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_v), n2, ref, cnt, tok, pl.N, pl.H, pl.k);
+    using T = __nv_bfloat16;
+    auto kfn = refine_kernel<T>;
+    cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, refine_smem<T>());
+    kfn<<<grid, kRefineWarps * 32, refine_smem<T>(), s>>>(
+        (const T*)K, (const T*)V, reinterpret_cast<const T*>(out + pl.L.off_anchors_k),
+        reinterpret_cast<const T*>(out + pl.L.off_anchors_v), inv, sq, ref, cnt, tok, pl.N, pl.H, pl.k, pl.kp16);
   } else {
-    refine_kernel<float><<<2 * 148, 256, 0, s>>>(
-        (const float*)K, (const float*)V, reinterpret_cast<const float*>(out + pl.L.off_anchors_k),
-        reinterpret_cast<const float*>(out + pl.L.off_anchors_v), n2, ref, cnt, tok, pl.N, pl.H, pl.k);
+    using T = float;
+    auto kfn = refine_kernel<T>;
+    cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, refine_smem<T>());
+    kfn<<<grid, kRefineWarps * 32, refine_smem<T>(), s>>>(
+        (const T*)K, (const T*)V, reinterpret_cast<const T*>(out + pl.L.off_anchors_k),
+        reinterpret_cast<const T*>(out + pl.L.off_anchors_v), inv, sq, ref, cnt, tok, pl.N, pl.H, pl.k, pl.kp16);
   }
   return cudaGetLastError();
 }

@@ -1,0 +1,445 @@
+// Nearest-anchor assignment on the 5th-generation tensor cores (bf16).
+//
+// "AnchorKV: Anchor-Residual KV Cache Compression" (pith.science review),
+// Referee "Summary": every key and value is assigned to its nearest anchor.
+// Reading: argmax over slots of <x, a_s>/||a_s|| (signed cosine), ties to the
+// lowest slot, a zero anchor scores 0, an anchor token keeps its own slot.
+//
+// The contraction S = X A^T (X: 128 token rows, A: all k anchors of the
+// KV head and side, D = 128) runs as tcgen05.mma (M = 128, N = chunk of
+// anchors, K = 16 per instruction) from 128-byte-swizzled shared-memory
+// tiles that TMA fills; accumulators live in TMEM.  The epilogue never
+// writes S: eight warps read their TMEM lanes, scale each column by
+// 1/||a_s|| and keep the best and second-best score per row; the two column
+// halves are merged through shared memory.  Rows whose fp32 margin between
+// best and second best is not above the accumulation error bound are listed
+// for the fp64 re-decision shared with the SIMT path.
+//
+// Warp roles (320 threads, one CTA per SM, persistent over (side, head,
+// 128-row tile) work items): warp 0 issues TMA, warp 1 owns TMEM and issues
+// MMAs, warps 2..9 run the epilogue.  Anchors of the current (side, head)
+// stay resident in shared memory; token tiles stream through a ring.
+// Every mbarrier wait is bounded: on timeout the kernel latches an error,
+// drains its own copies and MMAs, frees TMEM and returns.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_util.cuh"
+
+namespace akv {
+
+// Margin below which a row's decision is re-taken in fp64, relative to ||x||.
+// Per key, the error against the exact cosine score (plus a row-constant
+// offset) is at most: fp32 accumulation of 128 exact products <= 2^-16 ||x||
+// (a conservative bound for the tensor-core adder), rounding of 1/||a||
+// <= 2^-24 ||x||, and the FMA's rounding onto the key grid <= 2^-15 ||x||; two
+// keys therefore differ from the exact difference by < 2^-13.4 ||x||.
+constexpr float kRefineRelTC = 1.0f / 8192.0f;
+
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kXStageBytes = 128 * 256;       // 128 rows x 128 bf16
+constexpr int kMaxKpad = 448;
+constexpr int kAccCols = 256;                 // columns per accumulator buffer
+
+struct TcArgs {
+  int N, H, k, kp16, cw, n_chunks, kpad, stages, row_tiles;
+  int total_items;
+  const float* anc_inv;
+  const int* slot_of;
+  const float* xnorm;
+  uint32_t* tok;
+  int* refine;
+  int* counters;
+};
+
+// Best two packed keys of a row (see the epilogue).  Keys of distinct slots
+// never compare equal, so the max/min updates keep them ordered.
+struct Keys2 {
+  uint32_t b1, b2;
+};
+
+__device__ __forceinline__ void key2_push(Keys2& s, uint32_t key) {
+  const uint32_t n1 = max(s.b1, key);
+  const uint32_t n2 = max(s.b2, min(key, s.b1));
+  s.b1 = n1; s.b2 = n2;
+}
+
+// Slot of a key: the low 9 bits hold (1 - chunk) << 8 | (255 - column in chunk).
+__device__ __forceinline__ uint32_t key_slot(uint32_t key, int cw) {
+  const uint32_t bits = key & 511u;
+  return ((bits & 256u) ? 0u : (uint32_t)cw) + (255u - (bits & 255u));
+}
+
+// Per-row constants of the key: C = 2^(floor(log2 ||x||) + 9) makes
+// fmaf(acc, 1/||a||, ||x||(1 + 2^-7) + C) land in [C, 2C), i.e. rounded to a
+// grid step of 2^(floor(log2 ||x||) - 14) <= 2^-14 ||x||, and since C's
+// mantissa is zero, bits(result) * 512 (mod 2^32) = q * 512 with q the grid
+// index: key = bits * 512 + (511 - column) orders by (score, -column) exactly.
+struct RowKey {
+  float add;      // ||x|| (1 + 2^-7) + C
+  float step;     // grid step
+};
+__device__ __forceinline__ RowKey row_key(float xn) {
+  const float x = fmaxf(xn, 1e-30f);
+  const int e = (int)((__float_as_uint(x) >> 23) & 255u) - 127;
+  RowKey r;
+  r.add = x * (1.0f + 1.0f / 128.0f) + __uint_as_float((uint32_t)(e + 9 + 127) << 23);
+  r.step = __uint_as_float((uint32_t)(e - 14 + 127) << 23);
+  return r;
+}
+
+// One chunk's columns for the warps of column group G (16-column blocks
+// G, G+2, ..., at most 7 of them since a chunk has at most 224 columns).  The
+// block and column indices are compile-time after unrolling, so a key costs
+// one FFMA and one LOP3 with an immediate, and the best-two update three
+// FMNMX.  Up to four TMEM loads are in flight per wait.
+template <int BLK>
+__device__ __forceinline__ void scan_block(const uint32_t (&w)[16], const float* ivc, float bias, int kc, Keys2& ka,
+                                           Keys2& kb) {
+  asm volatile("" ::: "memory");   // keep this block's loads from being hoisted into earlier blocks
+  const float4* iv4 = reinterpret_cast<const float4*>(ivc + BLK * 16);
+  const float4 i0 = iv4[0], i1 = iv4[1], i2 = iv4[2], i3 = iv4[3];
+  const float ivs[16] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w,
+                         i2.x, i2.y, i2.z, i2.w, i3.x, i3.y, i3.z, i3.w};
+  if (BLK * 16 + 16 <= kc) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint32_t key = __float_as_uint(fmaf(__uint_as_float(w[e]), ivs[e], bias)) * 512u +
+                           (uint32_t)(511 - (BLK * 16 + e));
+      if (e & 1) key2_push(kb, key);
+      else key2_push(ka, key);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      uint32_t key = __float_as_uint(fmaf(__uint_as_float(w[e]), ivs[e], bias)) * 512u +
+                     (uint32_t)(511 - (BLK * 16 + e));
+      if (BLK * 16 + e >= kc) key = 0u;
+      key2_push(ka, key);
+    }
+  }
+}
+
+// Blocks G + 2J and G + 2(J+1): two TMEM loads in flight, then recurse.
+template <int G, int J>
+__device__ __forceinline__ void scan_from(uint32_t tbase, const float* ivc, float bias, int kc, int nblk, Keys2& ka,
+                                          Keys2& kb) {
+  if constexpr (J < 7) {
+    constexpr int B0 = G + 2 * J, B1 = G + 2 * (J + 1);
+    if (!(B0 < nblk && B0 * 16 < kc)) return;
+    const bool h1 = (J + 1 < 7) && B1 < nblk && B1 * 16 < kc;
+    uint32_t v0[16], v1[16];
+    tc::tmem_ld16(tbase + (uint32_t)(B0 * 16), v0);
+    if (h1) tc::tmem_ld16(tbase + (uint32_t)(B1 * 16), v1);
+    tc::tmem_wait_ld_dep2(v0, v1);
+    scan_block<B0>(v0, ivc, bias, kc, ka, kb);
+    if constexpr (J + 1 < 7) {
+      if (h1) scan_block<B1>(v1, ivc, bias, kc, ka, kb);
+    }
+    scan_from<G, J + 2>(tbase, ivc, bias, kc, nblk, ka, kb);
+  }
+}
+
+template <int G>
+__device__ __forceinline__ void scan_chunk(uint32_t tbase, const float* ivc, float bias, int kc, int nblk, Keys2& ka,
+                                           Keys2& kb) {
+  scan_from<G, 0>(tbase, ivc, bias, kc, nblk, ka, kb);
+}
+
+using Best = Keys2;
+
+struct Ctl {
+  uint64_t x_full[4], x_empty[4], acc_full[2], acc_empty[2], anc_full, anc_empty, drain;
+  uint64_t mrg_full[2], mrg_empty[2];
+  uint32_t tmem_base;
+  int err;
+};
+
+__device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t parity, Ctl& ctl, int* counters) {
+  uint64_t t0 = 0;
+  for (uint32_t i = 0; i < tc::kWaitLimit; ++i) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 255u) {
+      if (*(volatile int*)&ctl.err) return false;
+      const uint64_t now = tc::globaltimer_ns();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > tc::kWaitNs) break;
+    }
+  }
+  *(volatile int*)&ctl.err = 1;
+  latch_error(counters, kDevErrTimeout);
+  return false;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constant__ CUtensorMap mapXV,
+                 const __grid_constant__ CUtensorMap mapAK, const __grid_constant__ CUtensorMap mapAV, TcArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte aligned base for the swizzled operand tiles
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* anc = base;                                   // kpad x 256 B
+  unsigned char* xs = anc + (size_t)a.kpad * 256;              // stages x 32 KB
+  Ctl& ctl = *reinterpret_cast<Ctl*>(xs + (size_t)a.stages * kXStageBytes);
+  Best* mrg = reinterpret_cast<Best*>(&ctl + 1);               // [2][128]
+  float* winv = reinterpret_cast<float*>(
+      (reinterpret_cast<uintptr_t>(mrg + 2 * 128) + 15) & ~static_cast<uintptr_t>(15));   // [8][kpad]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = gridDim.x;
+  const int beg = (int)((int64_t)blockIdx.x * a.total_items / G);
+  const int end = (int)((int64_t)(blockIdx.x + 1) * a.total_items / G);
+  const int S = a.stages;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) { tc::mbar_init(&ctl.x_full[s], 1); tc::mbar_init(&ctl.x_empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { tc::mbar_init(&ctl.acc_full[b], 1); tc::mbar_init(&ctl.acc_empty[b], 256); }
+    tc::mbar_init(&ctl.anc_full, 1);
+    tc::mbar_init(&ctl.anc_empty, 1);
+    tc::mbar_init(&ctl.drain, 1);
+    for (int b = 0; b < 2; ++b) { tc::mbar_init(&ctl.mrg_full[b], 128); tc::mbar_init(&ctl.mrg_empty[b], 128); }
+    ctl.err = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&ctl.tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::prefetch_tensormap(&mapXK); tc::prefetch_tensormap(&mapXV);
+    tc::prefetch_tensormap(&mapAK); tc::prefetch_tensormap(&mapAV);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = ctl.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int cur_u = -1, anc_loads = 0, issued = 0;
+      for (int it = beg; it < end && !ctl.err; ++it) {
+        const int u = it / a.row_tiles, j = it % a.row_tiles;
+        const int side = u / a.H, h = u % a.H;
+        if (u != cur_u) {
+          if (anc_loads > 0 && !wait_or_fail(&ctl.anc_empty, (anc_loads - 1) & 1, ctl, a.counters)) break;
+          tc::mbar_expect_tx(&ctl.anc_full, (uint32_t)a.kpad * 256u);
+          const CUtensorMap* mA = side ? &mapAV : &mapAK;
+          for (int c = 0; c < a.n_chunks; ++c)
+            for (int kh = 0; kh < 2; ++kh)
+              tc::tma_load_2d(anc + (size_t)(c * 2 + kh) * a.cw * 128, mA, kh * 64, h * a.k + c * a.cw,
+                              &ctl.anc_full);
+          cur_u = u;
+          ++anc_loads;
+        }
+        const int n = it - beg, s = n % S, use = n / S;
+        if (use > 0 && !wait_or_fail(&ctl.x_empty[s], (use - 1) & 1, ctl, a.counters)) break;
+        tc::mbar_expect_tx(&ctl.x_full[s], kXStageBytes);
+        const CUtensorMap* mX = side ? &mapXV : &mapXK;
+        const int row = h * a.N + j * 128;
+        tc::tma_load_2d(xs + (size_t)s * kXStageBytes, mX, 0, row, &ctl.x_full[s]);
+        tc::tma_load_2d(xs + (size_t)s * kXStageBytes + kXStageBytes / 2, mX, 64, row, &ctl.x_full[s]);
+        ++issued;
+      }
+      // drain: every copy issued must have landed before the CTA exits
+      for (int s = 0; s < S && s < issued; ++s) {
+        const int last_use = (issued - 1 - s) / S;
+        tc::mbar_wait(&ctl.x_full[s], last_use & 1);
+      }
+      if (anc_loads > 0) tc::mbar_wait(&ctl.anc_full, (anc_loads - 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16_f32(128, a.cw);
+      int cur_u = -1, anc_loads = 0, q = 0;
+      for (int it = beg; it < end && !ctl.err; ++it) {
+        const int u = it / a.row_tiles;
+        if (u != cur_u) {
+          if (anc_loads > 0) tc::mma_commit(&ctl.anc_empty);     // old anchors free once MMAs finish
+          if (!wait_or_fail(&ctl.anc_full, anc_loads & 1, ctl, a.counters)) break;
+          cur_u = u;
+          ++anc_loads;
+        }
+        const int n = it - beg, s = n % S, use = n / S;
+        if (!wait_or_fail(&ctl.x_full[s], use & 1, ctl, a.counters)) break;
+        tc::fence_after_sync();
+        const uint32_t xa = tc::smem_u32(xs + (size_t)s * kXStageBytes);
+        bool ok = true;
+        for (int c = 0; c < a.n_chunks; ++c, ++q) {
+          const int b = q & 1, uq = q >> 1;
+          if (uq > 0 && !wait_or_fail(&ctl.acc_empty[b], (uq - 1) & 1, ctl, a.counters)) { ok = false; break; }
+          tc::fence_after_sync();
+          const uint32_t d = tmem + (uint32_t)(b * kAccCols);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t aoff = (uint32_t)((kk >> 2) * (kXStageBytes / 2) + (kk & 3) * 32);
+            const uint32_t boff = (uint32_t)(((c * 2 + (kk >> 2)) * a.cw) * 128 + (kk & 3) * 32);
+            tc::mma_bf16(d, tc::sw128_desc(xa + aoff), tc::sw128_desc(tc::smem_u32(anc) + boff), idesc,
+                         kk > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(&ctl.acc_full[b]);
+        }
+        if (!ok) break;
+        tc::mma_commit(&ctl.x_empty[s]);
+      }
+      tc::mma_commit(&ctl.drain);
+      tc::mbar_wait(&ctl.drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (8 warps)
+    // Each column score s = acc / ||a|| becomes one positive float key
+    //   key = bits(s + ||x|| (1 + 2^-7)) with the low 9 bits replaced by 511 - slot,
+    // so the largest key is the best score and, among equal keys, the lowest
+    // slot; the best three keys per row cost five fmax/fmin per column.
+    const int g = (warp - 2) >> 2;          // column half
+    const int qd = warp & 3;                // TMEM lane quarter this warp may access
+    const int row = qd * 32 + lane;
+    const int nblk = a.cw / 16;
+    float* inv = winv + (size_t)(warp - 2) * a.kpad;   // this warp's copy of 1/||a||
+    int q = 0, cur_u = -1;
+    for (int it = beg; it < end; ++it) {
+      const int u = it / a.row_tiles, j = it % a.row_tiles;
+      const int side = u / a.H, h = u % a.H;
+      if (u != cur_u) {
+        __syncwarp();
+        const float* src = a.anc_inv + (int64_t)u * a.kp16;
+        for (int i = lane; i < a.kpad; i += 32) inv[i] = (i < a.kp16) ? src[i] : 0.f;
+        __syncwarp();
+        cur_u = u;
+      }
+      const int t = j * 128 + row;
+      const int64_t f = ((int64_t)side * a.H + h) * a.N + t;
+      const float xn = (t < a.N) ? a.xnorm[f] : 0.f;
+      const int own = (t < a.N) ? a.slot_of[(int64_t)h * a.N + t] : -1;
+      const RowKey rk = row_key(xn);
+      Keys2 ka{0u, 0u};
+      bool ok = true;
+      for (int c = 0; c < a.n_chunks; ++c, ++q) {
+        const int b = q & 1, uq = q >> 1;
+        if (!wait_or_fail(&ctl.acc_full[b], uq & 1, ctl, a.counters)) { ok = false; break; }
+        tc::fence_after_sync();
+        const uint32_t tbase = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(b * kAccCols);
+        const int kc = a.k - c * a.cw;                   // valid columns in this chunk
+        const float* ivc = inv + c * a.cw;
+        // keys of one chunk carry bit 8 set; chunk 1's keys get it cleared
+        // afterwards, so equal scores prefer chunk 0 (the lower slots)
+        Keys2 ca{0u, 0u}, cb{0u, 0u};
+        if (g == 0) scan_chunk<0>(tbase, ivc, rk.add, kc, nblk, ca, cb);
+        else scan_chunk<1>(tbase, ivc, rk.add, kc, nblk, ca, cb);
+        key2_push(ca, cb.b1); key2_push(ca, cb.b2);
+        if (c == 1) {
+          if (ca.b1) ca.b1 &= ~256u;
+          if (ca.b2) ca.b2 &= ~256u;
+        }
+        key2_push(ka, ca.b1); key2_push(ka, ca.b2);
+        tc::fence_before_sync();
+        tc::mbar_arrive(&ctl.acc_empty[b]);
+      }
+      if (!ok) break;
+      // merge the two column halves: group 1 hands its keys to group 0
+      const int n = it - beg, bb = n & 1, use = n >> 1;
+      if (g == 1) {
+        if (use > 0 && !wait_or_fail(&ctl.mrg_empty[bb], (use - 1) & 1, ctl, a.counters)) break;
+        mrg[bb * 128 + row] = ka;
+        tc::mbar_arrive(&ctl.mrg_full[bb]);
+        continue;
+      }
+      if (!wait_or_fail(&ctl.mrg_full[bb], use & 1, ctl, a.counters)) break;
+      const Keys2 other = mrg[bb * 128 + row];
+      tc::mbar_arrive(&ctl.mrg_empty[bb]);
+      key2_push(ka, other.b1); key2_push(ka, other.b2);
+      if (t < a.N) {
+        uint32_t slot;
+        if (own >= 0) {
+          slot = (uint32_t)own;
+        } else {
+          slot = key_slot(ka.b1, a.cw);
+          const float gap = (float)((ka.b1 >> 9) - (ka.b2 >> 9)) * rk.step;
+          if (!(gap > kRefineRelTC * xn)) list_for_refine(a.refine, a.counters, u, a.N, t);
+        }
+        a.tok[f] = slot;
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix [rows][128] as a tiled map with boxes of 64 x box_rows
+// (128-byte rows, 128-byte swizzle).
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {256};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool assign_tc_supported(const Plan& pl) {
+  if (pl.p.dtype != ANCHORKV_BF16) return false;
+  const int n_chunks = (pl.k + kAccCols - 1) / kAccCols;
+  const int cw = ((pl.k + n_chunks - 1) / n_chunks + 15) / 16 * 16;
+  return n_chunks * cw <= kMaxKpad && encode_fn() != nullptr;
+}
+
+cudaError_t launch_assign_tc(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s) {
+  TcArgs a;
+  a.N = pl.N; a.H = pl.H; a.k = pl.k; a.kp16 = pl.kp16;
+  a.n_chunks = (pl.k + kAccCols - 1) / kAccCols;
+  a.cw = ((pl.k + a.n_chunks - 1) / a.n_chunks + 15) / 16 * 16;
+  a.kpad = a.n_chunks * a.cw;
+  a.row_tiles = (pl.N + 127) / 128;
+  a.total_items = 2 * pl.H * a.row_tiles;
+  const int fixed = 1024 + (int)sizeof(Ctl) + 16 + 2 * 128 * (int)sizeof(Best) + 16 + 8 * a.kpad * 4 +
+                    a.kpad * 256;
+  a.stages = std::min(4, (227 * 1024 - fixed) / kXStageBytes);
+  if (a.stages < 2) return cudaErrorInvalidValue;
+  a.anc_inv = reinterpret_cast<const float*>(ws + pl.o_anc_inv);
+  a.slot_of = reinterpret_cast<const int*>(ws + pl.o_slot_of);
+  a.xnorm = reinterpret_cast<const float*>(ws + pl.o_xnorm);
+  a.tok = reinterpret_cast<uint32_t*>(out + pl.L.off_tok);
+  a.refine = reinterpret_cast<int*>(ws + pl.o_refine);
+  a.counters = reinterpret_cast<int*>(ws + pl.o_counters);
+  CUtensorMap mXK, mXV, mAK, mAV;
+  const int64_t HN = (int64_t)pl.H * pl.N, Hk = (int64_t)pl.H * pl.k;
+  if (!make_map(&mXK, K, HN, 128) || !make_map(&mXV, V, HN, 128) ||
+      !make_map(&mAK, out + pl.L.off_anchors_k, Hk, a.cw) || !make_map(&mAV, out + pl.L.off_anchors_v, Hk, a.cw))
+    return cudaErrorInvalidValue;
+  const int smem = fixed + a.stages * kXStageBytes;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = std::min(sms, a.total_items);
+  cudaFuncSetAttribute(assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  assign_tc_kernel<<<grid, kThreads, smem, s>>>(mXK, mXV, mAK, mAV, a);
+  return cudaGetLastError();
+}
+
+}  // namespace akv

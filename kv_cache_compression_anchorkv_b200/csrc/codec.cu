@@ -30,55 +30,72 @@ namespace {
 
 // ---------------------------------------------------------------- project
 
+// grid (ceil(N / 128), H, 2), 128 threads: the block stages 128 token rows
+// of one (side, head) in shared memory (coalesced loads, rows padded to
+// D + 1 floats so that thread r reading row r is bank-conflict free); each
+// thread then takes one token end to end in fp64.
+constexpr int kProjRows = 128;
+
 template <typename T>
-__global__ void project_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ anc_k,
-                               const T* __restrict__ anc_v, const double* __restrict__ anc_n2,
-                               const int* __restrict__ slot_of, const float* __restrict__ a2s,
-                               const float* __restrict__ kus, uint32_t* __restrict__ tok,
-                               float* __restrict__ util, int N, int H, int k) {
-  const int lane = threadIdx.x & 31;
-  const int64_t total = 2LL * H * N;
-  for (int64_t f = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); f < total;
-       f += (int64_t)gridDim.x * (blockDim.x >> 5)) {
-    const int side = (int)(f / ((int64_t)H * N));
-    const int h = (int)((f / N) % H);
-    const int t = (int)(f % N);
-    const uint32_t slot = tok[f] & 0xFFFFu;
-    const T* x = (side ? V : K) + ((int64_t)h * N + t) * kD;
-    const T* a = (side ? anc_v : anc_k) + ((int64_t)h * k + slot) * kD;
-    float xf[4], af[4];
-    load4<T>(x + lane * 4, xf);
-    load4<T>(a + lane * 4, af);
-    const bool is_anchor = slot_of[(int64_t)h * N + t] >= 0;
-    double dot = 0.0;
+__global__ void __launch_bounds__(kProjRows)
+project_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ anc_k,
+               const T* __restrict__ anc_v, const double* __restrict__ anc_n2, const int* __restrict__ slot_of,
+               const float* __restrict__ a2s, const float* __restrict__ kus, uint32_t* __restrict__ tok,
+               float* __restrict__ util, int N, int H, int k, int obs_rb) {
+  extern __shared__ float xt[];                       // [kProjRows][kD + 1]
+  const int t0 = blockIdx.x * kProjRows, h = blockIdx.y, side = blockIdx.z;
+  const int nv = min(kProjRows, N - t0);
+  const T* X = (side ? V : K) + ((int64_t)h * N + t0) * kD;
+  for (int i = threadIdx.x; i < nv * (kD / 4); i += kProjRows) {
+    const int r = i / (kD / 4), c = (i % (kD / 4)) * 4;
+    float f[4];
+    load4<T>(X + (int64_t)r * kD + c, f);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) dot = fma((double)xf[e], (double)af[e], dot);
-    dot = warp_sum_d(dot);
-    const double n2 = anc_n2[((int64_t)side * H + h) * k + slot];
-    double gamma = (n2 > 0.0) ? dot / n2 : 0.0;
-    if (is_anchor) gamma = 1.0;
-    const uint16_t gb = half_bits_rn(gamma);
-    const double g = (double)half_bits_to_f(gb);
-    double r2 = 0.0;
+    for (int e = 0; e < 4; ++e) xt[r * (kD + 1) + c + e] = f[e];
+  }
+  __syncthreads();
+  const int r = threadIdx.x;
+  if (r >= nv) return;
+  const int t = t0 + r;
+  const int64_t f = ((int64_t)side * H + h) * N + t;
+  const uint32_t slot = tok[f] & 0xFFFFu;
+  const T* a = (side ? anc_v : anc_k) + ((int64_t)h * k + slot) * kD;
+  const float* xr = xt + r * (kD + 1);
+  const bool is_anchor = slot_of[(int64_t)h * N + t] >= 0;
+  double dot = 0.0;
+  for (int d = 0; d < kD; d += 4) {
+    float af[4];
+    load4<T>(a + d, af);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dot = fma((double)xr[d + e], (double)af[e], dot);
+  }
+  const double n2 = anc_n2[((int64_t)side * H + h) * k + slot];
+  double gamma = (n2 > 0.0) ? dot / n2 : 0.0;
+  if (is_anchor) gamma = 1.0;
+  const uint16_t gb = half_bits_rn(gamma);
+  const double g = (double)half_bits_to_f(gb);
+  double r2 = 0.0;
+  for (int d = 0; d < kD; d += 4) {
+    float af[4];
+    load4<T>(a + d, af);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const double r = (double)xf[e] - g * (double)af[e];
-      r2 = fma(r, r, r2);
-    }
-    r2 = warp_sum_d(r2);
-    if (lane == 0) {
-      tok[f] = slot | ((uint32_t)gb << 16);
-      float u;
-      if (is_anchor) {
-        u = -1.0f;
-      } else if (side) {
-        u = (float)(r2 * (double)a2s[(int64_t)h * N + t]);
-      } else {
-        u = (float)(r2 / (double)(kD * kD) * (double)kus[(int64_t)h * N + t]);
-      }
-      util[f] = u;
+      const double rr = (double)xr[d + e] - g * (double)af[e];
+      r2 = fma(rr, rr, r2);
     }
   }
+  tok[f] = slot | ((uint32_t)gb << 16);
+  float u;
+  if (is_anchor) {
+    u = -1.0f;
+  } else {
+    // sum of the observation-row-block partials, in order
+    const float* src = side ? a2s : kus;
+    float m = src[(int64_t)h * N + t];
+    for (int rb = 1; rb < obs_rb; ++rb) m += src[((int64_t)rb * H + h) * N + t];
+    u = side ? (float)(r2 * (double)m) : (float)(r2 / (double)(kD * kD) * (double)m);
+  }
+  util[f] = u;
 }
 
 // ---------------------------------------------------------------- top-R select
@@ -370,24 +387,27 @@ CodecConst make_cc(const Plan& pl) {
 }  // namespace
 
 cudaError_t launch_project(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s) {
-  const int blocks = 148 * 8;
+  const dim3 blocks((pl.N + kProjRows - 1) / kProjRows, pl.H, 2);
+  const int smem = kProjRows * (kD + 1) * (int)sizeof(float);
   auto* n2 = reinterpret_cast<const double*>(ws + pl.o_anc_n2);
   auto* slot_of = reinterpret_cast<const int*>(ws + pl.o_slot_of);
   auto* a2 = reinterpret_cast<const float*>(ws + pl.o_a2);
   auto* ku = reinterpret_cast<const float*>(ws + pl.o_ku);
   auto* tok = reinterpret_cast<uint32_t*>(out + pl.L.off_tok);
   auto* util = reinterpret_cast<float*>(ws + pl.o_util);
+  cudaFuncSetAttribute(project_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaFuncSetAttribute(project_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (pl.p.dtype == ANCHORKV_BF16) {
-    project_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+    project_kernel<__nv_bfloat16><<<blocks, kProjRows, smem, s>>>(
         (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
         reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_k),
         reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_v), n2, slot_of, a2, ku, tok, util,
-        pl.N, pl.H, pl.k);
+        pl.N, pl.H, pl.k, pl.obs_rb);
   } else {
-    project_kernel<float><<<blocks, 256, 0, s>>>(
+    project_kernel<float><<<blocks, kProjRows, smem, s>>>(
         (const float*)K, (const float*)V, reinterpret_cast<const float*>(out + pl.L.off_anchors_k),
         reinterpret_cast<const float*>(out + pl.L.off_anchors_v), n2, slot_of, a2, ku, tok, util,
-        pl.N, pl.H, pl.k);
+        pl.N, pl.H, pl.k, pl.obs_rb);
   }
   return cudaGetLastError();
 }

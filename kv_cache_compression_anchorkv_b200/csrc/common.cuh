@@ -14,16 +14,18 @@ constexpr int kD = 128;          // head_dim supported by every kernel
 constexpr int kTile = 128;       // token tile of the residual bitmap / prefix table
 constexpr int kCodeBytes = kD / 4;
 
-// Counter slots in the compress workspace (int32 [16] at offset 0).
+// Counter slots in the compress workspace (int32 at offset 0): 16 scalar
+// counters, then one re-decision list length per (side, head).
 enum Counter {
   kStatus = 0,        // non-zero: a device-side check failed (code below)
   kRefineRows = 1,    // nearest-anchor rows re-decided in fp64
   kSelectTies = 2,    // token-sides whose utility equals the selection threshold
   kRefineOverflow = 3,
   kUniformRetries = 4,
-  kCounterCount = 16
+  kCounterCount = 16,
+  kRefineListBase = 16
 };
-enum DeviceError { kDevErrNone = 0, kDevErrUniform = 1, kDevErrRefine = 2, kDevErrBounds = 3 };
+enum DeviceError { kDevErrNone = 0, kDevErrUniform = 1, kDevErrRefine = 2, kDevErrBounds = 3, kDevErrTimeout = 4 };
 
 __device__ __forceinline__ void latch_error(int* counters, int code) {
   atomicCAS(&counters[kStatus], 0, code);
@@ -71,6 +73,45 @@ __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
+}
+
+// Running best, second and third score of a row with the slots of the first
+// two; slots are pushed in ascending order, so strict comparisons keep the
+// lowest slot among equal scores.
+struct Top3 {
+  float b1, b2, b3;
+  int i1, i2;
+};
+
+__device__ __forceinline__ Top3 top3_init() { return Top3{-INFINITY, -INFINITY, -INFINITY, 0x7fffffff, 0x7fffffff}; }
+
+__device__ __forceinline__ void push(Top3& b, float v, int i) {
+  if (v > b.b1) { b.b3 = b.b2; b.b2 = b.b1; b.i2 = b.i1; b.b1 = v; b.i1 = i; }
+  else if (v > b.b2) { b.b3 = b.b2; b.b2 = v; b.i2 = i; }
+  else if (v > b.b3) { b.b3 = v; }
+}
+
+__device__ __forceinline__ bool before(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+__device__ __forceinline__ Top3 merge(const Top3& a, const Top3& b) {
+  const bool a_wins = before(a.b1, a.i1, b.b1, b.i1);
+  const Top3& w = a_wins ? a : b;
+  const Top3& l = a_wins ? b : a;
+  Top3 r;
+  r.b1 = w.b1; r.i1 = w.i1;
+  if (before(l.b1, l.i1, w.b2, w.i2)) { r.b2 = l.b1; r.i2 = l.i1; r.b3 = fmaxf(w.b2, l.b2); }
+  else { r.b2 = w.b2; r.i2 = w.i2; r.b3 = fmaxf(w.b3, l.b1); }
+  return r;
+}
+
+// Lists token t of (side, head) u (= side * H + head) for the fp64
+// re-decision of its nearest anchor; list u holds up to N tokens.
+__device__ __forceinline__ void list_for_refine(int* refine, int* counters, int u, int N, int t) {
+  const int at = atomicAdd(&counters[kRefineListBase + u], 1);
+  refine[(int64_t)u * N + at] = t;
+  atomicAdd(&counters[kRefineRows], 1);
 }
 
 // fp16 (IEEE half) round-to-nearest-even of a double, saturating at +-65504.

@@ -11,7 +11,7 @@ namespace akv {
 // Stages bracketed by the optional event timing (profile.cu).
 enum Stage {
   kStObsPass1 = 0, kStObsCombine, kStTokenStats, kStAnchorSelect, kStAssign, kStRefine, kStProject,
-  kStSelect, kStQuantize, kStDecodePrep, kStDecodeSplit, kStDecodeCombine, kStageCount
+  kStSelect, kStQuantize, kStDecodePrep, kStDecodeSplit, kStDecodeCombine, kStObsAlpha, kStObsKu, kStageCount
 };
 void stage_begin(int stage, cudaStream_t s);
 void stage_end(int stage, cudaStream_t s, int kernels);
@@ -20,15 +20,20 @@ void stage_end(int stage, cudaStream_t s, int kernels);
 struct Plan {
   anchorkv_params p;
   anchorkv_layout L;
-  int N, D, H, Hq, G, W, GW, k, n_s, n_u, n_tiles, elem;
+  int N, D, H, Hq, G, W, GW, k, kp16, n_s, n_u, n_tiles, elem;
   int64_t R, cap;
   bool all_anchors;
-  // pass-1 token chunks
+  // pass-1 token chunks (SIMT observation passes)
   int chunk1, n_chunk1;
+  // tensor-core observation passes: row blocks, token splits, tiles per split
+  int tc_rb, tc_split, tc_tps;
+  // row-block partials of score / sum alpha^2 / key term the consumers sum
+  int obs_rb;
   // workspace offsets (bytes from the workspace base)
   int64_t ws_total;
   int64_t o_counters, o_row_m, o_row_z, o_ybar, o_part_m, o_part_l, o_part_y;
-  int64_t o_score, o_a2, o_ku, o_pooled, o_slot_of, o_anc_n2, o_anc_inv;
+  int64_t o_tc_pm2, o_tc_pl, o_tc_rm2, o_tc_riz, o_tc_rq2, o_tc_ry2, o_tc_py, o_tc_yh, o_tc_yl;
+  int64_t o_score, o_a2, o_ku, o_pooled, o_slot_of, o_anc_n2, o_anc_inv, o_anc_sqrt, o_xnorm;
   int64_t o_util, o_refine, o_sel_state, o_hist, o_tile_gt, o_tile_eq, o_tie_before, o_tile_cnt;
   // codebook and Hadamard signs (bit j set: s_j = -1)
   double tau, l1, l2;
@@ -51,6 +56,10 @@ cudaError_t launch_token_stats(const Plan& pl, const void* K, const void* V, con
 cudaError_t launch_anchor_select(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s);
 cudaError_t launch_assign_simt(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s);
 cudaError_t launch_refine(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s);
+cudaError_t launch_assign_tc(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s);
+bool assign_tc_supported(const Plan& pl);
+cudaError_t launch_obs_tc(const Plan& pl, const void* K, const void* V, const void* Q, char* ws, cudaStream_t s);
+bool obs_tc_supported(const Plan& pl);
 cudaError_t launch_project(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s);
 cudaError_t launch_select(const Plan& pl, char* out, char* ws, cudaStream_t s);
 cudaError_t launch_quantize(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s);

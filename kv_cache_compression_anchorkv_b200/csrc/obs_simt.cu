@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 token_stats_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ Q,
                    int N, int G, int W, const float* __restrict__ row_m, const float* __restrict__ row_z,
                    const float* __restrict__ ybar, float* __restrict__ score, float* __restrict__ a2s,
-                   float* __restrict__ kus) {
+                   float* __restrict__ kus, float* __restrict__ xnorm, int H) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   StatSmem& sm = *reinterpret_cast<StatSmem*>(smem_raw);
   const int h = blockIdx.y;
@@ -222,6 +222,16 @@ token_stats_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __
   const float scale = rsqrtf((float)kD);
   load_tile<T>(sm.x, K + (int64_t)h * N * kD, t0, nv);
   load_tile<T>(sm.v, V + (int64_t)h * N * kD, t0, nv);
+  __syncthreads();
+  if (threadIdx.x < 2 * kTokTile) {
+    // row norms of the keys and values (fp32), used by the assignment's
+    // error bound
+    const int t = threadIdx.x % kTokTile, side = threadIdx.x / kTokTile;
+    const float* rowp = side ? sm.v[t] : sm.x[t];
+    float s2 = 0.f;
+    for (int d = 0; d < kD; ++d) s2 = fmaf(rowp[d], rowp[d], s2);
+    if (t < nv) xnorm[((int64_t)side * H + h) * N + t0 + t] = sqrtf(s2);
+  }
   float acc[3][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
   for (int r0 = 0; r0 < GW; r0 += kRowBlk) {
     const int nr = min(kRowBlk, GW - r0);
@@ -351,16 +361,17 @@ cudaError_t launch_token_stats(const Plan& pl, const void* K, const void* V, con
   auto* sc = reinterpret_cast<float*>(ws + pl.o_score);
   auto* a2 = reinterpret_cast<float*>(ws + pl.o_a2);
   auto* ku = reinterpret_cast<float*>(ws + pl.o_ku);
+  auto* xn = reinterpret_cast<float*>(ws + pl.o_xnorm);
   if (pl.p.dtype == ANCHORKV_BF16) {
     auto k = token_stats_kernel<__nv_bfloat16>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     k<<<grid, kThreads, smem, s>>>((const __nv_bfloat16*)K, (const __nv_bfloat16*)V, (const __nv_bfloat16*)Q,
-                                   pl.N, pl.G, pl.W, rm, rz, yb, sc, a2, ku);
+                                   pl.N, pl.G, pl.W, rm, rz, yb, sc, a2, ku, xn, pl.H);
   } else {
     auto k = token_stats_kernel<float>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     k<<<grid, kThreads, smem, s>>>((const float*)K, (const float*)V, (const float*)Q,
-                                   pl.N, pl.G, pl.W, rm, rz, yb, sc, a2, ku);
+                                   pl.N, pl.G, pl.W, rm, rz, yb, sc, a2, ku, xn, pl.H);
   }
   return cudaGetLastError();
 }

@@ -151,3 +151,32 @@ def test_full_size_layer_llama8b_shape():
     comp = torch.from_numpy(gb).cuda()
     o = api.decode_attn(p, comp, q)
     parity.check_decode(p, [gb], _f64(q), None, None, 0, o.cpu().double().numpy(), DECODE_TOL["bf16"])
+
+
+@pytest.mark.parametrize("name", ["bf16-ragged-n3000", "bf16-gqa8-n2500", "bf16-every-residual"])
+def test_tensor_core_and_simt_assignment_agree(name, monkeypatch):
+    """The tcgen05 assignment and the SIMT assignment both end in the same
+    fp64-certified decisions, so their layouts are identical."""
+    spec, theta = CASES[name]
+    K, V, Q = (x.cuda() for x in make_layer(spec, 0))
+    p = _params(spec, theta)
+    tc_out, tc_ws = api.compress(p, K, V, Q)
+    tc_refined = api.read_status(tc_ws)[1]
+    monkeypatch.setenv("ANCHORKV_SIMT_ASSIGN", "1")
+    simt_out, _ = api.compress(p, K, V, Q)
+    assert torch.equal(tc_out, simt_out)
+    print(name, "rows re-decided in fp64 (tensor-core path):", tc_refined)
+
+
+@pytest.mark.parametrize("name", ["bf16-ragged-n3000", "bf16-gqa8-n2500"])
+def test_simt_observation_path_parity(name, monkeypatch):
+    """The SIMT observation passes (used for fp32 caches) also match the
+    oracle on bf16 inputs, so both implementations stay covered."""
+    monkeypatch.setenv("ANCHORKV_SIMT_OBS", "1")
+    spec, theta = CASES[name]
+    K, V, Q = make_layer(spec, 0)
+    p = _params(spec, theta, layer=1)
+    gb, gpool, gutil, counters = parity.gpu_compress(p, K, V, Q)
+    assert counters[0] == 0
+    rep = parity.check_compress(p, _f64(K), _f64(V), _f64(Q), gb, gpool, gutil)
+    print(name, "simt observation passes", rep)
