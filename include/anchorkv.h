@@ -177,6 +177,32 @@ int anchorkv_decode_attn(const anchorkv_params* p, const void* compressed,
                          void* stream);
 
 /*
+ * Decode attention that allocates nothing.  The paper has no counterpart:
+ * this is a library service, not part of the method.  Same operation,
+ * arguments and errors as anchorkv_decode_attn, without the workspace: the
+ * scratch comes from one library-owned array of
+ * ANCHORKV_DECODE_NOALLOC_SCRATCH_BYTES per device, and the call makes no
+ * cudaMalloc, cudaFree or other allocating call.  It is meant for callers
+ * that cannot allocate device memory while decoding: a serving engine whose
+ * free HBM is all handed to its KV-cache pool, a plain-C caller without a
+ * device allocator, or a decode loop that must not take the device-wide
+ * synchronisation cudaMalloc / cudaFree bring.
+ *   - Sizes whose decode workspace (anchorkv_decode_workspace_bytes) exceeds
+ *     the maximum are rejected with ANCHORKV_ENOSPC before any launch.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call on a device shares the array, which keeps the last call's
+ *     contents (nothing in it needs to start at zero).  Calls that overlap on
+ *     the GPU (different streams, or different host threads without ordering
+ *     between their streams) race on it: order them on one stream.
+ */
+#define ANCHORKV_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20)
+int anchorkv_decode_attn_noalloc(const anchorkv_params* p, const void* compressed,
+                                 int64_t seq_stride_bytes, int32_t batch, const void* q,
+                                 const void* K_tail, const void* V_tail, int32_t tail_len,
+                                 int32_t tail_cap, float* out, void* stream);
+
+/*
  * Test and inspection hook: writes the dense reconstruction
  * x^_t = gamma~_t x_a(t) + r~_t of one compressed layer.
  *   K_hat, V_hat device [H][N][D] float32.

@@ -126,6 +126,40 @@ def decode_attn(p: AnchorKVParams, compressed: torch.Tensor, q: torch.Tensor,
     return out
 
 
+NOALLOC_SCRATCH_BYTES = 32 << 20   # ANCHORKV_DECODE_NOALLOC_SCRATCH_BYTES in include/anchorkv.h
+
+
+def decode_attn_noalloc(p: AnchorKVParams, compressed: torch.Tensor, q: torch.Tensor, out: torch.Tensor,
+                        K_tail: torch.Tensor | None = None, V_tail: torch.Tensor | None = None,
+                        tail_len: int = 0) -> torch.Tensor:
+    """Decode attention that allocates no device memory: the library's
+    per-device scratch array stands in for the workspace, and `out` must be
+    supplied.  For callers that cannot allocate while decoding (all free HBM
+    given to a KV-cache pool, no device allocator, or no room for the
+    device-wide synchronisation of cudaMalloc/cudaFree).  Calls that overlap
+    on the GPU share the scratch and race; sizes whose decode workspace
+    exceeds NOALLOC_SCRATCH_BYTES raise (ANCHORKV_ENOSPC)."""
+    if compressed.dim() == 1:
+        compressed = compressed[None]
+    batch, stride = compressed.shape
+    _check_tensor("q", q, (batch, p.n_q_heads, p.head_dim), p.torch_dtype)
+    _check_tensor("out", out, (batch, p.n_q_heads, p.head_dim), torch.float32)
+    cap = 0
+    if K_tail is not None:
+        cap = K_tail.shape[2]
+        _check_tensor("K_tail", K_tail, (batch, p.n_kv_heads, cap, p.head_dim), p.torch_dtype)
+        _check_tensor("V_tail", V_tail, (batch, p.n_kv_heads, cap, p.head_dim), p.torch_dtype)
+    st = capi.lib().anchorkv_decode_attn_noalloc(ctypes.byref(p.c()), _ptr(compressed), stride, batch, _ptr(q),
+                                                 _ptr(K_tail), _ptr(V_tail), tail_len, cap, _ptr(out),
+                                                 _stream(q.device))
+    if st == capi.ENOSPC:
+        raise capi.AnchorKVError(
+            f"anchorkv_decode_attn_noalloc (decode workspace {decode_workspace_bytes(p, batch)} B exceeds the "
+            f"{NOALLOC_SCRATCH_BYTES} B static scratch)", st)
+    capi.check("anchorkv_decode_attn_noalloc", st)
+    return out
+
+
 def reconstruct(p: AnchorKVParams, compressed: torch.Tensor):
     """Dense fp32 K^, V^ [H, N, D] of one compressed layer (inspection hook)."""
     H, N, D = p.n_kv_heads, p.n_tokens, p.head_dim
