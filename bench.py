@@ -314,6 +314,7 @@ def run_gpu(args, world, rank, local):
                        "decode_batch": 1, "parallelism": f"replicas{world}",
                        "l2": "inputs larger than L2 (%.1f GB of K/V per step)" % (Lr * 2 * H * N * 128 * 2 / 1e9)},
             "decode_us_per_step": dec_us,
+            "decode_launch": api.decode_config(params[0], 1),
             "decode_hbm_gbs": dec_bytes / (dec_us / 1e6) / 1e9,
             "compressed_bytes_per_layer": L["total_bytes"],
             "uncompressed_bytes_per_layer": L["uncompressed_bytes"],

@@ -177,6 +177,18 @@ int anchorkv_decode_attn(const anchorkv_params* p, const void* compressed,
                          void* stream);
 
 /*
+ * Launch shape of anchorkv_decode_attn for `batch` sequences on the current
+ * device (a diagnostic with no counterpart in the method): CTAs per
+ * (sequence, KV head) thread-block cluster and dynamic shared memory per CTA.
+ * Up to 8 query heads per KV head the decode runs as one cluster per
+ * (sequence, head) and needs no workspace; otherwise *cluster_ctas = 0 and
+ * the split-token kernels, which use the workspace, run.  Host; queries the
+ * device once per shape.  EUNSUPPORTED if no cluster shape fits the device.
+ */
+int anchorkv_decode_config(const anchorkv_params* p, int32_t batch, int32_t* cluster_ctas,
+                           int32_t* smem_bytes);
+
+/*
  * Decode attention that allocates nothing.  The paper has no counterpart:
  * this is a library service, not part of the method.  Same operation,
  * arguments and errors as anchorkv_decode_attn, without the workspace: the
@@ -225,7 +237,10 @@ int anchorkv_codebook(double* out4);
  * process-wide; recording adds a few microseconds per stage. */
 int anchorkv_stage_timing(int enable);
 
-/* Waits for the recorded events and returns, per stage (n >= 12 entries),
+/* Number of timed stages reported by anchorkv_stage_times. */
+#define ANCHORKV_N_STAGES 15
+
+/* Waits for the recorded events and returns, per stage (n >= ANCHORKV_N_STAGES entries),
  * the accumulated milliseconds and the number of timed calls since the last
  * anchorkv_stage_timing call.  Stage names: anchorkv_stage_name. */
 int anchorkv_stage_times(double* ms_out, int64_t* calls_out, int32_t n);

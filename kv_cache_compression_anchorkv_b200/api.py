@@ -126,6 +126,15 @@ def decode_attn(p: AnchorKVParams, compressed: torch.Tensor, q: torch.Tensor,
     return out
 
 
+def decode_config(p: AnchorKVParams, batch: int) -> dict:
+    """Launch shape of decode_attn on the current device: CTAs per (sequence,
+    head) cluster (0: split-token path with a workspace) and shared memory."""
+    c, m = ctypes.c_int32(), ctypes.c_int32()
+    capi.check("anchorkv_decode_config",
+               capi.lib().anchorkv_decode_config(ctypes.byref(p.c()), batch, ctypes.byref(c), ctypes.byref(m)))
+    return {"cluster_ctas": c.value, "smem_bytes": m.value}
+
+
 NOALLOC_SCRATCH_BYTES = 32 << 20   # ANCHORKV_DECODE_NOALLOC_SCRATCH_BYTES in include/anchorkv.h
 
 
@@ -215,7 +224,7 @@ class HostCompressor:
         return self.host_out
 
 
-N_STAGES = 14
+N_STAGES = 15   # ANCHORKV_N_STAGES
 
 
 def stage_timing(enable: bool) -> None:

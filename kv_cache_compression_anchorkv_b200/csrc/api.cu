@@ -318,7 +318,8 @@ int anchorkv_decode_attn(const anchorkv_params* p, const void* compressed, int64
   if (st) return st;
   if (batch < 0 || tail_len < 0 || tail_cap < tail_len) return ANCHORKV_EINVAL;
   if (batch == 0) return ANCHORKV_OK;
-  if (!compressed || !q || !out || !ws) return ANCHORKV_EINVAL;
+  if (batch > 65535) return ANCHORKV_EUNSUPPORTED;
+  if (!compressed || !q || !out) return ANCHORKV_EINVAL;
   if (tail_len > 0 && (!K_tail || !V_tail)) return ANCHORKV_EINVAL;
   if (tail_len > 4096) return ANCHORKV_EUNSUPPORTED;
   if (seq_stride_bytes < pl.L.total_bytes && batch > 1) return ANCHORKV_EINVAL;
@@ -327,14 +328,33 @@ int anchorkv_decode_attn(const anchorkv_params* p, const void* compressed, int64
   DecodePlan dp;
   make_decode_plan(pl, batch, &dp);
   if ((int64_t)ws_bytes < dp.ws_total) return ANCHORKV_ENOSPC;
-  const size_t smem_split = sizeof(float) * ((size_t)2 * pl.G * pl.k + (size_t)pl.G * dp.split_tokens + 2 * pl.G * kD);
-  if (smem_split > 220 * 1024 || sizeof(float) * ((size_t)pl.G * pl.k + (size_t)pl.G * std::max(tail_len, 1)) > 180 * 1024)
-    return ANCHORKV_EUNSUPPORTED;
+  if (dp.ws_total > 0 && !ws) return ANCHORKV_EINVAL;
+  st = check_decode_shape(pl, dp, tail_len);
+  if (st) return st;
   st = check_device();
   if (st) return st;
   AKV_LAUNCH(launch_decode(pl, dp, (const char*)compressed, seq_stride_bytes, q, K_tail, V_tail, tail_len,
                            tail_cap, out, (char*)ws, (cudaStream_t)stream));
   return ANCHORKV_OK;
+}
+
+int anchorkv_decode_config(const anchorkv_params* p, int32_t batch, int32_t* cluster_ctas, int32_t* smem_bytes) {
+  if (!cluster_ctas || !smem_bytes || batch < 1) return ANCHORKV_EINVAL;
+  Plan pl;
+  int st = make_plan(p, &pl);
+  if (st) return st;
+  DecodePlan dp;
+  make_decode_plan(pl, batch, &dp);
+  *cluster_ctas = 0;
+  *smem_bytes = 0;
+  if (!dp.cluster) return ANCHORKV_OK;
+  st = check_device();
+  if (st) return st;
+  int C = 0, smem = 0;
+  st = decode_cluster_size(pl, batch, &C, &smem);
+  *cluster_ctas = C;
+  *smem_bytes = smem;
+  return st;
 }
 
 int anchorkv_reconstruct(const anchorkv_params* p, const void* compressed, float* K_hat, float* V_hat,

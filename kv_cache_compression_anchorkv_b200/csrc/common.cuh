@@ -123,8 +123,9 @@ __device__ __forceinline__ float half_bits_to_f(uint32_t bits16) {
   return __half2float(__ushort_as_half((unsigned short)bits16));
 }
 
-// In-warp orthonormal Walsh-Hadamard transform of a 128-vector held as
-// 4 consecutive coordinates per lane (lane l owns 4l..4l+3), natural order.
+// In-warp Walsh-Hadamard transform (unnormalised: the Sylvester matrix of
+// +-1 entries) of a 128-vector held as 4 consecutive coordinates per lane
+// (lane l owns 4l..4l+3), natural order.
 template <typename F>
 __device__ __forceinline__ void fwht128(F (&v)[4]) {
   F a0 = v[0] + v[1], a1 = v[0] - v[1], a2 = v[2] + v[3], a3 = v[2] - v[3];

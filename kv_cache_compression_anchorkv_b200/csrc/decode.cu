@@ -329,6 +329,13 @@ decode_combine_kernel(DecodeArgs a, const T* __restrict__ q, const T* __restrict
 
 int make_decode_plan(const Plan& pl, int batch, DecodePlan* dp) {
   dp->batch = batch;
+  dp->cluster = decode_cluster_supported(pl);
+  if (dp->cluster) {
+    dp->n_split = 0; dp->split_tokens = 0;
+    dp->o_P = dp->o_qrot = dp->o_part_m = dp->o_part_l = dp->o_part_w = dp->o_part_z = 0;
+    dp->ws_total = 0;
+    return ANCHORKV_OK;
+  }
   const int units = std::max(1, batch * pl.H);
   int want = std::max(1, (2 * 148 + units - 1) / units);
   int tiles_per = std::max(1, (pl.n_tiles + want - 1) / want);
@@ -348,9 +355,23 @@ int make_decode_plan(const Plan& pl, int batch, DecodePlan* dp) {
   return ANCHORKV_OK;
 }
 
+int check_decode_shape(const Plan& pl, const DecodePlan& dp, int tail_len) {
+  if (dp.cluster) return ANCHORKV_OK;
+  const size_t smem_split = sizeof(float) * ((size_t)2 * pl.G * pl.k + (size_t)pl.G * dp.split_tokens + 2 * pl.G * kD);
+  const size_t smem_comb = sizeof(float) * ((size_t)pl.G * pl.k + (size_t)pl.G * std::max(tail_len, 1));
+  if (smem_split > 220 * 1024 || smem_comb > 180 * 1024) return ANCHORKV_EUNSUPPORTED;
+  return ANCHORKV_OK;
+}
+
 cudaError_t launch_decode(const Plan& pl, const DecodePlan& dp, const char* comp, int64_t stride, const void* q,
                           const void* Kt, const void* Vt, int tail_len, int tail_cap, float* out, char* ws,
                           cudaStream_t s) {
+  if (dp.cluster) {
+    cudaError_t e = cudaSuccess;
+    const int st = launch_decode_cluster(pl, dp.batch, comp, stride, q, Kt, Vt, tail_len, tail_cap, out, s, &e);
+    if (st == ANCHORKV_OK) return cudaSuccess;
+    return e != cudaSuccess ? e : cudaErrorNotSupported;
+  }
   DecodeArgs a;
   a.comp = reinterpret_cast<const uint8_t*>(comp);
   a.stride = stride;

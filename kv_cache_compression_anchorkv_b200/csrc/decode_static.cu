@@ -71,6 +71,7 @@ int anchorkv_decode_attn_noalloc(const anchorkv_params* p, const void* compresse
   if (st) return st;
   if (batch < 0 || tail_len < 0 || tail_cap < tail_len) return ANCHORKV_EINVAL;
   if (batch == 0) return ANCHORKV_OK;
+  if (batch > 65535) return ANCHORKV_EUNSUPPORTED;
   if (!compressed || !q || !out) return ANCHORKV_EINVAL;
   if (tail_len > 0 && (!K_tail || !V_tail)) return ANCHORKV_EINVAL;
   if (tail_len > 4096) return ANCHORKV_EUNSUPPORTED;
@@ -80,9 +81,8 @@ int anchorkv_decode_attn_noalloc(const anchorkv_params* p, const void* compresse
   DecodePlan dp;
   make_decode_plan(pl, batch, &dp);
   if (dp.ws_total > (int64_t)ANCHORKV_DECODE_NOALLOC_SCRATCH_BYTES) return ANCHORKV_ENOSPC;
-  const size_t smem_split = sizeof(float) * ((size_t)2 * pl.G * pl.k + (size_t)pl.G * dp.split_tokens + 2 * pl.G * kD);
-  if (smem_split > 220 * 1024 || sizeof(float) * ((size_t)pl.G * pl.k + (size_t)pl.G * std::max(tail_len, 1)) > 180 * 1024)
-    return ANCHORKV_EUNSUPPORTED;
+  st = check_decode_shape(pl, dp, tail_len);
+  if (st) return st;
   st = device_is_sm100();
   if (st) return st;
   char* scratch = nullptr;

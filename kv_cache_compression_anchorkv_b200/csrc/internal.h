@@ -11,7 +11,7 @@ namespace akv {
 // Stages bracketed by the optional event timing (profile.cu).
 enum Stage {
   kStObsPass1 = 0, kStObsCombine, kStTokenStats, kStAnchorSelect, kStAssign, kStRefine, kStProject,
-  kStSelect, kStQuantize, kStDecodePrep, kStDecodeSplit, kStDecodeCombine, kStObsAlpha, kStObsKu, kStageCount
+  kStSelect, kStQuantize, kStDecodePrep, kStDecodeSplit, kStDecodeCombine, kStObsAlpha, kStObsKu, kStDecodeCluster, kStageCount
 };
 void stage_begin(int stage, cudaStream_t s);
 void stage_end(int stage, cudaStream_t s, int kernels);
@@ -44,10 +44,18 @@ int make_plan(const anchorkv_params* p, Plan* out);
 void codebook(double* tau, double* l1, double* l2, double* mse);
 
 struct DecodePlan {
+  bool cluster;           // one cluster per (sequence, head), no workspace
   int batch, n_split, split_tokens;
   int64_t ws_total, o_P, o_qrot, o_part_m, o_part_l, o_part_w, o_part_z;
 };
 int make_decode_plan(const Plan& pl, int batch, DecodePlan* out);
+// Shape checks of a decode call (shared-memory limits of the chosen path).
+int check_decode_shape(const Plan& pl, const DecodePlan& dp, int tail_len);
+bool decode_cluster_supported(const Plan& pl);
+int decode_cluster_size(const Plan& pl, int batch, int* C, int* smem);
+int launch_decode_cluster(const Plan& pl, int batch, const char* comp, int64_t stride, const void* q,
+                          const void* Kt, const void* Vt, int tail_len, int tail_cap, float* out, cudaStream_t s,
+                          cudaError_t* err);
 
 // Kernel launchers (one per hot-path step), all asynchronous on `s`.
 cudaError_t launch_obs_pass1(const Plan& pl, const void* K, const void* V, const void* Q, char* ws, cudaStream_t s);

@@ -23,6 +23,7 @@ bool g_on = false;
 std::vector<Mark> g_marks;
 std::vector<cudaEvent_t> g_pool;
 int64_t g_launches = 0;
+static_assert(kStageCount == ANCHORKV_N_STAGES, "stage table and header disagree");
 double g_ms[kStageCount];
 int64_t g_calls[kStageCount];
 cudaEvent_t g_open[kStageCount];
@@ -40,7 +41,7 @@ cudaEvent_t get_event() {
 
 const char* kNames[kStageCount] = {"obs_pass1", "obs_combine", "token_stats", "anchor_select", "assign",
                                    "assign_refine", "project", "select_topR", "quantize", "decode_prep",
-                                   "decode_split", "decode_combine", "obs_alpha", "obs_key_term"};
+                                   "decode_split", "decode_combine", "obs_alpha", "obs_key_term", "decode_attn"};
 
 }  // namespace
 

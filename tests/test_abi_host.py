@@ -89,4 +89,8 @@ def test_workspace_view():
     v = api.compress_workspace(p)
     assert v["total_bytes"] > v["off_utility"] + 4 * 2 * 8 * 32768
     assert v["off_counters"] % 256 == 0 and v["off_pooled"] % 256 == 0
-    assert api.decode_workspace_bytes(p, 16) > api.decode_workspace_bytes(p, 1) > 0
+    # up to 8 query heads per KV head the decode runs in one cluster per
+    # (sequence, head) and needs no workspace; above that it splits tokens
+    assert api.decode_workspace_bytes(p, 1) == api.decode_workspace_bytes(p, 16) == 0
+    p16 = api.AnchorKVParams(n_tokens=32768, n_q_heads=128)
+    assert api.decode_workspace_bytes(p16, 16) > api.decode_workspace_bytes(p16, 1) > 0

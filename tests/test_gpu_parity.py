@@ -32,6 +32,10 @@ CASES = {
     "bf16-no-residual": (CacheSpec(1, 2, 4, 1000, n_dirs=16, seed=4), 0.01),
     "fp32-all-anchors": (CacheSpec(1, 2, 4, 33, dtype="fp32", n_dirs=8, seed=5), 0.5),
     "fp32-window8-n700": (CacheSpec(1, 3, 3, 700, window=8, dtype="fp32", n_dirs=8, seed=6), 0.3),
+    # 16 query heads per KV head (the split-K decode path)
+    "bf16-gqa16-n1500": (CacheSpec(1, 1, 16, 1500, n_dirs=32, seed=8), 0.2),
+    # enough tiles that every CTA of a 16-CTA decode cluster streams two chunks
+    "bf16-n20000": (CacheSpec(1, 1, 4, 20000, n_dirs=64, seed=9), 0.1),
 }
 
 
@@ -90,7 +94,9 @@ def test_reconstruct_matches_oracle():
 @pytest.mark.parametrize("name,batch,tail", [("tiny-fp32-n1024", 1, 0), ("tiny-fp32-n1024", 2, 5),
                                              ("bf16-ragged-n3000", 3, 17), ("bf16-gqa8-n2500", 2, 0),
                                              ("bf16-every-residual", 1, 3), ("bf16-no-residual", 2, 1),
-                                             ("fp32-all-anchors", 1, 2)])
+                                             ("fp32-all-anchors", 1, 2), ("fp32-window8-n700", 2, 9),
+                                             ("bf16-gqa16-n1500", 2, 4), ("bf16-n20000", 1, 0),
+                                             ("bf16-n20000", 2, 1500)])
 def test_decode_parity(name, batch, tail):
     spec, theta = CASES[name]
     p = _params(spec, theta)
@@ -111,6 +117,14 @@ def test_decode_parity(name, batch, tail):
     err = parity.check_decode(p, layouts, _f64(q), _f64(Kt), _f64(Vt), tail, o.cpu().double().numpy(),
                               DECODE_TOL[spec.dtype])
     print(name, batch, tail, "max abs err", err)
+
+
+def test_decode_config():
+    spec, theta = CASES["bf16-n20000"]
+    cfg = api.decode_config(_params(spec, theta), 1)
+    assert cfg["cluster_ctas"] in (1, 2, 4, 8, 16) and 0 < cfg["smem_bytes"] <= 227 * 1024
+    spec, theta = CASES["bf16-gqa16-n1500"]
+    assert api.decode_config(_params(spec, theta), 2)["cluster_ctas"] == 0
 
 
 def test_error_paths_on_device():

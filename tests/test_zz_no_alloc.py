@@ -62,6 +62,8 @@ def _decode_both(p, comp, stride, q, Kt, Vt, tail_len):
 CASES = {
     "bf16-ragged-n3000-batch2": (CacheSpec(1, 2, 8, 3000, n_dirs=64, seed=11), 0.1, 2),
     "fp32-window8-n700-batch3": (CacheSpec(1, 3, 3, 700, window=8, dtype="fp32", n_dirs=8, seed=12), 0.3, 3),
+    # 16 query heads per KV head: the decode path that uses the scratch
+    "bf16-gqa16-n1500-batch2": (CacheSpec(1, 1, 16, 1500, n_dirs=32, seed=13), 0.2, 2),
 }
 
 
@@ -90,7 +92,7 @@ def test_noalloc_rejects_sizes_beyond_the_scratch():
     the placeholder pointers below can never reach a kernel."""
     if torch.cuda.is_available():
         pytest.skip("host-only check")
-    p = api.AnchorKVParams(n_tokens=131072, n_kv_heads=8, n_q_heads=64)
+    p = api.AnchorKVParams(n_tokens=131072, n_kv_heads=8, n_q_heads=128)
     batch = 4
     assert api.decode_workspace_bytes(p, batch) > api.NOALLOC_SCRATCH_BYTES
     stride = (api.anchorkv_bytes(p)["total_bytes"] + 255) // 256 * 256
