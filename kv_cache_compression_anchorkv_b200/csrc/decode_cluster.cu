@@ -16,27 +16,30 @@
 // Work split.  The C CTAs of a cluster share one (sequence, head):
 //  1. CTA r computes P for anchor slots [r kc, (r+1) kc) and stores them into
 //     every CTA's shared memory (distributed shared memory);
-//  2. each CTA streams its 128-token tiles in chunks of 256 tokens, one per
-//     thread (warp w = bitmap word w).  A chunk's token records, bitmap words,
-//     residual codes and scales are copied into shared memory with cp.async
-//     one chunk ahead, so the loop reads only shared memory:
-//       a. anchor logits; each residual's rank in the chunk (= its staged
-//          record) from the word's prefix count;
-//       b. key residual logits over the chunk's key records, one warp per
-//          32/G records (lane = code byte), partial dot products reduced by a
-//          transposed butterfly, scattered to their tokens;
-//       c. the chunk maximum; the running maximum is only raised when a chunk
-//          exceeds it by 2^8 (so rescaling is rare);
-//       d. probabilities, value-anchor weights W by shared-memory atomics and
-//          each value record's weights p sigma~;
-//       e. value residual sums Z over the chunk's value records (lane = code
-//          byte, packed f32x2 FMAs);
+//  2. each CTA walks its 128-token tiles in chunks of at most 1024 tokens
+//     whose residual records fit the 768-record staging buffer.  A chunk's
+//     token records, bitmap words, residual codes and scales are copied into
+//     shared memory with cp.async; each thread owns 4 tokens (token
+//     tid + 256 u, so warp w reads bitmap words w + 8 u) and keeps their
+//     scores in registers:
+//       a. anchor logits, and each residual's rank in the chunk (= its staged
+//          record) from a prefix count over the chunk's bitmap words;
+//       b. key residual logits per key record, one warp per 32/G records
+//          (lane = code byte), partial dot products reduced by a transposed
+//          butterfly, stored by rank;
+//       c. each token adds its record's logit; the chunk maximum raises the
+//          running maximum only when it exceeds it by 2^8 (rescaling is rare);
+//       d. probabilities, value-anchor weights W by shared-memory atomics, and
+//          each value record's weights p sigma~ stored by rank;
+//       e. value residual sums Z over the value records (lane = code byte,
+//          packed f32x2 FMAs);
 //  3. the cluster merges (max, sum, W, Z) through distributed shared memory:
 //     CTA r forms W for its slot slice and multiplies it with its slice of
 //     value anchors, the CTA owning head j undoes the rotation of its Z, and
 //     the partial outputs are summed into the output rows.
 // Scores are kept in log2 units (q is pre-multiplied by log2 e).
 #include <algorithm>
+#include <cstddef>
 #include <mutex>
 
 #include "common.cuh"
@@ -47,14 +50,17 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kCH = 256;                   // tokens per chunk = threads
-constexpr int kTPC = kCH / kTile;          // tiles per chunk
-constexpr int kWPC = kCH / 32;             // bitmap words per chunk and side = warps
+constexpr int kTT = 1024;                  // most tokens per chunk
+constexpr int kTPT = kTT / kThreads;       // tokens per thread
+constexpr int kTilesPC = kTT / kTile;      // most tiles per chunk
+constexpr int kWordsPC = kTT / 32;         // bitmap words per chunk and side
+constexpr int kRC = 768;                   // residual records staged per chunk, both sides
 constexpr int kLutCopies = 8;              // lane l reads copy l % 8: conflict-free float4 lookups
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleGap = 8.0f;        // log2 units
 constexpr int kMaxC = 16;
-static_assert(kCH == kThreads && kWPC == kWarps, "one token per thread, one bitmap word per warp");
+static_assert(kRC >= 2 * kTile, "one tile's records must fit a chunk");
+static_assert(kWordsPC == 4 * kWarps, "warp w reads bitmap words w + 8u");
 
 struct CArgs {
   const uint8_t* comp;
@@ -71,21 +77,23 @@ struct CArgs {
   float* out;
 };
 
-// One chunk's token records, bitmap words, residual codes and scales, per side.
+// One chunk's token records, bitmap words (with prefix counts), residual
+// codes (key records, then value records) and scales.
 struct Stage {
-  uint32_t tok[2][kCH];
-  uint32_t bm[2][kWPC];
-  uint8_t codes[2][kCH * kCodeBytes];
-  uint16_t sig[2][kCH + 8];
+  uint8_t codes[kRC * kCodeBytes];   // 16-byte copies: first, at offset 0
+  uint32_t tok[2][kTT];
+  uint32_t bm[2][kWordsPC];          // 16-byte copies: offset 32 KB
+  int wpre[2][kWordsPC + 1];
+  uint16_t sig[2][kRC + 8];          // 4-byte copies
 };
+static_assert(offsetof(Stage, bm) % 16 == 0 && offsetof(Stage, sig) % 4 == 0, "cp.async alignment");
 
 // Shared-memory carve-up (bytes), identical on host and device.
 struct SmemPlan {
-  int lut, stage, pf, P, W, sc, listK, wV, vsl, zred, oacc, ofin, misc, total;
+  int lut, stage, pf, P, W, rbuf, vsl, zred, oacc, ofin, misc, total;
 };
 
 __host__ __device__ inline int align_up(int x, int a) { return (x + a - 1) / a * a; }
-__host__ __device__ inline int stage_bytes() { return align_up((int)sizeof(Stage), 16); }
 __host__ __device__ inline int gp_of(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8; }
 
 // tpc: most tiles one CTA owns (its tile prefixes are kept for the whole
@@ -94,13 +102,11 @@ __host__ __device__ inline SmemPlan smem_plan(int G, int k, int tpc, int kc, int
   SmemPlan s;
   int cur = 0;
   s.lut = cur; cur += 256 * kLutCopies * 16;
-  s.stage = cur; cur += 2 * stage_bytes();
+  s.stage = cur; cur = align_up(cur + (int)sizeof(Stage), 16);
   s.pf = cur; cur = align_up(cur + 4 * 2 * (tpc + 1), 16);
   s.P = cur; cur = align_up(cur + 4 * G * k, 16);
   s.W = cur; cur = align_up(cur + 4 * G * k, 16);
-  s.sc = cur; cur = align_up(cur + 4 * G * kCH, 16);
-  s.listK = cur; cur += 4 * kCH;
-  s.wV = cur; cur += 4 * gp_of(G) * kCH;
+  s.rbuf = cur; cur = align_up(cur + 4 * gp_of(G) * kRC, 16);
   s.vsl = cur; cur = align_up(cur + kc * kD * elem, 16);
   s.zred = cur; cur += 4 * G * kD;
   s.oacc = cur; cur += 4 * G * kD;
@@ -163,42 +169,58 @@ __device__ __forceinline__ void transpose_reduce32(float (&v)[32], int lane) {
   }
 }
 
-// Residual records of a chunk for one side: [r0, r0 + n) with codes staged
-// from record r0 and scales staged from the even record w0.
+// Records of tiles [i0, i1) of one side (relative prefix indices), clamped
+// to [0, R) and to `cap` records: [r0, r0 + n), scales staged from the even
+// record w0.
 struct RecRange {
   int64_t r0, w0;
   int n;
 };
-__device__ __forceinline__ RecRange rec_range(const int* pfs, int i0, int i1, int64_t R) {
+__device__ __forceinline__ RecRange rec_range(const int* pfs, int i0, int i1, int64_t R, int cap) {
   RecRange rr;
   int64_t lo = pfs[i0], hi = pfs[i1];
   lo = lo < 0 ? 0 : (lo > R ? R : lo);
   hi = hi > R ? R : hi;
   int64_t n = hi - lo;
-  n = n < 0 ? 0 : (n > kCH ? kCH : n);
+  n = n < 0 ? 0 : (n > cap ? cap : n);
   rr.r0 = lo;
   rr.n = (int)n;
   rr.w0 = lo & ~(int64_t)1;
   return rr;
 }
 
-// Issues cp.async copies of the chunk of tiles [t0, t1) (CTA tile range
-// starting at tb, tile prefixes pf[2][.]) into st.
+// End tile of the chunk that starts at tile t0: at most kTilesPC tiles and
+// kRC records of both sides (at least one tile).
+__device__ __forceinline__ int chunk_end(const int* pf, int pf_stride, int tb, int te, int t0) {
+  int t1 = t0 + 1;
+  while (t1 < te && t1 - t0 < kTilesPC) {
+    const int64_t nk = (int64_t)pf[t1 + 1 - tb] - pf[t0 - tb];
+    const int64_t nv = (int64_t)pf[pf_stride + t1 + 1 - tb] - pf[pf_stride + t0 - tb];
+    if (nk + nv > kRC) break;
+    ++t1;
+  }
+  return t1;
+}
+
+// Issues cp.async copies of the chunk of tiles [t0, t1) into st.
 __device__ __forceinline__ void stage_chunk(Stage& st, const CArgs& a, const uint8_t* comp, const int* pf,
                                             int pf_stride, int h, int tb, int t0, int t1) {
   const int tok0 = t0 * kTile, tok1 = min(a.N, t1 * kTile);
   const int ntok = tok1 - tok0, nt = t1 - t0;
   const uint8_t* codes = comp + a.L.off_res_codes;
   const uint16_t* sig = reinterpret_cast<const uint16_t*>(comp + a.L.off_res_sigma);
+  const RecRange rK = rec_range(pf, t0 - tb, t1 - tb, a.R, kRC);
+  const RecRange rV = rec_range(pf + pf_stride, t0 - tb, t1 - tb, a.R, kRC - rK.n);
   for (int side = 0; side < 2; ++side) {
     const uint32_t* tok = reinterpret_cast<const uint32_t*>(comp + a.L.off_tok) + ((int64_t)side * a.H + h) * a.N;
     const uint32_t* bm = reinterpret_cast<const uint32_t*>(comp + a.L.off_bitmap) +
                          ((int64_t)side * a.H + h) * a.n_tiles * 4;
     for (int i = threadIdx.x; i < ntok; i += kThreads) cp_async4(&st.tok[side][i], tok + tok0 + i);
     for (int i = threadIdx.x; i < nt; i += kThreads) cp_async16(&st.bm[side][4 * i], bm + (int64_t)(t0 + i) * 4);
-    const RecRange rr = rec_range(pf + side * pf_stride, t0 - tb, t1 - tb, a.R);
+    const RecRange& rr = side ? rV : rK;
+    uint8_t* dst = st.codes + (side ? rK.n * kCodeBytes : 0);
     for (int i = threadIdx.x; i < 2 * rr.n; i += kThreads)
-      cp_async16(&st.codes[side][16 * i], codes + rr.r0 * kCodeBytes + 16 * i);
+      cp_async16(dst + 16 * i, codes + rr.r0 * kCodeBytes + 16 * i);
     // scales: whole 4-byte words from the even record w0; a last record that
     // ends the array on an odd count is read on its own
     const int64_t end = rr.r0 + rr.n;
@@ -229,14 +251,12 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
   const int tpc = (a.n_tiles + (int)C - 1) / (int)C;
   const SmemPlan sp = smem_plan(G, k, tpc, kc, (int)sizeof(T));
   float4* lut = reinterpret_cast<float4*>(smem + sp.lut);
-  uint8_t* stg = smem + sp.stage;
+  Stage& st = *reinterpret_cast<Stage*>(smem + sp.stage);
   int* pf = reinterpret_cast<int*>(smem + sp.pf);        // [2][tpc + 1]
   const int pf_stride = tpc + 1;
   float* P = reinterpret_cast<float*>(smem + sp.P);
   float* W = reinterpret_cast<float*>(smem + sp.W);
-  float* sc = reinterpret_cast<float*>(smem + sp.sc);
-  int* listK = reinterpret_cast<int*>(smem + sp.listK);
-  float* wV = reinterpret_cast<float*>(smem + sp.wV);     // [kCH][GP]
+  float* rbuf = reinterpret_cast<float*>(smem + sp.rbuf);  // [kRC][GP] per-record values
   T* vsl = reinterpret_cast<T*>(smem + sp.vsl);
   float* zred = reinterpret_cast<float*>(smem + sp.zred);
   float* oacc = reinterpret_cast<float*>(smem + sp.oacc);
@@ -250,7 +270,6 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
   float* pm = scl + kMaxC * 8;          // [kMaxC][8] peers' running max
   float* pl = pm + kMaxC * 8;           // [kMaxC][8] peers' denominators
   float* red = pl + kMaxC * 8;          // [kWarps][8] block reductions
-  auto stage = [&](int c) -> Stage& { return *reinterpret_cast<Stage*>(stg + (c & 1) * stage_bytes()); };
 
   const uint8_t* comp = a.comp + (int64_t)b * a.stride;
   const T* qg = reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.H * G + (int64_t)h * G) * kD;
@@ -259,7 +278,6 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
 
   // token tiles of this CTA and anchor slots of its slice
   const int tb = (int)((int64_t)a.n_tiles * r / C), te = (int)((int64_t)a.n_tiles * (r + 1) / C);
-  const int n_chunks = (te - tb + kTPC - 1) / kTPC;
   const int s0 = min(k, (int)r * kc), s1 = min(k, s0 + kc), nsl = s1 - s0;
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
@@ -277,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
   cp_commit();
   float* qs = ofin;          // q * log2e / sqrt(D) until the merge
   float* qr = zred;          // H(s . q) * log2e / D until the merge
-  float* Pown = sc;          // this CTA's slots of P [G][kc] until the first chunk
+  float* Pown = rbuf;        // this CTA's slots of P [G][kc] until the first chunk
   const float isd = rsqrtf((float)kD);
   for (int i = tid; i < G * kD; i += kThreads) qs[i] = to_f<T>(qg[i]) * (isd * kLog2e);
   for (int i = tid; i < 256 * kLutCopies; i += kThreads) {
@@ -309,7 +327,8 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
   }
   cp_wait<0>();
   __syncthreads();
-  if (n_chunks > 0) stage_chunk(stage(0), a, comp, pf, pf_stride, h, tb, tb, min(te, tb + kTPC));
+  int t0 = tb, t1 = (te > tb) ? chunk_end(pf, pf_stride, tb, te, tb) : tb;
+  if (t1 > t0) stage_chunk(st, a, comp, pf, pf_stride, h, tb, t0, t1);
   cp_commit();
   // P into every CTA of the cluster, once all of them have started (the
   // arrive is at kernel entry)
@@ -336,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
 
   // Raises the running max of each head to the chunk's if it exceeds it by
   // kRescaleGap, rescaling W, Z, the tail sums and the partial sums.  `mine`
-  // holds this thread's score per head (-inf if it has none).
+  // holds this thread's maximum per head (-inf if it has none).
   auto update_max = [&](const float (&mine)[GP]) {
 #pragma unroll
     for (int j = 0; j < GP; ++j) {
@@ -373,41 +392,55 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
     }
   };
 
-  // ---- token chunks: thread tid <-> token tid of the chunk, warp <-> word
+  // ---- token chunks
   const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int c = 0; c < n_chunks; ++c) {
-    const int t0 = tb + c * kTPC, t1 = min(te, t0 + kTPC);
-    if (c + 1 < n_chunks) stage_chunk(stage(c + 1), a, comp, pf, pf_stride, h, tb, t1, min(te, t1 + kTPC));
-    cp_commit();
-    cp_wait<1>();
+  while (t1 > t0) {
+    cp_wait<0>();
     __syncthreads();
-    const Stage& st = stage(c);
     const int nt = min(a.N, t1 * kTile) - t0 * kTile;
-    const RecRange rK = rec_range(pf, t0 - tb, t1 - tb, a.R);
-    const RecRange rV = rec_range(pf + pf_stride, t0 - tb, t1 - tb, a.R);
-    // (a) anchor logits; residual ranks
-    const bool valid = tid < nt;
-    const uint32_t wK = st.bm[0][warp] & word_mask(warp, nt);
-    const uint32_t wV_ = st.bm[1][warp] & word_mask(warp, nt);
-    const int preK = __reduce_add_sync(0xffffffffu, lane < warp ? __popc(st.bm[0][lane & (kWPC - 1)] & word_mask(lane, nt)) : 0);
-    const int preV = __reduce_add_sync(0xffffffffu, lane < warp ? __popc(st.bm[1][lane & (kWPC - 1)] & word_mask(lane, nt)) : 0);
-    const int nK = min(rK.n, __reduce_add_sync(0xffffffffu, lane < kWPC ? __popc(st.bm[0][lane & (kWPC - 1)] & word_mask(lane, nt)) : 0));
-    const int nV = min(rV.n, __reduce_add_sync(0xffffffffu, lane < kWPC ? __popc(st.bm[1][lane & (kWPC - 1)] & word_mask(lane, nt)) : 0));
-    const bool hasK = (wK >> lane) & 1u, hasV = (wV_ >> lane) & 1u;
-    const int rankK = preK + __popc(wK & lt_mask), rankV = preV + __popc(wV_ & lt_mask);
-    uint32_t xV = 0u;
-    if (valid) {
-      const uint32_t x = st.tok[0][tid];
-      const int slot = min((int)(x & 0xFFFFu), k - 1);
-      const float g = half_bits_to_f(x >> 16);
+    const RecRange rK = rec_range(pf, t0 - tb, t1 - tb, a.R, kRC);
+    const RecRange rV = rec_range(pf + pf_stride, t0 - tb, t1 - tb, a.R, kRC - rK.n);
+    // prefix counts of the bitmap words (warp 0: keys, warp 1: values)
+    if (warp < 2) {
+      const int side = warp;
+      const uint32_t w0 = st.bm[side][lane] & word_mask(lane, nt);
+      int incl = __popc(w0);
 #pragma unroll
-      for (int j = 0; j < GP; ++j)
-        if (j < G) sc[j * kCH + tid] = g * P[j * k + slot];
-      if (hasK && rankK < nK) listK[rankK] = tid;
-      xV = st.tok[1][tid];
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      st.wpre[side][lane] = incl - __popc(w0);
+      if (lane == 31) st.wpre[side][kWordsPC] = incl;
     }
     __syncthreads();
-    // (b) key residual logits, groups of RB records per warp
+    const int nK = min(rK.n, st.wpre[0][kWordsPC]);
+    const int nV = min(rV.n, st.wpre[1][kWordsPC]);
+    // (a) anchor logits, residual ranks
+    float s[kTPT][GP];
+    int rankK[kTPT], rankV[kTPT];
+    uint32_t xV[kTPT];
+#pragma unroll
+    for (int u = 0; u < kTPT; ++u) {
+      const int i = tid + u * kThreads, wd = warp + u * kWarps;
+      const uint32_t wK = st.bm[0][wd] & word_mask(wd, nt);
+      const uint32_t wVv = st.bm[1][wd] & word_mask(wd, nt);
+      rankK[u] = ((wK >> lane) & 1u) ? st.wpre[0][wd] + __popc(wK & lt_mask) : kRC;
+      rankV[u] = ((wVv >> lane) & 1u) ? st.wpre[1][wd] + __popc(wVv & lt_mask) : kRC;
+      xV[u] = 0u;
+#pragma unroll
+      for (int j = 0; j < GP; ++j) s[u][j] = -INFINITY;
+      if (i < nt) {
+        const uint32_t x = st.tok[0][i];
+        const int slot = min((int)(x & 0xFFFFu), k - 1);
+        const float g = half_bits_to_f(x >> 16);
+#pragma unroll
+        for (int j = 0; j < GP; ++j)
+          if (j < G) s[u][j] = g * P[j * k + slot];
+        xV[u] = st.tok[1][i];
+      }
+    }
+    // (b) key residual logits, groups of RB records per warp, stored by rank
     {
       constexpr int RB = 32 / GP;
       const int64_t sk = rK.r0 - rK.w0;
@@ -419,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
           uint32_t byte = 0u;
           float sg = 0.f;
           if (rho < nK) {
-            byte = st.codes[0][rho * kCodeBytes + lane];
+            byte = st.codes[rho * kCodeBytes + lane];
             sg = half_bits_to_f(st.sig[0][rho + sk]);
           }
           const float4 lv = lut[byte * kLutCopies + (lane & (kLutCopies - 1))];
@@ -433,40 +466,56 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
           }
         }
         transpose_reduce32(v, lane);
-        const int rho = g0 + lane / GP, j = lane % GP;
-        if (rho < nK && j < G) sc[j * kCH + listK[rho]] += v[0];
+        if (g0 + lane / GP < nK) rbuf[(g0 + lane / GP) * GP + lane % GP] = v[0];
       }
     }
     __syncthreads();
-    // (c) chunk maximum
+    // (c) key residual logits into the scores, chunk maximum
     float mine[GP];
 #pragma unroll
-    for (int j = 0; j < GP; ++j) mine[j] = (valid && j < G) ? sc[j * kCH + tid] : -INFINITY;
-    update_max(mine);
-    // (d) probabilities, value-anchor weights, value-record weights
-    if (valid) {
-      const int slot = min((int)(xV & 0xFFFFu), k - 1);
-      const float g = half_bits_to_f(xV >> 16);
-      const bool rec = hasV && rankV < nV;
-      const float sg = rec ? half_bits_to_f(st.sig[1][rankV + (rV.r0 - rV.w0)]) : 0.f;
+    for (int j = 0; j < GP; ++j) mine[j] = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < GP; ++j) {
-        if (j < G) {
-          const float p = exp2f(mine[j] - mrun[j]);
-          lpart[j] += p;
-          atomicAdd(&W[j * k + slot], p * g);
-          if (rec) wV[rankV * GP + j] = p * sg;
+    for (int u = 0; u < kTPT; ++u) {
+      if (rankK[u] < nK) {
+#pragma unroll
+        for (int j = 0; j < GP; ++j) s[u][j] += rbuf[rankK[u] * GP + j];
+      }
+#pragma unroll
+      for (int j = 0; j < GP; ++j) mine[j] = fmaxf(mine[j], s[u][j]);
+    }
+    update_max(mine);
+    // (d) probabilities, value-anchor weights, value-record weights by rank
+    {
+      const int64_t sv = rV.r0 - rV.w0;
+#pragma unroll
+      for (int u = 0; u < kTPT; ++u) {
+        const int i = tid + u * kThreads;
+        if (i < nt) {
+          const int slot = min((int)(xV[u] & 0xFFFFu), k - 1);
+          const float g = half_bits_to_f(xV[u] >> 16);
+          const bool rec = rankV[u] < nV;
+          const float sg = rec ? half_bits_to_f(st.sig[1][rankV[u] + sv]) : 0.f;
+#pragma unroll
+          for (int j = 0; j < GP; ++j) {
+            if (j < G) {
+              const float p = exp2f(s[u][j] - mrun[j]);
+              lpart[j] += p;
+              atomicAdd(&W[j * k + slot], p * g);
+              if (rec) rbuf[rankV[u] * GP + j] = p * sg;
+            }
+          }
         }
       }
     }
     __syncthreads();
     // (e) value residuals: Z += (p sigma~) lev(c), lane = code byte
     {
+      const uint8_t* vcodes = st.codes + rK.n * kCodeBytes;
       int rho = warp;
       for (; rho + 3 * kWarps < nV; rho += 4 * kWarps) {
         uint32_t byte[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) byte[u] = st.codes[1][(rho + u * kWarps) * kCodeBytes + lane];
+        for (int u = 0; u < 4; ++u) byte[u] = vcodes[(rho + u * kWarps) * kCodeBytes + lane];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const float4 lv = lut[byte[u] * kLutCopies + (lane & (kLutCopies - 1))];
@@ -475,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
 #pragma unroll
           for (int j = 0; j < GP; ++j) {
             if (j < G) {
-              const float w = wV[rr * GP + j];
+              const float w = rbuf[rr * GP + j];
               const float2 ww = make_float2(w, w);
               z[j][0] = __ffma2_rn(l01, ww, z[j][0]);
               z[j][1] = __ffma2_rn(l23, ww, z[j][1]);
@@ -484,13 +533,13 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
         }
       }
       for (; rho < nV; rho += kWarps) {
-        const uint32_t byte = st.codes[1][rho * kCodeBytes + lane];
+        const uint32_t byte = vcodes[rho * kCodeBytes + lane];
         const float4 lv = lut[byte * kLutCopies + (lane & (kLutCopies - 1))];
         const float2 l01 = make_float2(lv.x, lv.y), l23 = make_float2(lv.z, lv.w);
 #pragma unroll
         for (int j = 0; j < GP; ++j) {
           if (j < G) {
-            const float w = wV[rho * GP + j];
+            const float w = rbuf[rho * GP + j];
             const float2 ww = make_float2(w, w);
             z[j][0] = __ffma2_rn(l01, ww, z[j][0]);
             z[j][1] = __ffma2_rn(l23, ww, z[j][1]);
@@ -499,18 +548,24 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
       }
     }
     __syncthreads();
+    // next chunk
+    t0 = t1;
+    t1 = (t0 < te) ? chunk_end(pf, pf_stride, tb, te, t0) : t0;
+    if (t1 > t0) stage_chunk(st, a, comp, pf, pf_stride, h, tb, t0, t1);
+    cp_commit();
   }
   cp_wait<0>();
   __syncthreads();
 
-  // ---- exact tail tokens, split over the cluster
+  // ---- exact tail tokens, split over the cluster (scores in rbuf [G][256])
   if (a.tail_len > 0) {
+    float* ts = rbuf;
     const int per = (a.tail_len + (int)C - 1) / (int)C;
     const int ta = min(a.tail_len, (int)r * per), tz = min(a.tail_len, ta + per);
     const T* Kt = reinterpret_cast<const T*>(a.Kt) + ((int64_t)b * a.H + h) * a.tail_cap * kD;
     const T* Vt = reinterpret_cast<const T*>(a.Vt) + ((int64_t)b * a.H + h) * a.tail_cap * kD;
-    for (int base = ta; base < tz; base += kCH) {
-      const int nt = min(kCH, tz - base);
+    for (int base = ta; base < tz; base += kThreads) {
+      const int nt = min(kThreads, tz - base);
       for (int i = warp; i < nt; i += kWarps) {
         float kf[4];
         load4<T>(Kt + (int64_t)(base + i) * kD + lane * 4, kf);
@@ -519,20 +574,20 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
 #pragma unroll
           for (int e = 0; e < 4; ++e) d = fmaf(qs[j * kD + lane * 4 + e], kf[e], d);
           d = warp_sum(d);
-          if (lane == 0) sc[j * kCH + i] = d;
+          if (lane == 0) ts[j * kThreads + i] = d;
         }
       }
       __syncthreads();
       float mine[GP];
 #pragma unroll
-      for (int j = 0; j < GP; ++j) mine[j] = (tid < nt && j < G) ? sc[j * kCH + tid] : -INFINITY;
+      for (int j = 0; j < GP; ++j) mine[j] = (tid < nt && j < G) ? ts[j * kThreads + tid] : -INFINITY;
       update_max(mine);
       if (tid < nt) {
 #pragma unroll
         for (int j = 0; j < GP; ++j) {
           if (j < G) {
             const float p = exp2f(mine[j] - mrun[j]);
-            sc[j * kCH + tid] = p;
+            ts[j * kThreads + tid] = p;
             lpart[j] += p;
           }
         }
@@ -542,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
         float vf[4];
         load4<T>(Vt + (int64_t)(base + i) * kD + lane * 4, vf);
         for (int j = 0; j < G; ++j) {
-          const float p = sc[j * kCH + i];
+          const float p = ts[j * kThreads + i];
 #pragma unroll
           for (int e = 0; e < 4; ++e) atomicAdd(&oacc[j * kD + lane * 4 + e], p * vf[e]);
         }
@@ -581,9 +636,9 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
     float Lj = 0.f;
     for (uint32_t rr = 0; rr < C; ++rr) {
       const float m = pm[rr * 8 + tid];
-      const float s = (m == -INFINITY) ? 0.f : exp2f(m - M);
-      scl[rr * 8 + tid] = s;
-      Lj = fmaf(pl[rr * 8 + tid], s, Lj);
+      const float sc = (m == -INFINITY) ? 0.f : exp2f(m - M);
+      scl[rr * 8 + tid] = sc;
+      Lj = fmaf(pl[rr * 8 + tid], sc, Lj);
     }
     Lfin[tid] = Lj;
   }
@@ -592,21 +647,21 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
   // reads any more), then W V_a
   float* wt = P;
   for (int i = tid; i < G * nsl; i += kThreads) {
-    const int j = i / nsl, s = s0 + i % nsl;
+    const int j = i / nsl, sl = s0 + i % nsl;
     float w = 0.f;
 #pragma unroll 4
-    for (uint32_t rr = 0; rr < C; ++rr) w = fmaf(*peer(&W[j * k + s], rr), scl[rr * 8 + j], w);
-    wt[j * kc + (s - s0)] = w;
+    for (uint32_t rr = 0; rr < C; ++rr) w = fmaf(*peer(&W[j * k + sl], rr), scl[rr * 8 + j], w);
+    wt[j * kc + (sl - s0)] = w;
   }
   __syncthreads();
   for (int i = tid; i < G * kD; i += kThreads) {
     const int j = i / kD, d = i % kD;
     float o = 0.f;
-    for (int s = 0; s < nsl; ++s) o = fmaf(wt[j * kc + s], to_f<T>(vsl[s * kD + d]), o);
+    for (int sl = 0; sl < nsl; ++sl) o = fmaf(wt[j * kc + sl], to_f<T>(vsl[sl * kD + d]), o);
     ofin[i] = o;
   }
   // residual sums and exact tail of the heads this CTA owns (j = r mod C),
-  // summed over the cluster into sc
+  // summed over the cluster into rbuf
   const int n_own = (G - (int)r + (int)C - 1) / (int)C;   // heads r, r + C, ...
   for (int i = tid; i < n_own * 2 * kD; i += kThreads) {
     const int jj = i / (2 * kD), kind = (i / kD) & 1, d = i % kD;
@@ -615,19 +670,19 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
     float acc = 0.f;
 #pragma unroll 4
     for (uint32_t rr = 0; rr < C; ++rr) acc = fmaf(*peer(&src[j * kD + d], rr), scl[rr * 8 + j], acc);
-    sc[i] = acc;
+    rbuf[i] = acc;
   }
   __syncthreads();
   for (int jj = warp; jj < n_own; jj += kWarps) {
     const int j = (int)r + jj * (int)C;
     float zv[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) zv[e] = sc[jj * 2 * kD + lane * 4 + e];
+    for (int e = 0; e < 4; ++e) zv[e] = rbuf[jj * 2 * kD + lane * 4 + e];
     fwht128<float>(zv);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int d = lane * 4 + e;
-      ofin[j * kD + d] += zv[e] * isd * sign_of(a, d) + sc[jj * 2 * kD + kD + d];
+      ofin[j * kD + d] += zv[e] * isd * sign_of(a, d) + rbuf[jj * 2 * kD + kD + d];
     }
   }
   __syncthreads();
@@ -718,9 +773,9 @@ int plan_bytes(const Plan& pl, int C) {
 }
 
 // Shared memory of a C-CTA cluster fits: the plan within 227 KB, and a CTA's
-// slots of P fit the chunk score buffer that holds them in the prologue.
+// slots of P fit the record buffer that holds them in the prologue.
 bool fits(const Plan& pl, int C) {
-  if ((pl.k + C - 1) / C > kCH) return false;
+  if ((pl.k + C - 1) / C > kRC) return false;
   return plan_bytes(pl, C) <= 227 * 1024;
 }
 
