@@ -30,60 +30,76 @@ namespace {
 
 // ---------------------------------------------------------------- project
 
-// grid (ceil(N / 128), H, 2), 128 threads: the block stages 128 token rows
-// of one (side, head) in shared memory (coalesced loads, rows padded to
-// D + 1 floats so that thread r reading row r is bank-conflict free); each
-// thread then takes one token end to end in fp64.
-constexpr int kProjRows = 128;
+// grid (ceil(N / 64), H, 2), 256 threads: 4 lanes per token (a warp takes 8
+// consecutive tokens of one (side, head)).  Lane q of a token reads the
+// 16-byte pieces q, q + 4, ... of the token's row and of its anchor's row,
+// so every load instruction reads 64 contiguous bytes of 8 rows, and one
+// pass accumulates d = <x, x_a> and n = ||x||^2 in fp64.  The 4 partial sums
+// are combined by two shuffles.  With the stored g = fp16(d / a2),
+// a2 = ||x_a||^2, the residual energy is r2 = n - 2 g d + g^2 a2: the sums of
+// exact bf16/fp32 products are exact or within fp64 rounding, so the
+// cancellation leaves an error near 1e-12 ||x||^2.
+constexpr int kProjTokens = 64;
 
 template <typename T>
-__global__ void __launch_bounds__(kProjRows)
+__device__ __forceinline__ void load16(const T* p, float (&o)[16 / sizeof(T)]);
+template <>
+__device__ __forceinline__ void load16<float>(const float* p, float (&o)[4]) {
+  const float4 v = *reinterpret_cast<const float4*>(p);
+  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfloat16* p, float (&o)[8]) {
+  const uint4 v = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    o[2 * i] = __uint_as_float(w[i] << 16);
+    o[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
 project_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ anc_k,
                const T* __restrict__ anc_v, const double* __restrict__ anc_n2, const int* __restrict__ slot_of,
                const float* __restrict__ a2s, const float* __restrict__ kus, uint32_t* __restrict__ tok,
                float* __restrict__ util, int N, int H, int k, int obs_rb) {
-  extern __shared__ float xt[];                       // [kProjRows][kD + 1]
-  const int t0 = blockIdx.x * kProjRows, h = blockIdx.y, side = blockIdx.z;
-  const int nv = min(kProjRows, N - t0);
-  const T* X = (side ? V : K) + ((int64_t)h * N + t0) * kD;
-  for (int i = threadIdx.x; i < nv * (kD / 4); i += kProjRows) {
-    const int r = i / (kD / 4), c = (i % (kD / 4)) * 4;
-    float f[4];
-    load4<T>(X + (int64_t)r * kD + c, f);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) xt[r * (kD + 1) + c + e] = f[e];
-  }
-  __syncthreads();
-  const int r = threadIdx.x;
-  if (r >= nv) return;
-  const int t = t0 + r;
-  const int64_t f = ((int64_t)side * H + h) * N + t;
-  const uint32_t slot = tok[f] & 0xFFFFu;
+  constexpr int EPV = 16 / (int)sizeof(T);        // elements per 16-byte load
+  constexpr int STEPS = kD / (4 * EPV);           // loads per lane and row
+  const int q = threadIdx.x & 3;
+  const int t = blockIdx.x * kProjTokens + (threadIdx.x >> 2), h = blockIdx.y, side = blockIdx.z;
+  const bool valid = t < N;
+  const int tt = valid ? t : N - 1;               // every lane takes part in the shuffles
+  const int64_t f = ((int64_t)side * H + h) * N + tt;
+  const uint32_t slot = min(tok[f] & 0xFFFFu, (uint32_t)(k - 1));
+  const T* x = (side ? V : K) + ((int64_t)h * N + tt) * kD;
   const T* a = (side ? anc_v : anc_k) + ((int64_t)h * k + slot) * kD;
-  const float* xr = xt + r * (kD + 1);
-  const bool is_anchor = slot_of[(int64_t)h * N + t] >= 0;
-  double dot = 0.0;
-  for (int d = 0; d < kD; d += 4) {
-    float af[4];
-    load4<T>(a + d, af);
+  double dot = 0.0, nx = 0.0;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) dot = fma((double)xr[d + e], (double)af[e], dot);
+  for (int i = 0; i < STEPS; ++i) {
+    const int d = (4 * i + q) * EPV;
+    float xf[EPV], af[EPV];
+    load16<T>(x + d, xf);
+    load16<T>(a + d, af);
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) {
+      dot = fma((double)xf[e], (double)af[e], dot);
+      nx = fma((double)xf[e], (double)xf[e], nx);
+    }
   }
+  dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+  nx += __shfl_xor_sync(0xffffffffu, nx, 1);
+  dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+  nx += __shfl_xor_sync(0xffffffffu, nx, 2);
+  if (!valid || q != 0) return;
+  const bool is_anchor = slot_of[(int64_t)h * N + t] >= 0;
   const double n2 = anc_n2[((int64_t)side * H + h) * k + slot];
   double gamma = (n2 > 0.0) ? dot / n2 : 0.0;
   if (is_anchor) gamma = 1.0;
   const uint16_t gb = half_bits_rn(gamma);
   const double g = (double)half_bits_to_f(gb);
-  double r2 = 0.0;
-  for (int d = 0; d < kD; d += 4) {
-    float af[4];
-    load4<T>(a + d, af);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const double rr = (double)xr[d + e] - g * (double)af[e];
-      r2 = fma(rr, rr, r2);
-    }
-  }
+  const double r2 = fmax(0.0, nx - 2.0 * g * dot + g * g * n2);
   tok[f] = slot | ((uint32_t)gb << 16);
   float u;
   if (is_anchor) {
@@ -387,24 +403,21 @@ CodecConst make_cc(const Plan& pl) {
 }  // namespace
 
 cudaError_t launch_project(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s) {
-  const dim3 blocks((pl.N + kProjRows - 1) / kProjRows, pl.H, 2);
-  const int smem = kProjRows * (kD + 1) * (int)sizeof(float);
+  const dim3 blocks((pl.N + kProjTokens - 1) / kProjTokens, pl.H, 2);
   auto* n2 = reinterpret_cast<const double*>(ws + pl.o_anc_n2);
   auto* slot_of = reinterpret_cast<const int*>(ws + pl.o_slot_of);
   auto* a2 = reinterpret_cast<const float*>(ws + pl.o_a2);
   auto* ku = reinterpret_cast<const float*>(ws + pl.o_ku);
   auto* tok = reinterpret_cast<uint32_t*>(out + pl.L.off_tok);
   auto* util = reinterpret_cast<float*>(ws + pl.o_util);
-  cudaFuncSetAttribute(project_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  cudaFuncSetAttribute(project_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (pl.p.dtype == ANCHORKV_BF16) {
-    project_kernel<__nv_bfloat16><<<blocks, kProjRows, smem, s>>>(
+    project_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
         (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
         reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_k),
         reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_v), n2, slot_of, a2, ku, tok, util,
         pl.N, pl.H, pl.k, pl.obs_rb);
   } else {
-    project_kernel<float><<<blocks, kProjRows, smem, s>>>(
+    project_kernel<float><<<blocks, 256, 0, s>>>(
         (const float*)K, (const float*)V, reinterpret_cast<const float*>(out + pl.L.off_anchors_k),
         reinterpret_cast<const float*>(out + pl.L.off_anchors_v), n2, slot_of, a2, ku, tok, util,
         pl.N, pl.H, pl.k, pl.obs_rb);

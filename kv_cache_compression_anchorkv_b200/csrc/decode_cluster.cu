@@ -60,6 +60,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleGap = 8.0f;        // log2 units
 constexpr int kMaxC = 16;
 static_assert(kRC >= 2 * kTile, "one tile's records must fit a chunk");
+static_assert(kWarps >= 8, "a warp per query head of a KV head (G <= 8)");
 static_assert(kWordsPC == 4 * kWarps, "warp w reads bitmap words w + 8u");
 
 struct CArgs {
@@ -281,8 +282,9 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
   const int s0 = min(k, (int)r * kc), s1 = min(k, s0 + kc), nsl = s1 - s0;
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
-  // ---- prologue: tile prefixes and value-anchor slice (async), query,
-  // tables, rotated query, P of this CTA's slots
+  // ---- prologue: every global load first (tile prefixes and value-anchor
+  // slice by cp.async, query and this warp's anchor keys into registers),
+  // then tables, rotated query and P of this CTA's slots
   for (int side = 0; side < 2; ++side) {
     const int* pfg = reinterpret_cast<const int*>(comp + a.L.off_tile_prefix) + ((int64_t)side * a.H + h) * (a.n_tiles + 1);
     for (int i = tid; i <= te - tb; i += kThreads) cp_async4(&pf[side * pf_stride + i], pfg + tb + i);
@@ -293,11 +295,28 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
     for (int i = tid; i < bytes / 16; i += kThreads) cp_async16(reinterpret_cast<uint8_t*>(vsl) + 16 * i, src + 16 * i);
   }
   cp_commit();
+  const float isd = rsqrtf((float)kD);
+  float qf[GP][4];                       // q * log2e / sqrt(D), this lane's 4 coordinates
+#pragma unroll
+  for (int j = 0; j < GP; ++j) {
+    if (j < G) {
+      load4<T>(qg + j * kD + lane * 4, qf[j]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) qf[j][e] *= isd * kLog2e;
+    } else {
+      qf[j][0] = qf[j][1] = qf[j][2] = qf[j][3] = 0.f;
+    }
+  }
+  constexpr int kPB = 4;                 // anchor rows in flight per warp
+  float af[kPB][4];
+#pragma unroll
+  for (int u = 0; u < kPB; ++u) {
+    const int sl = s0 + warp + u * kWarps;
+    if (sl < s1) load4<T>(ancK + (int64_t)sl * kD + lane * 4, af[u]);
+  }
   float* qs = ofin;          // q * log2e / sqrt(D) until the merge
   float* qr = zred;          // H(s . q) * log2e / D until the merge
   float* Pown = rbuf;        // this CTA's slots of P [G][kc] until the first chunk
-  const float isd = rsqrtf((float)kD);
-  for (int i = tid; i < G * kD; i += kThreads) qs[i] = to_f<T>(qg[i]) * (isd * kLog2e);
   for (int i = tid; i < 256 * kLutCopies; i += kThreads) {
     const int v = i / kLutCopies;
     lut[i] = make_float4(a.lev[v & 3], a.lev[(v >> 2) & 3], a.lev[(v >> 4) & 3], a.lev[(v >> 6) & 3]);
@@ -305,24 +324,41 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
   for (int i = tid; i < G * k; i += kThreads) W[i] = 0.f;
   for (int i = tid; i < G * kD; i += kThreads) oacc[i] = 0.f;
   if (tid < 8) { mrun[tid] = -INFINITY; lsum[tid] = 0.f; }
-  __syncthreads();
-  for (int j = warp; j < G; j += kWarps) {
-    float v[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) v[e] = qs[j * kD + lane * 4 + e] * sign_of(a, lane * 4 + e);
-    fwht128<float>(v);
+  for (int j = 0; j < GP; ++j) {          // warp j rotates head j (GP <= kWarps)
+    if (j < G && j == warp) {
+      float v[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) qr[j * kD + lane * 4 + e] = v[e] * isd;
+      for (int e = 0; e < 4; ++e) {
+        qs[j * kD + lane * 4 + e] = qf[j][e];
+        v[e] = qf[j][e] * sign_of(a, lane * 4 + e);
+      }
+      fwht128<float>(v);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) qr[j * kD + lane * 4 + e] = v[e] * isd;
+    }
   }
-  for (int s = s0 + warp; s < s1; s += kWarps) {
-    float af[4];
-    load4<T>(ancK + (int64_t)s * kD + lane * 4, af);
-    for (int j = 0; j < G; ++j) {
-      float d = 0.f;
+  for (int base = s0 + warp; base < s1; base += kPB * kWarps) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) d = fmaf(qs[j * kD + lane * 4 + e], af[e], d);
-      d = warp_sum(d);
-      if (lane == 0) Pown[j * kc + (s - s0)] = d;
+    for (int u = 0; u < kPB; ++u) {
+      const int sl = base + u * kWarps;
+      if (sl < s1) {
+#pragma unroll
+        for (int j = 0; j < GP; ++j) {
+          if (j < G) {
+            float d = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d = fmaf(qf[j][e], af[u][e], d);
+            d = warp_sum(d);
+            if (lane == 0) Pown[j * kc + (sl - s0)] = d;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kPB; ++u) {   // the next rows of this warp
+      const int sl = base + kPB * kWarps + u * kWarps;
+      if (sl < s1) load4<T>(ancK + (int64_t)sl * kD + lane * 4, af[u]);
     }
   }
   cp_wait<0>();
@@ -606,18 +642,30 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
     }
   }
 
-  // ---- per-CTA totals: Z into zred (qr is no longer needed), l into lsum
-  for (int i = tid; i < G * kD; i += kThreads) zred[i] = 0.f;
-  __syncthreads();
+  // ---- per-CTA totals: each warp's Z into the (free) stage buffer, summed
+  // over the warps into zred (qr is no longer needed); l into lsum
+  {
+    float* zw = reinterpret_cast<float*>(&st);       // [kWarps][G][kD]
 #pragma unroll
-  for (int j = 0; j < GP; ++j) {
-    if (j < G) {
-      atomicAdd(&zred[j * kD + lane * 4 + 0], z[j][0].x);
-      atomicAdd(&zred[j * kD + lane * 4 + 1], z[j][0].y);
-      atomicAdd(&zred[j * kD + lane * 4 + 2], z[j][1].x);
-      atomicAdd(&zred[j * kD + lane * 4 + 3], z[j][1].y);
-      const float l = warp_sum(lpart[j]);
-      if (lane == 0) atomicAdd(&lsum[j], l);
+    for (int j = 0; j < GP; ++j) {
+      if (j < G) {
+        *reinterpret_cast<float4*>(&zw[(warp * G + j) * kD + lane * 4]) =
+            make_float4(z[j][0].x, z[j][0].y, z[j][1].x, z[j][1].y);
+        const float l = warp_sum(lpart[j]);
+        if (lane == 0) red[warp * 8 + j] = l;
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < G * kD; i += kThreads) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) acc += zw[w * G * kD + i];
+      zred[i] = acc;
+    }
+    if (tid < G) {
+      float l = 0.f;
+      for (int w = 0; w < kWarps; ++w) l += red[w * 8 + tid];
+      lsum[tid] = l;
     }
   }
   __syncthreads();

@@ -441,22 +441,33 @@ obs_b_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
 }
 
 // ybar = sum of partials (split order); bf16 hi/lo copies and ||ybar_r||^2.
-__global__ void obs_ybar_kernel(ObsTc a, __nv_bfloat16* __restrict__ yh, __nv_bfloat16* __restrict__ yl,
-                                float* __restrict__ row_y2) {
-  __shared__ float red[4][128];
-  const int u = blockIdx.x, d = threadIdx.x, warp = d >> 5, lane = d & 31;
-  for (int r = 0; r < 128; ++r) {
-    float y = 0.f;
-    for (int s = 0; s < a.n_split; ++s) y += a.part_y[(((int64_t)u * a.n_split + s) * 128 + r) * 128 + d];
-    const __nv_bfloat16 hi = __float2bfloat16_rn(y);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(y - __bfloat162float(hi));
-    yh[((int64_t)u * 128 + r) * 128 + d] = hi;
-    yl[((int64_t)u * 128 + r) * 128 + d] = lo;
-    const float w = warp_sum(y * y);
-    if (lane == 0) red[warp][r] = w;
+// grid (U, 128 / kYbarRows), 128 threads: thread d sums coordinate d of
+// kYbarRows rows, all partial loads of a row in flight together.
+constexpr int kYbarRows = 4;
+__global__ void __launch_bounds__(128) obs_ybar_kernel(ObsTc a, __nv_bfloat16* __restrict__ yh,
+                                                       __nv_bfloat16* __restrict__ yl, float* __restrict__ row_y2) {
+  __shared__ float red[kYbarRows][4];
+  const int u = blockIdx.x, r0 = blockIdx.y * kYbarRows, d = threadIdx.x, warp = d >> 5, lane = d & 31;
+  const float* src = a.part_y + (int64_t)u * a.n_split * 128 * 128 + (int64_t)r0 * 128 + d;
+  float y[kYbarRows];
+#pragma unroll
+  for (int i = 0; i < kYbarRows; ++i) y[i] = 0.f;
+#pragma unroll 4
+  for (int sp = 0; sp < a.n_split; ++sp) {
+#pragma unroll
+    for (int i = 0; i < kYbarRows; ++i) y[i] += src[(int64_t)sp * 128 * 128 + i * 128];
+  }
+#pragma unroll
+  for (int i = 0; i < kYbarRows; ++i) {
+    const int64_t o = ((int64_t)u * 128 + r0 + i) * 128 + d;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(y[i]);
+    yh[o] = hi;
+    yl[o] = __float2bfloat16_rn(y[i] - __bfloat162float(hi));
+    const float w = warp_sum(y[i] * y[i]);
+    if (lane == 0) red[i][warp] = w;
   }
   __syncthreads();
-  row_y2[(int64_t)u * 128 + d] = red[0][d] + red[1][d] + red[2][d] + red[3][d];
+  if (d < kYbarRows) row_y2[(int64_t)u * 128 + r0 + d] = red[d][0] + red[d][1] + red[d][2] + red[d][3];
 }
 
 // ============================================================== pass C
@@ -666,7 +677,7 @@ cudaError_t launch_obs_tc(const Plan& pl, const void* K, const void* V, const vo
   obs_b_kernel<<<items, kThr, kSmemB, s>>>(mQ, mK, mV, a);
   stage_end(kStObsAlpha, s, 1);
   stage_begin(kStObsCombine, s);
-  obs_ybar_kernel<<<U, 128, 0, s>>>(a, reinterpret_cast<__nv_bfloat16*>(ws + pl.o_tc_yh),
+  obs_ybar_kernel<<<dim3(U, 128 / kYbarRows), 128, 0, s>>>(a, reinterpret_cast<__nv_bfloat16*>(ws + pl.o_tc_yh),
                                    reinterpret_cast<__nv_bfloat16*>(ws + pl.o_tc_yl),
                                    reinterpret_cast<float*>(ws + pl.o_tc_ry2));
   stage_end(kStObsCombine, s, 1);
