@@ -83,21 +83,37 @@ class ClockSampler:
 # ---------------------------------------------------------------- algorithmic units per stage
 
 def stage_units(spec, theta, L):
-    """Per-launch algorithmic bytes / flops of each stage (see the design notes).
-    Returns {stage: (kind, amount per launch)}; kind 'bytes' or 'flops'."""
+    """Algorithmic work of one launch of each timed stage (one layer):
+    {stage: (kind, amount, bound)}.  kind 'flops' (tensor contractions, counted
+    once even where the kernel splits an operand into bf16 hi/lo parts or
+    recomputes Q K^T) or 'bytes' (the bytes the stage must move at least)."""
     H, N, D, G, W = spec.n_kv_heads, spec.n_tokens, spec.head_dim, spec.n_q_heads // spec.n_kv_heads, spec.window
     e = 2 if spec.dtype == "bf16" else 4
     k = L["n_anchors"]
+    R = L["n_residuals"]
     GW = G * W
     kv = 2 * H * N * D * e
+    n_t = (N + 127) // 128
     return {
-        "obs_pass1": ("flops", 2 * 2 * H * GW * N * D),            # Q K^T and P V
-        "token_stats": ("flops", 2 * 2 * H * GW * N * D),          # Q K^T and V ybar^T
-        "assign": ("flops", 2 * 2 * H * N * k * D),                 # X A^T, both sides
-        "project": ("bytes", kv + 4 * 2 * H * N * 3),               # K, V + records + utilities
-        "quantize": ("bytes", L["n_residuals"] * (2 * D * e + 34)),
-        "decode_split": ("bytes", L["total_bytes"]),
+        "obs_pass1": ("flops", 2 * H * GW * N * D, "tensor"),          # S = Q K^T
+        "obs_alpha": ("flops", 2 * H * GW * N * D, "tensor"),          # ybar = alpha V
+        "obs_key_term": ("flops", 2 * H * GW * N * D, "tensor"),       # V ybar^T
+        "assign": ("flops", 2 * 2 * H * N * k * D, "tensor"),          # X A^T, both sides
+        "project": ("bytes", kv + 4 * 2 * H * N * 3, "hbm"),           # K, V; records, utilities
+        "select_topR": ("bytes", 4 * 2 * H * N + 16 * 2 * H * n_t, "hbm"),   # utilities, bitmap
+        "quantize": ("bytes", R * (2 * D * e + 34), "hbm"),            # residual rows, records
+        "decode_attn": ("bytes", L["total_bytes"], "hbm"),            # one compressed layer
     }
+
+
+def stage_roofline(stage, units, ms_per_launch, peaks):
+    kind, amount, bound = units[stage]
+    s = ms_per_launch / 1e3
+    if kind == "flops":
+        achieved, peak, unit = amount / s / 1e12, peaks["bf16_sust"] or peaks["bf16"], "TFLOP/s"
+    else:
+        achieved, peak, unit = amount / s / 1e9, peaks["hbm"], "GB/s"
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak}
 
 
 def main():
@@ -278,23 +294,16 @@ def run_gpu(args, world, rank, local):
 
     peaks = _peaks()
     units = stage_units(spec, theta, L)
-    dom = max((s for s in stages if s in units and stages[s][1]), key=lambda s: stages[s][0])
-    kind, amount = units[dom]
-    per_launch_s = stages[dom][0] / stages[dom][1] / 1e3
-    if kind == "flops":
-        achieved = amount / per_launch_s / 1e12
-        if dom == "assign" and os.environ.get("ANCHORKV_TC", "1") != "0" and _tc_assign():
-            roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16"], "unit": "TFLOP/s"}
-        else:
-            alu_peak = 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
-            roof = {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s"}
-    else:
-        achieved = amount / per_launch_s / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
+    per_launch = {st: stages[st][0] / stages[st][1] for st in stages if st in units and stages[st][1]}
+    dom = max(per_launch, key=lambda st: stages[st][0])
+    roof = stage_roofline(dom, units, per_launch[dom], peaks)
     roof["traffic"] = None
     roof["kernel"] = dom
-    roof["peak_source"] = peaks["source"]
+    roof["peak_source"] = ("measured" if peaks["source"] == "measured" else "fallback") + (
+        " (sustained bf16)" if roof["unit"] == "TFLOP/s" else " (copy)")
+    stage_roofs = {st: {kk: (round(v, 4) if isinstance(v, float) else v)
+                        for kk, v in stage_roofline(st, units, per_launch[st], peaks).items()}
+                   for st in per_launch}
 
     dec_bytes = Lr * L["total_bytes"]
     tokens_step = N * Lr * H * world
@@ -321,6 +330,7 @@ def run_gpu(args, world, rank, local):
             "compression_ratio": L["uncompressed_bytes"] / L["total_bytes"],
             "roofline": roof,
             "stage_ms_per_step": {s: v[0] / args.steps for s, v in stages.items() if v[1]},
+            "stage_roofline": stage_roofs,
             "gpu_launches": launches,
             "clocks": clk,
             "device_status": status[0],
@@ -333,11 +343,6 @@ def run_gpu(args, world, rank, local):
         dist.barrier()
         dist.destroy_process_group()
     return 0
-
-
-def _tc_assign() -> bool:
-    """True when the library's assignment stage runs on the tensor cores."""
-    return False
 
 
 def run_e2e(args, spec, theta, params, dev, stream, barrier, world):

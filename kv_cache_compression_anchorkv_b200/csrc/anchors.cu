@@ -12,9 +12,15 @@
 // other non-window positions, ties to the lower position; pooling is an
 // average with zero padding outside [0, N-W), divided by kappa.
 //
-// One CTA of 1024 threads per KV head; the per-head work is a few hundred
-// KB of L2-resident scores, so a single SM per head keeps every selection
-// exact and deterministic without grid-wide synchronisation.
+// One cluster of kC CTAs per KV head; CTA r owns a contiguous run of
+// positions and each thread a contiguous run inside it.  Both selections are
+// one cluster-wide radix select over 64-bit keys (smallest first, ties to the
+// lower position): per 8-bit digit every CTA builds a warp-aggregated
+// histogram of its keys, every CTA sums the kC histograms through
+// distributed shared memory and takes the same digit; the select stops as
+// soon as the threshold bin holds exactly the keys still needed (uniform
+// hash keys need two or three digits).  Ties at the full key are ranked by
+// position across the cluster.
 #include "common.cuh"
 #include "internal.h"
 
@@ -22,17 +28,27 @@ namespace akv {
 namespace {
 
 constexpr int kThreads = 1024;
-constexpr int kCandCap = 2048;
+constexpr int kWarps = kThreads / 32;
+constexpr int kC = 8;                 // CTAs per head (portable cluster size)
+constexpr int kSeg = 4096;            // pooling staging segment
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t b = __float_as_uint(f);
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+__device__ __forceinline__ void cl_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+template <typename U>
+__device__ __forceinline__ U* peer_ptr(U* p, unsigned rank) {
+  return static_cast<U*>(__cluster_map_shared_rank(p, rank));
+}
+
 // Exclusive block-wide prefix sum of v (one value per thread); returns the
 // thread's prefix and writes the block total to *total.
 __device__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -42,17 +58,17 @@ __device__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
   if (lane == 31) warp_tot[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int w = (lane < nw) ? warp_tot[lane] : 0;
+    int w = (lane < kWarps) ? warp_tot[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       int y = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += y;
     }
-    if (lane < nw) warp_tot[lane] = w;          // inclusive
+    if (lane < kWarps) warp_tot[lane] = w;          // inclusive
   }
   __syncthreads();
   const int before = (warp ? warp_tot[warp - 1] : 0) + x - v;
-  *total = warp_tot[nw - 1];
+  *total = warp_tot[kWarps - 1];
   __syncthreads();
   return before;
 }
@@ -65,12 +81,130 @@ struct PadList {
 };
 
 struct SelSmem {
-  unsigned int hist[256];
-  int warp_tot[32];
-  int scalar[8];
-  unsigned long long cand_key[kCandCap];
-  int cand_t[kCandCap];
+  unsigned int hist[2][256];         // double-buffered local digit histograms
+  unsigned int tot[256];             // cluster totals of the current digit
+  int warp_tot[kWarps];
+  int scal[8];
+  int cta_count;                     // this CTA's count exposed to the cluster
+  float stage[kSeg + 256];           // raw scores of one pooling segment (kappa <= 255)
 };
+
+// Result of a selection: keys below `prefix` at `bits` depth are taken; keys
+// equal to it are all taken if `all_ties`, else the first `need` of them in
+// position order.
+struct SelResult {
+  uint64_t prefix;
+  int bits;
+  int need;
+  bool all_ties;
+};
+
+// Cluster-wide radix select of the `want` smallest keys.  key(i, &k) returns
+// false for positions not taking part.  Every thread of every CTA returns the
+// same result.
+template <typename KeyF>
+__device__ SelResult cluster_select(SelSmem& sm, int lo, int hi, int ppt, int want, int key_bits, KeyF key) {
+  const unsigned C = kC;
+  SelResult res;
+  res.prefix = 0;
+  res.need = want;
+  res.all_ties = false;
+  int buf = 0;
+  int depth = 0;
+  for (; depth < key_bits; depth += 8) {
+    const int shift = 64 - depth - 8;
+    for (int i = threadIdx.x; i < 256; i += kThreads) sm.hist[buf][i] = 0u;
+    __syncthreads();
+    const uint64_t hmask = depth ? (~0ull << (64 - depth)) : 0ull;
+    for (int j = 0; j < ppt; ++j) {               // same trip count in every lane
+      const int i = lo + j;
+      uint64_t kk = 0;
+      const bool take = i < hi && key(i, kk) && ((kk & hmask) == (res.prefix & hmask));
+      const unsigned bin = take ? (unsigned)((kk >> shift) & 255u) : 256u;
+      // one atomic per distinct bin of the warp
+      const unsigned same = __match_any_sync(0xffffffffu, bin);
+      if (take && (threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&sm.hist[buf][bin], (unsigned)__popc(same));
+    }
+    __syncthreads();
+    cl_sync();
+    if (threadIdx.x < 256) {
+      unsigned t = 0;
+      for (unsigned rr = 0; rr < C; ++rr) t += peer_ptr(&sm.hist[buf][0], rr)[threadIdx.x];
+      sm.tot[threadIdx.x] = t;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      // digit: smallest d with sum_{b <= d} tot[b] >= need (8 bins per lane)
+      const int lane = threadIdx.x;
+      unsigned part = 0;
+      for (int b = 0; b < 8; ++b) part += sm.tot[lane * 8 + b];
+      unsigned incl = part;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const unsigned excl = incl - part;
+      const bool here = excl < (unsigned)res.need && incl >= (unsigned)res.need;
+      if (here) {
+        unsigned below = excl;
+        int d = lane * 8;
+        while (below + sm.tot[d] < (unsigned)res.need) { below += sm.tot[d]; ++d; }
+        sm.scal[0] = d;
+        sm.scal[1] = (int)below;
+        sm.scal[2] = (int)sm.tot[d];
+      }
+    }
+    __syncthreads();
+    const int d = sm.scal[0], below = sm.scal[1], cnt = sm.scal[2];
+    res.prefix |= (uint64_t)d << shift;
+    res.need -= below;
+    __syncthreads();
+    buf ^= 1;
+    if (cnt == res.need) { res.all_ties = true; depth += 8; break; }
+  }
+  res.bits = depth;
+  return res;
+}
+
+// Flags the selected positions of this thread's run [lo, hi): keys below the
+// threshold prefix, and keys equal to it either all or the first `need` in
+// position order across the cluster.
+template <typename KeyF>
+__device__ void mark_selected(SelSmem& sm, const SelResult& sr, int lo, int hi, uint8_t* flag, KeyF key) {
+  const uint64_t m = sr.bits >= 64 ? ~0ull : (sr.bits ? (~0ull << (64 - sr.bits)) : 0ull);
+  int ties = 0;
+  for (int i = lo; i < hi; ++i) {
+    uint64_t kk;
+    if (key(i, kk) && (kk & m) == sr.prefix) ++ties;
+  }
+  int rank0 = 0;
+  if (!sr.all_ties) {
+    int local_total;
+    const int before = block_exclusive_scan(ties, sm.warp_tot, &local_total);
+    if (threadIdx.x == 0) sm.cta_count = local_total;
+    cl_sync();
+    const unsigned r = blockIdx.x % kC;
+    int cta_before = 0;
+    for (unsigned rr = 0; rr < r; ++rr) cta_before += *peer_ptr(&sm.cta_count, rr);
+    rank0 = cta_before + before;
+  }
+  // keys are read before any flag of this thread changes (the value-sample
+  // key excludes flagged positions)
+  for (int i = lo; i < hi; ++i) {
+    uint64_t kk;
+    if (!key(i, kk)) continue;
+    const uint64_t top = kk & m;
+    if (top < sr.prefix) {
+      flag[i] = 1;
+    } else if (top == sr.prefix) {
+      if (sr.all_ties || rank0 < sr.need) flag[i] = 1;
+      ++rank0;
+    }
+  }
+  __syncthreads();
+  cl_sync();   // peers are done reading sm.cta_count / histograms of this select
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -81,170 +215,116 @@ anchor_select_kernel(const float* __restrict__ score, float* __restrict__ pooled
                      double* __restrict__ anc_n2, double* __restrict__ anc_sqrt, float* __restrict__ anc_inv,
                      int* __restrict__ counters,
                      int H, int kp16, int obs_rb, PadList pads) {
-  __shared__ SelSmem sm;
-  const int h = blockIdx.x;
+  extern __shared__ __align__(16) unsigned char dsm[];
+  SelSmem& sm = *reinterpret_cast<SelSmem*>(dsm);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(dsm + sizeof(SelSmem));   // pooled order keys of the run
+  const unsigned r = blockIdx.x % kC;
+  const int h = blockIdx.x / kC;
   const int tid = threadIdx.x;
   // alignment gaps between layout sections are part of the output: zero them
-  if (h == 0 && tid < PadList::kMax * 16) {
+  if (h == 0 && r == 0 && tid < PadList::kMax * 16) {
     const int i = tid / 16, b = tid % 16;
     if (b < pads.len[i]) pads.base[pads.off[i] + b] = 0;
   }
   const int NW = N - W;
+  const int per_cta = (N + kC - 1) / kC;
+  const int c0 = min(N, (int)r * per_cta), c1 = min(N, c0 + per_cta), np = c1 - c0;
+  const int ppt = (np + kThreads - 1) / kThreads;
+  const int lo = min(np, tid * ppt), hi = min(np, lo + ppt);         // this thread's run (local)
   float* pl = pooled + (int64_t)h * N;
-  int* flag = slot_of + (int64_t)h * N;       // flags first, slots after compaction
+  uint8_t* flag = reinterpret_cast<uint8_t*>(keys + np);               // [np] anchor flags
 
-  // 1. pooling (zero padding outside [0, N-W), divide by kappa); the score of
-  //    a position is the sum of its observation-row-block partials, in order
+  // 1. pooling of [c0, min(c1, NW)) in segments (zero padding outside
+  //    [0, N-W), divide by kappa); a position's score is the sum of its
+  //    observation-row-block partials, in order
   const int half = kappa / 2;
-  for (int t = tid; t < N; t += kThreads) {
-    if (t < NW) {
+  const int pend = min(c1, NW);
+  for (int sb = c0; sb < pend; sb += kSeg) {
+    const int se = min(pend, sb + kSeg);
+    for (int u = sb - half + tid; u < se + half; u += kThreads) {
+      float v = 0.f;
+      if (u >= 0 && u < NW) {
+        v = score[(int64_t)h * N + u];
+        for (int rb = 1; rb < obs_rb; ++rb) v += score[((int64_t)rb * H + h) * N + u];
+      }
+      sm.stage[u - (sb - half)] = v;
+    }
+    __syncthreads();
+    for (int t = sb + tid; t < se; t += kThreads) {
       float acc = 0.f;
       for (int d = -half; d <= half; ++d) {
         const int u = t + d;
-        if (u >= 0 && u < NW) {
-          float s = score[(int64_t)h * N + u];
-          for (int rb = 1; rb < obs_rb; ++rb) s += score[((int64_t)rb * H + h) * N + u];
-          acc += s;
-        }
+        if (u >= 0 && u < NW) acc += sm.stage[u - (sb - half)];
       }
-      pl[t] = acc / (float)kappa;
+      const float pv = acc / (float)kappa;
+      pl[t] = pv;
+      keys[t - c0] = ~order_key(pv);                 // smallest key = largest score
     }
-    flag[t] = (all_anchors || t >= NW) ? 1 : 0;
+    __syncthreads();
   }
+  for (int i = tid; i < np; i += kThreads) flag[i] = (all_anchors || c0 + i >= NW) ? 1 : 0;
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
   __syncthreads();
 
+  // 2. the n_s largest pooled scores, ties to the lower position
   if (!all_anchors && n_s > 0) {
-    // 2. radix select of the n_s largest pooled scores (32-bit order keys)
-    uint32_t prefix = 0;
-    int need = n_s;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += kThreads) sm.hist[i] = 0;
-      __syncthreads();
-      const uint32_t mask = (shift == 24) ? 0u : (0xFFFFFFFFu << (shift + 8));
-      for (int t = tid; t < NW; t += kThreads) {
-        const uint32_t key = order_key(pl[t]);
-        if ((key & mask) == (prefix & mask)) atomicAdd(&sm.hist[(key >> shift) & 255u], 1u);
-      }
-      __syncthreads();
-      if (tid == 0) {
-        int cum = 0, digit = 0;
-        for (int d = 255; d >= 0; --d) {
-          if (cum + (int)sm.hist[d] >= need) { digit = d; break; }
-          cum += sm.hist[d];
-        }
-        sm.scalar[0] = digit;
-        sm.scalar[1] = need - cum;
-      }
-      __syncthreads();
-      prefix |= (uint32_t)sm.scalar[0] << shift;
-      need = sm.scalar[1];
-      __syncthreads();
-    }
-    // mark keys above the threshold and the first `need` ties in position order
-    int taken = 0;
-    for (int base = 0; base < NW; base += kThreads) {
-      const int t = base + tid;
-      uint32_t key = (t < NW) ? order_key(pl[t]) : 0u;
-      const int tie = (t < NW && key == prefix) ? 1 : 0;
-      int tot;
-      const int rank = taken + block_exclusive_scan(tie, sm.warp_tot, &tot);
-      if (t < NW && (key > prefix || (tie && rank < need))) flag[t] = 1;
-      taken += tot;
-    }
-    __syncthreads();
+    auto key = [&](int i, uint64_t& kk) -> bool {
+      if (c0 + i >= NW) return false;
+      kk = (uint64_t)keys[i] << 32;
+      return true;
+    };
+    const SelResult sr = cluster_select(sm, lo, hi, ppt, n_s, 32, key);
+    mark_selected(sm, sr, lo, hi, flag, key);
   }
-
+  // 3. the n_u smallest hash keys among the other non-window positions
   if (!all_anchors && n_u > 0) {
-    // 3. uniform sample: the n_u smallest hash keys among unflagged non-window
-    //    positions.  A key threshold is chosen so that between n_u and
-    //    kCandCap candidates fall below it (bisection on the threshold); the
-    //    candidates are then sorted exactly by (key, position).
-    const int n_rest = NW - n_s;
-    double lo = 0.0, hi = 1.0;
-    double frac = fmin(1.0, (n_u + 4.0 * sqrt((double)n_u) + 32.0) / (double)n_rest);
-    unsigned long long thr = 0;
-    int count = -1, iter = 0;
-    for (; iter < 80; ++iter) {
-      thr = (frac >= 1.0) ? ~0ull : (unsigned long long)(frac * 18446744073709551616.0);
-      if (tid == 0) sm.scalar[2] = 0;
-      __syncthreads();
-      int local = 0;
-      for (int t = tid; t < NW; t += kThreads)
-        if (!flag[t] && (frac >= 1.0 || anchor_key(seed, layer, h, t) < thr)) ++local;
-      local = __reduce_add_sync(0xffffffffu, local);
-      if ((tid & 31) == 0) atomicAdd(&sm.scalar[2], local);
-      __syncthreads();
-      count = sm.scalar[2];
-      __syncthreads();
-      if (count >= n_u && count <= kCandCap) break;
-      if (count < n_u) lo = frac; else hi = frac;
-      frac = 0.5 * (lo + hi);
-    }
-    if (count < n_u || count > kCandCap) {
-      if (tid == 0) latch_error(counters, kDevErrUniform);
-      return;
-    }
-    if (tid == 0 && iter > 0) atomicAdd(&counters[kUniformRetries], iter);
-    if (tid == 0) sm.scalar[3] = 0;
-    __syncthreads();
-    for (int t = tid; t < NW; t += kThreads) {
-      if (flag[t]) continue;
-      const unsigned long long key = anchor_key(seed, layer, h, t);
-      if (frac >= 1.0 || key < thr) {
-        const int slot = atomicAdd(&sm.scalar[3], 1);
-        sm.cand_key[slot] = key;
-        sm.cand_t[slot] = t;
-      }
-    }
-    __syncthreads();
-    int P = 1;
-    while (P < count) P <<= 1;
-    for (int i = count + tid; i < P; i += kThreads) { sm.cand_key[i] = ~0ull; sm.cand_t[i] = 0x7fffffff; }
-    __syncthreads();
-    // bitonic sort by (key, t)
-    for (int size = 2; size <= P; size <<= 1) {
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int i = tid; i < P; i += kThreads) {
-          const int j = i ^ stride;
-          if (j > i) {
-            const bool up = ((i & size) == 0);
-            const unsigned long long ki = sm.cand_key[i], kj = sm.cand_key[j];
-            const int ti = sm.cand_t[i], tj = sm.cand_t[j];
-            const bool gt = (ki > kj) || (ki == kj && ti > tj);
-            if (gt == up) {
-              sm.cand_key[i] = kj; sm.cand_key[j] = ki;
-              sm.cand_t[i] = tj; sm.cand_t[j] = ti;
-            }
-          }
-        }
-        __syncthreads();
-      }
-    }
-    for (int i = tid; i < n_u; i += kThreads) flag[sm.cand_t[i]] = 1;
-    __syncthreads();
+    auto key = [&](int i, uint64_t& kk) -> bool {
+      if (c0 + i >= NW || flag[i]) return false;
+      kk = anchor_key(seed, layer, h, c0 + i);
+      return true;
+    };
+    const SelResult sr = cluster_select(sm, lo, hi, ppt, n_u, 64, key);
+    mark_selected(sm, sr, lo, hi, flag, key);
   }
 
   // 4. compaction in position order: slot s <-> anchor_pos[s]
-  int taken = 0;
-  int* apos = anchor_pos + (int64_t)h * k;
-  for (int base = 0; base < N; base += kThreads) {
-    const int t = base + tid;
-    const int f = (t < N) ? flag[t] : 0;
-    int tot;
-    const int s = taken + block_exclusive_scan(f, sm.warp_tot, &tot);
-    if (t < N) {
-      if (f && s < k) apos[s] = t;
-      flag[t] = f ? s : -1;
-    }
-    taken += tot;
+  int cnt = 0;
+  for (int i = lo; i < hi; ++i) cnt += flag[i];
+  int local_total;
+  const int before = block_exclusive_scan(cnt, sm.warp_tot, &local_total);
+  if (tid == 0) sm.cta_count = local_total;
+  cl_sync();
+  int cta_before = 0, all = 0;
+  for (unsigned rr = 0; rr < (unsigned)kC; ++rr) {
+    const int c = *peer_ptr(&sm.cta_count, rr);
+    if (rr < r) cta_before += c;
+    all += c;
   }
-  if (tid == 0 && taken != k) latch_error(counters, kDevErrBounds);
+  int* apos = anchor_pos + (int64_t)h * k;
+  int* sof = slot_of + (int64_t)h * N;
+  {
+    int s = cta_before + before;
+    for (int i = lo; i < hi; ++i) {
+      if (flag[i]) {
+        if (s < k) apos[s] = c0 + i;
+        sof[c0 + i] = s;
+        ++s;
+      } else {
+        sof[c0 + i] = -1;
+      }
+    }
+  }
+  if (all != k) {
+    if (r == 0 && tid == 0) latch_error(counters, kDevErrBounds);
+    cl_sync();
+    return;
+  }
   __syncthreads();
-  if (taken != k) return;
 
-  // 5. copy anchor rows into the layout; exact fp64 squared norms
+  // 5. this CTA's anchor rows into the layout; exact fp64 squared norms
   const int warp = tid >> 5, lane = tid & 31;
-  for (int s = warp; s < k; s += kThreads / 32) {
+  const int s_lo = cta_before, s_hi = cta_before + local_total;
+  for (int s = s_lo + warp; s < s_hi; s += kWarps) {
     const int t = apos[s];
     for (int side = 0; side < 2; ++side) {
       const T* src = (side ? V : K) + ((int64_t)h * N + t) * kD;
@@ -264,10 +344,13 @@ anchor_select_kernel(const float* __restrict__ score, float* __restrict__ pooled
     }
   }
   // 1/||a|| rows are padded to a multiple of 16 slots with zeros
-  for (int i = tid; i < 2 * (kp16 - k); i += kThreads) {
-    const int side = i / (kp16 - k), s = k + i % (kp16 - k);
-    anc_inv[((int64_t)side * H + h) * kp16 + s] = 0.f;
+  if (r == 0) {
+    for (int i = tid; i < 2 * (kp16 - k); i += kThreads) {
+      const int side = i / (kp16 - k), s = k + i % (kp16 - k);
+      anc_inv[((int64_t)side * H + h) * kp16 + s] = 0.f;
+    }
   }
+  cl_sync();   // no CTA leaves while a peer may still read its shared memory
 }
 
 }  // namespace
@@ -293,19 +376,43 @@ cudaError_t launch_anchor_select(const Plan& pl, const void* K, const void* V, c
     pads.off[i] = ends[i];
     pads.len[i] = (int)((16 - ends[i] % 16) % 16);
   }
+  const int per_cta = (int)((N + kC - 1) / kC);
+  const size_t smem = sizeof(SelSmem) + (size_t)per_cta * 5;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(pl.H * kC);
+  lc.blockDim = dim3(kThreads);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kC;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  cudaError_t e;
   if (pl.p.dtype == ANCHORKV_BF16) {
-    anchor_select_kernel<__nv_bfloat16><<<pl.H, kThreads, 0, s>>>(
-        score, pooled, pl.N, pl.W, pl.p.pool_kernel, pl.n_s, pl.n_u, pl.k, pl.all_anchors ? 1 : 0,
-        pl.p.seed, pl.p.layer, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
-        reinterpret_cast<__nv_bfloat16*>(out + pl.L.off_anchors_k),
-        reinterpret_cast<__nv_bfloat16*>(out + pl.L.off_anchors_v), apos, slot_of, n2, sq, inv, cnt, pl.H, pl.kp16, pl.obs_rb, pads);
+    using T = __nv_bfloat16;
+    auto kern = anchor_select_kernel<T>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaLaunchKernelEx(&lc, kern, score, pooled, pl.N, pl.W, pl.p.pool_kernel, pl.n_s, pl.n_u, pl.k,
+                           pl.all_anchors ? 1 : 0, (unsigned long long)pl.p.seed, pl.p.layer, (const T*)K,
+                           (const T*)V, reinterpret_cast<T*>(out + pl.L.off_anchors_k),
+                           reinterpret_cast<T*>(out + pl.L.off_anchors_v), apos, slot_of, n2, sq, inv, cnt, pl.H,
+                           pl.kp16, pl.obs_rb, pads);
   } else {
-    anchor_select_kernel<float><<<pl.H, kThreads, 0, s>>>(
-        score, pooled, pl.N, pl.W, pl.p.pool_kernel, pl.n_s, pl.n_u, pl.k, pl.all_anchors ? 1 : 0,
-        pl.p.seed, pl.p.layer, (const float*)K, (const float*)V,
-        reinterpret_cast<float*>(out + pl.L.off_anchors_k), reinterpret_cast<float*>(out + pl.L.off_anchors_v),
-        apos, slot_of, n2, sq, inv, cnt, pl.H, pl.kp16, pl.obs_rb, pads);
+    using T = float;
+    auto kern = anchor_select_kernel<T>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaLaunchKernelEx(&lc, kern, score, pooled, pl.N, pl.W, pl.p.pool_kernel, pl.n_s, pl.n_u, pl.k,
+                           pl.all_anchors ? 1 : 0, (unsigned long long)pl.p.seed, pl.p.layer, (const T*)K,
+                           (const T*)V, reinterpret_cast<T*>(out + pl.L.off_anchors_k),
+                           reinterpret_cast<T*>(out + pl.L.off_anchors_v), apos, slot_of, n2, sq, inv, cnt, pl.H,
+                           pl.kp16, pl.obs_rb, pads);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
