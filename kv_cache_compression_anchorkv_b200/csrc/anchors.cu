@@ -21,6 +21,7 @@
 // soon as the threshold bin holds exactly the keys still needed (uniform
 // hash keys need two or three digits).  Ties at the full key are ranked by
 // position across the cluster.
+#include "cluster_select.cuh"
 #include "common.cuh"
 #include "internal.h"
 
@@ -37,13 +38,9 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-__device__ __forceinline__ void cl_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
+__device__ __forceinline__ void cl_sync() { cluster_barrier(); }
 template <typename U>
-__device__ __forceinline__ U* peer_ptr(U* p, unsigned rank) {
-  return static_cast<U*>(__cluster_map_shared_rank(p, rank));
-}
+__device__ __forceinline__ U* peer_ptr(U* p, unsigned rank) { return cluster_peer(p, rank); }
 
 // Exclusive block-wide prefix sum of v (one value per thread); returns the
 // thread's prefix and writes the block total to *total.
@@ -81,102 +78,21 @@ struct PadList {
 };
 
 struct SelSmem {
-  unsigned int hist[2][256];         // double-buffered local digit histograms
-  unsigned int tot[256];             // cluster totals of the current digit
+  RadixSmem rs;
   int warp_tot[kWarps];
-  int scal[8];
   int cta_count;                     // this CTA's count exposed to the cluster
   float stage[kSeg + 256];           // raw scores of one pooling segment (kappa <= 255)
 };
-
-// Result of a selection: keys below `prefix` at `bits` depth are taken; keys
-// equal to it are all taken if `all_ties`, else the first `need` of them in
-// position order.
-struct SelResult {
-  uint64_t prefix;
-  int bits;
-  int need;
-  bool all_ties;
-};
-
-// Cluster-wide radix select of the `want` smallest keys.  key(i, &k) returns
-// false for positions not taking part.  Every thread of every CTA returns the
-// same result.
-template <typename KeyF>
-__device__ SelResult cluster_select(SelSmem& sm, int lo, int hi, int ppt, int want, int key_bits, KeyF key) {
-  const unsigned C = kC;
-  SelResult res;
-  res.prefix = 0;
-  res.need = want;
-  res.all_ties = false;
-  int buf = 0;
-  int depth = 0;
-  for (; depth < key_bits; depth += 8) {
-    const int shift = 64 - depth - 8;
-    for (int i = threadIdx.x; i < 256; i += kThreads) sm.hist[buf][i] = 0u;
-    __syncthreads();
-    const uint64_t hmask = depth ? (~0ull << (64 - depth)) : 0ull;
-    for (int j = 0; j < ppt; ++j) {               // same trip count in every lane
-      const int i = lo + j;
-      uint64_t kk = 0;
-      const bool take = i < hi && key(i, kk) && ((kk & hmask) == (res.prefix & hmask));
-      const unsigned bin = take ? (unsigned)((kk >> shift) & 255u) : 256u;
-      // one atomic per distinct bin of the warp
-      const unsigned same = __match_any_sync(0xffffffffu, bin);
-      if (take && (threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&sm.hist[buf][bin], (unsigned)__popc(same));
-    }
-    __syncthreads();
-    cl_sync();
-    if (threadIdx.x < 256) {
-      unsigned t = 0;
-      for (unsigned rr = 0; rr < C; ++rr) t += peer_ptr(&sm.hist[buf][0], rr)[threadIdx.x];
-      sm.tot[threadIdx.x] = t;
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      // digit: smallest d with sum_{b <= d} tot[b] >= need (8 bins per lane)
-      const int lane = threadIdx.x;
-      unsigned part = 0;
-      for (int b = 0; b < 8; ++b) part += sm.tot[lane * 8 + b];
-      unsigned incl = part;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const unsigned excl = incl - part;
-      const bool here = excl < (unsigned)res.need && incl >= (unsigned)res.need;
-      if (here) {
-        unsigned below = excl;
-        int d = lane * 8;
-        while (below + sm.tot[d] < (unsigned)res.need) { below += sm.tot[d]; ++d; }
-        sm.scal[0] = d;
-        sm.scal[1] = (int)below;
-        sm.scal[2] = (int)sm.tot[d];
-      }
-    }
-    __syncthreads();
-    const int d = sm.scal[0], below = sm.scal[1], cnt = sm.scal[2];
-    res.prefix |= (uint64_t)d << shift;
-    res.need -= below;
-    __syncthreads();
-    buf ^= 1;
-    if (cnt == res.need) { res.all_ties = true; depth += 8; break; }
-  }
-  res.bits = depth;
-  return res;
-}
 
 // Flags the selected positions of this thread's run [lo, hi): keys below the
 // threshold prefix, and keys equal to it either all or the first `need` in
 // position order across the cluster.
 template <typename KeyF>
-__device__ void mark_selected(SelSmem& sm, const SelResult& sr, int lo, int hi, uint8_t* flag, KeyF key) {
-  const uint64_t m = sr.bits >= 64 ? ~0ull : (sr.bits ? (~0ull << (64 - sr.bits)) : 0ull);
+__device__ void mark_selected(SelSmem& sm, const RadixResult& sr, int lo, int hi, uint8_t* flag, KeyF key) {
   int ties = 0;
   for (int i = lo; i < hi; ++i) {
     uint64_t kk;
-    if (key(i, kk) && (kk & m) == sr.prefix) ++ties;
+    if (key(i - lo, kk) && radix_top(kk, sr.bits) == sr.prefix) ++ties;
   }
   int rank0 = 0;
   if (!sr.all_ties) {
@@ -193,8 +109,8 @@ __device__ void mark_selected(SelSmem& sm, const SelResult& sr, int lo, int hi, 
   // key excludes flagged positions)
   for (int i = lo; i < hi; ++i) {
     uint64_t kk;
-    if (!key(i, kk)) continue;
-    const uint64_t top = kk & m;
+    if (!key(i - lo, kk)) continue;
+    const uint64_t top = radix_top(kk, sr.bits);
     if (top < sr.prefix) {
       flag[i] = 1;
     } else if (top == sr.prefix) {
@@ -268,22 +184,24 @@ anchor_select_kernel(const float* __restrict__ score, float* __restrict__ pooled
 
   // 2. the n_s largest pooled scores, ties to the lower position
   if (!all_anchors && n_s > 0) {
-    auto key = [&](int i, uint64_t& kk) -> bool {
-      if (c0 + i >= NW) return false;
+    auto key = [&](int j, uint64_t& kk) -> bool {
+      const int i = lo + j;
+      if (i >= hi || c0 + i >= NW) return false;
       kk = (uint64_t)keys[i] << 32;
       return true;
     };
-    const SelResult sr = cluster_select(sm, lo, hi, ppt, n_s, 32, key);
+    const RadixResult sr = cluster_radix_select<kThreads, kC>(sm.rs, ppt, n_s, 32, key);
     mark_selected(sm, sr, lo, hi, flag, key);
   }
   // 3. the n_u smallest hash keys among the other non-window positions
   if (!all_anchors && n_u > 0) {
-    auto key = [&](int i, uint64_t& kk) -> bool {
-      if (c0 + i >= NW || flag[i]) return false;
+    auto key = [&](int j, uint64_t& kk) -> bool {
+      const int i = lo + j;
+      if (i >= hi || c0 + i >= NW || flag[i]) return false;
       kk = anchor_key(seed, layer, h, c0 + i);
       return true;
     };
-    const SelResult sr = cluster_select(sm, lo, hi, ppt, n_u, 64, key);
+    const RadixResult sr = cluster_radix_select<kThreads, kC>(sm.rs, ppt, n_u, 64, key);
     mark_selected(sm, sr, lo, hi, flag, key);
   }
 

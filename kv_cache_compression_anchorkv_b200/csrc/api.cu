@@ -134,7 +134,8 @@ int make_plan(const anchorkv_params* p, Plan* pl) {
   pl->obs_rb = 1;
   const int64_t H = pl->H, N = pl->N, GW = pl->GW, k = pl->k, D = kD;
   const int64_t n_sh_t = 2 * H * pl->n_tiles;
-  const int64_t U = H * pl->tc_rb, nrb = pl->tc_rb;
+  // the tensor-core passes leave two row-block partials per 128-row block
+  const int64_t U = H * pl->tc_rb, nrb = 2 * pl->tc_rb;
   int64_t off = 0;
   auto take = [&](int64_t bytes) { int64_t o = off; off += (bytes + 255) / 256 * 256; return o; };
   pl->o_counters = take(4 * (kCounterCount + 2 * H));
@@ -144,8 +145,8 @@ int make_plan(const anchorkv_params* p, Plan* pl) {
   pl->o_part_m = take(4 * H * pl->n_chunk1 * GW);
   pl->o_part_l = take(4 * H * pl->n_chunk1 * GW);
   pl->o_part_y = take(4 * H * pl->n_chunk1 * GW * D);
-  pl->o_tc_pm2 = take(4 * U * pl->tc_split * 128);
-  pl->o_tc_pl = take(4 * U * pl->tc_split * 128);
+  pl->o_tc_pm2 = take(4 * U * 2 * pl->tc_split * 128);
+  pl->o_tc_pl = take(4 * U * 2 * pl->tc_split * 128);
   pl->o_tc_rm2 = take(4 * U * 128);
   pl->o_tc_riz = take(4 * U * 128);
   pl->o_tc_rq2 = take(4 * U * 128);
@@ -276,7 +277,7 @@ int anchorkv_compress(const anchorkv_params* p, const void* K, const void* V, co
 #define AKV_STAGE(st, nk, expr) \
   do { stage_begin(st, s); AKV_LAUNCH(expr); stage_end(st, s, nk); } while (0)
   if (use_tc_obs(pl)) {
-    pl.obs_rb = pl.tc_rb;
+    pl.obs_rb = 2 * pl.tc_rb;
     AKV_LAUNCH(launch_obs_tc(pl, K, V, Q_obs, w, s));
   } else {
     pl.obs_rb = 1;
@@ -292,7 +293,7 @@ int anchorkv_compress(const anchorkv_params* p, const void* K, const void* V, co
   }
   AKV_STAGE(kStRefine, 1, launch_refine(pl, K, V, o, w, s));
   AKV_STAGE(kStProject, 1, launch_project(pl, K, V, o, w, s));
-  const int sel_kernels = pl.R == 0 ? 0 : (pl.R == pl.cap ? 5 : 13);
+  const int sel_kernels = pl.R == 0 ? 0 : 1;
   AKV_STAGE(kStSelect, sel_kernels, launch_select(pl, o, w, s));
   AKV_STAGE(kStQuantize, pl.R ? 1 : 0, launch_quantize(pl, K, V, o, w, s));
 #undef AKV_STAGE

@@ -114,161 +114,6 @@ project_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __rest
   util[f] = u;
 }
 
-// ---------------------------------------------------------------- top-R select
-// Radix select over the utility bits (eligible utilities are >= 0, so their
-// IEEE bit patterns order like the values).  state[0] = threshold prefix,
-// state[1] = how many keys equal to the final threshold are still to take.
-
-__global__ void rs_hist_kernel(const float* __restrict__ util, int64_t n, const uint32_t* __restrict__ state,
-                               int shift, unsigned int* __restrict__ hist) {
-  __shared__ unsigned int sh[256];
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) sh[i] = 0;
-  __syncthreads();
-  const uint32_t prefix = state[0];
-  const uint32_t mask = (shift == 24) ? 0u : (0xFFFFFFFFu << (shift + 8));
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    const float u = util[i];
-    if (!(u >= 0.f)) continue;
-    const uint32_t key = __float_as_uint(u);
-    if ((key & mask) == (prefix & mask)) atomicAdd(&sh[(key >> shift) & 255u], 1u);
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < 256; i += blockDim.x)
-    if (sh[i]) atomicAdd(&hist[i], sh[i]);
-}
-
-__global__ void rs_pick_kernel(unsigned int* __restrict__ hist, uint32_t* __restrict__ state, int shift) {
-  if (threadIdx.x == 0) {
-    const int need = (int)state[1];
-    int cum = 0, digit = 0;
-    for (int d = 255; d >= 0; --d) {
-      if (cum + (int)hist[d] >= need) { digit = d; break; }
-      cum += (int)hist[d];
-    }
-    state[0] |= (uint32_t)digit << shift;
-    state[1] = (uint32_t)(need - cum);
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-}
-
-__global__ void rs_init_kernel(uint32_t* __restrict__ state, unsigned int* __restrict__ hist, int R, int take_all) {
-  if (threadIdx.x == 0) {
-    state[0] = 0;
-    state[1] = take_all ? 0x7fffffffu : (uint32_t)R;
-  }
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-}
-
-// One warp per 128-token tile of one (side, head): counts above/at threshold.
-__global__ void sel_tiles_kernel(const float* __restrict__ util, const uint32_t* __restrict__ state, int N,
-                                 int n_tiles, int n_sh, int* __restrict__ tile_gt, int* __restrict__ tile_eq) {
-  const int lane = threadIdx.x & 31;
-  const int tile = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (tile >= n_sh * n_tiles) return;
-  const int sh = tile / n_tiles, j = tile % n_tiles;
-  const uint32_t T = state[0];
-  int gt = 0, eq = 0;
-  for (int w = 0; w < 4; ++w) {
-    const int t = j * kTile + w * 32 + lane;
-    bool g = false, e = false;
-    if (t < N) {
-      const float u = util[(int64_t)sh * N + t];
-      if (u >= 0.f) {
-        const uint32_t key = __float_as_uint(u);
-        g = key > T;
-        e = key == T;
-      }
-    }
-    gt += __popc(__ballot_sync(0xffffffffu, g));
-    eq += __popc(__ballot_sync(0xffffffffu, e));
-  }
-  if (lane == 0) { tile_gt[tile] = gt; tile_eq[tile] = eq; }
-}
-
-// Single-block exclusive scan of n ints; out has n + 1 entries (out[n] = total).
-// With prefix_layout != 0 the result is written as [n_sh][n_tiles + 1] where
-// entry (sh, n_tiles) is the start of the next (side, head).
-__global__ void scan_kernel(const int* __restrict__ in, int n, int* __restrict__ out, int n_tiles,
-                            int prefix_layout) {
-  __shared__ int warp_tot[32];
-  __shared__ int carry;
-  if (threadIdx.x == 0) carry = 0;
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int base = 0; base <= n; base += blockDim.x) {
-    const int i = base + threadIdx.x;
-    const int v = (i < n) ? in[i] : 0;
-    int x = v;
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) warp_tot[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-      int w = (lane < nw) ? warp_tot[lane] : 0;
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, w, o);
-        if (lane >= o) w += y;
-      }
-      if (lane < nw) warp_tot[lane] = w;
-    }
-    __syncthreads();
-    const int excl = carry + (warp ? warp_tot[warp - 1] : 0) + x - v;
-    if (i <= n) {
-      if (!prefix_layout) {
-        out[i] = excl;
-      } else {
-        const int sh = i / n_tiles, j = i % n_tiles;
-        if (i < n) out[sh * (n_tiles + 1) + j] = excl;
-        if (j == 0 && sh > 0) out[(sh - 1) * (n_tiles + 1) + n_tiles] = excl;
-      }
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) carry += warp_tot[nw - 1];
-    __syncthreads();
-  }
-}
-
-__global__ void sel_bitmap_kernel(const float* __restrict__ util, const uint32_t* __restrict__ state, int N,
-                                  int n_tiles, int n_sh, const int* __restrict__ tie_before,
-                                  uint32_t* __restrict__ bitmap, int* __restrict__ tile_cnt,
-                                  int* __restrict__ counters) {
-  const int lane = threadIdx.x & 31;
-  const int tile = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (tile >= n_sh * n_tiles) return;
-  const int sh = tile / n_tiles, j = tile % n_tiles;
-  const uint32_t T = state[0];
-  const int need = (int)state[1];
-  int rank = tie_before[tile];
-  int cnt = 0, ties = 0;
-  for (int w = 0; w < 4; ++w) {
-    const int t = j * kTile + w * 32 + lane;
-    bool g = false, e = false;
-    if (t < N) {
-      const float u = util[(int64_t)sh * N + t];
-      if (u >= 0.f) {
-        const uint32_t key = __float_as_uint(u);
-        g = key > T;
-        e = key == T;
-      }
-    }
-    const uint32_t eqb = __ballot_sync(0xffffffffu, e);
-    const int my_rank = rank + __popc(eqb & ((1u << lane) - 1u));
-    const bool s = g || (e && my_rank < need);
-    const uint32_t sb = __ballot_sync(0xffffffffu, s);
-    if (lane == 0) bitmap[(int64_t)tile * 4 + w] = sb;
-    rank += __popc(eqb);
-    ties += __popc(eqb);
-    cnt += __popc(sb);
-  }
-  if (lane == 0) {
-    tile_cnt[tile] = cnt;
-    if (ties && need != 0x7fffffff) atomicAdd(&counters[kSelectTies], ties);
-  }
-}
-
 // ---------------------------------------------------------------- quantize
 
 struct CodecConst {
@@ -422,41 +267,6 @@ cudaError_t launch_project(const Plan& pl, const void* K, const void* V, char* o
         reinterpret_cast<const float*>(out + pl.L.off_anchors_v), n2, slot_of, a2, ku, tok, util,
         pl.N, pl.H, pl.k, pl.obs_rb);
   }
-  return cudaGetLastError();
-}
-
-cudaError_t launch_select(const Plan& pl, char* out, char* ws, cudaStream_t s) {
-  const int n_sh = 2 * pl.H, n_t = pl.n_tiles, n_tiles_all = n_sh * n_t;
-  auto* util = reinterpret_cast<const float*>(ws + pl.o_util);
-  auto* state = reinterpret_cast<uint32_t*>(ws + pl.o_sel_state);
-  auto* hist = reinterpret_cast<unsigned int*>(ws + pl.o_hist);
-  auto* gt = reinterpret_cast<int*>(ws + pl.o_tile_gt);
-  auto* eq = reinterpret_cast<int*>(ws + pl.o_tile_eq);
-  auto* tb = reinterpret_cast<int*>(ws + pl.o_tie_before);
-  auto* tc = reinterpret_cast<int*>(ws + pl.o_tile_cnt);
-  auto* cnt = reinterpret_cast<int*>(ws + pl.o_counters);
-  auto* bitmap = reinterpret_cast<uint32_t*>(out + pl.L.off_bitmap);
-  auto* prefix = reinterpret_cast<int*>(out + pl.L.off_tile_prefix);
-  if (pl.R == 0) {
-    cudaMemsetAsync(bitmap, 0, (size_t)n_tiles_all * 16, s);
-    cudaMemsetAsync(prefix, 0, (size_t)n_sh * (n_t + 1) * 4, s);
-    return cudaGetLastError();
-  }
-  const bool take_all = pl.R == pl.cap;
-  rs_init_kernel<<<1, 256, 0, s>>>(state, hist, (int)pl.R, take_all ? 1 : 0);
-  if (!take_all) {
-    const int64_t n = 2LL * pl.H * pl.N;
-    const int blocks = (int)std::min<int64_t>(148 * 4, (n + 255) / 256);
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      rs_hist_kernel<<<blocks, 256, 0, s>>>(util, n, state, shift, hist);
-      rs_pick_kernel<<<1, 256, 0, s>>>(hist, state, shift);
-    }
-  }
-  const int wb = (n_tiles_all + 7) / 8;
-  sel_tiles_kernel<<<wb, 256, 0, s>>>(util, state, pl.N, n_t, n_sh, gt, eq);
-  scan_kernel<<<1, 1024, 0, s>>>(eq, n_tiles_all, tb, n_t, 0);
-  sel_bitmap_kernel<<<wb, 256, 0, s>>>(util, state, pl.N, n_t, n_sh, tb, bitmap, tc, cnt);
-  scan_kernel<<<1, 1024, 0, s>>>(tc, n_tiles_all, prefix, n_t, 1);
   return cudaGetLastError();
 }
 

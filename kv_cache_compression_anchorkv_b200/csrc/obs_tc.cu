@@ -20,8 +20,12 @@
 // needed.  All operands are bf16 (K, V, Q exact; alpha and ybar split into
 // two bf16 terms, error 2^-17 relative), accumulators fp32 in TMEM, exp via
 // ex2.approx in the log2 domain.  Warp roles as in the assignment kernel:
-// warp 0 TMA, warp 1 TMEM owner + MMA issuer, warps 2..5 epilogue (one TMEM
-// lane = one row or token per thread).  Every wait is bounded.
+// warp 0 TMA, warp 1 TMEM owner + MMA issuer, warps 2..9 epilogue in two
+// column groups (warps 2..5 and 6..9; one TMEM lane = one row or token per
+// thread, each group half of the accumulator's columns).  Pass A's groups
+// split the tokens of a tile and leave separate (max, sum) partials; passes B
+// and C's groups split the observation rows, so their per-token sums are
+// written as two row blocks per 128-row block.  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -34,11 +38,12 @@ namespace {
 
 constexpr int kOp = 128 * 256;                 // one [128][128] bf16 operand tile
 constexpr int kHalf = kOp / 2;                 // its 64-column swizzled half
-constexpr int kThr = 192;
+constexpr int kThr = 320;
+constexpr int kEpi = 256;                      // epilogue threads (8 warps, 2 column groups)
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct ObsTc {
-  int N, H, G, W, GW, n_rb, n_split, tps, row_tiles;
+  int N, H, G, W, GW, n_rb, n_split, tps, row_tiles;   // part_m2/part_l hold 2 * n_split partials per unit
   float c2;                                     // log2(e) / sqrt(D)
   float* part_m2;                               // [U][n_split][128]
   float* part_l;
@@ -46,7 +51,7 @@ struct ObsTc {
   const float* row_iz;
   const float* row_q2;
   const float* row_y2;
-  float* score;                                 // [n_rb][H][N]
+  float* score;                                 // [2 n_rb][H][N] (row block rb, column group g at 2 rb + g)
   float* a2s;
   float* kus;
   float* part_y;                                // [U][n_split][128 rows][128 d]
@@ -96,6 +101,19 @@ __device__ __forceinline__ void ld128(uint32_t taddr, uint32_t (&v)[8][16]) {
   tc::tmem_wait_ld_dep4(v[4], v[5], v[6], v[7]);
 }
 
+__device__ __forceinline__ void ld64(uint32_t taddr, uint32_t (&v)[4][16]) {
+  tc::tmem_ld16(taddr + 0, v[0]);
+  tc::tmem_ld16(taddr + 16, v[1]);
+  tc::tmem_ld16(taddr + 32, v[2]);
+  tc::tmem_ld16(taddr + 48, v[3]);
+  tc::tmem_wait_ld_dep4(v[0], v[1], v[2], v[3]);
+}
+
+template <typename U>
+__device__ __forceinline__ float* align16f(U* p) {
+  return reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(p) + 15) & ~static_cast<uintptr_t>(15));
+}
+
 __device__ __forceinline__ unsigned char* aligned_base(unsigned char* raw) {
   return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~static_cast<uintptr_t>(1023));
 }
@@ -142,7 +160,7 @@ obs_a_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
   if (threadIdx.x == 0) {
     tc::mbar_init(&ctl.q_full, 1);
     for (int s = 0; s < S; ++s) { tc::mbar_init(&ctl.x_full[s], 1); tc::mbar_init(&ctl.x_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { tc::mbar_init(&ctl.acc_full[b], 1); tc::mbar_init(&ctl.acc_empty[b], 128); }
+    for (int b = 0; b < 2; ++b) { tc::mbar_init(&ctl.acc_full[b], 1); tc::mbar_init(&ctl.acc_empty[b], kEpi); }
     tc::mbar_init(&ctl.drain, 1);
     ctl.err = 0;
     tc::fence_barrier_init();
@@ -188,23 +206,24 @@ obs_a_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
       tc::mbar_wait(&ctl.drain, 0);
     }
   } else {
-    const int qd = warp & 3, r = qd * 32 + lane;
+    // group g takes tokens 64 g .. 64 g + 63 of every tile
+    const int qd = warp & 3, g = (warp - 2) >> 2, r = qd * 32 + lane;
     const int lim = row_limit(a, it.rb * 128 + r);
     float m = -INFINITY, l = 0.f;
     for (int i = 0; i < it.n; ++i) {
       const int b = i & 1, ub = i >> 1;
       if (!tc::wait_or_fail(&ctl.acc_full[b], ub & 1, &ctl.err, a.counters, kDevErrTimeout)) break;
       tc::fence_after_sync();
-      uint32_t v[8][16];
-      ld128(tmem + ((uint32_t)(qd * 32) << 16) + b * 128, v);
+      uint32_t v[4][16];
+      ld64(tmem + ((uint32_t)(qd * 32) << 16) + b * 128 + g * 64, v);
       tc::fence_before_sync();
       tc::mbar_arrive(&ctl.acc_empty[b]);
-      const int t0 = (it.tile0 + i) * 128;
+      const int t0 = (it.tile0 + i) * 128 + g * 64;
       if (lim < t0) continue;                       // nothing visible (or padding row)
-      const bool full = t0 + 127 <= lim;
+      const bool full = t0 + 63 <= lim;
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
+      for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float y = __uint_as_float(v[c][e]) * a.c2;
@@ -212,18 +231,19 @@ obs_a_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
           if (full || t0 + c * 16 + e <= lim) mx = fmaxf(mx, y);
         }
       const float mn = fmaxf(m, mx);
-      float sum = 0.f;
+      float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
+      for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float p = tc::ex2_approx(__uint_as_float(v[c][e]) - mn);
-          sum += (full || t0 + c * 16 + e <= lim) ? p : 0.f;
+          const float q = (full || t0 + c * 16 + e <= lim) ? p : 0.f;
+          if (e & 1) sum1 += q; else sum0 += q;
         }
-      l = l * tc::ex2_approx(m - mn) + sum;
+      l = l * tc::ex2_approx(m - mn) + (sum0 + sum1);
       m = mn;
     }
-    const int64_t pi = ((int64_t)it.u * a.n_split + it.s) * 128 + r;
+    const int64_t pi = ((int64_t)it.u * 2 * a.n_split + 2 * it.s + g) * 128 + r;
     a.part_m2[pi] = m;
     a.part_l[pi] = l;
   }
@@ -237,11 +257,12 @@ __global__ void obs_rows_kernel(const __nv_bfloat16* __restrict__ Q, ObsTc a, fl
                                 float* __restrict__ row_iz, float* __restrict__ row_q2) {
   const int u = blockIdx.x, r = threadIdx.x;
   const int h = u / a.n_rb, rb = u % a.n_rb, rr = rb * 128 + r;
+  const int np = 2 * a.n_split;
   float M = -INFINITY;
-  for (int s = 0; s < a.n_split; ++s) M = fmaxf(M, a.part_m2[((int64_t)u * a.n_split + s) * 128 + r]);
+  for (int s = 0; s < np; ++s) M = fmaxf(M, a.part_m2[((int64_t)u * np + s) * 128 + r]);
   float Z = 0.f;
-  for (int s = 0; s < a.n_split; ++s) {
-    const int64_t pi = ((int64_t)u * a.n_split + s) * 128 + r;
+  for (int s = 0; s < np; ++s) {
+    const int64_t pi = ((int64_t)u * np + s) * 128 + r;
     if (a.part_m2[pi] > -INFINITY) Z = fmaf(a.part_l[pi], exp2f(a.part_m2[pi] - M), Z);
   }
   float q2 = 0.f;
@@ -276,7 +297,7 @@ obs_b_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
   unsigned char* xs = q + kOp;                   // stage s: K at xs + 2s kOp, V at + kOp
   unsigned char* al = xs + S * 2 * kOp;          // alpha hi at al, lo at al + kOp (MN-major)
   CtlB& ctl = *reinterpret_cast<CtlB*>(al + 2 * kOp);
-  float* cm2 = reinterpret_cast<float*>(&ctl + 1);
+  float* cm2 = align16f(&ctl + 1);               // 16-byte aligned for float4 reads
   float* ciz = cm2 + 128;
   int* clim = reinterpret_cast<int*>(ciz + 128);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -284,8 +305,8 @@ obs_b_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
   if (threadIdx.x == 0) {
     tc::mbar_init(&ctl.q_full, 1);
     for (int s = 0; s < S; ++s) { tc::mbar_init(&ctl.x_full[s], 1); tc::mbar_init(&ctl.x_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { tc::mbar_init(&ctl.s_full[b], 1); tc::mbar_init(&ctl.s_empty[b], 128); }
-    tc::mbar_init(&ctl.al_full, 128);
+    for (int b = 0; b < 2; ++b) { tc::mbar_init(&ctl.s_full[b], 1); tc::mbar_init(&ctl.s_empty[b], kEpi); }
+    tc::mbar_init(&ctl.al_full, kEpi);
     tc::mbar_init(&ctl.al_empty, 1);
     tc::mbar_init(&ctl.y_full, 1);
     tc::mbar_init(&ctl.drain, 1);
@@ -293,7 +314,7 @@ obs_b_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
     tc::fence_barrier_init();
   }
   if (warp == 1) { tc::tmem_alloc(&ctl.tmem_base, 512); tc::tmem_relinquish(); }
-  if (threadIdx.x >= 64) {
+  if (threadIdx.x >= 64 && threadIdx.x < 64 + 128) {
     const int r = threadIdx.x - 64;
     cm2[r] = a.row_m2[(int64_t)it.u * 128 + r];
     ciz[r] = a.row_iz[(int64_t)it.u * 128 + r];
@@ -359,80 +380,88 @@ obs_b_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
       tc::mbar_wait(&ctl.drain, 0);
     }
   } else {
-    const int qd = warp & 3, tl = qd * 32 + lane;
+    // group g takes observation rows 64 g .. 64 g + 63 of every token
+    const int qd = warp & 3, g = (warp - 2) >> 2, tl = qd * 32 + lane;
+    const int rb2 = 2 * it.rb + g;
     bool ok = true;
     for (int i = 0; i < it.n; ++i) {
       const int b = i & 1, ub = i >> 1, s = i % S;
       if (!tc::wait_or_fail(&ctl.s_full[b], ub & 1, &ctl.err, a.counters, kDevErrTimeout)) { ok = false; break; }
       tc::fence_after_sync();
-      uint32_t v[8][16];
-      ld128(tmem + ((uint32_t)(qd * 32) << 16) + b * 128, v);
+      uint32_t v[4][16];
+      ld64(tmem + ((uint32_t)(qd * 32) << 16) + b * 128 + g * 64, v);
       tc::fence_before_sync();
       tc::mbar_arrive(&ctl.s_empty[b]);
       const int t = (it.tile0 + i) * 128 + tl;
       float sc = 0.f, a2 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
+      for (int c = 0; c < 4; ++c) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int r = c * 16 + e;
-          float al_ = tc::ex2_approx(fmaf(__uint_as_float(v[c][e]), a.c2, -cm2[r])) * ciz[r];
-          al_ = (t <= clim[r]) ? al_ : 0.f;
-          v[c][e] = __float_as_uint(al_);
-          sc += al_;
-          a2 = fmaf(al_, al_, a2);
+        for (int e4 = 0; e4 < 16; e4 += 4) {
+          const int r0 = g * 64 + c * 16 + e4;
+          const float4 m4 = *reinterpret_cast<const float4*>(&cm2[r0]);
+          const float4 z4 = *reinterpret_cast<const float4*>(&ciz[r0]);
+          const int4 l4 = *reinterpret_cast<const int4*>(&clim[r0]);
+          const float mm[4] = {m4.x, m4.y, m4.z, m4.w}, zz[4] = {z4.x, z4.y, z4.z, z4.w};
+          const int ll[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float al_ = tc::ex2_approx(fmaf(__uint_as_float(v[c][e4 + q]), a.c2, -mm[q])) * zz[q];
+            al_ = (t <= ll[q]) ? al_ : 0.f;
+            v[c][e4 + q] = __float_as_uint(al_);
+            sc += al_;
+            a2 = fmaf(al_, al_, a2);
+          }
         }
+      }
       if (it.rb == 0 && t < a.N) {
-        const unsigned char* kt = xs + 2 * s * kOp;
-        a.xnorm[(int64_t)it.h * a.N + t] = sqrtf(row_sumsq(kt, tl));
-        a.xnorm[((int64_t)a.H + it.h) * a.N + t] = sqrtf(row_sumsq(kt + kOp, tl));
+        const unsigned char* xt = xs + 2 * s * kOp + g * kOp;    // group 0: K, group 1: V
+        a.xnorm[((int64_t)g * a.H + it.h) * a.N + t] = sqrtf(row_sumsq(xt, tl));
       }
       if (i > 0 && !tc::wait_or_fail(&ctl.al_empty, (i - 1) & 1, &ctl.err, a.counters, kDevErrTimeout)) {
         ok = false;
         break;
       }
-      // alpha[t][r] as bf16 hi + lo, MN-major (r contiguous), 128-byte swizzle
+      // alpha[t][r] as bf16 hi + lo, MN-major (r contiguous), 128-byte
+      // swizzle; this group's rows are the 64-row half g of the tile
 #pragma unroll
-      for (int blk = 0; blk < 2; ++blk)
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t hw[4], lw[4];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint32_t hw[4], lw[4];
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            const int r = blk * 64 + ch * 8 + 2 * p;
-            const float x0 = __uint_as_float(v[r >> 4][r & 15]), x1 = __uint_as_float(v[(r + 1) >> 4][(r + 1) & 15]);
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(x0, x1);
-            const float2 hf = __bfloat1622float2(h2);
-            const __nv_bfloat162 l2 = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
-            hw[p] = *reinterpret_cast<const uint32_t*>(&h2);
-            lw[p] = *reinterpret_cast<const uint32_t*>(&l2);
-          }
-          const int off = blk * kHalf + tl * 128 + ((ch ^ (tl & 7)) << 4);
-          *reinterpret_cast<uint4*>(al + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(al + kOp + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        for (int p = 0; p < 4; ++p) {
+          const int r = ch * 8 + 2 * p;                 // within the group's 64 rows
+          const float x0 = __uint_as_float(v[r >> 4][r & 15]), x1 = __uint_as_float(v[(r + 1) >> 4][(r + 1) & 15]);
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(x0, x1);
+          const float2 hf = __bfloat1622float2(h2);
+          const __nv_bfloat162 l2 = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+          hw[p] = *reinterpret_cast<const uint32_t*>(&h2);
+          lw[p] = *reinterpret_cast<const uint32_t*>(&l2);
         }
+        const int off = g * kHalf + tl * 128 + ((ch ^ (tl & 7)) << 4);
+        *reinterpret_cast<uint4*>(al + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(al + kOp + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&ctl.al_full);
       if (t < a.N) {
-        const int64_t o = ((int64_t)it.rb * a.H + it.h) * a.N + t;
+        const int64_t o = ((int64_t)rb2 * a.H + it.h) * a.N + t;
         a.score[o] = sc;
         a.a2s[o] = a2;
       }
     }
-    // partial ybar^T: TMEM lane = d, column = row r
+    // partial ybar^T: TMEM lane = d, column = row r (this group's 64 rows)
+    float* py = a.part_y + ((int64_t)it.u * a.n_split + it.s) * 128 * 128;
     if (ok && it.n > 0 && tc::wait_or_fail(&ctl.y_full, 0, &ctl.err, a.counters, kDevErrTimeout)) {
       tc::fence_after_sync();
-      uint32_t v[8][16];
-      ld128(tmem + ((uint32_t)(qd * 32) << 16) + ycol, v);
+      uint32_t v[4][16];
+      ld64(tmem + ((uint32_t)(qd * 32) << 16) + ycol + g * 64, v);
       const int d = tl;
-      float* py = a.part_y + ((int64_t)it.u * a.n_split + it.s) * 128 * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
+      for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int e = 0; e < 16; ++e) py[(c * 16 + e) * 128 + d] = __uint_as_float(v[c][e]);
+        for (int e = 0; e < 16; ++e) py[(g * 64 + c * 16 + e) * 128 + d] = __uint_as_float(v[c][e]);
     } else if (it.n == 0) {
-      float* py = a.part_y + ((int64_t)it.u * a.n_split + it.s) * 128 * 128;
-      for (int r = 0; r < 128; ++r) py[r * 128 + tl] = 0.f;
+      for (int r = g * 64; r < g * 64 + 64; ++r) py[r * 128 + tl] = 0.f;
     }
   }
   tc::fence_before_sync();
@@ -489,7 +518,7 @@ obs_c_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
   unsigned char* yl = yh + kOp;
   unsigned char* xs = yl + kOp;                  // stage s: K at xs + 2s kOp, V at + kOp
   CtlC& ctl = *reinterpret_cast<CtlC*>(xs + S * 2 * kOp);
-  float* cm2 = reinterpret_cast<float*>(&ctl + 1);
+  float* cm2 = align16f(&ctl + 1);               // 16-byte aligned for float4 reads
   float* ciq = cm2 + 128;                       // ||q_r||^2 / Z_r^2
   float* cy2 = ciq + 128;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -497,13 +526,13 @@ obs_c_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
   if (threadIdx.x == 0) {
     tc::mbar_init(&ctl.b_full, 1);
     for (int s = 0; s < S; ++s) { tc::mbar_init(&ctl.x_full[s], 1); tc::mbar_init(&ctl.x_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { tc::mbar_init(&ctl.acc_full[b], 1); tc::mbar_init(&ctl.acc_empty[b], 128); }
+    for (int b = 0; b < 2; ++b) { tc::mbar_init(&ctl.acc_full[b], 1); tc::mbar_init(&ctl.acc_empty[b], kEpi); }
     tc::mbar_init(&ctl.drain, 1);
     ctl.err = 0;
     tc::fence_barrier_init();
   }
   if (warp == 1) { tc::tmem_alloc(&ctl.tmem_base, 512); tc::tmem_relinquish(); }
-  if (threadIdx.x >= 64) {
+  if (threadIdx.x >= 64 && threadIdx.x < 64 + 128) {
     const int r = threadIdx.x - 64;
     const int64_t o = (int64_t)it.u * 128 + r;
     cm2[r] = a.row_m2[o];
@@ -559,20 +588,30 @@ obs_c_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
       tc::mbar_wait(&ctl.drain, 0);
     }
   } else {
-    const int qd = warp & 3, tl = qd * 32 + lane;
+    // group g takes observation rows 64 g .. 64 g + 63 of every token
+    const int qd = warp & 3, g = (warp - 2) >> 2, tl = qd * 32 + lane;
+    const int rb2 = 2 * it.rb + g;
+    const float c2x2 = 2.f * a.c2;
+    // ||V_t||^2 of this thread's token, one tile ahead
+    auto vnorm2 = [&](int i) -> float {
+      const int t = (it.tile0 + i) * 128 + tl;
+      const float vn = (i < it.n && t < a.N) ? a.xnorm[((int64_t)a.H + it.h) * a.N + t] : 0.f;
+      return vn * vn;
+    };
+    float v2n = vnorm2(0);
     for (int i = 0; i < it.n; ++i) {
       const int b = i & 1, ub = i >> 1;
+      const float v2 = v2n;
+      v2n = vnorm2(i + 1);
       if (!tc::wait_or_fail(&ctl.acc_full[b], ub & 1, &ctl.err, a.counters, kDevErrTimeout)) break;
       tc::fence_after_sync();
       const int t = (it.tile0 + i) * 128 + tl;
-      const float vn = (t < a.N) ? a.xnorm[((int64_t)a.H + it.h) * a.N + t] : 0.f;
-      const float v2 = vn * vn;
-      const uint32_t base = tmem + ((uint32_t)(qd * 32) << 16) + b * 256;
+      const uint32_t base = tmem + ((uint32_t)(qd * 32) << 16) + b * 256 + g * 64;
       // every live row sees the whole tile unless it reaches into the window
       const bool full = (it.tile0 + i) * 128 + 127 <= a.N - a.W;
-      float ku = 0.f;
+      float ku0 = 0.f, ku1 = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t s0[16], s1[16], y0[16], y1[16];
         tc::tmem_ld16(base + c * 32, s0);
         tc::tmem_ld16(base + c * 32 + 16, s1);
@@ -580,20 +619,29 @@ obs_c_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
         tc::tmem_ld16(base + 128 + c * 32 + 16, y1);
         tc::tmem_wait_ld_dep4(s0, s1, y0, y1);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int r = c * 32 + e;
-          const float sv = __uint_as_float(e < 16 ? s0[e] : s1[e - 16]);
-          const float vy = __uint_as_float(e < 16 ? y0[e] : y1[e - 16]);
-          // alpha^2 ||q||^2 = 2^(2 (s c2 - M2)) ||q||^2 / Z^2
-          float w = tc::ex2_approx(2.f * fmaf(sv, a.c2, -cm2[r])) * ciq[r];
-          if (!full && t > row_limit(a, it.rb * 128 + r)) w = 0.f;
-          const float dist = fmaf(-2.f, vy, v2 + cy2[r]);
-          ku = fmaf(w, dist, ku);
+        for (int e4 = 0; e4 < 32; e4 += 4) {
+          const int r0 = g * 64 + c * 32 + e4;
+          const float4 m4 = *reinterpret_cast<const float4*>(&cm2[r0]);
+          const float4 q4 = *reinterpret_cast<const float4*>(&ciq[r0]);
+          const float4 y4 = *reinterpret_cast<const float4*>(&cy2[r0]);
+          const float mm[4] = {m4.x, m4.y, m4.z, m4.w}, qq[4] = {q4.x, q4.y, q4.z, q4.w};
+          const float yy[4] = {y4.x, y4.y, y4.z, y4.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int e = e4 + q;
+            const float sv = __uint_as_float(e < 16 ? s0[e] : s1[e - 16]);
+            const float vy = __uint_as_float(e < 16 ? y0[e] : y1[e - 16]);
+            // alpha^2 ||q||^2 = 2^(2 (s c2 - M2)) ||q||^2 / Z^2
+            float w = tc::ex2_approx(fmaf(sv, c2x2, -2.f * mm[q])) * qq[q];
+            if (!full && t > row_limit(a, it.rb * 128 + r0 + q)) w = 0.f;
+            const float dist = fmaf(-2.f, vy, v2 + yy[q]);
+            if (q & 1) ku1 = fmaf(w, dist, ku1); else ku0 = fmaf(w, dist, ku0);
+          }
         }
       }
       tc::fence_before_sync();
       tc::mbar_arrive(&ctl.acc_empty[b]);
-      if (t < a.N) a.kus[((int64_t)it.rb * a.H + it.h) * a.N + t] = ku;
+      if (t < a.N) a.kus[((int64_t)rb2 * a.H + it.h) * a.N + t] = ku0 + ku1;
     }
   }
   tc::fence_before_sync();
