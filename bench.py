@@ -116,6 +116,35 @@ def stage_roofline(stage, units, ms_per_launch, peaks):
     return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak}
 
 
+# ---------------------------------------------------------------- ranks (host logic, also used by the gloo tests)
+
+def rank_spec(spec, rank: int, layers: int = 0):
+    """The cache rank `rank` compresses: an independent seed per rank (the
+    layers of one model split over ranks share nothing), optionally fewer layers."""
+    out = type(spec)(**{**spec.__dict__, "seed": spec.seed + rank})
+    if layers:
+        out = type(spec)(**{**out.__dict__, "n_layers": min(layers, out.n_layers)})
+    return out
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    """Maximum of x over the ranks of the default process group (x itself
+    when running alone)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput in Mtok/s: every rank's layer-head tokens over the
+    slowest rank's step time."""
+    return tokens_per_rank * world / (ms_per_step / 1e3) / 1e6
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -214,9 +243,7 @@ def run_gpu(args, world, rank, local):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     wl = WORKLOADS[WORKLOAD]
     spec, theta = wl["spec"], wl["theta"]
-    spec = type(spec)(**{**spec.__dict__, "seed": spec.seed + rank})     # an independent cache per rank
-    if args.layers:
-        spec = type(spec)(**{**spec.__dict__, "n_layers": min(args.layers, spec.n_layers)})
+    spec = rank_spec(spec, rank, args.layers)     # an independent cache per rank
     Lr, H, N = spec.n_layers, spec.n_kv_heads, spec.n_tokens
 
     cpu_base = None
@@ -265,11 +292,7 @@ def run_gpu(args, world, rank, local):
     barrier()
     launches = api.launch_count() - n0
     clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(ev0.elapsed_time(ev1), world, dev)
     ms_step = ms / args.steps
 
     # decode alone and compress alone (same stream, CUDA events) for the metric's parts
@@ -281,7 +304,7 @@ def run_gpu(args, world, rank, local):
             api.decode_attn(params[l], outs[l], qd[l], out=dout[l], workspace=dws)
     ev3.record(stream)
     barrier()
-    dec_us = 1e3 * ev2.elapsed_time(ev3) / args.steps
+    dec_us = 1e3 * reduce_max(ev2.elapsed_time(ev3), world, dev) / args.steps
 
     # per-stage event timing over the same steps, for the roofline of the dominant kernel
     api.stage_timing(True)
@@ -306,8 +329,7 @@ def run_gpu(args, world, rank, local):
                    for st in per_launch}
 
     dec_bytes = Lr * L["total_bytes"]
-    tokens_step = N * Lr * H * world
-    value = tokens_step / (ms_step / 1e3) / 1e6
+    value = job_value(N * Lr * H, world, ms_step)
 
     e2e = None
     if not args.no_e2e:
@@ -387,16 +409,11 @@ def run_e2e(args, spec, theta, params, dev, stream, barrier, world):
         step()
     e1.record(stream)
     barrier()
-    ms = e0.elapsed_time(e1) / steps
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(e0.elapsed_time(e1), world, dev) / steps
     h2d = sum(x.numel() * x.element_size() for t3 in host for x in t3) + sum(q.numel() * q.element_size() for q in qh)
     d2h = sum(o.numel() for o in outs_h) + oh.numel() * 4
-    tokens = spec.n_tokens * Lr * spec.n_kv_heads * world
-    return {"value": tokens / (ms / 1e3) / 1e6, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+    return {"value": job_value(spec.n_tokens * Lr * spec.n_kv_heads, world, ms), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": ms, "steps": steps}
 
 

@@ -1,0 +1,64 @@
+"""Host logic of the multi-rank benchmark on CPU: two `gloo` ranks.
+
+Layers of a model are independent compression problems (the budget is per
+layer), so ranks shard them with no collective on the data path; the only
+exchange is the max-over-ranks reduction of the step time.  These tests run
+that host logic as two processes on the CPU, with the oracle standing in for
+the per-rank work.
+"""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from kv_cache_compression_anchorkv_b200.synthetic import CacheSpec, make_layer
+from oracle import anchorkv_oracle as O
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank: int, world: int, port: int, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        spec = bench.rank_spec(CacheSpec(4, 1, 4, 300, n_dirs=8, seed=3), rank, layers=2)
+        # per-rank work: the oracle's compress of this rank's first layer
+        K, V, Q = make_layer(spec, 0)
+        p = O.Params(n_tokens=spec.n_tokens, n_kv_heads=1, n_q_heads=4, theta=0.3, dtype="bf16", seed=spec.seed)
+        res = O.compress_layer(K.double().numpy(), V.double().numpy(), Q.double().numpy(), p)
+        n_anchor = int(len(res["anchor_pos"][0]))
+        ms = bench.reduce_max(10.0 + rank, world, "cpu")           # rank 1 is the slower one
+        value = bench.job_value(spec.n_tokens * spec.n_layers * spec.n_kv_heads, world, ms)
+        out[rank] = (spec.seed, spec.n_layers, ms, value, n_anchor, float(K.float().sum()))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_shard_and_reduce():
+    world = 2
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world, join=True, start_method="spawn")
+        r0, r1 = out[0], out[1]
+    # independent caches per rank, layers capped
+    assert (r0[0], r1[0]) == (3, 4) and r0[1] == r1[1] == 2
+    assert r0[5] != r1[5]
+    # both ranks see the slowest rank's time and the same whole-job value
+    assert r0[2] == r1[2] == 11.0
+    assert r0[3] == r1[3] == pytest.approx(300 * 2 * 1 * 2 / (11.0 / 1e3) / 1e6)
+    assert r0[4] == r1[4] == O.layout(O.Params(n_tokens=300, n_kv_heads=1, n_q_heads=4, theta=0.3))["k"]
+
+
+def test_single_rank_reduce_is_identity():
+    assert bench.reduce_max(7.5, 1, "cpu") == 7.5
+    assert bench.job_value(1000, 1, 1.0) == pytest.approx(1.0)
