@@ -44,6 +44,14 @@ def _peaks():
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
+    """SM clock and clock-event reasons of the benchmark's GPU, sampled every
+    10 ms from a thread through NVML while the timed region runs (read-only;
+    nvidia-smi at 200 ms when NVML is unavailable)."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -51,8 +59,41 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
+        self.thread = None
+        self.rows = []
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        pr = torch.cuda.get_device_properties(self.dev)
+        bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+        return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
 
     def start(self):
+        import threading
+        try:
+            nv, h = self._nvml_handle()
+        except Exception:
+            nv = None
+        if nv is not None:
+            self.stop_flag = threading.Event()
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+
+            def poll():
+                while not self.stop_flag.is_set():
+                    try:
+                        clk = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.rows.append((float(clk), float(mx), [n for n, c in self.REASONS
+                                                                   if rs & getattr(nv, c, 0)]))
+                    except Exception:
+                        pass
+                    self.stop_flag.wait(0.01)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
@@ -61,23 +102,30 @@ class ClockSampler:
             self.proc = None
 
     def stop(self) -> dict | None:
-        if self.proc is None:
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            rows = self.rows
+        elif self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            names = [n for n, _ in self.REASONS[:4]]
+            rows = [(float(r[1]), float(r[2]), [n for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"])
+                    for r in (x.split(",") for x in out.strip().splitlines()) if len(r) >= 9]
+        else:
             return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows]
-        mx = max(float(r[2]) for r in rows)
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
-        loaded = [s for s in sm if s > 0.5 * mx] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows)}
+        mx = max(r[1] for r in rows)
+        sm = [r[0] for r in rows]
+        loaded = [v for v in sm if v > 0.5 * mx] or sm
+        reasons = sorted({n for r in rows for n in r[2]})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows),
+                "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
 # ---------------------------------------------------------------- algorithmic units per stage
@@ -193,11 +241,18 @@ def _threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(spec, theta, n_heads=2):
-    dt, toks = _oracle_sample(spec, theta, n_heads)
-    return {"value": toks / dt / 1e6, "unit": UNIT, "cores": _threads(), "kind": "oracle",
-            "sample": f"one layer, {n_heads} of {spec.n_kv_heads} KV heads (N={spec.n_tokens}), fp64 numpy, "
-                      f"{dt:.1f} s"}
+def cpu_baseline(spec, theta, min_seconds=10.0, max_reps=4):
+    """The oracle on one full layer (all KV heads) of the workload, repeated
+    until about `min_seconds` of CPU work have been timed."""
+    total, toks, reps = 0.0, 0, 0
+    while reps < max_reps and (reps == 0 or total < min_seconds):
+        dt, t = _oracle_sample(spec, theta, spec.n_kv_heads)
+        total += dt
+        toks += t
+        reps += 1
+    return {"value": toks / total / 1e6, "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "sample": f"{reps} x one layer, all {spec.n_kv_heads} KV heads (N={spec.n_tokens}), fp64 numpy, "
+                      f"{total:.1f} s"}
 
 
 def run_reference(args):

@@ -78,7 +78,7 @@ struct PadList {
 };
 
 struct SelSmem {
-  RadixSmem rs;
+  RadixSmem<kThreads> rs;
   int warp_tot[kWarps];
   int cta_count;                     // this CTA's count exposed to the cluster
   float stage[kSeg + 256];           // raw scores of one pooling segment (kappa <= 255)
@@ -87,11 +87,11 @@ struct SelSmem {
 // Flags the selected positions of this thread's run [lo, hi): keys below the
 // threshold prefix, and keys equal to it either all or the first `need` in
 // position order across the cluster.
-template <typename KeyF>
-__device__ void mark_selected(SelSmem& sm, const RadixResult& sr, int lo, int hi, uint8_t* flag, KeyF key) {
+template <typename K, typename KeyF>
+__device__ void mark_selected(SelSmem& sm, const RadixResult<K>& sr, int lo, int hi, uint8_t* flag, KeyF key) {
   int ties = 0;
   for (int i = lo; i < hi; ++i) {
-    uint64_t kk;
+    K kk;
     if (key(i - lo, kk) && radix_top(kk, sr.bits) == sr.prefix) ++ties;
   }
   int rank0 = 0;
@@ -108,9 +108,9 @@ __device__ void mark_selected(SelSmem& sm, const RadixResult& sr, int lo, int hi
   // keys are read before any flag of this thread changes (the value-sample
   // key excludes flagged positions)
   for (int i = lo; i < hi; ++i) {
-    uint64_t kk;
+    K kk;
     if (!key(i - lo, kk)) continue;
-    const uint64_t top = radix_top(kk, sr.bits);
+    const K top = radix_top(kk, sr.bits);
     if (top < sr.prefix) {
       flag[i] = 1;
     } else if (top == sr.prefix) {
@@ -184,13 +184,13 @@ anchor_select_kernel(const float* __restrict__ score, float* __restrict__ pooled
 
   // 2. the n_s largest pooled scores, ties to the lower position
   if (!all_anchors && n_s > 0) {
-    auto key = [&](int j, uint64_t& kk) -> bool {
+    auto key = [&](int j, uint32_t& kk) -> bool {
       const int i = lo + j;
       if (i >= hi || c0 + i >= NW) return false;
-      kk = (uint64_t)keys[i] << 32;
+      kk = keys[i];
       return true;
     };
-    const RadixResult sr = cluster_radix_select<kThreads, kC>(sm.rs, ppt, n_s, 32, key);
+    const RadixResult<uint32_t> sr = cluster_radix_select<kThreads, kC, uint32_t>(sm.rs, ppt, n_s, key);
     mark_selected(sm, sr, lo, hi, flag, key);
   }
   // 3. the n_u smallest hash keys among the other non-window positions
@@ -201,7 +201,7 @@ anchor_select_kernel(const float* __restrict__ score, float* __restrict__ pooled
       kk = anchor_key(seed, layer, h, c0 + i);
       return true;
     };
-    const RadixResult sr = cluster_radix_select<kThreads, kC>(sm.rs, ppt, n_u, 64, key);
+    const RadixResult<uint64_t> sr = cluster_radix_select<kThreads, kC, uint64_t>(sm.rs, ppt, n_u, key);
     mark_selected(sm, sr, lo, hi, flag, key);
   }
 

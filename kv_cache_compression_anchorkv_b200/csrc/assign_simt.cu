@@ -143,8 +143,11 @@ assign_simt_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __
 constexpr int kRefineWarps = 8;
 constexpr int kRefineMaxK = 2048;
 template <typename T> struct RefineCfg;
+// kChunk slots per staging round; the transposed rows are kChunk + 1 pairs
+// apart so that the staging stores of consecutive pairs fall in different banks.
 template <> struct RefineCfg<__nv_bfloat16> { using P = __nv_bfloat162; static constexpr int kChunk = 448; };
 template <> struct RefineCfg<float> { using P = float2; static constexpr int kChunk = 192; };
+template <typename T> __host__ __device__ constexpr int refine_ld() { return RefineCfg<T>::kChunk + 1; }
 
 __device__ __forceinline__ float2 pair_f(__nv_bfloat162 p) { return __bfloat1622float2(p); }
 __device__ __forceinline__ float2 pair_f(float2 p) { return p; }
@@ -158,8 +161,9 @@ refine_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restr
   using P = typename RefineCfg<T>::P;
   constexpr int CH = RefineCfg<T>::kChunk;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  P* aT = reinterpret_cast<P*>(smem_raw);                              // [64][CH]
-  float* xs = reinterpret_cast<float*>(aT + 64 * CH);                  // [8][128]
+  constexpr int LD = refine_ld<T>();
+  P* aT = reinterpret_cast<P*>(smem_raw);                              // [64][LD]
+  float* xs = reinterpret_cast<float*>(aT + 64 * LD);                  // [8][128]
   float* sc = xs + kRefineWarps * kD;                                  // [8][kRefineMaxK]
   const int u = blockIdx.y, side = u / H, h = u % H;
   const int n = counters[kRefineListBase + u];
@@ -175,7 +179,7 @@ refine_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restr
     for (int i = threadIdx.x; i < cn * 64; i += blockDim.x) {
       const int j = i / 64, dp = i % 64;
       const T* src = A + (int64_t)(c0 + j) * kD + 2 * dp;
-      aT[dp * CH + j] = *reinterpret_cast<const P*>(src);
+      aT[dp * LD + j] = *reinterpret_cast<const P*>(src);
     }
     __syncthreads();
   };
@@ -201,7 +205,7 @@ refine_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restr
         float acc = 0.f;
 #pragma unroll 8
         for (int dp = 0; dp < 64; ++dp) {
-          const float2 av = pair_f(aT[dp * CH + j]);
+          const float2 av = pair_f(aT[dp * LD + j]);
           acc = fmaf(xw[2 * dp], av.x, acc);
           acc = fmaf(xw[2 * dp + 1], av.y, acc);
         }
@@ -238,7 +242,7 @@ refine_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restr
 
 template <typename T>
 constexpr int refine_smem() {
-  return 64 * RefineCfg<T>::kChunk * (int)sizeof(typename RefineCfg<T>::P) + kRefineWarps * kD * 4 +
+  return 64 * refine_ld<T>() * (int)sizeof(typename RefineCfg<T>::P) + kRefineWarps * kD * 4 +
          kRefineWarps * kRefineMaxK * 4;
 }
 

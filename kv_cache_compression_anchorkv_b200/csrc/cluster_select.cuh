@@ -1,14 +1,15 @@
-// Cluster-wide radix select over 64-bit keys, shared by the anchor selection
-// and the top-R residual selection.
+// Cluster-wide radix select, shared by the anchor selection and the top-R
+// residual selection.
 //
 // The `want` smallest keys of a set spread over the C CTAs of a thread-block
-// cluster are found digit by digit (8 bits from the top): every CTA builds a
-// histogram of its keys that match the prefix found so far (one shared-memory
-// atomic per distinct bin of a warp), every CTA sums the C histograms through
-// distributed shared memory and picks the same digit.  The select stops as
-// soon as the threshold bin holds exactly the keys still needed.  The caller
-// then takes the keys below the threshold prefix and, at the threshold, all
-// of them or the first `need` in its own tie order.
+// cluster are found digit by digit (8 bits from the top): every warp counts
+// its keys that match the prefix found so far in a private histogram (native
+// shared-memory integer atomics), the CTA sums its warps' histograms, every
+// CTA sums the C CTA histograms through distributed shared memory and picks
+// the same digit.  The select stops as soon as the threshold bin holds
+// exactly the keys still needed.  The caller then takes the keys below the
+// threshold prefix and, at the threshold, all of them or the first `need` in
+// its own tie order.
 #pragma once
 
 #include "common.cuh"
@@ -26,48 +27,61 @@ __device__ __forceinline__ U* cluster_peer(U* p, unsigned rank) {
   return static_cast<U*>(__cluster_map_shared_rank(p, rank));
 }
 
+template <int kThreads>
 struct RadixSmem {
-  unsigned int hist[2][256];   // double-buffered local digit histograms
-  unsigned int tot[256];       // cluster totals of the current digit
+  unsigned int whist[kThreads / 32][256];   // per-warp histograms of the current digit
+  unsigned int hist[2][256];                // CTA histograms, double-buffered (read by peers)
+  unsigned int tot[256];                    // cluster totals of the current digit
   int scal[4];
 };
 
 // Keys whose top `bits` bits are below `prefix` are selected; keys equal to
 // it are all selected if `all_ties`, else the first `need` in tie order.
+template <typename K>
 struct RadixResult {
-  uint64_t prefix;
+  K prefix;
   int bits;
   int need;
   bool all_ties;
 };
 
-__device__ __forceinline__ uint64_t radix_top(uint64_t key, int bits) {
-  return bits >= 64 ? key : (bits ? key & (~0ull << (64 - bits)) : 0ull);
+template <typename K>
+__device__ __forceinline__ K radix_top(K key, int bits) {
+  constexpr int kB = 8 * (int)sizeof(K);
+  return bits >= kB ? key : (bits ? (K)(key & (~(K)0 << (kB - bits))) : (K)0);
 }
 
 // key(j, kk) is called for j in [0, iters) with the same `iters` in every
-// thread of the CTA; it returns false for items that take no part.  Keys have
-// `key_bits` significant bits from the top.  Every thread of every CTA
+// thread of the CTA; it returns false for items that take no part.  K is
+// uint32_t or uint64_t (all bits significant).  Every thread of every CTA
 // returns the same result.  Requires kThreads >= 256.
-template <int kThreads, int C, typename KeyF>
-__device__ RadixResult cluster_radix_select(RadixSmem& sm, int iters, int want, int key_bits, KeyF key) {
+template <int kThreads, int C, typename K, typename KeyF>
+__device__ RadixResult<K> cluster_radix_select(RadixSmem<kThreads>& sm, int iters, int want, KeyF key) {
   static_assert(kThreads >= 256 && kThreads % 32 == 0, "one thread per bin");
-  RadixResult res;
+  constexpr int kB = 8 * (int)sizeof(K);
+  constexpr int kWarps = kThreads / 32;
+  const int warp = threadIdx.x >> 5;
+  RadixResult<K> res;
   res.prefix = 0;
   res.need = want;
   res.all_ties = false;
   int buf = 0;
   int depth = 0;
-  for (; depth < key_bits; depth += 8) {
-    const int shift = 64 - depth - 8;
-    for (int i = threadIdx.x; i < 256; i += kThreads) sm.hist[buf][i] = 0u;
+  for (; depth < kB; depth += 8) {
+    const int shift = kB - depth - 8;
+    for (int i = threadIdx.x; i < kWarps * 256; i += kThreads) (&sm.whist[0][0])[i] = 0u;
     __syncthreads();
+    unsigned* wh = sm.whist[warp];
     for (int j = 0; j < iters; ++j) {
-      uint64_t kk = 0;
-      const bool take = key(j, kk) && radix_top(kk, depth) == res.prefix;
-      const unsigned bin = take ? (unsigned)((kk >> shift) & 255u) : 256u;
-      const unsigned same = __match_any_sync(0xffffffffu, bin);
-      if (take && (int)(threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&sm.hist[buf][bin], (unsigned)__popc(same));
+      K kk = 0;
+      if (key(j, kk) && radix_top(kk, depth) == res.prefix) atomicAdd(&wh[(unsigned)(kk >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x < 256) {
+      unsigned t = 0;
+#pragma unroll 8
+      for (int w = 0; w < kWarps; ++w) t += sm.whist[w][threadIdx.x];
+      sm.hist[buf][threadIdx.x] = t;
     }
     __syncthreads();
     cluster_barrier();
@@ -100,7 +114,7 @@ __device__ RadixResult cluster_radix_select(RadixSmem& sm, int iters, int want, 
     }
     __syncthreads();
     const int d = sm.scal[0], below = sm.scal[1], cnt = sm.scal[2];
-    res.prefix |= (uint64_t)d << shift;
+    res.prefix |= (K)d << shift;
     res.need -= below;
     __syncthreads();
     buf ^= 1;

@@ -118,8 +118,10 @@ __device__ __forceinline__ unsigned char* aligned_base(unsigned char* raw) {
   return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~static_cast<uintptr_t>(1023));
 }
 
-// Sum of squares of one token row of a swizzled [128][128] bf16 tile (the
-// chunk order inside the row does not matter for a norm).
+// Sum of squares of one token row of a swizzled [128][128] bf16 tile.  The
+// chunk order inside the row does not matter for a norm, so row r reads its
+// 16-byte chunks in the order c ^ (r & 7): the 8 rows of a quarter-warp then
+// hit 8 different bank groups.
 __device__ __forceinline__ float row_sumsq(const unsigned char* tile, int r) {
   float s = 0.f;
 #pragma unroll
@@ -127,7 +129,7 @@ __device__ __forceinline__ float row_sumsq(const unsigned char* tile, int r) {
     const uint4* p = reinterpret_cast<const uint4*>(tile + half * kHalf + r * 128);
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      const uint4 q = p[c];
+      const uint4 q = p[c ^ (r & 7)];
       const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {

@@ -29,7 +29,7 @@ constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 
 struct SelectSmem {
-  RadixSmem rs;
+  RadixSmem<kThreads> rs;
   int warp_tot[kWarps];
   int scal[4];
   int cta_ties, cta_recs;            // exposed to the cluster
@@ -101,26 +101,24 @@ select_kernel(const float* __restrict__ util, int N, int n_t, int n_sh, int R, i
   asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 
   // 1. threshold
-  RadixResult sr;
+  RadixResult<uint32_t> sr;
   sr.prefix = 0; sr.bits = 0; sr.need = 0; sr.all_ties = true;
   if (!take_all) {
     const int iters = (nt * kTile + kThreads - 1) / kThreads;
-    auto key = [&](int j, uint64_t& kk) -> bool {
+    auto key = [&](int j, uint32_t& kk) -> bool {
       const int q = j * kThreads + tid;
       if (q >= nt * kTile) return false;
-      const uint32_t k32 = key_of(q);
-      if (!eligible(q, k32)) return false;
-      kk = (uint64_t)k32 << 32;
-      return true;
+      kk = key_of(q);
+      return eligible(q, kk);
     };
-    sr = cluster_radix_select<kThreads, C>(sm.rs, iters, R, 32, key);
+    sr = cluster_radix_select<kThreads, C, uint32_t>(sm.rs, iters, R, key);
   }
   // classification of slot q: 2 = above the threshold, 1 = at it
   auto cls = [&](int q) -> int {
     const uint32_t k32 = key_of(q);
     if (!eligible(q, k32)) return 0;
     if (take_all) return 2;
-    const uint64_t top = radix_top((uint64_t)k32 << 32, sr.bits);
+    const uint32_t top = radix_top(k32, sr.bits);
     return top < sr.prefix ? 2 : (top == sr.prefix ? 1 : 0);
   };
 
