@@ -202,6 +202,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--layers", type=int, default=0, help="compress only the first L layers (profiling runs)")
+    ap.add_argument("--compress-streams", type=int, default=4,
+                    help="compress layers round-robin on this many streams (independent layers overlap)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -319,10 +321,33 @@ def run_gpu(args, world, rank, local):
     dws = torch.empty(api.decode_workspace_bytes(params[0], 1), dtype=torch.uint8, device=dev)
     dout = [torch.empty(1, spec.n_q_heads, spec.head_dim, dtype=torch.float32, device=dev) for _ in range(Lr)]
     stream = torch.cuda.current_stream(dev)
+    # layers are independent compression problems: optionally several streams,
+    # each with its own workspace; decode stays sequential over layers (a
+    # layer's query depends on the previous layer's output)
+    n_cs = max(1, args.compress_streams)
+    cstreams = [torch.cuda.Stream(dev) for _ in range(n_cs)] if n_cs > 1 else []
+    wss = [ws] + [torch.empty_like(ws) for _ in range(n_cs - 1)]
 
-    def step():
+    def compress_all(single=False):
+        if single or not cstreams:
+            for l in range(Lr):
+                api.compress(params[l], Ks[l], Vs[l], Qs[l], out=outs[l], workspace=ws)
+            return
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        for cs in cstreams:
+            cs.wait_event(fork)
         for l in range(Lr):
-            api.compress(params[l], Ks[l], Vs[l], Qs[l], out=outs[l], workspace=ws)
+            i = l % n_cs
+            with torch.cuda.stream(cstreams[i]):
+                api.compress(params[l], Ks[l], Vs[l], Qs[l], out=outs[l], workspace=wss[i])
+        for cs in cstreams:
+            join = torch.cuda.Event()
+            join.record(cs)
+            stream.wait_event(join)
+
+    def step(single=False):
+        compress_all(single)
         for l in range(Lr):
             api.decode_attn(params[l], outs[l], qd[l], out=dout[l], workspace=dws)
 
@@ -333,7 +358,8 @@ def run_gpu(args, world, rank, local):
 
     for _ in range(args.warmup):
         step()
-    status = api.read_status(ws)
+    status = [api.read_status(w)[0] for w in wss]
+    status = [max(status, key=abs)]
     barrier()
     clocks = ClockSampler(local)
     clocks.start()
@@ -365,7 +391,7 @@ def run_gpu(args, world, rank, local):
     api.stage_timing(True)
     barrier()
     for _ in range(args.steps):
-        step()
+        step(single=True)     # one stream: stage events do not overlap
     barrier()
     stages = api.stage_times()
     api.stage_timing(False)
@@ -397,7 +423,7 @@ def run_gpu(args, world, rank, local):
             "vs_baseline": None, "dtype": spec.dtype, "data": "synthetic",
             "config": {"workload": WORKLOAD, "layers": Lr, "kv_heads": H, "q_heads": spec.n_q_heads,
                        "head_dim": spec.head_dim, "n_tokens": N, "window": spec.window, "theta": theta,
-                       "decode_batch": 1, "parallelism": f"replicas{world}",
+                       "decode_batch": 1, "parallelism": f"replicas{world}", "compress_streams": n_cs,
                        "l2": "inputs larger than L2 (%.1f GB of K/V per step)" % (Lr * 2 * H * N * 128 * 2 / 1e9)},
             "decode_us_per_step": dec_us,
             "decode_launch": api.decode_config(params[0], 1),
@@ -437,19 +463,32 @@ def run_e2e(args, spec, theta, params, dev, stream, barrier, world):
         K, V, Q = make_layer(spec, l, device=dev)
         host.append(tuple(x.cpu().pin_memory() for x in (K, V, Q)))
     qh = [make_decode_queries(spec, l, 0, 1, device=dev).cpu().pin_memory() for l in range(Lr)]
-    comp = api.HostCompressor(api.AnchorKVParams(**{**params[0].__dict__}), device=dev)
-    outs_h = [torch.empty_like(comp.host_out).pin_memory() for _ in range(Lr)]
+    n_cs = max(1, args.compress_streams)
+    comps = [api.HostCompressor(api.AnchorKVParams(**{**params[0].__dict__}), device=dev) for _ in range(n_cs)]
+    cstreams = [torch.cuda.Stream(dev) for _ in range(n_cs)] if n_cs > 1 else [stream]
+    outs_h = [torch.empty_like(comps[0].host_out).pin_memory() for _ in range(Lr)]
     qdev = torch.empty(1, spec.n_q_heads, spec.head_dim, dtype=params[0].torch_dtype, device=dev)
     odev = torch.empty(1, spec.n_q_heads, spec.head_dim, dtype=torch.float32, device=dev)
     oh = torch.empty(Lr, 1, spec.n_q_heads, spec.head_dim, dtype=torch.float32).pin_memory()
-    layouts = [torch.empty_like(comp.out) for _ in range(Lr)]
+    layouts = [torch.empty_like(comps[0].out) for _ in range(Lr)]
     dws = torch.empty(api.decode_workspace_bytes(params[0], 1), dtype=torch.uint8, device=dev)
 
     def step():
+        # compress: layer l on stream l % n_cs (copies of one layer overlap the
+        # compression of another); decode: sequential over layers
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        for cs in cstreams:
+            cs.wait_event(fork)
         for l in range(Lr):
-            comp(*host[l], layer=l)
-            layouts[l].copy_(comp.out)
-            outs_h[l].copy_(comp.host_out, non_blocking=True)
+            i = l % n_cs
+            with torch.cuda.stream(cstreams[i]):
+                comps[i](*host[l], layer=l, host_out=outs_h[l])
+                layouts[l].copy_(comps[i].out)
+        for cs in cstreams:
+            join = torch.cuda.Event()
+            join.record(cs)
+            stream.wait_event(join)
         for l in range(Lr):
             qdev.copy_(qh[l], non_blocking=True)
             api.decode_attn(params[l], layouts[l], qdev, out=odev, workspace=dws)

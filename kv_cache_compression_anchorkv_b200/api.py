@@ -213,15 +213,20 @@ class HostCompressor:
         self.ws = torch.empty(compress_workspace(p)["total_bytes"], dtype=torch.uint8, device=device)
         self.host_out = torch.empty(L["total_bytes"], dtype=torch.uint8, pin_memory=True)
 
-    def __call__(self, K_host, V_host, Q_host, layer: int | None = None):
+    def __call__(self, K_host, V_host, Q_host, layer: int | None = None, host_out: torch.Tensor | None = None):
+        """Compress one layer; the compressed bytes land in `host_out` (pinned,
+        total_bytes) or in the compressor's own pinned buffer.  Several
+        compressors on different streams overlap the copies of one layer with
+        the compression of another."""
         if layer is not None:
             self.p.layer = layer
         self.K.copy_(K_host, non_blocking=True)
         self.V.copy_(V_host, non_blocking=True)
         self.Q.copy_(Q_host, non_blocking=True)
         compress(self.p, self.K, self.V, self.Q, out=self.out, workspace=self.ws)
-        self.host_out.copy_(self.out, non_blocking=True)
-        return self.host_out
+        dst = self.host_out if host_out is None else host_out
+        dst.copy_(self.out, non_blocking=True)
+        return dst
 
 
 N_STAGES = 15   # ANCHORKV_N_STAGES
