@@ -328,28 +328,37 @@ def run_gpu(args, world, rank, local):
     cstreams = [torch.cuda.Stream(dev) for _ in range(n_cs)] if n_cs > 1 else []
     wss = [ws] + [torch.empty_like(ws) for _ in range(n_cs - 1)]
 
-    def compress_all(single=False):
+    dstream = torch.cuda.Stream(dev) if n_cs > 1 else None
+
+    def step(single=False):
         if single or not cstreams:
             for l in range(Lr):
                 api.compress(params[l], Ks[l], Vs[l], Qs[l], out=outs[l], workspace=ws)
+            for l in range(Lr):
+                api.decode_attn(params[l], outs[l], qd[l], out=dout[l], workspace=dws)
             return
+        # compress layer l on stream l % n_cs; the decode step runs on its own
+        # stream, layer after layer, each layer once its compression is done
         fork = torch.cuda.Event()
         fork.record(stream)
-        for cs in cstreams:
+        for cs in cstreams + [dstream]:
             cs.wait_event(fork)
+        done = []
         for l in range(Lr):
             i = l % n_cs
             with torch.cuda.stream(cstreams[i]):
                 api.compress(params[l], Ks[l], Vs[l], Qs[l], out=outs[l], workspace=wss[i])
-        for cs in cstreams:
+                ev = torch.cuda.Event()
+                ev.record(cstreams[i])
+                done.append(ev)
+        with torch.cuda.stream(dstream):
+            for l in range(Lr):
+                dstream.wait_event(done[l])
+                api.decode_attn(params[l], outs[l], qd[l], out=dout[l], workspace=dws)
+        for cs in cstreams + [dstream]:
             join = torch.cuda.Event()
             join.record(cs)
             stream.wait_event(join)
-
-    def step(single=False):
-        compress_all(single)
-        for l in range(Lr):
-            api.decode_attn(params[l], outs[l], qd[l], out=dout[l], workspace=dws)
 
     def barrier():
         if world > 1:
@@ -465,7 +474,8 @@ def run_e2e(args, spec, theta, params, dev, stream, barrier, world):
     qh = [make_decode_queries(spec, l, 0, 1, device=dev).cpu().pin_memory() for l in range(Lr)]
     n_cs = max(1, args.compress_streams)
     comps = [api.HostCompressor(api.AnchorKVParams(**{**params[0].__dict__}), device=dev) for _ in range(n_cs)]
-    cstreams = [torch.cuda.Stream(dev) for _ in range(n_cs)] if n_cs > 1 else [stream]
+    cstreams = [torch.cuda.Stream(dev) for _ in range(n_cs)]
+    dstream = torch.cuda.Stream(dev)
     outs_h = [torch.empty_like(comps[0].host_out).pin_memory() for _ in range(Lr)]
     qdev = torch.empty(1, spec.n_q_heads, spec.head_dim, dtype=params[0].torch_dtype, device=dev)
     odev = torch.empty(1, spec.n_q_heads, spec.head_dim, dtype=torch.float32, device=dev)
@@ -478,21 +488,27 @@ def run_e2e(args, spec, theta, params, dev, stream, barrier, world):
         # compression of another); decode: sequential over layers
         fork = torch.cuda.Event()
         fork.record(stream)
-        for cs in cstreams:
+        for cs in cstreams + [dstream]:
             cs.wait_event(fork)
+        done = []
         for l in range(Lr):
             i = l % n_cs
             with torch.cuda.stream(cstreams[i]):
                 comps[i](*host[l], layer=l, host_out=outs_h[l])
                 layouts[l].copy_(comps[i].out)
-        for cs in cstreams:
+                ev = torch.cuda.Event()
+                ev.record(cstreams[i])
+                done.append(ev)
+        with torch.cuda.stream(dstream):
+            for l in range(Lr):
+                dstream.wait_event(done[l])
+                qdev.copy_(qh[l], non_blocking=True)
+                api.decode_attn(params[l], layouts[l], qdev, out=odev, workspace=dws)
+                oh[l].copy_(odev, non_blocking=True)
+        for cs in cstreams + [dstream]:
             join = torch.cuda.Event()
             join.record(cs)
             stream.wait_event(join)
-        for l in range(Lr):
-            qdev.copy_(qh[l], non_blocking=True)
-            api.decode_attn(params[l], layouts[l], qdev, out=odev, workspace=dws)
-            oh[l].copy_(odev, non_blocking=True)
 
     steps = max(1, min(args.steps, 3))
     step()

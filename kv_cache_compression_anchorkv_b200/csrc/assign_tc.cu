@@ -301,9 +301,27 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
     const int nblk = a.cw / 16;
     float* inv = winv + (size_t)(warp - 2) * a.kpad;   // this warp's copy of 1/||a||
     int q = 0, cur_u = -1;
+    // this thread's row norm and own-slot flag, one item ahead
+    auto row_info = [&](int it2, float& xn2, int& own2) {
+      xn2 = 0.f;
+      own2 = -1;
+      if (it2 >= end) return;
+      const int u2 = it2 / a.row_tiles, j2 = it2 % a.row_tiles;
+      const int t2 = j2 * 128 + row;
+      if (t2 >= a.N) return;
+      const int side2 = u2 / a.H, h2 = u2 % a.H;
+      xn2 = a.xnorm[((int64_t)side2 * a.H + h2) * a.N + t2];
+      own2 = a.slot_of[(int64_t)h2 * a.N + t2];
+    };
+    float xn_next;
+    int own_next;
+    row_info(beg, xn_next, own_next);
     for (int it = beg; it < end; ++it) {
       const int u = it / a.row_tiles, j = it % a.row_tiles;
       const int side = u / a.H, h = u % a.H;
+      const float xn = xn_next;
+      const int own = own_next;
+      row_info(it + 1, xn_next, own_next);
       if (u != cur_u) {
         __syncwarp();
         const float* src = a.anc_inv + (int64_t)u * a.kp16;
@@ -313,8 +331,6 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
       }
       const int t = j * 128 + row;
       const int64_t f = ((int64_t)side * a.H + h) * a.N + t;
-      const float xn = (t < a.N) ? a.xnorm[f] : 0.f;
-      const int own = (t < a.N) ? a.slot_of[(int64_t)h * a.N + t] : -1;
       const RowKey rk = row_key(xn);
       Keys2 ka{0u, 0u};
       bool ok = true;
@@ -327,10 +343,16 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
         const float* ivc = inv + c * a.cw;
         // keys of one chunk carry bit 8 set; chunk 1's keys get it cleared
         // afterwards, so equal scores prefer chunk 0 (the lower slots)
+        // both column groups run the same code on their own blocks (group g
+        // owns blocks g, g + 2, ...): group 1 starts 16 columns further, which
+        // its keys absorb afterwards (the low 9 bits stay >= 256, no borrow)
         Keys2 ca{0u, 0u}, cb{0u, 0u};
-        if (g == 0) scan_chunk<0>(tbase, ivc, rk.add, kc, nblk, ca, cb);
-        else scan_chunk<1>(tbase, ivc, rk.add, kc, nblk, ca, cb);
+        scan_chunk<0>(tbase + 16u * (uint32_t)g, ivc + 16 * g, rk.add, kc - 16 * g, nblk - g, ca, cb);
         key2_push(ca, cb.b1); key2_push(ca, cb.b2);
+        if (g == 1) {
+          if (ca.b1) ca.b1 -= 16u;
+          if (ca.b2) ca.b2 -= 16u;
+        }
         if (c == 1) {
           if (ca.b1) ca.b1 &= ~256u;
           if (ca.b2) ca.b2 &= ~256u;
