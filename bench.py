@@ -154,6 +154,28 @@ def stage_units(spec, theta, L):
     }
 
 
+def recorded_traffic(stage):
+    """DRAM bytes per launch of `stage` from profiles/traffic.txt, or None when
+    there is no capture or the kernel source changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) < 5 or line.startswith("#") or parts[0] != stage:
+                continue
+            src = os.path.join(ROOT, parts[3])
+            if not os.path.exists(src):
+                return None
+            with open(src, "rb") as g:
+                if hashlib.sha256(g.read()).hexdigest() != parts[4]:
+                    return None
+            return int(parts[2])
+    return None
+
+
 def stage_roofline(stage, units, ms_per_launch, peaks):
     kind, amount, bound = units[stage]
     s = ms_per_launch / 1e3
@@ -410,7 +432,7 @@ def run_gpu(args, world, rank, local):
     per_launch = {st: stages[st][0] / stages[st][1] for st in stages if st in units and stages[st][1]}
     dom = max(per_launch, key=lambda st: stages[st][0])
     roof = stage_roofline(dom, units, per_launch[dom], peaks)
-    roof["traffic"] = None
+    roof["traffic"] = recorded_traffic(dom)
     roof["kernel"] = dom
     roof["peak_source"] = ("measured" if peaks["source"] == "measured" else "fallback") + (
         " (sustained bf16)" if roof["unit"] == "TFLOP/s" else " (copy)")

@@ -94,3 +94,20 @@ def test_workspace_view():
     assert api.decode_workspace_bytes(p, 1) == api.decode_workspace_bytes(p, 16) == 0
     p16 = api.AnchorKVParams(n_tokens=32768, n_q_heads=128)
     assert api.decode_workspace_bytes(p16, 16) > api.decode_workspace_bytes(p16, 1) > 0
+
+
+def test_recorded_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
+    import bench
+    # the committed record matches the committed kernel source
+    assert bench.recorded_traffic("assign") is None or bench.recorded_traffic("assign") > 0
+    assert bench.recorded_traffic("no_such_stage") is None
+    # a record whose hash does not match its source reads as unknown
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "k.cu").write_text("kernel v2\n")
+    (tmp_path / "profiles" / "traffic.txt").write_text("stage_x kern 123 k.cu " + "0" * 64 + " cap.md\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("stage_x") is None
+    import hashlib
+    h = hashlib.sha256(b"kernel v2\n").hexdigest()
+    (tmp_path / "profiles" / "traffic.txt").write_text(f"stage_x kern 123 k.cu {h} cap.md\n")
+    assert bench.recorded_traffic("stage_x") == 123
