@@ -126,16 +126,18 @@ int make_plan(const anchorkv_params* p, Plan* pl) {
   // that the (head, row block, split) items fill the SMs about once
   pl->tc_rb = (pl->GW + 127) / 128;
   {
+    // one CTA per SM (their shared memory allows no more): at most 148 items,
+    // so every item runs in the first wave
     const int units = pl->H * pl->tc_rb, row_tiles = (pl->N + 127) / 128;
-    const int want = std::max(1, (148 + units - 1) / units);
+    const int want = std::max(1, 148 / units);
     pl->tc_tps = std::max(1, (row_tiles + want - 1) / want);
     pl->tc_split = (row_tiles + pl->tc_tps - 1) / pl->tc_tps;
   }
   pl->obs_rb = 1;
   const int64_t H = pl->H, N = pl->N, GW = pl->GW, k = pl->k, D = kD;
   const int64_t n_sh_t = 2 * H * pl->n_tiles;
-  // the tensor-core passes leave two row-block partials per 128-row block
-  const int64_t U = H * pl->tc_rb, nrb = 2 * pl->tc_rb;
+  // the tensor-core passes leave kObsGroups row-block partials per 128-row block
+  const int64_t U = H * pl->tc_rb, nrb = kObsGroups * pl->tc_rb;
   int64_t off = 0;
   auto take = [&](int64_t bytes) { int64_t o = off; off += (bytes + 255) / 256 * 256; return o; };
   pl->o_counters = take(4 * (kCounterCount + 2 * H));
@@ -145,8 +147,8 @@ int make_plan(const anchorkv_params* p, Plan* pl) {
   pl->o_part_m = take(4 * H * pl->n_chunk1 * GW);
   pl->o_part_l = take(4 * H * pl->n_chunk1 * GW);
   pl->o_part_y = take(4 * H * pl->n_chunk1 * GW * D);
-  pl->o_tc_pm2 = take(4 * U * 2 * pl->tc_split * 128);
-  pl->o_tc_pl = take(4 * U * 2 * pl->tc_split * 128);
+  pl->o_tc_pm2 = take(4 * U * kObsGroups * pl->tc_split * 128);
+  pl->o_tc_pl = take(4 * U * kObsGroups * pl->tc_split * 128);
   pl->o_tc_rm2 = take(4 * U * 128);
   pl->o_tc_riz = take(4 * U * 128);
   pl->o_tc_rq2 = take(4 * U * 128);
@@ -277,7 +279,7 @@ int anchorkv_compress(const anchorkv_params* p, const void* K, const void* V, co
 #define AKV_STAGE(st, nk, expr) \
   do { stage_begin(st, s); AKV_LAUNCH(expr); stage_end(st, s, nk); } while (0)
   if (use_tc_obs(pl)) {
-    pl.obs_rb = 2 * pl.tc_rb;
+    pl.obs_rb = kObsGroups * pl.tc_rb;
     AKV_LAUNCH(launch_obs_tc(pl, K, V, Q_obs, w, s));
   } else {
     pl.obs_rb = 1;

@@ -16,6 +16,10 @@ enum Stage {
 void stage_begin(int stage, cudaStream_t s);
 void stage_end(int stage, cudaStream_t s, int kernels);
 
+// Epilogue column groups of the tensor-core observation passes: each leaves
+// its own (max, sum) partials (pass A) or per-token row-block sums (B, C).
+constexpr int kObsGroups = 4;
+
 // Everything one compress call needs to know, derived from the parameters.
 struct Plan {
   anchorkv_params p;

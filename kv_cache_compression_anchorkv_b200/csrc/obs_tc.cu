@@ -19,13 +19,17 @@
 // Row constants are global before passes B and C, so no online rescaling is
 // needed.  All operands are bf16 (K, V, Q exact; alpha and ybar split into
 // two bf16 terms, error 2^-17 relative), accumulators fp32 in TMEM, exp via
-// ex2.approx in the log2 domain.  Warp roles as in the assignment kernel:
-// warp 0 TMA, warp 1 TMEM owner + MMA issuer, warps 2..9 epilogue in two
-// column groups (warps 2..5 and 6..9; one TMEM lane = one row or token per
-// thread, each group half of the accumulator's columns).  Pass A's groups
+// ex2.approx in the log2 domain.  Warp roles: warp 0 TMA, warp 1 TMEM owner
+// + MMA issuer, warps 2..17 epilogue in four column groups of four warps (one
+// TMEM lane = one row or token per thread, each group a quarter of the
+// accumulator's 128 columns, so 32 values per thread and tile and four warps
+// per scheduler to hide the latency of the exp2 chains).  Pass A's groups
 // split the tokens of a tile and leave separate (max, sum) partials; passes B
 // and C's groups split the observation rows, so their per-token sums are
-// written as two row blocks per 128-row block.  Every wait is bounded.
+// written as four row blocks per 128-row block.  Per-row constants are folded
+// into the exp2 argument (log2 of the scale factors), the arithmetic runs on
+// packed fp32 pairs, and the window mask is applied only on the tiles that
+// reach into the window.  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -38,12 +42,13 @@ namespace {
 
 constexpr int kOp = 128 * 256;                 // one [128][128] bf16 operand tile
 constexpr int kHalf = kOp / 2;                 // its 64-column swizzled half
-constexpr int kThr = 320;
-constexpr int kEpi = 256;                      // epilogue threads (8 warps, 2 column groups)
+constexpr int kGroups = kObsGroups;            // epilogue column groups (32 columns each)
+constexpr int kEpi = 128 * kGroups;            // epilogue threads
+constexpr int kThr = 64 + kEpi;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct ObsTc {
-  int N, H, G, W, GW, n_rb, n_split, tps, row_tiles;   // part_m2/part_l hold 2 * n_split partials per unit
+  int N, H, G, W, GW, n_rb, n_split, tps, row_tiles;   // part_m2/part_l hold kGroups * n_split partials per unit
   float c2;                                     // log2(e) / sqrt(D)
   float* part_m2;                               // [U][n_split][128]
   float* part_l;
@@ -51,7 +56,7 @@ struct ObsTc {
   const float* row_iz;
   const float* row_q2;
   const float* row_y2;
-  float* score;                                 // [2 n_rb][H][N] (row block rb, column group g at 2 rb + g)
+  float* score;                                 // [kGroups n_rb][H][N] (row block rb, group g at kGroups rb + g)
   float* a2s;
   float* kus;
   float* part_y;                                // [U][n_split][128 rows][128 d]
@@ -88,26 +93,15 @@ __device__ __forceinline__ void load_op(unsigned char* dst, const CUtensorMap* m
   tc::tma_load_2d(dst + kHalf, m, 64, row, bar);
 }
 
-__device__ __forceinline__ void ld128(uint32_t taddr, uint32_t (&v)[8][16]) {
+__device__ __forceinline__ void ld32(uint32_t taddr, uint32_t (&v)[2][16]) {
   tc::tmem_ld16(taddr + 0, v[0]);
   tc::tmem_ld16(taddr + 16, v[1]);
-  tc::tmem_ld16(taddr + 32, v[2]);
-  tc::tmem_ld16(taddr + 48, v[3]);
-  tc::tmem_wait_ld_dep4(v[0], v[1], v[2], v[3]);
-  tc::tmem_ld16(taddr + 64, v[4]);
-  tc::tmem_ld16(taddr + 80, v[5]);
-  tc::tmem_ld16(taddr + 96, v[6]);
-  tc::tmem_ld16(taddr + 112, v[7]);
-  tc::tmem_wait_ld_dep4(v[4], v[5], v[6], v[7]);
+  tc::tmem_wait_ld_dep2(v[0], v[1]);
 }
 
-__device__ __forceinline__ void ld64(uint32_t taddr, uint32_t (&v)[4][16]) {
-  tc::tmem_ld16(taddr + 0, v[0]);
-  tc::tmem_ld16(taddr + 16, v[1]);
-  tc::tmem_ld16(taddr + 32, v[2]);
-  tc::tmem_ld16(taddr + 48, v[3]);
-  tc::tmem_wait_ld_dep4(v[0], v[1], v[2], v[3]);
-}
+__device__ __forceinline__ float2 f2(uint32_t x, uint32_t y) { return make_float2(__uint_as_float(x), __uint_as_float(y)); }
+__device__ __forceinline__ float2 ex2x2(float2 x) { return make_float2(tc::ex2_approx(x.x), tc::ex2_approx(x.y)); }
+constexpr uint32_t kNegInf = 0xFF800000u;
 
 template <typename U>
 __device__ __forceinline__ float* align16f(U* p) {
@@ -118,28 +112,25 @@ __device__ __forceinline__ unsigned char* aligned_base(unsigned char* raw) {
   return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~static_cast<uintptr_t>(1023));
 }
 
-// Sum of squares of one token row of a swizzled [128][128] bf16 tile.  The
-// chunk order inside the row does not matter for a norm, so row r reads its
-// 16-byte chunks in the order c ^ (r & 7): the 8 rows of a quarter-warp then
-// hit 8 different bank groups.
-__device__ __forceinline__ float row_sumsq(const unsigned char* tile, int r) {
-  float s = 0.f;
+// Sum of squares of the 64 columns of half `part` of token row r of a
+// swizzled [128][128] bf16 tile.  The chunk order inside the row does not
+// matter for a norm, so the row reads its 16-byte chunks in the order
+// c ^ (r & 7) ^ 4 part: the quarter-warp (4 rows x 2 halves, the rows 4-aligned)
+// then hits 8 different bank groups.
+__device__ __forceinline__ float half_sumsq(const unsigned char* tile, int r, int part) {
+  float2 s = make_float2(0.f, 0.f);
+  const uint4* p = reinterpret_cast<const uint4*>(tile + part * kHalf + r * 128);
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const uint4* p = reinterpret_cast<const uint4*>(tile + half * kHalf + r * 128);
+  for (int c = 0; c < 8; ++c) {
+    const uint4 q = p[c ^ (r & 7) ^ (part << 2)];
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const uint4 q = p[c ^ (r & 7)];
-      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
-        s = fmaf(lo, lo, s);
-        s = fmaf(hi, hi, s);
-      }
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = f2(w[e] << 16, w[e] & 0xFFFF0000u);
+      s = __ffma2_rn(x, x, s);
     }
   }
-  return s;
+  return s.x + s.y;
 }
 
 // ============================================================== pass A
@@ -208,44 +199,43 @@ obs_a_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
       tc::mbar_wait(&ctl.drain, 0);
     }
   } else {
-    // group g takes tokens 64 g .. 64 g + 63 of every tile
+    // group g takes tokens 32 g .. 32 g + 31 of every tile
     const int qd = warp & 3, g = (warp - 2) >> 2, r = qd * 32 + lane;
     const int lim = row_limit(a, it.rb * 128 + r);
+    const float2 cc = make_float2(a.c2, a.c2);
     float m = -INFINITY, l = 0.f;
     for (int i = 0; i < it.n; ++i) {
       const int b = i & 1, ub = i >> 1;
       if (!tc::wait_or_fail(&ctl.acc_full[b], ub & 1, &ctl.err, a.counters, kDevErrTimeout)) break;
       tc::fence_after_sync();
-      uint32_t v[4][16];
-      ld64(tmem + ((uint32_t)(qd * 32) << 16) + b * 128 + g * 64, v);
+      uint32_t v[2][16];
+      ld32(tmem + ((uint32_t)(qd * 32) << 16) + b * 128 + g * 32, v);
       tc::fence_before_sync();
       tc::mbar_arrive(&ctl.acc_empty[b]);
-      const int t0 = (it.tile0 + i) * 128 + g * 64;
+      const int t0 = (it.tile0 + i) * 128 + g * 32;
       if (lim < t0) continue;                       // nothing visible (or padding row)
-      const bool full = t0 + 63 <= lim;
-      float mx = -INFINITY;
+      if (t0 + 31 > lim) {                          // the window's edge: hidden scores -> -inf
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+        for (int e = 0; e < 32; ++e)
+          if (t0 + e > lim) v[e >> 4][e & 15] = kNegInf;
+      }
+      // the maximum of the raw scores (c2 > 0 commutes with it)
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float y = __uint_as_float(v[c][e]) * a.c2;
-          v[c][e] = __float_as_uint(y);
-          if (full || t0 + c * 16 + e <= lim) mx = fmaxf(mx, y);
-        }
-      const float mn = fmaxf(m, mx);
-      float sum0 = 0.f, sum1 = 0.f;
+      for (int e = 0; e < 32; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(v[e >> 4][e & 15]));
+      const float mn = fmaxf(m, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * a.c2);
+      const float2 nm = make_float2(-mn, -mn);
+      float2 sum0 = make_float2(0.f, 0.f), sum1 = sum0;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p = tc::ex2_approx(__uint_as_float(v[c][e]) - mn);
-          const float q = (full || t0 + c * 16 + e <= lim) ? p : 0.f;
-          if (e & 1) sum1 += q; else sum0 += q;
-        }
-      l = l * tc::ex2_approx(m - mn) + (sum0 + sum1);
+      for (int e = 0; e < 32; e += 4) {
+        const uint32_t* w = &v[e >> 4][e & 15];
+        sum0 = __fadd2_rn(sum0, ex2x2(__ffma2_rn(f2(w[0], w[1]), cc, nm)));
+        sum1 = __fadd2_rn(sum1, ex2x2(__ffma2_rn(f2(w[2], w[3]), cc, nm)));
+      }
+      l = l * tc::ex2_approx(m - mn) + ((sum0.x + sum0.y) + (sum1.x + sum1.y));
       m = mn;
     }
-    const int64_t pi = ((int64_t)it.u * 2 * a.n_split + 2 * it.s + g) * 128 + r;
+    const int64_t pi = ((int64_t)it.u * kGroups * a.n_split + kGroups * it.s + g) * 128 + r;
     a.part_m2[pi] = m;
     a.part_l[pi] = l;
   }
@@ -254,32 +244,39 @@ obs_a_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
   if (warp == 1) { tc::fence_after_sync(); tc::tmem_dealloc(tmem, 256); }
 }
 
-// Row constants: M_r (log2 domain), 1/Z_r and ||q_r||^2; one thread per row.
-__global__ void obs_rows_kernel(const __nv_bfloat16* __restrict__ Q, ObsTc a, float* __restrict__ row_m2,
-                                float* __restrict__ row_iz, float* __restrict__ row_q2) {
-  const int u = blockIdx.x, r = threadIdx.x;
+// Row constants: M_r (log2 domain), 1/Z_r and ||q_r||^2.  grid (U, 16),
+// 256 threads: one warp per row, the lanes striding over the row's pass-A
+// partials (merged in a fixed order: lane-strided, then a fixed butterfly)
+// and over its 128 query coordinates.
+__global__ void __launch_bounds__(256) obs_rows_kernel(const __nv_bfloat16* __restrict__ Q, ObsTc a,
+                                                       float* __restrict__ row_m2, float* __restrict__ row_iz,
+                                                       float* __restrict__ row_q2) {
+  const int u = blockIdx.x, lane = threadIdx.x & 31, r = blockIdx.y * 8 + (threadIdx.x >> 5);
   const int h = u / a.n_rb, rb = u % a.n_rb, rr = rb * 128 + r;
-  const int np = 2 * a.n_split;
+  const int np = kGroups * a.n_split;
   float M = -INFINITY;
-  for (int s = 0; s < np; ++s) M = fmaxf(M, a.part_m2[((int64_t)u * np + s) * 128 + r]);
+  for (int s = lane; s < np; s += 32) M = fmaxf(M, a.part_m2[((int64_t)u * np + s) * 128 + r]);
+  M = warp_max(M);
   float Z = 0.f;
-  for (int s = 0; s < np; ++s) {
+  for (int s = lane; s < np; s += 32) {
     const int64_t pi = ((int64_t)u * np + s) * 128 + r;
     if (a.part_m2[pi] > -INFINITY) Z = fmaf(a.part_l[pi], exp2f(a.part_m2[pi] - M), Z);
   }
+  Z = warp_sum(Z);
   float q2 = 0.f;
   if (rr < a.GW) {
-    const __nv_bfloat16* qr = Q + ((int64_t)h * a.GW + rr) * kD;
-    for (int d = 0; d < kD; ++d) {
-      const float x = __bfloat162float(qr[d]);
-      q2 = fmaf(x, x, q2);
-    }
+    float f[4];
+    load4<__nv_bfloat16>(Q + ((int64_t)h * a.GW + rr) * kD + lane * 4, f);
+    q2 = f[0] * f[0] + f[1] * f[1] + f[2] * f[2] + f[3] * f[3];
   }
-  const int64_t o = (int64_t)u * 128 + r;
-  const bool live = rr < a.GW && Z > 0.f;
-  row_m2[o] = live ? M : 0.f;
-  row_iz[o] = live ? 1.f / Z : 0.f;
-  row_q2[o] = q2;
+  q2 = warp_sum(q2);
+  if (lane == 0) {
+    const int64_t o = (int64_t)u * 128 + r;
+    const bool live = rr < a.GW && Z > 0.f;
+    row_m2[o] = live ? M : 0.f;
+    row_iz[o] = live ? 1.f / Z : 0.f;
+    row_q2[o] = q2;
+  }
 }
 
 // ============================================================== pass B
@@ -299,9 +296,8 @@ obs_b_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
   unsigned char* xs = q + kOp;                   // stage s: K at xs + 2s kOp, V at + kOp
   unsigned char* al = xs + S * 2 * kOp;          // alpha hi at al, lo at al + kOp (MN-major)
   CtlB& ctl = *reinterpret_cast<CtlB*>(al + 2 * kOp);
-  float* cm2 = align16f(&ctl + 1);               // 16-byte aligned for float4 reads
-  float* ciz = cm2 + 128;
-  int* clim = reinterpret_cast<int*>(ciz + 128);
+  float* cb = align16f(&ctl + 1);                // log2(1/Z_r) - M_r, 16-byte aligned for float4 reads
+  int* clim = reinterpret_cast<int*>(cb + 128);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Item it = item_of(a);
   if (threadIdx.x == 0) {
@@ -317,9 +313,9 @@ obs_b_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
   }
   if (warp == 1) { tc::tmem_alloc(&ctl.tmem_base, 512); tc::tmem_relinquish(); }
   if (threadIdx.x >= 64 && threadIdx.x < 64 + 128) {
+    // alpha = 2^(s c2 - M_r) / Z_r = 2^(s c2 + cb_r); padding rows (1/Z = 0) get -inf
     const int r = threadIdx.x - 64;
-    cm2[r] = a.row_m2[(int64_t)it.u * 128 + r];
-    ciz[r] = a.row_iz[(int64_t)it.u * 128 + r];
+    cb[r] = log2f(a.row_iz[(int64_t)it.u * 128 + r]) - a.row_m2[(int64_t)it.u * 128 + r];
     clim[r] = row_limit(a, it.rb * 128 + r);
   }
   tc::fence_before_sync();
@@ -382,88 +378,93 @@ obs_b_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
       tc::mbar_wait(&ctl.drain, 0);
     }
   } else {
-    // group g takes observation rows 64 g .. 64 g + 63 of every token
+    // group g takes observation rows 32 g .. 32 g + 31 of every token
     const int qd = warp & 3, g = (warp - 2) >> 2, tl = qd * 32 + lane;
-    const int rb2 = 2 * it.rb + g;
+    const int rb4 = kGroups * it.rb + g;
+    // norm work: epilogue thread e takes half (e & 1) of row (e >> 1) & 127 of
+    // the K (e < 256) or V tile
+    const int ne = threadIdx.x - 64, nrow = (ne >> 1) & 127, nside = ne >> 8, npart = ne & 1;
+    const float2 cc = make_float2(a.c2, a.c2);
     bool ok = true;
     for (int i = 0; i < it.n; ++i) {
       const int b = i & 1, ub = i >> 1, s = i % S;
       if (!tc::wait_or_fail(&ctl.s_full[b], ub & 1, &ctl.err, a.counters, kDevErrTimeout)) { ok = false; break; }
       tc::fence_after_sync();
-      uint32_t v[4][16];
-      ld64(tmem + ((uint32_t)(qd * 32) << 16) + b * 128 + g * 64, v);
+      uint32_t v[2][16];
+      ld32(tmem + ((uint32_t)(qd * 32) << 16) + b * 128 + g * 32, v);
       tc::fence_before_sync();
       tc::mbar_arrive(&ctl.s_empty[b]);
       const int t = (it.tile0 + i) * 128 + tl;
-      float sc = 0.f, a2 = 0.f;
+      if ((it.tile0 + i) * 128 + 127 > a.N - a.W) {   // the window's edge: hidden scores -> -inf
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-#pragma unroll
-        for (int e4 = 0; e4 < 16; e4 += 4) {
-          const int r0 = g * 64 + c * 16 + e4;
-          const float4 m4 = *reinterpret_cast<const float4*>(&cm2[r0]);
-          const float4 z4 = *reinterpret_cast<const float4*>(&ciz[r0]);
-          const int4 l4 = *reinterpret_cast<const int4*>(&clim[r0]);
-          const float mm[4] = {m4.x, m4.y, m4.z, m4.w}, zz[4] = {z4.x, z4.y, z4.z, z4.w};
-          const int ll[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float al_ = tc::ex2_approx(fmaf(__uint_as_float(v[c][e4 + q]), a.c2, -mm[q])) * zz[q];
-            al_ = (t <= ll[q]) ? al_ : 0.f;
-            v[c][e4 + q] = __float_as_uint(al_);
-            sc += al_;
-            a2 = fmaf(al_, al_, a2);
-          }
-        }
+        for (int e = 0; e < 32; ++e)
+          if (t > clim[g * 32 + e]) v[e >> 4][e & 15] = kNegInf;
       }
-      if (it.rb == 0 && t < a.N) {
-        const unsigned char* xt = xs + 2 * s * kOp + g * kOp;    // group 0: K, group 1: V
-        a.xnorm[((int64_t)g * a.H + it.h) * a.N + t] = sqrtf(row_sumsq(xt, tl));
+      float2 sc0 = make_float2(0.f, 0.f), sc1 = sc0, aa0 = sc0, aa1 = sc0;
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const float4 b4 = *reinterpret_cast<const float4*>(&cb[g * 32 + e]);
+        uint32_t* w = &v[e >> 4][e & 15];
+        const float2 al0 = ex2x2(__ffma2_rn(f2(w[0], w[1]), cc, make_float2(b4.x, b4.y)));
+        const float2 al1 = ex2x2(__ffma2_rn(f2(w[2], w[3]), cc, make_float2(b4.z, b4.w)));
+        w[0] = __float_as_uint(al0.x); w[1] = __float_as_uint(al0.y);
+        w[2] = __float_as_uint(al1.x); w[3] = __float_as_uint(al1.y);
+        sc0 = __fadd2_rn(sc0, al0);
+        sc1 = __fadd2_rn(sc1, al1);
+        aa0 = __ffma2_rn(al0, al0, aa0);
+        aa1 = __ffma2_rn(al1, al1, aa1);
+      }
+      if (it.rb == 0) {
+        float ss = half_sumsq(xs + (2 * s + nside) * kOp, nrow, npart);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        const int tn = (it.tile0 + i) * 128 + nrow;
+        if (npart == 0 && tn < a.N) a.xnorm[((int64_t)nside * a.H + it.h) * a.N + tn] = sqrtf(ss);
       }
       if (i > 0 && !tc::wait_or_fail(&ctl.al_empty, (i - 1) & 1, &ctl.err, a.counters, kDevErrTimeout)) {
         ok = false;
         break;
       }
       // alpha[t][r] as bf16 hi + lo, MN-major (r contiguous), 128-byte
-      // swizzle; this group's rows are the 64-row half g of the tile
+      // swizzle; this group's rows are chunks 4 (g & 1) .. + 3 of half g / 2
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int ch = 0; ch < 4; ++ch) {
         uint32_t hw[4], lw[4];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-          const int r = ch * 8 + 2 * p;                 // within the group's 64 rows
-          const float x0 = __uint_as_float(v[r >> 4][r & 15]), x1 = __uint_as_float(v[(r + 1) >> 4][(r + 1) & 15]);
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(x0, x1);
-          const float2 hf = __bfloat1622float2(h2);
-          const __nv_bfloat162 l2 = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+          const int r = ch * 8 + 2 * p;                 // within the group's 32 rows
+          const float2 x = f2(v[r >> 4][r & 15], v[r >> 4][(r & 15) + 1]);
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(x.x, x.y);
+          const float2 lo = __fadd2_rn(x, make_float2(-__low2float(h2), -__high2float(h2)));
+          const __nv_bfloat162 l2 = __floats2bfloat162_rn(lo.x, lo.y);
           hw[p] = *reinterpret_cast<const uint32_t*>(&h2);
           lw[p] = *reinterpret_cast<const uint32_t*>(&l2);
         }
-        const int off = g * kHalf + tl * 128 + ((ch ^ (tl & 7)) << 4);
+        const int cg = ((g & 1) << 2) + ch;
+        const int off = (g >> 1) * kHalf + tl * 128 + ((cg ^ (tl & 7)) << 4);
         *reinterpret_cast<uint4*>(al + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
         *reinterpret_cast<uint4*>(al + kOp + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&ctl.al_full);
       if (t < a.N) {
-        const int64_t o = ((int64_t)rb2 * a.H + it.h) * a.N + t;
-        a.score[o] = sc;
-        a.a2s[o] = a2;
+        const int64_t o = ((int64_t)rb4 * a.H + it.h) * a.N + t;
+        a.score[o] = (sc0.x + sc0.y) + (sc1.x + sc1.y);
+        a.a2s[o] = (aa0.x + aa0.y) + (aa1.x + aa1.y);
       }
     }
-    // partial ybar^T: TMEM lane = d, column = row r (this group's 64 rows)
+    // partial ybar^T: TMEM lane = d, column = row r (this group's 32 rows)
     float* py = a.part_y + ((int64_t)it.u * a.n_split + it.s) * 128 * 128;
     if (ok && it.n > 0 && tc::wait_or_fail(&ctl.y_full, 0, &ctl.err, a.counters, kDevErrTimeout)) {
       tc::fence_after_sync();
-      uint32_t v[4][16];
-      ld64(tmem + ((uint32_t)(qd * 32) << 16) + ycol + g * 64, v);
+      uint32_t v[2][16];
+      ld32(tmem + ((uint32_t)(qd * 32) << 16) + ycol + g * 32, v);
       const int d = tl;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int e = 0; e < 16; ++e) py[(g * 64 + c * 16 + e) * 128 + d] = __uint_as_float(v[c][e]);
+        for (int e = 0; e < 16; ++e) py[(g * 32 + c * 16 + e) * 128 + d] = __uint_as_float(v[c][e]);
     } else if (it.n == 0) {
-      for (int r = g * 64; r < g * 64 + 64; ++r) py[r * 128 + tl] = 0.f;
+      for (int r = g * 32; r < g * 32 + 32; ++r) py[r * 128 + tl] = 0.f;
     }
   }
   tc::fence_before_sync();
@@ -520,9 +521,10 @@ obs_c_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
   unsigned char* yl = yh + kOp;
   unsigned char* xs = yl + kOp;                  // stage s: K at xs + 2s kOp, V at + kOp
   CtlC& ctl = *reinterpret_cast<CtlC*>(xs + S * 2 * kOp);
-  float* cm2 = align16f(&ctl + 1);               // 16-byte aligned for float4 reads
-  float* ciq = cm2 + 128;                       // ||q_r||^2 / Z_r^2
-  float* cy2 = ciq + 128;
+  // per row pair (r, r + 1): {cw_r, cw_r+1, ||ybar_r||^2, ||ybar_r+1||^2}, where
+  // alpha_r^2 ||q_r||^2 = 2^(2 s c2 + cw_r); 16-byte aligned for float4 reads
+  float* cpk = align16f(&ctl + 1);
+  int* clim = reinterpret_cast<int*>(cpk + 256);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Item it = item_of(a);
   if (threadIdx.x == 0) {
@@ -535,11 +537,12 @@ obs_c_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
   }
   if (warp == 1) { tc::tmem_alloc(&ctl.tmem_base, 512); tc::tmem_relinquish(); }
   if (threadIdx.x >= 64 && threadIdx.x < 64 + 128) {
+    // cw_r = 2 log2(1/Z_r) + log2 ||q_r||^2 - 2 M_r (-inf for padding rows)
     const int r = threadIdx.x - 64;
     const int64_t o = (int64_t)it.u * 128 + r;
-    cm2[r] = a.row_m2[o];
-    ciq[r] = a.row_iz[o] * a.row_iz[o] * a.row_q2[o];
-    cy2[r] = a.row_y2[o];
+    cpk[(r >> 1) * 4 + (r & 1)] = 2.f * log2f(a.row_iz[o]) + log2f(a.row_q2[o]) - 2.f * a.row_m2[o];
+    cpk[(r >> 1) * 4 + 2 + (r & 1)] = a.row_y2[o];
+    clim[r] = row_limit(a, it.rb * 128 + r);
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -590,10 +593,11 @@ obs_c_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
       tc::mbar_wait(&ctl.drain, 0);
     }
   } else {
-    // group g takes observation rows 64 g .. 64 g + 63 of every token
+    // group g takes observation rows 32 g .. 32 g + 31 of every token
     const int qd = warp & 3, g = (warp - 2) >> 2, tl = qd * 32 + lane;
-    const int rb2 = 2 * it.rb + g;
-    const float c2x2 = 2.f * a.c2;
+    const int rb4 = kGroups * it.rb + g;
+    const float2 cc = make_float2(2.f * a.c2, 2.f * a.c2), m2 = make_float2(-2.f, -2.f);
+    const float4* pk = reinterpret_cast<const float4*>(cpk) + g * 16;
     // ||V_t||^2 of this thread's token, one tile ahead
     auto vnorm2 = [&](int i) -> float {
       const int t = (it.tile0 + i) * 128 + tl;
@@ -607,43 +611,40 @@ obs_c_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
       v2n = vnorm2(i + 1);
       if (!tc::wait_or_fail(&ctl.acc_full[b], ub & 1, &ctl.err, a.counters, kDevErrTimeout)) break;
       tc::fence_after_sync();
+      const uint32_t base = tmem + ((uint32_t)(qd * 32) << 16) + b * 256 + g * 32;
       const int t = (it.tile0 + i) * 128 + tl;
-      const uint32_t base = tmem + ((uint32_t)(qd * 32) << 16) + b * 256 + g * 64;
-      // every live row sees the whole tile unless it reaches into the window
-      const bool full = (it.tile0 + i) * 128 + 127 <= a.N - a.W;
-      float ku0 = 0.f, ku1 = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t s0[16], s1[16], y0[16], y1[16];
-        tc::tmem_ld16(base + c * 32, s0);
-        tc::tmem_ld16(base + c * 32 + 16, s1);
-        tc::tmem_ld16(base + 128 + c * 32, y0);
-        tc::tmem_ld16(base + 128 + c * 32 + 16, y1);
-        tc::tmem_wait_ld_dep4(s0, s1, y0, y1);
+      const bool edge = (it.tile0 + i) * 128 + 127 > a.N - a.W;
+      // sum_r w_r (||V_t||^2 - 2 V_t.ybar_r + ||ybar_r||^2), w_r = alpha_r^2 ||q_r||^2,
+      // in two rounds of 16 rows (the accumulator is released after the second load)
+      const float2 vv = make_float2(v2, v2);
+      float2 ku0 = make_float2(0.f, 0.f), ku1 = ku0;
 #pragma unroll
-        for (int e4 = 0; e4 < 32; e4 += 4) {
-          const int r0 = g * 64 + c * 32 + e4;
-          const float4 m4 = *reinterpret_cast<const float4*>(&cm2[r0]);
-          const float4 q4 = *reinterpret_cast<const float4*>(&ciq[r0]);
-          const float4 y4 = *reinterpret_cast<const float4*>(&cy2[r0]);
-          const float mm[4] = {m4.x, m4.y, m4.z, m4.w}, qq[4] = {q4.x, q4.y, q4.z, q4.w};
-          const float yy[4] = {y4.x, y4.y, y4.z, y4.w};
+      for (int hr = 0; hr < 2; ++hr) {
+        uint32_t sv[16], vy[16];
+        tc::tmem_ld16(base + hr * 16, sv);
+        tc::tmem_ld16(base + 128 + hr * 16, vy);
+        tc::tmem_wait_ld_dep2(sv, vy);
+        if (hr == 1) {
+          tc::fence_before_sync();
+          tc::mbar_arrive(&ctl.acc_empty[b]);
+        }
+        if (edge) {                                    // the window's edge: hidden scores -> -inf
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int e = e4 + q;
-            const float sv = __uint_as_float(e < 16 ? s0[e] : s1[e - 16]);
-            const float vy = __uint_as_float(e < 16 ? y0[e] : y1[e - 16]);
-            // alpha^2 ||q||^2 = 2^(2 (s c2 - M2)) ||q||^2 / Z^2
-            float w = tc::ex2_approx(fmaf(sv, c2x2, -2.f * mm[q])) * qq[q];
-            if (!full && t > row_limit(a, it.rb * 128 + r0 + q)) w = 0.f;
-            const float dist = fmaf(-2.f, vy, v2 + yy[q]);
-            if (q & 1) ku1 = fmaf(w, dist, ku1); else ku0 = fmaf(w, dist, ku0);
-          }
+          for (int e = 0; e < 16; ++e)
+            if (t > clim[g * 32 + hr * 16 + e]) sv[e] = kNegInf;
+        }
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const float4 p0 = pk[hr * 8 + (e >> 1)], p1 = pk[hr * 8 + (e >> 1) + 1];
+          const float2 w0 = ex2x2(__ffma2_rn(f2(sv[e], sv[e + 1]), cc, make_float2(p0.x, p0.y)));
+          const float2 w1 = ex2x2(__ffma2_rn(f2(sv[e + 2], sv[e + 3]), cc, make_float2(p1.x, p1.y)));
+          const float2 d0 = __ffma2_rn(f2(vy[e], vy[e + 1]), m2, __fadd2_rn(vv, make_float2(p0.z, p0.w)));
+          const float2 d1 = __ffma2_rn(f2(vy[e + 2], vy[e + 3]), m2, __fadd2_rn(vv, make_float2(p1.z, p1.w)));
+          ku0 = __ffma2_rn(w0, d0, ku0);
+          ku1 = __ffma2_rn(w1, d1, ku1);
         }
       }
-      tc::fence_before_sync();
-      tc::mbar_arrive(&ctl.acc_empty[b]);
-      if (t < a.N) a.kus[((int64_t)rb2 * a.H + it.h) * a.N + t] = ku0 + ku1;
+      if (t < a.N) a.kus[((int64_t)rb4 * a.H + it.h) * a.N + t] = (ku0.x + ku0.y) + (ku1.x + ku1.y);
     }
   }
   tc::fence_before_sync();
@@ -676,7 +677,7 @@ bool map128(CUtensorMap* m, const void* base, int64_t rows) {
 }
 
 constexpr int kSmemA = 1024 + kOp + 4 * kOp + (int)sizeof(CtlA) + 64;
-constexpr int kSmemB = 1024 + kOp + 4 * kOp + 2 * kOp + (int)sizeof(CtlB) + 3 * 128 * 4 + 64;
+constexpr int kSmemB = 1024 + kOp + 4 * kOp + 2 * kOp + (int)sizeof(CtlB) + 2 * 128 * 4 + 64;
 constexpr int kSmemC = 1024 + 3 * kOp + 4 * kOp + (int)sizeof(CtlC) + 3 * 128 * 4 + 64;
 static_assert(kSmemB <= 227 * 1024 && kSmemC <= 227 * 1024, "shared memory budget");
 
@@ -719,7 +720,7 @@ cudaError_t launch_obs_tc(const Plan& pl, const void* K, const void* V, const vo
   cudaFuncSetAttribute(obs_c_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemC);
   stage_begin(kStObsPass1, s);
   obs_a_kernel<<<items, kThr, kSmemA, s>>>(mQ, mK, a);
-  obs_rows_kernel<<<U, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(Q), a,
+  obs_rows_kernel<<<dim3(U, 16), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(Q), a,
                                    reinterpret_cast<float*>(ws + pl.o_tc_rm2), reinterpret_cast<float*>(ws + pl.o_tc_riz),
                                    reinterpret_cast<float*>(ws + pl.o_tc_rq2));
   stage_end(kStObsPass1, s, 2);
