@@ -6,19 +6,23 @@
 // lowest slot, a zero anchor scores 0, an anchor token keeps its own slot.
 //
 // The contraction S = X A^T (X: 128 token rows, A: all k anchors of the
-// KV head and side, D = 128) runs as tcgen05.mma (M = 128, N = chunk of
-// anchors, K = 16 per instruction) from 128-byte-swizzled shared-memory
-// tiles that TMA fills; accumulators live in TMEM.  The epilogue never
-// writes S: eight warps read their TMEM lanes, scale each column by
-// 1/||a_s|| and keep the best and second-best score per row; the two column
-// halves are merged through shared memory.  Rows whose fp32 margin between
-// best and second best is not above the accumulation error bound are listed
-// for the fp64 re-decision shared with the SIMT path.
+// KV head and side, D = 128) runs as tcgen05.mma (M = 128, N = chunk of at
+// most 128 anchors, K = 16 per instruction) from 128-byte-swizzled
+// shared-memory tiles that TMA fills; accumulators live in a ring of TMEM
+// chunk buffers (as many as fit in 512 columns).  The epilogue never writes
+// S: each thread reads its TMEM lane, scales each column by 1/||a_s|| and
+// keeps the best and second-best score of its row over all chunks.  Rows
+// whose fp32 margin between best and second best is not above the
+// accumulation error bound are listed for the fp64 re-decision shared with
+// the SIMT path.
 //
 // Warp roles (320 threads, one CTA per SM, persistent over (side, head,
 // 128-row tile) work items): warp 0 issues TMA, warp 1 owns TMEM and issues
-// MMAs, warps 2..9 run the epilogue.  Anchors of the current (side, head)
-// stay resident in shared memory; token tiles stream through a ring.
+// MMAs, warps 2..9 run the epilogue as two groups of four warps that take
+// alternate items whole (every column of their 128 rows), so the groups
+// never wait on each other and need no merge.  Anchors of the current
+// (side, head) stay resident in shared memory; token tiles stream through a
+// ring.
 // Every mbarrier wait is bounded: on timeout the kernel latches an error,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include <cudaTypedefs.h>
@@ -42,10 +46,11 @@ namespace {
 constexpr int kThreads = 320;
 constexpr int kXStageBytes = 128 * 256;       // 128 rows x 128 bf16
 constexpr int kMaxKpad = 448;
-constexpr int kAccCols = 256;                 // columns per accumulator buffer
+constexpr int kChunkMax = 128;                // anchors per MMA chunk (accumulator columns)
+constexpr int kMaxBuf = 8;                    // accumulator buffers in the TMEM ring
 
 struct TcArgs {
-  int N, H, k, kp16, cw, n_chunks, kpad, stages, row_tiles;
+  int N, H, k, kp16, cw, n_chunks, kpad, stages, row_tiles, nbuf;
   int total_items;
   const float* anc_inv;
   const int* slot_of;
@@ -56,7 +61,7 @@ struct TcArgs {
 };
 
 // Best two packed keys of a row (see the epilogue).  Keys of distinct slots
-// never compare equal, so the max/min updates keep them ordered.
+// never compare equal, so the max/min updates keep them ordered; 0 = none.
 struct Keys2 {
   uint32_t b1, b2;
 };
@@ -67,11 +72,8 @@ __device__ __forceinline__ void key2_push(Keys2& s, uint32_t key) {
   s.b1 = n1; s.b2 = n2;
 }
 
-// Slot of a key: the low 9 bits hold (1 - chunk) << 8 | (255 - column in chunk).
-__device__ __forceinline__ uint32_t key_slot(uint32_t key, int cw) {
-  const uint32_t bits = key & 511u;
-  return ((bits & 256u) ? 0u : (uint32_t)cw) + (255u - (bits & 255u));
-}
+// Slot of a key: the low 9 bits hold 511 - slot.
+__device__ __forceinline__ uint32_t key_slot(uint32_t key) { return 511u - (key & 511u); }
 
 // Per-row constants of the key: C = 2^(floor(log2 ||x||) + 9) makes
 // fmaf(acc, 1/||a||, ||x||(1 + 2^-7) + C) land in [C, 2C), i.e. rounded to a
@@ -91,11 +93,11 @@ __device__ __forceinline__ RowKey row_key(float xn) {
   return r;
 }
 
-// One chunk's columns for the warps of column group G (16-column blocks
-// G, G+2, ..., at most 7 of them since a chunk has at most 224 columns).  The
-// block and column indices are compile-time after unrolling, so a key costs
-// one FFMA and one LOP3 with an immediate, and the best-two update three
-// FMNMX.  Up to four TMEM loads are in flight per wait.
+// One 16-column block of a chunk (block BLK, columns 16 BLK ..): the block
+// and column indices are compile-time after unrolling, so a key costs one
+// FFMA and one shift-add, and the best-two update three integer min/max.
+// Keys carry 511 - (column in chunk); the chunk offset is applied to the
+// chunk's best two afterwards.
 template <int BLK>
 __device__ __forceinline__ void scan_block(const uint32_t (&w)[16], const float* ivc, float bias, int kc, Keys2& ka,
                                            Keys2& kb) {
@@ -123,37 +125,42 @@ __device__ __forceinline__ void scan_block(const uint32_t (&w)[16], const float*
   }
 }
 
-// Blocks G + 2J and G + 2(J+1): two TMEM loads in flight, then recurse.
-template <int G, int J>
-__device__ __forceinline__ void scan_from(uint32_t tbase, const float* ivc, float bias, int kc, int nblk, Keys2& ka,
-                                          Keys2& kb) {
-  if constexpr (J < 7) {
-    constexpr int B0 = G + 2 * J, B1 = G + 2 * (J + 1);
-    if (!(B0 < nblk && B0 * 16 < kc)) return;
-    const bool h1 = (J + 1 < 7) && B1 < nblk && B1 * 16 < kc;
-    uint32_t v0[16], v1[16];
-    tc::tmem_ld16(tbase + (uint32_t)(B0 * 16), v0);
-    if (h1) tc::tmem_ld16(tbase + (uint32_t)(B1 * 16), v1);
-    tc::tmem_wait_ld_dep2(v0, v1);
-    scan_block<B0>(v0, ivc, bias, kc, ka, kb);
-    if constexpr (J + 1 < 7) {
-      if (h1) scan_block<B1>(v1, ivc, bias, kc, ka, kb);
-    }
-    scan_from<G, J + 2>(tbase, ivc, bias, kc, nblk, ka, kb);
+// Blocks J and J + 1 are in c0/c1; the loads of blocks J + 2 and J + 3 go
+// out before c0/c1 are scanned, so the TMEM latency hides behind the scan.
+// nv = valid blocks of the chunk (at most kChunkMax / 16).
+template <int J>
+__device__ __forceinline__ void scan_pipe(uint32_t tbase, const float* ivc, float bias, int kc, int nv,
+                                          uint32_t (&c0)[16], uint32_t (&c1)[16], uint32_t (&n0)[16],
+                                          uint32_t (&n1)[16], Keys2& ka, Keys2& kb) {
+  constexpr int kB = kChunkMax / 16;
+  if constexpr (J < kB) {
+    if (J >= nv) return;
+    const bool l2 = J + 2 < nv, l3 = J + 3 < nv;
+    if constexpr (J + 2 < kB) { if (l2) tc::tmem_ld16(tbase + (uint32_t)((J + 2) * 16), n0); }
+    if constexpr (J + 3 < kB) { if (l3) tc::tmem_ld16(tbase + (uint32_t)((J + 3) * 16), n1); }
+    scan_block<J>(c0, ivc, bias, kc, ka, kb);
+    if constexpr (J + 1 < kB) { if (J + 1 < nv) scan_block<J + 1>(c1, ivc, bias, kc, ka, kb); }
+    if (l2) tc::tmem_wait_ld_dep2(n0, n1);
+    scan_pipe<J + 2>(tbase, ivc, bias, kc, nv, n0, n1, c0, c1, ka, kb);
   }
 }
 
-template <int G>
-__device__ __forceinline__ void scan_chunk(uint32_t tbase, const float* ivc, float bias, int kc, int nblk, Keys2& ka,
-                                           Keys2& kb) {
-  scan_from<G, 0>(tbase, ivc, bias, kc, nblk, ka, kb);
+// Best two keys of one chunk (kc valid columns of its TMEM buffer).
+__device__ __forceinline__ Keys2 scan_chunk(uint32_t tbase, const float* ivc, float bias, int kc) {
+  Keys2 ka{0u, 0u}, kb{0u, 0u};
+  const int nv = (kc + 15) >> 4;
+  uint32_t c0[16], c1[16], n0[16], n1[16];
+  tc::tmem_ld16(tbase, c0);
+  if (nv > 1) tc::tmem_ld16(tbase + 16u, c1);
+  tc::tmem_wait_ld_dep2(c0, c1);
+  scan_pipe<0>(tbase, ivc, bias, kc, nv, c0, c1, n0, n1, ka, kb);
+  key2_push(ka, kb.b1);
+  key2_push(ka, kb.b2);
+  return ka;
 }
 
-using Best = Keys2;
-
 struct Ctl {
-  uint64_t x_full[4], x_empty[4], acc_full[2], acc_empty[2], anc_full, anc_empty, drain;
-  uint64_t mrg_full[2], mrg_empty[2];
+  uint64_t x_full[4], x_empty[4], acc_full[kMaxBuf], acc_empty[kMaxBuf], anc_full, anc_empty, drain;
   uint32_t tmem_base;
   int err;
 };
@@ -184,9 +191,8 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
   unsigned char* anc = base;                                   // kpad x 256 B
   unsigned char* xs = anc + (size_t)a.kpad * 256;              // stages x 32 KB
   Ctl& ctl = *reinterpret_cast<Ctl*>(xs + (size_t)a.stages * kXStageBytes);
-  Best* mrg = reinterpret_cast<Best*>(&ctl + 1);               // [2][128]
   float* winv = reinterpret_cast<float*>(
-      (reinterpret_cast<uintptr_t>(mrg + 2 * 128) + 15) & ~static_cast<uintptr_t>(15));   // [8][kpad]
+      (reinterpret_cast<uintptr_t>(&ctl + 1) + 15) & ~static_cast<uintptr_t>(15));   // [8][kpad]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x;
@@ -196,11 +202,10 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { tc::mbar_init(&ctl.x_full[s], 1); tc::mbar_init(&ctl.x_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { tc::mbar_init(&ctl.acc_full[b], 1); tc::mbar_init(&ctl.acc_empty[b], 256); }
+    for (int b = 0; b < a.nbuf; ++b) { tc::mbar_init(&ctl.acc_full[b], 1); tc::mbar_init(&ctl.acc_empty[b], 128); }
     tc::mbar_init(&ctl.anc_full, 1);
     tc::mbar_init(&ctl.anc_empty, 1);
     tc::mbar_init(&ctl.drain, 1);
-    for (int b = 0; b < 2; ++b) { tc::mbar_init(&ctl.mrg_full[b], 128); tc::mbar_init(&ctl.mrg_empty[b], 128); }
     ctl.err = 0;
     tc::fence_barrier_init();
   }
@@ -270,10 +275,10 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
         const uint32_t xa = tc::smem_u32(xs + (size_t)s * kXStageBytes);
         bool ok = true;
         for (int c = 0; c < a.n_chunks; ++c, ++q) {
-          const int b = q & 1, uq = q >> 1;
+          const int b = q % a.nbuf, uq = q / a.nbuf;
           if (uq > 0 && !wait_or_fail(&ctl.acc_empty[b], (uq - 1) & 1, ctl, a.counters)) { ok = false; break; }
           tc::fence_after_sync();
-          const uint32_t d = tmem + (uint32_t)(b * kAccCols);
+          const uint32_t d = tmem + (uint32_t)(b * a.cw);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t aoff = (uint32_t)((kk >> 2) * (kXStageBytes / 2) + (kk & 3) * 32);
@@ -291,16 +296,15 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
     }
   } else {
     // ------------------------------------------------------------ epilogue (8 warps)
-    // Each column score s = acc / ||a|| becomes one positive float key
-    //   key = bits(s + ||x|| (1 + 2^-7)) with the low 9 bits replaced by 511 - slot,
+    // Each column score s = acc / ||a|| becomes one positive integer key
+    //   key = bits(s + ||x|| (1 + 2^-7) + C) * 512 + 511 - slot,
     // so the largest key is the best score and, among equal keys, the lowest
-    // slot; the best three keys per row cost five fmax/fmin per column.
-    const int g = (warp - 2) >> 2;          // column half
+    // slot.  Group g takes the items beg + g, beg + g + 2, ... whole.
+    const int g = (warp - 2) >> 2;          // item parity
     const int qd = warp & 3;                // TMEM lane quarter this warp may access
     const int row = qd * 32 + lane;
-    const int nblk = a.cw / 16;
     float* inv = winv + (size_t)(warp - 2) * a.kpad;   // this warp's copy of 1/||a||
-    int q = 0, cur_u = -1;
+    int cur_u = -1;
     // this thread's row norm and own-slot flag, one item ahead
     auto row_info = [&](int it2, float& xn2, int& own2) {
       xn2 = 0.f;
@@ -315,13 +319,13 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
     };
     float xn_next;
     int own_next;
-    row_info(beg, xn_next, own_next);
-    for (int it = beg; it < end; ++it) {
+    row_info(beg + g, xn_next, own_next);
+    for (int it = beg + g; it < end; it += 2) {
       const int u = it / a.row_tiles, j = it % a.row_tiles;
       const int side = u / a.H, h = u % a.H;
       const float xn = xn_next;
       const int own = own_next;
-      row_info(it + 1, xn_next, own_next);
+      row_info(it + 2, xn_next, own_next);
       if (u != cur_u) {
         __syncwarp();
         const float* src = a.anc_inv + (int64_t)u * a.kp16;
@@ -334,52 +338,29 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
       const RowKey rk = row_key(xn);
       Keys2 ka{0u, 0u};
       bool ok = true;
+      int q = (it - beg) * a.n_chunks;      // global chunk index of this item's first chunk
       for (int c = 0; c < a.n_chunks; ++c, ++q) {
-        const int b = q & 1, uq = q >> 1;
+        const int b = q % a.nbuf, uq = q / a.nbuf;
         if (!wait_or_fail(&ctl.acc_full[b], uq & 1, ctl, a.counters)) { ok = false; break; }
         tc::fence_after_sync();
-        const uint32_t tbase = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(b * kAccCols);
-        const int kc = a.k - c * a.cw;                   // valid columns in this chunk
-        const float* ivc = inv + c * a.cw;
-        // keys of one chunk carry bit 8 set; chunk 1's keys get it cleared
-        // afterwards, so equal scores prefer chunk 0 (the lower slots)
-        // both column groups run the same code on their own blocks (group g
-        // owns blocks g, g + 2, ...): group 1 starts 16 columns further, which
-        // its keys absorb afterwards (the low 9 bits stay >= 256, no borrow)
-        Keys2 ca{0u, 0u}, cb{0u, 0u};
-        scan_chunk<0>(tbase + 16u * (uint32_t)g, ivc + 16 * g, rk.add, kc - 16 * g, nblk - g, ca, cb);
-        key2_push(ca, cb.b1); key2_push(ca, cb.b2);
-        if (g == 1) {
-          if (ca.b1) ca.b1 -= 16u;
-          if (ca.b2) ca.b2 -= 16u;
-        }
-        if (c == 1) {
-          if (ca.b1) ca.b1 &= ~256u;
-          if (ca.b2) ca.b2 &= ~256u;
-        }
-        key2_push(ka, ca.b1); key2_push(ka, ca.b2);
+        const uint32_t tbase = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(b * a.cw);
+        Keys2 ca = scan_chunk(tbase, inv + c * a.cw, rk.add, min(a.cw, a.k - c * a.cw));
         tc::fence_before_sync();
         tc::mbar_arrive(&ctl.acc_empty[b]);
+        // column in chunk -> slot: the low 9 bits drop by c cw (no borrow, slot < 512)
+        const uint32_t off = (uint32_t)(c * a.cw);
+        if (ca.b1) ca.b1 -= off;
+        if (ca.b2) ca.b2 -= off;
+        key2_push(ka, ca.b1);
+        key2_push(ka, ca.b2);
       }
       if (!ok) break;
-      // merge the two column halves: group 1 hands its keys to group 0
-      const int n = it - beg, bb = n & 1, use = n >> 1;
-      if (g == 1) {
-        if (use > 0 && !wait_or_fail(&ctl.mrg_empty[bb], (use - 1) & 1, ctl, a.counters)) break;
-        mrg[bb * 128 + row] = ka;
-        tc::mbar_arrive(&ctl.mrg_full[bb]);
-        continue;
-      }
-      if (!wait_or_fail(&ctl.mrg_full[bb], use & 1, ctl, a.counters)) break;
-      const Keys2 other = mrg[bb * 128 + row];
-      tc::mbar_arrive(&ctl.mrg_empty[bb]);
-      key2_push(ka, other.b1); key2_push(ka, other.b2);
       if (t < a.N) {
         uint32_t slot;
         if (own >= 0) {
           slot = (uint32_t)own;
         } else {
-          slot = key_slot(ka.b1, a.cw);
+          slot = key_slot(ka.b1);
           const float gap = (float)((ka.b1 >> 9) - (ka.b2 >> 9)) * rk.step;
           if (!(gap > kRefineRelTC * xn)) list_for_refine(a.refine, a.counters, u, a.N, t);
         }
@@ -426,7 +407,7 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
 
 bool assign_tc_supported(const Plan& pl) {
   if (pl.p.dtype != ANCHORKV_BF16) return false;
-  const int n_chunks = (pl.k + kAccCols - 1) / kAccCols;
+  const int n_chunks = (pl.k + kChunkMax - 1) / kChunkMax;
   const int cw = ((pl.k + n_chunks - 1) / n_chunks + 15) / 16 * 16;
   return n_chunks * cw <= kMaxKpad && encode_fn() != nullptr;
 }
@@ -434,13 +415,13 @@ bool assign_tc_supported(const Plan& pl) {
 cudaError_t launch_assign_tc(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s) {
   TcArgs a;
   a.N = pl.N; a.H = pl.H; a.k = pl.k; a.kp16 = pl.kp16;
-  a.n_chunks = (pl.k + kAccCols - 1) / kAccCols;
+  a.n_chunks = (pl.k + kChunkMax - 1) / kChunkMax;
   a.cw = ((pl.k + a.n_chunks - 1) / a.n_chunks + 15) / 16 * 16;
   a.kpad = a.n_chunks * a.cw;
+  a.nbuf = std::min(kMaxBuf, 512 / a.cw);
   a.row_tiles = (pl.N + 127) / 128;
   a.total_items = 2 * pl.H * a.row_tiles;
-  const int fixed = 1024 + (int)sizeof(Ctl) + 16 + 2 * 128 * (int)sizeof(Best) + 16 + 8 * a.kpad * 4 +
-                    a.kpad * 256;
+  const int fixed = 1024 + (int)sizeof(Ctl) + 16 + 8 * a.kpad * 4 + a.kpad * 256;
   a.stages = std::min(4, (227 * 1024 - fixed) / kXStageBytes);
   if (a.stages < 2) return cudaErrorInvalidValue;
   a.anc_inv = reinterpret_cast<const float*>(ws + pl.o_anc_inv);
