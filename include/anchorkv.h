@@ -224,7 +224,11 @@ int anchorkv_reconstruct(const anchorkv_params* p, const void* compressed,
 
 /* Copies the device status word and counters of a compress workspace to
  * `host_counters` (16 int32) with a synchronous copy on `stream`.  Returns
- * ANCHORKV_EDEVICE if the status word is non-zero. */
+ * ANCHORKV_EDEVICE if the status word is non-zero.  The first failing check
+ * latches its code: 1 uniform anchor sample, 2 refine list, 3 an
+ * inconsistent record or selection (a write that would leave its bounds is
+ * skipped), 4 a bounded wait in a tensor-core kernel timed out (the kernel
+ * drained its own work and returned). */
 int anchorkv_read_device_status(const void* ws, int32_t* host_counters, void* stream);
 
 /* The fp32 codebook the kernels use: {tau, l1, l2, mse} of the four-level

@@ -180,12 +180,20 @@ def reconstruct(p: AnchorKVParams, compressed: torch.Tensor):
     return Kh, Vh
 
 
+# device status word values (the first kernel to fail latches its code)
+DEVICE_ERRORS = {1: "uniform anchor sample", 2: "refine list", 3: "inconsistent record or selection (bounds)",
+                 4: "bounded wait timed out"}
+
+
 def read_status(workspace: torch.Tensor) -> list[int]:
     """Device status word and counters of a compress workspace (synchronises
-    the current stream).  Raises if a device-side check failed."""
+    the current stream).  Raises if a device-side check failed, naming it."""
     buf = (ctypes.c_int32 * 16)()
     st = capi.lib().anchorkv_read_device_status(_ptr(workspace), buf, _stream(workspace.device))
     vals = list(buf)
+    if st == capi.EDEVICE:
+        raise capi.AnchorKVError("anchorkv_read_device_status", st,
+                                 f"status word {vals[0]} ({DEVICE_ERRORS.get(vals[0], 'unknown')})")
     capi.check("anchorkv_read_device_status", st)
     return vals
 

@@ -69,10 +69,11 @@ _lib = None
 
 
 class AnchorKVError(RuntimeError):
-    def __init__(self, fn: str, status: int):
+    def __init__(self, fn: str, status: int, detail: str | None = None):
         msg = _lib.anchorkv_strerror(status).decode() if _lib is not None else str(status)
-        super().__init__(f"{fn} failed: {msg} ({status})")
+        super().__init__(f"{fn} failed: {msg} ({status})" + (f": {detail}" if detail else ""))
         self.status = status
+        self.detail = detail
 
 
 def header_functions() -> list[str]:

@@ -6,20 +6,26 @@
 // lowest slot, a zero anchor scores 0, an anchor token keeps its own slot.
 //
 // The contraction S = X A^T (X: 128 token rows, A: all k anchors of the
-// KV head and side, D = 128) runs as tcgen05.mma (M = 128, N = chunk of at
-// most 128 anchors, K = 16 per instruction) from 128-byte-swizzled
-// shared-memory tiles that TMA fills; accumulators live in a ring of TMEM
-// chunk buffers (as many as fit in 512 columns).  The epilogue never writes
+// KV head and side, D = 128) runs as tcgen05.mma (M = 128, N = chunk of
+// anchors, K = 16 per instruction) from 128-byte-swizzled shared-memory
+// tiles that TMA fills; accumulators live in a ring of TMEM chunk buffers
+// (as many as fit in 512 columns).  Chunks are as wide as possible (up to
+// N = 256): the MMA issue rate per FLOP is best for wide N.  The ring is
+// shared by the epilogue groups, so a group may reach chunk q while the
+// buffer still waits for chunk q - nbuf; since a parity wait cannot tell
+// phase p from p + 2, a group first waits until the MMA warp has published
+// that it issued chunk q (which it does only after chunk q - nbuf was
+// released) and only then waits on the buffer's barrier.  The epilogue never writes
 // S: each thread reads its TMEM lane, scales each column by 1/||a_s|| and
 // keeps the best and second-best score of its row over all chunks.  Rows
 // whose fp32 margin between best and second best is not above the
 // accumulation error bound are listed for the fp64 re-decision shared with
 // the SIMT path.
 //
-// Warp roles (320 threads, one CTA per SM, persistent over (side, head,
-// 128-row tile) work items): warp 0 issues TMA, warp 1 owns TMEM and issues
-// MMAs, warps 2..9 run the epilogue as two groups of four warps that take
-// alternate items whole (every column of their 128 rows), so the groups
+// Warp roles (one CTA per SM, persistent over (side, head, 128-row tile)
+// work items): warp 0 issues TMA, warp 1 owns TMEM and issues MMAs, the
+// other warps run the epilogue as kGroups groups of four warps that take
+// items in turn, each whole (every column of its 128 rows), so the groups
 // never wait on each other and need no merge.  Anchors of the current
 // (side, head) stay resident in shared memory; token tiles stream through a
 // ring.
@@ -43,11 +49,13 @@ constexpr float kRefineRelTC = 1.0f / 8192.0f;
 
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kXStageBytes = 128 * 256;       // 128 rows x 128 bf16
-constexpr int kMaxKpad = 448;
-constexpr int kChunkMax = 128;                // anchors per MMA chunk (accumulator columns)
+constexpr int kGroups = 2;                    // epilogue groups (four warps each)
+constexpr int kEpiWarps = 4 * kGroups;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kChunkMax = 256;                // anchors per MMA chunk (N of one instruction)
 constexpr int kMaxBuf = 8;                    // accumulator buffers in the TMEM ring
+constexpr int kXStageBytes = 128 * 256;       // 128 rows x 128 bf16
+constexpr int kMaxKpad = 480;
 
 struct TcArgs {
   int N, H, k, kp16, cw, n_chunks, kpad, stages, row_tiles, nbuf;
@@ -163,7 +171,17 @@ struct Ctl {
   uint64_t x_full[4], x_empty[4], acc_full[kMaxBuf], acc_empty[kMaxBuf], anc_full, anc_empty, drain;
   uint32_t tmem_base;
   int err;
+  int issued;          // chunks the MMA warp has issued (store-release)
 };
+
+__device__ __forceinline__ void publish_issued(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(tc::smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int read_issued(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(tc::smem_u32(p)) : "memory");
+  return v;
+}
 
 __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t parity, Ctl& ctl, int* counters) {
   uint64_t t0 = 0;
@@ -181,6 +199,23 @@ __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t parity, Ctl
   return false;
 }
 
+// Bounded wait until the MMA warp has issued chunk q.
+__device__ __forceinline__ bool wait_issued(Ctl* ctl, int q, int* counters) {
+  uint64_t t0 = 0;
+  for (uint32_t i = 0; i < tc::kWaitLimit; ++i) {
+    if (read_issued(&ctl->issued) > q) return true;
+    if ((i & 255u) == 255u) {
+      if (*(volatile int*)&ctl->err) return false;
+      const uint64_t now = tc::globaltimer_ns();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > tc::kWaitNs) break;
+    }
+  }
+  *(volatile int*)&ctl->err = 1;
+  latch_error(counters, kDevErrTimeout);
+  return false;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constant__ CUtensorMap mapXV,
                  const __grid_constant__ CUtensorMap mapAK, const __grid_constant__ CUtensorMap mapAV, TcArgs a) {
@@ -192,7 +227,7 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
   unsigned char* xs = anc + (size_t)a.kpad * 256;              // stages x 32 KB
   Ctl& ctl = *reinterpret_cast<Ctl*>(xs + (size_t)a.stages * kXStageBytes);
   float* winv = reinterpret_cast<float*>(
-      (reinterpret_cast<uintptr_t>(&ctl + 1) + 15) & ~static_cast<uintptr_t>(15));   // [8][kpad]
+      (reinterpret_cast<uintptr_t>(&ctl + 1) + 15) & ~static_cast<uintptr_t>(15));   // [kEpiWarps][kpad]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x;
@@ -203,6 +238,7 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { tc::mbar_init(&ctl.x_full[s], 1); tc::mbar_init(&ctl.x_empty[s], 1); }
     for (int b = 0; b < a.nbuf; ++b) { tc::mbar_init(&ctl.acc_full[b], 1); tc::mbar_init(&ctl.acc_empty[b], 128); }
+    ctl.issued = 0;
     tc::mbar_init(&ctl.anc_full, 1);
     tc::mbar_init(&ctl.anc_empty, 1);
     tc::mbar_init(&ctl.drain, 1);
@@ -287,6 +323,7 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
                          kk > 0 ? 1u : 0u);
           }
           tc::mma_commit(&ctl.acc_full[b]);
+          publish_issued(&ctl.issued, q + 1);
         }
         if (!ok) break;
         tc::mma_commit(&ctl.x_empty[s]);
@@ -295,12 +332,12 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
       tc::mbar_wait(&ctl.drain, 0);
     }
   } else {
-    // ------------------------------------------------------------ epilogue (8 warps)
+    // ------------------------------------------------------------ epilogue (kEpiWarps warps)
     // Each column score s = acc / ||a|| becomes one positive integer key
     //   key = bits(s + ||x|| (1 + 2^-7) + C) * 512 + 511 - slot,
     // so the largest key is the best score and, among equal keys, the lowest
-    // slot.  Group g takes the items beg + g, beg + g + 2, ... whole.
-    const int g = (warp - 2) >> 2;          // item parity
+    // slot.  Group g takes the items beg + g, beg + g + kGroups, ... whole.
+    const int g = (warp - 2) >> 2;
     const int qd = warp & 3;                // TMEM lane quarter this warp may access
     const int row = qd * 32 + lane;
     float* inv = winv + (size_t)(warp - 2) * a.kpad;   // this warp's copy of 1/||a||
@@ -320,12 +357,12 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
     float xn_next;
     int own_next;
     row_info(beg + g, xn_next, own_next);
-    for (int it = beg + g; it < end; it += 2) {
+    for (int it = beg + g; it < end; it += kGroups) {
       const int u = it / a.row_tiles, j = it % a.row_tiles;
       const int side = u / a.H, h = u % a.H;
       const float xn = xn_next;
       const int own = own_next;
-      row_info(it + 2, xn_next, own_next);
+      row_info(it + kGroups, xn_next, own_next);
       if (u != cur_u) {
         __syncwarp();
         const float* src = a.anc_inv + (int64_t)u * a.kp16;
@@ -338,10 +375,14 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
       const RowKey rk = row_key(xn);
       Keys2 ka{0u, 0u};
       bool ok = true;
-      int q = (it - beg) * a.n_chunks;      // global chunk index of this item's first chunk
+      int q = (it - beg) * a.n_chunks;      // ring index of this item's first chunk
       for (int c = 0; c < a.n_chunks; ++c, ++q) {
         const int b = q % a.nbuf, uq = q / a.nbuf;
-        if (!wait_or_fail(&ctl.acc_full[b], uq & 1, ctl, a.counters)) { ok = false; break; }
+        // chunk q issued => chunk q - nbuf released => the barrier is at phase uq
+        if (!wait_issued(&ctl, q, a.counters) || !wait_or_fail(&ctl.acc_full[b], uq & 1, ctl, a.counters)) {
+          ok = false;
+          break;
+        }
         tc::fence_after_sync();
         const uint32_t tbase = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(b * a.cw);
         Keys2 ca = scan_chunk(tbase, inv + c * a.cw, rk.add, min(a.cw, a.k - c * a.cw));
@@ -421,7 +462,7 @@ cudaError_t launch_assign_tc(const Plan& pl, const void* K, const void* V, char*
   a.nbuf = std::min(kMaxBuf, 512 / a.cw);
   a.row_tiles = (pl.N + 127) / 128;
   a.total_items = 2 * pl.H * a.row_tiles;
-  const int fixed = 1024 + (int)sizeof(Ctl) + 16 + 8 * a.kpad * 4 + a.kpad * 256;
+  const int fixed = 1024 + (int)sizeof(Ctl) + 16 + kEpiWarps * a.kpad * 4 + a.kpad * 256;
   a.stages = std::min(4, (227 * 1024 - fixed) / kXStageBytes);
   if (a.stages < 2) return cudaErrorInvalidValue;
   a.anc_inv = reinterpret_cast<const float*>(ws + pl.o_anc_inv);

@@ -125,14 +125,42 @@ __device__ __forceinline__ double sign_of(const CodecConst& cc, int j) {
   return ((cc.sign_bits[j >> 5] >> (j & 31)) & 1u) ? -1.0 : 1.0;
 }
 
-// One warp per (tile, 32-token word); residual records in flat order.
+// 16 consecutive elements of a row (32-byte aligned for bf16, 64 for fp32).
+template <typename T> __device__ __forceinline__ void load16(const T* p, float (&o)[16]);
+template <> __device__ __forceinline__ void load16<float>(const float* p, float (&o)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 v = reinterpret_cast<const float4*>(p)[i];
+    o[4 * i] = v.x; o[4 * i + 1] = v.y; o[4 * i + 2] = v.z; o[4 * i + 3] = v.w;
+  }
+}
+template <> __device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfloat16* p, float (&o)[16]) {
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint4 v = reinterpret_cast<const uint4*>(p)[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      o[8 * i + 2 * e] = __uint_as_float(w[e] << 16);
+      o[8 * i + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+    }
+  }
+}
+
+// One warp per (tile, 32-token word); its residual records (flat order) go
+// four at a time, eight lanes per record, lane l8 holding elements
+// 16 l8 .. 16 l8 + 15.  The word's token records are gathered once (lane b
+// holds token b's), so each record costs one round of independent row loads.
+// The Hadamard transform runs its four low stages in registers and its three
+// high stages across the record's eight lanes, all in fp64.
 template <typename T>
-__global__ void quantize_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ anc_k,
-                                const T* __restrict__ anc_v, const uint32_t* __restrict__ tok,
-                                const uint32_t* __restrict__ bitmap, const int* __restrict__ tile_prefix,
-                                uint8_t* __restrict__ codes, uint16_t* __restrict__ sigma, int N, int H, int k,
-                                int n_tiles, int64_t R, int* __restrict__ counters, CodecConst cc) {
-  const int lane = threadIdx.x & 31;
+__global__ void __launch_bounds__(256, 2) quantize_kernel(const T* __restrict__ K, const T* __restrict__ V,
+                                const T* __restrict__ anc_k, const T* __restrict__ anc_v,
+                                const uint32_t* __restrict__ tok, const uint32_t* __restrict__ bitmap,
+                                const int* __restrict__ tile_prefix, uint8_t* __restrict__ codes,
+                                uint16_t* __restrict__ sigma, int N, int H, int k, int n_tiles, int64_t R,
+                                int* __restrict__ counters, CodecConst cc) {
+  const int lane = threadIdx.x & 31, grp = lane >> 3, l8 = lane & 7;
   const int n_words = 2 * H * n_tiles * 4;
   const int wid = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (wid >= n_words) return;
@@ -140,49 +168,83 @@ __global__ void quantize_kernel(const T* __restrict__ K, const T* __restrict__ V
   const int sh = tile / n_tiles, j = tile % n_tiles;
   const int side = sh / H, h = sh % H;
   const uint32_t* bw = bitmap + (int64_t)tile * 4;
-  int rec = tile_prefix[sh * (n_tiles + 1) + j];
-  for (int q = 0; q < w; ++q) rec += __popc(bw[q]);
-  uint32_t bits = bw[w];
+  int rec0 = tile_prefix[sh * (n_tiles + 1) + j];
+  for (int q = 0; q < w; ++q) rec0 += __popc(bw[q]);
+  const uint32_t bits = bw[w];
+  const int nrec = __popc(bits);
+  if (nrec == 0) return;
+  const int t0 = j * kTile + w * 32;
+  // token (t0 + lane)'s record word, if selected
+  uint32_t my_tok = 0;
+  if (((bits >> lane) & 1u) && t0 + lane < N) my_tok = tok[(int64_t)sh * N + t0 + lane];
   const double inv_sqrt_d = 1.0 / sqrt((double)kD);
-  double sgn[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) sgn[e] = sign_of(cc, lane * 4 + e);
-  while (bits) {
-    const int b = __ffs(bits) - 1;
-    bits &= bits - 1;
-    const int t = j * kTile + w * 32 + b;
-    if (rec >= R || t >= N) {                 // inconsistent selection: never write out of bounds
-      if (lane == 0) latch_error(counters, kDevErrBounds);
-      break;
-    }
-    const uint32_t rec_tok = tok[((int64_t)side * H + h) * N + t];
+  // sign bits of elements 16 l8 .. 16 l8 + 15 (bit i set: s = -1)
+  const uint32_t sw = l8 < 2 ? cc.sign_bits[0] : l8 < 4 ? cc.sign_bits[1] : l8 < 6 ? cc.sign_bits[2] : cc.sign_bits[3];
+  const uint32_t sgn = (sw >> ((l8 & 1) * 16)) & 0xFFFFu;
+  const T* X = (side ? V : K) + (int64_t)h * N * kD + l8 * 16;
+  const T* A = (side ? anc_v : anc_k) + (int64_t)h * k * kD + l8 * 16;
+  for (int base = 0; base < nrec; base += 4) {
+    const int i = base + grp;
+    const bool act = i < nrec;
+    const int b = act ? (int)__fns(bits, 0, i + 1) : 0;
+    const int t = t0 + b;
+    const int64_t rec = (int64_t)rec0 + i;
+    const uint32_t rec_tok = __shfl_sync(0xffffffffu, my_tok, b);
     const uint32_t slot = rec_tok & 0xFFFFu;
+    const bool bad = act && (rec >= R || t >= N || slot >= (uint32_t)k);
+    if (bad && l8 == 0) latch_error(counters, kDevErrBounds);   // inconsistent record: write nothing
+    const bool live = act && !bad;
     const double g = (double)half_bits_to_f(rec_tok >> 16);
-    float xf[4], af[4];
-    load4<T>((side ? V : K) + ((int64_t)h * N + t) * kD + lane * 4, xf);
-    load4<T>((side ? anc_v : anc_k) + ((int64_t)h * k + slot) * kD + lane * 4, af);
-    double y[4];
+    float xf[16], af[16];
+    if (live) {
+      load16<T>(X + (int64_t)t * kD, xf);
+      load16<T>(A + (int64_t)slot * kD, af);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) { xf[e] = 0.f; af[e] = 0.f; }
+    }
+    double y[16];
     double r2 = 0.0;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
+    for (int e = 0; e < 16; ++e) {
       const double r = (double)xf[e] - g * (double)af[e];
       r2 = fma(r, r, r2);
-      y[e] = r * sgn[e];
+      y[e] = ((sgn >> e) & 1u) ? -r : r;
     }
-    r2 = warp_sum_d(r2);
-    fwht128<double>(y);
+#pragma unroll
+    for (int m = 1; m < 8; m <<= 1) r2 += __shfl_xor_sync(0xffffffffu, r2, m);
+    // Hadamard transform (natural order): four stages on the element bits ...
+#pragma unroll
+    for (int m = 1; m < 16; m <<= 1)
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        if (!(e & m)) {
+          const double a0 = y[e], a1 = y[e | m];
+          y[e] = a0 + a1;
+          y[e | m] = a0 - a1;
+        }
+    // ... and three on the lane bits
+#pragma unroll
+    for (int m = 1; m < 8; m <<= 1) {
+      const bool upper = l8 & m;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const double other = __shfl_xor_sync(0xffffffffu, y[e], m);
+        y[e] = upper ? (other - y[e]) : (y[e] + other);
+      }
+    }
+    if (!live) continue;
     const uint16_t sb = half_bits_rn(sqrt(r2 / (double)kD));
     const double th = cc.tau * (double)half_bits_to_f(sb);
-    uint32_t byte = 0;
+    uint32_t word = 0;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
+    for (int e = 0; e < 16; ++e) {
       const double v = y[e] * inv_sqrt_d;
       const uint32_t c = (v >= th) ? 3u : (v >= 0.0) ? 2u : (v >= -th) ? 1u : 0u;
-      byte |= c << (2 * e);
+      word |= c << (2 * e);
     }
-    codes[(int64_t)rec * kCodeBytes + lane] = (uint8_t)byte;
-    if (lane == 0) sigma[rec] = sb;
-    ++rec;
+    reinterpret_cast<uint32_t*>(codes + rec * kCodeBytes)[l8] = word;
+    if (l8 == 0) sigma[rec] = sb;
   }
 }
 

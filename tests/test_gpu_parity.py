@@ -36,6 +36,10 @@ CASES = {
     "bf16-gqa16-n1500": (CacheSpec(1, 1, 16, 1500, n_dirs=32, seed=8), 0.2),
     # enough tiles that every CTA of a 16-CTA decode cluster streams two chunks
     "bf16-n20000": (CacheSpec(1, 1, 4, 20000, n_dirs=64, seed=9), 0.1),
+    # wide windows: k = W + ceil(N/128) anchors = 232 and 413 (up to six
+    # assignment chunks; eight 128-row observation blocks)
+    "bf16-window200-n4000": (CacheSpec(1, 1, 4, 4000, window=200, n_dirs=32, seed=10), 0.1),
+    "bf16-window256-n20000": (CacheSpec(1, 1, 4, 20000, window=256, n_dirs=64, seed=11), 0.1),
 }
 
 
