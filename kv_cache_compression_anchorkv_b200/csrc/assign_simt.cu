@@ -133,84 +133,100 @@ assign_simt_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __
 }
 
 // Re-decision of the listed rows of one (side, head) per blockIdx.y.
-// The block stages the head's anchors in shared memory transposed as
-// (d, d+1) pairs per slot, so that lanes scoring consecutive slots read
-// consecutive words.  Each warp takes one row: fp32 scores of every slot
-// (sequential FMA over D = 128 exact products: error <= 2^-17 ||x|| after
-// scaling), candidates within 2^-14 ||x|| of the best fp32 score, and the
-// exact fp64 score dot / sqrt(||a||^2) of each candidate (correctly rounded
-// sqrt and division) decides; ties go to the lowest slot.
+// The (side, head) lists are walked as one flat sequence (their lengths are
+// very uneven), one listed row per warp; nothing is staged: the anchors stay
+// in L2 (k x 256 bytes, shared by every row of the list).  Scores go 32 slots
+// at a time: lane l holds coordinates 4l .. 4l + 3 of the row and of each of
+// the 32 anchors (coalesced loads, all 32 in flight together), and a transposed butterfly
+// leaves slot j0 + l's dot product on lane l.  fp32 products of exact inputs
+// summed in any order err by at most 127 u sum|x_d a_d| <= 2^-17 ||x|| ||a||,
+// so after scaling by 1/||a|| every slot within 2^-14 ||x|| of the best fp32
+// score is a candidate.  Candidates are gathered 32 at a time and each lane
+// takes one: the exact fp64 score dot / sqrt(||a||^2) (correctly rounded
+// sqrt and division) decides, ties to the lowest slot.
 constexpr int kRefineWarps = 8;
 constexpr int kRefineMaxK = 2048;
-template <typename T> struct RefineCfg;
-// kChunk slots per staging round; the transposed rows are kChunk + 1 pairs
-// apart so that the staging stores of consecutive pairs fall in different banks.
-template <> struct RefineCfg<__nv_bfloat16> { using P = __nv_bfloat162; static constexpr int kChunk = 448; };
-template <> struct RefineCfg<float> { using P = float2; static constexpr int kChunk = 192; };
-template <typename T> __host__ __device__ constexpr int refine_ld() { return RefineCfg<T>::kChunk + 1; }
 
-__device__ __forceinline__ float2 pair_f(__nv_bfloat162 p) { return __bfloat1622float2(p); }
-__device__ __forceinline__ float2 pair_f(float2 p) { return p; }
+template <typename T> struct RawRow;    // 4 consecutive elements as loaded
+template <> struct RawRow<__nv_bfloat16> {
+  uint2 v;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { v = *reinterpret_cast<const uint2*>(p); }
+  __device__ __forceinline__ float dot(const float (&x)[4]) const {
+    return fmaf(x[3], __uint_as_float(v.y & 0xFFFF0000u), fmaf(x[2], __uint_as_float(v.y << 16),
+           fmaf(x[1], __uint_as_float(v.x & 0xFFFF0000u), x[0] * __uint_as_float(v.x << 16))));
+  }
+};
+template <> struct RawRow<float> {
+  float4 v;
+  __device__ __forceinline__ void load(const float* p) { v = *reinterpret_cast<const float4*>(p); }
+  __device__ __forceinline__ float dot(const float (&x)[4]) const {
+    return fmaf(x[3], v.w, fmaf(x[2], v.z, fmaf(x[1], v.y, x[0] * v.x)));
+  }
+};
+
+// One lane's exact fp64 score of slot s against the row held in shared memory.
+template <typename T>
+__device__ __forceinline__ double exact_score(const T* A, const float* xw, const double* sq, int s) {
+  const T* a = A + (int64_t)s * kD;
+  double d = 0.0;
+#pragma unroll 4
+  for (int c = 0; c < kD; c += 4) {
+    float af[4];
+    load4<T>(a + c, af);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) d = fma((double)xw[c + e], (double)af[e], d);
+  }
+  const double nn = sq[s];
+  return nn > 0.0 ? d / nn : 0.0;
+}
 
 template <typename T>
-__global__ void __launch_bounds__(kRefineWarps * 32)
+__global__ void __launch_bounds__(kRefineWarps * 32, 3)
 refine_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ anc_k,
               const T* __restrict__ anc_v, const float* __restrict__ anc_inv, const double* __restrict__ anc_sqrt,
               const int* __restrict__ refine, const int* __restrict__ counters, uint32_t* __restrict__ tok, int N,
               int H, int k, int kp16) {
-  using P = typename RefineCfg<T>::P;
-  constexpr int CH = RefineCfg<T>::kChunk;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  constexpr int LD = refine_ld<T>();
-  P* aT = reinterpret_cast<P*>(smem_raw);                              // [64][LD]
-  float* xs = reinterpret_cast<float*>(aT + 64 * LD);                  // [8][128]
-  float* sc = xs + kRefineWarps * kD;                                  // [8][kRefineMaxK]
-  const int u = blockIdx.y, side = u / H, h = u % H;
-  const int n = counters[kRefineListBase + u];
-  if ((int)blockIdx.x * kRefineWarps >= n) return;
+  float* sc = reinterpret_cast<float*>(smem_raw);                      // [8][kRefineMaxK]
+  float* xs = sc + kRefineWarps * kRefineMaxK;                         // [8][128]
+  int* cs_all = reinterpret_cast<int*>(xs + kRefineWarps * kD);        // [8][32]
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const T* A = (side ? anc_v : anc_k) + (int64_t)h * k * kD;
-  const float* inv = anc_inv + (int64_t)u * kp16;
-  const double* sq = anc_sqrt + (int64_t)u * k;
-  float* xw = xs + w * kD;
   float* sw = sc + w * kRefineMaxK;
-  auto stage = [&](int c0, int cn) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < cn * 64; i += blockDim.x) {
-      const int j = i / 64, dp = i % 64;
-      const T* src = A + (int64_t)(c0 + j) * kD + 2 * dp;
-      aT[dp * LD + j] = *reinterpret_cast<const P*>(src);
-    }
-    __syncthreads();
-  };
-  const bool one_chunk = k <= CH;
-  if (one_chunk) stage(0, k);
-  for (int base = blockIdx.x * kRefineWarps; base < n; base += gridDim.x * kRefineWarps) {
-    const int i = base + w;
-    const bool live = i < n;
-    const int t = live ? refine[(int64_t)u * N + i] : 0;
-    const T* x = (side ? V : K) + ((int64_t)h * N + t) * kD;
+  float* xw = xs + w * kD;
+  int* cl = cs_all + w * 32;
+  int total = 0;
+  for (int u = 0; u < 2 * H; ++u) total += counters[kRefineListBase + u];
+  for (int g = blockIdx.x * kRefineWarps + w; g < total; g += gridDim.x * kRefineWarps) {
+    int u = 0, i = g;
+    while (i >= counters[kRefineListBase + u]) i -= counters[kRefineListBase + u++];
+    const int side = u / H, h = u % H;
+    const T* A = (side ? anc_v : anc_k) + (int64_t)h * k * kD;
+    const float* inv = anc_inv + (int64_t)u * kp16;
+    const double* sq = anc_sqrt + (int64_t)u * k;
+    const int t = refine[(int64_t)u * N + i];
     float xf[4];
-    load4<T>(x + lane * 4, xf);
+    load4<T>((side ? V : K) + ((int64_t)h * N + t) * kD + lane * 4, xf);
     __syncwarp();
 #pragma unroll
     for (int e = 0; e < 4; ++e) xw[lane * 4 + e] = xf[e];
     const float xn = sqrtf(warp_sum(xf[0] * xf[0] + xf[1] * xf[1] + xf[2] * xf[2] + xf[3] * xf[3]));
-    __syncwarp();
     float best = -INFINITY;
-    for (int c0 = 0; c0 < k; c0 += CH) {
-      const int cn = min(CH, k - c0);
-      if (!one_chunk) stage(c0, cn);
-      for (int j = lane; j < cn; j += 32) {
-        float acc = 0.f;
-#pragma unroll 8
-        for (int dp = 0; dp < 64; ++dp) {
-          const float2 av = pair_f(aT[dp * LD + j]);
-          acc = fmaf(xw[2 * dp], av.x, acc);
-          acc = fmaf(xw[2 * dp + 1], av.y, acc);
-        }
-        const float s = acc * inv[c0 + j];
-        sw[c0 + j] = s;
+    const T* Al = A + lane * 4;
+    for (int j0 = 0; j0 < k; j0 += 32) {
+      RawRow<T> r[32];
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) {
+        if (j0 + jj < k) r[jj].load(Al + (int64_t)(j0 + jj) * kD);
+        else r[jj].v = {};
+      }
+      float v[32];
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) v[jj] = r[jj].dot(xf);
+      transpose_reduce32(v, lane);
+      const int j = j0 + lane;
+      if (j < k) {
+        const float s = v[0] * inv[j];
+        sw[j] = s;
         best = fmaxf(best, s);
       }
     }
@@ -219,31 +235,46 @@ refine_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restr
     const float thr = best - xn * (1.0f / 16384.0f);
     double cbest = -INFINITY;
     int cbi = 0x7fffffff;
+    int nb = 0;                               // candidates gathered in cl (warp-uniform)
+    auto evaluate = [&]() {
+      __syncwarp();
+      if (lane < nb) {
+        const int s = cl[lane];
+        const double c = exact_score<T>(A, xw, sq, s);
+        if (c > cbest || (c == cbest && s < cbi)) { cbest = c; cbi = s; }
+      }
+      __syncwarp();
+      nb = 0;
+    };
     for (int j0 = 0; j0 < k; j0 += 32) {
       const int j = j0 + lane;
-      uint32_t cand = __ballot_sync(0xffffffffu, j < k && sw[j] >= thr);
-      while (cand) {
-        const int s = j0 + __ffs(cand) - 1;
-        cand &= cand - 1;
-        float af[4];
-        load4<T>(A + (int64_t)s * kD + lane * 4, af);
-        double d = 0.0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) d = fma((double)xf[e], (double)af[e], d);
-        d = warp_sum_d(d);
-        const double nn = sq[s];
-        const double cs = (nn > 0.0) ? d / nn : 0.0;
-        if (cs > cbest) { cbest = cs; cbi = s; }
+      bool mine = j < k && sw[j] >= thr;
+      uint32_t m = __ballot_sync(0xffffffffu, mine);
+      while (m) {
+        const int take = min(__popc(m), 32 - nb);
+        const int rank = __popc(m & ((1u << lane) - 1u));
+        if (mine && rank < take) { cl[nb + rank] = j; mine = false; }
+        nb += take;
+        m = __ballot_sync(0xffffffffu, mine);
+        if (nb == 32) evaluate();
       }
     }
-    if (live && lane == 0 && cbi < k) tok[(int64_t)u * N + t] = (uint32_t)cbi;
+    if (nb) evaluate();
+    // warp argmax over (score, -slot)
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const double oc = __shfl_xor_sync(0xffffffffu, cbest, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, cbi, o);
+      if (oc > cbest || (oc == cbest && oi < cbi)) { cbest = oc; cbi = oi; }
+    }
+    if (lane == 0 && cbi < k) tok[(int64_t)u * N + t] = (uint32_t)cbi;
+    __syncwarp();
   }
 }
 
 template <typename T>
 constexpr int refine_smem() {
-  return 64 * refine_ld<T>() * (int)sizeof(typename RefineCfg<T>::P) + kRefineWarps * kD * 4 +
-         kRefineWarps * kRefineMaxK * 4;
+  return kRefineWarps * (kRefineMaxK + kD + 32) * 4;
 }
 
 }  // namespace
@@ -280,8 +311,11 @@ cudaError_t launch_refine(const Plan& pl, const void* K, const void* V, char* ou
   auto* ref = reinterpret_cast<const int*>(ws + pl.o_refine);
   auto* cnt = reinterpret_cast<const int*>(ws + pl.o_counters);
   auto* tok = reinterpret_cast<uint32_t*>(out + pl.L.off_tok);
-  // a few CTAs per (side, head) list; the lists are short (about 1% of rows)
-  const dim3 grid(std::max(1, 2 * 148 / (2 * pl.H)), 2 * pl.H);
+  // the lists are short (about 1% of rows) and uneven: a flat walk over all
+  // of them, a few resident CTAs per SM
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const dim3 grid(3 * sms);
   if (pl.p.dtype == ANCHORKV_BF16) {
     using T = __nv_bfloat16;
     auto kfn = refine_kernel<T>;

@@ -142,4 +142,19 @@ __device__ __forceinline__ void fwht128(F (&v)[4]) {
   }
 }
 
+// Transposed butterfly: on entry lane l holds 32 partial values v[i]; on
+// exit v[0] of lane l is the sum over lanes of value l (31 shuffles).
+__device__ __forceinline__ void transpose_reduce32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float keep = up ? v[i + off] : v[i];
+      const float send = up ? v[i] : v[i + off];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+}
+
 }  // namespace akv

@@ -155,21 +155,6 @@ __device__ __forceinline__ float sign_of(const CArgs& a, int d) {
   return ((a.sign_bits[d >> 5] >> (d & 31)) & 1u) ? -1.f : 1.f;
 }
 
-// Transposed butterfly: on entry lane l holds 32 partial values v[i]; on
-// exit v[0] of lane l is the sum over lanes of value l.
-__device__ __forceinline__ void transpose_reduce32(float (&v)[32], int lane) {
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) {
-    const bool up = (lane & off) != 0;
-#pragma unroll
-    for (int i = 0; i < off; ++i) {
-      const float keep = up ? v[i + off] : v[i];
-      const float send = up ? v[i] : v[i + off];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-    }
-  }
-}
-
 // Records of tiles [i0, i1) of one side (relative prefix indices), clamped
 // to [0, R) and to `cap` records: [r0, r0 + n), scales staged from the even
 // record w0.
