@@ -36,6 +36,14 @@ import numpy as np
 # Parameters and fixed hyper-parameters
 # --------------------------------------------------------------------------
 
+# Mode bits (Params.mode; the C ABI's anchorkv_params.mode):
+MODE_KEY_QUERIES = 1        # [VQ] "Adaptation notes": trailing key rows as proxy queries
+MODE_RANK_SHIFT = 1         # bits 1..3: ranking criterion of the residual budget
+MODE_RANK_MASK = 7 << MODE_RANK_SHIFT
+MODE_NAIVE_CODEC = 1 << 4   # [PITH] minor comments, Figure 5 "Naive 2 bit": no rotation
+RANK_UTILITY, RANK_RESIDUAL_NORM, RANK_ATTENTION, RANK_COSINE, RANK_RANDOM = 0, 1, 2, 3, 4
+RANK_SALT = 0x72616E6B5F726E64   # "rank_rnd": separates the ranking keys from the anchor sample
+
 B_INDEX = 2      # b_a: bytes per anchor index   [PITH] "Assumptions & free parameters", codec parameters
 B_GAMMA = 2      # b_gamma: bytes per coefficient [PITH] same entry
 CODE_BITS = 2    # 2-bit residual codes            [PITH] same entry
@@ -70,6 +78,19 @@ class Params:
     rho_num: int = 7
     rho_den: int = 10
     pool_kernel: int = 7
+    mode: int = 0                # MODE_* bits; 0 = the method as the pages describe it
+
+    @property
+    def key_queries(self) -> bool:
+        return bool(self.mode & MODE_KEY_QUERIES)
+
+    @property
+    def rank(self) -> int:
+        return (self.mode & MODE_RANK_MASK) >> MODE_RANK_SHIFT
+
+    @property
+    def naive_codec(self) -> bool:
+        return bool(self.mode & MODE_NAIVE_CODEC)
 
     @property
     def elem_bytes(self) -> int:
@@ -411,6 +432,78 @@ def utilities(alpha: np.ndarray, ybar: np.ndarray, Qh: np.ndarray, Vh: np.ndarra
     return uK, uV
 
 
+def key_queries(K: np.ndarray, p: Params) -> np.ndarray:
+    """Proxy observation queries built from the keys alone: [Hq, W, D].
+
+    [VQ] "Adaptation notes" (key-as-query proxy): a cache wrapper never sees
+    queries, so the trailing anchorkv_window key rows stand in as the queries
+    for both anchor selection and residual scoring.
+    Reading: every query head j of KV head h = j // G uses K[h, N-W : N]
+    (the G copies rank exactly like one copy); each proxy row keeps its
+    position N - W + w, so the causal mask is unchanged.
+    """
+    H, N, D = K.shape
+    W, G = p.window, p.group
+    Q = np.zeros((p.n_q_heads, W, D))
+    for j in range(p.n_q_heads):
+        Q[j] = K[j // G, N - W:N]
+    return Q
+
+
+def random_rank_key(seed: int, layer: int, f: int) -> float:
+    """Uniform ranking value in [0, 1) of flat token-side f: the top 24 bits of
+    a SplitMix64 output (a 24-bit integer over 2^24, exact in fp32)."""
+    z = splitmix64((seed ^ RANK_SALT ^ ((layer & 0x7FFF) << 48) ^ f) & _M64)
+    return float(z >> 40) / float(1 << 24)
+
+
+def ranking_values(p: Params, h: int, alpha: np.ndarray, ybar: np.ndarray, Qh: np.ndarray,
+                   K_h: np.ndarray, V_h: np.ndarray, r2: np.ndarray, cos: list, anchor_pos: np.ndarray):
+    """Per-side ranking values (uK, uV) of one head under the selected criterion.
+
+    [PITH] "Circularity Check": the utility ranking is validated against
+    random, attention, residual-norm and cosine alternatives (Figure 5).
+    Readings (the alternatives are named, not defined):
+      utility        the first-order utility (``utilities``);
+      residual norm  ||r_t||^2 of the side;
+      attention      sum over observation rows of alpha_rt (the un-pooled
+                     observation score), the same for both sides;
+      cosine         1 - cos(x_t, x_a(t)) (worst-approximated first; a zero
+                     vector has cosine 0);
+      random         ``random_rank_key`` of the flat index f.
+    Anchors get 0 and are ineligible.  cos: per side, the true cosine of each
+    token with its assigned anchor.
+    """
+    N = K_h.shape[0]
+    H = p.n_kv_heads
+    if p.rank == RANK_UTILITY:
+        return utilities(alpha, ybar, Qh, V_h, r2[0], r2[1], anchor_pos)
+    out = []
+    for side in range(2):
+        if p.rank == RANK_RESIDUAL_NORM:
+            u = r2[side].copy()
+        elif p.rank == RANK_ATTENTION:
+            u = alpha.sum(axis=0)
+        elif p.rank == RANK_COSINE:
+            u = 1.0 - cos[side]
+        elif p.rank == RANK_RANDOM:
+            base = (side * H + h) * N
+            u = np.array([random_rank_key(p.seed, p.layer, base + t) for t in range(N)])
+        else:
+            raise ValueError("unknown ranking criterion")
+        u[anchor_pos] = 0.0
+        out.append(u)
+    return out[0], out[1]
+
+
+def assigned_cosine(X: np.ndarray, anchor_pos: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """cos(x_t, x_a(t)) = <x, a> / (||x|| ||a||), 0 when either norm is 0."""
+    xa = X[anchor_pos][idx]
+    den = np.sqrt((X * X).sum(axis=1) * (xa * xa).sum(axis=1))
+    dot = (X * xa).sum(axis=1)
+    return np.where(den > 0, dot / np.where(den > 0, den, 1.0), 0.0)
+
+
 # --------------------------------------------------------------------------
 # a5: per-layer residual budget, pooled over heads and sides
 # --------------------------------------------------------------------------
@@ -438,7 +531,7 @@ def select_residuals(u: np.ndarray, eligible: np.ndarray, R: int) -> np.ndarray:
 # a6: randomized Hadamard rotation + 2-bit Lloyd-Max quantization + packing
 # --------------------------------------------------------------------------
 
-def quantize_residuals(r: np.ndarray, seed: int, codebook=None):
+def quantize_residuals(r: np.ndarray, seed: int, codebook=None, naive: bool = False):
     """Encode residual rows r [n, D] to (sigma~ fp16 [n], codes [n, D] in 0..3).
 
     [PITH] Referee "Summary": 2-bit Hadamard-rotated, Lloyd-Max-quantized
@@ -448,15 +541,21 @@ def quantize_residuals(r: np.ndarray, seed: int, codebook=None):
     shared signs s; one fp16 scale sigma~ = fp16(||r|| / sqrt(D)) per residual
     vector (group = the whole head vector); code = 3 if y >= tau sigma~,
     2 if y >= 0, 1 if y >= -tau sigma~, else 0.
+    naive: the ablation of [PITH] Figure 5 ("Naive 2 bit", minor comments);
+    Reading: the same scale and codebook applied to r itself (no sign flip,
+    no rotation), y = r.
     Returns (sigma16, codes, y).
     """
     D = r.shape[1]
     if codebook is None:
         codebook = lloyd_max_gaussian_4()
     tau = codebook[0]
-    s = hadamard_signs(seed, D)
-    H = hadamard_matrix(D)
-    y = (r * s[None, :]) @ H.T
+    if naive:
+        y = r.copy()
+    else:
+        s = hadamard_signs(seed, D)
+        H = hadamard_matrix(D)
+        y = (r * s[None, :]) @ H.T
     sigma = np.sqrt((r * r).sum(axis=1) / D)
     sig16 = to_fp16(sigma)
     th = tau * sig16.astype(np.float64)[:, None]
@@ -464,14 +563,17 @@ def quantize_residuals(r: np.ndarray, seed: int, codebook=None):
     return sig16, codes.astype(np.uint8), y
 
 
-def dequantize_residuals(sig16: np.ndarray, codes: np.ndarray, seed: int, codebook=None):
-    """r~ = s * H_D (sigma~ * level(code)); H_D is symmetric and its own inverse."""
+def dequantize_residuals(sig16: np.ndarray, codes: np.ndarray, seed: int, codebook=None, naive: bool = False):
+    """r~ = s * H_D (sigma~ * level(code)); H_D is symmetric and its own inverse.
+    naive: r~ = sigma~ * level(code)."""
     D = codes.shape[1]
     if codebook is None:
         codebook = lloyd_max_gaussian_4()
     _, l1, l2, _ = codebook
     lev = np.array([-l2, -l1, l1, l2])
     z = lev[codes.astype(np.int64)] * sig16.astype(np.float64)[:, None]
+    if naive:
+        return z
     H = hadamard_matrix(D)
     return (z @ H.T) * hadamard_signs(seed, D)[None, :]
 
@@ -517,6 +619,8 @@ def compress_layer(K: np.ndarray, V: np.ndarray, Q: np.ndarray, p: Params,
     stages = stages or {}
     H, N, D = K.shape
     G, W = p.group, p.window
+    if p.key_queries:
+        Q = key_queries(K, p)
     L = layout(p)
     k = L["k"]
     out = dict(layout=L, anchor_pos=np.zeros((H, k), np.int64),
@@ -536,6 +640,7 @@ def compress_layer(K: np.ndarray, V: np.ndarray, Q: np.ndarray, p: Params,
         ap = np.asarray(ap, np.int64)
         out["anchor_pos"][h] = ap
         out["eligible"][:, h, ap] = False
+        acos = []
         for side, X in enumerate((K[h], V[h])):
             idx, _, cos = assign(X, ap)
             if "idx" in stages:
@@ -545,12 +650,13 @@ def compress_layer(K: np.ndarray, V: np.ndarray, Q: np.ndarray, p: Params,
             g, g16, r, r2 = project(X, ap, idx)
             out["gamma"][side, h], out["g16"][side, h] = g, g16
             out["r"][side, h], out["r2"][side, h] = r, r2
-        uK, uV = utilities(att["alpha"], att["ybar"], Qh, V[h], out["r2"][0, h], out["r2"][1, h], ap)
+            acos.append(assigned_cosine(X, ap, idx))
+        uK, uV = ranking_values(p, h, att["alpha"], att["ybar"], Qh, K[h], V[h], out["r2"][:, h], acos, ap)
         out["u"][0, h], out["u"][1, h] = uK, uV
     sel = stages["sel"] if "sel" in stages else select_residuals(out["u"], out["eligible"], L["R"])
     out["sel"] = np.asarray(sel, bool)
     rows = out["r"][out["sel"]]                         # flat (side, h, t) order
-    sig16, codes, y = quantize_residuals(rows, p.seed)
+    sig16, codes, y = quantize_residuals(rows, p.seed, naive=p.naive_codec)
     out["sigma16"], out["codes"], out["y"] = sig16, codes, y
     out["bytes"] = pack_layout(p, K, V, out)
     return out
@@ -651,7 +757,7 @@ def reconstruct(parts: dict, p: Params, identity_residuals: np.ndarray | None = 
     out = []
     res_rows = None
     if parts["codes"].shape[0]:
-        res_rows = dequantize_residuals(parts["sigma16"], parts["codes"], p.seed)
+        res_rows = dequantize_residuals(parts["sigma16"], parts["codes"], p.seed, naive=p.naive_codec)
     cursor = 0
     flat_sel = parts["sel"].reshape(-1)
     rec_of = np.cumsum(flat_sel) - 1                    # record index per token-side
