@@ -68,8 +68,39 @@ typedef struct anchorkv_params {
   int32_t rho_num;      /* scored share of the m slots = rho_num/rho_den (7)   */
   int32_t rho_den;      /* (10)                                                */
   int32_t pool_kernel;  /* kappa, odd, positional pooling width (7)            */
-  int32_t reserved;     /* must be 0                                           */
+  int32_t mode;         /* ANCHORKV_MODE_* bits; 0 = the method as published   */
 } anchorkv_params;
+
+/*
+ * Mode bits of anchorkv_params.mode (compress and decode of one layout must
+ * use the same mode):
+ *   ANCHORKV_MODE_KEY_QUERIES  Q_obs may be NULL; the trailing W keys of each
+ *       KV head serve as the observation queries of its query heads (VeloxQuant
+ *       "Adaptation notes": key-as-query proxy, since a cache wrapper never
+ *       sees queries).
+ *   bits 1..3 (ANCHORKV_MODE_RANK(r)): the criterion that ranks token-sides
+ *       for the residual budget; UTILITY is the method, the others are the
+ *       alternatives the review's "Circularity Check" names for the Figure 5
+ *       ablation: residual norm ||r||^2, attention (sum of the observation
+ *       weights), cosine (1 - cos(x, x_a)), random (a seeded hash of the flat
+ *       index).  Values above ANCHORKV_RANK_RANDOM are rejected (EINVAL).
+ *   ANCHORKV_MODE_NAIVE_CODEC  the 2-bit codec without the sign flip and
+ *       Hadamard rotation (the review's "Naive 2 bit" ablation).
+ * Any other bit set: EINVAL.
+ */
+#define ANCHORKV_MODE_KEY_QUERIES 0x1
+#define ANCHORKV_MODE_RANK_SHIFT 1
+#define ANCHORKV_MODE_RANK_MASK 0xE
+#define ANCHORKV_MODE_RANK(r) ((int32_t)(r) << ANCHORKV_MODE_RANK_SHIFT)
+#define ANCHORKV_MODE_NAIVE_CODEC 0x10
+#define ANCHORKV_MODE_ALL 0x1F
+enum anchorkv_rank {
+  ANCHORKV_RANK_UTILITY = 0,
+  ANCHORKV_RANK_RESIDUAL_NORM = 1,
+  ANCHORKV_RANK_ATTENTION = 2,
+  ANCHORKV_RANK_COSINE = 3,
+  ANCHORKV_RANK_RANDOM = 4
+};
 
 /*
  * Byte accounting of one compressed layer (review, Referee "Summary": an exact
@@ -143,7 +174,8 @@ int anchorkv_compress_workspace(const anchorkv_params* p, anchorkv_workspace_vie
  * per-layer top-R residual selection pooled over heads and sides, randomized
  * Hadamard rotation + 2-bit Lloyd-Max codes.
  *   K, V   device [H][N][D] dtype     prefill keys (pre-RoPE) and values
- *   Q_obs  device [H_q][W][D] dtype   queries of the last W positions
+ *   Q_obs  device [H_q][W][D] dtype   queries of the last W positions (may be
+ *          NULL with ANCHORKV_MODE_KEY_QUERIES)
  *   out    device, out_bytes >= anchorkv_layout.total_bytes
  *   ws     device, ws_bytes >= anchorkv_workspace_view.total_bytes; the call
  *          overwrites it (no state is carried between calls)

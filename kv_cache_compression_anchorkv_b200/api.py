@@ -15,6 +15,17 @@ import torch
 from . import capi
 
 _DT = {"fp32": capi.FP32, "bf16": capi.BF16}
+
+# anchorkv_params.mode bits (include/anchorkv.h)
+MODE_KEY_QUERIES = 0x1       # Q_obs may be None: the trailing W keys serve as the observation queries
+MODE_RANK_SHIFT = 1
+RANK_UTILITY, RANK_RESIDUAL_NORM, RANK_ATTENTION, RANK_COSINE, RANK_RANDOM = 0, 1, 2, 3, 4
+MODE_NAIVE_CODEC = 0x10      # 2-bit codec without the sign flip and Hadamard rotation
+
+
+def mode_bits(key_queries: bool = False, rank: int = RANK_UTILITY, naive_codec: bool = False) -> int:
+    """The anchorkv_params.mode value of a combination of options."""
+    return (MODE_KEY_QUERIES if key_queries else 0) | (rank << MODE_RANK_SHIFT) | (MODE_NAIVE_CODEC if naive_codec else 0)
 _TORCH_DT = {"fp32": torch.float32, "bf16": torch.bfloat16}
 
 
@@ -34,11 +45,12 @@ class AnchorKVParams:
     rho_num: int = 7
     rho_den: int = 10
     pool_kernel: int = 7
+    mode: int = 0                # mode_bits(...); compress and decode of one layout use the same
 
     def c(self) -> capi.Params:
         return capi.Params(self.n_tokens, self.head_dim, self.n_kv_heads, self.n_q_heads, self.window,
                            _DT[self.dtype], float(self.theta), self.seed, self.layer, self.anchor_div,
-                           self.rho_num, self.rho_den, self.pool_kernel, 0)
+                           self.rho_num, self.rho_den, self.pool_kernel, self.mode)
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -73,14 +85,16 @@ def _check_tensor(name, t, shape, dtype):
         raise ValueError(f"{name}: expected contiguous {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
 
 
-def compress(p: AnchorKVParams, K: torch.Tensor, V: torch.Tensor, Q_obs: torch.Tensor,
+def compress(p: AnchorKVParams, K: torch.Tensor, V: torch.Tensor, Q_obs: torch.Tensor | None,
              out: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
-    """Compress one layer.  K, V: [H, N, D]; Q_obs: [H_q, W, D] (CUDA, p.dtype).
+    """Compress one layer.  K, V: [H, N, D]; Q_obs: [H_q, W, D] (CUDA, p.dtype),
+    or None with the key-as-query mode.
     Returns (compressed uint8 tensor of layout.total_bytes, workspace)."""
     H, N, D, W = p.n_kv_heads, p.n_tokens, p.head_dim, p.window
     _check_tensor("K", K, (H, N, D), p.torch_dtype)
     _check_tensor("V", V, (H, N, D), p.torch_dtype)
-    _check_tensor("Q_obs", Q_obs, (p.n_q_heads, W, D), p.torch_dtype)
+    if Q_obs is not None or not (p.mode & MODE_KEY_QUERIES):
+        _check_tensor("Q_obs", Q_obs, (p.n_q_heads, W, D), p.torch_dtype)
     L = anchorkv_bytes(p)
     ws = compress_workspace(p)
     if out is None:

@@ -20,7 +20,7 @@ class Params(ctypes.Structure):
         ("n_q_heads", ctypes.c_int32), ("window", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("theta", ctypes.c_double), ("seed", ctypes.c_uint64), ("layer", ctypes.c_int32),
         ("anchor_div", ctypes.c_int32), ("rho_num", ctypes.c_int32), ("rho_den", ctypes.c_int32),
-        ("pool_kernel", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("pool_kernel", ctypes.c_int32), ("mode", ctypes.c_int32),
     ]
 
 

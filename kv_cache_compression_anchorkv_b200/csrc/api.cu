@@ -98,7 +98,9 @@ static int validate(const anchorkv_params* p) {
   if (!(p->theta > 0.0) || !isfinite(p->theta)) return ANCHORKV_EINVAL;
   if (p->anchor_div < 1 || p->rho_den < 1 || p->rho_num < 0 || p->rho_num > p->rho_den) return ANCHORKV_EINVAL;
   if (p->pool_kernel < 1 || !(p->pool_kernel & 1) || p->pool_kernel > 255) return ANCHORKV_EINVAL;
-  if (p->layer < 0 || p->layer > 32767 || p->reserved != 0) return ANCHORKV_EINVAL;
+  if (p->layer < 0 || p->layer > 32767) return ANCHORKV_EINVAL;
+  if (p->mode & ~ANCHORKV_MODE_ALL) return ANCHORKV_EINVAL;
+  if (((p->mode & ANCHORKV_MODE_RANK_MASK) >> ANCHORKV_MODE_RANK_SHIFT) > ANCHORKV_RANK_RANDOM) return ANCHORKV_EINVAL;
   if ((int64_t)2 * p->n_kv_heads * p->n_tokens > (int64_t)1 << 30) return ANCHORKV_EINVAL;
   return ANCHORKV_OK;
 }
@@ -174,6 +176,8 @@ int make_plan(const anchorkv_params* p, Plan* pl) {
   pl->o_tile_eq = take(4 * n_sh_t);
   pl->o_tie_before = take(4 * (n_sh_t + 1));
   pl->o_tile_cnt = take(4 * n_sh_t);
+  // proxy observation queries (key-as-query mode)
+  pl->o_qproxy = (p->mode & ANCHORKV_MODE_KEY_QUERIES) ? take((int64_t)pl->Hq * pl->W * kD * pl->elem) : 0;
   pl->ws_total = off;
   double mse;
   codebook(&pl->tau, &pl->l1, &pl->l2, &mse);
@@ -267,7 +271,8 @@ int anchorkv_compress(const anchorkv_params* p, const void* K, const void* V, co
   Plan pl;
   int st = make_plan(p, &pl);
   if (st) return st;
-  if (!K || !V || !Q_obs || !out || !ws) return ANCHORKV_EINVAL;
+  const bool key_queries = (p->mode & ANCHORKV_MODE_KEY_QUERIES) != 0;
+  if (!K || !V || (!Q_obs && !key_queries) || !out || !ws) return ANCHORKV_EINVAL;
   if ((int64_t)out_bytes < pl.L.total_bytes || (int64_t)ws_bytes < pl.ws_total) return ANCHORKV_ENOSPC;
   if (((uintptr_t)K | (uintptr_t)V | (uintptr_t)Q_obs | (uintptr_t)out | (uintptr_t)ws) & 15) return ANCHORKV_EINVAL;
   st = check_device();
@@ -276,6 +281,10 @@ int anchorkv_compress(const anchorkv_params* p, const void* K, const void* V, co
   char* o = (char*)out;
   char* w = (char*)ws;
   AKV_LAUNCH(cudaMemsetAsync(w + pl.o_counters, 0, 4 * (kCounterCount + 2 * (size_t)pl.H), s));
+  if (key_queries) {
+    AKV_LAUNCH(launch_key_queries(pl, K, w + pl.o_qproxy, s));
+    Q_obs = w + pl.o_qproxy;
+  }
 #define AKV_STAGE(st, nk, expr) \
   do { stage_begin(st, s); AKV_LAUNCH(expr); stage_end(st, s, nk); } while (0)
   if (use_tc_obs(pl)) {

@@ -59,12 +59,15 @@ __device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfloat16* p, fl
   }
 }
 
-template <typename T>
+// kUtility: the method's ranking (the other criteria, an ablation, share the
+// second instantiation and switch on `rank`).
+template <typename T, bool kUtility>
 __global__ void __launch_bounds__(256)
 project_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ anc_k,
                const T* __restrict__ anc_v, const double* __restrict__ anc_n2, const int* __restrict__ slot_of,
-               const float* __restrict__ a2s, const float* __restrict__ kus, uint32_t* __restrict__ tok,
-               float* __restrict__ util, int N, int H, int k, int obs_rb) {
+               const float* __restrict__ a2s, const float* __restrict__ kus, const float* __restrict__ score,
+               uint32_t* __restrict__ tok, float* __restrict__ util, int N, int H, int k, int obs_rb, int rank,
+               uint64_t seed, int layer) {
   constexpr int EPV = 16 / (int)sizeof(T);        // elements per 16-byte load
   constexpr int STEPS = kD / (4 * EPV);           // loads per lane and row
   const int q = threadIdx.x & 3;
@@ -104,14 +107,43 @@ project_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __rest
   float u;
   if (is_anchor) {
     u = -1.0f;
-  } else {
+  } else if (kUtility) {
     // sum of the observation-row-block partials, in order
     const float* src = side ? a2s : kus;
     float m = src[(int64_t)h * N + t];
     for (int rb = 1; rb < obs_rb; ++rb) m += src[((int64_t)rb * H + h) * N + t];
     u = side ? (float)(r2 * (double)m) : (float)(r2 / (double)(kD * kD) * (double)m);
+  } else if (rank == ANCHORKV_RANK_RESIDUAL_NORM) {
+    u = (float)r2;
+  } else if (rank == ANCHORKV_RANK_ATTENTION) {
+    // sum over the observation rows of alpha (row-block partials, in order)
+    float m = score[(int64_t)h * N + t];
+    for (int rb = 1; rb < obs_rb; ++rb) m += score[((int64_t)rb * H + h) * N + t];
+    u = m;
+  } else if (rank == ANCHORKV_RANK_COSINE) {
+    const double den = sqrt(nx * n2);
+    u = (float)(1.0 - (den > 0.0 ? dot / den : 0.0));
+  } else {
+    // a seeded uniform value of the flat index: the top 24 bits of SplitMix64
+    const uint64_t z = splitmix64(seed ^ kRankSalt ^ ((uint64_t)(layer & 0x7FFF) << 48) ^ (uint64_t)f);
+    u = (float)(z >> 40) * (1.0f / 16777216.0f);
   }
   util[f] = u;
+}
+
+// ---------------------------------------------------------------- key-as-query proxies
+
+// Q[j][w] = K[j / G][N - W + w]: the trailing window keys of each KV head as
+// the observation queries of its query heads (VeloxQuant "Adaptation notes",
+// key-as-query proxy).  One thread per 16 bytes.
+__global__ void key_query_kernel(const uint4* __restrict__ K, uint4* __restrict__ Q, int N, int W, int G,
+                                 int chunks_per_row, int64_t total) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= total) return;
+  const int64_t row = i / chunks_per_row;
+  const int c = (int)(i % chunks_per_row);
+  const int j = (int)(row / W), w = (int)(row % W);
+  Q[i] = K[((int64_t)(j / G) * N + (N - W + w)) * chunks_per_row + c];
 }
 
 // ---------------------------------------------------------------- quantize
@@ -159,7 +191,7 @@ __global__ void __launch_bounds__(256, 2) quantize_kernel(const T* __restrict__ 
                                 const uint32_t* __restrict__ tok, const uint32_t* __restrict__ bitmap,
                                 const int* __restrict__ tile_prefix, uint8_t* __restrict__ codes,
                                 uint16_t* __restrict__ sigma, int N, int H, int k, int n_tiles, int64_t R,
-                                int* __restrict__ counters, CodecConst cc) {
+                                int* __restrict__ counters, CodecConst cc, int naive) {
   const int lane = threadIdx.x & 31, grp = lane >> 3, l8 = lane & 7;
   const int n_words = 2 * H * n_tiles * 4;
   const int wid = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -209,37 +241,40 @@ __global__ void __launch_bounds__(256, 2) quantize_kernel(const T* __restrict__ 
     for (int e = 0; e < 16; ++e) {
       const double r = (double)xf[e] - g * (double)af[e];
       r2 = fma(r, r, r2);
-      y[e] = ((sgn >> e) & 1u) ? -r : r;
+      y[e] = (!naive && ((sgn >> e) & 1u)) ? -r : r;
     }
 #pragma unroll
     for (int m = 1; m < 8; m <<= 1) r2 += __shfl_xor_sync(0xffffffffu, r2, m);
-    // Hadamard transform (natural order): four stages on the element bits ...
+    if (!naive) {                             // (uniform per launch)
+      // Hadamard transform (natural order): four stages on the element bits ...
 #pragma unroll
-    for (int m = 1; m < 16; m <<= 1)
+      for (int m = 1; m < 16; m <<= 1)
 #pragma unroll
-      for (int e = 0; e < 16; ++e)
-        if (!(e & m)) {
-          const double a0 = y[e], a1 = y[e | m];
-          y[e] = a0 + a1;
-          y[e | m] = a0 - a1;
+        for (int e = 0; e < 16; ++e)
+          if (!(e & m)) {
+            const double a0 = y[e], a1 = y[e | m];
+            y[e] = a0 + a1;
+            y[e | m] = a0 - a1;
+          }
+      // ... and three on the lane bits
+#pragma unroll
+      for (int m = 1; m < 8; m <<= 1) {
+        const bool upper = l8 & m;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const double other = __shfl_xor_sync(0xffffffffu, y[e], m);
+          y[e] = upper ? (other - y[e]) : (y[e] + other);
         }
-    // ... and three on the lane bits
-#pragma unroll
-    for (int m = 1; m < 8; m <<= 1) {
-      const bool upper = l8 & m;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const double other = __shfl_xor_sync(0xffffffffu, y[e], m);
-        y[e] = upper ? (other - y[e]) : (y[e] + other);
       }
     }
     if (!live) continue;
     const uint16_t sb = half_bits_rn(sqrt(r2 / (double)kD));
     const double th = cc.tau * (double)half_bits_to_f(sb);
+    const double ysc = naive ? 1.0 : inv_sqrt_d;
     uint32_t word = 0;
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      const double v = y[e] * inv_sqrt_d;
+      const double v = y[e] * ysc;
       const uint32_t c = (v >= th) ? 3u : (v >= 0.0) ? 2u : (v >= -th) ? 1u : 0u;
       word |= c << (2 * e);
     }
@@ -252,7 +287,7 @@ __global__ void __launch_bounds__(256, 2) quantize_kernel(const T* __restrict__ 
 
 template <typename T>
 __global__ void reconstruct_kernel(const uint8_t* __restrict__ comp, anchorkv_layout L, int N, int H, int k,
-                                   CodecConst cc, float* __restrict__ Kh, float* __restrict__ Vh) {
+                                   CodecConst cc, int naive, float* __restrict__ Kh, float* __restrict__ Vh) {
   const int lane = threadIdx.x & 31;
   const int64_t total = 2LL * H * N;
   const int n_tiles = L.n_tiles;
@@ -287,12 +322,17 @@ __global__ void reconstruct_kernel(const uint8_t* __restrict__ comp, anchorkv_la
       float z[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) z[e] = lev[(byte >> (2 * e)) & 3u] * sg;
-      fwht128<float>(z);
-      const float isd = rsqrtf((float)kD);
+      if (naive) {                              // unrotated codec: r~ = sigma~ level(code)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float s = ((cc.sign_bits[(lane * 4 + e) >> 5] >> ((lane * 4 + e) & 31)) & 1u) ? -1.f : 1.f;
-        o[e] += s * z[e] * isd;
+        for (int e = 0; e < 4; ++e) o[e] += z[e];
+      } else {
+        fwht128<float>(z);
+        const float isd = rsqrtf((float)kD);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float s = ((cc.sign_bits[(lane * 4 + e) >> 5] >> ((lane * 4 + e) & 31)) & 1u) ? -1.f : 1.f;
+          o[e] += s * z[e] * isd;
+        }
       }
     }
     float* dst = (side ? Vh : Kh) + ((int64_t)h * N + t) * kD + lane * 4;
@@ -315,20 +355,33 @@ cudaError_t launch_project(const Plan& pl, const void* K, const void* V, char* o
   auto* slot_of = reinterpret_cast<const int*>(ws + pl.o_slot_of);
   auto* a2 = reinterpret_cast<const float*>(ws + pl.o_a2);
   auto* ku = reinterpret_cast<const float*>(ws + pl.o_ku);
+  auto* sc = reinterpret_cast<const float*>(ws + pl.o_score);
   auto* tok = reinterpret_cast<uint32_t*>(out + pl.L.off_tok);
   auto* util = reinterpret_cast<float*>(ws + pl.o_util);
+  const int rank = rank_of(pl);
+  auto go = [&](auto kern, auto tag) {
+    using T = decltype(tag);
+    kern<<<blocks, 256, 0, s>>>(static_cast<const T*>(K), static_cast<const T*>(V),
+                                reinterpret_cast<const T*>(out + pl.L.off_anchors_k),
+                                reinterpret_cast<const T*>(out + pl.L.off_anchors_v), n2, slot_of, a2, ku, sc, tok,
+                                util, pl.N, pl.H, pl.k, pl.obs_rb, rank, pl.p.seed, pl.p.layer);
+  };
   if (pl.p.dtype == ANCHORKV_BF16) {
-    project_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-        (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
-        reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_k),
-        reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_v), n2, slot_of, a2, ku, tok, util,
-        pl.N, pl.H, pl.k, pl.obs_rb);
+    if (rank == ANCHORKV_RANK_UTILITY) go(project_kernel<__nv_bfloat16, true>, __nv_bfloat16{});
+    else go(project_kernel<__nv_bfloat16, false>, __nv_bfloat16{});
   } else {
-    project_kernel<float><<<blocks, 256, 0, s>>>(
-        (const float*)K, (const float*)V, reinterpret_cast<const float*>(out + pl.L.off_anchors_k),
-        reinterpret_cast<const float*>(out + pl.L.off_anchors_v), n2, slot_of, a2, ku, tok, util,
-        pl.N, pl.H, pl.k, pl.obs_rb);
+    if (rank == ANCHORKV_RANK_UTILITY) go(project_kernel<float, true>, float{});
+    else go(project_kernel<float, false>, float{});
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_key_queries(const Plan& pl, const void* K, void* Q, cudaStream_t s) {
+  const int chunks = kD * pl.elem / 16;
+  const int64_t total = (int64_t)pl.Hq * pl.W * chunks;
+  const int blocks = (int)((total + 255) / 256);
+  key_query_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(K), static_cast<uint4*>(Q), pl.N, pl.W, pl.G,
+                                          chunks, total);
   return cudaGetLastError();
 }
 
@@ -347,12 +400,12 @@ cudaError_t launch_quantize(const Plan& pl, const void* K, const void* V, char* 
         (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
         reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_k),
         reinterpret_cast<const __nv_bfloat16*>(out + pl.L.off_anchors_v), tok, bitmap, prefix, codes, sigma,
-        pl.N, pl.H, pl.k, pl.n_tiles, pl.R, reinterpret_cast<int*>(ws + pl.o_counters), cc);
+        pl.N, pl.H, pl.k, pl.n_tiles, pl.R, reinterpret_cast<int*>(ws + pl.o_counters), cc, naive_codec(pl));
   } else {
     quantize_kernel<float><<<blocks, 256, 0, s>>>(
         (const float*)K, (const float*)V, reinterpret_cast<const float*>(out + pl.L.off_anchors_k),
         reinterpret_cast<const float*>(out + pl.L.off_anchors_v), tok, bitmap, prefix, codes, sigma,
-        pl.N, pl.H, pl.k, pl.n_tiles, pl.R, reinterpret_cast<int*>(ws + pl.o_counters), cc);
+        pl.N, pl.H, pl.k, pl.n_tiles, pl.R, reinterpret_cast<int*>(ws + pl.o_counters), cc, naive_codec(pl));
   }
   return cudaGetLastError();
 }
@@ -361,9 +414,11 @@ cudaError_t launch_reconstruct(const Plan& pl, const char* comp, float* Kh, floa
   const CodecConst cc = make_cc(pl);
   const int blocks = 148 * 8;
   if (pl.p.dtype == ANCHORKV_BF16)
-    reconstruct_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>((const uint8_t*)comp, pl.L, pl.N, pl.H, pl.k, cc, Kh, Vh);
+    reconstruct_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>((const uint8_t*)comp, pl.L, pl.N, pl.H, pl.k, cc,
+                                                             naive_codec(pl), Kh, Vh);
   else
-    reconstruct_kernel<float><<<blocks, 256, 0, s>>>((const uint8_t*)comp, pl.L, pl.N, pl.H, pl.k, cc, Kh, Vh);
+    reconstruct_kernel<float><<<blocks, 256, 0, s>>>((const uint8_t*)comp, pl.L, pl.N, pl.H, pl.k, cc,
+                                                     naive_codec(pl), Kh, Vh);
   return cudaGetLastError();
 }
 

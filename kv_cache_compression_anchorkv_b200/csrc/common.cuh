@@ -31,6 +31,10 @@ __device__ __forceinline__ void latch_error(int* counters, int code) {
   atomicCAS(&counters[kStatus], 0, code);
 }
 
+// Salt of the random residual ranking ("rank_rnd"), keeping its keys apart
+// from the uniform anchor sample's.
+constexpr uint64_t kRankSalt = 0x72616E6B5F726E64ull;
+
 // SplitMix64 output for state x (Steele, Lea & Flood, OOPSLA 2014).
 __host__ __device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
   uint64_t z = x + 0x9E3779B97F4A7C15ull;

@@ -39,6 +39,7 @@ struct DecodeArgs {
   float* pz;     // [b][h][split][G][D]
   float lev[4];
   uint32_t sign_bits[4];
+  int naive;     // unrotated codec: residuals live in the token domain
 };
 
 __device__ __forceinline__ float sgnf(const DecodeArgs& a, int j) {
@@ -74,10 +75,15 @@ __global__ void decode_prep_kernel(DecodeArgs a, const T* __restrict__ q) {
   if (blockIdx.x == 0) {
     for (int j = warp; j < a.G; j += blockDim.x >> 5) {
       float v[4];
+      float* dst = a.qrot + ((int64_t)bh * a.G + j) * kD + lane * 4;
+      if (a.naive) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[e] = qs[j][lane * 4 + e] * isd;
+        continue;
+      }
 #pragma unroll
       for (int e = 0; e < 4; ++e) v[e] = qs[j][lane * 4 + e] * sgnf(a, lane * 4 + e);
       fwht128<float>(v);
-      float* dst = a.qrot + ((int64_t)bh * a.G + j) * kD + lane * 4;
 #pragma unroll
       for (int e = 0; e < 4; ++e) dst[e] = v[e] * isd * isd;   // orthonormal H, then 1/sqrt(D)
     }
@@ -304,8 +310,8 @@ decode_combine_kernel(DecodeArgs a, const T* __restrict__ q, const T* __restrict
     zrot[j][i % kD] = z;
   }
   __syncthreads();
-  // rotate Z back: s . H(Z), one warp per head
-  for (int j = warp; j < G; j += 8) {
+  // rotate Z back: s . H(Z), one warp per head (not for the unrotated codec)
+  for (int j = warp; j < G && !a.naive; j += 8) {
     float v[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) v[e] = zrot[j][lane * 4 + e];
@@ -387,6 +393,7 @@ cudaError_t launch_decode(const Plan& pl, const DecodePlan& dp, const char* comp
   a.pz = reinterpret_cast<float*>(ws + dp.o_part_z);
   a.lev[0] = (float)-pl.l2; a.lev[1] = (float)-pl.l1; a.lev[2] = (float)pl.l1; a.lev[3] = (float)pl.l2;
   for (int i = 0; i < 4; ++i) a.sign_bits[i] = pl.sign_bits[i];
+  a.naive = naive_codec(pl);
   const int bh = dp.batch * pl.H;
   dim3 gp((pl.k + 31) / 32, bh);
   const size_t smem_split = sizeof(float) * ((size_t)2 * pl.G * pl.k + (size_t)pl.G * dp.split_tokens + 2 * pl.G * kD);

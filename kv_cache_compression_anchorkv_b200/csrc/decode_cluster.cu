@@ -71,6 +71,7 @@ struct CArgs {
   int64_t R;
   float lev[4];
   uint32_t sign_bits[4];
+  int naive;                 // unrotated codec: residuals live in the token domain
   const void* q;
   const void* Kt;
   const void* Vt;
@@ -316,11 +317,15 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         qs[j * kD + lane * 4 + e] = qf[j][e];
-        v[e] = qf[j][e] * sign_of(a, lane * 4 + e);
+        v[e] = a.naive ? qf[j][e] : qf[j][e] * sign_of(a, lane * 4 + e);
       }
-      fwht128<float>(v);
+      if (!a.naive) {                      // (uniform per launch)
+        fwht128<float>(v);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) qr[j * kD + lane * 4 + e] = v[e] * isd;
+        for (int e = 0; e < 4; ++e) v[e] *= isd;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) qr[j * kD + lane * 4 + e] = v[e];
     }
   }
   for (int base = s0 + warp; base < s1; base += kPB * kWarps) {
@@ -711,11 +716,15 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) decode_cluster_kern
     float zv[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) zv[e] = rbuf[jj * 2 * kD + lane * 4 + e];
-    fwht128<float>(zv);
+    if (!a.naive) {                        // rotate the value residuals back (uniform per launch)
+      fwht128<float>(zv);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) zv[e] *= isd * sign_of(a, lane * 4 + e);
+    }
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int d = lane * 4 + e;
-      ofin[j * kD + d] += zv[e] * isd * sign_of(a, d) + rbuf[jj * 2 * kD + kD + d];
+      ofin[j * kD + d] += zv[e] + rbuf[jj * 2 * kD + kD + d];
     }
   }
   __syncthreads();
@@ -880,6 +889,7 @@ int launch_decode_cluster(const Plan& pl, int batch, const char* comp, int64_t s
   a.R = pl.R;
   a.lev[0] = (float)-pl.l2; a.lev[1] = (float)-pl.l1; a.lev[2] = (float)pl.l1; a.lev[3] = (float)pl.l2;
   for (int i = 0; i < 4; ++i) a.sign_bits[i] = pl.sign_bits[i];
+  a.naive = naive_codec(pl);
   a.q = q; a.Kt = Kt; a.Vt = Vt; a.tail_len = tail_len; a.tail_cap = tail_cap; a.out = out;
   const int GP = gp_of(pl.G);
   stage_begin(kStDecodeCluster, s);

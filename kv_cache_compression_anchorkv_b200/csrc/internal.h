@@ -39,6 +39,7 @@ struct Plan {
   int64_t o_tc_pm2, o_tc_pl, o_tc_rm2, o_tc_riz, o_tc_rq2, o_tc_ry2, o_tc_py, o_tc_yh, o_tc_yl;
   int64_t o_score, o_a2, o_ku, o_pooled, o_slot_of, o_anc_n2, o_anc_inv, o_anc_sqrt, o_xnorm;
   int64_t o_util, o_refine, o_sel_state, o_hist, o_tile_gt, o_tile_eq, o_tie_before, o_tile_cnt;
+  int64_t o_qproxy;          // proxy observation queries [Hq][W][D] (key-as-query mode), else 0
   // codebook and Hadamard signs (bit j set: s_j = -1)
   double tau, l1, l2;
   uint32_t sign_bits[4];
@@ -75,6 +76,10 @@ bool obs_tc_supported(const Plan& pl);
 cudaError_t launch_project(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s);
 cudaError_t launch_select(const Plan& pl, char* out, char* ws, cudaStream_t s);
 cudaError_t launch_quantize(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s);
+cudaError_t launch_key_queries(const Plan& pl, const void* K, void* Q, cudaStream_t s);
+// mode bits of the plan's parameters
+inline int rank_of(const Plan& pl) { return (pl.p.mode & ANCHORKV_MODE_RANK_MASK) >> ANCHORKV_MODE_RANK_SHIFT; }
+inline int naive_codec(const Plan& pl) { return (pl.p.mode & ANCHORKV_MODE_NAIVE_CODEC) ? 1 : 0; }
 cudaError_t launch_decode(const Plan& pl, const DecodePlan& dp, const char* comp, int64_t stride,
                           const void* q, const void* Kt, const void* Vt, int tail_len, int tail_cap,
                           float* out, char* ws, cudaStream_t s);

@@ -32,12 +32,16 @@ EPS_FP64 = 1e-12
 def oracle_params(p: api.AnchorKVParams) -> O.Params:
     return O.Params(n_tokens=p.n_tokens, n_kv_heads=p.n_kv_heads, n_q_heads=p.n_q_heads, theta=p.theta,
                     head_dim=p.head_dim, window=p.window, dtype=p.dtype, seed=p.seed, layer=p.layer,
-                    anchor_div=p.anchor_div, rho_num=p.rho_num, rho_den=p.rho_den, pool_kernel=p.pool_kernel)
+                    anchor_div=p.anchor_div, rho_num=p.rho_num, rho_den=p.rho_den, pool_kernel=p.pool_kernel,
+                    mode=p.mode)
 
 
 def gpu_compress(p: api.AnchorKVParams, K: torch.Tensor, V: torch.Tensor, Q: torch.Tensor):
-    """Run the CUDA compress on (device copies of) K, V, Q; return host arrays."""
+    """Run the CUDA compress on (device copies of) K, V, Q; return host arrays.
+    With the key-as-query mode the library gets no queries at all."""
     Kd, Vd, Qd = (x.cuda() if x.device.type != "cuda" else x for x in (K, V, Q))
+    if p.mode & api.MODE_KEY_QUERIES:
+        Qd = None
     out, ws = api.compress(p, Kd, Vd, Qd)
     counters = api.read_status(ws)
     view = api.compress_workspace(p)
@@ -64,6 +68,8 @@ def check_compress(p: api.AnchorKVParams, K: np.ndarray, V: np.ndarray, Q: np.nd
     rep = dict(near_tie_scored=0, near_tie_slot=0, near_tie_gamma=0, near_tie_select=0, near_tie_code=0,
                exact_ties_slot=0, max_rel_pooled=0.0, max_rel_util=0.0)
     assert gpu_bytes.shape[0] == L["total"]
+    if po.key_queries:
+        Q = O.key_queries(K, po)
     g = O.unpack_layout(gpu_bytes, po)
     eligible = np.ones((2, H, N), bool)
     att = []
@@ -100,6 +106,7 @@ def check_compress(p: api.AnchorKVParams, K: np.ndarray, V: np.ndarray, Q: np.nd
     # nearest-anchor slot and coefficient, per side
     r2 = np.zeros((2, H, N))
     r_all = np.zeros((2, H, N, D))
+    acos = np.zeros((2, H, N))
     for h in range(H):
         ap = g["anchor_pos"][h]
         for side, X in enumerate((K[h], V[h])):
@@ -129,11 +136,13 @@ def check_compress(p: api.AnchorKVParams, K: np.ndarray, V: np.ndarray, Q: np.nd
             r[ap] = 0.0
             r_all[side, h] = r
             r2[side, h] = (r * r).sum(axis=1)
-    # utilities (oracle formula on the GPU's decisions)
+            acos[side, h] = O.assigned_cosine(X, ap, idx_g)
+    # ranking values (the oracle's criterion for the mode, on the GPU's decisions)
     u_o = np.zeros((2, H, N))
     for h in range(H):
         Qh, a = att[h]
-        uK, uV = O.utilities(a["alpha"], a["ybar"], Qh, V[h], r2[0, h], r2[1, h], g["anchor_pos"][h])
+        uK, uV = O.ranking_values(po, h, a["alpha"], a["ybar"], Qh, K[h], V[h], r2[:, h], list(acos[:, h]),
+                                  g["anchor_pos"][h])
         u_o[0, h], u_o[1, h] = uK, uV
     assert np.all(gpu_util[~eligible] == -1.0)
     el = eligible
@@ -171,7 +180,7 @@ def check_compress(p: api.AnchorKVParams, K: np.ndarray, V: np.ndarray, Q: np.nd
     # residual codes and scales for the GPU-selected rows, in record order
     if R:
         rows = r_all[g["sel"]]
-        sig_o, codes_o, y = O.quantize_residuals(rows, p.seed)
+        sig_o, codes_o, y = O.quantize_residuals(rows, p.seed, naive=po.naive_codec)
         assert np.array_equal(sig_o.view(np.uint16), g["sigma16"].view(np.uint16)), "residual scales"
         badc = np.argwhere(codes_o != g["codes"])
         tau = O.lloyd_max_gaussian_4()[0]

@@ -49,7 +49,8 @@ def test_byte_accounting_matches_oracle(N, H, Hq, theta, dtype):
 @pytest.mark.parametrize("field,value", [
     ("head_dim", 64), ("n_kv_heads", 0), ("n_q_heads", 12), ("window", 0), ("n_tokens", 32),
     ("theta", 0.0), ("theta", float("nan")), ("theta", -1.0), ("pool_kernel", 6), ("rho_num", 11),
-    ("layer", -1), ("anchor_div", 0)])
+    ("layer", -1), ("anchor_div", 0), ("mode", 0x20), ("mode", api.mode_bits(rank=5)),
+    ("mode", api.mode_bits(rank=7)), ("mode", -1)])
 def test_invalid_params_rejected(field, value):
     p = api.AnchorKVParams(n_tokens=1024, n_kv_heads=8, n_q_heads=32)
     setattr(p, field, value)
@@ -111,3 +112,39 @@ def test_recorded_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
     h = hashlib.sha256(b"kernel v2\n").hexdigest()
     (tmp_path / "profiles" / "traffic.txt").write_text(f"stage_x kern 123 k.cu {h} cap.md\n")
     assert bench.recorded_traffic("stage_x") == 123
+
+
+def test_mode_bits_match_header():
+    text = open(capi.HEADER).read()
+    for name, val in [("ANCHORKV_MODE_KEY_QUERIES", api.MODE_KEY_QUERIES), ("ANCHORKV_MODE_NAIVE_CODEC", api.MODE_NAIVE_CODEC),
+                      ("ANCHORKV_MODE_RANK_SHIFT", api.MODE_RANK_SHIFT)]:
+        assert f"#define {name} {val:#x}" in text or f"#define {name} {val}" in text, name
+    for name, val in [("ANCHORKV_RANK_RESIDUAL_NORM", api.RANK_RESIDUAL_NORM), ("ANCHORKV_RANK_ATTENTION", api.RANK_ATTENTION),
+                      ("ANCHORKV_RANK_COSINE", api.RANK_COSINE), ("ANCHORKV_RANK_RANDOM", api.RANK_RANDOM)]:
+        assert f"{name} = {val}" in text, name
+    assert api.mode_bits(True, api.RANK_RANDOM, True) == 0x1 | (4 << 1) | 0x10
+    assert api.mode_bits(True, api.RANK_RANDOM, True) == O.MODE_KEY_QUERIES | (O.RANK_RANDOM << O.MODE_RANK_SHIFT) | O.MODE_NAIVE_CODEC
+
+
+def test_every_valid_mode_is_accepted():
+    for mode in range(0x20):
+        p = api.AnchorKVParams(n_tokens=1024, mode=mode)
+        rank = (mode >> 1) & 7
+        if rank > api.RANK_RANDOM:
+            with pytest.raises(capi.AnchorKVError):
+                api.anchorkv_bytes(p)
+        else:
+            assert api.anchorkv_bytes(p)["total_bytes"] > 0
+
+
+def test_queries_are_optional_only_with_key_queries():
+    """Q_obs = NULL is EINVAL unless the key-as-query mode is set; then the
+    proxy queries take workspace (size check first: never dereferenced)."""
+    L = capi.lib()
+    fake = ctypes.c_void_p(1 << 20)
+    p = api.AnchorKVParams(n_tokens=1024).c()
+    assert L.anchorkv_compress(ctypes.byref(p), fake, fake, None, fake, 1 << 40, fake, 1 << 40, None) == capi.EINVAL
+    pk = api.AnchorKVParams(n_tokens=1024, mode=api.MODE_KEY_QUERIES)
+    assert L.anchorkv_compress(ctypes.byref(pk.c()), fake, fake, None, fake, 16, fake, 16, None) == capi.ENOSPC
+    base = api.compress_workspace(api.AnchorKVParams(n_tokens=1024))["total_bytes"]
+    assert api.compress_workspace(pk)["total_bytes"] >= base + 32 * 32 * 128 * 2

@@ -198,3 +198,70 @@ def test_simt_observation_path_parity(name, monkeypatch):
     assert counters[0] == 0
     rep = parity.check_compress(p, _f64(K), _f64(V), _f64(Q), gb, gpool, gutil)
     print(name, "simt observation passes", rep)
+
+
+# optional modes: key-as-query proxies, the alternative rankings, the unrotated codec
+MODE_CASES = [
+    ("bf16-ragged-n3000", api.mode_bits(key_queries=True)),
+    ("fp32-window8-n700", api.mode_bits(key_queries=True)),
+    ("bf16-ragged-n3000", api.mode_bits(rank=api.RANK_RESIDUAL_NORM)),
+    ("bf16-gqa8-n2500", api.mode_bits(rank=api.RANK_ATTENTION)),
+    ("tiny-fp32-n1024", api.mode_bits(rank=api.RANK_ATTENTION)),
+    ("bf16-ragged-n3000", api.mode_bits(rank=api.RANK_COSINE)),
+    ("bf16-n20000", api.mode_bits(rank=api.RANK_RANDOM)),
+    ("bf16-ragged-n3000", api.mode_bits(naive_codec=True)),
+    ("tiny-fp32-n1024", api.mode_bits(naive_codec=True)),
+    ("bf16-gqa16-n1500", api.mode_bits(key_queries=True, rank=api.RANK_COSINE, naive_codec=True)),
+]
+
+
+@pytest.mark.parametrize("name,mode", MODE_CASES)
+def test_compress_modes(name, mode):
+    spec, theta = CASES[name]
+    K, V, Q = make_layer(spec, 0)
+    p = _params(spec, theta, layer=2)
+    p.mode = mode
+    gb, gpool, gutil, counters = parity.gpu_compress(p, K, V, Q)
+    assert counters[0] == 0
+    rep = parity.check_compress(p, _f64(K), _f64(V), _f64(Q), gb, gpool, gutil)
+    print(name, hex(mode), rep)
+
+
+@pytest.mark.parametrize("name,batch,tail", [("bf16-ragged-n3000", 2, 5), ("tiny-fp32-n1024", 1, 0),
+                                             ("bf16-gqa16-n1500", 2, 3), ("bf16-n20000", 1, 700)])
+def test_decode_naive_codec(name, batch, tail):
+    """Decode of layouts written with the unrotated codec (cluster path for
+    G <= 8, split-token path for G = 16)."""
+    spec, theta = CASES[name]
+    p = _params(spec, theta)
+    p.mode = api.mode_bits(naive_codec=True)
+    L = api.anchorkv_bytes(p)
+    stride = (L["total_bytes"] + 255) // 256 * 256
+    comp = torch.zeros(batch, stride, dtype=torch.uint8, device="cuda")
+    layouts = []
+    for b in range(batch):
+        sb = CacheSpec(**{**spec.__dict__, "seed": spec.seed + 50 * b})
+        K, V, Q = make_layer(sb, 0)
+        out, _ = api.compress(p, K.cuda(), V.cuda(), Q.cuda())
+        comp[b, :L["total_bytes"]] = out
+        layouts.append(out.cpu().numpy())
+    q = make_decode_queries(spec, 0, step=0, batch=batch)
+    cap = max(tail, 1) + 3
+    Kt, Vt = make_tail(spec, 0, cap, batch=batch)
+    o = api.decode_attn(p, comp, q.cuda(), Kt.cuda(), Vt.cuda(), tail_len=tail)
+    err = parity.check_decode(p, layouts, _f64(q), _f64(Kt), _f64(Vt), tail, o.cpu().double().numpy(),
+                              DECODE_TOL[spec.dtype])
+    print(name, "naive codec", batch, tail, "max abs err", err)
+
+
+def test_reconstruct_naive_codec():
+    spec, theta = CASES["bf16-ragged-n3000"]
+    K, V, Q = make_layer(spec, 0)
+    p = _params(spec, theta)
+    p.mode = api.mode_bits(naive_codec=True)
+    out, _ = api.compress(p, K.cuda(), V.cuda(), Q.cuda())
+    Kh, Vh = api.reconstruct(p, out)
+    po = parity.oracle_params(p)
+    Ko, Vo = O.reconstruct(O.unpack_layout(out.cpu().numpy(), po), po)
+    assert np.abs(Kh.cpu().double().numpy() - Ko).max() < 1e-5 * np.abs(Ko).max()
+    assert np.abs(Vh.cpu().double().numpy() - Vo).max() < 1e-5 * np.abs(Vo).max()
