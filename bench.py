@@ -8,6 +8,9 @@ cache (32 layers, 8 KV / 32 query heads, D = 128, N = 32768 tokens, bf16,
 theta = 0.05).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl anchorkv|reference]
+        python bench.py --sweep      (theta/length sweep of one 8B-shaped layer:
+                                      counts, speed, Theorem-1 bound vs measured
+                                      output error, ranking and codec ablations)
 Under torchrun (N > 1) every rank compresses its own independent cache (weak
 scaling, no collective on the data path); the timed region is bracketed by a
 barrier and device synchronisation and its duration is the max over ranks.
@@ -226,7 +229,12 @@ def main():
     ap.add_argument("--layers", type=int, default=0, help="compress only the first L layers (profiling runs)")
     ap.add_argument("--compress-streams", type=int, default=4,
                     help="compress layers round-robin on this many streams (independent layers overlap)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="theta/length sweep with output error vs the Theorem-1 bound and the ablations "
+                         "(one JSON line per point; not the benchmark line)")
     args = ap.parse_args()
+    if args.sweep:
+        return run_sweep(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -236,6 +244,118 @@ def main():
             return 0
         return run_reference(args)
     return run_gpu(args, world, rank, local)
+
+
+# ---------------------------------------------------------------- sweep and ablations
+
+def _output_error(p, comp, K, V, n_queries, seed):
+    """Output error of the compressed cache on n_queries N(0, I) queries per
+    KV head and the two Theorem-1 bounds (review, "What carries the argument",
+    Eq. 17: ||y^ - y|| <= sum_t alpha_t ||V^_t - V_t|| + 2 V_max tanh(mu),
+    mu = ||q|| max_t ||K_t - K^_t|| / sqrt(D); both pairings of weights and
+    V_max are provable and both are checked).  y^ comes from the library's
+    decode kernel on the compressed bytes; the exact attention and the bound
+    terms are evaluated in fp64 with torch (evaluation only)."""
+    import torch
+    from kv_cache_compression_anchorkv_b200 import api
+    from kv_cache_compression_anchorkv_b200.synthetic import gaussian_queries
+    H, Hq, D = p.n_kv_heads, p.n_q_heads, p.head_dim
+    G = Hq // H
+    dev = K.device
+    Kh, Vh = api.reconstruct(p, comp)
+    qs = gaussian_queries(H * n_queries, D, seed, device=dev).reshape(H, n_queries, D)
+    # the decode kernel takes Hq queries per call: G per KV head
+    yhat = torch.empty(H, n_queries, D, dtype=torch.float64, device=dev)
+    for c in range(0, n_queries, G):
+        q = qs[:, c:c + G].reshape(1, Hq, D).to(p.torch_dtype)
+        o = api.decode_attn(p, comp, q)
+        yhat[:, c:c + G] = o.reshape(H, G, D).double()
+    qd = qs.to(p.torch_dtype).double()          # the queries the kernel saw
+    err, rel, ba, bb, dks = [], [], [], [], []
+    for h in range(H):
+        k, v = K[h].double(), V[h].double()
+        kh, vh = Kh[h].double(), Vh[h].double()
+        dK = (k - kh).norm(dim=1).max()
+        dV = (v - vh).norm(dim=1)
+        vmax, vhmax = v.norm(dim=1).max(), vh.norm(dim=1).max()
+        a = torch.softmax(qd[h] @ k.T / D ** 0.5, dim=1)
+        ah = torch.softmax(qd[h] @ kh.T / D ** 0.5, dim=1)
+        y = a @ v
+        mu = qd[h].norm(dim=1) * dK / D ** 0.5
+        e = (yhat[h] - y).norm(dim=1)
+        err.append(e)
+        rel.append(e / y.norm(dim=1))
+        ba.append(ah @ dV + 2 * vmax * torch.tanh(mu))
+        bb.append(a @ dV + 2 * vhmax * torch.tanh(mu))
+        dks.append(float(dK))
+    err, rel, ba, bb = (torch.cat(x) for x in (err, rel, ba, bb))
+    bound = torch.minimum(ba, bb)
+    return {"queries": int(err.numel()), "err_mean": float(err.mean()), "err_max": float(err.max()),
+            "rel_err_mean": float(rel.mean()), "bound_a_mean": float(ba.mean()), "bound_b_mean": float(bb.mean()),
+            "bound_holds": float(((err <= ba) & (err <= bb)).double().mean()),
+            "err_over_bound_max": float((err / bound).max()), "max_key_error": max(dks)}
+
+
+def _time_ms(fn, reps, warm=2):
+    import torch
+    for _ in range(warm):
+        fn()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def run_sweep(args):
+    """Theta/length sweep of one 8B-shaped layer (8 KV / 32 query heads,
+    D = 128, bf16, window 32; N in {8K, 32K, 128K} x theta in {0.05, 0.1,
+    0.2}): anchor and residual counts, compress Mtok/s per layer-head, decode
+    at batch 1 (µs, GB/s over the compressed bytes), and the Theorem-1 bound
+    vs the measured output error on 256 N(0, I) queries per KV head.  Then,
+    at N = 32768 and theta = 0.05, the same error for every residual ranking
+    criterion and for the unrotated codec (the ablation of the review's
+    Figure 5).  Synthetic data as in the benchmark; one JSON line per point."""
+    import torch
+    from kv_cache_compression_anchorkv_b200 import api
+    from kv_cache_compression_anchorkv_b200.synthetic import CacheSpec, make_decode_queries, make_layer
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    n_queries = 256
+
+    def point(N, theta, mode, tag):
+        spec = CacheSpec(1, 8, 32, N, n_dirs=128, seed=0)
+        K, V, Q = make_layer(spec, 0, device=dev)
+        p = api.AnchorKVParams(n_tokens=N, n_kv_heads=8, n_q_heads=32, theta=theta, mode=mode)
+        L = api.anchorkv_bytes(p)
+        out, ws = api.compress(p, K, V, Q)
+        ms = _time_ms(lambda: api.compress(p, K, V, Q, out=out, workspace=ws), reps=5)
+        q = make_decode_queries(spec, 0, step=0, batch=1, device=dev)
+        dec_ms = _time_ms(lambda: api.decode_attn(p, out, q), reps=20)
+        st = api.read_status(ws)
+        line = {"sweep": tag, "n_tokens": N, "theta": theta, "mode": mode, "anchors": L["n_anchors"],
+                "residuals": L["n_residuals"], "residual_share": L["n_residuals"] / (2 * 8 * N),
+                "compressed_bytes": L["total_bytes"], "ratio": L["uncompressed_bytes"] / L["total_bytes"],
+                "compress_mtok_s_per_layer_head": 8 * N / (ms * 1e-3) / 1e6, "compress_ms": ms,
+                "decode_us": dec_ms * 1e3, "decode_gbs": L["total_bytes"] / (dec_ms * 1e-3) / 1e9,
+                "refined_rows": st[1]}
+        line.update(_output_error(p, out, K, V, n_queries, seed=1000 + N))
+        print(json.dumps(line), flush=True)
+
+    for N in (8192, 32768, 131072):
+        for theta in (0.05, 0.1, 0.2):
+            point(N, theta, 0, "theta-length")
+    for name, mode in [("utility", 0), ("residual-norm", api.mode_bits(rank=api.RANK_RESIDUAL_NORM)),
+                       ("attention", api.mode_bits(rank=api.RANK_ATTENTION)),
+                       ("cosine", api.mode_bits(rank=api.RANK_COSINE)),
+                       ("random", api.mode_bits(rank=api.RANK_RANDOM)),
+                       ("naive-2bit", api.mode_bits(naive_codec=True)),
+                       ("key-queries", api.mode_bits(key_queries=True))]:
+        point(32768, 0.05, mode, "ablation:" + name)
+    return 0
 
 
 # ---------------------------------------------------------------- oracle (CPU) arm

@@ -121,8 +121,11 @@ def decode_attn(p: AnchorKVParams, compressed: torch.Tensor, q: torch.Tensor,
     row) or [total_bytes]; q: [batch, H_q, D]; tails [batch, H, T_cap, D].
     Returns fp32 [batch, H_q, D]."""
     if compressed.dim() == 1:
-        compressed = compressed[None]
-    batch, stride = compressed.shape
+        # one layout: the stride never steps to a second sequence, it only has
+        # to satisfy the ABI (>= total bytes, a multiple of 16)
+        batch, stride = 1, (compressed.numel() + 15) // 16 * 16
+    else:
+        batch, stride = compressed.shape
     _check_tensor("q", q, (batch, p.n_q_heads, p.head_dim), p.torch_dtype)
     cap = 0
     if K_tail is not None:
@@ -163,8 +166,11 @@ def decode_attn_noalloc(p: AnchorKVParams, compressed: torch.Tensor, q: torch.Te
     on the GPU share the scratch and race; sizes whose decode workspace
     exceeds NOALLOC_SCRATCH_BYTES raise (ANCHORKV_ENOSPC)."""
     if compressed.dim() == 1:
-        compressed = compressed[None]
-    batch, stride = compressed.shape
+        # one layout: the stride never steps to a second sequence, it only has
+        # to satisfy the ABI (>= total bytes, a multiple of 16)
+        batch, stride = 1, (compressed.numel() + 15) // 16 * 16
+    else:
+        batch, stride = compressed.shape
     _check_tensor("q", q, (batch, p.n_q_heads, p.head_dim), p.torch_dtype)
     _check_tensor("out", out, (batch, p.n_q_heads, p.head_dim), torch.float32)
     cap = 0
