@@ -178,6 +178,7 @@ int make_plan(const anchorkv_params* p, Plan* pl) {
   pl->o_tile_cnt = take(4 * n_sh_t);
   // proxy observation queries (key-as-query mode)
   pl->o_qproxy = (p->mode & ANCHORKV_MODE_KEY_QUERIES) ? take((int64_t)pl->Hq * pl->W * kD * pl->elem) : 0;
+  pl->o_asg_keys = pl->k > kAssignGroupMax ? take(16 * 2 * H * N) : 0;
   pl->ws_total = off;
   double mse;
   codebook(&pl->tau, &pl->l1, &pl->l2, &mse);

@@ -22,6 +22,13 @@
 // accumulation error bound are listed for the fp64 re-decision shared with
 // the SIMT path.
 //
+// More anchors than fit in shared memory (k > kMaxKpad) are taken in groups
+// of at most kMaxKpad, one launch per group: each group's best two keys of a
+// row are widened to 64 bits (score grid index, then the inverted global
+// slot, so the order is still (score, -slot)) and merged with the previous
+// groups' through the workspace; the last group decides.  Every group uses
+// the row's same key grid, so keys of different groups compare exactly.
+//
 // Warp roles (one CTA per SM, persistent over (side, head, 128-row tile)
 // work items): warp 0 issues TMA, warp 1 owns TMEM and issues MMAs, the
 // other warps run the epilogue as kGroups groups of four warps that take
@@ -59,6 +66,8 @@ constexpr int kMaxKpad = 480;
 
 struct TcArgs {
   int N, H, k, kp16, cw, n_chunks, kpad, stages, row_tiles, nbuf;
+  int g0, gk, first, last;      // this launch's anchor group: slots [g0, g0 + gk)
+  ulonglong2* keys;             // [2][H][N] best two 64-bit keys after earlier groups
   int total_items;
   const float* anc_inv;
   const int* slot_of;
@@ -271,7 +280,7 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
           const CUtensorMap* mA = side ? &mapAV : &mapAK;
           for (int c = 0; c < a.n_chunks; ++c)
             for (int kh = 0; kh < 2; ++kh)
-              tc::tma_load_2d(anc + (size_t)(c * 2 + kh) * a.cw * 128, mA, kh * 64, h * a.k + c * a.cw,
+              tc::tma_load_2d(anc + (size_t)(c * 2 + kh) * a.cw * 128, mA, kh * 64, h * a.k + a.g0 + c * a.cw,
                               &ctl.anc_full);
           cur_u = u;
           ++anc_loads;
@@ -366,7 +375,7 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
       if (u != cur_u) {
         __syncwarp();
         const float* src = a.anc_inv + (int64_t)u * a.kp16;
-        for (int i = lane; i < a.kpad; i += 32) inv[i] = (i < a.kp16) ? src[i] : 0.f;
+        for (int i = lane; i < a.kpad; i += 32) inv[i] = (i < a.gk) ? src[a.g0 + i] : 0.f;
         __syncwarp();
         cur_u = u;
       }
@@ -385,7 +394,7 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
         }
         tc::fence_after_sync();
         const uint32_t tbase = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(b * a.cw);
-        Keys2 ca = scan_chunk(tbase, inv + c * a.cw, rk.add, min(a.cw, a.k - c * a.cw));
+        Keys2 ca = scan_chunk(tbase, inv + c * a.cw, rk.add, min(a.cw, a.gk - c * a.cw));
         tc::fence_before_sync();
         tc::mbar_arrive(&ctl.acc_empty[b]);
         // column in chunk -> slot: the low 9 bits drop by c cw (no borrow, slot < 512)
@@ -397,15 +406,32 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
       }
       if (!ok) break;
       if (t < a.N) {
-        uint32_t slot;
-        if (own >= 0) {
-          slot = (uint32_t)own;
-        } else {
-          slot = key_slot(ka.b1);
-          const float gap = (float)((ka.b1 >> 9) - (ka.b2 >> 9)) * rk.step;
-          if (!(gap > kRefineRelTC * xn)) list_for_refine(a.refine, a.counters, u, a.N, t);
+        // 64-bit keys: grid index, then ~(global slot); 0 = none
+        auto wide = [&](uint32_t k32) -> uint64_t {
+          return k32 ? ((uint64_t)(k32 >> 9) << 32) | (uint32_t)~(uint32_t)(a.g0 + key_slot(k32)) : 0ull;
+        };
+        uint64_t b1 = wide(ka.b1), b2 = wide(ka.b2);
+        if (!a.first) {
+          const ulonglong2 pv = a.keys[f];
+          const uint64_t p1 = pv.x, p2 = pv.y;
+          auto mx = [](uint64_t x, uint64_t y) { return x > y ? x : y; };
+          const uint64_t n1 = mx(b1, p1), n2 = mx(mx(b2, p2), b1 < p1 ? b1 : p1);
+          b1 = n1;
+          b2 = n2;
         }
-        a.tok[f] = slot;
+        if (!a.last) {
+          a.keys[f] = make_ulonglong2((unsigned long long)b1, (unsigned long long)b2);
+        } else {
+          uint32_t slot;
+          if (own >= 0) {
+            slot = (uint32_t)own;
+          } else {
+            slot = ~(uint32_t)b1;
+            const float gap = (float)((uint32_t)(b1 >> 32) - (uint32_t)(b2 >> 32)) * rk.step;
+            if (!(gap > kRefineRelTC * xn)) list_for_refine(a.refine, a.counters, u, a.N, t);
+          }
+          a.tok[f] = slot;
+        }
       }
     }
   }
@@ -446,44 +472,56 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
 
 }  // namespace
 
-bool assign_tc_supported(const Plan& pl) {
-  if (pl.p.dtype != ANCHORKV_BF16) return false;
-  const int n_chunks = (pl.k + kChunkMax - 1) / kChunkMax;
-  const int cw = ((pl.k + n_chunks - 1) / n_chunks + 15) / 16 * 16;
-  return n_chunks * cw <= kMaxKpad && encode_fn() != nullptr;
-}
+static_assert(kAssignGroupMax == kMaxKpad, "the plan's anchor groups are the kernel's resident anchor limit");
 
+bool assign_tc_supported(const Plan& pl) { return pl.p.dtype == ANCHORKV_BF16 && encode_fn() != nullptr; }
+
+// One launch per anchor group (a single one when k <= kMaxKpad); groups of
+// equal size, each split into chunks of at most kChunkMax anchors.
 cudaError_t launch_assign_tc(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s) {
-  TcArgs a;
-  a.N = pl.N; a.H = pl.H; a.k = pl.k; a.kp16 = pl.kp16;
-  a.n_chunks = (pl.k + kChunkMax - 1) / kChunkMax;
-  a.cw = ((pl.k + a.n_chunks - 1) / a.n_chunks + 15) / 16 * 16;
-  a.kpad = a.n_chunks * a.cw;
-  a.nbuf = std::min(kMaxBuf, 512 / a.cw);
-  a.row_tiles = (pl.N + 127) / 128;
-  a.total_items = 2 * pl.H * a.row_tiles;
-  const int fixed = 1024 + (int)sizeof(Ctl) + 16 + kEpiWarps * a.kpad * 4 + a.kpad * 256;
-  a.stages = std::min(4, (227 * 1024 - fixed) / kXStageBytes);
-  if (a.stages < 2) return cudaErrorInvalidValue;
-  a.anc_inv = reinterpret_cast<const float*>(ws + pl.o_anc_inv);
-  a.slot_of = reinterpret_cast<const int*>(ws + pl.o_slot_of);
-  a.xnorm = reinterpret_cast<const float*>(ws + pl.o_xnorm);
-  a.tok = reinterpret_cast<uint32_t*>(out + pl.L.off_tok);
-  a.refine = reinterpret_cast<int*>(ws + pl.o_refine);
-  a.counters = reinterpret_cast<int*>(ws + pl.o_counters);
-  CUtensorMap mXK, mXV, mAK, mAV;
-  const int64_t HN = (int64_t)pl.H * pl.N, Hk = (int64_t)pl.H * pl.k;
-  if (!make_map(&mXK, K, HN, 128) || !make_map(&mXV, V, HN, 128) ||
-      !make_map(&mAK, out + pl.L.off_anchors_k, Hk, a.cw) || !make_map(&mAV, out + pl.L.off_anchors_v, Hk, a.cw))
-    return cudaErrorInvalidValue;
-  const int smem = fixed + a.stages * kXStageBytes;
+  const int n_groups = (pl.k + kMaxKpad - 1) / kMaxKpad;
+  const int gsize = ((pl.k + n_groups - 1) / n_groups + 15) / 16 * 16;
   int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = std::min(sms, a.total_items);
-  cudaFuncSetAttribute(assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  assign_tc_kernel<<<grid, kThreads, smem, s>>>(mXK, mXV, mAK, mAV, a);
-  return cudaGetLastError();
+  CUtensorMap mXK, mXV;
+  const int64_t HN = (int64_t)pl.H * pl.N, Hk = (int64_t)pl.H * pl.k;
+  if (!make_map(&mXK, K, HN, 128) || !make_map(&mXV, V, HN, 128)) return cudaErrorInvalidValue;
+  for (int g = 0; g < n_groups; ++g) {
+    TcArgs a;
+    a.N = pl.N; a.H = pl.H; a.k = pl.k; a.kp16 = pl.kp16;
+    a.g0 = g * gsize;
+    a.gk = std::min(gsize, pl.k - a.g0);
+    a.first = g == 0;
+    a.last = g == n_groups - 1;
+    a.keys = n_groups > 1 ? reinterpret_cast<ulonglong2*>(ws + pl.o_asg_keys) : nullptr;
+    a.n_chunks = (a.gk + kChunkMax - 1) / kChunkMax;
+    a.cw = ((a.gk + a.n_chunks - 1) / a.n_chunks + 15) / 16 * 16;
+    a.kpad = a.n_chunks * a.cw;
+    if (a.kpad > kMaxKpad) return cudaErrorInvalidValue;
+    a.nbuf = std::min(kMaxBuf, 512 / a.cw);
+    a.row_tiles = (pl.N + 127) / 128;
+    a.total_items = 2 * pl.H * a.row_tiles;
+    const int fixed = 1024 + (int)sizeof(Ctl) + 16 + kEpiWarps * a.kpad * 4 + a.kpad * 256;
+    a.stages = std::min(4, (227 * 1024 - fixed) / kXStageBytes);
+    if (a.stages < 2) return cudaErrorInvalidValue;
+    a.anc_inv = reinterpret_cast<const float*>(ws + pl.o_anc_inv);
+    a.slot_of = reinterpret_cast<const int*>(ws + pl.o_slot_of);
+    a.xnorm = reinterpret_cast<const float*>(ws + pl.o_xnorm);
+    a.tok = reinterpret_cast<uint32_t*>(out + pl.L.off_tok);
+    a.refine = reinterpret_cast<int*>(ws + pl.o_refine);
+    a.counters = reinterpret_cast<int*>(ws + pl.o_counters);
+    CUtensorMap mAK, mAV;
+    if (!make_map(&mAK, out + pl.L.off_anchors_k, Hk, a.cw) || !make_map(&mAV, out + pl.L.off_anchors_v, Hk, a.cw))
+      return cudaErrorInvalidValue;
+    const int smem = fixed + a.stages * kXStageBytes;
+    const int grid = std::min(sms, a.total_items);
+    cudaFuncSetAttribute(assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    assign_tc_kernel<<<grid, kThreads, smem, s>>>(mXK, mXV, mAK, mAV, a);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace akv

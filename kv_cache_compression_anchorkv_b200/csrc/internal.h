@@ -20,6 +20,11 @@ void stage_end(int stage, cudaStream_t s, int kernels);
 // its own (max, sum) partials (pass A) or per-token row-block sums (B, C).
 constexpr int kObsGroups = 4;
 
+// Anchors the tensor-core assignment keeps resident in shared memory at once;
+// more are taken in groups of at most this many (best keys merged through
+// the workspace between groups).
+constexpr int kAssignGroupMax = 480;
+
 // Everything one compress call needs to know, derived from the parameters.
 struct Plan {
   anchorkv_params p;
@@ -40,6 +45,7 @@ struct Plan {
   int64_t o_score, o_a2, o_ku, o_pooled, o_slot_of, o_anc_n2, o_anc_inv, o_anc_sqrt, o_xnorm;
   int64_t o_util, o_refine, o_sel_state, o_hist, o_tile_gt, o_tile_eq, o_tie_before, o_tile_cnt;
   int64_t o_qproxy;          // proxy observation queries [Hq][W][D] (key-as-query mode), else 0
+  int64_t o_asg_keys;        // best two 64-bit keys per token-side between anchor groups (k > kAssignGroupMax)
   // codebook and Hadamard signs (bit j set: s_j = -1)
   double tau, l1, l2;
   uint32_t sign_bits[4];

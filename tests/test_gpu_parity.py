@@ -265,3 +265,18 @@ def test_reconstruct_naive_codec():
     Ko, Vo = O.reconstruct(O.unpack_layout(out.cpu().numpy(), po), po)
     assert np.abs(Kh.cpu().double().numpy() - Ko).max() < 1e-5 * np.abs(Ko).max()
     assert np.abs(Vh.cpu().double().numpy() - Vo).max() < 1e-5 * np.abs(Vo).max()
+
+
+@pytest.mark.parametrize("N,anchor_div,theta", [(8000, 16, 0.1), (8000, 8, 0.15)])
+def test_compress_anchor_groups(N, anchor_div, theta):
+    """More anchors than the tensor-core assignment keeps resident (k = 532
+    and 1032: two and three anchor groups merged through the workspace)."""
+    spec = CacheSpec(1, 1, 4, N, n_dirs=64, seed=12)
+    K, V, Q = make_layer(spec, 0)
+    p = _params(spec, theta, layer=1)
+    p.anchor_div = anchor_div
+    assert api.anchorkv_bytes(p)["n_anchors"] > 480
+    gb, gpool, gutil, counters = parity.gpu_compress(p, K, V, Q)
+    assert counters[0] == 0
+    rep = parity.check_compress(p, _f64(K), _f64(V), _f64(Q), gb, gpool, gutil)
+    print("anchor groups", N, anchor_div, rep, "refined rows:", counters[1])
