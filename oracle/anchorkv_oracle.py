@@ -808,6 +808,61 @@ def decode_attention(q: np.ndarray, Khat: np.ndarray, Vhat: np.ndarray,
 
 
 # --------------------------------------------------------------------------
+# a7 with rotary positions: keys stored pre-RoPE, rotated at decode
+# --------------------------------------------------------------------------
+
+def rope_rotate(X: np.ndarray, positions: np.ndarray, base: float) -> np.ndarray:
+    """R_p x for every row: the rotary position map of each row's position.
+
+    [PITH] "Assumptions & free parameters" (standard math, Section 3.2): RoPE
+    is a per-position orthogonal linear map R_t, so R_t K_t = R_t K~_t +
+    R_t r_t and ||R_t r_t|| = ||r_t||, which justifies storing keys pre-RoPE
+    and rotating them at decode time.
+    Reading (the pages name no convention): the rotate-half pairing of
+    Llama-family models, coordinate i paired with i + D/2 for i < D/2 and
+    turned by the angle p * base^(-2i/D).
+    X: [n, D]; positions: [n] integers.
+    """
+    n, D = X.shape
+    half = D // 2
+    inv = base ** (-2.0 * np.arange(half) / D)
+    ang = np.asarray(positions, np.float64)[:, None] * inv[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = X[:, :half], X[:, half:]
+    return np.concatenate([a * c - b * s, a * s + b * c], axis=1)
+
+
+def decode_attention_rope(q: np.ndarray, Khat: np.ndarray, Vhat: np.ndarray, base: float,
+                          Ktail: np.ndarray | None = None, Vtail: np.ndarray | None = None) -> np.ndarray:
+    """Decode attention when the cached keys are stored before the rotary map.
+
+    [PITH] "Assumptions & free parameters": pre-RoPE storage, rotation at
+    decode time.  Reading: cached token t sits at position t, appended tail
+    token i at N + i, and the decode query at N + T (the position of the token
+    being decoded); keys and the query are rotated at their positions, values
+    are not; no mask.  q: [Hq, D]; Khat, Vhat: [H, N, D]; tails [H, T, D].
+    """
+    Hq, D = q.shape
+    H, N, _ = Khat.shape
+    G = Hq // H
+    T = 0 if Ktail is None else Ktail.shape[1]
+    pos = np.arange(N + T)
+    o = np.zeros((Hq, D))
+    for j in range(Hq):
+        h = j // G
+        Kf, Vf = Khat[h], Vhat[h]
+        if T:
+            Kf = np.concatenate([Kf, Ktail[h]], axis=0)
+            Vf = np.concatenate([Vf, Vtail[h]], axis=0)
+        kr = rope_rotate(Kf, pos, base)
+        qr = rope_rotate(q[j][None, :], np.array([N + T]), base)[0]
+        s = kr @ qr / math.sqrt(D)
+        w = np.exp(s - s.max())
+        o[j] = (w / w.sum()) @ Vf
+    return o
+
+
+# --------------------------------------------------------------------------
 # Theorem 1 (output-error bound) terms
 # --------------------------------------------------------------------------
 

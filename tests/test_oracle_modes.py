@@ -239,3 +239,65 @@ def test_mode_pins_catch_planted_mistakes(monkeypatch):
     monkeypatch.setattr(O, "quantize_residuals", lambda r, seed, codebook=None, naive=False: orig_q(r, seed, codebook))
     with pytest.raises(AssertionError):
         test_naive_codec_codes_the_residual_itself()
+
+
+# ---------------------------------------------------------------- rotary positions
+
+def test_rope_is_orthogonal_and_linear():
+    """[PITH] Section 3.2 as quoted in the review: R_t is orthogonal and linear,
+    so it distributes over the anchor-residual decomposition."""
+    rng = np.random.default_rng(20)
+    X, Y = rng.normal(size=(50, 128)), rng.normal(size=(50, 128))
+    pos = rng.integers(0, 200000, 50)
+    RX = O.rope_rotate(X, pos, 500000.0)
+    assert np.allclose(np.linalg.norm(RX, axis=1), np.linalg.norm(X, axis=1), rtol=1e-13)
+    assert np.allclose(O.rope_rotate(2.5 * X - Y, pos, 500000.0), 2.5 * RX - O.rope_rotate(Y, pos, 500000.0),
+                       rtol=0, atol=1e-11)
+
+
+def test_rope_matches_complex_rotation_and_hand_values():
+    """Pair (x_i, x_{i+D/2}) as the complex number x_i + i x_{i+D/2}, turned by
+    exp(i p base^(-2i/D)); and a hand-worked D = 4 case."""
+    rng = np.random.default_rng(21)
+    X = rng.normal(size=(7, 128))
+    pos = np.array([0, 1, 2, 31, 1000, 32767, 131071])
+    z = X[:, :64] + 1j * X[:, 64:]
+    w = z * np.exp(1j * pos[:, None] * 10000.0 ** (-np.arange(64) / 64.0)[None, :])
+    assert np.allclose(O.rope_rotate(X, pos, 10000.0), np.concatenate([w.real, w.imag], axis=1), rtol=0, atol=1e-11)
+    # D = 4, base 100: frequencies 1 and 100^(-1/2) = 0.1; x = e_0 and e_1 at p = 1
+    got = O.rope_rotate(np.array([[1.0, 0, 0, 0], [0, 1.0, 0, 0]]), np.array([1, 1]), 100.0)
+    assert np.allclose(got[0], [math.cos(1), 0, math.sin(1), 0])
+    assert np.allclose(got[1], [0, math.cos(0.1), 0, math.sin(0.1)])
+
+
+def test_rope_scores_depend_on_relative_position():
+    rng = np.random.default_rng(22)
+    q, k = rng.normal(size=(1, 128)), rng.normal(size=(1, 128))
+    for a, b in [(5, 17), (1000, 1003), (70000, 12)]:
+        lhs = O.rope_rotate(q, [a], 500000.0) @ O.rope_rotate(k, [b], 500000.0).T
+        rhs = q @ O.rope_rotate(k, [b - a], 500000.0).T
+        assert abs(lhs - rhs) < 1e-10 * (1 + abs(rhs))
+
+
+def test_rope_decode_is_attention_over_rotated_keys():
+    """The decode with rotary positions equals textbook softmax attention of
+    the rotated query over the rotated keys (positions 0..N-1, then the tail,
+    query at N + T), values unrotated."""
+    rng = np.random.default_rng(23)
+    H, G, N, T, D = 2, 3, 40, 5, 128
+    q = rng.normal(size=(H * G, D))
+    K, V = rng.normal(size=(H, N, D)), rng.normal(size=(H, N, D))
+    Kt, Vt = rng.normal(size=(H, T, D)), rng.normal(size=(H, T, D))
+    o = O.decode_attention_rope(q, K, V, 1000.0, Kt, Vt)
+    for j in range(H * G):
+        h = j // G
+        keys = np.concatenate([K[h], Kt[h]])
+        vals = np.concatenate([V[h], Vt[h]])
+        z = keys[:, :64] + 1j * keys[:, 64:]
+        zq = q[j, :64] + 1j * q[j, 64:]
+        f = 1000.0 ** (-np.arange(64) / 64.0)
+        zr = z * np.exp(1j * np.arange(N + T)[:, None] * f[None, :])
+        zqr = zq * np.exp(1j * (N + T) * f)
+        s = (zr.real @ zqr.real + zr.imag @ zqr.imag) / math.sqrt(D)
+        p = np.exp(s - s.max())
+        assert np.allclose(o[j], (p / p.sum()) @ vals, rtol=0, atol=1e-12)
