@@ -209,6 +209,27 @@ int anchorkv_decode_attn(const anchorkv_params* p, const void* compressed,
                          void* stream);
 
 /*
+ * Decode attention when the cached keys were stored before the rotary
+ * position map (review, "Assumptions & free parameters": RoPE is a
+ * per-position orthogonal linear map, so it distributes over the
+ * anchor-residual split, which justifies pre-RoPE storage and rotation at
+ * decode time).  Same layouts and arguments as anchorkv_decode_attn, plus
+ * rope_base (> 1, e.g. 10000 or 500000).  Rotate-half pairing: coordinate i
+ * and i + D/2 turn by p * rope_base^(-2i/D); cached token t sits at
+ * position t, tail token i at N + i (the tail keys are passed pre-rotary as
+ * well), the query q at N + tail_len; values are not rotated.  Keys are
+ * rebuilt token by token (gamma~ K_a + r~), so this path reads the anchors
+ * once per token instead of once per slot.
+ *   ws  device, ws_bytes >= anchorkv_decode_rope_workspace_bytes
+ */
+int anchorkv_decode_rope_workspace_bytes(const anchorkv_params* p, int32_t batch, size_t* ws_bytes);
+int anchorkv_decode_attn_rope(const anchorkv_params* p, const void* compressed,
+                              int64_t seq_stride_bytes, int32_t batch, const void* q,
+                              const void* K_tail, const void* V_tail, int32_t tail_len,
+                              int32_t tail_cap, double rope_base, float* out, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/*
  * Launch shape of anchorkv_decode_attn for `batch` sequences on the current
  * device (a diagnostic with no counterpart in the method): CTAs per
  * (sequence, KV head) thread-block cluster and dynamic shared memory per CTA.
@@ -274,7 +295,7 @@ int anchorkv_codebook(double* out4);
 int anchorkv_stage_timing(int enable);
 
 /* Number of timed stages reported by anchorkv_stage_times. */
-#define ANCHORKV_N_STAGES 15
+#define ANCHORKV_N_STAGES 16
 
 /* Waits for the recorded events and returns, per stage (n >= ANCHORKV_N_STAGES entries),
  * the accumulated milliseconds and the number of timed calls since the last

@@ -143,6 +143,40 @@ def decode_attn(p: AnchorKVParams, compressed: torch.Tensor, q: torch.Tensor,
     return out
 
 
+def decode_rope_workspace_bytes(p: AnchorKVParams, batch: int) -> int:
+    n = ctypes.c_size_t()
+    capi.check("anchorkv_decode_rope_workspace_bytes",
+               capi.lib().anchorkv_decode_rope_workspace_bytes(ctypes.byref(p.c()), batch, ctypes.byref(n)))
+    return n.value
+
+
+def decode_attn_rope(p: AnchorKVParams, compressed: torch.Tensor, q: torch.Tensor, rope_base: float,
+                     K_tail: torch.Tensor | None = None, V_tail: torch.Tensor | None = None, tail_len: int = 0,
+                     out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Decode attention over layouts whose keys were stored before the rotary
+    map (anchorkv_decode_attn_rope): cached token t at position t, tail token
+    i at N + i, the query at N + tail_len.  Shapes as decode_attn."""
+    if compressed.dim() == 1:
+        batch, stride = 1, (compressed.numel() + 15) // 16 * 16
+    else:
+        batch, stride = compressed.shape
+    _check_tensor("q", q, (batch, p.n_q_heads, p.head_dim), p.torch_dtype)
+    cap = 0
+    if K_tail is not None:
+        cap = K_tail.shape[2]
+        _check_tensor("K_tail", K_tail, (batch, p.n_kv_heads, cap, p.head_dim), p.torch_dtype)
+        _check_tensor("V_tail", V_tail, (batch, p.n_kv_heads, cap, p.head_dim), p.torch_dtype)
+    if out is None:
+        out = torch.empty(batch, p.n_q_heads, p.head_dim, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(decode_rope_workspace_bytes(p, batch), dtype=torch.uint8, device=q.device)
+    st = capi.lib().anchorkv_decode_attn_rope(ctypes.byref(p.c()), _ptr(compressed), stride, batch, _ptr(q),
+                                              _ptr(K_tail), _ptr(V_tail), tail_len, cap, float(rope_base),
+                                              _ptr(out), _ptr(workspace), workspace.numel(), _stream(q.device))
+    capi.check("anchorkv_decode_attn_rope", st)
+    return out
+
+
 def decode_config(p: AnchorKVParams, batch: int) -> dict:
     """Launch shape of decode_attn on the current device: CTAs per (sequence,
     head) cluster (0: split-token path with a workspace) and shared memory."""
@@ -257,7 +291,7 @@ class HostCompressor:
         return dst
 
 
-N_STAGES = 15   # ANCHORKV_N_STAGES
+N_STAGES = 16   # ANCHORKV_N_STAGES
 
 
 def stage_timing(enable: bool) -> None:

@@ -55,6 +55,9 @@ _SIGS = {
     "anchorkv_decode_attn_noalloc": ([_P(Params), _vp, ctypes.c_int64, ctypes.c_int32, _vp, _vp, _vp,
                                       ctypes.c_int32, ctypes.c_int32, _vp, _vp], ctypes.c_int),
     "anchorkv_decode_config": ([_P(Params), ctypes.c_int32, _P(ctypes.c_int32), _P(ctypes.c_int32)], ctypes.c_int),
+    "anchorkv_decode_rope_workspace_bytes": ([_P(Params), ctypes.c_int32, _P(ctypes.c_size_t)], ctypes.c_int),
+    "anchorkv_decode_attn_rope": ([_P(Params), _vp, ctypes.c_int64, ctypes.c_int32, _vp, _vp, _vp, ctypes.c_int32,
+                                   ctypes.c_int32, ctypes.c_double, _vp, _vp, ctypes.c_size_t, _vp], ctypes.c_int),
     "anchorkv_reconstruct": ([_P(Params), _vp, _vp, _vp, _vp], ctypes.c_int),
     "anchorkv_read_device_status": ([_vp, _P(ctypes.c_int32), _vp], ctypes.c_int),
     "anchorkv_codebook": ([_P(ctypes.c_double)], ctypes.c_int),

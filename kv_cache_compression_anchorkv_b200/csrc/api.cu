@@ -351,6 +351,43 @@ int anchorkv_decode_attn(const anchorkv_params* p, const void* compressed, int64
   return ANCHORKV_OK;
 }
 
+int anchorkv_decode_rope_workspace_bytes(const anchorkv_params* p, int32_t batch, size_t* ws_bytes) {
+  if (!ws_bytes || batch < 0) return ANCHORKV_EINVAL;
+  Plan pl;
+  int st = make_plan(p, &pl);
+  if (st) return st;
+  *ws_bytes = (size_t)make_rope_plan(pl, std::max(batch, 1)).ws_total;
+  return ANCHORKV_OK;
+}
+
+int anchorkv_decode_attn_rope(const anchorkv_params* p, const void* compressed, int64_t seq_stride_bytes,
+                              int32_t batch, const void* q, const void* K_tail, const void* V_tail, int32_t tail_len,
+                              int32_t tail_cap, double rope_base, float* out, void* ws, size_t ws_bytes,
+                              void* stream) {
+  Plan pl;
+  int st = make_plan(p, &pl);
+  if (st) return st;
+  if (batch < 0 || tail_len < 0 || tail_cap < tail_len) return ANCHORKV_EINVAL;
+  if (!(rope_base > 1.0) || !isfinite(rope_base)) return ANCHORKV_EINVAL;
+  if (batch == 0) return ANCHORKV_OK;
+  if (batch > 65535) return ANCHORKV_EUNSUPPORTED;
+  if (!compressed || !q || !out || !ws) return ANCHORKV_EINVAL;
+  if (tail_len > 0 && (!K_tail || !V_tail)) return ANCHORKV_EINVAL;
+  if ((int64_t)pl.N + tail_len > (1 << 21)) return ANCHORKV_EUNSUPPORTED;
+  if (seq_stride_bytes < pl.L.total_bytes && batch > 1) return ANCHORKV_EINVAL;
+  if (seq_stride_bytes % 16) return ANCHORKV_EINVAL;
+  if (((uintptr_t)compressed | (uintptr_t)q | (uintptr_t)out | (uintptr_t)ws | (uintptr_t)K_tail |
+       (uintptr_t)V_tail) & 15)
+    return ANCHORKV_EINVAL;
+  const RopePlan rp = make_rope_plan(pl, batch);
+  if ((int64_t)ws_bytes < rp.ws_total) return ANCHORKV_ENOSPC;
+  st = check_device();
+  if (st) return st;
+  AKV_LAUNCH(launch_decode_rope(pl, rp, (const char*)compressed, seq_stride_bytes, batch, q, K_tail, V_tail, tail_len,
+                                tail_cap, rope_base, out, (char*)ws, (cudaStream_t)stream));
+  return ANCHORKV_OK;
+}
+
 int anchorkv_decode_config(const anchorkv_params* p, int32_t batch, int32_t* cluster_ctas, int32_t* smem_bytes) {
   if (!cluster_ctas || !smem_bytes || batch < 1) return ANCHORKV_EINVAL;
   Plan pl;

@@ -1,0 +1,273 @@
+// Decode attention with rotary positions: keys are stored before the rotary
+// map and rotated at decode time.
+//
+// "AnchorKV: Anchor-Residual KV Cache Compression" (pith.science review),
+// "Assumptions & free parameters" (standard math, Section 3.2): RoPE is a
+// per-position orthogonal linear map R_t, so R_t K_t = R_t K~_t + R_t r_t and
+// ||R_t r_t|| = ||r_t||, which justifies pre-RoPE storage and rotation at
+// decode time.  Reading: the rotate-half pairing (coordinate i with i + D/2,
+// angle p * base^(-2i/D)); cached token t at position t, tail token i at
+// N + i, the decode query at N + T.
+//
+// The per-slot factorisation q.K_a of the plain decode does not survive the
+// rotation (every token turns its anchor by a different angle, and the
+// rotation does not commute with the residual codec's Hadamard transform), so
+// each warp rebuilds K^_t = gamma~ K_a + r~_t for one token at a time in
+// registers (lane l holds coordinates 4l .. 4l + 3; the residual through a
+// warp FWHT), rotates it by its position (the partner coordinate is in lane
+// l ^ 16), scores it against the G rotated queries of the KV head and
+// updates an online softmax over V^_t.  Angles are reduced modulo 2 pi in
+// fp64 before the fast sine/cosine.  Splits of the tokens over CTAs fill the
+// SMs; a second kernel merges the splits in order.
+#include "common.cuh"
+#include "internal.h"
+
+namespace akv {
+namespace {
+
+constexpr int kRopeWarps = 8;
+constexpr float kLog2eR = 1.4426950408889634f;
+
+struct RopeArgs {
+  const uint8_t* comp;
+  int64_t stride;
+  anchorkv_layout L;
+  int N, H, G, k, n_tiles, n_split, split_tokens, tail_len, tail_cap, naive;
+  int64_t R;
+  float lev[4];
+  uint32_t sign_bits[4];
+  double inv_freq[kD / 2];      // base^(-2i/D)
+  float* part;                  // [b][h][split][G][D + 2]: m, l, acc
+};
+
+__device__ __forceinline__ float sgn_of(const RopeArgs& a, int d) {
+  return ((a.sign_bits[d >> 5] >> (d & 31)) & 1u) ? -1.f : 1.f;
+}
+
+template <typename T> __device__ __forceinline__ void load4r(const T* p, float (&o)[4]);
+template <> __device__ __forceinline__ void load4r<float>(const float* p, float (&o)[4]) {
+  const float4 v = *reinterpret_cast<const float4*>(p);
+  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+}
+template <> __device__ __forceinline__ void load4r<__nv_bfloat16>(const __nv_bfloat16* p, float (&o)[4]) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  o[0] = __uint_as_float(v.x << 16); o[1] = __uint_as_float(v.x & 0xFFFF0000u);
+  o[2] = __uint_as_float(v.y << 16); o[3] = __uint_as_float(v.y & 0xFFFF0000u);
+}
+
+// R_p x for this lane's four coordinates (lane l: 4l .. 4l + 3; the pair of
+// coordinate d < D/2 is d + D/2, held by lane l ^ 16).
+__device__ __forceinline__ void rope4(const RopeArgs& a, int64_t pos, float (&x)[4], int lane) {
+  const bool upper = lane >= 16;
+  const double two_pi = 6.283185307179586476925286766559;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int i = (lane & 15) * 4 + e;
+    const double ang = (double)pos * a.inv_freq[i];
+    const float r = (float)(ang - two_pi * rint(ang / two_pi));
+    float s, c;
+    __sincosf(r, &s, &c);
+    const float other = __shfl_xor_sync(0xffffffffu, x[e], 16);
+    x[e] = upper ? fmaf(other, s, x[e] * c) : fmaf(-other, s, x[e] * c);
+  }
+}
+
+// One side's reconstructed row x^_t (this lane's four coordinates): gamma~
+// times the anchor row, plus the decoded residual when the bitmap has it.
+template <typename T>
+__device__ __forceinline__ void rebuild(const RopeArgs& a, const uint8_t* comp, int side, int h, int t,
+                                        const T* anchors, float (&x)[4], int lane) {
+  const uint32_t rt = reinterpret_cast<const uint32_t*>(comp + a.L.off_tok)[((int64_t)side * a.H + h) * a.N + t];
+  const int slot = min((int)(rt & 0xFFFFu), a.k - 1);
+  const float g = half_bits_to_f(rt >> 16);
+  float av[4];
+  load4r<T>(anchors + ((int64_t)h * a.k + slot) * kD + lane * 4, av);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) x[e] = g * av[e];
+  const int sh = side * a.H + h, tile = t / kTile, w = (t % kTile) / 32, b = t % 32;
+  const uint32_t* bw = reinterpret_cast<const uint32_t*>(comp + a.L.off_bitmap) + ((int64_t)sh * a.n_tiles + tile) * 4;
+  const uint32_t word = bw[w];
+  if (!((word >> b) & 1u)) return;                   // (uniform over the warp)
+  int64_t rec = reinterpret_cast<const int*>(comp + a.L.off_tile_prefix)[(int64_t)sh * (a.n_tiles + 1) + tile];
+  for (int q = 0; q < w; ++q) rec += __popc(bw[q]);
+  rec += __popc(word & ((1u << b) - 1u));
+  if (rec >= a.R) return;                             // corrupt layout: anchor part only
+  const float sg = half_bits_to_f(reinterpret_cast<const uint16_t*>(comp + a.L.off_res_sigma)[rec]);
+  const uint32_t byte = (comp + a.L.off_res_codes)[rec * kCodeBytes + lane];
+  float z[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) z[e] = a.lev[(byte >> (2 * e)) & 3u] * sg;
+  if (a.naive) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] += z[e];
+    return;
+  }
+  fwht128<float>(z);
+  const float isd = rsqrtf((float)kD);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) x[e] = fmaf(z[e] * isd, sgn_of(a, lane * 4 + e), x[e]);
+}
+
+// grid (n_split, batch * H), kRopeWarps warps; each warp takes tokens
+// t0 + warp, t0 + warp + 8, ... of its split (the tail after the N cached
+// ones).  GM: a power of two >= G (register arrays per query head).
+template <typename T, int GM>
+__global__ void __launch_bounds__(kRopeWarps * 32) rope_split_kernel(RopeArgs a, const T* __restrict__ q,
+                                                                     const T* __restrict__ Kt,
+                                                                     const T* __restrict__ Vt) {
+  extern __shared__ __align__(16) float smr[];       // [8][G][D + 2]
+  const int split = blockIdx.x, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, G = a.G;
+  const uint8_t* comp = a.comp + (int64_t)b * a.stride;
+  const T* AK = reinterpret_cast<const T*>(comp + a.L.off_anchors_k);
+  const T* AV = reinterpret_cast<const T*>(comp + a.L.off_anchors_v);
+  const int T_ = a.tail_len, total = a.N + T_;
+  // this KV head's queries, rotated to the decode position, scaled for exp2
+  const float qs = kLog2eR * rsqrtf((float)kD);
+  float qr[GM][4], m[GM], l[GM], acc[GM][4];
+#pragma unroll
+  for (int j = 0; j < GM; ++j) {
+    m[j] = -INFINITY;
+    l[j] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) { acc[j][e] = 0.f; qr[j][e] = 0.f; }
+    if (j < G) {
+      float v[4];
+      load4r<T>(q + ((int64_t)b * a.H * G + h * G + j) * kD + lane * 4, v);
+      rope4(a, (int64_t)total, v, lane);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) qr[j][e] = v[e] * qs;
+    }
+  }
+  const int t0 = split * a.split_tokens, t1 = min(total, t0 + a.split_tokens);
+  for (int t = t0 + warp; t < t1; t += kRopeWarps) {
+    float kx[4], vx[4];
+    if (t < a.N) {
+      rebuild<T>(a, comp, 0, h, t, AK, kx, lane);
+      rebuild<T>(a, comp, 1, h, t, AV, vx, lane);
+    } else {
+      const int64_t row = (((int64_t)b * a.H + h) * a.tail_cap + (t - a.N)) * kD + lane * 4;
+      load4r<T>(Kt + row, kx);
+      load4r<T>(Vt + row, vx);
+    }
+    rope4(a, (int64_t)t, kx, lane);
+#pragma unroll
+    for (int j = 0; j < GM; ++j) {
+      if (j < G) {
+        float d = qr[j][0] * kx[0];
+#pragma unroll
+        for (int e = 1; e < 4; ++e) d = fmaf(qr[j][e], kx[e], d);
+        d = warp_sum(d);                             // log2-domain logit, uniform over the warp
+        const float mn = fmaxf(m[j], d);
+        const float sc = exp2f(m[j] - mn), p = exp2f(d - mn);
+        l[j] = fmaf(l[j], sc, p);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[j][e] = fmaf(acc[j][e], sc, p * vx[e]);
+        m[j] = mn;
+      }
+    }
+  }
+  // merge the warps of the CTA (fixed order) and write this split's partial
+  const int stride = kD + 2;
+#pragma unroll
+  for (int j = 0; j < GM; ++j) {
+    if (j < G) {
+      float* dst = smr + ((size_t)warp * G + j) * stride;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dst[lane * 4 + e] = acc[j][e];
+      if (lane == 0) { dst[kD] = m[j]; dst[kD + 1] = l[j]; }
+    }
+  }
+  __syncthreads();
+  float* out = a.part + (((int64_t)bh * a.n_split + split) * G) * stride;
+  for (int i = threadIdx.x; i < G * kD; i += blockDim.x) {
+    const int j = i / kD, d = i % kD;
+    float M = -INFINITY;
+    for (int w = 0; w < kRopeWarps; ++w) M = fmaxf(M, smr[((size_t)w * G + j) * stride + kD]);
+    float L = 0.f, O = 0.f;
+    for (int w = 0; w < kRopeWarps; ++w) {
+      const float* src = smr + ((size_t)w * G + j) * stride;
+      const float f = src[kD] > -INFINITY ? exp2f(src[kD] - M) : 0.f;
+      L = fmaf(src[kD + 1], f, L);
+      O = fmaf(src[d], f, O);
+    }
+    out[j * stride + d] = O;
+    if (d == 0) { out[j * stride + kD] = M; out[j * stride + kD + 1] = L; }
+  }
+}
+
+// grid (batch * H), 128 threads: merge the splits in order.
+__global__ void __launch_bounds__(128) rope_combine_kernel(RopeArgs a, float* __restrict__ o) {
+  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H, d = threadIdx.x, G = a.G;
+  const int stride = kD + 2;
+  const float* base = a.part + (int64_t)bh * a.n_split * G * stride;
+  for (int j = 0; j < G; ++j) {
+    float M = -INFINITY;
+    for (int s = 0; s < a.n_split; ++s) M = fmaxf(M, base[((int64_t)s * G + j) * stride + kD]);
+    float L = 0.f, O = 0.f;
+    for (int s = 0; s < a.n_split; ++s) {
+      const float* src = base + ((int64_t)s * G + j) * stride;
+      const float f = src[kD] > -INFINITY ? exp2f(src[kD] - M) : 0.f;
+      L = fmaf(src[kD + 1], f, L);
+      O = fmaf(src[d], f, O);
+    }
+    o[((int64_t)b * a.H * G + h * G + j) * kD + d] = O / L;
+  }
+}
+
+}  // namespace
+
+// Token splits of the rotary decode: about two CTAs per SM over batch * H
+// (sequence, head) pairs, at least 256 cached tokens per split.
+RopePlan make_rope_plan(const Plan& pl, int batch) {
+  RopePlan rp;
+  const int bh = std::max(1, batch * pl.H);
+  const int want = std::max(1, (2 * 148 + bh - 1) / bh);
+  rp.n_split = std::max(1, std::min(want, (pl.N + 255) / 256));
+  rp.ws_total = (int64_t)batch * pl.H * rp.n_split * pl.G * (kD + 2) * 4;
+  return rp;
+}
+
+cudaError_t launch_decode_rope(const Plan& pl, const RopePlan& rp, const char* comp, int64_t stride, int batch,
+                               const void* q, const void* Kt, const void* Vt, int tail_len, int tail_cap,
+                               double rope_base, float* out, char* ws, cudaStream_t s) {
+  RopeArgs a;
+  a.comp = reinterpret_cast<const uint8_t*>(comp);
+  a.stride = stride;
+  a.L = pl.L;
+  a.N = pl.N; a.H = pl.H; a.G = pl.G; a.k = pl.k; a.n_tiles = pl.n_tiles;
+  a.n_split = rp.n_split;
+  a.split_tokens = (pl.N + tail_len + rp.n_split - 1) / rp.n_split;
+  a.tail_len = tail_len; a.tail_cap = tail_cap;
+  a.naive = naive_codec(pl);
+  a.R = pl.R;
+  a.lev[0] = (float)-pl.l2; a.lev[1] = (float)-pl.l1; a.lev[2] = (float)pl.l1; a.lev[3] = (float)pl.l2;
+  for (int i = 0; i < 4; ++i) a.sign_bits[i] = pl.sign_bits[i];
+  for (int i = 0; i < kD / 2; ++i) a.inv_freq[i] = pow(rope_base, -2.0 * i / kD);
+  a.part = reinterpret_cast<float*>(ws);
+  const dim3 grid(rp.n_split, batch * pl.H);
+  const size_t smem = sizeof(float) * (size_t)kRopeWarps * pl.G * (kD + 2);
+  auto go = [&](auto kern, auto tag) {
+    using T = decltype(tag);
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    kern<<<grid, kRopeWarps * 32, smem, s>>>(a, static_cast<const T*>(q), static_cast<const T*>(Kt),
+                                             static_cast<const T*>(Vt));
+  };
+  stage_begin(kStDecodeRope, s);
+  if (pl.p.dtype == ANCHORKV_BF16) {
+    using T = __nv_bfloat16;
+    if (pl.G <= 4) go(rope_split_kernel<T, 4>, T{});
+    else if (pl.G <= 8) go(rope_split_kernel<T, 8>, T{});
+    else go(rope_split_kernel<T, 16>, T{});
+  } else {
+    using T = float;
+    if (pl.G <= 4) go(rope_split_kernel<T, 4>, T{});
+    else if (pl.G <= 8) go(rope_split_kernel<T, 8>, T{});
+    else go(rope_split_kernel<T, 16>, T{});
+  }
+  rope_combine_kernel<<<batch * pl.H, 128, 0, s>>>(a, out);
+  stage_end(kStDecodeRope, s, 2);
+  return cudaGetLastError();
+}
+
+}  // namespace akv

@@ -11,7 +11,8 @@ namespace akv {
 // Stages bracketed by the optional event timing (profile.cu).
 enum Stage {
   kStObsPass1 = 0, kStObsCombine, kStTokenStats, kStAnchorSelect, kStAssign, kStRefine, kStProject,
-  kStSelect, kStQuantize, kStDecodePrep, kStDecodeSplit, kStDecodeCombine, kStObsAlpha, kStObsKu, kStDecodeCluster, kStageCount
+  kStSelect, kStQuantize, kStDecodePrep, kStDecodeSplit, kStDecodeCombine, kStObsAlpha, kStObsKu, kStDecodeCluster,
+  kStDecodeRope, kStageCount
 };
 void stage_begin(int stage, cudaStream_t s);
 void stage_end(int stage, cudaStream_t s, int kernels);
@@ -83,6 +84,16 @@ cudaError_t launch_project(const Plan& pl, const void* K, const void* V, char* o
 cudaError_t launch_select(const Plan& pl, char* out, char* ws, cudaStream_t s);
 cudaError_t launch_quantize(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s);
 cudaError_t launch_key_queries(const Plan& pl, const void* K, void* Q, cudaStream_t s);
+
+// Decode attention with rotary positions (keys stored before the rotary map).
+struct RopePlan {
+  int n_split;
+  int64_t ws_total;
+};
+RopePlan make_rope_plan(const Plan& pl, int batch);
+cudaError_t launch_decode_rope(const Plan& pl, const RopePlan& rp, const char* comp, int64_t stride, int batch,
+                               const void* q, const void* Kt, const void* Vt, int tail_len, int tail_cap,
+                               double rope_base, float* out, char* ws, cudaStream_t s);
 // mode bits of the plan's parameters
 inline int rank_of(const Plan& pl) { return (pl.p.mode & ANCHORKV_MODE_RANK_MASK) >> ANCHORKV_MODE_RANK_SHIFT; }
 inline int naive_codec(const Plan& pl) { return (pl.p.mode & ANCHORKV_MODE_NAIVE_CODEC) ? 1 : 0; }

@@ -41,7 +41,8 @@ cudaEvent_t get_event() {
 
 const char* kNames[kStageCount] = {"obs_pass1", "obs_combine", "token_stats", "anchor_select", "assign",
                                    "assign_refine", "project", "select_topR", "quantize", "decode_prep",
-                                   "decode_split", "decode_combine", "obs_alpha", "obs_key_term", "decode_attn"};
+                                   "decode_split", "decode_combine", "obs_alpha", "obs_key_term", "decode_attn",
+                                   "decode_rope"};
 
 }  // namespace
 

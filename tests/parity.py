@@ -212,3 +212,19 @@ def check_decode(p: api.AnchorKVParams, layouts: list, q: np.ndarray, Kt, Vt, ta
         worst = max(worst, float(np.abs(o - out[b]).max()))
     assert worst <= tol, f"decode max-abs error {worst} > {tol}"
     return worst
+
+
+def check_decode_rope(p: api.AnchorKVParams, layouts: list, q: np.ndarray, Kt, Vt, tail_len: int, base: float,
+                      out: np.ndarray, tol: float) -> float:
+    """Decode attention with rotary positions vs the oracle on the GPU's layout."""
+    po = oracle_params(p)
+    worst = 0.0
+    for b, buf in enumerate(layouts):
+        parts = O.unpack_layout(buf, po)
+        Kh, Vh = O.reconstruct(parts, po)
+        kt = Kt[b][:, :tail_len] if tail_len else None
+        vt = Vt[b][:, :tail_len] if tail_len else None
+        o = O.decode_attention_rope(q[b], Kh, Vh, base, kt, vt)
+        worst = max(worst, float(np.abs(o - out[b]).max()))
+    assert worst <= tol, f"rotary decode max-abs error {worst} > {tol}"
+    return worst

@@ -148,3 +148,16 @@ def test_queries_are_optional_only_with_key_queries():
     assert L.anchorkv_compress(ctypes.byref(pk.c()), fake, fake, None, fake, 16, fake, 16, None) == capi.ENOSPC
     base = api.compress_workspace(api.AnchorKVParams(n_tokens=1024))["total_bytes"]
     assert api.compress_workspace(pk)["total_bytes"] >= base + 32 * 32 * 128 * 2
+
+
+def test_rope_decode_arguments_checked_on_the_host():
+    L = capi.lib()
+    p = api.AnchorKVParams(n_tokens=1024).c()
+    fake = ctypes.c_void_p(1 << 20)
+    n = ctypes.c_size_t()
+    assert L.anchorkv_decode_rope_workspace_bytes(ctypes.byref(p), 4, ctypes.byref(n)) == capi.OK and n.value > 0
+    for base in (1.0, 0.5, float("nan"), float("inf")):
+        assert L.anchorkv_decode_attn_rope(ctypes.byref(p), fake, 1 << 20, 1, fake, None, None, 0, 0, base,
+                                           fake, fake, 1 << 30, None) == capi.EINVAL
+    assert L.anchorkv_decode_attn_rope(ctypes.byref(p), fake, 1 << 20, 1, fake, None, None, 0, 0, 10000.0,
+                                       fake, fake, 16, None) == capi.ENOSPC

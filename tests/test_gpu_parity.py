@@ -280,3 +280,33 @@ def test_compress_anchor_groups(N, anchor_div, theta):
     assert counters[0] == 0
     rep = parity.check_compress(p, _f64(K), _f64(V), _f64(Q), gb, gpool, gutil)
     print("anchor groups", N, anchor_div, rep, "refined rows:", counters[1])
+
+
+@pytest.mark.parametrize("name,batch,tail,base,mode", [
+    ("tiny-fp32-n1024", 1, 0, 10000.0, 0), ("tiny-fp32-n1024", 2, 5, 500000.0, 0),
+    ("bf16-ragged-n3000", 2, 17, 500000.0, 0), ("bf16-gqa8-n2500", 1, 3, 10000.0, 0),
+    ("bf16-gqa16-n1500", 2, 4, 500000.0, 0), ("bf16-n20000", 1, 40, 500000.0, 0),
+    ("bf16-ragged-n3000", 1, 2, 10000.0, 0x10)])
+def test_decode_rope_parity(name, batch, tail, base, mode):
+    """Keys stored before the rotary map, rotated at decode (cached token t at
+    position t, tail token i at N + i, the query at N + T)."""
+    spec, theta = CASES[name]
+    p = _params(spec, theta)
+    p.mode = mode
+    L = api.anchorkv_bytes(p)
+    stride = (L["total_bytes"] + 255) // 256 * 256
+    comp = torch.zeros(batch, stride, dtype=torch.uint8, device="cuda")
+    layouts = []
+    for b in range(batch):
+        sb = CacheSpec(**{**spec.__dict__, "seed": spec.seed + 70 * b})
+        K, V, Q = make_layer(sb, 0)
+        out, _ = api.compress(p, K.cuda(), V.cuda(), Q.cuda())
+        comp[b, :L["total_bytes"]] = out
+        layouts.append(out.cpu().numpy())
+    q = make_decode_queries(spec, 0, step=1, batch=batch)
+    cap = max(tail, 1) + 2
+    Kt, Vt = make_tail(spec, 0, cap, batch=batch)
+    o = api.decode_attn_rope(p, comp, q.cuda(), base, Kt.cuda(), Vt.cuda(), tail_len=tail)
+    err = parity.check_decode_rope(p, layouts, _f64(q), _f64(Kt), _f64(Vt), tail, base, o.cpu().double().numpy(),
+                                   DECODE_TOL[spec.dtype])
+    print(name, "rope", batch, tail, base, "max abs err", err)
