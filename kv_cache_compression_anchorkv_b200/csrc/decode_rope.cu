@@ -56,15 +56,15 @@ template <> __device__ __forceinline__ void load4r<__nv_bfloat16>(const __nv_bfl
 }
 
 // R_p x for this lane's four coordinates (lane l: 4l .. 4l + 3; the pair of
-// coordinate d < D/2 is d + D/2, held by lane l ^ 16).
-__device__ __forceinline__ void rope4(const RopeArgs& a, int64_t pos, float (&x)[4], int lane) {
+// coordinate d < D/2 is d + D/2, held by lane l ^ 16).  f: this lane's four
+// frequencies base^(-2i/D), i = 4 (l mod 16) + e.
+__device__ __forceinline__ void rope4(const double (&f)[4], int64_t pos, float (&x)[4], int lane) {
   const bool upper = lane >= 16;
-  const double two_pi = 6.283185307179586476925286766559;
+  const double two_pi = 6.283185307179586476925286766559, inv_two_pi = 0.15915494309189533576888376337251;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    const int i = (lane & 15) * 4 + e;
-    const double ang = (double)pos * a.inv_freq[i];
-    const float r = (float)(ang - two_pi * rint(ang / two_pi));
+    const double ang = (double)pos * f[e];
+    const float r = (float)(ang - two_pi * rint(ang * inv_two_pi));
     float s, c;
     __sincosf(r, &s, &c);
     const float other = __shfl_xor_sync(0xffffffffu, x[e], 16);
@@ -72,47 +72,112 @@ __device__ __forceinline__ void rope4(const RopeArgs& a, int64_t pos, float (&x)
   }
 }
 
-// One side's reconstructed row x^_t (this lane's four coordinates): gamma~
-// times the anchor row, plus the decoded residual when the bitmap has it.
-template <typename T>
-__device__ __forceinline__ void rebuild(const RopeArgs& a, const uint8_t* comp, int side, int h, int t,
-                                        const T* anchors, float (&x)[4], int lane) {
-  const uint32_t rt = reinterpret_cast<const uint32_t*>(comp + a.L.off_tok)[((int64_t)side * a.H + h) * a.N + t];
-  const int slot = min((int)(rt & 0xFFFFu), a.k - 1);
-  const float g = half_bits_to_f(rt >> 16);
-  float av[4];
-  load4r<T>(anchors + ((int64_t)h * a.k + slot) * kD + lane * 4, av);
+// Per-token words that do not depend on one another (both sides): record
+// word, the tile's four bitmap words, the tile's first record index.
+struct TokWords {
+  uint32_t rt[2];
+  uint4 bw[2];
+  int pf[2];
+};
+
+__device__ __forceinline__ void load_words(const RopeArgs& a, const uint8_t* comp, int h, int t, TokWords& w) {
+  const int tile = t / kTile;
 #pragma unroll
-  for (int e = 0; e < 4; ++e) x[e] = g * av[e];
-  const int sh = side * a.H + h, tile = t / kTile, w = (t % kTile) / 32, b = t % 32;
-  const uint32_t* bw = reinterpret_cast<const uint32_t*>(comp + a.L.off_bitmap) + ((int64_t)sh * a.n_tiles + tile) * 4;
-  const uint32_t word = bw[w];
-  if (!((word >> b) & 1u)) return;                   // (uniform over the warp)
-  int64_t rec = reinterpret_cast<const int*>(comp + a.L.off_tile_prefix)[(int64_t)sh * (a.n_tiles + 1) + tile];
-  for (int q = 0; q < w; ++q) rec += __popc(bw[q]);
-  rec += __popc(word & ((1u << b) - 1u));
-  if (rec >= a.R) return;                             // corrupt layout: anchor part only
-  const float sg = half_bits_to_f(reinterpret_cast<const uint16_t*>(comp + a.L.off_res_sigma)[rec]);
-  const uint32_t byte = (comp + a.L.off_res_codes)[rec * kCodeBytes + lane];
-  float z[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) z[e] = a.lev[(byte >> (2 * e)) & 3u] * sg;
-  if (a.naive) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) x[e] += z[e];
-    return;
+  for (int side = 0; side < 2; ++side) {
+    const int sh = side * a.H + h;
+    w.rt[side] = reinterpret_cast<const uint32_t*>(comp + a.L.off_tok)[(int64_t)sh * a.N + t];
+    w.bw[side] = reinterpret_cast<const uint4*>(comp + a.L.off_bitmap)[(int64_t)sh * a.n_tiles + tile];
+    w.pf[side] = reinterpret_cast<const int*>(comp + a.L.off_tile_prefix)[(int64_t)sh * (a.n_tiles + 1) + tile];
   }
-  fwht128<float>(z);
+}
+
+// Both sides' reconstructed rows x^_t (this lane's four coordinates): gamma~
+// times the anchor row plus the decoded residual when the bitmap has it.  The
+// anchor rows and the residual records of both sides are loaded before any
+// of them is used.
+template <typename T>
+__device__ __forceinline__ void rebuild2(const RopeArgs& a, const uint8_t* comp, int t, const TokWords& w,
+                                         const T* AK, const T* AV, int h, float (&kx)[4], float (&vx)[4], int lane) {
+  const int wi = (t % kTile) / 32, b = t % 32;
+  float av[2][4], z[2][4];
+  bool has[2];
+#pragma unroll
+  for (int side = 0; side < 2; ++side) {
+    const int slot = min((int)(w.rt[side] & 0xFFFFu), a.k - 1);
+    load4r<T>((side ? AV : AK) + ((int64_t)h * a.k + slot) * kD + lane * 4, av[side]);
+    const uint32_t words[4] = {w.bw[side].x, w.bw[side].y, w.bw[side].z, w.bw[side].w};
+    uint32_t word = words[0];
+    int64_t rec = w.pf[side];
+#pragma unroll
+    for (int q = 1; q < 4; ++q) {
+      if (q <= wi) rec += __popc(words[q - 1]);
+      if (q == wi) word = words[q];
+    }
+    rec += __popc(word & ((1u << b) - 1u));
+    has[side] = ((word >> b) & 1u) && rec < a.R;      // (uniform over the warp)
+    if (has[side]) {
+      const float sg = half_bits_to_f(reinterpret_cast<const uint16_t*>(comp + a.L.off_res_sigma)[rec]);
+      const uint32_t byte = (comp + a.L.off_res_codes)[rec * kCodeBytes + lane];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) z[side][e] = a.lev[(byte >> (2 * e)) & 3u] * sg;
+    }
+  }
   const float isd = rsqrtf((float)kD);
 #pragma unroll
-  for (int e = 0; e < 4; ++e) x[e] = fmaf(z[e] * isd, sgn_of(a, lane * 4 + e), x[e]);
+  for (int side = 0; side < 2; ++side) {
+    float* x = side ? vx : kx;
+    const float g = half_bits_to_f(w.rt[side] >> 16);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = g * av[side][e];
+    if (!has[side]) continue;
+    if (a.naive) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[e] += z[side][e];
+    } else {
+      fwht128<float>(z[side]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[e] = fmaf(z[side][e] * isd, sgn_of(a, lane * 4 + e), x[e]);
+    }
+  }
+}
+
+// Sums over the warp of GM values at once (GM a power of two <= 32): a
+// transposed butterfly leaves value j's sum in lanes whose top log2(GM) bits
+// are j, and one shuffle per value hands every lane all of them.
+template <int GM>
+__device__ __forceinline__ void warp_sums(float (&d)[GM], int lane) {
+  constexpr int kBits = GM == 1 ? 0 : GM == 2 ? 1 : GM == 4 ? 2 : GM == 8 ? 3 : 4;
+  float v[GM];
+#pragma unroll
+  for (int i = 0; i < GM; ++i) v[i] = d[i];
+#pragma unroll
+  for (int st = 0; st < kBits; ++st) {
+    const int off = 16 >> st, half = GM >> (st + 1);
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float keep = up ? v[i + half] : v[i];
+      const float send = up ? v[i] : v[i + half];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+#pragma unroll
+  for (int off = 16 >> kBits; off >= 1; off >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+#pragma unroll
+  for (int j = 0; j < GM; ++j) d[j] = __shfl_sync(0xffffffffu, v[0], j << (5 - kBits));
+}
+
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // grid (n_split, batch * H), kRopeWarps warps; each warp takes tokens
 // t0 + warp, t0 + warp + 8, ... of its split (the tail after the N cached
 // ones).  GM: a power of two >= G (register arrays per query head).
 template <typename T, int GM>
-__global__ void __launch_bounds__(kRopeWarps * 32) rope_split_kernel(RopeArgs a, const T* __restrict__ q,
+__global__ void __launch_bounds__(kRopeWarps * 32, GM <= 4 ? 2 : 1) rope_split_kernel(RopeArgs a, const T* __restrict__ q,
                                                                      const T* __restrict__ Kt,
                                                                      const T* __restrict__ Vt) {
   extern __shared__ __align__(16) float smr[];       // [8][G][D + 2]
@@ -124,6 +189,9 @@ __global__ void __launch_bounds__(kRopeWarps * 32) rope_split_kernel(RopeArgs a,
   const int T_ = a.tail_len, total = a.N + T_;
   // this KV head's queries, rotated to the decode position, scaled for exp2
   const float qs = kLog2eR * rsqrtf((float)kD);
+  double fr[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) fr[e] = a.inv_freq[(lane & 15) * 4 + e];
   float qr[GM][4], m[GM], l[GM], acc[GM][4];
 #pragma unroll
   for (int j = 0; j < GM; ++j) {
@@ -134,32 +202,41 @@ __global__ void __launch_bounds__(kRopeWarps * 32) rope_split_kernel(RopeArgs a,
     if (j < G) {
       float v[4];
       load4r<T>(q + ((int64_t)b * a.H * G + h * G + j) * kD + lane * 4, v);
-      rope4(a, (int64_t)total, v, lane);
+      rope4(fr, (int64_t)total, v, lane);
 #pragma unroll
       for (int e = 0; e < 4; ++e) qr[j][e] = v[e] * qs;
     }
   }
   const int t0 = split * a.split_tokens, t1 = min(total, t0 + a.split_tokens);
+  // the words of the next token of this warp are loaded one token ahead
+  TokWords cur, nxt;
+  if (t0 + warp < min(t1, a.N)) load_words(a, comp, h, t0 + warp, cur);
   for (int t = t0 + warp; t < t1; t += kRopeWarps) {
     float kx[4], vx[4];
+    if (t + kRopeWarps < min(t1, a.N)) load_words(a, comp, h, t + kRopeWarps, nxt);
     if (t < a.N) {
-      rebuild<T>(a, comp, 0, h, t, AK, kx, lane);
-      rebuild<T>(a, comp, 1, h, t, AV, vx, lane);
+      rebuild2<T>(a, comp, t, cur, AK, AV, h, kx, vx, lane);
+      cur = nxt;
     } else {
       const int64_t row = (((int64_t)b * a.H + h) * a.tail_cap + (t - a.N)) * kD + lane * 4;
       load4r<T>(Kt + row, kx);
       load4r<T>(Vt + row, vx);
     }
-    rope4(a, (int64_t)t, kx, lane);
+    rope4(fr, (int64_t)t, kx, lane);
+    float dl[GM];
+#pragma unroll
+    for (int j = 0; j < GM; ++j) {
+      dl[j] = qr[j][0] * kx[0];
+#pragma unroll
+      for (int e = 1; e < 4; ++e) dl[j] = fmaf(qr[j][e], kx[e], dl[j]);
+    }
+    warp_sums<GM>(dl, lane);                         // log2-domain logits, on every lane
 #pragma unroll
     for (int j = 0; j < GM; ++j) {
       if (j < G) {
-        float d = qr[j][0] * kx[0];
-#pragma unroll
-        for (int e = 1; e < 4; ++e) d = fmaf(qr[j][e], kx[e], d);
-        d = warp_sum(d);                             // log2-domain logit, uniform over the warp
+        const float d = dl[j];
         const float mn = fmaxf(m[j], d);
-        const float sc = exp2f(m[j] - mn), p = exp2f(d - mn);
+        const float sc = ex2f(m[j] - mn), p = ex2f(d - mn);
         l[j] = fmaf(l[j], sc, p);
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[j][e] = fmaf(acc[j][e], sc, p * vx[e]);
