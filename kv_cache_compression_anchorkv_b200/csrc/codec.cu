@@ -186,7 +186,7 @@ template <> __device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfl
 // The Hadamard transform runs its four low stages in registers and its three
 // high stages across the record's eight lanes, all in fp64.
 template <typename T>
-__global__ void __launch_bounds__(256, 2) quantize_kernel(const T* __restrict__ K, const T* __restrict__ V,
+__global__ void __launch_bounds__(256, 3) quantize_kernel(const T* __restrict__ K, const T* __restrict__ V,
                                 const T* __restrict__ anc_k, const T* __restrict__ anc_v,
                                 const uint32_t* __restrict__ tok, const uint32_t* __restrict__ bitmap,
                                 const int* __restrict__ tile_prefix, uint8_t* __restrict__ codes,
