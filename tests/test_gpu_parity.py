@@ -310,3 +310,89 @@ def test_decode_rope_parity(name, batch, tail, base, mode):
     err = parity.check_decode_rope(p, layouts, _f64(q), _f64(Kt), _f64(Vt), tail, base, o.cpu().double().numpy(),
                                    DECODE_TOL[spec.dtype])
     print(name, "rope", batch, tail, base, "max abs err", err)
+
+
+@pytest.mark.slow
+def test_batched_decode_8b_shape_sampled():
+    """Batched decode as benchmarked for many sequences: 16 compressed
+    sequences of the 8B shape (8 KV / 32 query heads, N = 32768, theta = 0.1)
+    decoded in one launch; sequences 0 and 15 checked against the oracle."""
+    spec = CacheSpec(32, 8, 32, 32768, n_dirs=128, seed=0)
+    p = _params(spec, 0.1, layer=0)
+    L = api.anchorkv_bytes(p)
+    stride = (L["total_bytes"] + 255) // 256 * 256
+    batch = 16
+    comp = torch.zeros(batch, stride, dtype=torch.uint8, device="cuda")
+    for b in range(batch):
+        sb = CacheSpec(**{**spec.__dict__, "seed": 1000 + b})
+        K, V, Q = make_layer(sb, 0, device="cuda")
+        out, ws = api.compress(p, K, V, Q)
+        assert api.read_status(ws)[0] == 0
+        comp[b, :L["total_bytes"]] = out
+    q = make_decode_queries(spec, 0, step=0, batch=batch, device="cuda")
+    o = api.decode_attn(p, comp, q)
+    po = parity.oracle_params(p)
+    for b in (0, batch - 1):
+        parts = O.unpack_layout(comp[b, :L["total_bytes"]].cpu().numpy(), po)
+        Kh, Vh = O.reconstruct(parts, po)
+        want = O.decode_attention(_f64(q[b]), Kh, Vh)
+        err = float(np.abs(o[b].cpu().double().numpy() - want).max())
+        assert err <= DECODE_TOL["bf16"], (b, err)
+        print("batched decode sequence", b, "max abs err", err)
+
+
+@pytest.mark.slow
+def test_70b_shape_layer_sampled():
+    """One layer of the 70B-shaped cache (8 KV / 64 query heads, N = 131072,
+    theta = 0.05; k = 1056 anchors, three assignment groups): byte accounting,
+    window anchors, a sample of nearest-anchor slots and coefficients against
+    fp64 (mismatches only as counted near-ties), and the decode after 128
+    appended tokens against the oracle."""
+    spec = CacheSpec(80, 8, 64, 131072, n_dirs=256, seed=0)
+    p = _params(spec, 0.05, layer=7)
+    K, V, Q = make_layer(spec, 7, device="cuda")
+    out, ws = api.compress(p, K, V, Q)
+    st = api.read_status(ws)
+    assert st[0] == 0
+    L = api.anchorkv_bytes(p)
+    po = parity.oracle_params(p)
+    Lo = O.layout(po)
+    assert L["total_bytes"] == Lo["total"] and L["n_residuals"] == Lo["R"] and L["n_anchors"] == Lo["k"] == 1056
+    g = O.unpack_layout(out.cpu().numpy(), po)
+    N, W = spec.n_tokens, spec.window
+    rng = np.random.default_rng(3)
+    near = 0
+    for h in (0, 5):
+        ap = g["anchor_pos"][h]
+        assert np.all(np.isin(np.arange(N - W, N), ap)) and np.all(np.diff(ap) > 0)
+        for side, X in enumerate((K[h], V[h])):
+            Xh = _f64(X)
+            A = Xh[ap]
+            an = np.linalg.norm(A, axis=1)
+            for t in rng.choice(N, 400, replace=False):
+                cos = np.where(an > 0, A @ Xh[t] / np.where(an > 0, an, 1.0), 0.0)
+                s_o = int(np.argmax(cos)) if t not in set(ap.tolist()) else int(np.searchsorted(ap, t))
+                s_g = int(g["idx"][side, h, t])
+                if s_o != s_g:
+                    assert cos[s_o] - cos[s_g] <= 1e-12 * np.linalg.norm(Xh[t]), (h, side, t)
+                    near += 1
+                    continue
+                xa = A[s_g]
+                n2 = float(xa @ xa)
+                gam = 1.0 if t in set(ap.tolist()) else (float(Xh[t] @ xa) / n2 if n2 > 0 else 0.0)
+                assert np.float16(gam).view(np.uint16) == g["g16"][side, h, t].view(np.uint16) or \
+                    abs(gam - float(g["g16"][side, h, t])) <= 2 ** -11 * abs(gam) + 1e-300, (h, side, t)
+    q = make_decode_queries(spec, 7, step=128, batch=1, device="cuda")
+    Kt, Vt = make_tail(spec, 7, 128, batch=1, device="cuda")
+    o = api.decode_attn(p, out, q, Kt, Vt, tail_len=128)
+    Kh, Vh = O.reconstruct(g, po)
+    for j in (0, 63):
+        h = j // 8
+        Kf = np.concatenate([Kh[h], _f64(Kt[0, h])])
+        Vf = np.concatenate([Vh[h], _f64(Vt[0, h])])
+        s = Kf @ _f64(q[0, j]) / np.sqrt(128)
+        w = np.exp(s - s.max())
+        want = (w / w.sum()) @ Vf
+        err = float(np.abs(o[0, j].cpu().double().numpy() - want).max())
+        assert err <= DECODE_TOL["bf16"], (j, err)
+    print("70B-shaped layer: refined rows", st[1], "sampled near-ties", near)
