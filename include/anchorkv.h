@@ -221,6 +221,8 @@ int anchorkv_decode_attn(const anchorkv_params* p, const void* compressed,
  * rebuilt token by token (gamma~ K_a + r~), so this path reads the anchors
  * once per token instead of once per slot.
  *   ws  device, ws_bytes >= anchorkv_decode_rope_workspace_bytes
+ * Errors: EINVAL for a bad base, pointer, size or stride; EUNSUPPORTED when
+ * batch * H > 65535 or N + tail_len > 2^21; ENOSPC for a small workspace.
  */
 int anchorkv_decode_rope_workspace_bytes(const anchorkv_params* p, int32_t batch, size_t* ws_bytes);
 int anchorkv_decode_attn_rope(const anchorkv_params* p, const void* compressed,

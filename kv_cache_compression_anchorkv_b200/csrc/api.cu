@@ -370,7 +370,7 @@ int anchorkv_decode_attn_rope(const anchorkv_params* p, const void* compressed, 
   if (batch < 0 || tail_len < 0 || tail_cap < tail_len) return ANCHORKV_EINVAL;
   if (!(rope_base > 1.0) || !isfinite(rope_base)) return ANCHORKV_EINVAL;
   if (batch == 0) return ANCHORKV_OK;
-  if (batch > 65535) return ANCHORKV_EUNSUPPORTED;
+  if ((int64_t)batch * pl.H > 65535) return ANCHORKV_EUNSUPPORTED;     // (sequence, head) pairs: grid y
   if (!compressed || !q || !out || !ws) return ANCHORKV_EINVAL;
   if (tail_len > 0 && (!K_tail || !V_tail)) return ANCHORKV_EINVAL;
   if ((int64_t)pl.N + tail_len > (1 << 21)) return ANCHORKV_EUNSUPPORTED;

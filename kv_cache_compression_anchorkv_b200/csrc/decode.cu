@@ -363,6 +363,7 @@ int make_decode_plan(const Plan& pl, int batch, DecodePlan* dp) {
 
 int check_decode_shape(const Plan& pl, const DecodePlan& dp, int tail_len) {
   if (dp.cluster) return ANCHORKV_OK;
+  if ((int64_t)dp.batch * pl.H > 65535) return ANCHORKV_EUNSUPPORTED;   // (sequence, head) pairs: grid y
   const size_t smem_split = sizeof(float) * ((size_t)2 * pl.G * pl.k + (size_t)pl.G * dp.split_tokens + 2 * pl.G * kD);
   const size_t smem_comb = sizeof(float) * ((size_t)pl.G * pl.k + (size_t)pl.G * std::max(tail_len, 1));
   if (smem_split > 220 * 1024 || smem_comb > 180 * 1024) return ANCHORKV_EUNSUPPORTED;

@@ -161,3 +161,20 @@ def test_rope_decode_arguments_checked_on_the_host():
                                            fake, fake, 1 << 30, None) == capi.EINVAL
     assert L.anchorkv_decode_attn_rope(ctypes.byref(p), fake, 1 << 20, 1, fake, None, None, 0, 0, 10000.0,
                                        fake, fake, 16, None) == capi.ENOSPC
+    # (sequence, head) pairs beyond one grid dimension
+    assert L.anchorkv_decode_attn_rope(ctypes.byref(p), fake, 1 << 24, 10000, fake, None, None, 0, 0, 10000.0,
+                                       fake, fake, 1 << 40, None) == capi.EUNSUPPORTED
+
+
+def test_split_token_decode_grid_limit_on_the_host():
+    """The split-token decode (more than 8 query heads per KV head) puts
+    batch x H (sequence, head) pairs in one grid dimension: beyond 65535 it
+    is refused before any launch."""
+    L = capi.lib()
+    p = api.AnchorKVParams(n_tokens=1024, n_kv_heads=8, n_q_heads=128).c()
+    fake = ctypes.c_void_p(1 << 20)
+    n = ctypes.c_size_t()
+    assert L.anchorkv_decode_workspace_bytes(ctypes.byref(p), 9000, ctypes.byref(n)) == capi.OK
+    st = L.anchorkv_decode_attn(ctypes.byref(p), fake, 1 << 24, 9000, fake, None, None, 0, 0, fake, fake,
+                                n.value, None)
+    assert st == capi.EUNSUPPORTED
