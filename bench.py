@@ -314,7 +314,8 @@ def run_sweep(args):
     """Theta/length sweep of one 8B-shaped layer (8 KV / 32 query heads,
     D = 128, bf16, window 32; N in {8K, 32K, 128K} x theta in {0.05, 0.1,
     0.2}): anchor and residual counts, compress Mtok/s per layer-head, decode
-    at batch 1 (µs, GB/s over the compressed bytes), and the Theorem-1 bound
+    at batch 1 (µs, GB/s over the compressed bytes; also the decode with
+    rotary positions, keys taken as stored before RoPE), and the Theorem-1 bound
     vs the measured output error on 256 N(0, I) queries per KV head.  Then,
     at N = 32768 and theta = 0.05, the same error for every residual ranking
     criterion and for the unrotated codec (the ablation of the review's
@@ -335,12 +336,14 @@ def run_sweep(args):
         ms = _time_ms(lambda: api.compress(p, K, V, Q, out=out, workspace=ws), reps=5)
         q = make_decode_queries(spec, 0, step=0, batch=1, device=dev)
         dec_ms = _time_ms(lambda: api.decode_attn(p, out, q), reps=20)
+        rope_ms = _time_ms(lambda: api.decode_attn_rope(p, out, q, 500000.0), reps=10)
         st = api.read_status(ws)
         line = {"sweep": tag, "n_tokens": N, "theta": theta, "mode": mode, "anchors": L["n_anchors"],
                 "residuals": L["n_residuals"], "residual_share": L["n_residuals"] / (2 * 8 * N),
                 "compressed_bytes": L["total_bytes"], "ratio": L["uncompressed_bytes"] / L["total_bytes"],
                 "compress_mtok_s_per_layer_head": 8 * N / (ms * 1e-3) / 1e6, "compress_ms": ms,
                 "decode_us": dec_ms * 1e3, "decode_gbs": L["total_bytes"] / (dec_ms * 1e-3) / 1e9,
+                "decode_rope_us": rope_ms * 1e3,
                 "refined_rows": st[1]}
         line.update(_output_error(p, out, K, V, n_queries, seed=1000 + N))
         print(json.dumps(line), flush=True)
