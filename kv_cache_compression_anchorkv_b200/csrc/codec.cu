@@ -78,6 +78,15 @@ project_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __rest
   const uint32_t slot = min(tok[f] & 0xFFFFu, (uint32_t)(k - 1));
   const T* x = (side ? V : K) + ((int64_t)h * N + tt) * kD;
   const T* a = (side ? anc_v : anc_k) + ((int64_t)h * k + slot) * kD;
+  // Loads that depend only on the token go out with the row loads: the
+  // anchor flag, the anchor's squared norm, and (utility ranking) lane q's observation-row-block
+  // partial q, for the first npre of the obs_rb partials.
+  const bool is_anchor = slot_of[(int64_t)h * N + tt] >= 0;
+  const double n2 = anc_n2[((int64_t)side * H + h) * k + slot];
+  const float* src = side ? a2s : kus;
+  static_assert(kObsGroups <= 4, "one partial per lane of the quad");
+  const int npre = min(obs_rb, kObsGroups);
+  const float part = (kUtility && q < npre) ? src[((int64_t)q * H + h) * N + tt] : 0.0f;
   double dot = 0.0, nx = 0.0;
 #pragma unroll
   for (int i = 0; i < STEPS; ++i) {
@@ -95,9 +104,11 @@ project_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __rest
   nx += __shfl_xor_sync(0xffffffffu, nx, 1);
   dot += __shfl_xor_sync(0xffffffffu, dot, 2);
   nx += __shfl_xor_sync(0xffffffffu, nx, 2);
+  // partials 0 .. npre-1 to the quad's lane 0, summed in row-block order
+  const int l0 = threadIdx.x & 31 & ~3;
+  float m = __shfl_sync(0xffffffffu, part, l0);
+  for (int rb = 1; rb < npre; ++rb) m += __shfl_sync(0xffffffffu, part, l0 + rb);
   if (!valid || q != 0) return;
-  const bool is_anchor = slot_of[(int64_t)h * N + t] >= 0;
-  const double n2 = anc_n2[((int64_t)side * H + h) * k + slot];
   double gamma = (n2 > 0.0) ? dot / n2 : 0.0;
   if (is_anchor) gamma = 1.0;
   const uint16_t gb = half_bits_rn(gamma);
@@ -109,17 +120,15 @@ project_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __rest
     u = -1.0f;
   } else if (kUtility) {
     // sum of the observation-row-block partials, in order
-    const float* src = side ? a2s : kus;
-    float m = src[(int64_t)h * N + t];
-    for (int rb = 1; rb < obs_rb; ++rb) m += src[((int64_t)rb * H + h) * N + t];
+    for (int rb = npre; rb < obs_rb; ++rb) m += src[((int64_t)rb * H + h) * N + t];
     u = side ? (float)(r2 * (double)m) : (float)(r2 / (double)(kD * kD) * (double)m);
   } else if (rank == ANCHORKV_RANK_RESIDUAL_NORM) {
     u = (float)r2;
   } else if (rank == ANCHORKV_RANK_ATTENTION) {
     // sum over the observation rows of alpha (row-block partials, in order)
-    float m = score[(int64_t)h * N + t];
-    for (int rb = 1; rb < obs_rb; ++rb) m += score[((int64_t)rb * H + h) * N + t];
-    u = m;
+    float sa = score[(int64_t)h * N + t];
+    for (int rb = 1; rb < obs_rb; ++rb) sa += score[((int64_t)rb * H + h) * N + t];
+    u = sa;
   } else if (rank == ANCHORKV_RANK_COSINE) {
     const double den = sqrt(nx * n2);
     u = (float)(1.0 - (den > 0.0 ? dot / den : 0.0));
