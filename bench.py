@@ -232,6 +232,8 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="theta/length sweep with output error vs the Theorem-1 bound and the ablations "
                          "(one JSON line per point; not the benchmark line)")
+    ap.add_argument("--sweep-point", default="",
+                    help="with --sweep: only the theta-length point N,THETA (e.g. 32768,0.05; profiling runs)")
     args = ap.parse_args()
     if args.sweep:
         return run_sweep(args)
@@ -348,6 +350,10 @@ def run_sweep(args):
         line.update(_output_error(p, out, K, V, n_queries, seed=1000 + N))
         print(json.dumps(line), flush=True)
 
+    if args.sweep_point:
+        N, theta = args.sweep_point.split(",")
+        point(int(N), float(theta), 0, "theta-length")
+        return 0
     for N in (8192, 32768, 131072):
         for theta in (0.05, 0.1, 0.2):
             point(N, theta, 0, "theta-length")

@@ -17,8 +17,16 @@
 // warp FWHT), rotates it by its position (the partner coordinate is in lane
 // l ^ 16), scores it against the G rotated queries of the KV head and
 // updates an online softmax over V^_t.  Angles are reduced modulo 2 pi in
-// fp64 before the fast sine/cosine.  Splits of the tokens over CTAs fill the
-// SMs; a second kernel merges the splits in order.
+// fp64 before the fast sine/cosine.
+//
+// A warp walks 32-token chunks (one bitmap word each): its lanes decode the
+// chunk's record words, one token per lane (slot, gamma~, residual record
+// index), and the per-token loop then takes them by shuffle, with the next
+// token's anchor rows and residual codes already in flight; the next chunk's
+// words are loaded a chunk ahead.  Tail tokens take the same path, their raw
+// row standing in for the anchor row with gamma~ = 1 and no residual.
+// Splits of the tokens (multiples of 32) over CTAs fill the SMs; a second
+// kernel merges the splits in order.
 #include "common.cuh"
 #include "internal.h"
 
@@ -58,7 +66,7 @@ template <> __device__ __forceinline__ void load4r<__nv_bfloat16>(const __nv_bfl
 // R_p x for this lane's four coordinates (lane l: 4l .. 4l + 3; the pair of
 // coordinate d < D/2 is d + D/2, held by lane l ^ 16).  f: this lane's four
 // frequencies base^(-2i/D), i = 4 (l mod 16) + e.
-__device__ __forceinline__ void rope4(const double (&f)[4], int64_t pos, float (&x)[4], int lane) {
+__device__ __forceinline__ void rope4(const double* f, int64_t pos, float (&x)[4], int lane) {
   const bool upper = lane >= 16;
   const double two_pi = 6.283185307179586476925286766559, inv_two_pi = 0.15915494309189533576888376337251;
 #pragma unroll
@@ -72,71 +80,142 @@ __device__ __forceinline__ void rope4(const double (&f)[4], int64_t pos, float (
   }
 }
 
-// Per-token words that do not depend on one another (both sides): record
-// word, the tile's four bitmap words, the tile's first record index.
-struct TokWords {
+// Four coordinates of a row as loaded (bf16: 8 bytes, fp32: 16 bytes).
+template <typename T> struct Raw4 { using type = uint4; };
+template <> struct Raw4<__nv_bfloat16> { using type = uint2; };
+
+template <typename T>
+__device__ __forceinline__ typename Raw4<T>::type load_raw4(const T* p) {
+  return *reinterpret_cast<const typename Raw4<T>::type*>(p);
+}
+__device__ __forceinline__ void unpack4(const uint2& v, float (&o)[4]) {
+  o[0] = __uint_as_float(v.x << 16); o[1] = __uint_as_float(v.x & 0xFFFF0000u);
+  o[2] = __uint_as_float(v.y << 16); o[3] = __uint_as_float(v.y & 0xFFFF0000u);
+}
+__device__ __forceinline__ void unpack4(const uint4& v, float (&o)[4]) {
+  o[0] = __uint_as_float(v.x); o[1] = __uint_as_float(v.y);
+  o[2] = __uint_as_float(v.z); o[3] = __uint_as_float(v.w);
+}
+
+// The raw words of a 32-token chunk (tc a multiple of 32): lane l's token
+// record words (both sides), and one word of the chunk's tile spread over
+// lanes 0 .. 9 (lane 4s + w: bitmap word w of side s; lane 8 + s: the tile's
+// first record index of side s).
+struct ChunkRaw {
   uint32_t rt[2];
-  uint4 bw[2];
-  int pf[2];
+  uint32_t wv;
 };
 
-__device__ __forceinline__ void load_words(const RopeArgs& a, const uint8_t* comp, int h, int t, TokWords& w) {
-  const int tile = t / kTile;
+__device__ __forceinline__ void chunk_load(const RopeArgs& a, const uint8_t* comp, int h, int tc, int lane,
+                                           ChunkRaw& cr) {
+  cr.rt[0] = cr.rt[1] = 0u;
+  cr.wv = 0u;
+  if (tc >= a.N) return;                            // tail tokens only
+  const int t = tc + lane, tile = tc / kTile;
+  const uint32_t* tok = reinterpret_cast<const uint32_t*>(comp + a.L.off_tok);
+#pragma unroll
+  for (int side = 0; side < 2; ++side)
+    if (t < a.N) cr.rt[side] = tok[(int64_t)(side * a.H + h) * a.N + t];
+  if (lane < 8) {
+    const int sh = (lane >> 2) * a.H + h;
+    cr.wv = reinterpret_cast<const uint32_t*>(comp + a.L.off_bitmap)[((int64_t)sh * a.n_tiles + tile) * 4 + (lane & 3)];
+  } else if (lane < 10) {
+    const int sh = (lane - 8) * a.H + h;
+    cr.wv = (uint32_t)reinterpret_cast<const int*>(comp + a.L.off_tile_prefix)[(int64_t)sh * (a.n_tiles + 1) + tile];
+  }
+}
+
+// Lane l's token of the chunk: its record words and its residual record index
+// per side (-1: no residual).
+struct Chunk {
+  uint32_t rt[2];
+  int rec[2];
+};
+
+__device__ __forceinline__ void chunk_decode(const RopeArgs& a, int tc, int lane, const ChunkRaw& cr, Chunk& ck) {
+  const int w = (tc % kTile) / 32;
+  const bool cached = tc + lane < a.N;
 #pragma unroll
   for (int side = 0; side < 2; ++side) {
-    const int sh = side * a.H + h;
-    w.rt[side] = reinterpret_cast<const uint32_t*>(comp + a.L.off_tok)[(int64_t)sh * a.N + t];
-    w.bw[side] = reinterpret_cast<const uint4*>(comp + a.L.off_bitmap)[(int64_t)sh * a.n_tiles + tile];
-    w.pf[side] = reinterpret_cast<const int*>(comp + a.L.off_tile_prefix)[(int64_t)sh * (a.n_tiles + 1) + tile];
+    int rec = (int)__shfl_sync(0xffffffffu, cr.wv, 8 + side);
+    uint32_t word = 0u;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t wq = __shfl_sync(0xffffffffu, cr.wv, 4 * side + q);
+      if (q < w) rec += __popc(wq);
+      if (q == w) word = wq;
+    }
+    rec += __popc(word & ((1u << lane) - 1u));
+    const bool has = cached && ((word >> lane) & 1u) && (int64_t)rec < a.R;
+    ck.rec[side] = has ? rec : -1;
+    ck.rt[side] = cr.rt[side];
+  }
+}
+
+// One token's loads (both sides): the anchor row (a tail token: its raw row),
+// the gamma~ bits, and the residual code byte and sigma when it has a record.
+template <typename T>
+struct TokRaw {
+  typename Raw4<T>::type row[2];
+  uint32_t gb[2];
+  uint32_t code[2];
+  uint32_t sig[2];
+  bool has[2];
+};
+
+template <typename T>
+__device__ __forceinline__ void tok_issue(const RopeArgs& a, const uint8_t* comp, const T* AK, const T* AV,
+                                          const T* Kt, const T* Vt, int bb, int h, int t, int b, const Chunk& ck,
+                                          int lane, TokRaw<T>& r) {
+#pragma unroll
+  for (int side = 0; side < 2; ++side) {
+    const uint32_t rt = __shfl_sync(0xffffffffu, ck.rt[side], b);
+    const int rec = __shfl_sync(0xffffffffu, ck.rec[side], b);
+    r.has[side] = rec >= 0;                           // (uniform over the warp)
+    r.code[side] = 0u;
+    r.sig[side] = 0u;
+    if (t < a.N) {
+      const int slot = min((int)(rt & 0xFFFFu), a.k - 1);
+      r.row[side] = load_raw4<T>((side ? AV : AK) + ((int64_t)h * a.k + slot) * kD + lane * 4);
+      r.gb[side] = rt >> 16;
+      if (rec >= 0) {
+        r.code[side] = (comp + a.L.off_res_codes)[(int64_t)rec * kCodeBytes + lane];
+        r.sig[side] = reinterpret_cast<const uint16_t*>(comp + a.L.off_res_sigma)[rec];
+      }
+    } else {
+      const int64_t row = (((int64_t)bb * a.H + h) * a.tail_cap + (t - a.N)) * kD + lane * 4;
+      r.row[side] = load_raw4<T>((side ? Vt : Kt) + row);
+      r.gb[side] = 0x3C00u;                           // gamma~ = 1
+    }
   }
 }
 
 // Both sides' reconstructed rows x^_t (this lane's four coordinates): gamma~
-// times the anchor row plus the decoded residual when the bitmap has it.  The
-// anchor rows and the residual records of both sides are loaded before any
-// of them is used.
+// times the anchor row plus the decoded residual when the bitmap has it.
 template <typename T>
-__device__ __forceinline__ void rebuild2(const RopeArgs& a, const uint8_t* comp, int t, const TokWords& w,
-                                         const T* AK, const T* AV, int h, float (&kx)[4], float (&vx)[4], int lane) {
-  const int wi = (t % kTile) / 32, b = t % 32;
-  float av[2][4], z[2][4];
-  bool has[2];
-#pragma unroll
-  for (int side = 0; side < 2; ++side) {
-    const int slot = min((int)(w.rt[side] & 0xFFFFu), a.k - 1);
-    load4r<T>((side ? AV : AK) + ((int64_t)h * a.k + slot) * kD + lane * 4, av[side]);
-    const uint32_t words[4] = {w.bw[side].x, w.bw[side].y, w.bw[side].z, w.bw[side].w};
-    uint32_t word = words[0];
-    int64_t rec = w.pf[side];
-#pragma unroll
-    for (int q = 1; q < 4; ++q) {
-      if (q <= wi) rec += __popc(words[q - 1]);
-      if (q == wi) word = words[q];
-    }
-    rec += __popc(word & ((1u << b) - 1u));
-    has[side] = ((word >> b) & 1u) && rec < a.R;      // (uniform over the warp)
-    if (has[side]) {
-      const float sg = half_bits_to_f(reinterpret_cast<const uint16_t*>(comp + a.L.off_res_sigma)[rec]);
-      const uint32_t byte = (comp + a.L.off_res_codes)[rec * kCodeBytes + lane];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) z[side][e] = a.lev[(byte >> (2 * e)) & 3u] * sg;
-    }
-  }
+__device__ __forceinline__ void tok_rebuild(const RopeArgs& a, const TokRaw<T>& r, float (&kx)[4], float (&vx)[4],
+                                            int lane) {
   const float isd = rsqrtf((float)kD);
 #pragma unroll
   for (int side = 0; side < 2; ++side) {
     float* x = side ? vx : kx;
-    const float g = half_bits_to_f(w.rt[side] >> 16);
+    float av[4];
+    unpack4(r.row[side], av);
+    const float g = half_bits_to_f((uint16_t)r.gb[side]);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) x[e] = g * av[side][e];
-    if (!has[side]) continue;
+    for (int e = 0; e < 4; ++e) x[e] = g * av[e];
+    if (!r.has[side]) continue;
+    const float sg = half_bits_to_f((uint16_t)r.sig[side]);
+    float z[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) z[e] = a.lev[(r.code[side] >> (2 * e)) & 3u] * sg;
     if (a.naive) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) x[e] += z[side][e];
+      for (int e = 0; e < 4; ++e) x[e] += z[e];
     } else {
-      fwht128<float>(z[side]);
+      fwht128<float>(z);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) x[e] = fmaf(z[side][e] * isd, sgn_of(a, lane * 4 + e), x[e]);
+      for (int e = 0; e < 4; ++e) x[e] = fmaf(z[e] * isd, sgn_of(a, lane * 4 + e), x[e]);
     }
   }
 }
@@ -173,25 +252,27 @@ __device__ __forceinline__ float ex2f(float x) {
   return y;
 }
 
-// grid (n_split, batch * H), kRopeWarps warps; each warp takes tokens
-// t0 + warp, t0 + warp + 8, ... of its split (the tail after the N cached
-// ones).  GM: a power of two >= G (register arrays per query head).
+// grid (n_split, batch * H), kRopeWarps warps; each warp takes the 32-token
+// chunks t0 + 32 warp, t0 + 32 (warp + 8), ... of its split (the tail after
+// the N cached ones).  GM: a power of two >= G (register arrays per query
+// head).
 template <typename T, int GM>
 __global__ void __launch_bounds__(kRopeWarps * 32, GM <= 4 ? 2 : 1) rope_split_kernel(RopeArgs a, const T* __restrict__ q,
                                                                      const T* __restrict__ Kt,
                                                                      const T* __restrict__ Vt) {
   extern __shared__ __align__(16) float smr[];       // [8][G][D + 2]
-  const int split = blockIdx.x, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  __shared__ double s_freq[kD / 2];
+  const int split = blockIdx.x, bh = blockIdx.y, bb = bh / a.H, h = bh % a.H;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, G = a.G;
-  const uint8_t* comp = a.comp + (int64_t)b * a.stride;
+  const uint8_t* comp = a.comp + (int64_t)bb * a.stride;
   const T* AK = reinterpret_cast<const T*>(comp + a.L.off_anchors_k);
   const T* AV = reinterpret_cast<const T*>(comp + a.L.off_anchors_v);
-  const int T_ = a.tail_len, total = a.N + T_;
+  const int total = a.N + a.tail_len;
+  for (int i = threadIdx.x; i < kD / 2; i += blockDim.x) s_freq[i] = a.inv_freq[i];
+  __syncthreads();
+  const double* fr = s_freq + (lane & 15) * 4;
   // this KV head's queries, rotated to the decode position, scaled for exp2
   const float qs = kLog2eR * rsqrtf((float)kD);
-  double fr[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) fr[e] = a.inv_freq[(lane & 15) * 4 + e];
   float qr[GM][4], m[GM], l[GM], acc[GM][4];
 #pragma unroll
   for (int j = 0; j < GM; ++j) {
@@ -201,47 +282,50 @@ __global__ void __launch_bounds__(kRopeWarps * 32, GM <= 4 ? 2 : 1) rope_split_k
     for (int e = 0; e < 4; ++e) { acc[j][e] = 0.f; qr[j][e] = 0.f; }
     if (j < G) {
       float v[4];
-      load4r<T>(q + ((int64_t)b * a.H * G + h * G + j) * kD + lane * 4, v);
+      load4r<T>(q + ((int64_t)bb * a.H * G + h * G + j) * kD + lane * 4, v);
       rope4(fr, (int64_t)total, v, lane);
 #pragma unroll
       for (int e = 0; e < 4; ++e) qr[j][e] = v[e] * qs;
     }
   }
   const int t0 = split * a.split_tokens, t1 = min(total, t0 + a.split_tokens);
-  // the words of the next token of this warp are loaded one token ahead
-  TokWords cur, nxt;
-  if (t0 + warp < min(t1, a.N)) load_words(a, comp, h, t0 + warp, cur);
-  for (int t = t0 + warp; t < t1; t += kRopeWarps) {
-    float kx[4], vx[4];
-    if (t + kRopeWarps < min(t1, a.N)) load_words(a, comp, h, t + kRopeWarps, nxt);
-    if (t < a.N) {
-      rebuild2<T>(a, comp, t, cur, AK, AV, h, kx, vx, lane);
-      cur = nxt;
-    } else {
-      const int64_t row = (((int64_t)b * a.H + h) * a.tail_cap + (t - a.N)) * kD + lane * 4;
-      load4r<T>(Kt + row, kx);
-      load4r<T>(Vt + row, vx);
-    }
-    rope4(fr, (int64_t)t, kx, lane);
-    float dl[GM];
+  ChunkRaw cr;
+  int tc = t0 + 32 * warp;
+  if (tc < t1) chunk_load(a, comp, h, tc, lane, cr);
+  for (; tc < t1; tc += 32 * kRopeWarps) {
+    Chunk ck;
+    chunk_decode(a, tc, lane, cr, ck);
+    if (tc + 32 * kRopeWarps < t1) chunk_load(a, comp, h, tc + 32 * kRopeWarps, lane, cr);
+    const int nb = min(32, t1 - tc);
+    TokRaw<T> cur, nxt;
+    tok_issue<T>(a, comp, AK, AV, Kt, Vt, bb, h, tc, 0, ck, lane, cur);
+    for (int b = 0; b < nb; ++b) {
+      const int t = tc + b;
+      if (b + 1 < nb) tok_issue<T>(a, comp, AK, AV, Kt, Vt, bb, h, t + 1, b + 1, ck, lane, nxt);
+      float kx[4], vx[4];
+      tok_rebuild<T>(a, cur, kx, vx, lane);
+      rope4(fr, (int64_t)t, kx, lane);
+      float dl[GM];
 #pragma unroll
-    for (int j = 0; j < GM; ++j) {
-      dl[j] = qr[j][0] * kx[0];
+      for (int j = 0; j < GM; ++j) {
+        dl[j] = qr[j][0] * kx[0];
 #pragma unroll
-      for (int e = 1; e < 4; ++e) dl[j] = fmaf(qr[j][e], kx[e], dl[j]);
-    }
-    warp_sums<GM>(dl, lane);                         // log2-domain logits, on every lane
-#pragma unroll
-    for (int j = 0; j < GM; ++j) {
-      if (j < G) {
-        const float d = dl[j];
-        const float mn = fmaxf(m[j], d);
-        const float sc = ex2f(m[j] - mn), p = ex2f(d - mn);
-        l[j] = fmaf(l[j], sc, p);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[j][e] = fmaf(acc[j][e], sc, p * vx[e]);
-        m[j] = mn;
+        for (int e = 1; e < 4; ++e) dl[j] = fmaf(qr[j][e], kx[e], dl[j]);
       }
+      warp_sums<GM>(dl, lane);                       // log2-domain logits, on every lane
+#pragma unroll
+      for (int j = 0; j < GM; ++j) {
+        if (j < G) {
+          const float d = dl[j];
+          const float mn = fmaxf(m[j], d);
+          const float sc = ex2f(m[j] - mn), p = ex2f(d - mn);
+          l[j] = fmaf(l[j], sc, p);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[j][e] = fmaf(acc[j][e], sc, p * vx[e]);
+          m[j] = mn;
+        }
+      }
+      cur = nxt;
     }
   }
   // merge the warps of the CTA (fixed order) and write this split's partial
@@ -314,7 +398,7 @@ cudaError_t launch_decode_rope(const Plan& pl, const RopePlan& rp, const char* c
   a.L = pl.L;
   a.N = pl.N; a.H = pl.H; a.G = pl.G; a.k = pl.k; a.n_tiles = pl.n_tiles;
   a.n_split = rp.n_split;
-  a.split_tokens = (pl.N + tail_len + rp.n_split - 1) / rp.n_split;
+  a.split_tokens = ((pl.N + tail_len + rp.n_split - 1) / rp.n_split + 31) / 32 * 32;   // whole chunks
   a.tail_len = tail_len; a.tail_cap = tail_cap;
   a.naive = naive_codec(pl);
   a.R = pl.R;
