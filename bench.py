@@ -403,9 +403,19 @@ def cpu_baseline(spec, theta, min_seconds=10.0, max_reps=4):
         total += dt
         toks += t
         reps += 1
-    return {"value": toks / total / 1e6, "unit": UNIT, "cores": _threads(), "kind": "oracle",
-            "sample": f"{reps} x one layer, all {spec.n_kv_heads} KV heads (N={spec.n_tokens}), fp64 numpy, "
-                      f"{total:.1f} s"}
+    out = {"value": toks / total / 1e6, "unit": UNIT, "cores": _threads(), "kind": "oracle",
+           "sample": f"{reps} x one layer, all {spec.n_kv_heads} KV heads (N={spec.n_tokens}), fp64 numpy, "
+                     f"{total:.1f} s"}
+    # the same oracle on one thread (its parallelism is numpy's BLAS threads)
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            dt, t = _oracle_sample(spec, theta, 1)
+        out["single_thread"] = {"value": t / dt / 1e6, "unit": UNIT, "cores": 1,
+                                "sample": f"one layer, 1 of {spec.n_kv_heads} KV heads, {dt:.1f} s"}
+    except ImportError:
+        pass
+    return out
 
 
 def run_reference(args):
@@ -547,6 +557,33 @@ def run_gpu(args, world, rank, local):
     barrier()
     dec_us = 1e3 * reduce_max(ev2.elapsed_time(ev3), world, dev) / args.steps
 
+    # the same decode step captured once as one CUDA graph over the layers
+    # (no collective inside the try, so every rank takes the same steps)
+    graph, graph_note = None, None
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for l in range(Lr):
+                api.decode_attn(params[l], outs[l], qd[l], out=dout[l], workspace=dws)
+    except Exception as e:  # reported in the line, not fatal to the bench
+        graph, graph_note = None, f"{type(e).__name__}: {e}"[:200]
+    barrier()
+    graph_local = 1e30
+    if graph is not None:
+        graph.replay()
+        torch.cuda.synchronize(dev)
+        ev4, ev5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev4.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        ev5.record(stream)
+        torch.cuda.synchronize(dev)
+        graph_local = ev4.elapsed_time(ev5)
+    barrier()
+    graph_ms = reduce_max(graph_local, world, dev)
+    dec_graph_us = 1e3 * graph_ms / args.steps if graph_ms < 1e29 else None
+    del graph
+
     # per-stage event timing over the same steps, for the roofline of the dominant kernel
     api.stage_timing(True)
     barrier()
@@ -586,8 +623,11 @@ def run_gpu(args, world, rank, local):
                        "decode_batch": 1, "parallelism": f"replicas{world}", "compress_streams": n_cs,
                        "l2": "inputs larger than L2 (%.1f GB of K/V per step)" % (Lr * 2 * H * N * 128 * 2 / 1e9)},
             "decode_us_per_step": dec_us,
+            "decode_graph_us_per_step": dec_graph_us,
             "decode_launch": api.decode_config(params[0], 1),
             "decode_hbm_gbs": dec_bytes / (dec_us / 1e6) / 1e9,
+            "decode_graph": ({"note": "one CUDA graph holding the 32 per-layer launches, replayed per step"}
+                             if dec_graph_us is not None else {"unavailable": graph_note or "capture failed on a rank"}),
             "compressed_bytes_per_layer": L["total_bytes"],
             "uncompressed_bytes_per_layer": L["uncompressed_bytes"],
             "compression_ratio": L["uncompressed_bytes"] / L["total_bytes"],
