@@ -212,6 +212,14 @@ def reduce_max(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def graph_us_over_ranks(local_ms, steps: int, world: int, device):
+    """Microseconds per step of a replayed graph, the max over ranks, or None
+    when any rank has no time (its capture failed: local_ms is None).  One
+    collective on every rank either way."""
+    ms = reduce_max(local_ms if local_ms is not None else 1e30, world, device)
+    return 1e3 * ms / steps if ms < 1e29 else None
+
+
 def job_value(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
     """Whole-job throughput in Mtok/s: every rank's layer-head tokens over the
     slowest rank's step time."""
@@ -568,7 +576,7 @@ def run_gpu(args, world, rank, local):
     except Exception as e:  # reported in the line, not fatal to the bench
         graph, graph_note = None, f"{type(e).__name__}: {e}"[:200]
     barrier()
-    graph_local = 1e30
+    graph_local = 0.0
     if graph is not None:
         graph.replay()
         torch.cuda.synchronize(dev)
@@ -580,8 +588,7 @@ def run_gpu(args, world, rank, local):
         torch.cuda.synchronize(dev)
         graph_local = ev4.elapsed_time(ev5)
     barrier()
-    graph_ms = reduce_max(graph_local, world, dev)
-    dec_graph_us = 1e3 * graph_ms / args.steps if graph_ms < 1e29 else None
+    dec_graph_us = graph_us_over_ranks(graph_local if graph is not None else None, args.steps, world, dev)
     del graph
 
     # per-stage event timing over the same steps, for the roofline of the dominant kernel

@@ -38,7 +38,10 @@ def _worker(rank: int, world: int, port: int, out):
         n_anchor = int(len(res["anchor_pos"][0]))
         ms = bench.reduce_max(10.0 + rank, world, "cpu")           # rank 1 is the slower one
         value = bench.job_value(spec.n_tokens * spec.n_layers * spec.n_kv_heads, world, ms)
-        out[rank] = (spec.seed, spec.n_layers, ms, value, n_anchor, float(K.float().sum()))
+        # replayed-graph time: both ranks timed, then rank 1's capture failed
+        g_ok = bench.graph_us_over_ranks(4.0 + rank, 2, world, "cpu")
+        g_fail = bench.graph_us_over_ranks(4.0 if rank == 0 else None, 2, world, "cpu")
+        out[rank] = (spec.seed, spec.n_layers, ms, value, n_anchor, float(K.float().sum()), g_ok, g_fail)
     finally:
         dist.barrier()
         dist.destroy_process_group()
@@ -57,8 +60,13 @@ def test_two_gloo_ranks_shard_and_reduce():
     assert r0[2] == r1[2] == 11.0
     assert r0[3] == r1[3] == pytest.approx(300 * 2 * 1 * 2 / (11.0 / 1e3) / 1e6)
     assert r0[4] == r1[4] == O.layout(O.Params(n_tokens=300, n_kv_heads=1, n_q_heads=4, theta=0.3))["k"]
+    # the graph time is the slowest rank's, and a failed capture anywhere is reported everywhere
+    assert r0[6] == r1[6] == pytest.approx(1e3 * 5.0 / 2)
+    assert r0[7] is None and r1[7] is None
 
 
 def test_single_rank_reduce_is_identity():
     assert bench.reduce_max(7.5, 1, "cpu") == 7.5
     assert bench.job_value(1000, 1, 1.0) == pytest.approx(1.0)
+    assert bench.graph_us_over_ranks(3.0, 3, 1, "cpu") == pytest.approx(1000.0)
+    assert bench.graph_us_over_ranks(None, 3, 1, "cpu") is None
