@@ -162,10 +162,6 @@ struct CodecConst {
   uint32_t sign_bits[4];
 };
 
-__device__ __forceinline__ double sign_of(const CodecConst& cc, int j) {
-  return ((cc.sign_bits[j >> 5] >> (j & 31)) & 1u) ? -1.0 : 1.0;
-}
-
 // 16 consecutive elements of a row (32-byte aligned for bf16, 64 for fp32).
 template <typename T> __device__ __forceinline__ void load16(const T* p, float (&o)[16]);
 template <> __device__ __forceinline__ void load16<float>(const float* p, float (&o)[16]) {
