@@ -286,7 +286,11 @@ def test_compress_anchor_groups(N, anchor_div, theta):
     ("tiny-fp32-n1024", 1, 0, 10000.0, 0), ("tiny-fp32-n1024", 2, 5, 500000.0, 0),
     ("bf16-ragged-n3000", 2, 17, 500000.0, 0), ("bf16-gqa8-n2500", 1, 3, 10000.0, 0),
     ("bf16-gqa16-n1500", 2, 4, 500000.0, 0), ("bf16-n20000", 1, 40, 500000.0, 0),
-    ("bf16-ragged-n3000", 1, 2, 10000.0, 0x10)])
+    ("bf16-ragged-n3000", 1, 2, 10000.0, 0x10),
+    # one and two query heads per KV head, no residuals, every residual, and a
+    # 33-token all-anchor cache whose tail makes a second, partial 32-token chunk
+    ("fp32-window8-n700", 1, 3, 10000.0, 0), ("bf16-no-residual", 2, 0, 500000.0, 0),
+    ("bf16-every-residual", 1, 1, 10000.0, 0), ("fp32-all-anchors", 1, 2, 10000.0, 0)])
 def test_decode_rope_parity(name, batch, tail, base, mode):
     """Keys stored before the rotary map, rotated at decode (cached token t at
     position t, tail token i at N + i, the query at N + T)."""
