@@ -211,6 +211,36 @@ def test_pooling_of_a_spike():
     assert np.allclose(O.pool_scores(e, 7)[:4], 1.0) and np.all(O.pool_scores(e, 7)[4:] == 0)
 
 
+def _textbook_pooled_scores(K, Q, p, h):
+    """The anchor score of KV head h recomputed from first principles: for
+    every query head j of the head and every window row w, a textbook softmax
+    (scipy) over the positions query (j, w) can see (t <= N - W + w); the
+    weights are summed over all (j, w) at the non-window positions t < N - W,
+    then averaged over a centred kappa-wide window with zero padding (numpy's
+    'same' convolution with a box of ones, divided by kappa)."""
+    N, D = K.shape[1], K.shape[2]
+    W, G = p.window, p.group
+    score = np.zeros(N - W)
+    for j in range(h * G, (h + 1) * G):
+        for w in range(W):
+            vis = N - W + w + 1
+            a = scipy.special.softmax(K[h, :vis] @ Q[j, w] / math.sqrt(D))
+            score += a[:N - W]
+    return np.convolve(score, np.ones(p.pool_kernel), mode="same") / p.pool_kernel
+
+
+def test_pooled_scores_against_textbook_softmax():
+    """[PITH] "Assumptions & free parameters": the last W queries' attention,
+    pooled over every GQA query head of the KV head, then kappa = 7 pooling
+    (Eq. 14).  The oracle's pooled scores (the values the GPU is compared
+    with) must equal an independent per-row recomputation."""
+    K, V, Q, p = _small_layer(N=300, H=2, Hq=8)
+    st = O.compress_layer(K, V, Q, p)
+    for h in range(p.n_kv_heads):
+        ref = _textbook_pooled_scores(K, Q, p, h)
+        assert np.abs(st["pooled"][h] - ref).max() <= 1e-12 * ref.max(), h
+
+
 def test_anchor_sets():
     K, V, Q, p = _small_layer(N=700)
     L = O.layout(p)
@@ -451,3 +481,35 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     monkeypatch.setattr(O, "project", bad_proj)
     with pytest.raises(AssertionError):
         test_gamma_orthogonality_and_exact_reconstruction()
+    monkeypatch.setattr(O, "project", orig_proj)
+
+
+def test_score_pin_catches_planted_mistakes(monkeypatch):
+    """Anchor-score mistakes the textbook recomputation must catch: summing the
+    window rows of one query head only, and pooling the weights of the window
+    positions into the scores next to the window."""
+    orig_scores, orig_pool = O.token_scores, O.pool_scores
+
+    def one_head_only(alpha, n_tokens, window):
+        return alpha[:window, : n_tokens - window].sum(axis=0)
+    monkeypatch.setattr(O, "token_scores", one_head_only)
+    with pytest.raises(AssertionError):
+        test_pooled_scores_against_textbook_softmax()
+
+    # the window's weights leak into the pooling: score over all N positions,
+    # pooled, and only then cut to the non-window positions
+    n_cut = {}
+
+    def full_length(alpha, n_tokens, window):
+        n_cut["n"] = n_tokens - window
+        return alpha.sum(axis=0)
+
+    def pool_then_cut(score, kappa):
+        return orig_pool(score, kappa)[: n_cut["n"]]
+    monkeypatch.setattr(O, "token_scores", full_length)
+    monkeypatch.setattr(O, "pool_scores", pool_then_cut)
+    with pytest.raises(AssertionError):
+        test_pooled_scores_against_textbook_softmax()
+    monkeypatch.setattr(O, "token_scores", orig_scores)
+    monkeypatch.setattr(O, "pool_scores", orig_pool)
+    test_pooled_scores_against_textbook_softmax()
