@@ -191,13 +191,24 @@ def stage_roofline(stage, units, ms_per_launch, peaks):
 
 # ---------------------------------------------------------------- ranks (host logic, also used by the gloo tests)
 
-def rank_spec(spec, rank: int, layers: int = 0):
-    """The cache rank `rank` compresses: an independent seed per rank (the
-    layers of one model split over ranks share nothing), optionally fewer layers."""
-    out = type(spec)(**{**spec.__dict__, "seed": spec.seed + rank})
+def rank_spec(spec, rank: int, layers: int = 0, shard: str = "replicas"):
+    """The cache rank `rank` works on: with replicas, an independent cache per
+    rank (its own seed); with layer sharding, the one model's cache, the same
+    on every rank.  Optionally fewer layers."""
+    out = type(spec)(**{**spec.__dict__, "seed": spec.seed + (rank if shard == "replicas" else 0)})
     if layers:
         out = type(spec)(**{**out.__dict__, "n_layers": min(layers, out.n_layers)})
     return out
+
+
+def rank_layers(n_layers: int, rank: int, world: int, shard: str = "replicas") -> list:
+    """Layer indices rank `rank` compresses and decodes: every layer of its own
+    cache (replicas), or layers l = rank (mod world) of the shared model
+    (layer sharding: each layer's budget is its own, so no layer needs
+    another rank's data and no collective runs on the data path)."""
+    if shard == "replicas" or world <= 1:
+        return list(range(n_layers))
+    return [l for l in range(n_layers) if l % world == rank]
 
 
 def reduce_max(x: float, world: int, device) -> float:
@@ -235,6 +246,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--layers", type=int, default=0, help="compress only the first L layers (profiling runs)")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "layers"],
+                    help="under torchrun: every rank its own cache (replicas, weak scaling) or the layers "
+                         "of one model split over the ranks (layers, strong scaling)")
     ap.add_argument("--compress-streams", type=int, default=4,
                     help="compress layers round-robin on this many streams (independent layers overlap)")
     ap.add_argument("--sweep", action="store_true",
@@ -526,8 +540,11 @@ def run_gpu(args, world, rank, local):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     wl = WORKLOADS[WORKLOAD]
     spec, theta = wl["spec"], wl["theta"]
-    spec = rank_spec(spec, rank, args.layers)     # an independent cache per rank
-    Lr, H, N = spec.n_layers, spec.n_kv_heads, spec.n_tokens
+    spec = rank_spec(spec, rank, args.layers, args.shard)
+    ids = rank_layers(spec.n_layers, rank, world, args.shard)    # this rank's layers
+    Lr, H, N = len(ids), spec.n_kv_heads, spec.n_tokens
+    # layer-heads of the whole job per step: every rank's own cache, or the one model
+    job_layers = Lr * world if args.shard == "replicas" else spec.n_layers
 
     cpu_base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -535,12 +552,12 @@ def run_gpu(args, world, rank, local):
 
     # inputs resident in HBM: every layer's K, V, Q_obs (4.3 GB at the 8B shape)
     Ks, Vs, Qs, qd = [], [], [], []
-    for l in range(Lr):
+    for l in ids:
         K, V, Q = make_layer(spec, l, device=dev)
         Ks.append(K); Vs.append(V); Qs.append(Q)
         qd.append(make_decode_queries(spec, l, step=0, batch=1, device=dev))
     params = [api.AnchorKVParams(n_tokens=N, n_kv_heads=H, n_q_heads=spec.n_q_heads, theta=theta,
-                                 window=spec.window, dtype=spec.dtype, seed=spec.seed, layer=l) for l in range(Lr)]
+                                 window=spec.window, dtype=spec.dtype, seed=spec.seed, layer=l) for l in ids]
     L = api.anchorkv_bytes(params[0])
     outs = [torch.empty(L["total_bytes"], dtype=torch.uint8, device=dev) for _ in range(Lr)]
     ws = torch.empty(api.compress_workspace(params[0])["total_bytes"], dtype=torch.uint8, device=dev)
@@ -671,20 +688,21 @@ def run_gpu(args, world, rank, local):
                    for st in per_launch}
 
     dec_bytes = Lr * L["total_bytes"]
-    value = job_value(N * Lr * H, world, ms_step)
+    value = job_value(N * job_layers * H, 1, ms_step)
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, spec, theta, params, dev, stream, barrier, world)
+        e2e = run_e2e(args, spec, theta, params, ids, job_layers, dev, stream, barrier, world)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak" if args.shard == "replicas" else "strong",
             "vs_baseline": None, "dtype": spec.dtype, "data": "synthetic",
             "config": {"workload": WORKLOAD, "layers": Lr, "kv_heads": H, "q_heads": spec.n_q_heads,
                        "head_dim": spec.head_dim, "n_tokens": N, "window": spec.window, "theta": theta,
-                       "decode_batch": 1, "parallelism": f"replicas{world}", "compress_streams": n_cs,
+                       "decode_batch": 1, "parallelism": f"{args.shard}{world}", "compress_streams": n_cs,
                        "l2": "inputs larger than L2 (%.1f GB of K/V per step)" % (Lr * 2 * H * N * 128 * 2 / 1e9)},
             "decode_us_per_step": dec_us,
             "decode_graph_us_per_step": dec_graph_us,
@@ -712,7 +730,7 @@ def run_gpu(args, world, rank, local):
     return 0
 
 
-def run_e2e(args, spec, theta, params, dev, stream, barrier, world):
+def run_e2e(args, spec, theta, params, ids, job_layers, dev, stream, barrier, world):
     """Same step through the public API with host buffers: per layer, pinned
     K, V, Q_obs are copied in, compressed and the layout copied back; then the
     decode step copies each layer's query in and its output back."""
@@ -720,13 +738,13 @@ def run_e2e(args, spec, theta, params, dev, stream, barrier, world):
 
     from kv_cache_compression_anchorkv_b200 import api
     from kv_cache_compression_anchorkv_b200.synthetic import make_decode_queries, make_layer
-    Lr = spec.n_layers
+    Lr = len(ids)
     # host copies of the layers (pinned); the step moves all of them
     host = []
-    for l in range(Lr):
+    for l in ids:
         K, V, Q = make_layer(spec, l, device=dev)
         host.append(tuple(x.cpu().pin_memory() for x in (K, V, Q)))
-    qh = [make_decode_queries(spec, l, 0, 1, device=dev).cpu().pin_memory() for l in range(Lr)]
+    qh = [make_decode_queries(spec, l, 0, 1, device=dev).cpu().pin_memory() for l in ids]
     n_cs = max(1, args.compress_streams)
     comps = [api.HostCompressor(api.AnchorKVParams(**{**params[0].__dict__}), device=dev) for _ in range(n_cs)]
     cstreams = [torch.cuda.Stream(dev) for _ in range(n_cs)]
@@ -749,7 +767,7 @@ def run_e2e(args, spec, theta, params, dev, stream, barrier, world):
         for l in range(Lr):
             i = l % n_cs
             with torch.cuda.stream(cstreams[i]):
-                comps[i](*host[l], layer=l, host_out=outs_h[l])
+                comps[i](*host[l], layer=ids[l], host_out=outs_h[l])
                 layouts[l].copy_(comps[i].out)
                 ev = torch.cuda.Event()
                 ev.record(cstreams[i])
@@ -777,7 +795,7 @@ def run_e2e(args, spec, theta, params, dev, stream, barrier, world):
     ms = reduce_max(e0.elapsed_time(e1), world, dev) / steps
     h2d = sum(x.numel() * x.element_size() for t3 in host for x in t3) + sum(q.numel() * q.element_size() for q in qh)
     d2h = sum(o.numel() for o in outs_h) + oh.numel() * 4
-    return {"value": job_value(spec.n_tokens * Lr * spec.n_kv_heads, world, ms), "unit": UNIT,
+    return {"value": job_value(spec.n_tokens * job_layers * spec.n_kv_heads, 1, ms), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": ms, "steps": steps}
 
