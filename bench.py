@@ -183,7 +183,8 @@ def stage_roofline(stage, units, ms_per_launch, peaks):
     kind, amount, bound = units[stage]
     s = ms_per_launch / 1e3
     if kind == "flops":
-        achieved, peak, unit = amount / s / 1e12, peaks["bf16_sust"] or peaks["bf16"], "TFLOP/s"
+        # per-launch event times run at full clock: the burst bf16 peak
+        achieved, peak, unit = amount / s / 1e12, peaks["bf16"], "TFLOP/s"
     else:
         achieved, peak, unit = amount / s / 1e9, peaks["hbm"], "GB/s"
     return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak}
@@ -245,6 +246,8 @@ def main():
     ap.add_argument("--impl", default="anchorkv", choices=["anchorkv", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the 70B-shaped compress + 128-step decode and the batch-16 decode blocks")
     ap.add_argument("--layers", type=int, default=0, help="compress only the first L layers (profiling runs)")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "layers"],
                     help="under torchrun: every rank its own cache (replicas, weak scaling) or the layers "
@@ -426,11 +429,30 @@ def run_batched_decode(args):
     dws = torch.empty(api.decode_workspace_bytes(p, batch), dtype=torch.uint8, device=dev)
     rws = torch.empty(api.decode_rope_workspace_bytes(p, batch), dtype=torch.uint8, device=dev)
     reps = max(1, args.steps) * 10
-    ms = _time_ms(lambda: api.decode_attn(p, comp, q, out=o, workspace=dws), reps=reps, warm=max(3, args.warmup))
-    rope_ms = _time_ms(lambda: api.decode_attn_rope(p, comp, q, 500000.0, out=o, workspace=rws), reps=reps,
-                       warm=max(3, args.warmup))
-    peaks = _peaks()
+    # layouts below the L2 size would be re-read from L2 between repetitions:
+    # flush it with a write larger than L2 before every repetition then, and
+    # time the flush alone to take it out
     nbytes = batch * L["total_bytes"]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if nbytes < (160 << 20) else None
+
+    def timed(fn):
+        if flush is None:
+            return _time_ms(fn, reps=reps, warm=max(3, args.warmup))
+        both = _time_ms(lambda: (flush.zero_(), fn()), reps=reps, warm=max(3, args.warmup))
+        return both - _time_ms(lambda: flush.zero_(), reps=reps, warm=2)
+
+    ms = timed(lambda: api.decode_attn(p, comp, q, out=o, workspace=dws))
+    finite = bool(torch.isfinite(o).all())
+    # the same decode with the key-residual logits on the tensor cores first
+    os.environ["ANCHORKV_DECODE_KLOGIT"] = "1"
+    kws = torch.empty(api.decode_workspace_bytes(p, batch), dtype=torch.uint8, device=dev)
+    ok_ = torch.empty_like(o)
+    k_ms = timed(lambda: api.decode_attn(p, comp, q, out=ok_, workspace=kws))
+    del os.environ["ANCHORKV_DECODE_KLOGIT"]
+    k_diff = float((ok_ - o).abs().max())
+    rope_ms = timed(lambda: api.decode_attn_rope(p, comp, q, 500000.0, out=o, workspace=rws))
+    finite = finite and bool(torch.isfinite(o).all())
+    peaks = _peaks()
     gbs = nbytes / (ms * 1e-3) / 1e9
     line = {"decode_batch": batch, "n_tokens": spec.n_tokens, "kv_heads": spec.n_kv_heads,
             "q_heads": spec.n_q_heads, "theta": theta, "compressed_bytes_per_sequence": L["total_bytes"],
@@ -439,11 +461,197 @@ def run_batched_decode(args):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm"], "traffic": None, "algorithmic_bytes": nbytes,
                          "peak_source": peaks["source"] + " (copy)"},
+            "decode_tc_key_logits_us_per_layer": k_ms * 1e3,
+            "decode_tc_key_logits_gbs": nbytes / (k_ms * 1e-3) / 1e9,
+            "decode_tc_key_logits_max_abs_diff": k_diff,
             "decode_rope_us_per_layer": rope_ms * 1e3,
             "decode_rope_gbs": nbytes / (rope_ms * 1e-3) / 1e9,
-            "device_status": status, "data": "synthetic"}
+            "l2": "layouts larger than L2" if flush is None else "L2 flushed before every repetition",
+            "output_finite": finite, "device_status": status, "data": "synthetic"}
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ---------------------------------------------------------------- other configurations (one GPU)
+
+def _event_ms(fn, stream, reps):
+    """Milliseconds per call of fn() (all calls on `stream`, CUDA events)."""
+    import torch
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def run_config2(args, dev):
+    """Llama-3-70B-shaped cache: 80 layers, 8 KV / 64 query heads, D = 128,
+    N = 131072, bf16, theta = 0.05 (43 GB of K/V resident in HBM).  The full
+    compress pass (layers on four streams, as in the main step), then a
+    128-step decode at batch 1 in which step i sees i + 1 exact tokens
+    appended after the compressed prefix; per layer launch, and as one CUDA
+    graph holding all 128 steps x 80 layers."""
+    import torch
+    from kv_cache_compression_anchorkv_b200 import api
+    from kv_cache_compression_anchorkv_b200.synthetic import WORKLOADS, make_decode_queries, make_layer, make_tail
+    wl = WORKLOADS["llama70b-n128k-bf16"]
+    spec, theta = wl["spec"], wl["theta"]
+    Lr, H, N, n_steps = spec.n_layers, spec.n_kv_heads, spec.n_tokens, 128
+    stream = torch.cuda.current_stream(dev)
+    Ks, Vs, Qs, qs, tails = [], [], [], [], []
+    for l in range(Lr):
+        K, V, Q = make_layer(spec, l, device=dev)
+        Ks.append(K); Vs.append(V); Qs.append(Q)
+        qs.append(make_decode_queries(spec, l, step=0, batch=n_steps, device=dev))   # row i: step i's query
+        tails.append(make_tail(spec, l, n_steps, batch=1, device=dev))
+    params = [api.AnchorKVParams(n_tokens=N, n_kv_heads=H, n_q_heads=spec.n_q_heads, theta=theta, layer=l)
+              for l in range(Lr)]
+    L = api.anchorkv_bytes(params[0])
+    outs = [torch.empty(L["total_bytes"], dtype=torch.uint8, device=dev) for _ in range(Lr)]
+    n_cs = 4
+    cstreams = [torch.cuda.Stream(dev) for _ in range(n_cs)]
+    wss = [torch.empty(api.compress_workspace(params[0])["total_bytes"], dtype=torch.uint8, device=dev)
+           for _ in range(n_cs)]
+
+    def compress_all():
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        for cs in cstreams:
+            cs.wait_event(fork)
+        for l in range(Lr):
+            with torch.cuda.stream(cstreams[l % n_cs]):
+                api.compress(params[l], Ks[l], Vs[l], Qs[l], out=outs[l], workspace=wss[l % n_cs])
+        for cs in cstreams:
+            j = torch.cuda.Event()
+            j.record(cs)
+            stream.wait_event(j)
+
+    compress_all()
+    status = max((api.read_status(w)[0] for w in wss), key=abs)
+    reps = max(1, min(args.steps, 3))
+    c_ms = _event_ms(compress_all, stream, reps)
+    del Ks, Vs, Qs, wss
+    torch.cuda.empty_cache()
+
+    dws = torch.empty(api.decode_workspace_bytes(params[0], 1), dtype=torch.uint8, device=dev)
+    dout = torch.empty(1, spec.n_q_heads, spec.head_dim, dtype=torch.float32, device=dev)
+
+    def decode_all():
+        for i in range(n_steps):
+            for l in range(Lr):
+                api.decode_attn(params[l], outs[l], qs[l][i:i + 1], tails[l][0], tails[l][1], tail_len=i + 1,
+                                out=dout, workspace=dws)
+
+    decode_all()
+    d_ms = _event_ms(decode_all, stream, 1)
+    ok = bool(torch.isfinite(dout).all())
+    graph_us, note = None, None
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            decode_all()
+        g.replay()
+        torch.cuda.synchronize()
+        graph_us = 1e3 * _event_ms(g.replay, stream, max(1, min(args.steps, 3))) / n_steps
+        del g
+    except Exception as e:
+        note = f"{type(e).__name__}: {e}"[:200]
+    peaks = _peaks()
+    step_bytes = Lr * L["total_bytes"]
+    dec_us = 1e3 * d_ms / n_steps
+    return {"workload": "llama70b-n128k-bf16", "layers": Lr, "kv_heads": H, "q_heads": spec.n_q_heads,
+            "n_tokens": N, "theta": theta, "anchors": L["n_anchors"], "residuals_per_layer": L["n_residuals"],
+            "compressed_bytes_per_layer": L["total_bytes"],
+            "compress_ms": c_ms, "compress_mtok_s_per_layer_head": Lr * H * N / (c_ms / 1e3) / 1e6,
+            "decode_steps": n_steps, "decode_tail": "step i decodes N compressed + (i + 1) exact tokens",
+            "decode_us_per_step": dec_us, "decode_us_per_layer": dec_us / Lr,
+            "decode_graph_us_per_step": graph_us,
+            **({"decode_graph_unavailable": note} if note else {}),
+            "decode_hbm_gbs": step_bytes / (dec_us / 1e6) / 1e9,
+            "decode_hbm_frac": step_bytes / (dec_us / 1e6) / 1e9 / peaks["hbm"],
+            "output_finite": ok, "device_status": status,
+            "l2": "inputs larger than L2 (43 GB of K/V; 2.1 GB of layouts per decode step)"}
+
+
+def run_config3(args, dev):
+    """Batched decode: 16 sequences of the 8B shape (32 layers, 8 KV / 32 query
+    heads, N = 32768, bf16), each compressed on its own at theta = 0.1; one
+    decode step = 32 layer launches of batch 16.  Microseconds per step and
+    GB/s over the compressed bytes the step reads, next to the bytes an
+    uncompressed cache would read."""
+    import torch
+    from kv_cache_compression_anchorkv_b200 import api
+    from kv_cache_compression_anchorkv_b200.synthetic import WORKLOADS, make_decode_queries, make_layer
+    wl = WORKLOADS["llama8b-n32k-bf16-batch16"]
+    spec, theta, batch = wl["spec"], wl["theta"], wl["batch"]
+    Lr, H, N = spec.n_layers, spec.n_kv_heads, spec.n_tokens
+    stream = torch.cuda.current_stream(dev)
+    params = [api.AnchorKVParams(n_tokens=N, n_kv_heads=H, n_q_heads=spec.n_q_heads, theta=theta, layer=l)
+              for l in range(Lr)]
+    L = api.anchorkv_bytes(params[0])
+    stride = (L["total_bytes"] + 255) // 256 * 256
+    comp = torch.zeros(Lr, batch, stride, dtype=torch.uint8, device=dev)
+    ws, status = None, 0
+    for l in range(Lr):
+        for b in range(batch):
+            sb = type(spec)(**{**spec.__dict__, "seed": 1000 + b})
+            K, V, Q = make_layer(sb, l, device=dev)
+            out, ws = api.compress(params[l], K, V, Q, out=comp[l, b, :L["total_bytes"]], workspace=ws)
+        status = status or api.read_status(ws)[0]
+    del K, V, Q, ws
+    torch.cuda.empty_cache()
+    q = [make_decode_queries(spec, l, step=0, batch=batch, device=dev) for l in range(Lr)]
+    dws = torch.empty(api.decode_workspace_bytes(params[0], batch), dtype=torch.uint8, device=dev)
+    o = torch.empty(Lr, batch, spec.n_q_heads, spec.head_dim, dtype=torch.float32, device=dev)
+
+    def step():
+        for l in range(Lr):
+            api.decode_attn(params[l], comp[l], q[l], out=o[l], workspace=dws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    ok = bool(torch.isfinite(o).all())
+    us = 1e3 * _event_ms(step, stream, max(3, args.steps))
+    graph_us = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        g.replay()
+        graph_us = 1e3 * _event_ms(g.replay, stream, max(3, args.steps))
+        del g
+    except Exception:
+        pass
+    # the same step with the key-residual logits on the tensor cores first
+    os.environ["ANCHORKV_DECODE_KLOGIT"] = "1"
+    kws = torch.empty(api.decode_workspace_bytes(params[0], batch), dtype=torch.uint8, device=dev)
+    ko = torch.empty_like(o)
+
+    def kstep():
+        for l in range(Lr):
+            api.decode_attn(params[l], comp[l], q[l], out=ko[l], workspace=kws)
+
+    kstep()
+    k_us = 1e3 * _event_ms(kstep, stream, max(3, args.steps))
+    del os.environ["ANCHORKV_DECODE_KLOGIT"]
+    k_diff = float((ko - o).abs().max())
+    peaks = _peaks()
+    step_bytes = Lr * batch * L["total_bytes"]
+    gbs = step_bytes / (us / 1e6) / 1e9
+    return {"workload": "llama8b-n32k-bf16-batch16", "layers": Lr, "batch": batch, "theta": theta,
+            "decode_tc_key_logits_us_per_step": k_us,
+            "decode_tc_key_logits_hbm_frac": step_bytes / (k_us / 1e6) / 1e9 / peaks["hbm"],
+            "decode_tc_key_logits_max_abs_diff": k_diff,
+            "compressed_bytes_per_sequence_layer": L["total_bytes"],
+            "decode_us_per_step": us, "decode_us_per_layer": us / Lr, "decode_graph_us_per_step": graph_us,
+            "decode_hbm_gbs": gbs, "decode_hbm_frac": gbs / peaks["hbm"],
+            "decode_launch": api.decode_config(params[0], batch),
+            "uncompressed_bytes_per_step": Lr * batch * L["uncompressed_bytes"],
+            "output_finite": ok, "device_status": status,
+            "l2": "layouts larger than L2 (%.1f GB per step)" % (step_bytes / 1e9)}
 
 
 # ---------------------------------------------------------------- oracle (CPU) arm
@@ -682,7 +890,7 @@ def run_gpu(args, world, rank, local):
     roof["traffic"] = recorded_traffic(dom)
     roof["kernel"] = dom
     roof["peak_source"] = ("measured" if peaks["source"] == "measured" else "fallback") + (
-        " (sustained bf16)" if roof["unit"] == "TFLOP/s" else " (copy)")
+        " (burst bf16)" if roof["unit"] == "TFLOP/s" else " (copy)")
     stage_roofs = {st: {kk: (round(v, 4) if isinstance(v, float) else v)
                         for kk, v in stage_roofline(st, units, per_launch[st], peaks).items()}
                    for st in per_launch}
@@ -693,6 +901,16 @@ def run_gpu(args, world, rank, local):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, spec, theta, params, ids, job_layers, dev, stream, barrier, world)
+
+    # the other single-GPU configurations, on this GPU alone (not under torchrun)
+    extra = {}
+    if world == 1 and not args.no_configs:
+        del Ks, Vs, Qs, outs, wss, ws
+        torch.cuda.empty_cache()
+        extra["config2"] = run_config2(args, dev)
+        torch.cuda.empty_cache()
+        extra["config3"] = run_config3(args, dev)
+        torch.cuda.empty_cache()
 
     if rank == 0:
         line = {
@@ -720,6 +938,7 @@ def run_gpu(args, world, rank, local):
             "clocks": clk,
             "device_status": status[0],
             "e2e": e2e,
+            **extra,
         }
         if cpu_base is not None:
             line["cpu_baseline"] = cpu_base

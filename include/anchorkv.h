@@ -152,6 +152,15 @@ typedef struct anchorkv_workspace_view {
   int64_t off_pooled;      /* float [H][N]: pooled score (first N-W valid)     */
   int64_t off_utility;     /* float [2][H][N]: utility, -1 for anchors         */
   int64_t off_counters;    /* int32 [16]                                       */
+  /* float [512][kpad]: the tensor-core assignment's raw fp32 accumulators
+   * <x_t, a_s> for tokens t < min(N, 512) of the key side of KV head 0
+   * against the slots s of the first anchor group (kpad = that group's width
+   * rounded up to its chunking, at most 480); written only on the bf16
+   * tensor-core path and only when the environment variable
+   * ANCHORKV_ASSIGN_PROBE is 1 at the call.  A diagnostic that lets a test
+   * measure the accumulation error the nearest-anchor certification relies
+   * on. */
+  int64_t off_assign_probe;
 } anchorkv_workspace_view;
 
 /* Fills `p` with the pages' defaults (D = 128, W = 32, k = S/128, rho = 0.7,
@@ -185,7 +194,8 @@ int anchorkv_compress(const anchorkv_params* p, const void* K, const void* V,
                       const void* Q_obs, void* out, size_t out_bytes,
                       void* ws, size_t ws_bytes, void* stream);
 
-/* Workspace bytes anchorkv_decode_attn needs for `batch` sequences. */
+/* Workspace bytes anchorkv_decode_attn needs for `batch` sequences (0 when
+ * every (sequence, head) is decoded by a single CTA). */
 int anchorkv_decode_workspace_bytes(const anchorkv_params* p, int32_t batch, size_t* ws_bytes);
 
 /*
@@ -198,9 +208,16 @@ int anchorkv_decode_workspace_bytes(const anchorkv_params* p, int32_t batch, siz
  *               `seq_stride_bytes` bytes (>= total_bytes, multiple of 16)
  *   q           device [batch][H_q][D] dtype
  *   K_tail, V_tail device [batch][H][tail_cap][D] dtype, first tail_len valid
- *               (may be NULL when tail_len == 0)
+ *               (may be NULL when tail_len == 0), 16-byte aligned
  *   out         device [batch][H_q][D] float32
- *   ws          device, ws_bytes >= anchorkv_decode_workspace_bytes
+ *   ws          device, ws_bytes >= anchorkv_decode_workspace_bytes; the call
+ *               overwrites it (it clears its own counters on `stream` first)
+ * Every device pointer must be 16-byte aligned (EINVAL otherwise, checked
+ * before any launch).  Errors: EINVAL for a bad pointer, size or stride;
+ * ENOSPC for a small workspace; EUNSUPPORTED when batch * H > 65535,
+ * tail_len > 4096 or no launch shape fits the device.
+ * Work split: each (sequence, KV head) is cut into token slices that run on
+ * separate CTAs across the GPU; the last slice to finish merges the others.
  */
 int anchorkv_decode_attn(const anchorkv_params* p, const void* compressed,
                          int64_t seq_stride_bytes, int32_t batch, const void* q,
@@ -233,15 +250,14 @@ int anchorkv_decode_attn_rope(const anchorkv_params* p, const void* compressed,
 
 /*
  * Launch shape of anchorkv_decode_attn for `batch` sequences on the current
- * device (a diagnostic with no counterpart in the method): CTAs per
- * (sequence, KV head) thread-block cluster and dynamic shared memory per CTA.
- * Up to 8 query heads per KV head the decode runs as one cluster per
- * (sequence, head) and needs no workspace; otherwise *cluster_ctas = 0 and
- * the split-token kernels, which use the workspace, run.  Host; queries the
- * device once per shape.  EUNSUPPORTED if no cluster shape fits the device.
+ * device (a diagnostic with no counterpart in the method): token slices (one
+ * CTA each) per (sequence, KV head) and dynamic shared memory per CTA.  When
+ * the slice decode's shared-memory plan does not fit (many query heads per KV
+ * head together with many anchors), *slices = 0 and the split-token kernels
+ * run.  Host; queries the device once per shape.  EUNSUPPORTED if the slice
+ * kernel cannot be resident on the device.
  */
-int anchorkv_decode_config(const anchorkv_params* p, int32_t batch, int32_t* cluster_ctas,
-                           int32_t* smem_bytes);
+int anchorkv_decode_config(const anchorkv_params* p, int32_t batch, int32_t* slices, int32_t* smem_bytes);
 
 /*
  * Decode attention that allocates nothing.  The paper has no counterpart:
@@ -259,9 +275,12 @@ int anchorkv_decode_config(const anchorkv_params* p, int32_t batch, int32_t* clu
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
  *   - Every call on a device shares the array, which keeps the last call's
- *     contents (nothing in it needs to start at zero).  Calls that overlap on
- *     the GPU (different streams, or different host threads without ordering
- *     between their streams) race on it: order them on one stream.
+ *     contents; the words that must start at zero (per-(sequence, head)
+ *     tickets of the slice merge) are cleared by the call on its stream.
+ *     Calls that overlap on the GPU (different streams, or different host
+ *     threads without ordering between their streams) race on it: order
+ *     them on one stream.
+ *   - Pointers as for anchorkv_decode_attn (16-byte aligned, tails included).
  */
 #define ANCHORKV_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20)
 int anchorkv_decode_attn_noalloc(const anchorkv_params* p, const void* compressed,

@@ -178,12 +178,13 @@ def decode_attn_rope(p: AnchorKVParams, compressed: torch.Tensor, q: torch.Tenso
 
 
 def decode_config(p: AnchorKVParams, batch: int) -> dict:
-    """Launch shape of decode_attn on the current device: CTAs per (sequence,
-    head) cluster (0: split-token path with a workspace) and shared memory."""
+    """Launch shape of decode_attn on the current device: token slices (CTAs)
+    per (sequence, head) of the slice decode (0: the split-token kernels run)
+    and shared memory per CTA."""
     c, m = ctypes.c_int32(), ctypes.c_int32()
     capi.check("anchorkv_decode_config",
                capi.lib().anchorkv_decode_config(ctypes.byref(p.c()), batch, ctypes.byref(c), ctypes.byref(m)))
-    return {"cluster_ctas": c.value, "smem_bytes": m.value}
+    return {"slices": c.value, "smem_bytes": m.value}
 
 
 NOALLOC_SCRATCH_BYTES = 32 << 20   # ANCHORKV_DECODE_NOALLOC_SCRATCH_BYTES in include/anchorkv.h

@@ -39,7 +39,8 @@ class Layout(ctypes.Structure):
 
 class WorkspaceView(ctypes.Structure):
     _fields_ = [("total_bytes", ctypes.c_int64), ("off_pooled", ctypes.c_int64),
-                ("off_utility", ctypes.c_int64), ("off_counters", ctypes.c_int64)]
+                ("off_utility", ctypes.c_int64), ("off_counters", ctypes.c_int64),
+                ("off_assign_probe", ctypes.c_int64)]
 
 
 _P = ctypes.POINTER

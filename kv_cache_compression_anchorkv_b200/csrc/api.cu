@@ -179,6 +179,7 @@ int make_plan(const anchorkv_params* p, Plan* pl) {
   // proxy observation queries (key-as-query mode)
   pl->o_qproxy = (p->mode & ANCHORKV_MODE_KEY_QUERIES) ? take((int64_t)pl->Hq * pl->W * kD * pl->elem) : 0;
   pl->o_asg_keys = pl->k > kAssignGroupMax ? take(16 * 2 * H * N) : 0;
+  pl->o_asg_probe = take(4 * 512 * kAssignGroupMax);
   pl->ws_total = off;
   double mse;
   codebook(&pl->tau, &pl->l1, &pl->l2, &mse);
@@ -264,6 +265,7 @@ int anchorkv_compress_workspace(const anchorkv_params* p, anchorkv_workspace_vie
   out->off_pooled = pl.o_pooled;
   out->off_utility = pl.o_util;
   out->off_counters = pl.o_counters;
+  out->off_assign_probe = pl.o_asg_probe;
   return ANCHORKV_OK;
 }
 
@@ -337,7 +339,9 @@ int anchorkv_decode_attn(const anchorkv_params* p, const void* compressed, int64
   if (tail_len > 4096) return ANCHORKV_EUNSUPPORTED;
   if (seq_stride_bytes < pl.L.total_bytes && batch > 1) return ANCHORKV_EINVAL;
   if (seq_stride_bytes % 16) return ANCHORKV_EINVAL;
-  if (((uintptr_t)compressed | (uintptr_t)q | (uintptr_t)out | (uintptr_t)ws) & 15) return ANCHORKV_EINVAL;
+  if (((uintptr_t)compressed | (uintptr_t)q | (uintptr_t)out | (uintptr_t)ws | (uintptr_t)K_tail |
+       (uintptr_t)V_tail) & 15)
+    return ANCHORKV_EINVAL;
   DecodePlan dp;
   make_decode_plan(pl, batch, &dp);
   if ((int64_t)ws_bytes < dp.ws_total) return ANCHORKV_ENOSPC;
@@ -346,9 +350,8 @@ int anchorkv_decode_attn(const anchorkv_params* p, const void* compressed, int64
   if (st) return st;
   st = check_device();
   if (st) return st;
-  AKV_LAUNCH(launch_decode(pl, dp, (const char*)compressed, seq_stride_bytes, q, K_tail, V_tail, tail_len,
-                           tail_cap, out, (char*)ws, (cudaStream_t)stream));
-  return ANCHORKV_OK;
+  return launch_decode(pl, dp, (const char*)compressed, seq_stride_bytes, q, K_tail, V_tail, tail_len, tail_cap, out,
+                       (char*)ws, (cudaStream_t)stream);
 }
 
 int anchorkv_decode_rope_workspace_bytes(const anchorkv_params* p, int32_t batch, size_t* ws_bytes) {
@@ -388,23 +391,22 @@ int anchorkv_decode_attn_rope(const anchorkv_params* p, const void* compressed, 
   return ANCHORKV_OK;
 }
 
-int anchorkv_decode_config(const anchorkv_params* p, int32_t batch, int32_t* cluster_ctas, int32_t* smem_bytes) {
-  if (!cluster_ctas || !smem_bytes || batch < 1) return ANCHORKV_EINVAL;
+int anchorkv_decode_config(const anchorkv_params* p, int32_t batch, int32_t* slices, int32_t* smem_bytes) {
+  if (!slices || !smem_bytes || batch < 1) return ANCHORKV_EINVAL;
   Plan pl;
   int st = make_plan(p, &pl);
   if (st) return st;
   DecodePlan dp;
   make_decode_plan(pl, batch, &dp);
-  *cluster_ctas = 0;
+  *slices = 0;
   *smem_bytes = 0;
-  if (!dp.cluster) return ANCHORKV_OK;
+  if (!dp.flash) return ANCHORKV_OK;
   st = check_device();
   if (st) return st;
-  int C = 0, smem = 0;
-  st = decode_cluster_size(pl, batch, &C, &smem);
-  *cluster_ctas = C;
-  *smem_bytes = smem;
-  return st;
+  if (flash_ctas_per_sm(pl, dp.fs) < 1) return ANCHORKV_EUNSUPPORTED;
+  *slices = dp.fs.S;
+  *smem_bytes = dp.fs.smem;
+  return ANCHORKV_OK;
 }
 
 int anchorkv_reconstruct(const anchorkv_params* p, const void* compressed, float* K_hat, float* V_hat,

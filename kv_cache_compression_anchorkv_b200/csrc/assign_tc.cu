@@ -40,6 +40,8 @@
 // drains its own copies and MMAs, frees TMEM and returns.
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tc_util.cuh"
@@ -56,10 +58,20 @@ constexpr float kRefineRelTC = 1.0f / 8192.0f;
 
 namespace {
 
-constexpr int kGroups = 2;                    // epilogue groups (four warps each)
-constexpr int kEpiWarps = 4 * kGroups;
+#ifndef AKV_ASSIGN_COL_GROUPS
+#define AKV_ASSIGN_COL_GROUPS 1
+#endif
+#ifndef AKV_ASSIGN_ITEM_GROUPS
+#define AKV_ASSIGN_ITEM_GROUPS 2
+#endif
+#ifndef AKV_ASSIGN_CHUNK
+#define AKV_ASSIGN_CHUNK 256
+#endif
+constexpr int kGroups = AKV_ASSIGN_ITEM_GROUPS;   // item groups: epilogue groups that take whole items in turn
+constexpr int kColGroups = AKV_ASSIGN_COL_GROUPS;   // groups of four warps sharing an item's columns
+constexpr int kEpiWarps = 4 * kGroups * kColGroups;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr int kChunkMax = 256;                // anchors per MMA chunk (N of one instruction)
+constexpr int kChunkMax = AKV_ASSIGN_CHUNK;   // anchors per MMA chunk (N of one instruction)
 constexpr int kMaxBuf = 8;                    // accumulator buffers in the TMEM ring
 constexpr int kXStageBytes = 128 * 256;       // 128 rows x 128 bf16
 constexpr int kMaxKpad = 480;
@@ -69,6 +81,7 @@ struct TcArgs {
   int g0, gk, first, last;      // this launch's anchor group: slots [g0, g0 + gk)
   ulonglong2* keys;             // [2][H][N] best two 64-bit keys after earlier groups
   int total_items;
+  float* probe;                 // [512][kpad] raw accumulators of the probe rows, or null
   const float* anc_inv;
   const int* slot_of;
   const float* xnorm;
@@ -162,6 +175,37 @@ __device__ __forceinline__ void scan_pipe(uint32_t tbase, const float* ivc, floa
   }
 }
 
+// Blocks P, P + 2, ... of a chunk (one of two column groups sharing it): the
+// load of block J + 2 goes out before block J is scanned.
+template <int J>
+__device__ __forceinline__ void scan_alt(uint32_t tbase, const float* ivc, float bias, int kc, int nv,
+                                         uint32_t (&c0)[16], uint32_t (&n0)[16], Keys2& ka, Keys2& kb) {
+  constexpr int kB = kChunkMax / 16;
+  if constexpr (J < kB) {
+    if (J >= nv) return;
+    const bool l2 = J + 2 < nv;
+    if constexpr (J + 2 < kB) { if (l2) tc::tmem_ld16(tbase + (uint32_t)((J + 2) * 16), n0); }
+    scan_block<J>(c0, ivc, bias, kc, ka, kb);
+    if (l2) tc::tmem_wait_ld_dep(n0);
+    scan_alt<J + 2>(tbase, ivc, bias, kc, nv, n0, c0, ka, kb);
+  }
+}
+
+template <int P>
+__device__ __forceinline__ Keys2 scan_chunk_alt(uint32_t tbase, const float* ivc, float bias, int kc) {
+  Keys2 ka{0u, 0u}, kb{0u, 0u};
+  const int nv = (kc + 15) >> 4;
+  if (P < nv) {
+    uint32_t c0[16], n0[16];
+    tc::tmem_ld16(tbase + (uint32_t)(P * 16), c0);
+    tc::tmem_wait_ld_dep(c0);
+    scan_alt<P>(tbase, ivc, bias, kc, nv, c0, n0, ka, kb);
+  }
+  key2_push(ka, kb.b1);
+  key2_push(ka, kb.b2);
+  return ka;
+}
+
 // Best two keys of one chunk (kc valid columns of its TMEM buffer).
 __device__ __forceinline__ Keys2 scan_chunk(uint32_t tbase, const float* ivc, float bias, int kc) {
   Keys2 ka{0u, 0u}, kb{0u, 0u};
@@ -181,6 +225,10 @@ struct Ctl {
   uint32_t tmem_base;
   int err;
   int issued;          // chunks the MMA warp has issued (store-release)
+  // column groups of one item group: the second group's best two keys per
+  // row (by item parity) and a failure flag both read after their barrier
+  uint2 xchg[kGroups][2][128];
+  int pair_fail[kGroups];
 };
 
 __device__ __forceinline__ void publish_issued(int* p, int v) {
@@ -246,8 +294,12 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { tc::mbar_init(&ctl.x_full[s], 1); tc::mbar_init(&ctl.x_empty[s], 1); }
-    for (int b = 0; b < a.nbuf; ++b) { tc::mbar_init(&ctl.acc_full[b], 1); tc::mbar_init(&ctl.acc_empty[b], 128); }
+    for (int b = 0; b < a.nbuf; ++b) {
+      tc::mbar_init(&ctl.acc_full[b], 1);
+      tc::mbar_init(&ctl.acc_empty[b], 128 * kColGroups);
+    }
     ctl.issued = 0;
+    for (int i = 0; i < kGroups; ++i) ctl.pair_fail[i] = 0;
     tc::mbar_init(&ctl.anc_full, 1);
     tc::mbar_init(&ctl.anc_empty, 1);
     tc::mbar_init(&ctl.drain, 1);
@@ -345,8 +397,12 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
     // Each column score s = acc / ||a|| becomes one positive integer key
     //   key = bits(s + ||x|| (1 + 2^-7) + C) * 512 + 511 - slot,
     // so the largest key is the best score and, among equal keys, the lowest
-    // slot.  Group g takes the items beg + g, beg + g + kGroups, ... whole.
-    const int g = (warp - 2) >> 2;
+    // slot.  Item group g takes the items beg + g, beg + g + kGroups, ...;
+    // with two column groups per item group, column group cg scans the
+    // 16-column blocks cg, cg + 2, ... of every chunk and the pair merges its
+    // rows' best two keys through shared memory after each item.
+    const int g = (warp - 2) / (4 * kColGroups);
+    const int cg = ((warp - 2) >> 2) % kColGroups;
     const int qd = warp & 3;                // TMEM lane quarter this warp may access
     const int row = qd * 32 + lane;
     float* inv = winv + (size_t)(warp - 2) * a.kpad;   // this warp's copy of 1/||a||
@@ -394,7 +450,25 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
         }
         tc::fence_after_sync();
         const uint32_t tbase = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(b * a.cw);
-        Keys2 ca = scan_chunk(tbase, inv + c * a.cw, rk.add, min(a.cw, a.gk - c * a.cw));
+        const int kc = min(a.cw, a.gk - c * a.cw);
+        Keys2 ca;
+        if constexpr (kColGroups == 1) ca = scan_chunk(tbase, inv + c * a.cw, rk.add, kc);
+        else ca = cg == 0 ? scan_chunk_alt<0>(tbase, inv + c * a.cw, rk.add, kc)
+                          : scan_chunk_alt<1>(tbase, inv + c * a.cw, rk.add, kc);
+        if (a.probe && a.first && u == 0 && j < 4 && cg == 0) {
+          // diagnostic: the raw fp32 accumulators <x_t, a_s> of tokens
+          // 0..511 of the key side of head 0 (first anchor group), so a test
+          // can measure the tensor-core accumulation error directly
+          for (int blk = 0; blk < (kc + 15) / 16; ++blk) {
+            uint32_t w[16];
+            tc::tmem_ld16(tbase + (uint32_t)(blk * 16), w);
+            tc::tmem_wait_ld_dep(w);
+            float* dst = a.probe + (int64_t)(j * 128 + row) * a.kpad + c * a.cw + blk * 16;
+#pragma unroll
+            for (int e2 = 0; e2 < 16; ++e2)
+              if (blk * 16 + e2 < kc) dst[e2] = __uint_as_float(w[e2]);
+          }
+        }
         tc::fence_before_sync();
         tc::mbar_arrive(&ctl.acc_empty[b]);
         // column in chunk -> slot: the low 9 bits drop by c cw (no borrow, slot < 512)
@@ -403,6 +477,19 @@ assign_tc_kernel(const __grid_constant__ CUtensorMap mapXK, const __grid_constan
         if (ca.b2) ca.b2 -= off;
         key2_push(ka, ca.b1);
         key2_push(ka, ca.b2);
+      }
+      if constexpr (kColGroups > 1) {
+        // both column groups reach this barrier once per item, failed or
+        // not, and decide together whether to go on
+        const int par = ((it - beg) / kGroups) & 1;
+        if (cg == 1) ctl.xchg[g][par][row] = make_uint2(ka.b1, ka.b2);
+        if (!ok) ctl.pair_fail[g] = 1;
+        tc::named_bar(1 + g, 32 * 4 * kColGroups);
+        if (*(volatile int*)&ctl.pair_fail[g]) break;
+        if (cg == 1) continue;
+        const uint2 o2 = ctl.xchg[g][par][row];
+        key2_push(ka, o2.x);
+        key2_push(ka, o2.y);
       }
       if (!ok) break;
       if (t < a.N) {
@@ -505,6 +592,12 @@ cudaError_t launch_assign_tc(const Plan& pl, const void* K, const void* V, char*
     const int fixed = 1024 + (int)sizeof(Ctl) + 16 + kEpiWarps * a.kpad * 4 + a.kpad * 256;
     a.stages = std::min(4, (227 * 1024 - fixed) / kXStageBytes);
     if (a.stages < 2) return cudaErrorInvalidValue;
+    // the accumulator probe is a test hook (ANCHORKV_ASSIGN_PROBE=1): its
+    // scattered stores would hold up the CTA that owns the probe rows
+    {
+      const char* e = getenv("ANCHORKV_ASSIGN_PROBE");
+      a.probe = (e && e[0] == '1') ? reinterpret_cast<float*>(ws + pl.o_asg_probe) : nullptr;
+    }
     a.anc_inv = reinterpret_cast<const float*>(ws + pl.o_anc_inv);
     a.slot_of = reinterpret_cast<const int*>(ws + pl.o_slot_of);
     a.xnorm = reinterpret_cast<const float*>(ws + pl.o_xnorm);

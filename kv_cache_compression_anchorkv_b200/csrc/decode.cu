@@ -335,11 +335,11 @@ decode_combine_kernel(DecodeArgs a, const T* __restrict__ q, const T* __restrict
 
 int make_decode_plan(const Plan& pl, int batch, DecodePlan* dp) {
   dp->batch = batch;
-  dp->cluster = decode_cluster_supported(pl);
-  if (dp->cluster) {
+  dp->flash = flash_decode_plan(pl, batch, &dp->fs);
+  if (dp->flash) {
     dp->n_split = 0; dp->split_tokens = 0;
     dp->o_P = dp->o_qrot = dp->o_part_m = dp->o_part_l = dp->o_part_w = dp->o_part_z = 0;
-    dp->ws_total = 0;
+    dp->ws_total = dp->fs.ws_total;
     return ANCHORKV_OK;
   }
   const int units = std::max(1, batch * pl.H);
@@ -362,7 +362,8 @@ int make_decode_plan(const Plan& pl, int batch, DecodePlan* dp) {
 }
 
 int check_decode_shape(const Plan& pl, const DecodePlan& dp, int tail_len) {
-  if (dp.cluster) return ANCHORKV_OK;
+  if ((int64_t)dp.batch * pl.H > 65535) return ANCHORKV_EUNSUPPORTED;   // (sequence, head) pairs: grid y
+  if (dp.flash) return ANCHORKV_OK;
   if ((int64_t)dp.batch * pl.H > 65535) return ANCHORKV_EUNSUPPORTED;   // (sequence, head) pairs: grid y
   const size_t smem_split = sizeof(float) * ((size_t)2 * pl.G * pl.k + (size_t)pl.G * dp.split_tokens + 2 * pl.G * kD);
   const size_t smem_comb = sizeof(float) * ((size_t)pl.G * pl.k + (size_t)pl.G * std::max(tail_len, 1));
@@ -370,15 +371,9 @@ int check_decode_shape(const Plan& pl, const DecodePlan& dp, int tail_len) {
   return ANCHORKV_OK;
 }
 
-cudaError_t launch_decode(const Plan& pl, const DecodePlan& dp, const char* comp, int64_t stride, const void* q,
-                          const void* Kt, const void* Vt, int tail_len, int tail_cap, float* out, char* ws,
-                          cudaStream_t s) {
-  if (dp.cluster) {
-    cudaError_t e = cudaSuccess;
-    const int st = launch_decode_cluster(pl, dp.batch, comp, stride, q, Kt, Vt, tail_len, tail_cap, out, s, &e);
-    if (st == ANCHORKV_OK) return cudaSuccess;
-    return e != cudaSuccess ? e : cudaErrorNotSupported;
-  }
+int launch_decode(const Plan& pl, const DecodePlan& dp, const char* comp, int64_t stride, const void* q,
+                  const void* Kt, const void* Vt, int tail_len, int tail_cap, float* out, char* ws, cudaStream_t s) {
+  if (dp.flash) return launch_flash_decode(pl, dp.fs, dp.batch, comp, stride, q, Kt, Vt, tail_len, tail_cap, out, ws, s);
   DecodeArgs a;
   a.comp = reinterpret_cast<const uint8_t*>(comp);
   a.stride = stride;
@@ -430,7 +425,7 @@ cudaError_t launch_decode(const Plan& pl, const DecodePlan& dp, const char* comp
     kc<<<bh, 256, smem_comb, s>>>(a, (const T*)q, (const T*)Kt, (const T*)Vt, tail_len, tail_cap, out);
     stage_end(kStDecodeCombine, s, 1);
   }
-  return cudaGetLastError();
+  return cudaGetLastError() == cudaSuccess ? ANCHORKV_OK : ANCHORKV_ECUDA;
 }
 
 }  // namespace akv

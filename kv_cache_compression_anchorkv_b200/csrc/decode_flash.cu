@@ -1,0 +1,978 @@
+// Decode attention over compressed layouts: every (sequence, KV head) is cut
+// into token slices that run on their own CTAs across the whole GPU, one
+// launch per layer; the slices of a (sequence, head) are merged by whichever
+// of its CTAs finishes last.
+//
+// "AnchorKV: Anchor-Residual KV Cache Compression" (pith.science review),
+// Referee "Summary": a FlashAttention-style decoder rebuilds tiles when they
+// are consumed; "AnchorKV-adapted" (VeloxQuant-MLX), "Adaptation notes":
+// tokens appended during decode stay at full precision.
+//
+// The rebuild is factored so that only compressed bytes are read per token
+// (log2 units, q' = q log2(e) / sqrt(D)):
+//   q' . K^_t = g^K_t P[i(t)] + sigma~_t <qr, lev(c_t)>,   P[a] = q' . K_a[a],
+//   qr = H(s . q') / sqrt(D)      (H the unnormalised Sylvester matrix,
+//                                  s the shared sign vector; qr = q' unrotated)
+//   sum_t p_t V^_t = sum_a W[a] V_a[a] + s . H(Z) / sqrt(D),
+//   W[a] = sum_{t: i(t)=a} p_t g^V_t,  Z = sum_t p_t sigma~_t lev(c_t).
+//
+// One CTA (256 threads) owns tiles [s tps, (s+1) tps) of its (sequence, head)
+// and walks them in chunks of up to 512 tokens whose token words, bitmap
+// words, residual codes and scales are staged into shared memory by cp.async
+// (chunk c + 1 lands while chunk c is worked on).  Per chunk:
+//   a. key-residual logits, one warp per 32/G records (lane = code byte,
+//      levels from a 16-entry nibble table held in 16 bank-disjoint copies,
+//      partial dots reduced by a transposed butterfly);
+//   b. every token's logit for the G query heads (anchor term + its record's
+//      residual term, the record found by a popcount in the bitmap word);
+//   c. the chunk maximum; the running maximum moves only when the chunk beats
+//      it by 2^8, so rescaling is rare;
+//   d. probabilities, value-anchor weights W (shared-memory atomics) and the
+//      weights p sigma~ of the chunk's value records;
+//   e. value-residual sums Z in registers (lane = code byte, packed f32x2).
+// The CTA that owns the last tile also takes the exact tail tokens.  At the
+// end each CTA forms its partial output (W times the value anchors, Z turned
+// back by one Hadamard transform) and, when the (sequence, head) has several
+// slices, writes (max, sum, output) to the workspace; the last CTA to finish
+// (an atomic ticket) merges them.
+#include <algorithm>
+#include <cstdlib>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace akv {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kCTMax = 512;                // most tokens per chunk
+constexpr int kKT = kCTMax / kThreads;     // most tokens per thread and chunk
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleGap = 8.0f;        // log2 units
+// dynamic shared memory a CTA may plan for: the 227 KB opt-in limit less
+// room for the kernel's static shared memory
+constexpr int kSmemBudget = 227 * 1024 - 256;
+// most slices per (sequence, head): the merge keeps 2 x S x G floats in the
+// logit buffers (ct x G floats each, ct >= 128)
+constexpr int kMaxSlices = 128;
+
+struct FArgs {
+  const uint8_t* comp;
+  int64_t stride;
+  int64_t total;                            // layout bytes of one sequence
+  int64_t off_ak, off_av, off_tok, off_bm, off_pf, off_codes, off_sig;
+  int N, H, G, k, kp, n_tiles;
+  int64_t R;
+  float lev[4];
+  uint32_t sign_bits[4];
+  int naive;
+  const void* q;
+  const void* Kt;
+  const void* Vt;
+  int tail_len, tail_cap;
+  float* out;
+  int S, tps, ct;                           // slices per (sequence, head), tiles per slice, tokens per chunk
+  const float* rlg;                         // [B][R][GP] key-record logits from the pre-pass, or null
+  float* part;                              // [B*H][S][GP*(2+128)] partial (max, sum, output)
+  int* tickets;                             // [B*H] zeroed before the launch when S > 1
+};
+
+// Shared-memory carve-up (bytes), the same on host and device.
+struct FPlan {
+  int qs, qr, P, W, Wi, lut, pfs, wpre, red, rlog, wz, stage, stage_bytes, total;
+  // offsets inside one stage
+  int s_codes, s_sig, s_tok, s_bm;
+};
+
+__host__ __device__ inline int fa_align(int x, int a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline FPlan fplan(int GP, int kp, int ct, int tps) {
+  FPlan f;
+  int cur = 0;
+  f.qs = cur; cur += GP * kD * 4;
+  f.qr = cur; cur += GP * kD * 4;
+  f.P = cur; cur += GP * kp * 4;
+  f.W = cur; cur += GP * kp * 4;
+  f.Wi = cur; cur += 2 * GP * kp * 4;
+  f.lut = cur; cur += 16 * 16 * 8;
+  f.pfs = cur; cur = fa_align(cur + 2 * (tps + 1) * 4, 16);
+  f.wpre = cur; cur = fa_align(cur + 2 * (ct / 32 + 1) * 4, 16);
+  f.red = cur; cur = fa_align(cur + 2 * kWarps * GP * 4, 16);
+  f.rlog = cur; cur = fa_align(cur + ct * GP * 4, 16);
+  f.wz = cur; cur = fa_align(cur + ct * GP * 4, 16);
+  // stage: codes [2][ct][32], scales [2][ct + 8] (16-byte spans), token words
+  // [2][ct + 4], bitmap words [2][ct / 32]
+  int sc = 0;
+  f.s_codes = sc; sc += 2 * ct * kCodeBytes;
+  f.s_sig = sc; sc += 2 * (ct + 8) * 2;
+  f.s_tok = sc; sc += 2 * (ct + 4) * 4;
+  f.s_bm = sc; sc += 2 * (ct / 32) * 4;
+  f.stage_bytes = fa_align(sc, 16);
+  // the two stages also hold the cross-warp sums at the end ([2][warps][GP][128])
+  f.stage = fa_align(cur, 16);
+  cur = f.stage + (2 * f.stage_bytes > 2 * kWarps * GP * kD * 4 ? 2 * f.stage_bytes : 2 * kWarps * GP * kD * 4);
+  f.total = fa_align(cur, 16);
+  return f;
+}
+
+__host__ __device__ inline int gp_of(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : G <= 8 ? 8 : 16; }
+
+// ---------------------------------------------------------------- small device helpers
+
+__device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// 16-byte cp.async that copies the first `n` bytes of the source (0 < n <= 16)
+// and fills the rest of the destination with zeros.
+__device__ __forceinline__ void cp16(void* dst, const void* src, int n) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr(dst)), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Copies layout bytes [off, off + n) of one sequence into shared memory
+// starting at `dst` (16-byte aligned) from the 16-byte boundary at or below
+// `off`: the first wanted byte lands at dst + (off & 15).  Units past the end
+// of the layout are clamped (zero-filled).
+__device__ __forceinline__ void copy_span(uint8_t* dst, const uint8_t* comp, int64_t total, int64_t off, int64_t n,
+                                          int tid) {
+  if (n <= 0) return;
+  const int64_t a0 = off & ~(int64_t)15;
+  const int units = (int)((off + n - a0 + 15) >> 4);
+  for (int u = tid; u < units; u += kThreads) {
+    const int64_t o = a0 + 16 * (int64_t)u;
+    const int64_t left = total - o;
+    if (left <= 0) continue;
+    cp16(dst + 16 * u, comp + o, left >= 16 ? 16 : (int)left);
+  }
+}
+
+// Brings the 128-byte line at p into L2 (no register result, no wait).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+__device__ __forceinline__ float sign_of(const FArgs& a, int d) {
+  return ((a.sign_bits[d >> 5] >> (d & 31)) & 1u) ? -1.f : 1.f;
+}
+
+// Four consecutive elements of row `row` (lane's coordinates 4 lane ..) kept
+// raw until used; rows at or past `rows` read as zeros.
+template <typename T> struct RawRow;
+template <> struct RawRow<__nv_bfloat16> {
+  using type = uint2;
+  __device__ __forceinline__ static uint2 load(const __nv_bfloat16* base, int row, int rows, int lane) {
+    return row < rows ? *reinterpret_cast<const uint2*>(base + (int64_t)row * kD + 4 * lane) : make_uint2(0u, 0u);
+  }
+  __device__ __forceinline__ static void to_f(const uint2 v, float (&o)[4]) {
+    o[0] = __uint_as_float(v.x << 16); o[1] = __uint_as_float(v.x & 0xFFFF0000u);
+    o[2] = __uint_as_float(v.y << 16); o[3] = __uint_as_float(v.y & 0xFFFF0000u);
+  }
+};
+template <> struct RawRow<float> {
+  using type = float4;
+  __device__ __forceinline__ static float4 load(const float* base, int row, int rows, int lane) {
+    return row < rows ? *reinterpret_cast<const float4*>(base + (int64_t)row * kD + 4 * lane)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  __device__ __forceinline__ static void to_f(const float4 v, float (&o)[4]) {
+    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+  }
+};
+
+// ---------------------------------------------------------------- the kernel
+
+template <typename T, int GP>
+__global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel(FArgs a) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H, s = blockIdx.x;
+  const int G = a.G, kp = a.kp, ct = a.ct;
+  const FPlan F = fplan(GP, kp, ct, a.tps);
+  float* qs = reinterpret_cast<float*>(sm + F.qs);       // [GP][128] q' (log2 units)
+  float* qr = reinterpret_cast<float*>(sm + F.qr);       // [GP][128] rotated q'
+  float* P = reinterpret_cast<float*>(sm + F.P);         // [GP][kp]
+  float* Wt = reinterpret_cast<float*>(sm + F.W);        // [GP][kp]
+  int* Wi = reinterpret_cast<int*>(sm + F.Wi);           // [2][GP][kp] this chunk's W in fixed point (hi, lo)
+  float2* lut = reinterpret_cast<float2*>(sm + F.lut);   // [16 nibbles][16 copies]
+  int* pfs = reinterpret_cast<int*>(sm + F.pfs);         // [2][tps + 1]
+  int* wpre = reinterpret_cast<int*>(sm + F.wpre);       // [2][ct/32 + 1]
+  float* red = reinterpret_cast<float*>(sm + F.red);     // [2][kWarps][GP]
+  float* rlog = reinterpret_cast<float*>(sm + F.rlog);   // [ct][GP] key-record logits by rank
+  float* wz = reinterpret_cast<float*>(sm + F.wz);       // [ct][GP] value-record weights by rank
+
+  const uint8_t* comp = a.comp + (int64_t)b * a.stride;
+  const int t_beg = s * a.tps, t_end = min(a.n_tiles, t_beg + a.tps);
+  const int nt = t_end - t_beg;
+  const int n_chunks = (nt * kTile + ct - 1) / ct;
+  const int tiles_pc = ct / kTile;
+  const bool has_tail = (s == a.S - 1) && a.tail_len > 0;
+
+  // ---- 1. prefixes of the slice's tiles, the query, the nibble table; first token words
+  {
+    // the anchor rows are read twice later (keys for P, values at the end):
+    // start their trip to L2 now
+    const int64_t arow = (int64_t)kD * sizeof(T), abytes = (int64_t)a.k * arow;
+    const uint8_t* ak = comp + a.off_ak + (int64_t)h * abytes;
+    const uint8_t* av = comp + a.off_av + (int64_t)h * abytes;
+    for (int64_t o = (int64_t)tid * 128; o < abytes; o += (int64_t)kThreads * 128) {
+      prefetch_l2(ak + o);
+      prefetch_l2(av + o);
+    }
+    const int* pf = reinterpret_cast<const int*>(comp + a.off_pf);
+    for (int i = tid; i < 2 * (nt + 1); i += kThreads) {
+      const int side = i / (nt + 1), j = i % (nt + 1);
+      int64_t v = pf[((int64_t)side * a.H + h) * (a.n_tiles + 1) + t_beg + j];
+      v = v < 0 ? 0 : (v > a.R ? a.R : v);
+      pfs[side * (a.tps + 1) + j] = (int)v;
+    }
+    const T* q = reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.H * G + (int64_t)h * G) * kD;
+    const float qscale = kLog2e * rsqrtf((float)kD);
+    for (int i = tid; i < GP * kD; i += kThreads) {
+      const int g = i / kD;
+      qs[i] = g < G ? to_f(q[(int64_t)g * kD + (i % kD)]) * qscale : 0.f;
+    }
+    if (tid < 256) {
+      const int n = tid >> 4;
+      lut[tid] = make_float2(a.lev[n & 3], a.lev[n >> 2]);
+    }
+  }
+  // token words and bitmap words of a chunk (no prefix needed); records need the prefixes
+  auto stage_of = [&](int c) -> uint8_t* { return sm + F.stage + (c & 1) * F.stage_bytes; };
+  auto issue_words = [&](int c) {
+    uint8_t* st = stage_of(c);
+    const int c0 = t_beg + c * tiles_pc, c1 = min(t_end, c0 + tiles_pc);
+    const int tok0 = c0 * kTile, tok1 = min(a.N, c1 * kTile);
+    for (int side = 0; side < 2; ++side) {
+      const int64_t toff = a.off_tok + 4 * (((int64_t)side * a.H + h) * a.N + tok0);
+      copy_span(st + F.s_tok + side * (ct + 4) * 4, comp, a.total, toff, 4 * (int64_t)(tok1 - tok0), tid);
+      const int64_t boff = a.off_bm + 16 * (((int64_t)side * a.H + h) * a.n_tiles + c0);
+      copy_span(st + F.s_bm + side * (ct / 32) * 4, comp, a.total, boff, 16 * (int64_t)(c1 - c0), tid);
+    }
+  };
+  auto issue_records = [&](int c) {
+    uint8_t* st = stage_of(c);
+    const int j0 = c * tiles_pc, j1 = min(nt, j0 + tiles_pc);
+    for (int side = a.rlg ? 1 : 0; side < 2; ++side) {   // key logits precomputed: no key records
+      const int r0 = pfs[side * (a.tps + 1) + j0];
+      int n = pfs[side * (a.tps + 1) + j1] - r0;
+      n = n < 0 ? 0 : (n > ct ? ct : n);
+      copy_span(st + F.s_codes + side * ct * kCodeBytes, comp, a.total, a.off_codes + (int64_t)kCodeBytes * r0,
+                (int64_t)kCodeBytes * n, tid);
+      copy_span(st + F.s_sig + side * (ct + 8) * 2, comp, a.total, a.off_sig + 2 * (int64_t)r0, 2 * (int64_t)n, tid);
+    }
+  };
+  issue_words(0);
+  __syncthreads();
+  issue_records(0);
+  cp_commit();
+
+  // ---- 2. rotated query and anchor logits P (while the copies fly)
+  for (int g = warp; g < GP; g += kWarps) {
+    float v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = qs[g * kD + 4 * lane + i];
+    if (!a.naive) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] *= sign_of(a, 4 * lane + i);
+      fwht128(v);
+      const float r = rsqrtf((float)kD);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] *= r;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) qr[g * kD + 4 * lane + i] = v[i];
+  }
+  {
+    float4 q4[GP];
+#pragma unroll
+    for (int g = 0; g < GP; ++g) q4[g] = *reinterpret_cast<const float4*>(qs + g * kD + 4 * lane);
+    const T* Ka = reinterpret_cast<const T*>(comp + a.off_ak) + (int64_t)h * a.k * kD;
+    constexpr int SB = 32 / GP;
+    // the rows of the warp's next batch are loaded before this batch is
+    // reduced, so one L2 round trip overlaps the other's arithmetic
+    using Raw = typename RawRow<T>::type;
+    Raw nx[SB];
+    auto fetch = [&](int base2) {
+#pragma unroll
+      for (int i = 0; i < SB; ++i) nx[i] = RawRow<T>::load(Ka, base2 + i, a.k, lane);
+    };
+    // (with 16 or more slots per batch the batch's own loads are enough in flight)
+    constexpr bool kPipe = SB <= 8;
+    int base = warp * SB;
+    if (kPipe && base < a.k) fetch(base);
+    for (; base < a.k; base += kWarps * SB) {
+      Raw cx[SB];
+      if (kPipe) {
+#pragma unroll
+        for (int i = 0; i < SB; ++i) cx[i] = nx[i];
+        if (base + kWarps * SB < a.k) fetch(base + kWarps * SB);
+      } else {
+#pragma unroll
+        for (int i = 0; i < SB; ++i) cx[i] = RawRow<T>::load(Ka, base + i, a.k, lane);
+      }
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < SB; ++i) {
+        float x[4];
+        RawRow<T>::to_f(cx[i], x);
+#pragma unroll
+        for (int g = 0; g < GP; ++g)
+          v[i * GP + g] = fmaf(q4[g].x, x[0], fmaf(q4[g].y, x[1], fmaf(q4[g].z, x[2], q4[g].w * x[3])));
+      }
+      transpose_reduce32(v, lane);
+      const int slot = base + lane / GP;
+      if (slot < a.k) P[(lane % GP) * kp + slot] = v[0];
+    }
+  }
+  for (int i = tid; i < GP * kp; i += kThreads) {
+    Wt[i] = 0.f;
+    Wi[i] = 0;
+    Wi[GP * kp + i] = 0;
+  }
+
+  // running state (identical in every thread): max per head; per-thread sums
+  float mrun[GP], lsum[GP];
+  float2 z01[GP], z23[GP];          // value-residual sums for dims 4 lane .. 4 lane + 3
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    mrun[g] = -INFINITY;
+    lsum[g] = 0.f;
+    z01[g] = make_float2(0.f, 0.f);
+    z23[g] = make_float2(0.f, 0.f);
+  }
+  float2 qr01[GP], qr23[GP];
+  __syncthreads();
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    const float4 t4 = *reinterpret_cast<const float4*>(qr + g * kD + 4 * lane);
+    qr01[g] = make_float2(t4.x, t4.y);
+    qr23[g] = make_float2(t4.z, t4.w);
+  }
+  const float2* lutc = lut + (lane & 15);
+
+  // Raises the running maximum to the chunk maximum `cm` when it beats it by
+  // the gap, rescaling every accumulator (CTA-uniform decision).
+  // Raises the running maximum to the chunk maximum `cm` when it beats it by
+  // the gap, rescaling the running sums and W (a CTA-uniform decision); the
+  // factors applied are left in f (1 where the maximum stayed).
+  auto update_max = [&](const float (&cm)[GP], float (&f)[GP]) {
+    bool any = false;
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      f[g] = 1.f;
+      if (mrun[g] == -INFINITY) {
+        mrun[g] = cm[g];
+      } else if (cm[g] > mrun[g] + kRescaleGap) {
+        f[g] = exp2f(mrun[g] - cm[g]);
+        mrun[g] = cm[g];
+        any = true;
+      }
+    }
+    if (any) {
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        lsum[g] *= f[g];
+        z01[g].x *= f[g]; z01[g].y *= f[g]; z23[g].x *= f[g]; z23[g].y *= f[g];
+        for (int i = tid; i < kp; i += kThreads) Wt[g * kp + i] *= f[g];
+      }
+      __syncthreads();
+    }
+  };
+  // CTA-wide maximum per head of per-thread values (all threads get it).
+  auto block_max = [&](float (&v)[GP], float (&out)[GP]) {
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      const float m = warp_max(v[g]);
+      if (lane == 0) red[warp * GP + g] = m;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      float m = red[g];
+#pragma unroll
+      for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red[w * GP + g]);
+      out[g] = m;
+    }
+  };
+
+  // CTA-wide maxima per head of per-thread values, and of one more value.
+  auto block_max2 = [&](float (&v)[GP], float x, float (&out)[GP], float& xout) {
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      const float m = warp_max(v[g]);
+      if (lane == 0) red[warp * (GP + 1) + g] = m;
+    }
+    const float mx = warp_max(x);
+    if (lane == 0) red[warp * (GP + 1) + GP] = mx;
+    __syncthreads();
+#pragma unroll
+    for (int g = 0; g <= GP; ++g) {
+      float m = red[g];
+#pragma unroll
+      for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red[w * (GP + 1) + g]);
+      if (g < GP) out[g] = m;
+      else xout = m;
+    }
+  };
+
+  // ---- 3. chunks
+  for (int c = 0; c < n_chunks; ++c) {
+    // chunk c has landed; past this barrier every thread is done with chunk
+    // c - 1, so its buffer takes chunk c + 1 while chunk c is worked on
+    cp_wait<0>();
+    __syncthreads();
+    if (c + 1 < n_chunks) {
+      issue_words(c + 1);
+      issue_records(c + 1);
+      cp_commit();
+    }
+    const uint8_t* st = stage_of(c);
+    const uint8_t* codes = st + F.s_codes;
+    const int j0 = c * tiles_pc, j1 = min(nt, j0 + tiles_pc);
+    const int tok0 = (t_beg + j0) * kTile, ntok = min(a.N, (t_beg + j1) * kTile) - tok0;
+    int rbase[2], nrec[2], sh_sig[2], sh_tok[2];
+#pragma unroll
+    for (int side = 0; side < 2; ++side) {
+      rbase[side] = pfs[side * (a.tps + 1) + j0];
+      int n = pfs[side * (a.tps + 1) + j1] - rbase[side];
+      nrec[side] = n < 0 ? 0 : (n > ct ? ct : n);
+      sh_sig[side] = (int)((a.off_sig + 2 * (int64_t)rbase[side]) & 15) / 2;
+      sh_tok[side] = (int)((a.off_tok + 4 * (((int64_t)side * a.H + h) * a.N + tok0)) & 15) / 4;
+    }
+    const uint32_t* bm0 = reinterpret_cast<const uint32_t*>(st + F.s_bm);
+    const uint16_t* sig0 = reinterpret_cast<const uint16_t*>(st + F.s_sig);
+    const uint32_t* tok0p = reinterpret_cast<const uint32_t*>(st + F.s_tok);
+    const int nwords = (ntok + 31) >> 5;
+
+    // a. bitmap word prefixes (warp = side) and key-residual logits
+    if (warp < 2) {
+      const int side = warp;
+      const uint32_t w = lane < nwords ? bm0[side * (ct / 32) + lane] : 0u;
+      int x = __popc(w);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane < ct / 32) wpre[side * (ct / 32 + 1) + lane + 1] = x;
+      if (lane == 0) wpre[side * (ct / 32 + 1)] = 0;
+    }
+    if (a.rlg) {
+      // key-record logits from the tensor-core pre-pass (sigma~ included)
+      const int nK = nrec[0];
+      const float* src = a.rlg + ((int64_t)b * a.R + rbase[0]) * GP;
+      for (int i = tid; i < nK * GP; i += kThreads) rlog[i] = src[i];
+    } else {
+      constexpr int RB = 32 / GP;
+      const int nK = nrec[0];
+      for (int base = warp * RB; base < nK; base += kWarps * RB) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < RB; ++i) {
+          const int r = base + i;
+          const uint32_t byte = r < nK ? codes[r * kCodeBytes + lane] : 0u;
+          const float2 l01 = lutc[(byte & 15u) * 16], l23 = lutc[(byte >> 4) * 16];
+#pragma unroll
+          for (int g = 0; g < GP; ++g) {
+            float2 t2 = __fmul2_rn(l01, qr01[g]);
+            t2 = __ffma2_rn(l23, qr23[g], t2);
+            v[i * GP + g] = t2.x + t2.y;
+          }
+        }
+        transpose_reduce32(v, lane);
+        const int r = base + lane / GP;
+        if (r < nK) rlog[r * GP + (lane % GP)] = v[0] * half_bits_to_f(sig0[sh_sig[0] + r]);
+      }
+    }
+    __syncthreads();
+
+    // b. token logits (their maximum only; phase d recomputes them) and the
+    //    value side's slot and coefficient
+    float cmx[GP];
+    int slv[kKT];
+    float gmv[kKT];
+    float gabs = 0.f;
+#pragma unroll
+    for (int g = 0; g < GP; ++g) cmx[g] = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kKT; ++i) {
+      const int t = tid + i * kThreads;
+      slv[i] = 0;
+      gmv[i] = 0.f;
+      if (t < ntok) {
+        const uint32_t wv = tok0p[(ct + 4) + sh_tok[1] + t];
+        slv[i] = min((int)(wv & 0xFFFFu), a.k - 1);
+        gmv[i] = half_bits_to_f(wv >> 16);
+        gabs = fmaxf(gabs, fabsf(gmv[i]));
+        const uint32_t wk = tok0p[sh_tok[0] + t];
+        const int slot = min((int)(wk & 0xFFFFu), a.k - 1);
+        const float gam = half_bits_to_f(wk >> 16);
+        const uint32_t word = bm0[t >> 5];
+        const uint32_t below = word & ((1u << (t & 31)) - 1u);
+        const int rank = wpre[t >> 5] + __popc(below);
+        const bool res = ((word >> (t & 31)) & 1u) && rank < nrec[0];
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          float x = gam * P[g * kp + slot];
+          if (res) x += rlog[rank * GP + g];
+          cmx[g] = fmaxf(cmx[g], x);
+        }
+      }
+    }
+    // c. chunk maximum, running maximum; fixed-point scale of the chunk's
+    //    anchor weights: |p gamma| <= 2^(cm - m) max|gamma|, ntok terms per
+    //    slot at most, so sum * 2^e stays below 2^30
+    float cm[GP], gmax, fsc[GP];
+    block_max2(cmx, gabs, cm, gmax);
+    update_max(cm, fsc);
+    // wsc = 2^e, winv = 2^-e, e = 30 - ceil(log2 ntok) - ceil(log2 bound)
+    float wsc[GP], winv[GP];
+    const int en = 32 - __clz(ntok);
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      const float bound = exp2f(cm[g] - mrun[g]) * gmax;
+      int eb = bound > 0.f ? (int)((__float_as_uint(bound) >> 23) & 255u) - 126 : 0;   // bound < 2^eb
+      int e = 30 - en - eb;
+      e = max(-100, min(100, e));
+      wsc[g] = __uint_as_float((uint32_t)(e + 127) << 23);
+      winv[g] = __uint_as_float((uint32_t)(127 - e) << 23);
+    }
+    // d. probabilities, anchor weights (native integer atomics on the fixed
+    //    point), value-record weights
+#pragma unroll
+    for (int i = 0; i < kKT; ++i) {
+      const int t = tid + i * kThreads;
+      if (t < ntok) {
+        // this token's logits again (anchor term + key residual term)
+        float lgt[GP];
+        {
+          const uint32_t wk = tok0p[sh_tok[0] + t];
+          const int kslot = min((int)(wk & 0xFFFFu), a.k - 1);
+          const float kgam = half_bits_to_f(wk >> 16);
+          const uint32_t kword = bm0[t >> 5];
+          const int krank = wpre[t >> 5] + __popc(kword & ((1u << (t & 31)) - 1u));
+          const bool kres = ((kword >> (t & 31)) & 1u) && krank < nrec[0];
+#pragma unroll
+          for (int g = 0; g < GP; ++g) {
+            float x = kgam * P[g * kp + kslot];
+            if (kres) x += rlog[krank * GP + g];
+            lgt[g] = x;
+          }
+        }
+        const int slot = slv[i];
+        const float gam = gmv[i];
+        const uint32_t word = bm0[ct / 32 + (t >> 5)];
+        const int rank = wpre[ct / 32 + 1 + (t >> 5)] + __popc(word & ((1u << (t & 31)) - 1u));
+        const bool res = ((word >> (t & 31)) & 1u) && rank < nrec[1];
+        const float sg = res ? half_bits_to_f(sig0[(ct + 8) + sh_sig[1] + rank]) : 0.f;
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          const float p = exp2f(lgt[g] - mrun[g]);
+          lsum[g] += p;
+          // two native integer adds: the scaled term's integer part, then its
+          // rounded remainder scaled by 2^20 (2^-(e+20) resolution overall)
+          const float x = p * gam * wsc[g];
+          const float xh = rintf(x);
+          atomicAdd(&Wi[g * kp + slot], (int)xh);
+          atomicAdd(&Wi[GP * kp + g * kp + slot], __float2int_rn((x - xh) * 1048576.0f));
+          if (res) wz[rank * GP + g] = p * sg;
+        }
+      }
+    }
+    __syncthreads();
+    // e. the chunk's fixed-point anchor weights into W (and cleared); value-residual sums
+    {
+      int4* hi4 = reinterpret_cast<int4*>(Wi);
+      int4* lo4 = reinterpret_cast<int4*>(Wi + GP * kp);
+      float4* w4 = reinterpret_cast<float4*>(Wt);
+      const int per = kp >> 2;          // kp is a multiple of 4
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        const float ih = winv[g], il = winv[g] * (1.0f / 1048576.0f);
+        for (int i = tid; i < per; i += kThreads) {
+          const int4 vh = hi4[g * per + i], vl = lo4[g * per + i];
+          float4 w = w4[g * per + i];
+          w.x += fmaf((float)vl.x, il, (float)vh.x * ih);
+          w.y += fmaf((float)vl.y, il, (float)vh.y * ih);
+          w.z += fmaf((float)vl.z, il, (float)vh.z * ih);
+          w.w += fmaf((float)vl.w, il, (float)vh.w * ih);
+          w4[g * per + i] = w;
+          hi4[g * per + i] = make_int4(0, 0, 0, 0);
+          lo4[g * per + i] = make_int4(0, 0, 0, 0);
+        }
+      }
+    }
+    {
+      const int nV = nrec[1];
+      const uint8_t* vcodes = codes + ct * kCodeBytes;
+      // four records per step, their loads issued before any arithmetic
+      constexpr int kU = 4;
+      for (int r0 = warp; r0 < nV; r0 += kU * kWarps) {
+        uint32_t byte[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int r = r0 + u * kWarps;
+          byte[u] = r < nV ? vcodes[r * kCodeBytes + lane] : 0u;
+        }
+        float2 l01[kU], l23[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          l01[u] = lutc[(byte[u] & 15u) * 16];
+          l23[u] = lutc[(byte[u] >> 4) * 16];
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int r = r0 + u * kWarps;
+          if (r < nV) {
+            const float* wr = wz + r * GP;
+#pragma unroll
+            for (int g = 0; g < GP; ++g) {
+              const float2 ww = make_float2(wr[g], wr[g]);
+              z01[g] = __ffma2_rn(l01[u], ww, z01[g]);
+              z23[g] = __ffma2_rn(l23[u], ww, z23[g]);
+            }
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- 4. exact tail tokens (last slice): logits in rlog, then values
+  float4 oacc[GP];                  // tail values, then anchor values, dims 4 lane ..
+#pragma unroll
+  for (int g = 0; g < GP; ++g) oacc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (has_tail) {
+    float4 q4[GP];
+#pragma unroll
+    for (int g = 0; g < GP; ++g) q4[g] = *reinterpret_cast<const float4*>(qs + g * kD + 4 * lane);
+    const T* Kt = reinterpret_cast<const T*>(a.Kt) + ((int64_t)b * a.H + h) * a.tail_cap * kD;
+    const T* Vt = reinterpret_cast<const T*>(a.Vt) + ((int64_t)b * a.H + h) * a.tail_cap * kD;
+    for (int t0 = 0; t0 < a.tail_len; t0 += ct) {
+      const int n = min(ct, a.tail_len - t0);
+      for (int i = warp; i < n; i += kWarps) {
+        float x[4];
+        load4(Kt + (int64_t)(t0 + i) * kD + 4 * lane, x);
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          const float d = warp_sum(fmaf(q4[g].x, x[0], fmaf(q4[g].y, x[1], fmaf(q4[g].z, x[2], q4[g].w * x[3]))));
+          if (lane == 0) rlog[i * GP + g] = d;
+        }
+      }
+      __syncthreads();
+      float cmx[GP], cm[GP];
+#pragma unroll
+      for (int g = 0; g < GP; ++g) cmx[g] = -INFINITY;
+      for (int i = tid; i < n; i += kThreads)
+#pragma unroll
+        for (int g = 0; g < GP; ++g) cmx[g] = fmaxf(cmx[g], rlog[i * GP + g]);
+      float fsc[GP];
+      block_max(cmx, cm);
+      update_max(cm, fsc);
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        oacc[g].x *= fsc[g]; oacc[g].y *= fsc[g]; oacc[g].z *= fsc[g]; oacc[g].w *= fsc[g];
+      }
+      for (int i = tid; i < n * GP; i += kThreads) {
+        const float p = exp2f(rlog[i] - mrun[i % GP]);
+        rlog[i] = p;
+      }
+      __syncthreads();
+      // probabilities were written by other threads: sum them per head here
+      for (int i = tid; i < n; i += kThreads)
+#pragma unroll
+        for (int g = 0; g < GP; ++g) lsum[g] += rlog[i * GP + g];
+      for (int i = warp; i < n; i += kWarps) {
+        float x[4];
+        load4(Vt + (int64_t)(t0 + i) * kD + 4 * lane, x);
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          const float p = rlog[i * GP + g];
+          oacc[g].x = fmaf(p, x[0], oacc[g].x); oacc[g].y = fmaf(p, x[1], oacc[g].y);
+          oacc[g].z = fmaf(p, x[2], oacc[g].z); oacc[g].w = fmaf(p, x[3], oacc[g].w);
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  // ---- 5. partial output of this slice
+  // sum of probabilities per head (per warp; summed where used)
+  {
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      const float v = warp_sum(lsum[g]);
+      if (lane == 0) red[kWarps * GP + warp * GP + g] = v;
+    }
+  }
+  // value anchors weighted by W (W is final after the last chunk's barrier)
+  {
+    const T* Va = reinterpret_cast<const T*>(comp + a.off_av) + (int64_t)h * a.k * kD;
+#pragma unroll 16
+    for (int slot = warp; slot < a.k; slot += kWarps) {
+      float x[4];
+      load4(Va + (int64_t)slot * kD + 4 * lane, x);
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        const float w = Wt[g * kp + slot];
+        oacc[g].x = fmaf(w, x[0], oacc[g].x); oacc[g].y = fmaf(w, x[1], oacc[g].y);
+        oacc[g].z = fmaf(w, x[2], oacc[g].z); oacc[g].w = fmaf(w, x[3], oacc[g].w);
+      }
+    }
+  }
+  // cross-warp sums of the anchor/tail values and of Z, through the stage buffers
+  float* ored = reinterpret_cast<float*>(sm + F.stage);          // [kWarps][GP][128]
+  float* zred = ored + kWarps * GP * kD;                           // [kWarps][GP][128]
+  __syncthreads();    // every chunk is consumed and no copy is in flight
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    *reinterpret_cast<float4*>(ored + (warp * GP + g) * kD + 4 * lane) = oacc[g];
+    *reinterpret_cast<float4*>(zred + (warp * GP + g) * kD + 4 * lane) =
+        make_float4(z01[g].x, z01[g].y, z23[g].x, z23[g].y);
+  }
+  __syncthreads();
+  // Z turned back to the token domain: s . H(Z) / sqrt(D) (unrotated codec: Z)
+  for (int g = warp; g < GP; g += kWarps) {
+    float z[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int w = 0; w < kWarps; ++w) {
+      const float4 t4 = *reinterpret_cast<const float4*>(zred + (w * GP + g) * kD + 4 * lane);
+      z[0] += t4.x; z[1] += t4.y; z[2] += t4.z; z[3] += t4.w;
+    }
+    if (!a.naive) {
+      fwht128(z);
+      const float r = rsqrtf((float)kD);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) z[i] *= sign_of(a, 4 * lane + i) * r;
+    }
+    // slot 0 of the warp sums takes the total (read only by this warp below)
+    *reinterpret_cast<float4*>(zred + g * kD + 4 * lane) = make_float4(z[0], z[1], z[2], z[3]);
+  }
+  __syncthreads();
+  // o[g][d] = sum over warps of the anchor/tail values + Z term, relative to mrun
+  float* opart = qr;   // reuse: [GP][128]
+  for (int i = tid; i < GP * kD; i += kThreads) {
+    const int g = i / kD;
+    float v = zred[i];
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) v += ored[(w * GP + g) * kD + (i % kD)];
+    opart[i] = v;
+  }
+  __syncthreads();
+  const int Hq = a.H * G;
+  float* out = a.out + ((int64_t)b * Hq + (int64_t)h * G) * kD;
+  auto total_l = [&](int g) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) v += red[kWarps * GP + w * GP + g];
+    return v;
+  };
+  if (a.S == 1) {
+    for (int i = tid; i < G * kD; i += kThreads) out[i] = opart[i] / total_l(i / kD);
+    return;
+  }
+  // several slices: publish this one, the last to finish merges
+  const int PW = GP * (2 + kD);
+  float* mine = a.part + ((int64_t)bh * a.S + s) * PW;
+  for (int i = tid; i < GP * kD; i += kThreads) mine[2 * GP + i] = opart[i];
+#pragma unroll
+  for (int g = 0; g < GP; ++g)
+    if (tid == g) {
+      mine[g] = mrun[g];
+      mine[GP + g] = total_l(g);
+    }
+  __threadfence();
+  __syncthreads();
+  __shared__ int last;
+  if (tid == 0) last = atomicAdd(&a.tickets[bh], 1) == a.S - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  const float* all = a.part + (int64_t)bh * a.S * PW;
+  // every slice's (max, sum) per head in one round of loads, then the
+  // slices' weights 2^(m_s - M) / L per head; the outputs' loads go out together
+  float* ms = rlog;                    // [S][GP] maxima, then weights (S <= kMaxSlices)
+  float* ls = wz;                      // [S][GP] sums
+  for (int i = tid; i < a.S * GP; i += kThreads) {
+    const int j = i / GP, g = i % GP;
+    ms[i] = __ldcg(all + (int64_t)j * PW + g);
+    ls[i] = __ldcg(all + (int64_t)j * PW + GP + g);
+  }
+  __syncthreads();
+  if (tid < GP) {
+    float M = -INFINITY;
+    for (int j = 0; j < a.S; ++j) M = fmaxf(M, ms[j * GP + tid]);
+    float lt = 0.f;
+    for (int j = 0; j < a.S; ++j) {
+      const float f = exp2f(ms[j * GP + tid] - M);
+      ms[j * GP + tid] = f;
+      lt = fmaf(ls[j * GP + tid], f, lt);
+    }
+    for (int j = 0; j < a.S; ++j) ms[j * GP + tid] /= lt;
+  }
+  __syncthreads();
+  for (int i = tid; i < G * kD; i += kThreads) {
+    const int g = i / kD;
+    float o = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < a.S; ++j) o = fmaf(__ldcg(all + (int64_t)j * PW + 2 * GP + i), ms[j * GP + g], o);
+    out[i] = o;
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+// Resident CTAs per SM at `smem` bytes of dynamic shared memory (0: none).
+// The kernel's dynamic shared-memory limit is raised once to the largest a
+// CTA may use, so every later shape launches without touching it.
+template <typename T, int GP>
+int max_ctas_per_sm(int smem) {
+  static std::mutex mu;
+  static int cache_smem[8] = {0}, cache_n[8] = {0}, n_cache = 0;
+  static int dev_set = -1;
+  std::lock_guard<std::mutex> lock(mu);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev != dev_set) {
+    // the opt-in maximum per block, less the kernel's static shared memory
+    int optin = 0;
+    cudaFuncAttributes fa;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa, flash_decode_kernel<T, GP>) != cudaSuccess)
+      return 0;
+    if (cudaFuncSetAttribute(flash_decode_kernel<T, GP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             optin - (int)fa.sharedSizeBytes) != cudaSuccess)
+      return 0;
+    dev_set = dev;
+    n_cache = 0;
+  }
+  for (int i = 0; i < n_cache; ++i)
+    if (cache_smem[i] == smem) return cache_n[i];
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, flash_decode_kernel<T, GP>, kThreads, smem) != cudaSuccess)
+    n = 0;
+  if (n_cache < 8) { cache_smem[n_cache] = smem; cache_n[n_cache] = n; ++n_cache; }
+  return n;
+}
+
+}  // namespace
+
+// Shape of the slice decode for `batch` sequences: tokens per chunk, slices
+// per (sequence, head) and the workspace.  Returns false when no chunk size
+// fits the shared memory (the split-token kernels take over).
+bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs) {
+  const int GP = gp_of(pl.G);
+  const int kp = (pl.k + 3) & ~3;
+  // CTAs resident per SM: two when the registers allow it (G <= 4) and the
+  // shared memory of the largest chunk size that fits does; the slice plan
+  // is sized for the whole head, which bounds every slice
+  static const int kChunkSizes[4] = {512, 384, 256, 128};
+  int per_sm = GP <= 4 ? 2 : 1;
+  const char* env = getenv("ANCHORKV_DECODE_CTAS_PER_SM");
+  if (env && env[0]) per_sm = std::max(1, std::min(per_sm, atoi(env)));
+  fs->ct = 0;
+  for (; per_sm >= 1 && !fs->ct; --per_sm)
+    for (int ct : kChunkSizes) {
+      const int need = fplan(GP, kp, ct, pl.n_tiles).total;
+      if (need <= kSmemBudget && (need + 1024) * per_sm <= 228 * 1024) { fs->ct = ct; break; }
+    }
+  if (!fs->ct) return false;
+  ++per_sm;                      // the loop stepped past the count that fit
+  const int units = std::max(1, batch * pl.H);
+  const int target = 148 * per_sm;
+  int S = std::max(1, std::min({pl.n_tiles, target / units, kMaxSlices}));
+  int tps = (pl.n_tiles + S - 1) / S;
+  S = (pl.n_tiles + tps - 1) / tps;
+  fs->S = S;
+  fs->tps = tps;
+  fs->smem = fplan(GP, kp, fs->ct, tps).total;
+  // key-residual logits on the tensor cores ahead of the decode: worth it
+  // when the launch is throughput-bound (a slice or two per head), not at
+  // batch 1 where latency rules; ANCHORKV_DECODE_KLOGIT=0/1 forces it
+  const char* kenv = getenv("ANCHORKV_DECODE_KLOGIT");
+  fs->klogit = klogit_tc_supported(pl) && pl.R > 0 &&
+               (kenv && kenv[0] ? kenv[0] == '1' : false);
+  int64_t off = 0;
+  auto take = [&](int64_t bytes) { int64_t o = off; off += (bytes + 255) / 256 * 256; return o; };
+  fs->o_tickets = S > 1 ? take(4 * (int64_t)units) : 0;
+  fs->o_part = S > 1 ? take(4 * (int64_t)units * S * GP * (2 + kD)) : 0;
+  fs->o_rlog = fs->klogit ? take(klogit_ws_bytes(pl, batch)) : 0;
+  fs->ws_total = off;
+  return true;
+}
+
+int launch_flash_decode(const Plan& pl, const FlashShape& fs, int batch, const char* comp, int64_t stride,
+                        const void* q, const void* Kt, const void* Vt, int tail_len, int tail_cap, float* out,
+                        char* ws, cudaStream_t s) {
+  FArgs a;
+  a.comp = reinterpret_cast<const uint8_t*>(comp);
+  a.stride = stride;
+  a.total = pl.L.total_bytes;
+  a.off_ak = pl.L.off_anchors_k; a.off_av = pl.L.off_anchors_v; a.off_tok = pl.L.off_tok;
+  a.off_bm = pl.L.off_bitmap; a.off_pf = pl.L.off_tile_prefix; a.off_codes = pl.L.off_res_codes;
+  a.off_sig = pl.L.off_res_sigma;
+  a.N = pl.N; a.H = pl.H; a.G = pl.G; a.k = pl.k; a.kp = (pl.k + 3) & ~3; a.n_tiles = pl.n_tiles;
+  a.R = pl.R;
+  a.lev[0] = (float)-pl.l2; a.lev[1] = (float)-pl.l1; a.lev[2] = (float)pl.l1; a.lev[3] = (float)pl.l2;
+  for (int i = 0; i < 4; ++i) a.sign_bits[i] = pl.sign_bits[i];
+  a.naive = naive_codec(pl);
+  a.q = q; a.Kt = Kt; a.Vt = Vt; a.tail_len = tail_len; a.tail_cap = tail_cap; a.out = out;
+  a.S = fs.S; a.tps = fs.tps; a.ct = fs.ct;
+  a.rlg = fs.klogit ? reinterpret_cast<const float*>(ws + fs.o_rlog) : nullptr;
+  a.part = fs.S > 1 ? reinterpret_cast<float*>(ws + fs.o_part) : nullptr;
+  a.tickets = fs.S > 1 ? reinterpret_cast<int*>(ws + fs.o_tickets) : nullptr;
+  if (fs.S > 1 && cudaMemsetAsync(a.tickets, 0, 4 * (size_t)batch * pl.H, s) != cudaSuccess) return ANCHORKV_ECUDA;
+  if (fs.klogit) {
+    const int st = launch_klogit_tc(pl, batch, comp, stride, q, reinterpret_cast<float*>(ws + fs.o_rlog), s);
+    if (st) return st;
+  }
+  const dim3 grid(fs.S, batch * pl.H);
+  const int GP = gp_of(pl.G);
+  cudaError_t e = cudaSuccess;
+  auto go = [&](auto kernel, int n_ok) {
+    if (n_ok < 1) { e = cudaErrorNotSupported; return; }
+    kernel<<<grid, kThreads, fs.smem, s>>>(a);
+    e = cudaGetLastError();
+  };
+  stage_begin(kStDecodeCluster, s);
+  if (pl.p.dtype == ANCHORKV_BF16) {
+    using T = __nv_bfloat16;
+    switch (GP) {
+      case 1: go(flash_decode_kernel<T, 1>, max_ctas_per_sm<T, 1>(fs.smem)); break;
+      case 2: go(flash_decode_kernel<T, 2>, max_ctas_per_sm<T, 2>(fs.smem)); break;
+      case 4: go(flash_decode_kernel<T, 4>, max_ctas_per_sm<T, 4>(fs.smem)); break;
+      case 8: go(flash_decode_kernel<T, 8>, max_ctas_per_sm<T, 8>(fs.smem)); break;
+      default: go(flash_decode_kernel<T, 16>, max_ctas_per_sm<T, 16>(fs.smem)); break;
+    }
+  } else {
+    using T = float;
+    switch (GP) {
+      case 1: go(flash_decode_kernel<T, 1>, max_ctas_per_sm<T, 1>(fs.smem)); break;
+      case 2: go(flash_decode_kernel<T, 2>, max_ctas_per_sm<T, 2>(fs.smem)); break;
+      case 4: go(flash_decode_kernel<T, 4>, max_ctas_per_sm<T, 4>(fs.smem)); break;
+      case 8: go(flash_decode_kernel<T, 8>, max_ctas_per_sm<T, 8>(fs.smem)); break;
+      default: go(flash_decode_kernel<T, 16>, max_ctas_per_sm<T, 16>(fs.smem)); break;
+    }
+  }
+  stage_end(kStDecodeCluster, s, 1);
+  if (e == cudaErrorNotSupported) return ANCHORKV_EUNSUPPORTED;
+  return e == cudaSuccess ? ANCHORKV_OK : ANCHORKV_ECUDA;
+}
+
+int flash_ctas_per_sm(const Plan& pl, const FlashShape& fs) {
+  const int GP = gp_of(pl.G);
+  if (pl.p.dtype == ANCHORKV_BF16) {
+    using T = __nv_bfloat16;
+    return GP == 1 ? max_ctas_per_sm<T, 1>(fs.smem) : GP == 2 ? max_ctas_per_sm<T, 2>(fs.smem)
+         : GP == 4 ? max_ctas_per_sm<T, 4>(fs.smem) : GP == 8 ? max_ctas_per_sm<T, 8>(fs.smem)
+         : max_ctas_per_sm<T, 16>(fs.smem);
+  }
+  using T = float;
+  return GP == 1 ? max_ctas_per_sm<T, 1>(fs.smem) : GP == 2 ? max_ctas_per_sm<T, 2>(fs.smem)
+       : GP == 4 ? max_ctas_per_sm<T, 4>(fs.smem) : GP == 8 ? max_ctas_per_sm<T, 8>(fs.smem)
+       : max_ctas_per_sm<T, 16>(fs.smem);
+}
+
+}  // namespace akv

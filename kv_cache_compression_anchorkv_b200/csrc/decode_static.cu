@@ -24,8 +24,10 @@ namespace akv {
 namespace {
 
 // Shared scratch of every anchorkv_decode_attn_noalloc call on a device.  It
-// keeps the previous call's contents; the decode kernels write every scratch
-// word before they read it, so nothing in it has to start at zero.
+// keeps the previous call's contents; the only words that must start at zero
+// (the slice decode's per-(sequence, head) tickets) are cleared on the call's
+// stream before its kernel runs, and every other word is written before it
+// is read.
 static __device__ __align__(256) char g_decode_scratch[ANCHORKV_DECODE_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
@@ -77,7 +79,8 @@ int anchorkv_decode_attn_noalloc(const anchorkv_params* p, const void* compresse
   if (tail_len > 4096) return ANCHORKV_EUNSUPPORTED;
   if (seq_stride_bytes < pl.L.total_bytes && batch > 1) return ANCHORKV_EINVAL;
   if (seq_stride_bytes % 16) return ANCHORKV_EINVAL;
-  if (((uintptr_t)compressed | (uintptr_t)q | (uintptr_t)out) & 15) return ANCHORKV_EINVAL;
+  if (((uintptr_t)compressed | (uintptr_t)q | (uintptr_t)out | (uintptr_t)K_tail | (uintptr_t)V_tail) & 15)
+    return ANCHORKV_EINVAL;
   DecodePlan dp;
   make_decode_plan(pl, batch, &dp);
   if (dp.ws_total > (int64_t)ANCHORKV_DECODE_NOALLOC_SCRATCH_BYTES) return ANCHORKV_ENOSPC;
@@ -88,10 +91,8 @@ int anchorkv_decode_attn_noalloc(const anchorkv_params* p, const void* compresse
   char* scratch = nullptr;
   st = scratch_on_current_device(&scratch);
   if (st) return st;
-  if (launch_decode(pl, dp, (const char*)compressed, seq_stride_bytes, q, K_tail, V_tail, tail_len, tail_cap, out,
-                    scratch, (cudaStream_t)stream) != cudaSuccess)
-    return ANCHORKV_ECUDA;
-  return ANCHORKV_OK;
+  return launch_decode(pl, dp, (const char*)compressed, seq_stride_bytes, q, K_tail, V_tail, tail_len, tail_cap, out,
+                       scratch, (cudaStream_t)stream);
 }
 
 }  // extern "C"

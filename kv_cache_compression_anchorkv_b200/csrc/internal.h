@@ -47,6 +47,7 @@ struct Plan {
   int64_t o_util, o_refine, o_sel_state, o_hist, o_tile_gt, o_tile_eq, o_tie_before, o_tile_cnt;
   int64_t o_qproxy;          // proxy observation queries [Hq][W][D] (key-as-query mode), else 0
   int64_t o_asg_keys;        // best two 64-bit keys per token-side between anchor groups (k > kAssignGroupMax)
+  int64_t o_asg_probe;       // [512][kAssignGroupMax] fp32 tensor-core accumulators of the probe rows
   // codebook and Hadamard signs (bit j set: s_j = -1)
   double tau, l1, l2;
   uint32_t sign_bits[4];
@@ -55,19 +56,33 @@ struct Plan {
 int make_plan(const anchorkv_params* p, Plan* out);
 void codebook(double* tau, double* l1, double* l2, double* mse);
 
+// Slice decode (decode_flash.cu): chunk size, slices per (sequence, head),
+// shared memory per CTA and its workspace (tickets, slice partials).
+struct FlashShape {
+  int ct, S, tps, smem;
+  bool klogit;            // key-residual logits from the tensor-core pre-pass
+  int64_t ws_total, o_tickets, o_part, o_rlog;
+};
+// Tensor-core pre-pass of the slice decode: sigma~ <qr, lev(c)> of every key
+// record, [batch][R][GP] floats in the workspace.
+bool klogit_tc_supported(const Plan& pl);
+int64_t klogit_ws_bytes(const Plan& pl, int batch);
+int launch_klogit_tc(const Plan& pl, int batch, const char* comp, int64_t stride, const void* q, float* out,
+                     cudaStream_t s);
 struct DecodePlan {
-  bool cluster;           // one cluster per (sequence, head), no workspace
+  bool flash;             // slice decode; otherwise the split-token kernels
+  FlashShape fs;
   int batch, n_split, split_tokens;
   int64_t ws_total, o_P, o_qrot, o_part_m, o_part_l, o_part_w, o_part_z;
 };
 int make_decode_plan(const Plan& pl, int batch, DecodePlan* out);
 // Shape checks of a decode call (shared-memory limits of the chosen path).
 int check_decode_shape(const Plan& pl, const DecodePlan& dp, int tail_len);
-bool decode_cluster_supported(const Plan& pl);
-int decode_cluster_size(const Plan& pl, int batch, int* C, int* smem);
-int launch_decode_cluster(const Plan& pl, int batch, const char* comp, int64_t stride, const void* q,
-                          const void* Kt, const void* Vt, int tail_len, int tail_cap, float* out, cudaStream_t s,
-                          cudaError_t* err);
+bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs);
+int launch_flash_decode(const Plan& pl, const FlashShape& fs, int batch, const char* comp, int64_t stride,
+                        const void* q, const void* Kt, const void* Vt, int tail_len, int tail_cap, float* out,
+                        char* ws, cudaStream_t s);
+int flash_ctas_per_sm(const Plan& pl, const FlashShape& fs);
 
 // Kernel launchers (one per hot-path step), all asynchronous on `s`.
 cudaError_t launch_obs_pass1(const Plan& pl, const void* K, const void* V, const void* Q, char* ws, cudaStream_t s);
@@ -97,9 +112,10 @@ cudaError_t launch_decode_rope(const Plan& pl, const RopePlan& rp, const char* c
 // mode bits of the plan's parameters
 inline int rank_of(const Plan& pl) { return (pl.p.mode & ANCHORKV_MODE_RANK_MASK) >> ANCHORKV_MODE_RANK_SHIFT; }
 inline int naive_codec(const Plan& pl) { return (pl.p.mode & ANCHORKV_MODE_NAIVE_CODEC) ? 1 : 0; }
-cudaError_t launch_decode(const Plan& pl, const DecodePlan& dp, const char* comp, int64_t stride,
-                          const void* q, const void* Kt, const void* Vt, int tail_len, int tail_cap,
-                          float* out, char* ws, cudaStream_t s);
+// Returns an ANCHORKV_* status.
+int launch_decode(const Plan& pl, const DecodePlan& dp, const char* comp, int64_t stride,
+                  const void* q, const void* Kt, const void* Vt, int tail_len, int tail_cap,
+                  float* out, char* ws, cudaStream_t s);
 cudaError_t launch_reconstruct(const Plan& pl, const char* comp, float* Kh, float* Vh, cudaStream_t s);
 
 }  // namespace akv

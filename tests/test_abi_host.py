@@ -21,6 +21,7 @@ def test_library_exports_every_declared_symbol():
 def test_struct_sizes_match_header_layout():
     assert ctypes.sizeof(capi.Params) == 4 * 6 + 8 + 8 + 4 * 6
     assert ctypes.sizeof(capi.Layout) == 8 * 7 + 4 * 4 + 8 * 8
+    assert ctypes.sizeof(capi.WorkspaceView) == 8 * 5
 
 
 CASES = [
@@ -90,11 +91,30 @@ def test_workspace_view():
     v = api.compress_workspace(p)
     assert v["total_bytes"] > v["off_utility"] + 4 * 2 * 8 * 32768
     assert v["off_counters"] % 256 == 0 and v["off_pooled"] % 256 == 0
-    # up to 8 query heads per KV head the decode runs in one cluster per
-    # (sequence, head) and needs no workspace; above that it splits tokens
-    assert api.decode_workspace_bytes(p, 1) == api.decode_workspace_bytes(p, 16) == 0
-    p16 = api.AnchorKVParams(n_tokens=32768, n_q_heads=128)
+    # the slice decode needs tickets and slice partials only when a (sequence,
+    # head) is cut into several slices: at batch 1 (8 heads on ~148 CTAs) it
+    # is, at batch 32 (256 heads) every head is one slice and needs nothing
+    assert api.decode_workspace_bytes(p, 1) > 0
+    assert api.decode_workspace_bytes(p, 32) == 0
+    # 16 query heads per KV head with 1056 anchors do not fit the slice
+    # decode's shared memory: the split-token kernels and their workspace
+    p16 = api.AnchorKVParams(n_tokens=131072, n_q_heads=128)
     assert api.decode_workspace_bytes(p16, 16) > api.decode_workspace_bytes(p16, 1) > 0
+
+
+def test_misaligned_tails_rejected_before_any_launch():
+    """K_tail / V_tail are read with 16-byte vector loads: a tail pointer off
+    a 16-byte boundary is EINVAL on the host, for the workspace and the
+    no-alloc entry points alike (placeholder pointers, never dereferenced)."""
+    L = capi.lib()
+    p = api.AnchorKVParams(n_tokens=1024).c()
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 21) + 2)
+    for kt, vt in ((odd, fake), (fake, odd)):
+        assert L.anchorkv_decode_attn(ctypes.byref(p), fake, 1 << 20, 1, fake, kt, vt, 4, 8, fake, fake,
+                                      1 << 30, None) == capi.EINVAL
+        assert L.anchorkv_decode_attn_noalloc(ctypes.byref(p), fake, 1 << 20, 1, fake, kt, vt, 4, 8, fake,
+                                              None) == capi.EINVAL
 
 
 def test_recorded_traffic_follows_the_kernel_source(tmp_path, monkeypatch):

@@ -51,6 +51,7 @@ def test_compress_parity(name):
     gb, gpool, gutil, counters = parity.gpu_compress(p, K, V, Q)
     assert counters[0] == 0
     rep = parity.check_compress(p, _f64(K), _f64(V), _f64(Q), gb, gpool, gutil)
+    parity.log_report(name, rep, refined_rows=counters[1])
     print(name, rep, "refined rows:", counters[1])
 
 
@@ -67,6 +68,7 @@ def test_compress_exact_ties():
     rep = parity.check_compress(p, _f64(K), _f64(V), _f64(Q), gb, gpool, gutil)
     g = O.unpack_layout(gb, parity.oracle_params(p))
     assert np.all(g["idx"][0, 0, 300:310] == 0) or 300 in g["anchor_pos"][0]
+    parity.log_report("exact-ties-n600", rep, refined_rows=counters[1])
     print(rep)
 
 
@@ -123,12 +125,47 @@ def test_decode_parity(name, batch, tail):
     print(name, batch, tail, "max abs err", err)
 
 
+@pytest.mark.parametrize("name,batch,tail,mode", [("tiny-fp32-n1024", 2, 5, 0), ("bf16-ragged-n3000", 3, 17, 0),
+                                                  ("bf16-gqa8-n2500", 2, 0, 0), ("bf16-every-residual", 1, 3, 0),
+                                                  ("fp32-window8-n700", 2, 9, 0), ("bf16-n20000", 2, 1500, 0),
+                                                  ("bf16-ragged-n3000", 2, 4, 0x10)])
+def test_decode_tensor_core_key_logits(name, batch, tail, mode, monkeypatch):
+    """The key-residual logits computed ahead of the decode on the tensor
+    cores (bit planes of the codes times a fixed-point query, kind::i8)
+    give the same decode as the oracle."""
+    monkeypatch.setenv("ANCHORKV_DECODE_KLOGIT", "1")
+    spec, theta = CASES[name]
+    p = _params(spec, theta)
+    p.mode = mode
+    L = api.anchorkv_bytes(p)
+    stride = (L["total_bytes"] + 255) // 256 * 256
+    comp = torch.zeros(batch, stride, dtype=torch.uint8, device="cuda")
+    layouts = []
+    for b in range(batch):
+        sb = CacheSpec(**{**spec.__dict__, "seed": spec.seed + 100 * b})
+        K, V, Q = make_layer(sb, 0)
+        out, _ = api.compress(p, K.cuda(), V.cuda(), Q.cuda())
+        comp[b, :L["total_bytes"]] = out
+        layouts.append(out.cpu().numpy())
+    q = make_decode_queries(spec, 0, step=3, batch=batch)
+    cap = max(tail, 1) + 3
+    Kt, Vt = make_tail(spec, 0, cap, batch=batch)
+    o = api.decode_attn(p, comp, q.cuda(), Kt.cuda(), Vt.cuda(), tail_len=tail)
+    err = parity.check_decode(p, layouts, _f64(q), _f64(Kt), _f64(Vt), tail, o.cpu().double().numpy(),
+                              DECODE_TOL[spec.dtype])
+    print(name, "tensor-core key logits", batch, tail, "max abs err", err)
+
+
 def test_decode_config():
     spec, theta = CASES["bf16-n20000"]
     cfg = api.decode_config(_params(spec, theta), 1)
-    assert cfg["cluster_ctas"] in (1, 2, 4, 8, 16) and 0 < cfg["smem_bytes"] <= 227 * 1024
-    spec, theta = CASES["bf16-gqa16-n1500"]
-    assert api.decode_config(_params(spec, theta), 2)["cluster_ctas"] == 0
+    n_tiles = (spec.n_tokens + 127) // 128
+    assert 1 < cfg["slices"] <= n_tiles and 0 < cfg["smem_bytes"] <= 227 * 1024
+    # a batch with more (sequence, head) pairs than SMs: one slice each
+    assert api.decode_config(_params(spec, theta), 200)["slices"] == 1
+    # 16 query heads per KV head and 1056 anchors: the split-token kernels
+    p = api.AnchorKVParams(n_tokens=131072, n_kv_heads=8, n_q_heads=128)
+    assert api.decode_config(p, 1)["slices"] == 0
 
 
 def test_error_paths_on_device():
@@ -164,11 +201,50 @@ def test_full_size_layer_llama8b_shape():
     p = _params(spec, 0.05, layer=layer)
     gb, gpool, gutil, counters = parity.gpu_compress(p, K, V, Q)
     rep = parity.check_compress(p, _f64(K), _f64(V), _f64(Q), gb, gpool, gutil, full_chain=False)
+    parity.log_report("llama8b-layer5-n32768", rep, refined_rows=counters[1])
     print("full-size layer", rep, "refined rows:", counters[1])
+    # decisions the fp32 paths cannot certify are re-taken in fp64, so near-ties
+    # can only come from the fp32 observation scores and utilities at the
+    # selection boundaries: a handful at most on half a million token-sides
+    assert rep["near_ties"] <= 8, rep
     q = make_decode_queries(spec, layer, step=0, batch=1, device="cuda")
     comp = torch.from_numpy(gb).cuda()
     o = api.decode_attn(p, comp, q)
     parity.check_decode(p, [gb], _f64(q), None, None, 0, o.cpu().double().numpy(), DECODE_TOL["bf16"])
+
+
+@pytest.mark.slow
+def test_tensor_core_accumulation_error_on_8b_layer(monkeypatch):
+    """The nearest-anchor decision is certified from fp32 scores: a row whose
+    best two differ by more than 2^-13 ||x|| is not re-taken in fp64.  That
+    margin assumes the tensor core's fp32 accumulation of the 128 exact bf16
+    products of <x, a> errs by at most 2^-16 ||x|| ||a||.  Measured here on
+    every (token, slot) pair of tokens 0..511 of the key side of head 0 of an
+    8B-shaped layer (512 x 288 raw accumulators exported by the kernel)
+    against the exact dot products."""
+    monkeypatch.setenv("ANCHORKV_ASSIGN_PROBE", "1")
+    spec = CacheSpec(32, 8, 32, 32768, n_dirs=128, seed=0)
+    K, V, Q = make_layer(spec, 5, device="cuda")
+    p = _params(spec, 0.05, layer=5)
+    out, ws = api.compress(p, K, V, Q)
+    assert api.read_status(ws)[0] == 0
+    L = api.anchorkv_bytes(p)
+    k = L["n_anchors"]
+    assert k == 288            # one anchor group, chunked 2 x 144 (or 3 x 96): 288 columns
+    view = api.compress_workspace(p)
+    raw = ws[view["off_assign_probe"]:view["off_assign_probe"] + 4 * 512 * k].cpu().numpy()
+    acc = raw.view(np.float32).reshape(512, k).astype(np.float64)
+    ap = O.unpack_layout(out.cpu().numpy(), parity.oracle_params(p))["anchor_pos"][0]
+    X = _f64(K[0, :512])
+    A = _f64(K[0])[ap]
+    exact = X @ A.T                      # products of bf16 values are exact in fp64
+    scale = np.linalg.norm(X, axis=1)[:, None] * np.linalg.norm(A, axis=1)[None, :]
+    rel = np.abs(acc - exact) / np.where(scale > 0, scale, 1.0)
+    print("tensor-core accumulation: max |acc - <x,a>| / (||x|| ||a||) =", rel.max(),
+          "= 2^%.1f" % np.log2(max(rel.max(), 1e-300)))
+    parity.log_report("tc-accumulation-8b-layer5", {"max_rel_acc_err": float(rel.max()),
+                                                     "pairs": int(rel.size)})
+    assert rel.max() <= 2.0 ** -16
 
 
 @pytest.mark.parametrize("name", ["bf16-ragged-n3000", "bf16-gqa8-n2500", "bf16-every-residual"])
@@ -197,6 +273,7 @@ def test_simt_observation_path_parity(name, monkeypatch):
     gb, gpool, gutil, counters = parity.gpu_compress(p, K, V, Q)
     assert counters[0] == 0
     rep = parity.check_compress(p, _f64(K), _f64(V), _f64(Q), gb, gpool, gutil)
+    parity.log_report(name + " (SIMT observation passes)", rep, refined_rows=counters[1])
     print(name, "simt observation passes", rep)
 
 
@@ -224,6 +301,7 @@ def test_compress_modes(name, mode):
     gb, gpool, gutil, counters = parity.gpu_compress(p, K, V, Q)
     assert counters[0] == 0
     rep = parity.check_compress(p, _f64(K), _f64(V), _f64(Q), gb, gpool, gutil)
+    parity.log_report(f"{name} mode {mode:#x}", rep, refined_rows=counters[1])
     print(name, hex(mode), rep)
 
 
@@ -279,6 +357,7 @@ def test_compress_anchor_groups(N, anchor_div, theta):
     gb, gpool, gutil, counters = parity.gpu_compress(p, K, V, Q)
     assert counters[0] == 0
     rep = parity.check_compress(p, _f64(K), _f64(V), _f64(Q), gb, gpool, gutil)
+    parity.log_report(f"anchor-groups-n{N}-k{api.anchorkv_bytes(p)['n_anchors']}", rep, refined_rows=counters[1])
     print("anchor groups", N, anchor_div, rep, "refined rows:", counters[1])
 
 
@@ -320,7 +399,7 @@ def test_decode_rope_parity(name, batch, tail, base, mode):
 def test_batched_decode_8b_shape_sampled():
     """Batched decode as benchmarked for many sequences: 16 compressed
     sequences of the 8B shape (8 KV / 32 query heads, N = 32768, theta = 0.1)
-    decoded in one launch; sequences 0 and 15 checked against the oracle."""
+    decoded in one launch; every sequence checked against the oracle."""
     spec = CacheSpec(32, 8, 32, 32768, n_dirs=128, seed=0)
     p = _params(spec, 0.1, layer=0)
     L = api.anchorkv_bytes(p)
@@ -336,7 +415,8 @@ def test_batched_decode_8b_shape_sampled():
     q = make_decode_queries(spec, 0, step=0, batch=batch, device="cuda")
     o = api.decode_attn(p, comp, q)
     po = parity.oracle_params(p)
-    for b in (0, batch - 1):
+    assert torch.isfinite(o).all()
+    for b in range(batch):
         parts = O.unpack_layout(comp[b, :L["total_bytes"]].cpu().numpy(), po)
         Kh, Vh = O.reconstruct(parts, po)
         want = O.decode_attention(_f64(q[b]), Kh, Vh)
@@ -346,57 +426,55 @@ def test_batched_decode_8b_shape_sampled():
 
 
 @pytest.mark.slow
-def test_70b_shape_layer_sampled():
+def test_70b_shape_layer_stage_by_stage():
     """One layer of the 70B-shaped cache (8 KV / 64 query heads, N = 131072,
-    theta = 0.05; k = 1056 anchors, three assignment groups): byte accounting,
-    window anchors, a sample of nearest-anchor slots and coefficients against
-    fp64 (mismatches only as counted near-ties), and the decode after 128
-    appended tokens against the oracle."""
+    theta = 0.05; k = 1056 anchors in three assignment groups), every stage
+    against the oracle on every head and side: pooled scores, anchor sets,
+    nearest-anchor slots, coefficients, utilities, the top-R selection, the
+    residual codes and scales (mismatches only as counted near-ties); then the
+    decode of all 64 query heads after 128 appended exact tokens."""
     spec = CacheSpec(80, 8, 64, 131072, n_dirs=256, seed=0)
     p = _params(spec, 0.05, layer=7)
     K, V, Q = make_layer(spec, 7, device="cuda")
-    out, ws = api.compress(p, K, V, Q)
-    st = api.read_status(ws)
-    assert st[0] == 0
     L = api.anchorkv_bytes(p)
     po = parity.oracle_params(p)
     Lo = O.layout(po)
     assert L["total_bytes"] == Lo["total"] and L["n_residuals"] == Lo["R"] and L["n_anchors"] == Lo["k"] == 1056
-    g = O.unpack_layout(out.cpu().numpy(), po)
-    N, W = spec.n_tokens, spec.window
-    rng = np.random.default_rng(3)
-    near = 0
-    for h in (0, 5):
-        ap = g["anchor_pos"][h]
-        assert np.all(np.isin(np.arange(N - W, N), ap)) and np.all(np.diff(ap) > 0)
-        for side, X in enumerate((K[h], V[h])):
-            Xh = _f64(X)
-            A = Xh[ap]
-            an = np.linalg.norm(A, axis=1)
-            for t in rng.choice(N, 400, replace=False):
-                cos = np.where(an > 0, A @ Xh[t] / np.where(an > 0, an, 1.0), 0.0)
-                s_o = int(np.argmax(cos)) if t not in set(ap.tolist()) else int(np.searchsorted(ap, t))
-                s_g = int(g["idx"][side, h, t])
-                if s_o != s_g:
-                    assert cos[s_o] - cos[s_g] <= 1e-12 * np.linalg.norm(Xh[t]), (h, side, t)
-                    near += 1
-                    continue
-                xa = A[s_g]
-                n2 = float(xa @ xa)
-                gam = 1.0 if t in set(ap.tolist()) else (float(Xh[t] @ xa) / n2 if n2 > 0 else 0.0)
-                assert np.float16(gam).view(np.uint16) == g["g16"][side, h, t].view(np.uint16) or \
-                    abs(gam - float(g["g16"][side, h, t])) <= 2 ** -11 * abs(gam) + 1e-300, (h, side, t)
+    gb, gpool, gutil, counters = parity.gpu_compress(p, K, V, Q)
+    assert counters[0] == 0
+    rep = parity.check_compress(p, _f64(K), _f64(V), _f64(Q), gb, gpool, gutil, full_chain=False)
+    parity.log_report("llama70b-layer7-n131072", rep, refined_rows=counters[1])
+    print("70B-shaped layer", rep, "refined rows:", counters[1])
+    assert rep["near_ties"] <= 16, rep
+    out = torch.from_numpy(gb).cuda()
     q = make_decode_queries(spec, 7, step=128, batch=1, device="cuda")
     Kt, Vt = make_tail(spec, 7, 128, batch=1, device="cuda")
     o = api.decode_attn(p, out, q, Kt, Vt, tail_len=128)
-    Kh, Vh = O.reconstruct(g, po)
-    for j in (0, 63):
-        h = j // 8
-        Kf = np.concatenate([Kh[h], _f64(Kt[0, h])])
-        Vf = np.concatenate([Vh[h], _f64(Vt[0, h])])
-        s = Kf @ _f64(q[0, j]) / np.sqrt(128)
-        w = np.exp(s - s.max())
-        want = (w / w.sum()) @ Vf
-        err = float(np.abs(o[0, j].cpu().double().numpy() - want).max())
-        assert err <= DECODE_TOL["bf16"], (j, err)
-    print("70B-shaped layer: refined rows", st[1], "sampled near-ties", near)
+    parity.check_decode(p, [gb], _f64(q), _f64(Kt), _f64(Vt), 128, o.cpu().double().numpy(), DECODE_TOL["bf16"])
+
+
+@pytest.mark.slow
+def test_multi_stream_compress_matches_single_stream():
+    """The benchmark compresses independent layers on four streams, each with
+    its own workspace: the layouts must equal the single-stream ones byte for
+    byte (8B-shaped layers, N = 32768, theta = 0.05)."""
+    spec = CacheSpec(4, 8, 32, 32768, n_dirs=128, seed=0)
+    layers = [make_layer(spec, l, device="cuda") for l in range(spec.n_layers)]
+    params = [_params(spec, 0.05, layer=l) for l in range(spec.n_layers)]
+    single = []
+    ws = None
+    for l, (K, V, Q) in enumerate(layers):
+        out, ws = api.compress(params[l], K, V, Q, workspace=ws)
+        single.append(out.clone())
+    streams = [torch.cuda.Stream() for _ in range(4)]
+    wss = [torch.empty_like(ws) for _ in range(4)]
+    multi = [torch.empty_like(x) for x in single]
+    torch.cuda.synchronize()
+    for l, (K, V, Q) in enumerate(layers):
+        with torch.cuda.stream(streams[l % 4]):
+            api.compress(params[l], K, V, Q, out=multi[l], workspace=wss[l % 4])
+    torch.cuda.synchronize()
+    for w in wss:
+        assert api.read_status(w)[0] == 0
+    for l in range(spec.n_layers):
+        assert torch.equal(single[l], multi[l]), l

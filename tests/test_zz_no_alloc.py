@@ -1,9 +1,11 @@
 """anchorkv_decode_attn_noalloc (library-owned scratch, no workspace argument)
 against anchorkv_decode_attn (caller workspace), both through the C ABI.
 
-Collected last on purpose: it must pass in a fresh process, where its first
-call performs the per-device scratch look-up, and after every other test,
-where the shared scratch holds whatever earlier calls left in it.
+The file is collected last, so that a run stopping at the first failure has
+already run every other test, and so that in a full run its calls find the
+shared scratch holding whatever earlier decode calls left in it.  Run on its
+own (pytest tests/test_zz_no_alloc.py), its first call is the one that looks
+up the scratch array's device address.
 """
 import ctypes
 
@@ -88,15 +90,26 @@ def test_noalloc_matches_workspace_entry_point(name):
 
 def test_noalloc_rejects_sizes_beyond_the_scratch():
     """A decode workspace above the static maximum is refused with ENOSPC
-    before any device work.  Host logic: run only where no GPU is present, so
-    the placeholder pointers below can never reach a kernel."""
-    if torch.cuda.is_available():
-        pytest.skip("host-only check")
+    before any device work.  With a GPU the arguments are real device buffers
+    of the right sizes (a zeroed layout batch, queries, output), so nothing
+    could read out of bounds even if a launch happened; without one they are
+    aligned placeholders that the size check turns away first."""
     p = api.AnchorKVParams(n_tokens=131072, n_kv_heads=8, n_q_heads=128)
     batch = 4
     assert api.decode_workspace_bytes(p, batch) > api.NOALLOC_SCRATCH_BYTES
     stride = (api.anchorkv_bytes(p)["total_bytes"] + 255) // 256 * 256
-    fake = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced: the size check comes first
-    st = capi.lib().anchorkv_decode_attn_noalloc(ctypes.byref(p.c()), fake, stride, batch, fake, None, None, 0,
-                                                 0, fake, None)
+    if torch.cuda.is_available():
+        comp = torch.zeros(batch, stride, dtype=torch.uint8, device="cuda")
+        q = torch.zeros(batch, p.n_q_heads, p.head_dim, dtype=torch.bfloat16, device="cuda")
+        out = torch.zeros(batch, p.n_q_heads, p.head_dim, dtype=torch.float32, device="cuda")
+        ptrs = (_vp(comp), _vp(q), _vp(out))
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    else:
+        fake = ctypes.c_void_p(1 << 20)
+        ptrs, stream = (fake, fake, fake), None
+    st = capi.lib().anchorkv_decode_attn_noalloc(ctypes.byref(p.c()), ptrs[0], stride, batch, ptrs[1], None, None,
+                                                 0, 0, ptrs[2], stream)
     assert st == capi.ENOSPC
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+        assert torch.count_nonzero(out).item() == 0     # nothing ran
