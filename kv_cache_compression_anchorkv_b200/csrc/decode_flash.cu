@@ -81,7 +81,7 @@ struct FArgs {
 
 // Shared-memory carve-up (bytes), the same on host and device.
 struct FPlan {
-  int qs, qr, P, W, Wi, lut, pfs, wpre, red, rlog, wz, stage, stage_bytes, total;
+  int qs, qr, P, W, Wi, Wf, lut, pfs, wpre, red, rlog, wz, stage, stage_bytes, total;
   // offsets inside one stage
   int s_codes, s_sig, s_tok, s_bm;
 };
@@ -91,15 +91,18 @@ __host__ __device__ inline int fa_align(int x, int a) { return (x + a - 1) / a *
 __host__ __device__ inline FPlan fplan(int GP, int kp, int ct, int tps) {
   FPlan f;
   int cur = 0;
+  // persistent small arrays first; from P on, the region is reused at the
+  // end for the cross-warp sums ([2][warps][GP][128] floats)
   f.qs = cur; cur += GP * kD * 4;
   f.qr = cur; cur += GP * kD * 4;
-  f.P = cur; cur += GP * kp * 4;
-  f.W = cur; cur += GP * kp * 4;
-  f.Wi = cur; cur += 2 * GP * kp * 4;
   f.lut = cur; cur += 16 * 16 * 8;
   f.pfs = cur; cur = fa_align(cur + 2 * (tps + 1) * 4, 16);
   f.wpre = cur; cur = fa_align(cur + 2 * (ct / 32 + 1) * 4, 16);
   f.red = cur; cur = fa_align(cur + 2 * kWarps * GP * 4, 16);
+  f.P = cur; cur += GP * kp * 4;
+  f.W = cur; cur += GP * kp * 4;
+  f.Wi = cur; cur += 2 * GP * kp * 4;
+  f.Wf = cur; cur += kp * 4;
   f.rlog = cur; cur = fa_align(cur + ct * GP * 4, 16);
   f.wz = cur; cur = fa_align(cur + ct * GP * 4, 16);
   // stage: codes [2][ct][32], scales [2][ct + 8] (16-byte spans), token words
@@ -110,9 +113,9 @@ __host__ __device__ inline FPlan fplan(int GP, int kp, int ct, int tps) {
   f.s_tok = sc; sc += 2 * (ct + 4) * 4;
   f.s_bm = sc; sc += 2 * (ct / 32) * 4;
   f.stage_bytes = fa_align(sc, 16);
-  // the two stages also hold the cross-warp sums at the end ([2][warps][GP][128])
   f.stage = fa_align(cur, 16);
-  cur = f.stage + (2 * f.stage_bytes > 2 * kWarps * GP * kD * 4 ? 2 * f.stage_bytes : 2 * kWarps * GP * kD * 4);
+  cur = f.stage + 2 * f.stage_bytes;
+  if (cur < f.P + 2 * kWarps * GP * kD * 4) cur = f.P + 2 * kWarps * GP * kD * 4;
   f.total = fa_align(cur, 16);
   return f;
 }
@@ -196,6 +199,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
   float* P = reinterpret_cast<float*>(sm + F.P);         // [GP][kp]
   float* Wt = reinterpret_cast<float*>(sm + F.W);        // [GP][kp]
   int* Wi = reinterpret_cast<int*>(sm + F.Wi);           // [2][GP][kp] this chunk's W in fixed point (hi, lo)
+  int* Wf = reinterpret_cast<int*>(sm + F.Wf);           // [kp] slots the chunk touched
   float2* lut = reinterpret_cast<float2*>(sm + F.lut);   // [16 nibbles][16 copies]
   int* pfs = reinterpret_cast<int*>(sm + F.pfs);         // [2][tps + 1]
   int* wpre = reinterpret_cast<int*>(sm + F.wpre);       // [2][ct/32 + 1]
@@ -332,6 +336,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
     Wi[i] = 0;
     Wi[GP * kp + i] = 0;
   }
+  for (int i = tid; i < kp; i += kThreads) Wf[i] = 0;
 
   // running state (identical in every thread): max per head; per-thread sums
   float mrun[GP], lsum[GP];
@@ -528,7 +533,9 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
     float cm[GP], gmax, fsc[GP];
     block_max2(cmx, gabs, cm, gmax);
     update_max(cm, fsc);
-    // wsc = 2^e, winv = 2^-e, e = 30 - ceil(log2 ntok) - ceil(log2 bound)
+    // wsc = 2^e, winv = 2^-e, e = 30 - ceil(log2 ntok) - ceil(log2 bound):
+    // the chunk's sum of |terms| stays below 2^30 (the integer parts) and the
+    // remainders, scaled by 2^20, below 2^29
     float wsc[GP], winv[GP];
     const int en = 32 - __clz(ntok);
 #pragma unroll
@@ -580,28 +587,26 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
           atomicAdd(&Wi[GP * kp + g * kp + slot], __float2int_rn((x - xh) * 1048576.0f));
           if (res) wz[rank * GP + g] = p * sg;
         }
+        Wf[slot] = 1;        // a plain store: any writer leaves 1
       }
     }
     __syncthreads();
-    // e. the chunk's fixed-point anchor weights into W (and cleared); value-residual sums
-    {
-      int4* hi4 = reinterpret_cast<int4*>(Wi);
-      int4* lo4 = reinterpret_cast<int4*>(Wi + GP * kp);
-      float4* w4 = reinterpret_cast<float4*>(Wt);
-      const int per = kp >> 2;          // kp is a multiple of 4
+    // e. the chunk's fixed-point anchor weights into W, per token: the first
+    //    thread to take a touched slot's flag (atomic exchange with 0) folds
+    //    that slot for every head and is its only writer; value-residual sums
 #pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        const float ih = winv[g], il = winv[g] * (1.0f / 1048576.0f);
-        for (int i = tid; i < per; i += kThreads) {
-          const int4 vh = hi4[g * per + i], vl = lo4[g * per + i];
-          float4 w = w4[g * per + i];
-          w.x += fmaf((float)vl.x, il, (float)vh.x * ih);
-          w.y += fmaf((float)vl.y, il, (float)vh.y * ih);
-          w.z += fmaf((float)vl.z, il, (float)vh.z * ih);
-          w.w += fmaf((float)vl.w, il, (float)vh.w * ih);
-          w4[g * per + i] = w;
-          hi4[g * per + i] = make_int4(0, 0, 0, 0);
-          lo4[g * per + i] = make_int4(0, 0, 0, 0);
+    for (int i = 0; i < kKT; ++i) {
+      const int t = tid + i * kThreads;
+      if (t < ntok) {
+        const int slot = slv[i];
+        if (atomicExch(&Wf[slot], 0)) {
+#pragma unroll
+          for (int g = 0; g < GP; ++g) {
+            const int vh = Wi[g * kp + slot], vl = Wi[GP * kp + g * kp + slot];
+            Wt[g * kp + slot] += fmaf((float)vl, winv[g] * (1.0f / 1048576.0f), (float)vh * winv[g]);
+            Wi[g * kp + slot] = 0;
+            Wi[GP * kp + g * kp + slot] = 0;
+          }
         }
       }
     }
@@ -724,7 +729,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
     }
   }
   // cross-warp sums of the anchor/tail values and of Z, through the stage buffers
-  float* ored = reinterpret_cast<float*>(sm + F.stage);          // [kWarps][GP][128]
+  float* ored = reinterpret_cast<float*>(sm + F.P);              // [kWarps][GP][128]
   float* zred = ored + kWarps * GP * kD;                           // [kWarps][GP][128]
   __syncthreads();    // every chunk is consumed and no copy is in flight
 #pragma unroll
@@ -813,12 +818,33 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
     for (int j = 0; j < a.S; ++j) ms[j * GP + tid] /= lt;
   }
   __syncthreads();
-  for (int i = tid; i < G * kD; i += kThreads) {
-    const int g = i / kD;
-    float o = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < a.S; ++j) o = fmaf(__ldcg(all + (int64_t)j * PW + 2 * GP + i), ms[j * GP + g], o);
-    out[i] = o;
+  // warp w sums the partials j = w (mod warps) over every (head, coordinate),
+  // all of a partial's loads in flight at once; the warps' sums meet in
+  // shared memory (the region from P on is free by now)
+  {
+    constexpr int EPL = GP * kD / 32;
+    float acc[EPL];
+#pragma unroll
+    for (int m = 0; m < EPL; ++m) acc[m] = 0.f;
+    for (int j = warp; j < a.S; j += kWarps) {
+      const float* pj = all + (int64_t)j * PW + 2 * GP;
+#pragma unroll
+      for (int m = 0; m < EPL; ++m) {
+        const int e = lane + 32 * m;
+        acc[m] = fmaf(__ldcg(pj + e), ms[j * GP + e / kD], acc[m]);
+      }
+    }
+    float* mred = reinterpret_cast<float*>(sm + F.P);
+    __syncthreads();           // every warp is done with the weights mred may cover
+#pragma unroll
+    for (int m = 0; m < EPL; ++m) mred[warp * GP * kD + lane + 32 * m] = acc[m];
+    __syncthreads();
+    for (int i = tid; i < G * kD; i += kThreads) {
+      float o = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) o += mred[w * GP * kD + i];
+      out[i] = o;
+    }
   }
 }
 
