@@ -891,8 +891,9 @@ def run_gpu(args, world, rank, local):
     roof["kernel"] = dom
     roof["peak_source"] = ("measured" if peaks["source"] == "measured" else "fallback") + (
         " (burst bf16)" if roof["unit"] == "TFLOP/s" else " (copy)")
-    stage_roofs = {st: {kk: (round(v, 4) if isinstance(v, float) else v)
-                        for kk, v in stage_roofline(st, units, per_launch[st], peaks).items()}
+    stage_roofs = {st: {**{kk: (round(v, 4) if isinstance(v, float) else v)
+                           for kk, v in stage_roofline(st, units, per_launch[st], peaks).items()},
+                        "traffic": recorded_traffic(st)}
                    for st in per_launch}
 
     dec_bytes = Lr * L["total_bytes"]

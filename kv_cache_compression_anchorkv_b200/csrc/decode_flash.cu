@@ -81,7 +81,7 @@ struct FArgs {
 
 // Shared-memory carve-up (bytes), the same on host and device.
 struct FPlan {
-  int qs, qr, P, W, Wi, Wf, lut, pfs, wpre, red, rlog, wz, stage, stage_bytes, total;
+  int qs, qr, P, W, lut, pfs, wpre, red, rlog, wz, stage, stage_bytes, total;
   // offsets inside one stage
   int s_codes, s_sig, s_tok, s_bm;
 };
@@ -100,9 +100,7 @@ __host__ __device__ inline FPlan fplan(int GP, int kp, int ct, int tps) {
   f.wpre = cur; cur = fa_align(cur + 2 * (ct / 32 + 1) * 4, 16);
   f.red = cur; cur = fa_align(cur + 2 * kWarps * GP * 4, 16);
   f.P = cur; cur += GP * kp * 4;
-  f.W = cur; cur += GP * kp * 4;
-  f.Wi = cur; cur += 2 * GP * kp * 4;
-  f.Wf = cur; cur += kp * 4;
+  f.W = cur; cur += GP * kp * 8;
   f.rlog = cur; cur = fa_align(cur + ct * GP * 4, 16);
   f.wz = cur; cur = fa_align(cur + ct * GP * 4, 16);
   // stage: codes [2][ct][32], scales [2][ct + 8] (16-byte spans), token words
@@ -152,6 +150,24 @@ __device__ __forceinline__ void copy_span(uint8_t* dst, const uint8_t* comp, int
   }
 }
 
+// GP consecutive floats of shared memory (16-byte aligned for GP >= 4) in as
+// few vector loads as they allow.
+template <int GP>
+__device__ __forceinline__ void load_row(const float* src, float (&v)[GP]) {
+  if constexpr (GP >= 4) {
+#pragma unroll
+    for (int j = 0; j < GP / 4; ++j) {
+      const float4 t = reinterpret_cast<const float4*>(src)[j];
+      v[4 * j] = t.x; v[4 * j + 1] = t.y; v[4 * j + 2] = t.z; v[4 * j + 3] = t.w;
+    }
+  } else if constexpr (GP == 2) {
+    const float2 t = *reinterpret_cast<const float2*>(src);
+    v[0] = t.x; v[1] = t.y;
+  } else {
+    v[0] = src[0];
+  }
+}
+
 // Brings the 128-byte line at p into L2 (no register result, no wait).
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
@@ -197,9 +213,9 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
   float* qs = reinterpret_cast<float*>(sm + F.qs);       // [GP][128] q' (log2 units)
   float* qr = reinterpret_cast<float*>(sm + F.qr);       // [GP][128] rotated q'
   float* P = reinterpret_cast<float*>(sm + F.P);         // [GP][kp]
-  float* Wt = reinterpret_cast<float*>(sm + F.W);        // [GP][kp]
-  int* Wi = reinterpret_cast<int*>(sm + F.Wi);           // [2][GP][kp] this chunk's W in fixed point (hi, lo)
-  int* Wf = reinterpret_cast<int*>(sm + F.Wf);           // [kp] slots the chunk touched
+  // [GP][kp] anchor weights W in 64-bit fixed point (value 2^-e W64) for the
+  // whole slice; turned into floats in P's place after the last chunk
+  long long* W64 = reinterpret_cast<long long*>(sm + F.W);
   float2* lut = reinterpret_cast<float2*>(sm + F.lut);   // [16 nibbles][16 copies]
   int* pfs = reinterpret_cast<int*>(sm + F.pfs);         // [2][tps + 1]
   int* wpre = reinterpret_cast<int*>(sm + F.wpre);       // [2][ct/32 + 1]
@@ -259,6 +275,14 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
   auto issue_records = [&](int c) {
     uint8_t* st = stage_of(c);
     const int j0 = c * tiles_pc, j1 = min(nt, j0 + tiles_pc);
+    if (a.rlg) {
+      // key logits precomputed: the chunk's rows of them take the key codes' place
+      const int r0 = pfs[j0];
+      int n = pfs[j1] - r0;
+      n = n < 0 ? 0 : (n > ct ? ct : n);
+      copy_span(st + F.s_codes, reinterpret_cast<const uint8_t*>(a.rlg), (int64_t)(b + 1) * a.R * GP * 4,
+                ((int64_t)b * a.R + r0) * GP * 4, (int64_t)n * GP * 4, tid);
+    }
     for (int side = a.rlg ? 1 : 0; side < 2; ++side) {   // key logits precomputed: no key records
       const int r0 = pfs[side * (a.tps + 1) + j0];
       int n = pfs[side * (a.tps + 1) + j1] - r0;
@@ -331,12 +355,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
       if (slot < a.k) P[(lane % GP) * kp + slot] = v[0];
     }
   }
-  for (int i = tid; i < GP * kp; i += kThreads) {
-    Wt[i] = 0.f;
-    Wi[i] = 0;
-    Wi[GP * kp + i] = 0;
-  }
-  for (int i = tid; i < kp; i += kThreads) Wf[i] = 0;
+  for (int i = tid; i < GP * kp; i += kThreads) W64[i] = 0;
 
   // running state (identical in every thread): max per head; per-thread sums
   float mrun[GP], lsum[GP];
@@ -348,6 +367,13 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
     z01[g] = make_float2(0.f, 0.f);
     z23[g] = make_float2(0.f, 0.f);
   }
+  // W's fixed-point scale 2^e: terms p gamma 2^e with p <= 2^gap and
+  // |gamma| < 2^eg, at most 2^lt of them per slot, stay below 2^62 in sum
+  const int ntok_slice = min(a.N, t_end * kTile) - t_beg * kTile;
+  const int lt = 32 - __clz(ntok_slice);
+  int eg = -1000;                   // no gamma seen yet
+  float gbound = 0.f;               // 2^eg: |gamma| below it needs no rescale
+  float wsc = 1.f;                  // 2^e
   float2 qr01[GP], qr23[GP];
   __syncthreads();
 #pragma unroll
@@ -358,21 +384,37 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
   }
   const float2* lutc = lut + (lane & 15);
 
-  // Raises the running maximum to the chunk maximum `cm` when it beats it by
-  // the gap, rescaling every accumulator (CTA-uniform decision).
-  // Raises the running maximum to the chunk maximum `cm` when it beats it by
-  // the gap, rescaling the running sums and W (a CTA-uniform decision); the
-  // factors applied are left in f (1 where the maximum stayed).
-  auto update_max = [&](const float (&cm)[GP], float (&f)[GP]) {
+  // Raises the running maximum of head g to ceil(cm[g]) when cm[g] beats it by
+  // the gap (or on the first values), and the bound on |gamma| to the power of
+  // two above gm; the factors are exact powers of two, so the fixed-point W
+  // takes them as arithmetic right shifts.  CTA-uniform; f gets the factors of
+  // the float accumulators (1 where the maximum stayed).
+  auto update_max = [&](const float (&cm)[GP], float gm, float (&f)[GP]) {
+    int shw[GP];
     bool any = false;
+    int sh_all = 0;
+    if (gm >= gbound) {
+      int eg2 = gm > 0.f ? (int)((__float_as_uint(gm) >> 23) & 255u) - 126 : -40;   // gm < 2^eg2
+      eg2 = max(eg2, -40);
+      if (eg != -1000) sh_all = eg2 - eg;
+      eg = eg2;
+      gbound = __uint_as_float((uint32_t)(eg + 127) << 23);
+      const int e = 62 - lt - (int)kRescaleGap - eg;
+      wsc = __uint_as_float((uint32_t)(e + 127) << 23);
+      any = sh_all > 0;
+    }
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
       f[g] = 1.f;
+      shw[g] = sh_all;
       if (mrun[g] == -INFINITY) {
-        mrun[g] = cm[g];
+        mrun[g] = ceilf(cm[g]);
       } else if (cm[g] > mrun[g] + kRescaleGap) {
-        f[g] = exp2f(mrun[g] - cm[g]);
-        mrun[g] = cm[g];
+        const float nm = ceilf(cm[g]);
+        const float d = fminf(nm - mrun[g], 200.f);
+        f[g] = exp2f(-d);
+        shw[g] += (int)d;
+        mrun[g] = nm;
         any = true;
       }
     }
@@ -381,7 +423,11 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
       for (int g = 0; g < GP; ++g) {
         lsum[g] *= f[g];
         z01[g].x *= f[g]; z01[g].y *= f[g]; z23[g].x *= f[g]; z23[g].y *= f[g];
-        for (int i = tid; i < kp; i += kThreads) Wt[g * kp + i] *= f[g];
+        if (shw[g] > 0)
+          for (int i = tid; i < kp; i += kThreads) {
+            const long long w = W64[g * kp + i];
+            W64[g * kp + i] = shw[g] >= 63 ? (w < 0 ? -1ll : 0ll) : (w >> shw[g]);
+          }
       }
       __syncthreads();
     }
@@ -465,12 +511,12 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
       if (lane < ct / 32) wpre[side * (ct / 32 + 1) + lane + 1] = x;
       if (lane == 0) wpre[side * (ct / 32 + 1)] = 0;
     }
-    if (a.rlg) {
-      // key-record logits from the tensor-core pre-pass (sigma~ included)
-      const int nK = nrec[0];
-      const float* src = a.rlg + ((int64_t)b * a.R + rbase[0]) * GP;
-      for (int i = tid; i < nK * GP; i += kThreads) rlog[i] = src[i];
-    } else {
+    // key-record logits by rank: staged from the tensor-core pre-pass (sigma~
+    // included), or computed here into rlog
+    const float* klg = a.rlg ? reinterpret_cast<const float*>(codes) +
+                                   (int)((((int64_t)b * a.R + rbase[0]) * GP * 4) & 15) / 4
+                             : rlog;
+    if (!a.rlg) {
       constexpr int RB = 32 / GP;
       const int nK = nrec[0];
       for (int base = warp * RB; base < nK; base += kWarps * RB) {
@@ -494,8 +540,9 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
     }
     __syncthreads();
 
-    // b. token logits (their maximum only; phase d recomputes them) and the
-    //    value side's slot and coefficient
+    // b. every token's logit for the G heads (anchor term + its record's
+    //    residual term), kept in registers; the value side's slot and coefficient
+    float lg[kKT][GP];
     float cmx[GP];
     int slv[kKT];
     float gmv[kKT];
@@ -507,6 +554,8 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
       const int t = tid + i * kThreads;
       slv[i] = 0;
       gmv[i] = 0.f;
+#pragma unroll
+      for (int g = 0; g < GP; ++g) lg[i][g] = -INFINITY;
       if (t < ntok) {
         const uint32_t wv = tok0p[(ct + 4) + sh_tok[1] + t];
         slv[i] = min((int)(wv & 0xFFFFu), a.k - 1);
@@ -522,94 +571,49 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
 #pragma unroll
         for (int g = 0; g < GP; ++g) {
           float x = gam * P[g * kp + slot];
-          if (res) x += rlog[rank * GP + g];
+          if (res) x += klg[rank * GP + g];
+          lg[i][g] = x;
           cmx[g] = fmaxf(cmx[g], x);
         }
       }
     }
-    // c. chunk maximum, running maximum; fixed-point scale of the chunk's
-    //    anchor weights: |p gamma| <= 2^(cm - m) max|gamma|, ntok terms per
-    //    slot at most, so sum * 2^e stays below 2^30
-    float cm[GP], gmax, fsc[GP];
-    block_max2(cmx, gabs, cm, gmax);
-    update_max(cm, fsc);
-    // wsc = 2^e, winv = 2^-e, e = 30 - ceil(log2 ntok) - ceil(log2 bound):
-    // the chunk's sum of |terms| stays below 2^30 (the integer parts) and the
-    // remainders, scaled by 2^20, below 2^29
-    float wsc[GP], winv[GP];
-    const int en = 32 - __clz(ntok);
+    // c. the running maximum and W's scale change only when a logit beats the
+    //    maximum by the gap or a |gamma| reaches the scale's bound: one CTA
+    //    vote, and the reductions only when it says so (rare after the first chunk)
+    {
+      bool up = gabs >= gbound;
 #pragma unroll
-    for (int g = 0; g < GP; ++g) {
-      const float bound = exp2f(cm[g] - mrun[g]) * gmax;
-      int eb = bound > 0.f ? (int)((__float_as_uint(bound) >> 23) & 255u) - 126 : 0;   // bound < 2^eb
-      int e = 30 - en - eb;
-      e = max(-100, min(100, e));
-      wsc[g] = __uint_as_float((uint32_t)(e + 127) << 23);
-      winv[g] = __uint_as_float((uint32_t)(127 - e) << 23);
+      for (int g = 0; g < GP; ++g) up |= cmx[g] > mrun[g] + kRescaleGap;
+      if (__syncthreads_or(up)) {
+        float cm[GP], gmax, fsc[GP];
+        block_max2(cmx, gabs, cm, gmax);
+        update_max(cm, gmax, fsc);
+      }
     }
-    // d. probabilities, anchor weights (native integer atomics on the fixed
-    //    point), value-record weights
+    // d. probabilities, anchor weights (one native 64-bit integer atomic per
+    //    head on the fixed point), value-record weights p sigma~
 #pragma unroll
     for (int i = 0; i < kKT; ++i) {
       const int t = tid + i * kThreads;
       if (t < ntok) {
-        // this token's logits again (anchor term + key residual term)
-        float lgt[GP];
-        {
-          const uint32_t wk = tok0p[sh_tok[0] + t];
-          const int kslot = min((int)(wk & 0xFFFFu), a.k - 1);
-          const float kgam = half_bits_to_f(wk >> 16);
-          const uint32_t kword = bm0[t >> 5];
-          const int krank = wpre[t >> 5] + __popc(kword & ((1u << (t & 31)) - 1u));
-          const bool kres = ((kword >> (t & 31)) & 1u) && krank < nrec[0];
-#pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            float x = kgam * P[g * kp + kslot];
-            if (kres) x += rlog[krank * GP + g];
-            lgt[g] = x;
-          }
-        }
         const int slot = slv[i];
-        const float gam = gmv[i];
+        const float gs = gmv[i] * wsc;
         const uint32_t word = bm0[ct / 32 + (t >> 5)];
         const int rank = wpre[ct / 32 + 1 + (t >> 5)] + __popc(word & ((1u << (t & 31)) - 1u));
         const bool res = ((word >> (t & 31)) & 1u) && rank < nrec[1];
         const float sg = res ? half_bits_to_f(sig0[(ct + 8) + sh_sig[1] + rank]) : 0.f;
 #pragma unroll
         for (int g = 0; g < GP; ++g) {
-          const float p = exp2f(lgt[g] - mrun[g]);
-          lsum[g] += p;
-          // two native integer adds: the scaled term's integer part, then its
-          // rounded remainder scaled by 2^20 (2^-(e+20) resolution overall)
-          const float x = p * gam * wsc[g];
-          const float xh = rintf(x);
-          atomicAdd(&Wi[g * kp + slot], (int)xh);
-          atomicAdd(&Wi[GP * kp + g * kp + slot], __float2int_rn((x - xh) * 1048576.0f));
-          if (res) wz[rank * GP + g] = p * sg;
+          const float pr = exp2f(lg[i][g] - mrun[g]);
+          lsum[g] += pr;
+          atomicAdd(reinterpret_cast<unsigned long long*>(&W64[g * kp + slot]),
+                    (unsigned long long)__float2ll_rn(pr * gs));
+          if (res) wz[rank * GP + g] = pr * sg;
         }
-        Wf[slot] = 1;        // a plain store: any writer leaves 1
       }
     }
     __syncthreads();
-    // e. the chunk's fixed-point anchor weights into W, per token: the first
-    //    thread to take a touched slot's flag (atomic exchange with 0) folds
-    //    that slot for every head and is its only writer; value-residual sums
-#pragma unroll
-    for (int i = 0; i < kKT; ++i) {
-      const int t = tid + i * kThreads;
-      if (t < ntok) {
-        const int slot = slv[i];
-        if (atomicExch(&Wf[slot], 0)) {
-#pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            const int vh = Wi[g * kp + slot], vl = Wi[GP * kp + g * kp + slot];
-            Wt[g * kp + slot] += fmaf((float)vl, winv[g] * (1.0f / 1048576.0f), (float)vh * winv[g]);
-            Wi[g * kp + slot] = 0;
-            Wi[GP * kp + g * kp + slot] = 0;
-          }
-        }
-      }
-    }
+    // e. value-residual sums
     {
       const int nV = nrec[1];
       const uint8_t* vcodes = codes + ct * kCodeBytes;
@@ -632,7 +636,8 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
         for (int u = 0; u < kU; ++u) {
           const int r = r0 + u * kWarps;
           if (r < nV) {
-            const float* wr = wz + r * GP;
+            float wr[GP];
+            load_row<GP>(wz + r * GP, wr);
 #pragma unroll
             for (int g = 0; g < GP; ++g) {
               const float2 ww = make_float2(wr[g], wr[g]);
@@ -676,15 +681,15 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
         for (int g = 0; g < GP; ++g) cmx[g] = fmaxf(cmx[g], rlog[i * GP + g]);
       float fsc[GP];
       block_max(cmx, cm);
-      update_max(cm, fsc);
+      update_max(cm, 0.f, fsc);
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         oacc[g].x *= fsc[g]; oacc[g].y *= fsc[g]; oacc[g].z *= fsc[g]; oacc[g].w *= fsc[g];
       }
-      for (int i = tid; i < n * GP; i += kThreads) {
-        const float p = exp2f(rlog[i] - mrun[i % GP]);
-        rlog[i] = p;
-      }
+      // (heads unrolled: mrun stays in registers)
+      for (int i = tid; i < n; i += kThreads)
+#pragma unroll
+        for (int g = 0; g < GP; ++g) rlog[i * GP + g] = exp2f(rlog[i * GP + g] - mrun[g]);
       __syncthreads();
       // probabilities were written by other threads: sum them per head here
       for (int i = tid; i < n; i += kThreads)
@@ -713,7 +718,14 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
       if (lane == 0) red[kWarps * GP + warp * GP + g] = v;
     }
   }
-  // value anchors weighted by W (W is final after the last chunk's barrier)
+  // W as floats in P's place (P is no longer read), then the value anchors
+  // weighted by W
+  float* Wt = P;
+  {
+    const float winv = 1.f / wsc;    // an exact power of two
+    for (int i = tid; i < GP * kp; i += kThreads) Wt[i] = (float)W64[i] * winv;
+  }
+  __syncthreads();
   {
     const T* Va = reinterpret_cast<const T*>(comp + a.off_av) + (int64_t)h * a.k * kD;
 #pragma unroll 16
