@@ -51,6 +51,13 @@ constexpr int kCTMax = 512;                // most tokens per chunk
 constexpr int kKT = kCTMax / kThreads;     // most tokens per thread and chunk
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleGap = 8.0f;        // log2 units
+// anchor-weight terms in fixed point: below 2^kFixBits, split at 2^kSplit into
+// two int32 parts whose sums over kFoldChunks chunks (at most 2^13 terms per
+// slot) stay below 2^30
+constexpr int kFixBits = 34;
+constexpr int kSplit = 17;
+constexpr float kSplitScale = (float)(1u << kSplit);
+constexpr int kFoldChunks = 16;
 // dynamic shared memory a CTA may plan for: the 227 KB opt-in limit less
 // room for the kernel's static shared memory
 constexpr int kSmemBudget = 227 * 1024 - 256;
@@ -81,7 +88,7 @@ struct FArgs {
 
 // Shared-memory carve-up (bytes), the same on host and device.
 struct FPlan {
-  int qs, qr, P, W, lut, pfs, wpre, red, rlog, wz, stage, stage_bytes, total;
+  int qs, qr, P, W, Wi, lut, pfs, wpre, red, rlog, wz, stage, stage_bytes, total;
   // offsets inside one stage
   int s_codes, s_sig, s_tok, s_bm;
 };
@@ -100,9 +107,10 @@ __host__ __device__ inline FPlan fplan(int GP, int kp, int ct, int tps) {
   f.wpre = cur; cur = fa_align(cur + 2 * (ct / 32 + 1) * 4, 16);
   f.red = cur; cur = fa_align(cur + 2 * kWarps * GP * 4, 16);
   f.P = cur; cur += GP * kp * 4;
-  f.W = cur; cur += GP * kp * 8;
+  f.W = cur; cur += GP * kp * 4;
+  f.Wi = cur; cur += 2 * GP * kp * 4;
   f.rlog = cur; cur = fa_align(cur + ct * GP * 4, 16);
-  f.wz = cur; cur = fa_align(cur + ct * GP * 4, 16);
+  f.wz = cur; cur = fa_align(cur + ct * GP * 8, 16);
   // stage: codes [2][ct][32], scales [2][ct + 8] (16-byte spans), token words
   // [2][ct + 4], bitmap words [2][ct / 32]
   int sc = 0;
@@ -117,6 +125,11 @@ __host__ __device__ inline FPlan fplan(int GP, int kp, int ct, int tps) {
   f.total = fa_align(cur, 16);
   return f;
 }
+
+// Words of one slice's partial: (max, sum) per head padded to 16 bytes, then
+// the GP x 128 outputs (16-byte aligned, for the merge's 16-byte copies).
+__host__ __device__ constexpr int part_out(int GP) { return 4 * ((2 * GP + 3) / 4); }
+__host__ __device__ constexpr int part_words(int GP) { return part_out(GP) + GP * kD; }
 
 __host__ __device__ inline int gp_of(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : G <= 8 ? 8 : 16; }
 
@@ -150,19 +163,16 @@ __device__ __forceinline__ void copy_span(uint8_t* dst, const uint8_t* comp, int
   }
 }
 
-// GP consecutive floats of shared memory (16-byte aligned for GP >= 4) in as
-// few vector loads as they allow.
+// GP consecutive float2 of shared memory (16-byte aligned for GP >= 2).
 template <int GP>
-__device__ __forceinline__ void load_row(const float* src, float (&v)[GP]) {
-  if constexpr (GP >= 4) {
+__device__ __forceinline__ void load_pairs(const float2* src, float2 (&v)[GP]) {
+  if constexpr (GP >= 2) {
 #pragma unroll
-    for (int j = 0; j < GP / 4; ++j) {
+    for (int j = 0; j < GP / 2; ++j) {
       const float4 t = reinterpret_cast<const float4*>(src)[j];
-      v[4 * j] = t.x; v[4 * j + 1] = t.y; v[4 * j + 2] = t.z; v[4 * j + 3] = t.w;
+      v[2 * j] = make_float2(t.x, t.y);
+      v[2 * j + 1] = make_float2(t.z, t.w);
     }
-  } else if constexpr (GP == 2) {
-    const float2 t = *reinterpret_cast<const float2*>(src);
-    v[0] = t.x; v[1] = t.y;
   } else {
     v[0] = src[0];
   }
@@ -213,15 +223,20 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
   float* qs = reinterpret_cast<float*>(sm + F.qs);       // [GP][128] q' (log2 units)
   float* qr = reinterpret_cast<float*>(sm + F.qr);       // [GP][128] rotated q'
   float* P = reinterpret_cast<float*>(sm + F.P);         // [GP][kp]
-  // [GP][kp] anchor weights W in 64-bit fixed point (value 2^-e W64) for the
-  // whole slice; turned into floats in P's place after the last chunk
-  long long* W64 = reinterpret_cast<long long*>(sm + F.W);
+  // [GP][kp] anchor weights W: floats, plus the latest chunks' terms in
+  // fixed point (value 2^-e (hi 2^kSplit + lo), native 32-bit atomics),
+  // folded into the floats every kFoldChunks chunks and before any rescale
+  float* Wt = reinterpret_cast<float*>(sm + F.W);
+  int* Whi = reinterpret_cast<int*>(sm + F.Wi);
+  int* Wlo = Whi + GP * kp;
   float2* lut = reinterpret_cast<float2*>(sm + F.lut);   // [16 nibbles][16 copies]
   int* pfs = reinterpret_cast<int*>(sm + F.pfs);         // [2][tps + 1]
   int* wpre = reinterpret_cast<int*>(sm + F.wpre);       // [2][ct/32 + 1]
   float* red = reinterpret_cast<float*>(sm + F.red);     // [2][kWarps][GP]
   float* rlog = reinterpret_cast<float*>(sm + F.rlog);   // [ct][GP] key-record logits by rank
-  float* wz = reinterpret_cast<float*>(sm + F.wz);       // [ct][GP] value-record weights by rank
+  // [ct][GP] value-record weights by rank, each stored twice (an f32x2 operand)
+  float2* wz2 = reinterpret_cast<float2*>(sm + F.wz);
+  float* wz = reinterpret_cast<float*>(sm + F.wz);         // the merge's scratch
 
   const uint8_t* comp = a.comp + (int64_t)b * a.stride;
   const int t_beg = s * a.tps, t_end = min(a.n_tiles, t_beg + a.tps);
@@ -355,7 +370,11 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
       if (slot < a.k) P[(lane % GP) * kp + slot] = v[0];
     }
   }
-  for (int i = tid; i < GP * kp; i += kThreads) W64[i] = 0;
+  for (int i = tid; i < GP * kp; i += kThreads) {
+    Wt[i] = 0.f;
+    Whi[i] = 0;
+    Wlo[i] = 0;
+  }
 
   // running state (identical in every thread): max per head; per-thread sums
   float mrun[GP], lsum[GP];
@@ -367,13 +386,13 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
     z01[g] = make_float2(0.f, 0.f);
     z23[g] = make_float2(0.f, 0.f);
   }
-  // W's fixed-point scale 2^e: terms p gamma 2^e with p <= 2^gap and
-  // |gamma| < 2^eg, at most 2^lt of them per slot, stay below 2^62 in sum
-  const int ntok_slice = min(a.N, t_end * kTile) - t_beg * kTile;
-  const int lt = 32 - __clz(ntok_slice);
+  // W's fixed-point scale 2^e: a term p gamma 2^e with p <= 2^gap and
+  // |gamma| < 2^eg stays below 2^kFixBits; split at 2^kSplit into two int32
+  // parts, kFoldChunks chunks of terms fit either part's sum
   int eg = -1000;                   // no gamma seen yet
   float gbound = 0.f;               // 2^eg: |gamma| below it needs no rescale
-  float wsc = 1.f;                  // 2^e
+  float wsc = 1.f, winv = 1.f;      // 2^e, 2^-e
+  bool folded_all = true;           // no term since the last fold
   float2 qr01[GP], qr23[GP];
   __syncthreads();
 #pragma unroll
@@ -384,52 +403,56 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
   }
   const float2* lutc = lut + (lane & 15);
 
+  // Adds the fixed-point parts into the float weights (times f[g] for head g
+  // afterwards) and clears them.  Each thread touches its own entries only.
+  auto fold = [&](const float (&f)[GP]) {
+#pragma unroll
+    for (int g = 0; g < GP; ++g)
+      for (int i = tid; i < kp; i += kThreads) {
+        const int j = g * kp + i;
+        const float add = fmaf((float)Whi[j], kSplitScale, (float)Wlo[j]) * winv;
+        Wt[j] = (Wt[j] + add) * f[g];
+        Whi[j] = 0;
+        Wlo[j] = 0;
+      }
+  };
   // Raises the running maximum of head g to ceil(cm[g]) when cm[g] beats it by
   // the gap (or on the first values), and the bound on |gamma| to the power of
-  // two above gm; the factors are exact powers of two, so the fixed-point W
-  // takes them as arithmetic right shifts.  CTA-uniform; f gets the factors of
-  // the float accumulators (1 where the maximum stayed).
+  // two above gm (a new fixed-point scale).  CTA-uniform; the factors (exact
+  // powers of two) are left in f, 1 where the maximum stayed.
   auto update_max = [&](const float (&cm)[GP], float gm, float (&f)[GP]) {
-    int shw[GP];
     bool any = false;
-    int sh_all = 0;
-    if (gm >= gbound) {
-      int eg2 = gm > 0.f ? (int)((__float_as_uint(gm) >> 23) & 255u) - 126 : -40;   // gm < 2^eg2
-      eg2 = max(eg2, -40);
-      if (eg != -1000) sh_all = eg2 - eg;
-      eg = eg2;
-      gbound = __uint_as_float((uint32_t)(eg + 127) << 23);
-      const int e = 62 - lt - (int)kRescaleGap - eg;
-      wsc = __uint_as_float((uint32_t)(e + 127) << 23);
-      any = sh_all > 0;
-    }
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
       f[g] = 1.f;
-      shw[g] = sh_all;
       if (mrun[g] == -INFINITY) {
         mrun[g] = ceilf(cm[g]);
       } else if (cm[g] > mrun[g] + kRescaleGap) {
         const float nm = ceilf(cm[g]);
-        const float d = fminf(nm - mrun[g], 200.f);
-        f[g] = exp2f(-d);
-        shw[g] += (int)d;
+        f[g] = exp2f(-fminf(nm - mrun[g], 200.f));
         mrun[g] = nm;
         any = true;
       }
     }
-    if (any) {
+    const bool rescale = gm >= gbound;
+    if (any || rescale) {
+      // the parts so far go in at the old scale; a raised maximum rescales
+      // the floats as well
+      if (!folded_all || any) fold(f);
+      folded_all = true;
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         lsum[g] *= f[g];
         z01[g].x *= f[g]; z01[g].y *= f[g]; z23[g].x *= f[g]; z23[g].y *= f[g];
-        if (shw[g] > 0)
-          for (int i = tid; i < kp; i += kThreads) {
-            const long long w = W64[g * kp + i];
-            W64[g * kp + i] = shw[g] >= 63 ? (w < 0 ? -1ll : 0ll) : (w >> shw[g]);
-          }
       }
       __syncthreads();
+    }
+    if (rescale) {
+      eg = max(gm > 0.f ? (int)((__float_as_uint(gm) >> 23) & 255u) - 126 : -40, -40);   // gm < 2^eg
+      gbound = __uint_as_float((uint32_t)(eg + 127) << 23);
+      const int e = kFixBits - (int)kRescaleGap - eg;
+      wsc = __uint_as_float((uint32_t)(e + 127) << 23);
+      winv = __uint_as_float((uint32_t)(127 - e) << 23);
     }
   };
   // CTA-wide maximum per head of per-thread values (all threads get it).
@@ -523,8 +546,9 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
         float v[32];
 #pragma unroll
         for (int i = 0; i < RB; ++i) {
-          const int r = base + i;
-          const uint32_t byte = r < nK ? codes[r * kCodeBytes + lane] : 0u;
+          // records past nK (up to the batch's end, inside the chunk's buffer)
+          // are computed from stale codes and not stored
+          const uint32_t byte = codes[(base + i) * kCodeBytes + lane];
           const float2 l01 = lutc[(byte & 15u) * 16], l23 = lutc[(byte >> 4) * 16];
 #pragma unroll
           for (int g = 0; g < GP; ++g) {
@@ -590,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
         update_max(cm, gmax, fsc);
       }
     }
-    // d. probabilities, anchor weights (one native 64-bit integer atomic per
+    // d. probabilities, anchor weights (two native 32-bit integer atomics per
     //    head on the fixed point), value-record weights p sigma~
 #pragma unroll
     for (int i = 0; i < kKT; ++i) {
@@ -606,26 +630,44 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
         for (int g = 0; g < GP; ++g) {
           const float pr = exp2f(lg[i][g] - mrun[g]);
           lsum[g] += pr;
-          atomicAdd(reinterpret_cast<unsigned long long*>(&W64[g * kp + slot]),
-                    (unsigned long long)__float2ll_rn(pr * gs));
-          if (res) wz[rank * GP + g] = pr * sg;
+          const float x = pr * gs;                              // |x| < 2^kFixBits
+          const float xh = floorf(x * (1.0f / kSplitScale));
+          atomicAdd(&Whi[g * kp + slot], (int)xh);
+          atomicAdd(&Wlo[g * kp + slot], __float2int_rn(fmaf(-xh, kSplitScale, x)));
+          if (res) wz2[rank * GP + g] = make_float2(pr * sg, pr * sg);
         }
       }
     }
+    // the value records up to the next multiple of 32 get zero weights, so
+    // the value loop below runs whole steps (their codes are stale but in
+    // the chunk's buffer)
+    {
+      const int nV = nrec[1], pad = (((nV + 31) & ~31) - nV) * GP;
+      for (int i = tid; i < pad; i += kThreads) wz2[nV * GP + i] = make_float2(0.f, 0.f);
+    }
     __syncthreads();
+    folded_all = false;
+    // every kFoldChunks chunks the parts go into the floats (the next chunk's
+    // atomics come after its own barriers)
+    if ((c + 1) % kFoldChunks == 0 && c + 1 < n_chunks) {
+      float f1[GP];
+#pragma unroll
+      for (int g = 0; g < GP; ++g) f1[g] = 1.f;
+      fold(f1);
+      folded_all = true;
+    }
     // e. value-residual sums
     {
       const int nV = nrec[1];
       const uint8_t* vcodes = codes + ct * kCodeBytes;
-      // four records per step, their loads issued before any arithmetic
+      // four records per step, their loads issued before any arithmetic; the
+      // records run to a multiple of 32 (zero weights past nV)
       constexpr int kU = 4;
-      for (int r0 = warp; r0 < nV; r0 += kU * kWarps) {
+      const int nV32 = (nV + 31) & ~31;
+      for (int r0 = warp; r0 < nV32; r0 += kU * kWarps) {
         uint32_t byte[kU];
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int r = r0 + u * kWarps;
-          byte[u] = r < nV ? vcodes[r * kCodeBytes + lane] : 0u;
-        }
+        for (int u = 0; u < kU; ++u) byte[u] = vcodes[(r0 + u * kWarps) * kCodeBytes + lane];
         float2 l01[kU], l23[kU];
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
@@ -634,16 +676,12 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
         }
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
-          const int r = r0 + u * kWarps;
-          if (r < nV) {
-            float wr[GP];
-            load_row<GP>(wz + r * GP, wr);
+          float2 ww[GP];
+          load_pairs<GP>(wz2 + (r0 + u * kWarps) * GP, ww);
 #pragma unroll
-            for (int g = 0; g < GP; ++g) {
-              const float2 ww = make_float2(wr[g], wr[g]);
-              z01[g] = __ffma2_rn(l01[u], ww, z01[g]);
-              z23[g] = __ffma2_rn(l23[u], ww, z23[g]);
-            }
+          for (int g = 0; g < GP; ++g) {
+            z01[g] = __ffma2_rn(l01[u], ww[g], z01[g]);
+            z23[g] = __ffma2_rn(l23[u], ww[g], z23[g]);
           }
         }
       }
@@ -718,12 +756,12 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
       if (lane == 0) red[kWarps * GP + warp * GP + g] = v;
     }
   }
-  // W as floats in P's place (P is no longer read), then the value anchors
-  // weighted by W
-  float* Wt = P;
+  // the last parts into the float weights, then the value anchors weighted by W
   {
-    const float winv = 1.f / wsc;    // an exact power of two
-    for (int i = tid; i < GP * kp; i += kThreads) Wt[i] = (float)W64[i] * winv;
+    float f1[GP];
+#pragma unroll
+    for (int g = 0; g < GP; ++g) f1[g] = 1.f;
+    fold(f1);
   }
   __syncthreads();
   {
@@ -791,9 +829,9 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
     return;
   }
   // several slices: publish this one, the last to finish merges
-  const int PW = GP * (2 + kD);
+  constexpr int PW = part_words(GP), PO = part_out(GP);
   float* mine = a.part + ((int64_t)bh * a.S + s) * PW;
-  for (int i = tid; i < GP * kD; i += kThreads) mine[2 * GP + i] = opart[i];
+  for (int i = tid; i < GP * kD; i += kThreads) mine[PO + i] = opart[i];
 #pragma unroll
   for (int g = 0; g < GP; ++g)
     if (tid == g) {
@@ -808,8 +846,19 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
   if (!last) return;
   __threadfence();
   const float* all = a.part + (int64_t)bh * a.S * PW;
-  // every slice's (max, sum) per head in one round of loads, then the
-  // slices' weights 2^(m_s - M) / L per head; the outputs' loads go out together
+  // the slices' partials come into the (now idle) stage buffers by cp.async,
+  // as many per round as fit: all of them at once for the usual slice counts
+  uint8_t* mbuf = sm + F.stage;
+  const int cap = max(1, 2 * F.stage_bytes / (PW * 4));
+  auto issue = [&](int j0, int j1) {
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(all + (int64_t)j0 * PW);
+    const int units = (j1 - j0) * PW / 4;
+    for (int u = tid; u < units; u += kThreads) cp16(mbuf + 16 * u, src + 16 * u, 16);
+    cp_commit();
+  };
+  issue(0, min(a.S, cap));
+  // every slice's (max, sum) per head, then the weights 2^(m_s - M) / L (one
+  // warp per head, lanes over slices)
   float* ms = rlog;                    // [S][GP] maxima, then weights (S <= kMaxSlices)
   float* ls = wz;                      // [S][GP] sums
   for (int i = tid; i < a.S * GP; i += kThreads) {
@@ -818,45 +867,62 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
     ls[i] = __ldcg(all + (int64_t)j * PW + GP + g);
   }
   __syncthreads();
-  if (tid < GP) {
+  for (int g = warp; g < GP; g += kWarps) {
     float M = -INFINITY;
-    for (int j = 0; j < a.S; ++j) M = fmaxf(M, ms[j * GP + tid]);
+    for (int j = lane; j < a.S; j += 32) M = fmaxf(M, ms[j * GP + g]);
+    M = warp_max(M);
     float lt = 0.f;
-    for (int j = 0; j < a.S; ++j) {
-      const float f = exp2f(ms[j * GP + tid] - M);
-      ms[j * GP + tid] = f;
-      lt = fmaf(ls[j * GP + tid], f, lt);
+    for (int j = lane; j < a.S; j += 32) {
+      const float f = exp2f(ms[j * GP + g] - M);
+      ms[j * GP + g] = f;
+      lt = fmaf(ls[j * GP + g], f, lt);
     }
-    for (int j = 0; j < a.S; ++j) ms[j * GP + tid] /= lt;
+    const float inv = 1.f / warp_sum(lt);
+    for (int j = lane; j < a.S; j += 32) ms[j * GP + g] *= inv;
   }
-  __syncthreads();
-  // warp w sums the partials j = w (mod warps) over every (head, coordinate),
-  // all of a partial's loads in flight at once; the warps' sums meet in
-  // shared memory (the region from P on is free by now)
-  {
-    constexpr int EPL = GP * kD / 32;
-    float acc[EPL];
+  // thread t sums float4 column q = t mod NQ of the outputs over the slices
+  // j = t / NQ (mod NG)
+  constexpr int NQ = GP * kD / 4;
+  constexpr int NG = NQ >= kThreads ? 1 : kThreads / NQ;
+  constexpr int QPT = NQ > kThreads ? NQ / kThreads : 1;   // columns per thread
+  float4 acc[QPT];
 #pragma unroll
-    for (int m = 0; m < EPL; ++m) acc[m] = 0.f;
-    for (int j = warp; j < a.S; j += kWarps) {
-      const float* pj = all + (int64_t)j * PW + 2 * GP;
+  for (int m = 0; m < QPT; ++m) acc[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int grp = NQ >= kThreads ? 0 : tid / NQ;
+  for (int j0 = 0; j0 < a.S; j0 += cap) {
+    const int j1 = min(a.S, j0 + cap);
+    cp_wait<0>();
+    __syncthreads();
+    for (int j = j0 + grp; j < j1; j += NG) {
+      const float* pj = reinterpret_cast<const float*>(mbuf) + (j - j0) * PW + PO;
 #pragma unroll
-      for (int m = 0; m < EPL; ++m) {
-        const int e = lane + 32 * m;
-        acc[m] = fmaf(__ldcg(pj + e), ms[j * GP + e / kD], acc[m]);
+      for (int m = 0; m < QPT; ++m) {
+        const int q = (NQ >= kThreads ? tid + m * kThreads : tid % NQ);
+        const float w = ms[j * GP + (4 * q) / kD];
+        const float4 v = reinterpret_cast<const float4*>(pj)[q];
+        acc[m].x = fmaf(v.x, w, acc[m].x); acc[m].y = fmaf(v.y, w, acc[m].y);
+        acc[m].z = fmaf(v.z, w, acc[m].z); acc[m].w = fmaf(v.w, w, acc[m].w);
       }
     }
-    float* mred = reinterpret_cast<float*>(sm + F.P);
-    __syncthreads();           // every warp is done with the weights mred may cover
-#pragma unroll
-    for (int m = 0; m < EPL; ++m) mred[warp * GP * kD + lane + 32 * m] = acc[m];
     __syncthreads();
-    for (int i = tid; i < G * kD; i += kThreads) {
-      float o = 0.f;
+    if (j1 < a.S) issue(j1, min(a.S, j1 + cap));
+  }
+  // the groups' sums meet in the stage buffers
+  float4* mred = reinterpret_cast<float4*>(mbuf);
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) o += mred[w * GP * kD + i];
-      out[i] = o;
+  for (int m = 0; m < QPT; ++m) {
+    const int q = (NQ >= kThreads ? tid + m * kThreads : tid % NQ);
+    mred[grp * NQ + q] = acc[m];
+  }
+  __syncthreads();
+  for (int q = tid; q < G * kD / 4; q += kThreads) {
+    float4 o = mred[q];
+#pragma unroll
+    for (int r = 1; r < NG; ++r) {
+      const float4 t = mred[r * NQ + q];
+      o.x += t.x; o.y += t.y; o.z += t.z; o.w += t.w;
     }
+    reinterpret_cast<float4*>(out)[q] = o;
   }
 }
 
@@ -935,7 +1001,7 @@ bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs) {
   int64_t off = 0;
   auto take = [&](int64_t bytes) { int64_t o = off; off += (bytes + 255) / 256 * 256; return o; };
   fs->o_tickets = S > 1 ? take(4 * (int64_t)units) : 0;
-  fs->o_part = S > 1 ? take(4 * (int64_t)units * S * GP * (2 + kD)) : 0;
+  fs->o_part = S > 1 ? take(4 * (int64_t)units * S * part_words(GP)) : 0;
   fs->o_rlog = fs->klogit ? take(klogit_ws_bytes(pl, batch)) : 0;
   fs->ws_total = off;
   return true;
