@@ -163,6 +163,23 @@ __device__ __forceinline__ void copy_span(uint8_t* dst, const uint8_t* comp, int
   }
 }
 
+// GP consecutive floats of shared memory (16-byte aligned for GP >= 4).
+template <int GP>
+__device__ __forceinline__ void load_slot(const float* src, float (&v)[GP]) {
+  if constexpr (GP >= 4) {
+#pragma unroll
+    for (int j = 0; j < GP / 4; ++j) {
+      const float4 t = reinterpret_cast<const float4*>(src)[j];
+      v[4 * j] = t.x; v[4 * j + 1] = t.y; v[4 * j + 2] = t.z; v[4 * j + 3] = t.w;
+    }
+  } else if constexpr (GP == 2) {
+    const float2 t = *reinterpret_cast<const float2*>(src);
+    v[0] = t.x; v[1] = t.y;
+  } else {
+    v[0] = src[0];
+  }
+}
+
 // GP consecutive float2 of shared memory (16-byte aligned for GP >= 2).
 template <int GP>
 __device__ __forceinline__ void load_pairs(const float2* src, float2 (&v)[GP]) {
@@ -210,6 +227,63 @@ template <> struct RawRow<float> {
     o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
   }
 };
+
+// Eight consecutive elements (8 hl .. 8 hl + 7) of row `row` kept raw until
+// used; rows at or past `rows` read as zeros.
+template <typename T> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+  using type = uint4;
+  __device__ __forceinline__ static uint4 load(const __nv_bfloat16* base, int row, int rows, int hl) {
+    return row < rows ? *reinterpret_cast<const uint4*>(base + (int64_t)row * kD + 8 * hl) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  __device__ __forceinline__ static void to_f2(const uint4 v, float2 (&o)[4]) {
+    o[0] = make_float2(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u));
+    o[1] = make_float2(__uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
+    o[2] = make_float2(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xFFFF0000u));
+    o[3] = make_float2(__uint_as_float(v.w << 16), __uint_as_float(v.w & 0xFFFF0000u));
+  }
+};
+template <> struct Raw8<float> {
+  struct type { float4 a, b; };
+  __device__ __forceinline__ static type load(const float* base, int row, int rows, int hl) {
+    type t;
+    if (row < rows) {
+      t.a = *reinterpret_cast<const float4*>(base + (int64_t)row * kD + 8 * hl);
+      t.b = *reinterpret_cast<const float4*>(base + (int64_t)row * kD + 8 * hl + 4);
+    } else {
+      t.a = t.b = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    return t;
+  }
+  __device__ __forceinline__ static void to_f2(const type& v, float2 (&o)[4]) {
+    o[0] = make_float2(v.a.x, v.a.y); o[1] = make_float2(v.a.z, v.a.w);
+    o[2] = make_float2(v.b.x, v.b.y); o[3] = make_float2(v.b.z, v.b.w);
+  }
+};
+
+// Sums V values over the 16 lanes of each half-warp, transposed: afterwards
+// lane l holds the total of value (l & 15) / (16 / V).
+template <int V>
+__device__ __forceinline__ void transpose_reduce16(float (&v)[V], int lane) {
+  int n = V;
+#pragma unroll
+  for (int off = 8; off >= 1; off >>= 1) {
+    if (n > 1) {
+      const int hf = n / 2;
+      const bool up = (lane & off) != 0;
+#pragma unroll
+      for (int i = 0; i < V / 2; ++i)
+        if (i < hf) {
+          const float keep = up ? v[i + hf] : v[i];
+          const float send = up ? v[i] : v[i + hf];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      n = hf;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+    }
+  }
+}
 
 // ---------------------------------------------------------------- the kernel
 
@@ -328,7 +402,54 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
 #pragma unroll
     for (int i = 0; i < 4; ++i) qr[g * kD + 4 * lane + i] = v[i];
   }
-  {
+  if constexpr (GP <= 8) {
+    // half-warp per slot, 8 coordinates per lane: the query's 8 x GP values
+    // stay in registers, the row is one 16-byte load (bf16), and the GP dot
+    // products meet in a 16-lane transposed reduction
+    const int half = lane >> 4, hl = lane & 15;
+    float2 q2[GP][4];
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      const float4 a4 = *reinterpret_cast<const float4*>(qs + g * kD + 8 * hl);
+      const float4 b4 = *reinterpret_cast<const float4*>(qs + g * kD + 8 * hl + 4);
+      q2[g][0] = make_float2(a4.x, a4.y); q2[g][1] = make_float2(a4.z, a4.w);
+      q2[g][2] = make_float2(b4.x, b4.y); q2[g][3] = make_float2(b4.z, b4.w);
+    }
+    const T* Ka = reinterpret_cast<const T*>(comp + a.off_ak) + (int64_t)h * a.k * kD;
+    using R8 = Raw8<T>;
+    // four slot pairs per step, the next step's rows in flight meanwhile
+    constexpr int kPS = 4;
+    typename R8::type nx[kPS];
+    const int npair = (a.k + 1) / 2;
+    auto fetch = [&](int sp0) {
+#pragma unroll
+      for (int u = 0; u < kPS; ++u) nx[u] = R8::load(Ka, 2 * (sp0 + u * kWarps) + half, a.k, hl);
+    };
+    if (warp < npair) fetch(warp);
+    for (int sp0 = warp; sp0 < npair; sp0 += kPS * kWarps) {
+      typename R8::type cx[kPS];
+#pragma unroll
+      for (int u = 0; u < kPS; ++u) cx[u] = nx[u];
+      if (sp0 + kPS * kWarps < npair) fetch(sp0 + kPS * kWarps);
+#pragma unroll
+      for (int u = 0; u < kPS; ++u) {
+        float2 x2[4];
+        R8::to_f2(cx[u], x2);
+        float v[GP];
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          float2 acc = __fmul2_rn(x2[0], q2[g][0]);
+          acc = __ffma2_rn(x2[1], q2[g][1], acc);
+          acc = __ffma2_rn(x2[2], q2[g][2], acc);
+          acc = __ffma2_rn(x2[3], q2[g][3], acc);
+          v[g] = acc.x + acc.y;
+        }
+        transpose_reduce16<GP>(v, lane);
+        const int slot = 2 * (sp0 + u * kWarps) + half;
+        if (slot < a.k && (hl % (16 / GP)) == 0) P[slot * GP + hl / (16 / GP)] = v[0];
+      }
+    }
+  } else   {
     float4 q4[GP];
 #pragma unroll
     for (int g = 0; g < GP; ++g) q4[g] = *reinterpret_cast<const float4*>(qs + g * kD + 4 * lane);
@@ -367,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
       }
       transpose_reduce32(v, lane);
       const int slot = base + lane / GP;
-      if (slot < a.k) P[(lane % GP) * kp + slot] = v[0];
+      if (slot < a.k) P[slot * GP + (lane % GP)] = v[0];
     }
   }
   for (int i = tid; i < GP * kp; i += kThreads) {
@@ -409,9 +530,9 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
 #pragma unroll
     for (int g = 0; g < GP; ++g)
       for (int i = tid; i < kp; i += kThreads) {
-        const int j = g * kp + i;
+        const int j = g * kp + i, jt = i * GP + g;
         const float add = fmaf((float)Whi[j], kSplitScale, (float)Wlo[j]) * winv;
-        Wt[j] = (Wt[j] + add) * f[g];
+        Wt[jt] = (Wt[jt] + add) * f[g];
         Whi[j] = 0;
         Wlo[j] = 0;
       }
@@ -592,9 +713,11 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
         const uint32_t below = word & ((1u << (t & 31)) - 1u);
         const int rank = wpre[t >> 5] + __popc(below);
         const bool res = ((word >> (t & 31)) & 1u) && rank < nrec[0];
+        float pv[GP];
+        load_slot<GP>(P + slot * GP, pv);
 #pragma unroll
         for (int g = 0; g < GP; ++g) {
-          float x = gam * P[g * kp + slot];
+          float x = gam * pv[g];
           if (res) x += klg[rank * GP + g];
           lg[i][g] = x;
           cmx[g] = fmaxf(cmx[g], x);
@@ -766,15 +889,41 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
   __syncthreads();
   {
     const T* Va = reinterpret_cast<const T*>(comp + a.off_av) + (int64_t)h * a.k * kD;
-#pragma unroll 16
-    for (int slot = warp; slot < a.k; slot += kWarps) {
-      float x[4];
-      load4(Va + (int64_t)slot * kD + 4 * lane, x);
+    if constexpr (GP >= 2) {
+      // heads in pairs: (o_2j, o_2j+1)[d] += (W_2j, W_2j+1) x[d], one f32x2 FMA
+      float2 acc[GP / 2][4];
 #pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        const float w = Wt[g * kp + slot];
-        oacc[g].x = fmaf(w, x[0], oacc[g].x); oacc[g].y = fmaf(w, x[1], oacc[g].y);
-        oacc[g].z = fmaf(w, x[2], oacc[g].z); oacc[g].w = fmaf(w, x[3], oacc[g].w);
+      for (int j = 0; j < GP / 2; ++j)
+#pragma unroll
+        for (int d = 0; d < 4; ++d) acc[j][d] = make_float2(0.f, 0.f);
+#pragma unroll 8
+      for (int slot = warp; slot < a.k; slot += kWarps) {
+        float x[4];
+        load4(Va + (int64_t)slot * kD + 4 * lane, x);
+        float w[GP];
+        load_slot<GP>(Wt + slot * GP, w);
+#pragma unroll
+        for (int j = 0; j < GP / 2; ++j) {
+          const float2 w2 = make_float2(w[2 * j], w[2 * j + 1]);
+#pragma unroll
+          for (int d = 0; d < 4; ++d) acc[j][d] = __ffma2_rn(w2, make_float2(x[d], x[d]), acc[j][d]);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < GP / 2; ++j) {
+        oacc[2 * j].x += acc[j][0].x; oacc[2 * j].y += acc[j][1].x;
+        oacc[2 * j].z += acc[j][2].x; oacc[2 * j].w += acc[j][3].x;
+        oacc[2 * j + 1].x += acc[j][0].y; oacc[2 * j + 1].y += acc[j][1].y;
+        oacc[2 * j + 1].z += acc[j][2].y; oacc[2 * j + 1].w += acc[j][3].y;
+      }
+    } else {
+#pragma unroll 16
+      for (int slot = warp; slot < a.k; slot += kWarps) {
+        float x[4];
+        load4(Va + (int64_t)slot * kD + 4 * lane, x);
+        const float w = Wt[slot];
+        oacc[0].x = fmaf(w, x[0], oacc[0].x); oacc[0].y = fmaf(w, x[1], oacc[0].y);
+        oacc[0].z = fmaf(w, x[2], oacc[0].z); oacc[0].w = fmaf(w, x[3], oacc[0].w);
       }
     }
   }
@@ -993,11 +1142,12 @@ bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs) {
   fs->tps = tps;
   fs->smem = fplan(GP, kp, fs->ct, tps).total;
   // key-residual logits on the tensor cores ahead of the decode: worth it
-  // when the launch is throughput-bound (a slice or two per head), not at
-  // batch 1 where latency rules; ANCHORKV_DECODE_KLOGIT=0/1 forces it
+  // when the launch is throughput-bound (two slices per head or fewer, i.e.
+  // many sequences), not when a few heads are cut into many slices and
+  // latency rules; ANCHORKV_DECODE_KLOGIT=0/1 forces it either way
   const char* kenv = getenv("ANCHORKV_DECODE_KLOGIT");
   fs->klogit = klogit_tc_supported(pl) && pl.R > 0 &&
-               (kenv && kenv[0] ? kenv[0] == '1' : false);
+               (kenv && kenv[0] ? kenv[0] == '1' : S <= 2);
   int64_t off = 0;
   auto take = [&](int64_t bytes) { int64_t o = off; off += (bytes + 255) / 256 * 256; return o; };
   fs->o_tickets = S > 1 ? take(4 * (int64_t)units) : 0;

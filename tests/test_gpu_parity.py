@@ -129,11 +129,13 @@ def test_decode_parity(name, batch, tail):
                                                   ("bf16-gqa8-n2500", 2, 0, 0), ("bf16-every-residual", 1, 3, 0),
                                                   ("fp32-window8-n700", 2, 9, 0), ("bf16-n20000", 2, 1500, 0),
                                                   ("bf16-ragged-n3000", 2, 4, 0x10)])
-def test_decode_tensor_core_key_logits(name, batch, tail, mode, monkeypatch):
-    """The key-residual logits computed ahead of the decode on the tensor
-    cores (bit planes of the codes times a fixed-point query, kind::i8)
-    give the same decode as the oracle."""
-    monkeypatch.setenv("ANCHORKV_DECODE_KLOGIT", "1")
+@pytest.mark.parametrize("klogit", ["1", "0"])
+def test_decode_tensor_core_key_logits(name, batch, tail, mode, klogit, monkeypatch):
+    """Both ways to the key-residual logits give the oracle's decode, whatever
+    the launch shape would pick by default: ahead of the decode on the tensor
+    cores (bit planes of the codes times a fixed-point query, kind::i8), or
+    inside the decode on the CUDA cores."""
+    monkeypatch.setenv("ANCHORKV_DECODE_KLOGIT", klogit)
     spec, theta = CASES[name]
     p = _params(spec, theta)
     p.mode = mode
