@@ -218,6 +218,10 @@ int anchorkv_decode_workspace_bytes(const anchorkv_params* p, int32_t batch, siz
  * tail_len > 4096 or no launch shape fits the device.
  * Work split: each (sequence, KV head) is cut into token slices that run on
  * separate CTAs across the GPU; the last slice to finish merges the others.
+ * When a head gets two slices or fewer (many sequences), a tensor-core pass
+ * first computes every key record's residual logits into the workspace
+ * (batch x R x G floats); ANCHORKV_DECODE_KLOGIT=0 or 1 in the environment
+ * turns that pass off or on for every shape.
  */
 int anchorkv_decode_attn(const anchorkv_params* p, const void* compressed,
                          int64_t seq_stride_bytes, int32_t batch, const void* q,
@@ -270,8 +274,11 @@ int anchorkv_decode_config(const anchorkv_params* p, int32_t batch, int32_t* sli
  * free HBM is all handed to its KV-cache pool, a plain-C caller without a
  * device allocator, or a decode loop that must not take the device-wide
  * synchronisation cudaMalloc / cudaFree bring.
- *   - Sizes whose decode workspace (anchorkv_decode_workspace_bytes) exceeds
- *     the maximum are rejected with ANCHORKV_ENOSPC before any launch.
+ *   - When anchorkv_decode_workspace_bytes exceeds the array, the call first
+ *     drops the tensor-core key-logit pre-pass (whose batch x R x G floats
+ *     dominate that workspace at large batch) and computes those logits
+ *     inside the decode instead; sizes that still do not fit are rejected
+ *     with ANCHORKV_ENOSPC before any launch.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
  *   - Every call on a device shares the array, which keeps the last call's

@@ -333,9 +333,9 @@ decode_combine_kernel(DecodeArgs a, const T* __restrict__ q, const T* __restrict
 
 }  // namespace
 
-int make_decode_plan(const Plan& pl, int batch, DecodePlan* dp) {
+int make_decode_plan(const Plan& pl, int batch, DecodePlan* dp, bool allow_prepass) {
   dp->batch = batch;
-  dp->flash = flash_decode_plan(pl, batch, &dp->fs);
+  dp->flash = flash_decode_plan(pl, batch, &dp->fs, allow_prepass);
   if (dp->flash) {
     dp->n_split = 0; dp->split_tokens = 0;
     dp->o_P = dp->o_qrot = dp->o_part_m = dp->o_part_l = dp->o_part_w = dp->o_part_z = 0;

@@ -330,6 +330,14 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
       prefetch_l2(ak + o);
       prefetch_l2(av + o);
     }
+    if (has_tail) {
+      // the exact tail's rows too, read after the last chunk
+      const int64_t tb = (int64_t)a.tail_len * kD * sizeof(T), base = ((int64_t)b * a.H + h) * a.tail_cap * kD * sizeof(T);
+      for (int64_t o = (int64_t)tid * 128; o < tb; o += (int64_t)kThreads * 128) {
+        prefetch_l2(reinterpret_cast<const uint8_t*>(a.Kt) + base + o);
+        prefetch_l2(reinterpret_cast<const uint8_t*>(a.Vt) + base + o);
+      }
+    }
     const int* pf = reinterpret_cast<const int*>(comp + a.off_pf);
     for (int i = tid; i < 2 * (nt + 1); i += kThreads) {
       const int side = i / (nt + 1), j = i % (nt + 1);
@@ -824,13 +832,31 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
     const T* Vt = reinterpret_cast<const T*>(a.Vt) + ((int64_t)b * a.H + h) * a.tail_cap * kD;
     for (int t0 = 0; t0 < a.tail_len; t0 += ct) {
       const int n = min(ct, a.tail_len - t0);
-      for (int i = warp; i < n; i += kWarps) {
-        float x[4];
-        load4(Kt + (int64_t)(t0 + i) * kD + 4 * lane, x);
+      // logits: TB tokens per warp step, their rows loaded together and their
+      // TB x GP dot products finished by one transposed reduction
+      {
+        constexpr int TB = GP >= 4 ? 32 / GP : 8;
+        for (int base = warp * TB; base < n; base += kWarps * TB) {
+          float x[TB][4];
 #pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          const float d = warp_sum(fmaf(q4[g].x, x[0], fmaf(q4[g].y, x[1], fmaf(q4[g].z, x[2], q4[g].w * x[3]))));
-          if (lane == 0) rlog[i * GP + g] = d;
+          for (int i = 0; i < TB; ++i) {
+            if (base + i < n) {
+              load4(Kt + (int64_t)(t0 + base + i) * kD + 4 * lane, x[i]);
+            } else {
+              x[i][0] = x[i][1] = x[i][2] = x[i][3] = 0.f;
+            }
+          }
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+#pragma unroll
+          for (int i = 0; i < TB; ++i)
+#pragma unroll
+            for (int g = 0; g < GP; ++g)
+              v[i * GP + g] = fmaf(q4[g].x, x[i][0], fmaf(q4[g].y, x[i][1], fmaf(q4[g].z, x[i][2], q4[g].w * x[i][3])));
+          transpose_reduce32(v, lane);
+          const int i = base + lane / GP;
+          if (lane < TB * GP && i < n) rlog[i * GP + (lane % GP)] = v[0];
         }
       }
       __syncthreads();
@@ -856,14 +882,29 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
       for (int i = tid; i < n; i += kThreads)
 #pragma unroll
         for (int g = 0; g < GP; ++g) lsum[g] += rlog[i * GP + g];
-      for (int i = warp; i < n; i += kWarps) {
-        float x[4];
-        load4(Vt + (int64_t)(t0 + i) * kD + 4 * lane, x);
+      // values: four rows per warp step, loaded together
+      for (int i0 = warp; i0 < n; i0 += 4 * kWarps) {
+        float x[4][4];
 #pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          const float p = rlog[i * GP + g];
-          oacc[g].x = fmaf(p, x[0], oacc[g].x); oacc[g].y = fmaf(p, x[1], oacc[g].y);
-          oacc[g].z = fmaf(p, x[2], oacc[g].z); oacc[g].w = fmaf(p, x[3], oacc[g].w);
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * kWarps;
+          if (i < n) {
+            load4(Vt + (int64_t)(t0 + i) * kD + 4 * lane, x[u]);
+          } else {
+            x[u][0] = x[u][1] = x[u][2] = x[u][3] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * kWarps;
+          if (i < n) {
+#pragma unroll
+            for (int g = 0; g < GP; ++g) {
+              const float p = rlog[i * GP + g];
+              oacc[g].x = fmaf(p, x[u][0], oacc[g].x); oacc[g].y = fmaf(p, x[u][1], oacc[g].y);
+              oacc[g].z = fmaf(p, x[u][2], oacc[g].z); oacc[g].w = fmaf(p, x[u][3], oacc[g].w);
+            }
+          }
         }
       }
       __syncthreads();
@@ -1115,7 +1156,7 @@ int max_ctas_per_sm(int smem) {
 // Shape of the slice decode for `batch` sequences: tokens per chunk, slices
 // per (sequence, head) and the workspace.  Returns false when no chunk size
 // fits the shared memory (the split-token kernels take over).
-bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs) {
+bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs, bool allow_prepass) {
   const int GP = gp_of(pl.G);
   const int kp = (pl.k + 3) & ~3;
   // CTAs resident per SM: two when the registers allow it (G <= 4) and the
@@ -1146,7 +1187,7 @@ bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs) {
   // many sequences), not when a few heads are cut into many slices and
   // latency rules; ANCHORKV_DECODE_KLOGIT=0/1 forces it either way
   const char* kenv = getenv("ANCHORKV_DECODE_KLOGIT");
-  fs->klogit = klogit_tc_supported(pl) && pl.R > 0 &&
+  fs->klogit = allow_prepass && klogit_tc_supported(pl) && pl.R > 0 &&
                (kenv && kenv[0] ? kenv[0] == '1' : S <= 2);
   int64_t off = 0;
   auto take = [&](int64_t bytes) { int64_t o = off; off += (bytes + 255) / 256 * 256; return o; };

@@ -83,6 +83,9 @@ int anchorkv_decode_attn_noalloc(const anchorkv_params* p, const void* compresse
     return ANCHORKV_EINVAL;
   DecodePlan dp;
   make_decode_plan(pl, batch, &dp);
+  // the key-logit pre-pass needs batch x R x G floats of scratch: without it
+  // if the array cannot hold them (the decode computes those logits itself)
+  if (dp.ws_total > (int64_t)ANCHORKV_DECODE_NOALLOC_SCRATCH_BYTES) make_decode_plan(pl, batch, &dp, false);
   if (dp.ws_total > (int64_t)ANCHORKV_DECODE_NOALLOC_SCRATCH_BYTES) return ANCHORKV_ENOSPC;
   st = check_decode_shape(pl, dp, tail_len);
   if (st) return st;

@@ -75,10 +75,12 @@ struct DecodePlan {
   int batch, n_split, split_tokens;
   int64_t ws_total, o_P, o_qrot, o_part_m, o_part_l, o_part_w, o_part_z;
 };
-int make_decode_plan(const Plan& pl, int batch, DecodePlan* out);
+// allow_prepass = false keeps the key logits inside the decode (no pre-pass
+// workspace), for callers whose scratch is fixed.
+int make_decode_plan(const Plan& pl, int batch, DecodePlan* out, bool allow_prepass = true);
 // Shape checks of a decode call (shared-memory limits of the chosen path).
 int check_decode_shape(const Plan& pl, const DecodePlan& dp, int tail_len);
-bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs);
+bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs, bool allow_prepass = true);
 int launch_flash_decode(const Plan& pl, const FlashShape& fs, int batch, const char* comp, int64_t stride,
                         const void* q, const void* Kt, const void* Vt, int tail_len, int tail_cap, float* out,
                         char* ws, cudaStream_t s);

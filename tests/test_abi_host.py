@@ -86,7 +86,7 @@ def test_library_codebook_matches_oracle():
         assert abs(a - b) < 1e-13
 
 
-def test_workspace_view():
+def test_workspace_view(monkeypatch):
     p = api.AnchorKVParams(n_tokens=32768)
     v = api.compress_workspace(p)
     assert v["total_bytes"] > v["off_utility"] + 4 * 2 * 8 * 32768
@@ -94,8 +94,16 @@ def test_workspace_view():
     # the slice decode needs tickets and slice partials only when a (sequence,
     # head) is cut into several slices: at batch 1 (8 heads on ~148 CTAs) it
     # is, at batch 32 (256 heads) every head is one slice and needs nothing
+    # but the key-logit pre-pass's batch x R x G floats, which that shape
+    # turns on by default
     assert api.decode_workspace_bytes(p, 1) > 0
+    R = api.anchorkv_bytes(p)["n_residuals"]
+    assert api.decode_workspace_bytes(p, 32) == (32 * R * 4 * 4 + 255) // 256 * 256
+    monkeypatch.setenv("ANCHORKV_DECODE_KLOGIT", "0")
     assert api.decode_workspace_bytes(p, 32) == 0
+    monkeypatch.setenv("ANCHORKV_DECODE_KLOGIT", "1")
+    assert api.decode_workspace_bytes(p, 1) > (R * 4 * 4 + 255) // 256 * 256
+    monkeypatch.delenv("ANCHORKV_DECODE_KLOGIT")
     # 16 query heads per KV head with 1056 anchors do not fit the slice
     # decode's shared memory: the split-token kernels and their workspace
     p16 = api.AnchorKVParams(n_tokens=131072, n_q_heads=128)
