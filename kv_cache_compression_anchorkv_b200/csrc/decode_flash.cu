@@ -41,6 +41,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc_util.cuh"
 
 namespace akv {
 namespace {
@@ -195,6 +196,14 @@ __device__ __forceinline__ void load_pairs(const float2* src, float2 (&v)[GP]) {
   }
 }
 
+// One contiguous global -> shared copy by the bulk-copy engine (16-byte
+// aligned addresses, size a multiple of 16), completing on `bar`.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(tc::smem_u32(dst)), "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+               : "memory");
+}
+
 // Brings the 128-byte line at p into L2 (no register result, no wait).
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
@@ -318,6 +327,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
   const int n_chunks = (nt * kTile + ct - 1) / ct;
   const int tiles_pc = ct / kTile;
   const bool has_tail = (s == a.S - 1) && a.tail_len > 0;
+  bool copy_failed = false;         // a chunk's bulk copy never completed (bounded wait)
 
   // ---- 1. prefixes of the slice's tiles, the query, the nibble table; first token words
   {
@@ -369,26 +379,49 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
       copy_span(st + F.s_bm + side * (ct / 32) * 4, comp, a.total, boff, 16 * (int64_t)(c1 - c0), tid);
     }
   };
+  // residual codes (and the pre-pass key logits) by the bulk-copy engine, one
+  // instruction per section issued by thread 0 and completing on the stage's
+  // barrier; the 2-byte scales by cp.async (their spans are not 16-byte aligned)
+  __shared__ __align__(8) uint64_t sbar[2];
   auto issue_records = [&](int c) {
     uint8_t* st = stage_of(c);
     const int j0 = c * tiles_pc, j1 = min(nt, j0 + tiles_pc);
-    if (a.rlg) {
-      // key logits precomputed: the chunk's rows of them take the key codes' place
-      const int r0 = pfs[j0];
-      int n = pfs[j1] - r0;
-      n = n < 0 ? 0 : (n > ct ? ct : n);
+    int r0s[2], ns[2];
+#pragma unroll
+    for (int side = 0; side < 2; ++side) {
+      r0s[side] = pfs[side * (a.tps + 1) + j0];
+      const int n = pfs[side * (a.tps + 1) + j1] - r0s[side];
+      ns[side] = n < 0 ? 0 : (n > ct ? ct : n);
+    }
+    const bool rlg_bulk = a.rlg && GP >= 4;   // 16-byte aligned rows of GP floats
+    if (tid == 0) {
+      tc::fence_proxy_async_smem();   // the buffer's last generic reads precede these writes
+      uint32_t bytes = (uint32_t)ns[1] * kCodeBytes;
+      if (!a.rlg) bytes += (uint32_t)ns[0] * kCodeBytes;
+      else if (rlg_bulk) bytes += (uint32_t)ns[0] * GP * 4;
+      tc::mbar_expect_tx(&sbar[c & 1], bytes);
+#pragma unroll
+      for (int side = 0; side < 2; ++side)
+        if (ns[side] > 0 && !(side == 0 && a.rlg))
+          bulk_g2s(st + F.s_codes + side * ct * kCodeBytes, comp + a.off_codes + (int64_t)kCodeBytes * r0s[side],
+                   (uint32_t)ns[side] * kCodeBytes, &sbar[c & 1]);
+      if (rlg_bulk && ns[0] > 0)
+        bulk_g2s(st + F.s_codes, a.rlg + ((int64_t)b * a.R + r0s[0]) * GP, (uint32_t)ns[0] * GP * 4, &sbar[c & 1]);
+    }
+    if (a.rlg && !rlg_bulk)
       copy_span(st + F.s_codes, reinterpret_cast<const uint8_t*>(a.rlg), (int64_t)(b + 1) * a.R * GP * 4,
-                ((int64_t)b * a.R + r0) * GP * 4, (int64_t)n * GP * 4, tid);
-    }
-    for (int side = a.rlg ? 1 : 0; side < 2; ++side) {   // key logits precomputed: no key records
-      const int r0 = pfs[side * (a.tps + 1) + j0];
-      int n = pfs[side * (a.tps + 1) + j1] - r0;
-      n = n < 0 ? 0 : (n > ct ? ct : n);
-      copy_span(st + F.s_codes + side * ct * kCodeBytes, comp, a.total, a.off_codes + (int64_t)kCodeBytes * r0,
-                (int64_t)kCodeBytes * n, tid);
-      copy_span(st + F.s_sig + side * (ct + 8) * 2, comp, a.total, a.off_sig + 2 * (int64_t)r0, 2 * (int64_t)n, tid);
-    }
+                ((int64_t)b * a.R + r0s[0]) * GP * 4, (int64_t)ns[0] * GP * 4, tid);
+#pragma unroll
+    for (int side = 0; side < 2; ++side)
+      if (!(side == 0 && a.rlg))
+        copy_span(st + F.s_sig + side * (ct + 8) * 2, comp, a.total, a.off_sig + 2 * (int64_t)r0s[side],
+                  2 * (int64_t)ns[side], tid);
   };
+  if (tid == 0) {
+    tc::mbar_init(&sbar[0], 1);
+    tc::mbar_init(&sbar[1], 1);
+    tc::fence_barrier_init();
+  }
   issue_words(0);
   __syncthreads();
   issue_records(0);
@@ -626,6 +659,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
     // chunk c has landed; past this barrier every thread is done with chunk
     // c - 1, so its buffer takes chunk c + 1 while chunk c is worked on
     cp_wait<0>();
+    if (!tc::mbar_wait(&sbar[c & 1], (c >> 1) & 1)) copy_failed = true;
     __syncthreads();
     if (c + 1 < n_chunks) {
       issue_words(c + 1);
@@ -912,7 +946,12 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
   }
 
   // ---- 5. partial output of this slice
-  // sum of probabilities per head (per warp; summed where used)
+  // sum of probabilities per head (per warp; summed where used); a slice
+  // whose data never arrived poisons its heads' sums
+  if (copy_failed) {
+#pragma unroll
+    for (int g = 0; g < GP; ++g) lsum[g] = __int_as_float(0x7fc00000);
+  }
   {
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
