@@ -443,13 +443,19 @@ def run_batched_decode(args):
 
     ms = timed(lambda: api.decode_attn(p, comp, q, out=o, workspace=dws))
     finite = bool(torch.isfinite(o).all())
-    # the same decode with the key-residual logits on the tensor cores first
-    os.environ["ANCHORKV_DECODE_KLOGIT"] = "1"
-    kws = torch.empty(api.decode_workspace_bytes(p, batch), dtype=torch.uint8, device=dev)
-    ok_ = torch.empty_like(o)
-    k_ms = timed(lambda: api.decode_attn(p, comp, q, out=ok_, workspace=kws))
-    del os.environ["ANCHORKV_DECODE_KLOGIT"]
-    k_diff = float((ok_ - o).abs().max())
+    # the same decode with the key-residual logits forced onto each path: the
+    # tensor-core pre-pass (the default from two slices per head down) and
+    # inside the decode
+    alt = {}
+    for flag, name in (("1", "prepass_key_logits"), ("0", "in_kernel_key_logits")):
+        os.environ["ANCHORKV_DECODE_KLOGIT"] = flag
+        kws = torch.empty(api.decode_workspace_bytes(p, batch), dtype=torch.uint8, device=dev)
+        ok_ = torch.empty_like(o)
+        k_ms = timed(lambda: api.decode_attn(p, comp, q, out=ok_, workspace=kws))
+        del os.environ["ANCHORKV_DECODE_KLOGIT"]
+        alt[f"decode_{name}_us_per_layer"] = k_ms * 1e3
+        alt[f"decode_{name}_gbs"] = nbytes / (k_ms * 1e-3) / 1e9
+        alt[f"decode_{name}_max_abs_diff"] = float((ok_ - o).abs().max())
     rope_ms = timed(lambda: api.decode_attn_rope(p, comp, q, 500000.0, out=o, workspace=rws))
     finite = finite and bool(torch.isfinite(o).all())
     peaks = _peaks()
@@ -461,9 +467,7 @@ def run_batched_decode(args):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm"], "traffic": None, "algorithmic_bytes": nbytes,
                          "peak_source": peaks["source"] + " (copy)"},
-            "decode_tc_key_logits_us_per_layer": k_ms * 1e3,
-            "decode_tc_key_logits_gbs": nbytes / (k_ms * 1e-3) / 1e9,
-            "decode_tc_key_logits_max_abs_diff": k_diff,
+            **alt,
             "decode_rope_us_per_layer": rope_ms * 1e3,
             "decode_rope_gbs": nbytes / (rope_ms * 1e-3) / 1e9,
             "l2": "layouts larger than L2" if flush is None else "L2 flushed before every repetition",
@@ -625,26 +629,29 @@ def run_config3(args, dev):
         del g
     except Exception:
         pass
-    # the same step with the key-residual logits on the tensor cores first
-    os.environ["ANCHORKV_DECODE_KLOGIT"] = "1"
-    kws = torch.empty(api.decode_workspace_bytes(params[0], batch), dtype=torch.uint8, device=dev)
-    ko = torch.empty_like(o)
-
-    def kstep():
-        for l in range(Lr):
-            api.decode_attn(params[l], comp[l], q[l], out=ko[l], workspace=kws)
-
-    kstep()
-    k_us = 1e3 * _event_ms(kstep, stream, max(3, args.steps))
-    del os.environ["ANCHORKV_DECODE_KLOGIT"]
-    k_diff = float((ko - o).abs().max())
+    # the same step with the key-residual logits forced onto each path: the
+    # tensor-core pre-pass (this shape's default) and inside the decode
     peaks = _peaks()
     step_bytes = Lr * batch * L["total_bytes"]
+    alt = {}
+    for flag, name in (("1", "prepass_key_logits"), ("0", "in_kernel_key_logits")):
+        os.environ["ANCHORKV_DECODE_KLOGIT"] = flag
+        kws = torch.empty(api.decode_workspace_bytes(params[0], batch), dtype=torch.uint8, device=dev)
+        ko = torch.empty_like(o)
+
+        def kstep():
+            for l in range(Lr):
+                api.decode_attn(params[l], comp[l], q[l], out=ko[l], workspace=kws)
+
+        kstep()
+        k_us = 1e3 * _event_ms(kstep, stream, max(3, args.steps))
+        alt[f"decode_{name}_us_per_step"] = k_us
+        alt[f"decode_{name}_hbm_frac"] = step_bytes / (k_us / 1e6) / 1e9 / peaks["hbm"]
+        alt[f"decode_{name}_max_abs_diff"] = float((ko - o).abs().max())
+        del os.environ["ANCHORKV_DECODE_KLOGIT"], kws, ko
     gbs = step_bytes / (us / 1e6) / 1e9
     return {"workload": "llama8b-n32k-bf16-batch16", "layers": Lr, "batch": batch, "theta": theta,
-            "decode_tc_key_logits_us_per_step": k_us,
-            "decode_tc_key_logits_hbm_frac": step_bytes / (k_us / 1e6) / 1e9 / peaks["hbm"],
-            "decode_tc_key_logits_max_abs_diff": k_diff,
+            **alt,
             "compressed_bytes_per_sequence_layer": L["total_bytes"],
             "decode_us_per_step": us, "decode_us_per_layer": us / Lr, "decode_graph_us_per_step": graph_us,
             "decode_hbm_gbs": gbs, "decode_hbm_frac": gbs / peaks["hbm"],
