@@ -84,7 +84,8 @@ struct FArgs {
   int S, tps, ct;                           // slices per (sequence, head), tiles per slice, tokens per chunk
   const float* rlg;                         // [B][R][GP] key-record logits from the pre-pass, or null
   float* part;                              // [B*H][S][GP*(2+128)] partial (max, sum, output)
-  int* tickets;                             // [B*H] zeroed before the launch when S > 1
+  int* tickets;                             // [B*H] zeroed by the anchor-logit pre-kernel when S > 1
+  float* Pw;                                // [B*H][kp][GP] anchor logits from the pre-kernel
 };
 
 // Shared-memory carve-up (bytes), the same on host and device.
@@ -213,30 +214,6 @@ __device__ __forceinline__ float sign_of(const FArgs& a, int d) {
   return ((a.sign_bits[d >> 5] >> (d & 31)) & 1u) ? -1.f : 1.f;
 }
 
-// Four consecutive elements of row `row` (lane's coordinates 4 lane ..) kept
-// raw until used; rows at or past `rows` read as zeros.
-template <typename T> struct RawRow;
-template <> struct RawRow<__nv_bfloat16> {
-  using type = uint2;
-  __device__ __forceinline__ static uint2 load(const __nv_bfloat16* base, int row, int rows, int lane) {
-    return row < rows ? *reinterpret_cast<const uint2*>(base + (int64_t)row * kD + 4 * lane) : make_uint2(0u, 0u);
-  }
-  __device__ __forceinline__ static void to_f(const uint2 v, float (&o)[4]) {
-    o[0] = __uint_as_float(v.x << 16); o[1] = __uint_as_float(v.x & 0xFFFF0000u);
-    o[2] = __uint_as_float(v.y << 16); o[3] = __uint_as_float(v.y & 0xFFFF0000u);
-  }
-};
-template <> struct RawRow<float> {
-  using type = float4;
-  __device__ __forceinline__ static float4 load(const float* base, int row, int rows, int lane) {
-    return row < rows ? *reinterpret_cast<const float4*>(base + (int64_t)row * kD + 4 * lane)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  __device__ __forceinline__ static void to_f(const float4 v, float (&o)[4]) {
-    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
-  }
-};
-
 // Eight consecutive elements (8 hl .. 8 hl + 7) of row `row` kept raw until
 // used; rows at or past `rows` read as zeros.
 template <typename T> struct Raw8;
@@ -290,6 +267,88 @@ __device__ __forceinline__ void transpose_reduce16(float (&v)[V], int lane) {
       n = hf;
     } else {
       v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- anchor logits
+
+constexpr int kPSlots = 64;   // slots per CTA of the anchor-logit pre-kernel
+
+// P = q . K_a (log2 units) of every slot, for each (sequence, head): CTA
+// (x, bh) takes slots [64 x, 64 x + 64), heads in passes of up to 8.  A
+// half-warp per slot, 8 coordinates per lane (the query's 8 x 8 values in
+// registers, one 16-byte row load), and a 16-lane transposed reduction of the
+// dot products.  Block x = 0 also clears the (sequence, head)'s merge ticket.
+// The decode is launched as a programmatic dependent of this kernel.
+template <typename T, int GP>
+__global__ void __launch_bounds__(kThreads) anchor_logit_kernel(FArgs a) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ __align__(16) float qs[GP * kD];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H, G = a.G, kp = a.kp;
+  if (blockIdx.x == 0 && tid == 0 && a.tickets) a.tickets[bh] = 0;
+  const int s0 = blockIdx.x * kPSlots, s1 = min(a.k, s0 + kPSlots);
+  const uint8_t* comp = a.comp + (int64_t)b * a.stride;
+  {
+    const T* q = reinterpret_cast<const T*>(a.q) + ((int64_t)b * a.H * G + (int64_t)h * G) * kD;
+    const float qscale = kLog2e * rsqrtf((float)kD);
+    for (int i = tid; i < GP * kD; i += kThreads) {
+      const int g = i / kD;
+      qs[i] = g < G ? to_f(q[(int64_t)g * kD + (i % kD)]) * qscale : 0.f;
+    }
+  }
+  __syncthreads();
+  float* Pw = a.Pw + (int64_t)bh * kp * GP;
+  constexpr int HG = GP < 8 ? GP : 8;
+#pragma unroll 1
+  for (int g0 = 0; g0 < GP; g0 += HG)
+  {
+    // half-warp per slot, 8 coordinates per lane: the query's 8 x GP values
+    // stay in registers, the row is one 16-byte load (bf16), and the GP dot
+    // products meet in a 16-lane transposed reduction
+    const int half = lane >> 4, hl = lane & 15;
+    float2 q2[HG][4];
+#pragma unroll
+    for (int g = 0; g < HG; ++g) {
+      const float4 a4 = *reinterpret_cast<const float4*>(qs + (g0 + g) * kD + 8 * hl);
+      const float4 b4 = *reinterpret_cast<const float4*>(qs + (g0 + g) * kD + 8 * hl + 4);
+      q2[g][0] = make_float2(a4.x, a4.y); q2[g][1] = make_float2(a4.z, a4.w);
+      q2[g][2] = make_float2(b4.x, b4.y); q2[g][3] = make_float2(b4.z, b4.w);
+    }
+    const T* Ka = reinterpret_cast<const T*>(comp + a.off_ak) + (int64_t)h * a.k * kD;
+    using R8 = Raw8<T>;
+    // four slot pairs per step, the next step's rows in flight meanwhile
+    constexpr int kPS = 4;
+    typename R8::type nx[kPS];
+    const int npair = (s1 - s0 + 1) / 2;
+    auto fetch = [&](int sp0) {
+#pragma unroll
+      for (int u = 0; u < kPS; ++u) nx[u] = R8::load(Ka, s0 + 2 * (sp0 + u * kWarps) + half, s1, hl);
+    };
+    if (warp < npair) fetch(warp);
+    for (int sp0 = warp; sp0 < npair; sp0 += kPS * kWarps) {
+      typename R8::type cx[kPS];
+#pragma unroll
+      for (int u = 0; u < kPS; ++u) cx[u] = nx[u];
+      if (sp0 + kPS * kWarps < npair) fetch(sp0 + kPS * kWarps);
+#pragma unroll
+      for (int u = 0; u < kPS; ++u) {
+        float2 x2[4];
+        R8::to_f2(cx[u], x2);
+        float v[HG];
+#pragma unroll
+        for (int g = 0; g < HG; ++g) {
+          float2 acc = __fmul2_rn(x2[0], q2[g][0]);
+          acc = __ffma2_rn(x2[1], q2[g][1], acc);
+          acc = __ffma2_rn(x2[2], q2[g][2], acc);
+          acc = __ffma2_rn(x2[3], q2[g][3], acc);
+          v[g] = acc.x + acc.y;
+        }
+        transpose_reduce16<HG>(v, lane);
+        const int slot = s0 + 2 * (sp0 + u * kWarps) + half;
+        if (slot < s1 && (hl % (16 / HG)) == 0) Pw[slot * GP + g0 + hl / (16 / HG)] = v[0];
+      }
     }
   }
 }
@@ -443,94 +502,15 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
 #pragma unroll
     for (int i = 0; i < 4; ++i) qr[g * kD + 4 * lane + i] = v[i];
   }
-  if constexpr (GP <= 8) {
-    // half-warp per slot, 8 coordinates per lane: the query's 8 x GP values
-    // stay in registers, the row is one 16-byte load (bf16), and the GP dot
-    // products meet in a 16-lane transposed reduction
-    const int half = lane >> 4, hl = lane & 15;
-    float2 q2[GP][4];
-#pragma unroll
-    for (int g = 0; g < GP; ++g) {
-      const float4 a4 = *reinterpret_cast<const float4*>(qs + g * kD + 8 * hl);
-      const float4 b4 = *reinterpret_cast<const float4*>(qs + g * kD + 8 * hl + 4);
-      q2[g][0] = make_float2(a4.x, a4.y); q2[g][1] = make_float2(a4.z, a4.w);
-      q2[g][2] = make_float2(b4.x, b4.y); q2[g][3] = make_float2(b4.z, b4.w);
-    }
-    const T* Ka = reinterpret_cast<const T*>(comp + a.off_ak) + (int64_t)h * a.k * kD;
-    using R8 = Raw8<T>;
-    // four slot pairs per step, the next step's rows in flight meanwhile
-    constexpr int kPS = 4;
-    typename R8::type nx[kPS];
-    const int npair = (a.k + 1) / 2;
-    auto fetch = [&](int sp0) {
-#pragma unroll
-      for (int u = 0; u < kPS; ++u) nx[u] = R8::load(Ka, 2 * (sp0 + u * kWarps) + half, a.k, hl);
-    };
-    if (warp < npair) fetch(warp);
-    for (int sp0 = warp; sp0 < npair; sp0 += kPS * kWarps) {
-      typename R8::type cx[kPS];
-#pragma unroll
-      for (int u = 0; u < kPS; ++u) cx[u] = nx[u];
-      if (sp0 + kPS * kWarps < npair) fetch(sp0 + kPS * kWarps);
-#pragma unroll
-      for (int u = 0; u < kPS; ++u) {
-        float2 x2[4];
-        R8::to_f2(cx[u], x2);
-        float v[GP];
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          float2 acc = __fmul2_rn(x2[0], q2[g][0]);
-          acc = __ffma2_rn(x2[1], q2[g][1], acc);
-          acc = __ffma2_rn(x2[2], q2[g][2], acc);
-          acc = __ffma2_rn(x2[3], q2[g][3], acc);
-          v[g] = acc.x + acc.y;
-        }
-        transpose_reduce16<GP>(v, lane);
-        const int slot = 2 * (sp0 + u * kWarps) + half;
-        if (slot < a.k && (hl % (16 / GP)) == 0) P[slot * GP + hl / (16 / GP)] = v[0];
-      }
-    }
-  } else   {
-    float4 q4[GP];
-#pragma unroll
-    for (int g = 0; g < GP; ++g) q4[g] = *reinterpret_cast<const float4*>(qs + g * kD + 4 * lane);
-    const T* Ka = reinterpret_cast<const T*>(comp + a.off_ak) + (int64_t)h * a.k * kD;
-    constexpr int SB = 32 / GP;
-    // the rows of the warp's next batch are loaded before this batch is
-    // reduced, so one L2 round trip overlaps the other's arithmetic
-    using Raw = typename RawRow<T>::type;
-    Raw nx[SB];
-    auto fetch = [&](int base2) {
-#pragma unroll
-      for (int i = 0; i < SB; ++i) nx[i] = RawRow<T>::load(Ka, base2 + i, a.k, lane);
-    };
-    // (with 16 or more slots per batch the batch's own loads are enough in flight)
-    constexpr bool kPipe = SB <= 8;
-    int base = warp * SB;
-    if (kPipe && base < a.k) fetch(base);
-    for (; base < a.k; base += kWarps * SB) {
-      Raw cx[SB];
-      if (kPipe) {
-#pragma unroll
-        for (int i = 0; i < SB; ++i) cx[i] = nx[i];
-        if (base + kWarps * SB < a.k) fetch(base + kWarps * SB);
-      } else {
-#pragma unroll
-        for (int i = 0; i < SB; ++i) cx[i] = RawRow<T>::load(Ka, base + i, a.k, lane);
-      }
-      float v[32];
-#pragma unroll
-      for (int i = 0; i < SB; ++i) {
-        float x[4];
-        RawRow<T>::to_f(cx[i], x);
-#pragma unroll
-        for (int g = 0; g < GP; ++g)
-          v[i * GP + g] = fmaf(q4[g].x, x[0], fmaf(q4[g].y, x[1], fmaf(q4[g].z, x[2], q4[g].w * x[3])));
-      }
-      transpose_reduce32(v, lane);
-      const int slot = base + lane / GP;
-      if (slot < a.k) P[slot * GP + (lane % GP)] = v[0];
-    }
+  // anchor logits P = q . K_a of this (sequence, head), computed by the
+  // pre-kernel that this launch depends on (programmatic dependent launch: the
+  // prologue above overlapped it); its writes, the cleared ticket included,
+  // are visible past this wait
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  {
+    const float* src = a.Pw + (int64_t)bh * kp * GP;
+    for (int u = tid; u < GP * kp / 4; u += kThreads) cp16(P + 4 * u, src + 4 * u, 16);
+    cp_commit();
   }
   for (int i = tid; i < GP * kp; i += kThreads) {
     Wt[i] = 0.f;
@@ -1233,6 +1213,7 @@ bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs, bool allow_pre
   fs->o_tickets = S > 1 ? take(4 * (int64_t)units) : 0;
   fs->o_part = S > 1 ? take(4 * (int64_t)units * S * part_words(GP)) : 0;
   fs->o_rlog = fs->klogit ? take(klogit_ws_bytes(pl, batch)) : 0;
+  fs->o_P = take(4 * (int64_t)units * ((pl.k + 3) & ~3) * GP);
   fs->ws_total = off;
   return true;
 }
@@ -1257,40 +1238,56 @@ int launch_flash_decode(const Plan& pl, const FlashShape& fs, int batch, const c
   a.rlg = fs.klogit ? reinterpret_cast<const float*>(ws + fs.o_rlog) : nullptr;
   a.part = fs.S > 1 ? reinterpret_cast<float*>(ws + fs.o_part) : nullptr;
   a.tickets = fs.S > 1 ? reinterpret_cast<int*>(ws + fs.o_tickets) : nullptr;
-  if (fs.S > 1 && cudaMemsetAsync(a.tickets, 0, 4 * (size_t)batch * pl.H, s) != cudaSuccess) return ANCHORKV_ECUDA;
+  a.Pw = reinterpret_cast<float*>(ws + fs.o_P);
+  stage_begin(kStDecodeCluster, s);
   if (fs.klogit) {
     const int st = launch_klogit_tc(pl, batch, comp, stride, q, reinterpret_cast<float*>(ws + fs.o_rlog), s);
     if (st) return st;
   }
   const dim3 grid(fs.S, batch * pl.H);
+  const dim3 pgrid((pl.k + kPSlots - 1) / kPSlots, batch * pl.H);
   const int GP = gp_of(pl.G);
   cudaError_t e = cudaSuccess;
-  auto go = [&](auto kernel, int n_ok) {
+  // the anchor-logit pre-kernel (it also clears the merge tickets), then the
+  // decode as its programmatic dependent: the decode's CTAs start once every
+  // pre-kernel CTA is running and wait for its results where they need them
+  auto go = [&](auto kernel, auto pkernel, int n_ok) {
     if (n_ok < 1) { e = cudaErrorNotSupported; return; }
-    kernel<<<grid, kThreads, fs.smem, s>>>(a);
+    pkernel<<<pgrid, kThreads, 0, s>>>(a);
     e = cudaGetLastError();
+    if (e != cudaSuccess) return;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = fs.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kernel, a);
   };
-  stage_begin(kStDecodeCluster, s);
   if (pl.p.dtype == ANCHORKV_BF16) {
     using T = __nv_bfloat16;
     switch (GP) {
-      case 1: go(flash_decode_kernel<T, 1>, max_ctas_per_sm<T, 1>(fs.smem)); break;
-      case 2: go(flash_decode_kernel<T, 2>, max_ctas_per_sm<T, 2>(fs.smem)); break;
-      case 4: go(flash_decode_kernel<T, 4>, max_ctas_per_sm<T, 4>(fs.smem)); break;
-      case 8: go(flash_decode_kernel<T, 8>, max_ctas_per_sm<T, 8>(fs.smem)); break;
-      default: go(flash_decode_kernel<T, 16>, max_ctas_per_sm<T, 16>(fs.smem)); break;
+      case 1: go(flash_decode_kernel<T, 1>, anchor_logit_kernel<T, 1>, max_ctas_per_sm<T, 1>(fs.smem)); break;
+      case 2: go(flash_decode_kernel<T, 2>, anchor_logit_kernel<T, 2>, max_ctas_per_sm<T, 2>(fs.smem)); break;
+      case 4: go(flash_decode_kernel<T, 4>, anchor_logit_kernel<T, 4>, max_ctas_per_sm<T, 4>(fs.smem)); break;
+      case 8: go(flash_decode_kernel<T, 8>, anchor_logit_kernel<T, 8>, max_ctas_per_sm<T, 8>(fs.smem)); break;
+      default: go(flash_decode_kernel<T, 16>, anchor_logit_kernel<T, 16>, max_ctas_per_sm<T, 16>(fs.smem)); break;
     }
   } else {
     using T = float;
     switch (GP) {
-      case 1: go(flash_decode_kernel<T, 1>, max_ctas_per_sm<T, 1>(fs.smem)); break;
-      case 2: go(flash_decode_kernel<T, 2>, max_ctas_per_sm<T, 2>(fs.smem)); break;
-      case 4: go(flash_decode_kernel<T, 4>, max_ctas_per_sm<T, 4>(fs.smem)); break;
-      case 8: go(flash_decode_kernel<T, 8>, max_ctas_per_sm<T, 8>(fs.smem)); break;
-      default: go(flash_decode_kernel<T, 16>, max_ctas_per_sm<T, 16>(fs.smem)); break;
+      case 1: go(flash_decode_kernel<T, 1>, anchor_logit_kernel<T, 1>, max_ctas_per_sm<T, 1>(fs.smem)); break;
+      case 2: go(flash_decode_kernel<T, 2>, anchor_logit_kernel<T, 2>, max_ctas_per_sm<T, 2>(fs.smem)); break;
+      case 4: go(flash_decode_kernel<T, 4>, anchor_logit_kernel<T, 4>, max_ctas_per_sm<T, 4>(fs.smem)); break;
+      case 8: go(flash_decode_kernel<T, 8>, anchor_logit_kernel<T, 8>, max_ctas_per_sm<T, 8>(fs.smem)); break;
+      default: go(flash_decode_kernel<T, 16>, anchor_logit_kernel<T, 16>, max_ctas_per_sm<T, 16>(fs.smem)); break;
     }
   }
-  stage_end(kStDecodeCluster, s, 1);
+  stage_end(kStDecodeCluster, s, fs.klogit ? 3 : 2);   // pre-pass, anchor logits, decode
   if (e == cudaErrorNotSupported) return ANCHORKV_EUNSUPPORTED;
   return e == cudaSuccess ? ANCHORKV_OK : ANCHORKV_ECUDA;
 }

@@ -61,7 +61,7 @@ void codebook(double* tau, double* l1, double* l2, double* mse);
 struct FlashShape {
   int ct, S, tps, smem;
   bool klogit;            // key-residual logits from the tensor-core pre-pass
-  int64_t ws_total, o_tickets, o_part, o_rlog;
+  int64_t ws_total, o_tickets, o_part, o_rlog, o_P;
 };
 // Tensor-core pre-pass of the slice decode: sigma~ <qr, lev(c)> of every key
 // record, [batch][R][GP] floats in the workspace.

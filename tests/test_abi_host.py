@@ -93,14 +93,15 @@ def test_workspace_view(monkeypatch):
     assert v["off_counters"] % 256 == 0 and v["off_pooled"] % 256 == 0
     # the slice decode needs tickets and slice partials only when a (sequence,
     # head) is cut into several slices: at batch 1 (8 heads on ~148 CTAs) it
-    # is, at batch 32 (256 heads) every head is one slice and needs nothing
-    # but the key-logit pre-pass's batch x R x G floats, which that shape
-    # turns on by default
+    # is, at batch 32 (256 heads) every head is one slice; every shape needs
+    # the anchor logits P (batch x H x k x G floats), and the key-logit
+    # pre-pass's batch x R x G floats when it runs (by default at batch 32)
     assert api.decode_workspace_bytes(p, 1) > 0
     R = api.anchorkv_bytes(p)["n_residuals"]
-    assert api.decode_workspace_bytes(p, 32) == (32 * R * 4 * 4 + 255) // 256 * 256
+    P32 = (32 * 8 * 288 * 4 * 4 + 255) // 256 * 256
+    assert api.decode_workspace_bytes(p, 32) == (32 * R * 4 * 4 + 255) // 256 * 256 + P32
     monkeypatch.setenv("ANCHORKV_DECODE_KLOGIT", "0")
-    assert api.decode_workspace_bytes(p, 32) == 0
+    assert api.decode_workspace_bytes(p, 32) == P32
     monkeypatch.setenv("ANCHORKV_DECODE_KLOGIT", "1")
     assert api.decode_workspace_bytes(p, 1) > (R * 4 * 4 + 255) // 256 * 256
     monkeypatch.delenv("ANCHORKV_DECODE_KLOGIT")
