@@ -86,18 +86,20 @@ struct FArgs {
   float* part;                              // [B*H][S][GP*(2+128)] partial (max, sum, output)
   int* tickets;                             // [B*H] zeroed by the anchor-logit pre-kernel when S > 1
   float* Pw;                                // [B*H][kp][GP] anchor logits from the pre-kernel
+  int rope;                                 // keys stored before the rotary map: rotate at decode
+  double inv_freq[kD / 2];                  // rotary frequencies base^(-2i/D)
 };
 
 // Shared-memory carve-up (bytes), the same on host and device.
 struct FPlan {
-  int qs, qr, P, W, Wi, lut, pfs, wpre, red, rlog, wz, stage, stage_bytes, total;
+  int qs, qr, P, W, Wi, lut, pfs, wpre, red, rlog, wz, rot, stage, stage_bytes, total;
   // offsets inside one stage
   int s_codes, s_sig, s_tok, s_bm;
 };
 
 __host__ __device__ inline int fa_align(int x, int a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline FPlan fplan(int GP, int kp, int ct, int tps) {
+__host__ __device__ inline FPlan fplan(int GP, int kp, int ct, int tps, bool rope) {
   FPlan f;
   int cur = 0;
   // persistent small arrays first; from P on, the region is reused at the
@@ -113,6 +115,9 @@ __host__ __device__ inline FPlan fplan(int GP, int kp, int ct, int tps) {
   f.Wi = cur; cur += 2 * GP * kp * 4;
   f.rlog = cur; cur = fa_align(cur + ct * GP * 4, 16);
   f.wz = cur; cur = fa_align(cur + ct * GP * 8, 16);
+  // rotary decode: (cos, sin) of b w_i (b < 32) and of the chunk's 32-token
+  // steps (T0 + 32 a) w_i, [32 + ct / 32][64] float2
+  f.rot = cur; cur += rope ? (32 + ct / 32) * (kD / 2) * 8 : 0;
   // stage: codes [2][ct][32], scales [2][ct + 8] (16-byte spans), token words
   // [2][ct + 4], bitmap words [2][ct / 32]
   int sc = 0;
@@ -162,6 +167,28 @@ __device__ __forceinline__ void copy_span(uint8_t* dst, const uint8_t* comp, int
     const int64_t left = total - o;
     if (left <= 0) continue;
     cp16(dst + 16 * u, comp + o, left >= 16 ? 16 : (int)left);
+  }
+}
+
+// (cos, sin) of pos * w with the angle reduced modulo 2 pi in fp64 first.
+__device__ __forceinline__ float2 rot_cs(double pos, double w) {
+  const double two_pi = 6.283185307179586476925286766559, inv_two_pi = 0.15915494309189533576888376337251;
+  const double ang = pos * w;
+  float sn, cs;
+  sincosf((float)(ang - two_pi * rint(ang * inv_two_pi)), &sn, &cs);
+  return make_float2(cs, sn);
+}
+
+// The rotary map at position pos on this lane's four coordinates (lane l:
+// 4l .. 4l + 3): coordinate d < D/2 pairs with d + D/2, held by lane l ^ 16,
+// and turns by pos * base^(-2 (d mod D/2) / D).
+__device__ __forceinline__ void rotate4(const FArgs& a, double pos, float (&x)[4], int lane) {
+  const bool upper = lane >= 16;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 c = rot_cs(pos, a.inv_freq[4 * (lane & 15) + e]);
+    const float other = __shfl_xor_sync(0xffffffffu, x[e], 16);
+    x[e] = upper ? fmaf(other, c.y, x[e] * c.x) : fmaf(-other, c.y, x[e] * c.x);
   }
 }
 
@@ -288,6 +315,7 @@ __global__ void __launch_bounds__(kThreads) anchor_logit_kernel(FArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H, G = a.G, kp = a.kp;
   if (blockIdx.x == 0 && tid == 0 && a.tickets) a.tickets[bh] = 0;
+  if (a.rope) return;            // the rotary decode has no per-slot logits
   const int s0 = blockIdx.x * kPSlots, s1 = min(a.k, s0 + kPSlots);
   const uint8_t* comp = a.comp + (int64_t)b * a.stride;
   {
@@ -355,13 +383,13 @@ __global__ void __launch_bounds__(kThreads) anchor_logit_kernel(FArgs a) {
 
 // ---------------------------------------------------------------- the kernel
 
-template <typename T, int GP>
+template <typename T, int GP, bool ROPE>
 __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel(FArgs a) {
   extern __shared__ __align__(16) uint8_t sm[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H, s = blockIdx.x;
   const int G = a.G, kp = a.kp, ct = a.ct;
-  const FPlan F = fplan(GP, kp, ct, a.tps);
+  const FPlan F = fplan(GP, kp, ct, a.tps, ROPE);
   float* qs = reinterpret_cast<float*>(sm + F.qs);       // [GP][128] q' (log2 units)
   float* qr = reinterpret_cast<float*>(sm + F.qr);       // [GP][128] rotated q'
   float* P = reinterpret_cast<float*>(sm + F.P);         // [GP][kp]
@@ -486,8 +514,23 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
   issue_records(0);
   cp_commit();
 
-  // ---- 2. rotated query and anchor logits P (while the copies fly)
-  for (int g = warp; g < GP; g += kWarps) {
+  // ---- 2. rotated query and anchor logits P (while the copies fly); the
+  //    rotary decode instead turns the query to its position N + tail_len
+  //    and tabulates (cos, sin)(b w_i) for b < 32
+  if constexpr (ROPE) {
+    for (int g = warp; g < GP; g += kWarps) {
+      float v[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = qs[g * kD + 4 * lane + i];
+      rotate4(a, (double)a.N + a.tail_len, v, lane);
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 4; ++i) qs[g * kD + 4 * lane + i] = v[i];
+    }
+    float2* tb = reinterpret_cast<float2*>(sm + F.rot);
+    for (int i = tid; i < 32 * (kD / 2); i += kThreads) tb[i] = rot_cs((double)(i / (kD / 2)), a.inv_freq[i % (kD / 2)]);
+  }
+  for (int g = warp; g < GP && !ROPE; g += kWarps) {
     float v[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) v[i] = qs[g * kD + 4 * lane + i];
@@ -507,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
   // prologue above overlapped it); its writes, the cleared ticket included,
   // are visible past this wait
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  {
+  if (!ROPE) {
     const float* src = a.Pw + (int64_t)bh * kp * GP;
     for (int u = tid; u < GP * kp / 4; u += kThreads) cp16(P + 4 * u, src + 4 * u, 16);
     cp_commit();
@@ -682,7 +725,13 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
     const float* klg = a.rlg ? reinterpret_cast<const float*>(codes) +
                                    (int)((((int64_t)b * a.R + rbase[0]) * GP * 4) & 15) / 4
                              : rlog;
-    if (!a.rlg) {
+    if constexpr (ROPE) {
+      // (cos, sin) of the chunk's 32-token steps (T0 + 32 a) w_i
+      float2* ta = reinterpret_cast<float2*>(sm + F.rot) + 32 * (kD / 2);
+      for (int i = tid; i < (ct / 32) * (kD / 2); i += kThreads)
+        ta[i] = rot_cs((double)tok0 + 32.0 * (i / (kD / 2)), a.inv_freq[i % (kD / 2)]);
+    }
+    if (!ROPE && !a.rlg) {
       constexpr int RB = 32 / GP;
       const int nK = nrec[0];
       for (int base = warp * RB; base < nK; base += kWarps * RB) {
@@ -707,6 +756,88 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
     }
     __syncthreads();
 
+    if constexpr (ROPE) {
+      // b'. rotary logits: every key rebuilt as gamma~ K_a + r~ (the residual
+      //     through one warp Hadamard transform), turned to its position by
+      //     the tabulated angles, dotted with the turned query; 32 / G tokens
+      //     per warp step (their anchor rows loaded eight at a time), the
+      //     products finished by one transposed reduction, into rlog
+      constexpr int TB = 32 / GP;
+      constexpr int TL = TB < 8 ? TB : 8;
+      const T* Ka = reinterpret_cast<const T*>(comp + a.off_ak) + (int64_t)h * a.k * kD;
+      const float2* tbl = reinterpret_cast<const float2*>(sm + F.rot);
+      const float2* tal = tbl + 32 * (kD / 2);
+      const int fi = 4 * (lane & 15);
+      const bool upper = lane >= 16;
+      float4 q4[GP];
+#pragma unroll
+      for (int g = 0; g < GP; ++g) q4[g] = *reinterpret_cast<const float4*>(qs + g * kD + 4 * lane);
+      const float rs = rsqrtf((float)kD);
+      for (int base = warp * TB; base < ntok; base += kWarps * TB) {
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+#pragma unroll
+        for (int i0 = 0; i0 < TB; i0 += TL) {
+          float xr[TL][4];
+          float gam[TL];
+          int rk[TL];
+#pragma unroll
+          for (int u = 0; u < TL; ++u) {
+            const int t = base + i0 + u;
+            gam[u] = 0.f;
+            rk[u] = -1;
+            if (t < ntok) {
+              const uint32_t wk = tok0p[sh_tok[0] + t];
+              const int slot = min((int)(wk & 0xFFFFu), a.k - 1);
+              gam[u] = half_bits_to_f(wk >> 16);
+              const uint32_t word = bm0[t >> 5];
+              const int rank = wpre[t >> 5] + __popc(word & ((1u << (t & 31)) - 1u));
+              if (((word >> (t & 31)) & 1u) && rank < nrec[0]) rk[u] = rank;
+              load4(Ka + (int64_t)slot * kD + 4 * lane, xr[u]);
+            } else {
+              xr[u][0] = xr[u][1] = xr[u][2] = xr[u][3] = 0.f;
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < TL; ++u) {
+            const int t = base + i0 + u;
+            if (t >= ntok) continue;                        // warp-uniform
+            float k4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) k4[e] = gam[u] * xr[u][e];
+            if (rk[u] >= 0) {                               // warp-uniform
+              const uint32_t cb = codes[rk[u] * kCodeBytes + lane];
+              const float sg = half_bits_to_f(sig0[sh_sig[0] + rk[u]]);
+              const float2 l01 = lutc[(cb & 15u) * 16], l23 = lutc[(cb >> 4) * 16];
+              float y[4] = {l01.x * sg, l01.y * sg, l23.x * sg, l23.y * sg};
+              if (!a.naive) {
+                fwht128(y);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) y[e] *= sign_of(a, 4 * lane + e) * rs;
+              }
+#pragma unroll
+              for (int e = 0; e < 4; ++e) k4[e] += y[e];
+            }
+            // turn by position tok0 + t: angle (T0 + 32 (t >> 5)) w + (t & 31) w
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 A = tal[(t >> 5) * (kD / 2) + fi + e], B = tbl[(t & 31) * (kD / 2) + fi + e];
+              const float c = fmaf(A.x, B.x, -A.y * B.y), sn = fmaf(A.x, B.y, A.y * B.x);
+              const float other = __shfl_xor_sync(0xffffffffu, k4[e], 16);
+              k4[e] = upper ? fmaf(other, sn, k4[e] * c) : fmaf(-other, sn, k4[e] * c);
+            }
+#pragma unroll
+            for (int g = 0; g < GP; ++g)
+              v[(i0 + u) * GP + g] = fmaf(q4[g].x, k4[0], fmaf(q4[g].y, k4[1], fmaf(q4[g].z, k4[2], q4[g].w * k4[3])));
+          }
+        }
+        transpose_reduce32(v, lane);
+        const int t = base + lane / GP;
+        if (lane < TB * GP && t < ntok) rlog[t * GP + (lane % GP)] = v[0];
+      }
+      __syncthreads();
+    }
     // b. every token's logit for the G heads (anchor term + its record's
     //    residual term), kept in registers; the value side's slot and coefficient
     float lg[kKT][GP];
@@ -728,21 +859,29 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
         slv[i] = min((int)(wv & 0xFFFFu), a.k - 1);
         gmv[i] = half_bits_to_f(wv >> 16);
         gabs = fmaxf(gabs, fabsf(gmv[i]));
-        const uint32_t wk = tok0p[sh_tok[0] + t];
-        const int slot = min((int)(wk & 0xFFFFu), a.k - 1);
-        const float gam = half_bits_to_f(wk >> 16);
-        const uint32_t word = bm0[t >> 5];
-        const uint32_t below = word & ((1u << (t & 31)) - 1u);
-        const int rank = wpre[t >> 5] + __popc(below);
-        const bool res = ((word >> (t & 31)) & 1u) && rank < nrec[0];
-        float pv[GP];
-        load_slot<GP>(P + slot * GP, pv);
+        if constexpr (ROPE) {
 #pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          float x = gam * pv[g];
-          if (res) x += klg[rank * GP + g];
-          lg[i][g] = x;
-          cmx[g] = fmaxf(cmx[g], x);
+          for (int g = 0; g < GP; ++g) {
+            lg[i][g] = rlog[t * GP + g];
+            cmx[g] = fmaxf(cmx[g], lg[i][g]);
+          }
+        } else {
+          const uint32_t wk = tok0p[sh_tok[0] + t];
+          const int slot = min((int)(wk & 0xFFFFu), a.k - 1);
+          const float gam = half_bits_to_f(wk >> 16);
+          const uint32_t word = bm0[t >> 5];
+          const uint32_t below = word & ((1u << (t & 31)) - 1u);
+          const int rank = wpre[t >> 5] + __popc(below);
+          const bool res = ((word >> (t & 31)) & 1u) && rank < nrec[0];
+          float pv[GP];
+          load_slot<GP>(P + slot * GP, pv);
+#pragma unroll
+          for (int g = 0; g < GP; ++g) {
+            float x = gam * pv[g];
+            if (res) x += klg[rank * GP + g];
+            lg[i][g] = x;
+            cmx[g] = fmaxf(cmx[g], x);
+          }
         }
       }
     }
@@ -859,6 +998,10 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
             } else {
               x[i][0] = x[i][1] = x[i][2] = x[i][3] = 0.f;
             }
+          }
+          if constexpr (ROPE) {
+#pragma unroll
+            for (int i = 0; i < TB; ++i) rotate4(a, (double)a.N + t0 + base + i, x[i], lane);
           }
           float v[32];
 #pragma unroll
@@ -1140,7 +1283,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
 // Resident CTAs per SM at `smem` bytes of dynamic shared memory (0: none).
 // The kernel's dynamic shared-memory limit is raised once to the largest a
 // CTA may use, so every later shape launches without touching it.
-template <typename T, int GP>
+template <typename T, int GP, bool ROPE>
 int max_ctas_per_sm(int smem) {
   static std::mutex mu;
   static int cache_smem[8] = {0}, cache_n[8] = {0}, n_cache = 0;
@@ -1153,9 +1296,9 @@ int max_ctas_per_sm(int smem) {
     int optin = 0;
     cudaFuncAttributes fa;
     if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
-        cudaFuncGetAttributes(&fa, flash_decode_kernel<T, GP>) != cudaSuccess)
+        cudaFuncGetAttributes(&fa, flash_decode_kernel<T, GP, ROPE>) != cudaSuccess)
       return 0;
-    if (cudaFuncSetAttribute(flash_decode_kernel<T, GP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(flash_decode_kernel<T, GP, ROPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              optin - (int)fa.sharedSizeBytes) != cudaSuccess)
       return 0;
     dev_set = dev;
@@ -1164,7 +1307,7 @@ int max_ctas_per_sm(int smem) {
   for (int i = 0; i < n_cache; ++i)
     if (cache_smem[i] == smem) return cache_n[i];
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, flash_decode_kernel<T, GP>, kThreads, smem) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, flash_decode_kernel<T, GP, ROPE>, kThreads, smem) != cudaSuccess)
     n = 0;
   if (n_cache < 8) { cache_smem[n_cache] = smem; cache_n[n_cache] = n; ++n_cache; }
   return n;
@@ -1175,7 +1318,7 @@ int max_ctas_per_sm(int smem) {
 // Shape of the slice decode for `batch` sequences: tokens per chunk, slices
 // per (sequence, head) and the workspace.  Returns false when no chunk size
 // fits the shared memory (the split-token kernels take over).
-bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs, bool allow_prepass) {
+bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs, bool allow_prepass, bool rope) {
   const int GP = gp_of(pl.G);
   const int kp = (pl.k + 3) & ~3;
   // CTAs resident per SM: two when the registers allow it (G <= 4) and the
@@ -1188,7 +1331,7 @@ bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs, bool allow_pre
   fs->ct = 0;
   for (; per_sm >= 1 && !fs->ct; --per_sm)
     for (int ct : kChunkSizes) {
-      const int need = fplan(GP, kp, ct, pl.n_tiles).total;
+      const int need = fplan(GP, kp, ct, pl.n_tiles, rope).total;
       if (need <= kSmemBudget && (need + 1024) * per_sm <= 228 * 1024) { fs->ct = ct; break; }
     }
   if (!fs->ct) return false;
@@ -1200,13 +1343,13 @@ bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs, bool allow_pre
   S = (pl.n_tiles + tps - 1) / tps;
   fs->S = S;
   fs->tps = tps;
-  fs->smem = fplan(GP, kp, fs->ct, tps).total;
+  fs->smem = fplan(GP, kp, fs->ct, tps, rope).total;
   // key-residual logits on the tensor cores ahead of the decode: worth it
   // when the launch is throughput-bound (two slices per head or fewer, i.e.
   // many sequences), not when a few heads are cut into many slices and
   // latency rules; ANCHORKV_DECODE_KLOGIT=0/1 forces it either way
   const char* kenv = getenv("ANCHORKV_DECODE_KLOGIT");
-  fs->klogit = allow_prepass && klogit_tc_supported(pl) && pl.R > 0 &&
+  fs->klogit = allow_prepass && !rope && klogit_tc_supported(pl) && pl.R > 0 &&
                (kenv && kenv[0] ? kenv[0] == '1' : S <= 2);
   int64_t off = 0;
   auto take = [&](int64_t bytes) { int64_t o = off; off += (bytes + 255) / 256 * 256; return o; };
@@ -1220,8 +1363,10 @@ bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs, bool allow_pre
 
 int launch_flash_decode(const Plan& pl, const FlashShape& fs, int batch, const char* comp, int64_t stride,
                         const void* q, const void* Kt, const void* Vt, int tail_len, int tail_cap, float* out,
-                        char* ws, cudaStream_t s) {
+                        char* ws, cudaStream_t s, double rope_base) {
   FArgs a;
+  a.rope = rope_base > 0.0;
+  for (int i = 0; i < kD / 2; ++i) a.inv_freq[i] = a.rope ? pow(rope_base, -2.0 * i / kD) : 0.0;
   a.comp = reinterpret_cast<const uint8_t*>(comp);
   a.stride = stride;
   a.total = pl.L.total_bytes;
@@ -1268,25 +1413,28 @@ int launch_flash_decode(const Plan& pl, const FlashShape& fs, int batch, const c
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kernel, a);
   };
-  if (pl.p.dtype == ANCHORKV_BF16) {
-    using T = __nv_bfloat16;
-    switch (GP) {
-      case 1: go(flash_decode_kernel<T, 1>, anchor_logit_kernel<T, 1>, max_ctas_per_sm<T, 1>(fs.smem)); break;
-      case 2: go(flash_decode_kernel<T, 2>, anchor_logit_kernel<T, 2>, max_ctas_per_sm<T, 2>(fs.smem)); break;
-      case 4: go(flash_decode_kernel<T, 4>, anchor_logit_kernel<T, 4>, max_ctas_per_sm<T, 4>(fs.smem)); break;
-      case 8: go(flash_decode_kernel<T, 8>, anchor_logit_kernel<T, 8>, max_ctas_per_sm<T, 8>(fs.smem)); break;
-      default: go(flash_decode_kernel<T, 16>, anchor_logit_kernel<T, 16>, max_ctas_per_sm<T, 16>(fs.smem)); break;
+  auto pick = [&](auto tag) {
+    using T = decltype(tag);
+    if (a.rope) {
+      switch (GP) {
+        case 1: go(flash_decode_kernel<T, 1, true>, anchor_logit_kernel<T, 1>, max_ctas_per_sm<T, 1, true>(fs.smem)); break;
+        case 2: go(flash_decode_kernel<T, 2, true>, anchor_logit_kernel<T, 2>, max_ctas_per_sm<T, 2, true>(fs.smem)); break;
+        case 4: go(flash_decode_kernel<T, 4, true>, anchor_logit_kernel<T, 4>, max_ctas_per_sm<T, 4, true>(fs.smem)); break;
+        case 8: go(flash_decode_kernel<T, 8, true>, anchor_logit_kernel<T, 8>, max_ctas_per_sm<T, 8, true>(fs.smem)); break;
+        default: e = cudaErrorNotSupported; break;
+      }
+      return;
     }
-  } else {
-    using T = float;
     switch (GP) {
-      case 1: go(flash_decode_kernel<T, 1>, anchor_logit_kernel<T, 1>, max_ctas_per_sm<T, 1>(fs.smem)); break;
-      case 2: go(flash_decode_kernel<T, 2>, anchor_logit_kernel<T, 2>, max_ctas_per_sm<T, 2>(fs.smem)); break;
-      case 4: go(flash_decode_kernel<T, 4>, anchor_logit_kernel<T, 4>, max_ctas_per_sm<T, 4>(fs.smem)); break;
-      case 8: go(flash_decode_kernel<T, 8>, anchor_logit_kernel<T, 8>, max_ctas_per_sm<T, 8>(fs.smem)); break;
-      default: go(flash_decode_kernel<T, 16>, anchor_logit_kernel<T, 16>, max_ctas_per_sm<T, 16>(fs.smem)); break;
+      case 1: go(flash_decode_kernel<T, 1, false>, anchor_logit_kernel<T, 1>, max_ctas_per_sm<T, 1, false>(fs.smem)); break;
+      case 2: go(flash_decode_kernel<T, 2, false>, anchor_logit_kernel<T, 2>, max_ctas_per_sm<T, 2, false>(fs.smem)); break;
+      case 4: go(flash_decode_kernel<T, 4, false>, anchor_logit_kernel<T, 4>, max_ctas_per_sm<T, 4, false>(fs.smem)); break;
+      case 8: go(flash_decode_kernel<T, 8, false>, anchor_logit_kernel<T, 8>, max_ctas_per_sm<T, 8, false>(fs.smem)); break;
+      default: go(flash_decode_kernel<T, 16, false>, anchor_logit_kernel<T, 16>, max_ctas_per_sm<T, 16, false>(fs.smem)); break;
     }
-  }
+  };
+  if (pl.p.dtype == ANCHORKV_BF16) pick(__nv_bfloat16{});
+  else pick(0.f);
   stage_end(kStDecodeCluster, s, fs.klogit ? 3 : 2);   // pre-pass, anchor logits, decode
   if (e == cudaErrorNotSupported) return ANCHORKV_EUNSUPPORTED;
   return e == cudaSuccess ? ANCHORKV_OK : ANCHORKV_ECUDA;
@@ -1296,14 +1444,14 @@ int flash_ctas_per_sm(const Plan& pl, const FlashShape& fs) {
   const int GP = gp_of(pl.G);
   if (pl.p.dtype == ANCHORKV_BF16) {
     using T = __nv_bfloat16;
-    return GP == 1 ? max_ctas_per_sm<T, 1>(fs.smem) : GP == 2 ? max_ctas_per_sm<T, 2>(fs.smem)
-         : GP == 4 ? max_ctas_per_sm<T, 4>(fs.smem) : GP == 8 ? max_ctas_per_sm<T, 8>(fs.smem)
-         : max_ctas_per_sm<T, 16>(fs.smem);
+    return GP == 1 ? max_ctas_per_sm<T, 1, false>(fs.smem) : GP == 2 ? max_ctas_per_sm<T, 2, false>(fs.smem)
+         : GP == 4 ? max_ctas_per_sm<T, 4, false>(fs.smem) : GP == 8 ? max_ctas_per_sm<T, 8, false>(fs.smem)
+         : max_ctas_per_sm<T, 16, false>(fs.smem);
   }
   using T = float;
-  return GP == 1 ? max_ctas_per_sm<T, 1>(fs.smem) : GP == 2 ? max_ctas_per_sm<T, 2>(fs.smem)
-       : GP == 4 ? max_ctas_per_sm<T, 4>(fs.smem) : GP == 8 ? max_ctas_per_sm<T, 8>(fs.smem)
-       : max_ctas_per_sm<T, 16>(fs.smem);
+  return GP == 1 ? max_ctas_per_sm<T, 1, false>(fs.smem) : GP == 2 ? max_ctas_per_sm<T, 2, false>(fs.smem)
+       : GP == 4 ? max_ctas_per_sm<T, 4, false>(fs.smem) : GP == 8 ? max_ctas_per_sm<T, 8, false>(fs.smem)
+       : max_ctas_per_sm<T, 16, false>(fs.smem);
 }
 
 }  // namespace akv

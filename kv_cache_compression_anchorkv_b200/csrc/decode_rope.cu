@@ -382,6 +382,12 @@ __global__ void __launch_bounds__(128) rope_combine_kernel(RopeArgs a, float* __
 // (sequence, head) pairs, at least 256 cached tokens per split.
 RopePlan make_rope_plan(const Plan& pl, int batch) {
   RopePlan rp;
+  rp.flash = pl.G <= 8 && flash_decode_plan(pl, batch, &rp.fs, false, true);
+  if (rp.flash) {
+    rp.n_split = 0;
+    rp.ws_total = rp.fs.ws_total;
+    return rp;
+  }
   const int bh = std::max(1, batch * pl.H);
   const int want = std::max(1, (2 * 148 + bh - 1) / bh);
   rp.n_split = std::max(1, std::min(want, (pl.N + 255) / 256));
@@ -392,6 +398,11 @@ RopePlan make_rope_plan(const Plan& pl, int batch) {
 cudaError_t launch_decode_rope(const Plan& pl, const RopePlan& rp, const char* comp, int64_t stride, int batch,
                                const void* q, const void* Kt, const void* Vt, int tail_len, int tail_cap,
                                double rope_base, float* out, char* ws, cudaStream_t s) {
+  if (rp.flash) {
+    const int st = launch_flash_decode(pl, rp.fs, batch, comp, stride, q, Kt, Vt, tail_len, tail_cap, out, ws, s,
+                                       rope_base);
+    return st == ANCHORKV_OK ? cudaSuccess : st == ANCHORKV_EUNSUPPORTED ? cudaErrorNotSupported : cudaErrorUnknown;
+  }
   RopeArgs a;
   a.comp = reinterpret_cast<const uint8_t*>(comp);
   a.stride = stride;

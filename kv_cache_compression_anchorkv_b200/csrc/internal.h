@@ -80,10 +80,11 @@ struct DecodePlan {
 int make_decode_plan(const Plan& pl, int batch, DecodePlan* out, bool allow_prepass = true);
 // Shape checks of a decode call (shared-memory limits of the chosen path).
 int check_decode_shape(const Plan& pl, const DecodePlan& dp, int tail_len);
-bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs, bool allow_prepass = true);
+// rope: the rotary decode (keys stored before the rotary map), G <= 8
+bool flash_decode_plan(const Plan& pl, int batch, FlashShape* fs, bool allow_prepass = true, bool rope = false);
 int launch_flash_decode(const Plan& pl, const FlashShape& fs, int batch, const char* comp, int64_t stride,
                         const void* q, const void* Kt, const void* Vt, int tail_len, int tail_cap, float* out,
-                        char* ws, cudaStream_t s);
+                        char* ws, cudaStream_t s, double rope_base = 0.0);
 int flash_ctas_per_sm(const Plan& pl, const FlashShape& fs);
 
 // Kernel launchers (one per hot-path step), all asynchronous on `s`.
@@ -104,6 +105,8 @@ cudaError_t launch_key_queries(const Plan& pl, const void* K, void* Q, cudaStrea
 
 // Decode attention with rotary positions (keys stored before the rotary map).
 struct RopePlan {
+  bool flash;             // the slice decode with its rotary phase (G <= 8); else the split-token kernels
+  FlashShape fs;
   int n_split;
   int64_t ws_total;
 };
