@@ -527,8 +527,13 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
 #pragma unroll
       for (int i = 0; i < 4; ++i) qs[g * kD + 4 * lane + i] = v[i];
     }
+    // rows of 64 entries ordered [e][l16] for frequency 4 l16 + e: a warp's
+    // lookups for one e are 16 consecutive float2 (no bank conflicts)
     float2* tb = reinterpret_cast<float2*>(sm + F.rot);
-    for (int i = tid; i < 32 * (kD / 2); i += kThreads) tb[i] = rot_cs((double)(i / (kD / 2)), a.inv_freq[i % (kD / 2)]);
+    for (int i = tid; i < 32 * (kD / 2); i += kThreads) {
+      const int r = i % (kD / 2);
+      tb[i] = rot_cs((double)(i / (kD / 2)), a.inv_freq[4 * (r % 16) + r / 16]);
+    }
   }
   for (int g = warp; g < GP && !ROPE; g += kWarps) {
     float v[4];
@@ -728,8 +733,10 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
     if constexpr (ROPE) {
       // (cos, sin) of the chunk's 32-token steps (T0 + 32 a) w_i
       float2* ta = reinterpret_cast<float2*>(sm + F.rot) + 32 * (kD / 2);
-      for (int i = tid; i < (ct / 32) * (kD / 2); i += kThreads)
-        ta[i] = rot_cs((double)tok0 + 32.0 * (i / (kD / 2)), a.inv_freq[i % (kD / 2)]);
+      for (int i = tid; i < (ct / 32) * (kD / 2); i += kThreads) {
+        const int r = i % (kD / 2);
+        ta[i] = rot_cs((double)tok0 + 32.0 * (i / (kD / 2)), a.inv_freq[4 * (r % 16) + r / 16]);
+      }
     }
     if (!ROPE && !a.rlg) {
       constexpr int RB = 32 / GP;
@@ -767,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
       const T* Ka = reinterpret_cast<const T*>(comp + a.off_ak) + (int64_t)h * a.k * kD;
       const float2* tbl = reinterpret_cast<const float2*>(sm + F.rot);
       const float2* tal = tbl + 32 * (kD / 2);
-      const int fi = 4 * (lane & 15);
+      const int l16 = lane & 15;
       const bool upper = lane >= 16;
       float4 q4[GP];
 #pragma unroll
@@ -822,7 +829,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
             // turn by position tok0 + t: angle (T0 + 32 (t >> 5)) w + (t & 31) w
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float2 A = tal[(t >> 5) * (kD / 2) + fi + e], B = tbl[(t & 31) * (kD / 2) + fi + e];
+              const float2 A = tal[(t >> 5) * (kD / 2) + e * 16 + l16], B = tbl[(t & 31) * (kD / 2) + e * 16 + l16];
               const float c = fmaf(A.x, B.x, -A.y * B.y), sn = fmaf(A.x, B.y, A.y * B.x);
               const float other = __shfl_xor_sync(0xffffffffu, k4[e], 16);
               k4[e] = upper ? fmaf(other, sn, k4[e] * c) : fmaf(-other, sn, k4[e] * c);
