@@ -158,6 +158,52 @@ def test_decode_tensor_core_key_logits(name, batch, tail, mode, klogit, monkeypa
     print(name, "tensor-core key logits", batch, tail, "max abs err", err)
 
 
+@pytest.mark.parametrize("name,batch,tail,klogit", [("bf16-ragged-n3000", 1, 5, "0"), ("bf16-gqa8-n2500", 3, 0, "1"),
+                                                    ("bf16-n20000", 1, 64, "0")])
+def test_decode_replayed_in_a_cuda_graph(name, batch, tail, klogit, monkeypatch):
+    """A decode captured in a CUDA graph (the anchor-logit pre-kernel, the
+    decode launched as its programmatic dependent, and the pre-pass when on)
+    and replayed gives the eager call's output bit for bit, replay after
+    replay; the rotary decode likewise."""
+    monkeypatch.setenv("ANCHORKV_DECODE_KLOGIT", klogit)
+    spec, theta = CASES[name]
+    p = _params(spec, theta)
+    L = api.anchorkv_bytes(p)
+    stride = (L["total_bytes"] + 255) // 256 * 256
+    comp = torch.zeros(batch, stride, dtype=torch.uint8, device="cuda")
+    for b in range(batch):
+        sb = CacheSpec(**{**spec.__dict__, "seed": spec.seed + 100 * b})
+        K, V, Q = make_layer(sb, 0)
+        out, _ = api.compress(p, K.cuda(), V.cuda(), Q.cuda())
+        comp[b, :L["total_bytes"]] = out
+    q = make_decode_queries(spec, 0, step=0, batch=batch).cuda()
+    Kt, Vt = (x.cuda() for x in make_tail(spec, 0, max(tail, 1) + 3, batch=batch))
+    ws = torch.empty(api.decode_workspace_bytes(p, batch), dtype=torch.uint8, device="cuda")
+    rws = torch.empty(api.decode_rope_workspace_bytes(p, batch), dtype=torch.uint8, device="cuda")
+    eager = api.decode_attn(p, comp, q, Kt, Vt, tail_len=tail, workspace=ws).clone()
+    eager_r = api.decode_attn_rope(p, comp, q, 500000.0, Kt, Vt, tail_len=tail, workspace=rws).clone()
+    o = torch.empty_like(eager)
+    orr = torch.empty_like(eager_r)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):          # warm the launch path on the capture stream
+        api.decode_attn(p, comp, q, Kt, Vt, tail_len=tail, out=o, workspace=ws)
+        api.decode_attn_rope(p, comp, q, 500000.0, Kt, Vt, tail_len=tail, out=orr, workspace=rws)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        api.decode_attn(p, comp, q, Kt, Vt, tail_len=tail, out=o, workspace=ws)
+        api.decode_attn_rope(p, comp, q, 500000.0, Kt, Vt, tail_len=tail, out=orr, workspace=rws)
+    for _ in range(3):
+        o.zero_()
+        orr.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(o, eager)
+        assert torch.equal(orr, eager_r)
+    del g
+
+
 def test_decode_config():
     spec, theta = CASES["bf16-n20000"]
     cfg = api.decode_config(_params(spec, theta), 1)
