@@ -282,7 +282,8 @@ __global__ void __launch_bounds__(256) obs_rows_kernel(const __nv_bfloat16* __re
 // ============================================================== pass B
 
 struct CtlB {
-  uint64_t q_full, x_full[2], x_empty[2], s_full[2], s_empty[2], al_full, al_empty, y_full, drain;
+  uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], s_empty[2], al_full, al_empty, y_full,
+      drain;
   uint32_t tmem_base;
   int err;
 };
@@ -302,7 +303,12 @@ obs_b_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
   const Item it = item_of(a);
   if (threadIdx.x == 0) {
     tc::mbar_init(&ctl.q_full, 1);
-    for (int s = 0; s < S; ++s) { tc::mbar_init(&ctl.x_full[s], 1); tc::mbar_init(&ctl.x_empty[s], 1); }
+    // a K stage is free once its S MMA is done and the epilogue has read the
+    // tile's norms (kEpi arrivals + the MMA's commit); a V stage once its Y MMA is
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(&ctl.k_full[s], 1); tc::mbar_init(&ctl.k_empty[s], kEpi + 1);
+      tc::mbar_init(&ctl.v_full[s], 1); tc::mbar_init(&ctl.v_empty[s], 1);
+    }
     for (int b = 0; b < 2; ++b) { tc::mbar_init(&ctl.s_full[b], 1); tc::mbar_init(&ctl.s_empty[b], kEpi); }
     tc::mbar_init(&ctl.al_full, kEpi);
     tc::mbar_init(&ctl.al_empty, 1);
@@ -328,17 +334,30 @@ obs_b_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
     if (lane == 0) {
       tc::mbar_expect_tx(&ctl.q_full, kOp);
       load_op(q, &mapQ, it.h * a.GW + it.rb * 128, &ctl.q_full);
-      int issued = 0;
-      for (int i = 0; i < it.n && !ctl.err; ++i) {
-        const int s = i % S, use = i / S;
-        if (use > 0 && !tc::wait_or_fail(&ctl.x_empty[s], (use - 1) & 1, &ctl.err, a.counters, kDevErrTimeout)) break;
-        tc::mbar_expect_tx(&ctl.x_full[s], 2 * kOp);
-        const int row = it.h * a.N + (it.tile0 + i) * 128;
-        load_op(xs + 2 * s * kOp, &mapK, row, &ctl.x_full[s]);
-        load_op(xs + 2 * s * kOp + kOp, &mapV, row, &ctl.x_full[s]);
-        ++issued;
+      // K and V in separate rings, K one tile ahead: tile i + 1's K goes out
+      // before tile i's V, so the S MMA of the next tile never waits behind
+      // the Y MMA of the current one
+      int kissued = 0, vissued = 0;
+      for (int i = 0; i <= it.n && !ctl.err; ++i) {
+        if (i < it.n) {
+          const int s = i % S, use = i / S;
+          if (use > 0 && !tc::wait_or_fail(&ctl.k_empty[s], (use - 1) & 1, &ctl.err, a.counters, kDevErrTimeout))
+            break;
+          tc::mbar_expect_tx(&ctl.k_full[s], kOp);
+          load_op(xs + 2 * s * kOp, &mapK, it.h * a.N + (it.tile0 + i) * 128, &ctl.k_full[s]);
+          ++kissued;
+        }
+        if (i >= 1) {
+          const int j = i - 1, s = j % S, use = j / S;
+          if (use > 0 && !tc::wait_or_fail(&ctl.v_empty[s], (use - 1) & 1, &ctl.err, a.counters, kDevErrTimeout))
+            break;
+          tc::mbar_expect_tx(&ctl.v_full[s], kOp);
+          load_op(xs + 2 * s * kOp + kOp, &mapV, it.h * a.N + (it.tile0 + j) * 128, &ctl.v_full[s]);
+          ++vissued;
+        }
       }
-      for (int s = 0; s < S && s < issued; ++s) tc::mbar_wait(&ctl.x_full[s], ((issued - 1 - s) / S) & 1);
+      for (int s = 0; s < S && s < kissued; ++s) tc::mbar_wait(&ctl.k_full[s], ((kissued - 1 - s) / S) & 1);
+      for (int s = 0; s < S && s < vissued; ++s) tc::mbar_wait(&ctl.v_full[s], ((vissued - 1 - s) / S) & 1);
       tc::mbar_wait(&ctl.q_full, 0);
     }
   } else if (warp == 1) {
@@ -348,19 +367,21 @@ obs_b_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
       bool ok = tc::wait_or_fail(&ctl.q_full, 0, &ctl.err, a.counters, kDevErrTimeout);
       auto mma1 = [&](int i) -> bool {
         const int s = i % S, use = i / S, b = i & 1, ub = i >> 1;
-        if (!tc::wait_or_fail(&ctl.x_full[s], use & 1, &ctl.err, a.counters, kDevErrTimeout)) return false;
+        if (!tc::wait_or_fail(&ctl.k_full[s], use & 1, &ctl.err, a.counters, kDevErrTimeout)) return false;
         if (ub > 0 && !tc::wait_or_fail(&ctl.s_empty[b], (ub - 1) & 1, &ctl.err, a.counters, kDevErrTimeout))
           return false;
         tc::fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) tc::mma_bf16(tmem + b * 128, kdesc(xs + 2 * s * kOp, kk), kdesc(q, kk), id1, kk > 0);
         tc::mma_commit(&ctl.s_full[b]);
+        tc::mma_commit(&ctl.k_empty[s]);      // with the epilogue's arrivals, frees the K stage
         return true;
       };
       if (ok && it.n > 0) ok = mma1(0);
       for (int i = 0; ok && i < it.n; ++i) {
         if (i + 1 < it.n && !mma1(i + 1)) break;
         if (!tc::wait_or_fail(&ctl.al_full, i & 1, &ctl.err, a.counters, kDevErrTimeout)) break;
+        if (!tc::wait_or_fail(&ctl.v_full[i % S], (i / S) & 1, &ctl.err, a.counters, kDevErrTimeout)) break;
         tc::fence_after_sync();
         const uint32_t vaddr = tc::smem_u32(xs + 2 * (i % S) * kOp + kOp);
         const uint32_t hi = tc::smem_u32(al), lo = tc::smem_u32(al + kOp);
@@ -371,7 +392,7 @@ obs_b_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
           tc::mma_bf16(tmem + ycol, da, tc::sw128_mn_desc(lo + kk * 2048, kHalf), id2, 1u);
         }
         tc::mma_commit(&ctl.al_empty);
-        tc::mma_commit(&ctl.x_empty[i % S]);
+        tc::mma_commit(&ctl.v_empty[i % S]);
       }
       tc::mma_commit(&ctl.y_full);
       tc::mma_commit(&ctl.drain);
@@ -415,11 +436,18 @@ obs_b_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
         aa1 = __ffma2_rn(al1, al1, aa1);
       }
       if (it.rb == 0) {
+        // the K tile has landed (its S MMA is done); the V side's norm
+        // threads wait for the V tile
+        if (nside == 1 && !tc::wait_or_fail(&ctl.v_full[s], (i / S) & 1, &ctl.err, a.counters, kDevErrTimeout)) {
+          ok = false;
+          break;
+        }
         float ss = half_sumsq(xs + (2 * s + nside) * kOp, nrow, npart);
         ss += __shfl_xor_sync(0xffffffffu, ss, 1);
         const int tn = (it.tile0 + i) * 128 + nrow;
         if (npart == 0 && tn < a.N) a.xnorm[((int64_t)nside * a.H + it.h) * a.N + tn] = sqrtf(ss);
       }
+      tc::mbar_arrive(&ctl.k_empty[s]);      // this thread is done with the K tile
       if (i > 0 && !tc::wait_or_fail(&ctl.al_empty, (i - 1) & 1, &ctl.err, a.counters, kDevErrTimeout)) {
         ok = false;
         break;
