@@ -40,6 +40,7 @@ namespace {
 // exact bf16/fp32 products are exact or within fp64 rounding, so the
 // cancellation leaves an error near 1e-12 ||x||^2.
 constexpr int kProjTokens = 64;
+constexpr int kProjTPQ = 2;      // tokens per quad of lanes (kProjTPQ x kProjTokens per block)
 
 template <typename T>
 __device__ __forceinline__ void load16(const T* p, float (&o)[16 / sizeof(T)]);
@@ -71,73 +72,102 @@ project_kernel(const T* __restrict__ K, const T* __restrict__ V, const T* __rest
   constexpr int EPV = 16 / (int)sizeof(T);        // elements per 16-byte load
   constexpr int STEPS = kD / (4 * EPV);           // loads per lane and row
   const int q = threadIdx.x & 3;
-  const int t = blockIdx.x * kProjTokens + (threadIdx.x >> 2), h = blockIdx.y, side = blockIdx.z;
-  const bool valid = t < N;
-  const int tt = valid ? t : N - 1;               // every lane takes part in the shuffles
-  const int64_t f = ((int64_t)side * H + h) * N + tt;
-  const uint32_t slot = min(tok[f] & 0xFFFFu, (uint32_t)(k - 1));
-  const T* x = (side ? V : K) + ((int64_t)h * N + tt) * kD;
-  const T* a = (side ? anc_v : anc_k) + ((int64_t)h * k + slot) * kD;
+  const int h = blockIdx.y, side = blockIdx.z;
+  // each quad takes kProjTPQ tokens kProjTokens apart, all their loads in
+  // flight together (record words, then rows and token-only values)
+  int tq[kProjTPQ], ttq[kProjTPQ];
+  int64_t fq[kProjTPQ];
+  uint32_t tw[kProjTPQ];
+#pragma unroll
+  for (int u = 0; u < kProjTPQ; ++u) {
+    tq[u] = (blockIdx.x * kProjTPQ + u) * kProjTokens + (threadIdx.x >> 2);
+    ttq[u] = tq[u] < N ? tq[u] : N - 1;           // every lane takes part in the shuffles
+    fq[u] = ((int64_t)side * H + h) * N + ttq[u];
+    tw[u] = tok[fq[u]];
+  }
   // Loads that depend only on the token go out with the row loads: the
   // anchor flag, the anchor's squared norm, and (utility ranking) lane q's observation-row-block
   // partial q, for the first npre of the obs_rb partials.
-  const bool is_anchor = slot_of[(int64_t)h * N + tt] >= 0;
-  const double n2 = anc_n2[((int64_t)side * H + h) * k + slot];
-  const float* src = side ? a2s : kus;
   static_assert(kObsGroups <= 4, "one partial per lane of the quad");
   const int npre = min(obs_rb, kObsGroups);
-  const float part = (kUtility && q < npre) ? src[((int64_t)q * H + h) * N + tt] : 0.0f;
-  double dot = 0.0, nx = 0.0;
+  const float* src = side ? a2s : kus;
+  uint32_t slotq[kProjTPQ];
+  bool anc[kProjTPQ];
+  double n2q[kProjTPQ], dotq[kProjTPQ], nxq[kProjTPQ];
+  float partq[kProjTPQ];
 #pragma unroll
-  for (int i = 0; i < STEPS; ++i) {
-    const int d = (4 * i + q) * EPV;
-    float xf[EPV], af[EPV];
-    load16<T>(x + d, xf);
-    load16<T>(a + d, af);
+  for (int u = 0; u < kProjTPQ; ++u) {
+    slotq[u] = min(tw[u] & 0xFFFFu, (uint32_t)(k - 1));
+    anc[u] = slot_of[(int64_t)h * N + ttq[u]] >= 0;
+    n2q[u] = anc_n2[((int64_t)side * H + h) * k + slotq[u]];
+    partq[u] = (kUtility && q < npre) ? src[((int64_t)q * H + h) * N + ttq[u]] : 0.0f;
+    dotq[u] = 0.0;
+    nxq[u] = 0.0;
+  }
 #pragma unroll
-    for (int e = 0; e < EPV; ++e) {
-      dot = fma((double)xf[e], (double)af[e], dot);
-      nx = fma((double)xf[e], (double)xf[e], nx);
+  for (int u = 0; u < kProjTPQ; ++u) {
+    const T* x = (side ? V : K) + ((int64_t)h * N + ttq[u]) * kD;
+    const T* a = (side ? anc_v : anc_k) + ((int64_t)h * k + slotq[u]) * kD;
+#pragma unroll
+    for (int i = 0; i < STEPS; ++i) {
+      const int d = (4 * i + q) * EPV;
+      float xf[EPV], af[EPV];
+      load16<T>(x + d, xf);
+      load16<T>(a + d, af);
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) {
+        dotq[u] = fma((double)xf[e], (double)af[e], dotq[u]);
+        nxq[u] = fma((double)xf[e], (double)xf[e], nxq[u]);
+      }
     }
   }
-  dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-  nx += __shfl_xor_sync(0xffffffffu, nx, 1);
-  dot += __shfl_xor_sync(0xffffffffu, dot, 2);
-  nx += __shfl_xor_sync(0xffffffffu, nx, 2);
-  // partials 0 .. npre-1 to the quad's lane 0, summed in row-block order
   const int l0 = threadIdx.x & 31 & ~3;
-  float m = __shfl_sync(0xffffffffu, part, l0);
-  for (int rb = 1; rb < npre; ++rb) m += __shfl_sync(0xffffffffu, part, l0 + rb);
-  if (!valid || q != 0) return;
-  double gamma = (n2 > 0.0) ? dot / n2 : 0.0;
-  if (is_anchor) gamma = 1.0;
-  const uint16_t gb = half_bits_rn(gamma);
-  const double g = (double)half_bits_to_f(gb);
-  const double r2 = fmax(0.0, nx - 2.0 * g * dot + g * g * n2);
-  tok[f] = slot | ((uint32_t)gb << 16);
-  float u;
-  if (is_anchor) {
-    u = -1.0f;
-  } else if (kUtility) {
-    // sum of the observation-row-block partials, in order
-    for (int rb = npre; rb < obs_rb; ++rb) m += src[((int64_t)rb * H + h) * N + t];
-    u = side ? (float)(r2 * (double)m) : (float)(r2 / (double)(kD * kD) * (double)m);
-  } else if (rank == ANCHORKV_RANK_RESIDUAL_NORM) {
-    u = (float)r2;
-  } else if (rank == ANCHORKV_RANK_ATTENTION) {
-    // sum over the observation rows of alpha (row-block partials, in order)
-    float sa = score[(int64_t)h * N + t];
-    for (int rb = 1; rb < obs_rb; ++rb) sa += score[((int64_t)rb * H + h) * N + t];
-    u = sa;
-  } else if (rank == ANCHORKV_RANK_COSINE) {
-    const double den = sqrt(nx * n2);
-    u = (float)(1.0 - (den > 0.0 ? dot / den : 0.0));
-  } else {
-    // a seeded uniform value of the flat index: the top 24 bits of SplitMix64
-    const uint64_t z = splitmix64(seed ^ kRankSalt ^ ((uint64_t)(layer & 0x7FFF) << 48) ^ (uint64_t)f);
-    u = (float)(z >> 40) * (1.0f / 16777216.0f);
+#pragma unroll
+  for (int u = 0; u < kProjTPQ; ++u) {
+    double dot = dotq[u], nx = nxq[u];
+    dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+    nx += __shfl_xor_sync(0xffffffffu, nx, 1);
+    dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+    nx += __shfl_xor_sync(0xffffffffu, nx, 2);
+    // partials 0 .. npre-1 to the quad's lane 0, summed in row-block order
+    float m = __shfl_sync(0xffffffffu, partq[u], l0);
+    for (int rb = 1; rb < npre; ++rb) m += __shfl_sync(0xffffffffu, partq[u], l0 + rb);
+    const int t = tq[u];
+    if (t >= N || q != 0) continue;
+    const int64_t f = fq[u];
+    const uint32_t slot = slotq[u];
+    const double n2 = n2q[u];
+    const bool is_anchor = anc[u];
+    double gamma = (n2 > 0.0) ? dot / n2 : 0.0;
+    if (is_anchor) gamma = 1.0;
+    const uint16_t gb = half_bits_rn(gamma);
+    const double g = (double)half_bits_to_f(gb);
+    const double r2 = fmax(0.0, nx - 2.0 * g * dot + g * g * n2);
+    tok[f] = slot | ((uint32_t)gb << 16);
+    float uval;
+    if (is_anchor) {
+      uval = -1.0f;
+    } else if (kUtility) {
+      // sum of the observation-row-block partials, in order
+      for (int rb = npre; rb < obs_rb; ++rb) m += src[((int64_t)rb * H + h) * N + t];
+      uval = side ? (float)(r2 * (double)m) : (float)(r2 / (double)(kD * kD) * (double)m);
+    } else if (rank == ANCHORKV_RANK_RESIDUAL_NORM) {
+      uval = (float)r2;
+    } else if (rank == ANCHORKV_RANK_ATTENTION) {
+      // sum over the observation rows of alpha (row-block partials, in order)
+      float sa = score[(int64_t)h * N + t];
+      for (int rb = 1; rb < obs_rb; ++rb) sa += score[((int64_t)rb * H + h) * N + t];
+      uval = sa;
+    } else if (rank == ANCHORKV_RANK_COSINE) {
+      const double den = sqrt(nx * n2);
+      uval = (float)(1.0 - (den > 0.0 ? dot / den : 0.0));
+    } else {
+      // a seeded uniform value of the flat index: the top 24 bits of SplitMix64
+      const uint64_t z = splitmix64(seed ^ kRankSalt ^ ((uint64_t)(layer & 0x7FFF) << 48) ^ (uint64_t)f);
+      uval = (float)(z >> 40) * (1.0f / 16777216.0f);
+    }
+    util[f] = uval;
   }
-  util[f] = u;
 }
 
 // ---------------------------------------------------------------- key-as-query proxies
@@ -355,7 +385,7 @@ CodecConst make_cc(const Plan& pl) {
 }  // namespace
 
 cudaError_t launch_project(const Plan& pl, const void* K, const void* V, char* out, char* ws, cudaStream_t s) {
-  const dim3 blocks((pl.N + kProjTokens - 1) / kProjTokens, pl.H, 2);
+  const dim3 blocks((pl.N + kProjTokens * kProjTPQ - 1) / (kProjTokens * kProjTPQ), pl.H, 2);
   auto* n2 = reinterpret_cast<const double*>(ws + pl.o_anc_n2);
   auto* slot_of = reinterpret_cast<const int*>(ws + pl.o_slot_of);
   auto* a2 = reinterpret_cast<const float*>(ws + pl.o_a2);
