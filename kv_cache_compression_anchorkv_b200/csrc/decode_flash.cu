@@ -92,7 +92,7 @@ struct FArgs {
 
 // Shared-memory carve-up (bytes), the same on host and device.
 struct FPlan {
-  int qs, qr, P, W, Wi, lut, pfs, wpre, red, rlog, wz, rot, stage, stage_bytes, total;
+  int qs, qr, P, W, Wi, lut, pfs, wpre, red, rlog, wz, rot, rtok, stage, stage_bytes, total;
   // offsets inside one stage
   int s_codes, s_sig, s_tok, s_bm;
 };
@@ -116,8 +116,10 @@ __host__ __device__ inline FPlan fplan(int GP, int kp, int ct, int tps, bool rop
   f.rlog = cur; cur = fa_align(cur + ct * GP * 4, 16);
   f.wz = cur; cur = fa_align(cur + ct * GP * 8, 16);
   // rotary decode: (cos, sin) of b w_i (b < 32) and of the chunk's 32-token
-  // steps (T0 + 32 a) w_i, [32 + ct / 32][64] float2
+  // blocks (T0 + 32 a) w_i, [32 + ct / 32][64] float2; the token of each
+  // key record of the chunk, [ct] int
   f.rot = cur; cur += rope ? (32 + ct / 32) * (kD / 2) * 8 : 0;
+  f.rtok = cur; cur += rope ? ct * 4 : 0;
   // stage: codes [2][ct][32], scales [2][ct + 8] (16-byte spans), token words
   // [2][ct + 4], bitmap words [2][ct / 32]
   int sc = 0;
@@ -189,6 +191,85 @@ __device__ __forceinline__ void rotate4(const FArgs& a, double pos, float (&x)[4
     const float2 c = rot_cs(pos, a.inv_freq[4 * (lane & 15) + e]);
     const float other = __shfl_xor_sync(0xffffffffu, x[e], 16);
     x[e] = upper ? fmaf(other, c.y, x[e] * c.x) : fmaf(-other, c.y, x[e] * c.x);
+  }
+}
+
+// Frequency of entry i of a rotary table row ([2][16] words of two (cos,
+// sin) pairs: word (j, l) holds frequencies 4 l + 2 j and 4 l + 2 j + 1).
+__device__ __forceinline__ int rot_freq(int i) {
+  const int w = (i % (kD / 2)) >> 1;
+  return 4 * (w & 15) + 2 * (w >> 4) + (i & 1);
+}
+
+// Coordinates 4 l + e and 64 + 4 l + e (e < 4) of one row, kept raw until used.
+template <typename T> struct Row8;
+template <> struct Row8<__nv_bfloat16> {
+  uint2 lo, hi;
+  __device__ __forceinline__ void load(const __nv_bfloat16* row) {
+    lo = *reinterpret_cast<const uint2*>(row);
+    hi = *reinterpret_cast<const uint2*>(row + kD / 2);
+  }
+  __device__ __forceinline__ void to_f(float (&x)[8]) const {
+    x[0] = __uint_as_float(lo.x << 16); x[1] = __uint_as_float(lo.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(lo.y << 16); x[3] = __uint_as_float(lo.y & 0xFFFF0000u);
+    x[4] = __uint_as_float(hi.x << 16); x[5] = __uint_as_float(hi.x & 0xFFFF0000u);
+    x[6] = __uint_as_float(hi.y << 16); x[7] = __uint_as_float(hi.y & 0xFFFF0000u);
+  }
+};
+template <> struct Row8<float> {
+  float4 lo, hi;
+  __device__ __forceinline__ void load(const float* row) {
+    lo = *reinterpret_cast<const float4*>(row);
+    hi = *reinterpret_cast<const float4*>(row + kD / 2);
+  }
+  __device__ __forceinline__ void to_f(float (&x)[8]) const {
+    x[0] = lo.x; x[1] = lo.y; x[2] = lo.z; x[3] = lo.w;
+    x[4] = hi.x; x[5] = hi.y; x[6] = hi.z; x[7] = hi.w;
+  }
+};
+
+// Turns the pairs (x[e], x[4 + e]) of a half-warp row by the angles of one
+// table row (lane l16's two words) and returns the G dot products with the
+// turned query qa (coordinates in the same order) into v[g].
+template <int GP>
+__device__ __forceinline__ void turn_dot(const float (&x)[8], const float4 c01, const float4 c23,
+                                         const float2 (&qa)[GP][4], float* v) {
+  const float cb[4] = {c01.x, c01.z, c23.x, c23.z}, sb[4] = {c01.y, c01.w, c23.y, c23.w};
+  float xr[4], yr[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    xr[e] = fmaf(x[e], cb[e], -x[4 + e] * sb[e]);
+    yr[e] = fmaf(x[4 + e], cb[e], x[e] * sb[e]);
+  }
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    float2 d = __fmul2_rn(make_float2(xr[0], xr[1]), qa[g][0]);
+    d = __ffma2_rn(make_float2(xr[2], xr[3]), qa[g][1], d);
+    d = __ffma2_rn(make_float2(yr[0], yr[1]), qa[g][2], d);
+    d = __ffma2_rn(make_float2(yr[2], yr[3]), qa[g][3], d);
+    v[g] = d.x + d.y;
+  }
+}
+
+// Unnormalised Walsh-Hadamard transform of a 128-vector spread over a
+// half-warp: lane l (of 16) holds coordinates 4 l + e in x[e] and
+// 64 + 4 l + e in x[4 + e] (e < 4).  Coordinate bits 0, 1 and 6 are register
+// bits, bits 2 .. 5 the lane bits; both halves of the warp must call it.
+__device__ __forceinline__ void fwht128_half(float (&x)[8], int lane) {
+#pragma unroll
+  for (int m = 1; m < 8; m <<= 1)
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (!(e & m)) {
+        const float u = x[e], v = x[e | m];
+        x[e] = u + v;
+        x[e | m] = u - v;
+      }
+#pragma unroll
+  for (int m = 1; m < 16; m <<= 1) {
+    const float sg = (lane & m) ? -1.f : 1.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = fmaf(x[e], sg, __shfl_xor_sync(0xffffffffu, x[e], m));
   }
 }
 
@@ -527,13 +608,11 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
 #pragma unroll
       for (int i = 0; i < 4; ++i) qs[g * kD + 4 * lane + i] = v[i];
     }
-    // rows of 64 entries ordered [e][l16] for frequency 4 l16 + e: a warp's
-    // lookups for one e are 16 consecutive float2 (no bank conflicts)
+    // rows of 64 entries as [2][16] 16-byte words: word (j, l16) holds the
+    // pairs of frequencies 4 l16 + 2 j and 4 l16 + 2 j + 1, so a half-warp's
+    // read of one word per lane is 256 contiguous bytes
     float2* tb = reinterpret_cast<float2*>(sm + F.rot);
-    for (int i = tid; i < 32 * (kD / 2); i += kThreads) {
-      const int r = i % (kD / 2);
-      tb[i] = rot_cs((double)(i / (kD / 2)), a.inv_freq[4 * (r % 16) + r / 16]);
-    }
+    for (int i = tid; i < 32 * (kD / 2); i += kThreads) tb[i] = rot_cs((double)(i / (kD / 2)), a.inv_freq[rot_freq(i)]);
   }
   for (int g = warp; g < GP && !ROPE; g += kWarps) {
     float v[4];
@@ -724,19 +803,26 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
       }
       if (lane < ct / 32) wpre[side * (ct / 32 + 1) + lane + 1] = x;
       if (lane == 0) wpre[side * (ct / 32 + 1)] = 0;
+      if (ROPE && side == 0) {
+        // the token of every key record (rank), for the rotary residual pass
+        int* rtok = reinterpret_cast<int*>(sm + F.rtok);
+        int r = x - __popc(w);
+        for (uint32_t m = w; m != 0u && r < nrec[0]; m &= m - 1u, ++r) rtok[r] = 32 * lane + __ffs(m) - 1;
+      }
     }
     // key-record logits by rank: staged from the tensor-core pre-pass (sigma~
     // included), or computed here into rlog
-    const float* klg = a.rlg ? reinterpret_cast<const float*>(codes) +
+    // (the rotary decode keeps its residual terms by rank in the wz buffer,
+    // free until step d)
+    const float* klg = ROPE ? reinterpret_cast<const float*>(sm + F.wz)
+                     : a.rlg ? reinterpret_cast<const float*>(codes) +
                                    (int)((((int64_t)b * a.R + rbase[0]) * GP * 4) & 15) / 4
                              : rlog;
     if constexpr (ROPE) {
-      // (cos, sin) of the chunk's 32-token steps (T0 + 32 a) w_i
+      // (cos, sin) of the chunk's 32-token blocks (T0 + 32 a) w_i
       float2* ta = reinterpret_cast<float2*>(sm + F.rot) + 32 * (kD / 2);
-      for (int i = tid; i < (ct / 32) * (kD / 2); i += kThreads) {
-        const int r = i % (kD / 2);
-        ta[i] = rot_cs((double)tok0 + 32.0 * (i / (kD / 2)), a.inv_freq[4 * (r % 16) + r / 16]);
-      }
+      for (int i = tid; i < (ct / 32) * (kD / 2); i += kThreads)
+        ta[i] = rot_cs((double)tok0 + 32.0 * (i / (kD / 2)), a.inv_freq[rot_freq(i)]);
     }
     if (!ROPE && !a.rlg) {
       constexpr int RB = 32 / GP;
@@ -764,84 +850,119 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
     __syncthreads();
 
     if constexpr (ROPE) {
-      // b'. rotary logits: every key rebuilt as gamma~ K_a + r~ (the residual
-      //     through one warp Hadamard transform), turned to its position by
-      //     the tabulated angles, dotted with the turned query; 32 / G tokens
-      //     per warp step (their anchor rows loaded eight at a time), the
-      //     products finished by one transposed reduction, into rlog
-      constexpr int TB = 32 / GP;
-      constexpr int TL = TB < 8 ? TB : 8;
-      const T* Ka = reinterpret_cast<const T*>(comp + a.off_ak) + (int64_t)h * a.k * kD;
-      const float2* tbl = reinterpret_cast<const float2*>(sm + F.rot);
-      const float2* tal = tbl + 32 * (kD / 2);
-      const int l16 = lane & 15;
-      const bool upper = lane >= 16;
-      float4 q4[GP];
+      // b'. rotary logits, on half-warps whose lane l16 holds coordinates
+      //     4 l16 + e and 64 + 4 l16 + e (e < 4), so that each rotary pair
+      //     (d, d + 64) sits in one lane.  Each warp takes 32-token blocks; the
+      //     query (at its own position) is turned back once by the block's
+      //     start T0 + 32 blk, and every key of the block is then turned only
+      //     by its offset b = t mod 32 (one table row):
+      //     - anchor terms: gamma~ times the dot product with the token's
+      //       anchor row goes to rlog by token (the rows of the next TL
+      //       tokens are in flight while TL tokens are worked on);
+      //     - residual terms of the block's key records: the residual is
+      //       rebuilt by one half-warp Hadamard transform; sigma~ times its
+      //       dot product goes to klg by rank.
+      //     16 / G tokens (records) per half-warp step, the 16 G products
+      //     finished by one transposed reduction.
+      constexpr int TBH = 16 / GP;
+      constexpr int TL0 = sizeof(T) == 2 ? 4 : 2;
+      constexpr int TL = TBH < TL0 ? TBH : TL0;   // rows per load batch
+      constexpr int BPS = TBH / TL;               // load batches per step
+      constexpr int NS = 16 / TBH;                // steps per 32-token block
+      const int half = lane >> 4, l16 = lane & 15;
+      const T* Ka = reinterpret_cast<const T*>(comp + a.off_ak) + (int64_t)h * a.k * kD + 4 * l16;
+      const float4* tbB = reinterpret_cast<const float4*>(sm + F.rot) + l16;   // [32][2][16]
+      const float4* tbA = tbB + 32 * 32;                                       // [ct / 32][2][16]
+      const int nK = nrec[0];
+      const int* rtok = reinterpret_cast<const int*>(sm + F.rtok);
+      float* rres = reinterpret_cast<float*>(sm + F.wz);
+      // the shared signs and 1 / sqrt(D) of the inverse rotation
+      float sg[8];
+      {
+        const float rs = rsqrtf((float)kD);
 #pragma unroll
-      for (int g = 0; g < GP; ++g) q4[g] = *reinterpret_cast<const float4*>(qs + g * kD + 4 * lane);
-      const float rs = rsqrtf((float)kD);
-      for (int base = warp * TB; base < ntok; base += kWarps * TB) {
-        float v[32];
+        for (int e = 0; e < 4; ++e) {
+          sg[e] = a.naive ? 1.f : sign_of(a, 4 * l16 + e) * rs;
+          sg[4 + e] = a.naive ? 1.f : sign_of(a, kD / 2 + 4 * l16 + e) * rs;
+        }
+      }
+      for (int blk = warp; blk * 32 < ntok; blk += kWarps) {
+        float2 qa[GP][4];
+        {
+          const float4 c01 = tbA[blk * 32], c23 = tbA[blk * 32 + 16];
+          const float ca[4] = {c01.x, c01.z, c23.x, c23.z}, sa[4] = {c01.y, c01.w, c23.y, c23.w};
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = 0.f;
-#pragma unroll
-        for (int i0 = 0; i0 < TB; i0 += TL) {
-          float xr[TL][4];
-          float gam[TL];
-          int rk[TL];
-#pragma unroll
-          for (int u = 0; u < TL; ++u) {
-            const int t = base + i0 + u;
-            gam[u] = 0.f;
-            rk[u] = -1;
-            if (t < ntok) {
-              const uint32_t wk = tok0p[sh_tok[0] + t];
-              const int slot = min((int)(wk & 0xFFFFu), a.k - 1);
-              gam[u] = half_bits_to_f(wk >> 16);
-              const uint32_t word = bm0[t >> 5];
-              const int rank = wpre[t >> 5] + __popc(word & ((1u << (t & 31)) - 1u));
-              if (((word >> (t & 31)) & 1u) && rank < nrec[0]) rk[u] = rank;
-              load4(Ka + (int64_t)slot * kD + 4 * lane, xr[u]);
-            } else {
-              xr[u][0] = xr[u][1] = xr[u][2] = xr[u][3] = 0.f;
-            }
-          }
-#pragma unroll
-          for (int u = 0; u < TL; ++u) {
-            const int t = base + i0 + u;
-            if (t >= ntok) continue;                        // warp-uniform
-            float k4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) k4[e] = gam[u] * xr[u][e];
-            if (rk[u] >= 0) {                               // warp-uniform
-              const uint32_t cb = codes[rk[u] * kCodeBytes + lane];
-              const float sg = half_bits_to_f(sig0[sh_sig[0] + rk[u]]);
-              const float2 l01 = lutc[(cb & 15u) * 16], l23 = lutc[(cb >> 4) * 16];
-              float y[4] = {l01.x * sg, l01.y * sg, l23.x * sg, l23.y * sg};
-              if (!a.naive) {
-                fwht128(y);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) y[e] *= sign_of(a, 4 * lane + e) * rs;
-              }
-#pragma unroll
-              for (int e = 0; e < 4; ++e) k4[e] += y[e];
-            }
-            // turn by position tok0 + t: angle (T0 + 32 (t >> 5)) w + (t & 31) w
+          for (int g = 0; g < GP; ++g) {
+            const float4 x4 = *reinterpret_cast<const float4*>(qs + g * kD + 4 * l16);
+            const float4 y4 = *reinterpret_cast<const float4*>(qs + g * kD + kD / 2 + 4 * l16);
+            const float xs[4] = {x4.x, x4.y, x4.z, x4.w}, ys[4] = {y4.x, y4.y, y4.z, y4.w};
+            float xq[4], yq[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float2 A = tal[(t >> 5) * (kD / 2) + e * 16 + l16], B = tbl[(t & 31) * (kD / 2) + e * 16 + l16];
-              const float c = fmaf(A.x, B.x, -A.y * B.y), sn = fmaf(A.x, B.y, A.y * B.x);
-              const float other = __shfl_xor_sync(0xffffffffu, k4[e], 16);
-              k4[e] = upper ? fmaf(other, sn, k4[e] * c) : fmaf(-other, sn, k4[e] * c);
+              xq[e] = fmaf(xs[e], ca[e], ys[e] * sa[e]);
+              yq[e] = fmaf(ys[e], ca[e], -xs[e] * sa[e]);
             }
-#pragma unroll
-            for (int g = 0; g < GP; ++g)
-              v[(i0 + u) * GP + g] = fmaf(q4[g].x, k4[0], fmaf(q4[g].y, k4[1], fmaf(q4[g].z, k4[2], q4[g].w * k4[3])));
+            qa[g][0] = make_float2(xq[0], xq[1]); qa[g][1] = make_float2(xq[2], xq[3]);
+            qa[g][2] = make_float2(yq[0], yq[1]); qa[g][3] = make_float2(yq[2], yq[3]);
           }
         }
-        transpose_reduce32(v, lane);
-        const int t = base + lane / GP;
-        if (lane < TB * GP && t < ntok) rlog[t * GP + (lane % GP)] = v[0];
+        const int bend = min(ntok, blk * 32 + 32);
+        // anchor terms: this half's tokens of step st are
+        // blk * 32 + st * 2 TBH + half * TBH + [0, TBH); rows past bend are
+        // read from stale token words (slots clamped) and not stored
+        const int tb0 = blk * 32 + half * TBH;
+        auto fetch = [&](int bi, Row8<T> (&r)[TL]) {
+          const int t1 = tb0 + (bi / BPS) * 2 * TBH + (bi % BPS) * TL;
+#pragma unroll
+          for (int w = 0; w < TL; ++w)
+            r[w].load(Ka + (int64_t)min((int)(tok0p[sh_tok[0] + t1 + w] & 0xFFFFu), a.k - 1) * kD);
+        };
+        Row8<T> cur[TL], nxt[TL];
+        fetch(0, cur);
+#pragma unroll 1
+        for (int st = 0; st < NS && blk * 32 + st * 2 * TBH < bend; ++st) {
+          float v[16];
+#pragma unroll
+          for (int j = 0; j < BPS; ++j) {
+            const int bi = st * BPS + j;
+            if (bi + 1 < NS * BPS) fetch(bi + 1, nxt);
+#pragma unroll
+            for (int w = 0; w < TL; ++w) {
+              const int bo = (tb0 + st * 2 * TBH + j * TL + w) & 31;
+              float x[8];
+              cur[w].to_f(x);
+              turn_dot<GP>(x, tbB[bo * 32], tbB[bo * 32 + 16], qa, v + (j * TL + w) * GP);
+            }
+#pragma unroll
+            for (int w = 0; w < TL; ++w) cur[w] = nxt[w];
+          }
+          transpose_reduce16<16>(v, lane);
+          const int t = tb0 + st * 2 * TBH + l16 / GP;
+          if (t < bend) rlog[t * GP + l16 % GP] = v[0] * half_bits_to_f(tok0p[sh_tok[0] + t] >> 16);
+        }
+        // residual terms of the block's key records
+        const int rlo = min(wpre[blk], nK), rhi = min(wpre[blk + 1], nK);
+        for (int r0 = rlo; r0 < rhi; r0 += 2 * TBH) {
+          float v[16];
+#pragma unroll
+          for (int u = 0; u < TBH; ++u) {
+            // records past rhi repeat the last one (every lane takes part in
+            // the transform's shuffles); their terms are not stored
+            const int r = min(r0 + half * TBH + u, rhi - 1);
+            const int bo = rtok[r] & 31;
+            const uint32_t b0 = codes[r * kCodeBytes + l16], b1 = codes[r * kCodeBytes + 16 + l16];
+            const float2 p0 = lutc[(b0 & 15u) * 16], p1 = lutc[(b0 >> 4) * 16];
+            const float2 p2 = lutc[(b1 & 15u) * 16], p3 = lutc[(b1 >> 4) * 16];
+            float y[8] = {p0.x, p0.y, p1.x, p1.y, p2.x, p2.y, p3.x, p3.y};
+            if (!a.naive) fwht128_half(y, lane);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] *= sg[e];
+            turn_dot<GP>(y, tbB[bo * 32], tbB[bo * 32 + 16], qa, v + u * GP);
+          }
+          transpose_reduce16<16>(v, lane);
+          const int r = r0 + half * TBH + l16 / GP;
+          if (r < rhi) rres[r * GP + l16 % GP] = v[0] * half_bits_to_f(sig0[sh_sig[0] + r]);
+        }
       }
       __syncthreads();
     }
@@ -866,29 +987,26 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
         slv[i] = min((int)(wv & 0xFFFFu), a.k - 1);
         gmv[i] = half_bits_to_f(wv >> 16);
         gabs = fmaxf(gabs, fabsf(gmv[i]));
+        const uint32_t word = bm0[t >> 5];
+        const uint32_t below = word & ((1u << (t & 31)) - 1u);
+        const int rank = wpre[t >> 5] + __popc(below);
+        const bool res = ((word >> (t & 31)) & 1u) && rank < nrec[0];
+        float pv[GP];
+        float gam = 1.f;
         if constexpr (ROPE) {
-#pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            lg[i][g] = rlog[t * GP + g];
-            cmx[g] = fmaxf(cmx[g], lg[i][g]);
-          }
+          load_slot<GP>(rlog + t * GP, pv);             // anchor terms, gamma~ included
         } else {
           const uint32_t wk = tok0p[sh_tok[0] + t];
           const int slot = min((int)(wk & 0xFFFFu), a.k - 1);
-          const float gam = half_bits_to_f(wk >> 16);
-          const uint32_t word = bm0[t >> 5];
-          const uint32_t below = word & ((1u << (t & 31)) - 1u);
-          const int rank = wpre[t >> 5] + __popc(below);
-          const bool res = ((word >> (t & 31)) & 1u) && rank < nrec[0];
-          float pv[GP];
+          gam = half_bits_to_f(wk >> 16);
           load_slot<GP>(P + slot * GP, pv);
+        }
 #pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            float x = gam * pv[g];
-            if (res) x += klg[rank * GP + g];
-            lg[i][g] = x;
-            cmx[g] = fmaxf(cmx[g], x);
-          }
+        for (int g = 0; g < GP; ++g) {
+          float x = gam * pv[g];
+          if (res) x += klg[rank * GP + g];
+          lg[i][g] = x;
+          cmx[g] = fmaxf(cmx[g], x);
         }
       }
     }
