@@ -39,8 +39,6 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 }
 
 __device__ __forceinline__ void cl_sync() { cluster_barrier(); }
-template <typename U>
-__device__ __forceinline__ U* peer_ptr(U* p, unsigned rank) { return cluster_peer(p, rank); }
 
 // Exclusive block-wide prefix sum of v (one value per thread); returns the
 // thread's prefix and writes the block total to *total.
@@ -81,6 +79,7 @@ struct SelSmem {
   RadixSmem<kThreads> rs;
   int warp_tot[kWarps];
   int cta_count;                     // this CTA's count exposed to the cluster
+  int csum[2];                       // cluster sums of the counts (before this CTA, all)
   float stage[kSeg + 256];           // raw scores of one pooling segment (kappa <= 255)
 };
 
@@ -100,9 +99,8 @@ __device__ void mark_selected(SelSmem& sm, const RadixResult<K>& sr, int lo, int
     const int before = block_exclusive_scan(ties, sm.warp_tot, &local_total);
     if (threadIdx.x == 0) sm.cta_count = local_total;
     cl_sync();
-    const unsigned r = blockIdx.x % kC;
-    int cta_before = 0;
-    for (unsigned rr = 0; rr < r; ++rr) cta_before += *peer_ptr(&sm.cta_count, rr);
+    int cta_before = 0, cta_all = 0;
+    cluster_sums<kC>(&sm.cta_count, sm.csum, blockIdx.x % kC, cta_before, cta_all);
     rank0 = cta_before + before;
   }
   // keys are read before any flag of this thread changes (the value-sample
@@ -157,13 +155,35 @@ anchor_select_kernel(const float* __restrict__ score, float* __restrict__ pooled
   const int pend = min(c1, NW);
   for (int sb = c0; sb < pend; sb += kSeg) {
     const int se = min(pend, sb + kSeg);
-    for (int u = sb - half + tid; u < se + half; u += kThreads) {
-      float v = 0.f;
-      if (u >= 0 && u < NW) {
-        v = score[(int64_t)h * N + u];
-        for (int rb = 1; rb < obs_rb; ++rb) v += score[((int64_t)rb * H + h) * N + u];
+    // a thread's staging entries u = sb - half + tid + i kThreads, their
+    // partials loaded kRB row blocks at a time (all in flight together) and
+    // summed in row-block order
+    constexpr int kE = (kSeg + 256 + kThreads - 1) / kThreads;
+    constexpr int kRB = 4;
+    const int ub = sb - half + tid, ue = se + half;
+    float acc[kE];
+#pragma unroll
+    for (int i = 0; i < kE; ++i) acc[i] = 0.f;
+    for (int rb0 = 0; rb0 < obs_rb; rb0 += kRB) {
+      float part[kE][kRB];
+#pragma unroll
+      for (int i = 0; i < kE; ++i) {
+        const int u = ub + i * kThreads;
+        const bool in = u < ue && u >= 0 && u < NW;
+#pragma unroll
+        for (int q = 0; q < kRB; ++q)
+          part[i][q] = (in && rb0 + q < obs_rb) ? score[((int64_t)(rb0 + q) * H + h) * N + u] : 0.f;
       }
-      sm.stage[u - (sb - half)] = v;
+#pragma unroll
+      for (int i = 0; i < kE; ++i)
+#pragma unroll
+        for (int q = 0; q < kRB; ++q)
+          if (rb0 + q < obs_rb) acc[i] = (rb0 + q == 0) ? part[i][q] : acc[i] + part[i][q];
+    }
+#pragma unroll
+    for (int i = 0; i < kE; ++i) {
+      const int u = ub + i * kThreads;
+      if (u < ue) sm.stage[u - (sb - half)] = (u >= 0 && u < NW) ? acc[i] : 0.f;
     }
     __syncthreads();
     for (int t = sb + tid; t < se; t += kThreads) {
@@ -213,18 +233,16 @@ anchor_select_kernel(const float* __restrict__ score, float* __restrict__ pooled
   if (tid == 0) sm.cta_count = local_total;
   cl_sync();
   int cta_before = 0, all = 0;
-  for (unsigned rr = 0; rr < (unsigned)kC; ++rr) {
-    const int c = *peer_ptr(&sm.cta_count, rr);
-    if (rr < r) cta_before += c;
-    all += c;
-  }
+  cluster_sums<kC>(&sm.cta_count, sm.csum, r, cta_before, all);
   int* apos = anchor_pos + (int64_t)h * k;
   int* sof = slot_of + (int64_t)h * N;
+  int* spos = reinterpret_cast<int*>(keys);   // this CTA's anchor positions (the keys are spent)
   {
     int s = cta_before + before;
     for (int i = lo; i < hi; ++i) {
       if (flag[i]) {
         if (s < k) apos[s] = c0 + i;
+        spos[s - cta_before] = c0 + i;
         sof[c0 + i] = s;
         ++s;
       } else {
@@ -243,13 +261,24 @@ anchor_select_kernel(const float* __restrict__ score, float* __restrict__ pooled
   const int warp = tid >> 5, lane = tid & 31;
   const int s_lo = cta_before, s_hi = cta_before + local_total;
   for (int s = s_lo + warp; s < s_hi; s += kWarps) {
-    const int t = apos[s];
+    const int t = spos[s - s_lo];
+    // both sides' rows in flight together
+    T raw[2][4];
+#pragma unroll
     for (int side = 0; side < 2; ++side) {
       const T* src = (side ? V : K) + ((int64_t)h * N + t) * kD;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) raw[side][e] = src[lane * 4 + e];
+    }
+#pragma unroll
+    for (int side = 0; side < 2; ++side) {
       T* dst = (side ? anc_v : anc_k) + ((int64_t)h * k + s) * kD;
       float f[4];
-      load4<T>(src + lane * 4, f);
-      for (int e = 0; e < 4; ++e) dst[lane * 4 + e] = src[lane * 4 + e];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        dst[lane * 4 + e] = raw[side][e];
+        f[e] = to_f(raw[side][e]);
+      }
       double n2 = 0.0;
       for (int e = 0; e < 4; ++e) n2 += (double)f[e] * (double)f[e];
       n2 = warp_sum_d(n2);

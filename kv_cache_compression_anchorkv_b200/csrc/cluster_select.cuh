@@ -4,7 +4,8 @@
 // The `want` smallest keys of a set spread over the C CTAs of a thread-block
 // cluster are found digit by digit (8 bits from the top): every warp counts
 // its keys that match the prefix found so far in a private histogram (native
-// shared-memory integer atomics), the CTA sums its warps' histograms, every
+// shared-memory integer atomics; with at most 8 keys per thread, straight
+// into the CTA histogram), the CTA sums its warps' histograms, every
 // CTA sums the C CTA histograms through distributed shared memory and picks
 // the same digit.  The select stops as soon as the threshold bin holds
 // exactly the keys still needed.  The caller then takes the keys below the
@@ -25,6 +26,29 @@ __device__ __forceinline__ void cluster_barrier() {
 template <typename U>
 __device__ __forceinline__ U* cluster_peer(U* p, unsigned rank) {
   return static_cast<U*>(__cluster_map_shared_rank(p, rank));
+}
+
+// Sum over the CTAs of the cluster of the int at `p` in each, and the sum over
+// the CTAs ranked below this one: one warp reads the peers (lane rr reads CTA
+// rr), the results go through `out` ([2]) to the whole CTA.  Call between
+// cluster barriers that order the peers' writes of *p before the reads.
+template <int C>
+__device__ __forceinline__ void cluster_sums(int* p, int* out, unsigned rank, int& before, int& all) {
+  static_assert(C <= 32, "one lane per CTA");
+  if (threadIdx.x < 32) {
+    const unsigned lane = threadIdx.x;
+    const int v = lane < (unsigned)C ? *cluster_peer(p, lane) : 0;
+    int b = lane < rank ? v : 0, a = v;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      b += __shfl_xor_sync(0xffffffffu, b, o);
+      a += __shfl_xor_sync(0xffffffffu, a, o);
+    }
+    if (lane == 0) { out[0] = b; out[1] = a; }
+  }
+  __syncthreads();
+  before = out[0];
+  all = out[1];
 }
 
 template <int kThreads>
@@ -67,23 +91,32 @@ __device__ RadixResult<K> cluster_radix_select(RadixSmem<kThreads>& sm, int iter
   res.all_ties = false;
   int buf = 0;
   int depth = 0;
+  // few keys per thread: count straight into the CTA histogram (no per-warp
+  // histograms to clear and add up)
+  const bool direct = iters <= 8;
   for (; depth < kB; depth += 8) {
     const int shift = kB - depth - 8;
-    for (int i = threadIdx.x; i < kWarps * 256; i += kThreads) (&sm.whist[0][0])[i] = 0u;
+    if (direct) {
+      if (threadIdx.x < 256) sm.hist[buf][threadIdx.x] = 0u;
+    } else {
+      for (int i = threadIdx.x; i < kWarps * 256; i += kThreads) (&sm.whist[0][0])[i] = 0u;
+    }
     __syncthreads();
-    unsigned* wh = sm.whist[warp];
+    unsigned* wh = direct ? sm.hist[buf] : sm.whist[warp];
     for (int j = 0; j < iters; ++j) {
       K kk = 0;
       if (key(j, kk) && radix_top(kk, depth) == res.prefix) atomicAdd(&wh[(unsigned)(kk >> shift) & 255u], 1u);
     }
     __syncthreads();
-    if (threadIdx.x < 256) {
-      unsigned t = 0;
+    if (!direct) {
+      if (threadIdx.x < 256) {
+        unsigned t = 0;
 #pragma unroll 8
-      for (int w = 0; w < kWarps; ++w) t += sm.whist[w][threadIdx.x];
-      sm.hist[buf][threadIdx.x] = t;
+        for (int w = 0; w < kWarps; ++w) t += sm.whist[w][threadIdx.x];
+        sm.hist[buf][threadIdx.x] = t;
+      }
+      __syncthreads();
     }
-    __syncthreads();
     cluster_barrier();
     if (threadIdx.x < 256) {
       unsigned t = 0;

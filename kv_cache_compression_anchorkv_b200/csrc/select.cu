@@ -84,17 +84,38 @@ select_kernel(const float* __restrict__ util, int N, int n_t, int n_sh, int R, i
   // u >= 0 maps to ~bits(u) - 2^31 in [0, 2^31) (smallest first = largest
   // utility), everything else to kNone.
   constexpr uint32_t kNone = 0xFFFFFFFFu;
-  uint32_t* keys = resident ? reinterpret_cast<uint32_t*>(tcount + ((nt + 3) & ~3)) : nullptr;
+  // per 32-token word, ballots of the slots at the threshold and above it
+  uint32_t* eqw = reinterpret_cast<uint32_t*>(tcount + ((nt + 3) & ~3));   // [4 nt]
+  uint32_t* abw = eqw + 4 * nt;                                            // [4 nt]
+  uint32_t* keys = resident ? abw + 4 * nt : nullptr;
+  auto key_of_u = [](float u) -> uint32_t { return (u >= 0.f) ? (~__float_as_uint(u)) & 0x7FFFFFFFu : kNone; };
+  // when N is a multiple of the tile, slot q of this CTA is utility
+  // tb * 128 + q (no per-slot division)
+  const bool dense = (N % kTile) == 0;
+  const float* ub = util + (int64_t)tb * kTile;
   auto key_from_global = [&](int q) -> uint32_t {
+    if (dense) return key_of_u(ub[q]);
     const int tile = tb + (q >> 7);
     if (tile >= te) return kNone;
     const int sh = tile / n_t, t = (tile % n_t) * kTile + (q & 127);
     if (t >= N) return kNone;
-    const float u = util[(int64_t)sh * N + t];
-    return (u >= 0.f) ? (~__float_as_uint(u)) & 0x7FFFFFFFu : kNone;
+    return key_of_u(util[(int64_t)sh * N + t]);
   };
-  if (resident)
-    for (int q = tid; q < nt * kTile; q += kThreads) keys[q] = key_from_global(q);
+  if (resident) {
+    const int n = nt * kTile;
+    int q = tid;
+    if (dense) {
+      // four independent loads per thread in flight
+      for (; q + 3 * kThreads < n; q += 4 * kThreads) {
+        const float u0 = ub[q], u1 = ub[q + kThreads], u2 = ub[q + 2 * kThreads], u3 = ub[q + 3 * kThreads];
+        keys[q] = key_of_u(u0);
+        keys[q + kThreads] = key_of_u(u1);
+        keys[q + 2 * kThreads] = key_of_u(u2);
+        keys[q + 3 * kThreads] = key_of_u(u3);
+      }
+    }
+    for (; q < n; q += kThreads) keys[q] = key_from_global(q);
+  }
   auto key_of = [&](int q) -> uint32_t { return resident ? keys[q] : key_from_global(q); };
   auto eligible = [&](int, uint32_t k32) -> bool { return k32 != kNone; };
   __syncthreads();
@@ -122,44 +143,55 @@ select_kernel(const float* __restrict__ util, int N, int n_t, int n_sh, int R, i
     return top < sr.prefix ? 2 : (top == sr.prefix ? 1 : 0);
   };
 
-  // 2. tie counts per tile
+  // 2. one warp per tile: ballots of "at the threshold" and "above it" per
+  //    32-token word, kept in shared memory; tie counts per tile
+  uint32_t eqv[4], abv[4];
   for (int i = warp; i < nt; i += kWarps) {
     int eq = 0;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) eq += __popc(__ballot_sync(0xffffffffu, cls(i * kTile + w * 32 + lane) == 1));
-    if (lane == 0) tcount[i] = eq;
+    for (int w = 0; w < 4; ++w) {
+      const int c = cls(i * kTile + w * 32 + lane);
+      eqv[w] = __ballot_sync(0xffffffffu, c == 1);
+      abv[w] = __ballot_sync(0xffffffffu, c == 2);
+      eq += __popc(eqv[w]);
+    }
+    __syncwarp();
+    if (lane == 0) {
+      tcount[i] = eq;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) { eqw[4 * i + w] = eqv[w]; abw[4 * i + w] = abv[w]; }
+    }
   }
   __syncthreads();
   const int ties = block_scan_inplace(tcount, nt, sm.warp_tot);
   if (tid == 0) sm.cta_ties = ties;
   cluster_barrier();
   int ties_before = 0, ties_all = 0;
-  for (unsigned rr = 0; rr < (unsigned)C; ++rr) {
-    const int c = *cluster_peer(&sm.cta_ties, rr);
-    if (rr < r) ties_before += c;
-    ties_all += c;
-  }
+  cluster_sums<C>(&sm.cta_ties, sm.scal, r, ties_before, ties_all);
   if (r == 0 && tid == 0 && !take_all && !sr.all_ties && ties_all > 0) atomicAdd(&counters[kSelectTies], ties_all);
 
-  // 3. bitmap words; record counts per tile
-  for (int i = warp; i < nt; i += kWarps) {
-    const int tile = tb + i;
-    int rank = ties_before + tcount[i];
-    int cnt = 0;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const int c = cls(i * kTile + w * 32 + lane);
-      const uint32_t eqb = __ballot_sync(0xffffffffu, c == 1);
-      const int my = rank + __popc(eqb & ((1u << lane) - 1u));
-      const bool s = c == 2 || (c == 1 && (sr.all_ties || my < sr.need));
-      const uint32_t sb = __ballot_sync(0xffffffffu, s);
-      if (lane == 0) bitmap[(int64_t)tile * 4 + w] = sb;
-      rank += __popc(eqb);
-      cnt += __popc(sb);
+  // 3. one thread per bitmap word: the words above the threshold, and of the
+  //    words at it the first `need` bits over the cluster in flat order
+  //    (lowest bit = lowest token); record counts per tile
+  for (int x = tid; x < 4 * nt; x += kThreads) {
+    const int i = x >> 2, w = x & 3;
+    const uint32_t eq = eqw[x];
+    uint32_t sel = eq;
+    if (!sr.all_ties && eq) {
+      int rank = ties_before + tcount[i];
+      for (int v = 0; v < w; ++v) rank += __popc(eqw[4 * i + v]);
+      const int n = min(max(sr.need - rank, 0), __popc(eq));
+      if (n < __popc(eq)) {
+        const int pos = n ? (int)__fns(eq, 0, n) : -1;     // the n-th set bit
+        sel = pos < 0 ? 0u : (pos == 31 ? eq : eq & ((2u << pos) - 1u));
+      }
     }
-    __syncwarp();
-    if (lane == 0) tcount[i] = cnt;
+    const uint32_t sb = abw[x] | sel;
+    bitmap[(int64_t)(tb + i) * 4 + w] = sb;
+    abw[x] = (uint32_t)__popc(sb);     // only this thread reads abw[x]
   }
+  __syncthreads();
+  for (int i = tid; i < nt; i += kThreads) tcount[i] = (int)(abw[4 * i] + abw[4 * i + 1] + abw[4 * i + 2] + abw[4 * i + 3]);
   __syncthreads();
 
   // 4. tile prefixes [n_sh][n_t + 1]; entry n_t of (side, head) sh is the
@@ -167,8 +199,8 @@ select_kernel(const float* __restrict__ util, int N, int n_t, int n_sh, int R, i
   const int recs = block_scan_inplace(tcount, nt, sm.warp_tot);
   if (tid == 0) sm.cta_recs = recs;
   cluster_barrier();
-  int recs_before = 0;
-  for (unsigned rr = 0; rr < r; ++rr) recs_before += *cluster_peer(&sm.cta_recs, rr);
+  int recs_before = 0, recs_all = 0;
+  cluster_sums<C>(&sm.cta_recs, sm.scal + 2, r, recs_before, recs_all);
   for (int i = tid; i < nt; i += kThreads) {
     const int tile = tb + i, sh = tile / n_t, j = tile % n_t;
     const int v = recs_before + tcount[i];
@@ -231,7 +263,7 @@ cudaError_t launch_select(const Plan& pl, char* out, char* ws, cudaStream_t s) {
   const int n_all = n_sh * n_t;
   auto plan = [&](int C, int* resident) -> size_t {
     const int tiles = (n_all + C - 1) / C;
-    const size_t base = sizeof(SelectSmem) + 4 * (size_t)((tiles + 3) & ~3);
+    const size_t base = sizeof(SelectSmem) + 4 * (size_t)((tiles + 3) & ~3) + 32 * (size_t)tiles;
     const size_t with_keys = base + 4 * (size_t)tiles * kTile;
     *resident = with_keys <= 227 * 1024 ? 1 : 0;
     return *resident ? with_keys : base;
