@@ -862,7 +862,7 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
       //     - residual terms of the block's key records: the residual is
       //       rebuilt by one half-warp Hadamard transform; sigma~ times its
       //       dot product goes to klg by rank.
-      //     16 / G tokens (records) per half-warp step, the 16 G products
+      //     Anchor terms: 16 / G tokens per half-warp step, the 16 G products
       //     finished by one transposed reduction.
       constexpr int TBH = 16 / GP;
       constexpr int TL0 = sizeof(T) == 2 ? 4 : 2;
@@ -940,28 +940,28 @@ __global__ void __launch_bounds__(kThreads, GP <= 4 ? 2 : 1) flash_decode_kernel
           const int t = tb0 + st * 2 * TBH + l16 / GP;
           if (t < bend) rlog[t * GP + l16 % GP] = v[0] * half_bits_to_f(tok0p[sh_tok[0] + t] >> 16);
         }
-        // residual terms of the block's key records
+        // residual terms of the block's key records, one record per
+        // half-warp per step (a rolled loop: the transform is the bulk of
+        // the code), its G dot products finished by a 16-lane reduction
         const int rlo = min(wpre[blk], nK), rhi = min(wpre[blk + 1], nK);
-        for (int r0 = rlo; r0 < rhi; r0 += 2 * TBH) {
-          float v[16];
+#pragma unroll 1
+        for (int r0 = rlo; r0 < rhi; r0 += 2) {
+          // a record past rhi repeats the last one (every lane takes part
+          // in the shuffles); its terms are not stored
+          const int r = min(r0 + half, rhi - 1);
+          const int bo = rtok[r] & 31;
+          const uint32_t b0 = codes[r * kCodeBytes + l16], b1 = codes[r * kCodeBytes + 16 + l16];
+          const float2 p0 = lutc[(b0 & 15u) * 16], p1 = lutc[(b0 >> 4) * 16];
+          const float2 p2 = lutc[(b1 & 15u) * 16], p3 = lutc[(b1 >> 4) * 16];
+          float y[8] = {p0.x, p0.y, p1.x, p1.y, p2.x, p2.y, p3.x, p3.y};
+          if (!a.naive) fwht128_half(y, lane);
 #pragma unroll
-          for (int u = 0; u < TBH; ++u) {
-            // records past rhi repeat the last one (every lane takes part in
-            // the transform's shuffles); their terms are not stored
-            const int r = min(r0 + half * TBH + u, rhi - 1);
-            const int bo = rtok[r] & 31;
-            const uint32_t b0 = codes[r * kCodeBytes + l16], b1 = codes[r * kCodeBytes + 16 + l16];
-            const float2 p0 = lutc[(b0 & 15u) * 16], p1 = lutc[(b0 >> 4) * 16];
-            const float2 p2 = lutc[(b1 & 15u) * 16], p3 = lutc[(b1 >> 4) * 16];
-            float y[8] = {p0.x, p0.y, p1.x, p1.y, p2.x, p2.y, p3.x, p3.y};
-            if (!a.naive) fwht128_half(y, lane);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] *= sg[e];
-            turn_dot<GP>(y, tbB[bo * 32], tbB[bo * 32 + 16], qa, v + u * GP);
-          }
-          transpose_reduce16<16>(v, lane);
-          const int r = r0 + half * TBH + l16 / GP;
-          if (r < rhi) rres[r * GP + l16 % GP] = v[0] * half_bits_to_f(sig0[sh_sig[0] + r]);
+          for (int e = 0; e < 8; ++e) y[e] *= sg[e];
+          float d[GP];
+          turn_dot<GP>(y, tbB[bo * 32], tbB[bo * 32 + 16], qa, d);
+          transpose_reduce16<GP>(d, lane);
+          if (r0 + half < rhi && (l16 % (16 / GP)) == 0)
+            rres[r * GP + l16 / (16 / GP)] = d[0] * half_bits_to_f(sig0[sh_sig[0] + r]);
         }
       }
       __syncthreads();
