@@ -291,15 +291,13 @@ __global__ void __launch_bounds__(256, 3) quantize_kernel(const T* __restrict__ 
             y[e] = a0 + a1;
             y[e | m] = a0 - a1;
           }
-      // ... and three on the lane bits
+      // ... and three on the lane bits: y + other below, other - y above,
+      // both one fma with a sign of +-1 (exact: one rounding, as the add)
 #pragma unroll
       for (int m = 1; m < 8; m <<= 1) {
-        const bool upper = l8 & m;
+        const double sg = (l8 & m) ? -1.0 : 1.0;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const double other = __shfl_xor_sync(0xffffffffu, y[e], m);
-          y[e] = upper ? (other - y[e]) : (y[e] + other);
-        }
+        for (int e = 0; e < 16; ++e) y[e] = fma(y[e], sg, __shfl_xor_sync(0xffffffffu, y[e], m));
       }
     }
     if (!live) continue;
