@@ -9,14 +9,16 @@
 // KV head and side, D = 128) runs as tcgen05.mma (M = 128, N = chunk of
 // anchors, K = 16 per instruction) from 128-byte-swizzled shared-memory
 // tiles that TMA fills; accumulators live in a ring of TMEM chunk buffers
-// (as many as fit in 512 columns).  Chunks are as wide as possible (up to
-// N = 256): the MMA issue rate per FLOP is best for wide N.  The ring is
-// shared by the epilogue groups, so a group may reach chunk q while the
-// buffer still waits for chunk q - nbuf; since a parity wait cannot tell
-// phase p from p + 2, a group first waits until the MMA warp has published
-// that it issued chunk q (which it does only after chunk q - nbuf was
-// released) and only then waits on the buffer's barrier.  The epilogue never writes
-// S: each thread reads its TMEM lane, scales each column by 1/||a_s|| and
+// (as many as fit in 512 columns).  Chunks are at most 128 anchors wide: the
+// epilogue and the MMA wait on each other through the ring, and a deeper ring
+// of narrower chunks (five buffers of 96 for 288 anchors) measured faster than
+// fewer wide ones (three of 144), although wide N issues MMAs at a better rate
+// per FLOP.  The ring is shared by the epilogue groups, so a group may reach
+// chunk q while the buffer still waits for chunk q - nbuf; since a parity
+// wait cannot tell phase p from p + 2, a group first waits until the MMA warp
+// has published that it issued chunk q (which it does only after chunk
+// q - nbuf was released) and only then waits on the buffer's barrier.  The
+// epilogue never writes S: each thread reads its TMEM lane, scales each column by 1/||a_s|| and
 // keeps the best and second-best score of its row over all chunks.  Rows
 // whose fp32 margin between best and second best is not above the
 // accumulation error bound are listed for the fp64 re-decision shared with
@@ -65,7 +67,7 @@ namespace {
 #define AKV_ASSIGN_ITEM_GROUPS 2
 #endif
 #ifndef AKV_ASSIGN_CHUNK
-#define AKV_ASSIGN_CHUNK 256
+#define AKV_ASSIGN_CHUNK 128
 #endif
 constexpr int kGroups = AKV_ASSIGN_ITEM_GROUPS;   // item groups: epilogue groups that take whole items in turn
 constexpr int kColGroups = AKV_ASSIGN_COL_GROUPS;   // groups of four warps sharing an item's columns
