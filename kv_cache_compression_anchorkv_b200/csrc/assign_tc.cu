@@ -9,11 +9,11 @@
 // KV head and side, D = 128) runs as tcgen05.mma (M = 128, N = chunk of
 // anchors, K = 16 per instruction) from 128-byte-swizzled shared-memory
 // tiles that TMA fills; accumulators live in a ring of TMEM chunk buffers
-// (as many as fit in 512 columns).  Chunks are at most 128 anchors wide: the
+// (as many as fit in 512 columns).  Chunks are at most 96 anchors wide: the
 // epilogue and the MMA wait on each other through the ring, and a deeper ring
 // of narrower chunks (five buffers of 96 for 288 anchors) measured faster than
-// fewer wide ones (three of 144), although wide N issues MMAs at a better rate
-// per FLOP.  The ring is shared by the epilogue groups, so a group may reach
+// fewer wide ones (three of 144, or of 128 at most), although wide N issues
+// MMAs at a better rate per FLOP.  The ring is shared by the epilogue groups, so a group may reach
 // chunk q while the buffer still waits for chunk q - nbuf; since a parity
 // wait cannot tell phase p from p + 2, a group first waits until the MMA warp
 // has published that it issued chunk q (which it does only after chunk
@@ -67,7 +67,7 @@ namespace {
 #define AKV_ASSIGN_ITEM_GROUPS 2
 #endif
 #ifndef AKV_ASSIGN_CHUNK
-#define AKV_ASSIGN_CHUNK 128
+#define AKV_ASSIGN_CHUNK 96
 #endif
 constexpr int kGroups = AKV_ASSIGN_ITEM_GROUPS;   // item groups: epilogue groups that take whole items in turn
 constexpr int kColGroups = AKV_ASSIGN_COL_GROUPS;   // groups of four warps sharing an item's columns
