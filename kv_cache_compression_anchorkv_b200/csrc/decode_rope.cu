@@ -27,6 +27,10 @@
 // row standing in for the anchor row with gamma~ = 1 and no residual.
 // Splits of the tokens (multiples of 32) over CTAs fill the SMs; a second
 // kernel merges the splits in order.
+//
+// These kernels serve 16 query heads per KV head.  Up to 8, the rotary decode
+// runs on the slice decode (decode_flash.cu) with its rotary key phase, which
+// the plan below picks first.
 #include "common.cuh"
 #include "internal.h"
 
