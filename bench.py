@@ -958,8 +958,9 @@ def run_gpu(args, world, rank, local):
 
 
 def run_e2e(args, spec, theta, params, ids, job_layers, dev, stream, barrier, world):
-    """Same step through the public API with host buffers: per layer, pinned
-    K, V, Q_obs are copied in, compressed and the layout copied back; then the
+    """Same step through the public API with host buffers: per layer, the
+    C ABI's anchorkv_compress_host copies the pinned K, V, Q_obs in, compresses
+    and copies the layout back (the copies inside the library); then the
     decode step copies each layer's query in and its output back."""
     import torch
 

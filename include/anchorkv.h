@@ -194,6 +194,33 @@ int anchorkv_compress(const anchorkv_params* p, const void* K, const void* V,
                       const void* Q_obs, void* out, size_t out_bytes,
                       void* ws, size_t ws_bytes, void* stream);
 
+/* Device staging bytes anchorkv_compress_host needs for `p`: K, V, Q_obs and
+ * the compressed layout of one layer, each 256-byte aligned.  Host, pure. */
+int anchorkv_compress_host_staging_bytes(const anchorkv_params* p, size_t* bytes);
+
+/*
+ * anchorkv_compress from host buffers: copies K, V and Q_obs into `staging`,
+ * compresses there and copies the layout back, everything queued on
+ * `stream` (one cudaMemcpyAsync per buffer, so page-locked host buffers make
+ * the copies asynchronous and let them overlap work on other streams).
+ *   K_host, V_host  host [H][N][D] dtype
+ *   Q_host          host [H_q][W][D] dtype (may be NULL with
+ *                   ANCHORKV_MODE_KEY_QUERIES)
+ *   out_host        host, out_bytes >= anchorkv_layout.total_bytes; valid once
+ *                   `stream` has completed the call's work
+ *   staging         device, 16-byte aligned, staging_bytes >=
+ *                   anchorkv_compress_host_staging_bytes; owned by the caller.
+ *                   It holds K, V, Q_obs and the layout in that order, each
+ *                   section rounded up to 256 bytes; the layout (its last
+ *                   section) stays there for the caller's device-side use
+ *   ws, ws_bytes    as for anchorkv_compress
+ * The host buffers must stay alive and unmodified until the stream completes.
+ * Errors as anchorkv_compress; ENOSPC also for a small staging buffer.
+ */
+int anchorkv_compress_host(const anchorkv_params* p, const void* K_host, const void* V_host,
+                           const void* Q_host, void* out_host, size_t out_bytes, void* staging,
+                           size_t staging_bytes, void* ws, size_t ws_bytes, void* stream);
+
 /* Workspace bytes anchorkv_decode_attn needs for `batch` sequences (0 when
  * every (sequence, head) is decoded by a single CTA). */
 int anchorkv_decode_workspace_bytes(const anchorkv_params* p, int32_t batch, size_t* ws_bytes);

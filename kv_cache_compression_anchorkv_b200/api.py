@@ -107,6 +107,41 @@ def compress(p: AnchorKVParams, K: torch.Tensor, V: torch.Tensor, Q_obs: torch.T
     return out, workspace
 
 
+def compress_host_staging_bytes(p: AnchorKVParams) -> int:
+    """Device staging bytes compress_host needs (K, V, Q_obs and the layout)."""
+    n = ctypes.c_size_t()
+    capi.check("anchorkv_compress_host_staging_bytes",
+               capi.lib().anchorkv_compress_host_staging_bytes(ctypes.byref(p.c()), ctypes.byref(n)))
+    return n.value
+
+
+def _check_host(name, t, shape, dtype):
+    if t.device.type != "cpu":
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
+def compress_host(p: AnchorKVParams, K: torch.Tensor, V: torch.Tensor, Q_obs: torch.Tensor | None,
+                  out: torch.Tensor, staging: torch.Tensor, workspace: torch.Tensor, device="cuda") -> torch.Tensor:
+    """Compress one layer from host buffers through anchorkv_compress_host: the
+    library copies K, V, Q_obs (host, ideally pinned) into `staging` (device),
+    compresses there and copies the layout into `out` (host uint8), all on the
+    current stream of `device`.  `out` is valid once that stream has run."""
+    H, N, D, W = p.n_kv_heads, p.n_tokens, p.head_dim, p.window
+    _check_host("K", K, (H, N, D), p.torch_dtype)
+    _check_host("V", V, (H, N, D), p.torch_dtype)
+    if Q_obs is not None or not (p.mode & MODE_KEY_QUERIES):
+        _check_host("Q_obs", Q_obs, (p.n_q_heads, W, D), p.torch_dtype)
+    if out.device.type != "cpu" or out.dtype != torch.uint8:
+        raise ValueError("out must be a host uint8 tensor")
+    st = capi.lib().anchorkv_compress_host(ctypes.byref(p.c()), _ptr(K), _ptr(V), _ptr(Q_obs), _ptr(out),
+                                           out.numel(), _ptr(staging), staging.numel(), _ptr(workspace),
+                                           workspace.numel(), _stream(torch.device(device)))
+    capi.check("anchorkv_compress_host", st)
+    return out
+
+
 def decode_workspace_bytes(p: AnchorKVParams, batch: int) -> int:
     n = ctypes.c_size_t()
     capi.check("anchorkv_decode_workspace_bytes",
@@ -260,21 +295,22 @@ def codebook() -> tuple[float, float, float, float]:
 
 
 class HostCompressor:
-    """End-to-end compress from host (pinned) buffers: per call, the layer's
-    K, V, Q_obs are copied to preallocated device buffers, compressed, and the
-    compressed bytes copied back into a pinned host buffer, all on the current
-    stream.  Allocation happens once, in the constructor."""
+    """End-to-end compress from host (pinned) buffers through the C ABI's
+    anchorkv_compress_host: per call, the library copies the layer's K, V,
+    Q_obs into a preallocated device staging buffer, compresses there and
+    copies the compressed bytes back into a pinned host buffer, all on the
+    current stream.  Allocation happens once, in the constructor; `out` is a
+    device view of the staged layout."""
 
     def __init__(self, p: AnchorKVParams, device="cuda"):
         self.p = p
-        H, N, D = p.n_kv_heads, p.n_tokens, p.head_dim
-        self.K = torch.empty(H, N, D, dtype=p.torch_dtype, device=device)
-        self.V = torch.empty_like(self.K)
-        self.Q = torch.empty(p.n_q_heads, p.window, D, dtype=p.torch_dtype, device=device)
+        self.device = torch.device(device)
         L = anchorkv_bytes(p)
-        self.out = torch.empty(L["total_bytes"], dtype=torch.uint8, device=device)
+        self.staging = torch.empty(compress_host_staging_bytes(p), dtype=torch.uint8, device=device)
         self.ws = torch.empty(compress_workspace(p)["total_bytes"], dtype=torch.uint8, device=device)
         self.host_out = torch.empty(L["total_bytes"], dtype=torch.uint8, pin_memory=True)
+        # the staged layout: the staging buffer's last section (256-byte aligned)
+        self.out = self.staging[-((L["total_bytes"] + 255) // 256 * 256):][:L["total_bytes"]]
 
     def __call__(self, K_host, V_host, Q_host, layer: int | None = None, host_out: torch.Tensor | None = None):
         """Compress one layer; the compressed bytes land in `host_out` (pinned,
@@ -283,13 +319,8 @@ class HostCompressor:
         the compression of another."""
         if layer is not None:
             self.p.layer = layer
-        self.K.copy_(K_host, non_blocking=True)
-        self.V.copy_(V_host, non_blocking=True)
-        self.Q.copy_(Q_host, non_blocking=True)
-        compress(self.p, self.K, self.V, self.Q, out=self.out, workspace=self.ws)
         dst = self.host_out if host_out is None else host_out
-        dst.copy_(self.out, non_blocking=True)
-        return dst
+        return compress_host(self.p, K_host, V_host, Q_host, dst, self.staging, self.ws, device=self.device)
 
 
 N_STAGES = 16   # ANCHORKV_N_STAGES

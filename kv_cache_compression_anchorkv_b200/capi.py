@@ -50,6 +50,9 @@ _SIGS = {
     "anchorkv_bytes": ([_P(Params), _P(Layout)], ctypes.c_int),
     "anchorkv_compress_workspace": ([_P(Params), _P(WorkspaceView)], ctypes.c_int),
     "anchorkv_compress": ([_P(Params), _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp, ctypes.c_size_t, _vp], ctypes.c_int),
+    "anchorkv_compress_host_staging_bytes": ([_P(Params), _P(ctypes.c_size_t)], ctypes.c_int),
+    "anchorkv_compress_host": ([_P(Params), _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp, ctypes.c_size_t, _vp,
+                                ctypes.c_size_t, _vp], ctypes.c_int),
     "anchorkv_decode_workspace_bytes": ([_P(Params), ctypes.c_int32, _P(ctypes.c_size_t)], ctypes.c_int),
     "anchorkv_decode_attn": ([_P(Params), _vp, ctypes.c_int64, ctypes.c_int32, _vp, _vp, _vp, ctypes.c_int32,
                               ctypes.c_int32, _vp, _vp, ctypes.c_size_t, _vp], ctypes.c_int),

@@ -222,6 +222,25 @@ static int check_device() {
     if (e_ != cudaSuccess) return ANCHORKV_ECUDA; \
   } while (0)
 
+// Device staging of anchorkv_compress_host: K, V, Q_obs and the layout, each
+// section 256-byte aligned.
+struct HostStaging {
+  int64_t kv, q, out, o_k, o_v, o_q, o_out, total;
+};
+HostStaging host_staging(const Plan& pl) {
+  auto al = [](int64_t x) { return (x + 255) / 256 * 256; };
+  HostStaging h;
+  h.kv = (int64_t)pl.H * pl.N * kD * pl.elem;
+  h.q = (int64_t)pl.Hq * pl.W * kD * pl.elem;
+  h.out = pl.L.total_bytes;
+  h.o_k = 0;
+  h.o_v = al(h.kv);
+  h.o_q = h.o_v + al(h.kv);
+  h.o_out = h.o_q + al(h.q);
+  h.total = h.o_out + al(h.out);
+  return h;
+}
+
 }  // namespace akv
 
 using namespace akv;
@@ -311,6 +330,40 @@ int anchorkv_compress(const anchorkv_params* p, const void* K, const void* V, co
   AKV_STAGE(kStSelect, sel_kernels, launch_select(pl, o, w, s));
   AKV_STAGE(kStQuantize, pl.R ? 1 : 0, launch_quantize(pl, K, V, o, w, s));
 #undef AKV_STAGE
+  return ANCHORKV_OK;
+}
+
+int anchorkv_compress_host_staging_bytes(const anchorkv_params* p, size_t* bytes) {
+  if (!bytes) return ANCHORKV_EINVAL;
+  Plan pl;
+  const int st = make_plan(p, &pl);
+  if (st) return st;
+  *bytes = (size_t)host_staging(pl).total;
+  return ANCHORKV_OK;
+}
+
+int anchorkv_compress_host(const anchorkv_params* p, const void* K_host, const void* V_host, const void* Q_host,
+                           void* out_host, size_t out_bytes, void* staging, size_t staging_bytes, void* ws,
+                           size_t ws_bytes, void* stream) {
+  Plan pl;
+  int st = make_plan(p, &pl);
+  if (st) return st;
+  const bool key_queries = (p->mode & ANCHORKV_MODE_KEY_QUERIES) != 0;
+  if (!K_host || !V_host || (!Q_host && !key_queries) || !out_host || !staging || !ws) return ANCHORKV_EINVAL;
+  const HostStaging hs = host_staging(pl);
+  if ((int64_t)out_bytes < pl.L.total_bytes || (int64_t)staging_bytes < hs.total) return ANCHORKV_ENOSPC;
+  if (((uintptr_t)staging | (uintptr_t)ws) & 15) return ANCHORKV_EINVAL;
+  st = check_device();
+  if (st) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* d = (char*)staging;
+  AKV_LAUNCH(cudaMemcpyAsync(d + hs.o_k, K_host, (size_t)hs.kv, cudaMemcpyHostToDevice, s));
+  AKV_LAUNCH(cudaMemcpyAsync(d + hs.o_v, V_host, (size_t)hs.kv, cudaMemcpyHostToDevice, s));
+  if (Q_host) AKV_LAUNCH(cudaMemcpyAsync(d + hs.o_q, Q_host, (size_t)hs.q, cudaMemcpyHostToDevice, s));
+  st = anchorkv_compress(p, d + hs.o_k, d + hs.o_v, Q_host ? d + hs.o_q : nullptr, d + hs.o_out, (size_t)hs.out, ws,
+                         ws_bytes, stream);
+  if (st) return st;
+  AKV_LAUNCH(cudaMemcpyAsync(out_host, d + hs.o_out, (size_t)hs.out, cudaMemcpyDeviceToHost, s));
   return ANCHORKV_OK;
 }
 

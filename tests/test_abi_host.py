@@ -68,6 +68,8 @@ def test_null_arguments_are_errors_not_crashes():
     n = ctypes.c_size_t()
     assert L.anchorkv_decode_workspace_bytes(ctypes.byref(p), -1, ctypes.byref(n)) == capi.EINVAL
     assert L.anchorkv_read_device_status(None, None, None) == capi.EINVAL
+    assert L.anchorkv_compress_host(ctypes.byref(p), None, None, None, None, 0, None, 0, None, 0, None) == capi.EINVAL
+    assert L.anchorkv_compress_host_staging_bytes(ctypes.byref(p), None) == capi.EINVAL
     assert L.anchorkv_strerror(capi.ENOSPC) == b"buffer too small"
 
 
@@ -77,6 +79,29 @@ def test_small_output_buffer_is_enospc():
     fake = ctypes.c_void_p(1 << 20)   # never dereferenced: size check fails first
     st = L.anchorkv_compress(ctypes.byref(p), fake, fake, fake, fake, 16, fake, 16, None)
     assert st == capi.ENOSPC
+
+
+def test_host_compress_staging_and_checks():
+    """The host-buffer compress: its staging size is K, V, Q_obs and the layout,
+    each rounded up to 256 bytes, and a small staging or output buffer is
+    refused before any copy (the fake pointers are never dereferenced)."""
+    L = capi.lib()
+    pp = api.AnchorKVParams(n_tokens=1000)
+    n = api.compress_host_staging_bytes(pp)
+    al = lambda x: (x + 255) // 256 * 256
+    kv = pp.n_kv_heads * pp.n_tokens * pp.head_dim * 2
+    q = pp.n_q_heads * pp.window * pp.head_dim * 2
+    total = api.anchorkv_bytes(pp)["total_bytes"]
+    assert n == 2 * al(kv) + al(q) + al(total)
+    p = pp.c()
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.anchorkv_compress_host(ctypes.byref(p), fake, fake, fake, fake, total, fake, n - 1, fake, 1 << 40,
+                                    None) == capi.ENOSPC
+    assert L.anchorkv_compress_host(ctypes.byref(p), fake, fake, fake, fake, total - 1, fake, n, fake, 1 << 40,
+                                    None) == capi.ENOSPC
+    misaligned = ctypes.c_void_p((1 << 20) + 8)
+    assert L.anchorkv_compress_host(ctypes.byref(p), fake, fake, fake, fake, total, misaligned, n, fake, 1 << 40,
+                                    None) == capi.EINVAL
 
 
 def test_library_codebook_matches_oracle():

@@ -81,6 +81,26 @@ def test_compress_deterministic():
     assert torch.equal(a, b)
 
 
+def test_host_buffer_compress_matches_device_compress():
+    """anchorkv_compress_host (copies inside the library, from pinned host
+    buffers) gives the device compress's bytes, in the host buffer and in the
+    staged layout; with key-as-query mode it takes no queries."""
+    spec, theta = CASES["bf16-ragged-n3000"]
+    K, V, Q = make_layer(spec, 0)
+    for mode in (0, api.MODE_KEY_QUERIES):
+        p = _params(spec, theta)
+        p.mode = mode
+        Qd = None if mode else Q.cuda()
+        ref, _ = api.compress(p, K.cuda(), V.cuda(), Qd)
+        hc = api.HostCompressor(p)
+        Kh, Vh = K.pin_memory(), V.pin_memory()
+        Qh = None if mode else Q.pin_memory()
+        out = hc(Kh, Vh, Qh)
+        torch.cuda.current_stream().synchronize()
+        assert torch.equal(out, ref.cpu())
+        assert torch.equal(hc.out, ref)
+
+
 def test_reconstruct_matches_oracle():
     spec, theta = CASES["bf16-ragged-n3000"]
     K, V, Q = make_layer(spec, 0)
